@@ -1,0 +1,367 @@
+"""Benchmark: MoE-layer expert forwards per second at batch 1 on B200.
+
+Workload: one 4-bit MoE layer of hidden 4096, expert intermediate 1024, 512
+routed experts (top-4, softmax renormalised over the selected) plus one
+shared expert, group-64 affine codes with bf16 scale/bias (6.75 MiB per
+expert, 3.62 GB per layer).  `--layers` (default 20) copies of that layer are
+resident in HBM (72.5 GB) and a token is carried through them as a stack, so
+that every step reads a new router, a new shared expert and the 4 routed
+experts the token picks: one step = one layer forward of one token, and the
+same weights come back only after 19 other layers (> 800 MB of other reads,
+well above the 126 MB L2).  All inputs are synthetic and seeded.
+
+Prints one JSON line (rank 0).  Under torchrun (N > 1) every rank runs its own
+replica (the path has no exchange step) and the time is the max over ranks.
+`--impl reference` times the fp64 CPU oracle on the same workload instead.
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import os
+import statistics
+import sys
+import threading
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
+
+METRIC = "MoE-layer expert fwd/s at batch 1; weight-stream HBM GB/s vs B200 peak"
+UNIT = "layer_fwd/s"
+FALLBACK_HBM_GBS = 6650.0
+
+
+def parse():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=4000)
+    ap.add_argument("--warmup", type=int, default=200)
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--layers", type=int, default=20, help="resident layer copies (L2 rotation)")
+    ap.add_argument("--e2e-steps", type=int, default=None)
+    ap.add_argument("--cpu-seconds", type=float, default=15.0, help="budget of the oracle CPU baseline sample")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    return ap.parse_args()
+
+
+def workload_config(layers: int) -> dict:
+    return {
+        "workload": "moe_layer_int4_batch1: hidden 4096, expert inter 1024, 512 experts top-4 + 1 shared, "
+                    f"group-64 int4 bf16 scale/bias, {layers} resident layer copies chained (one step = one layer of one token)",
+        "hidden": 4096, "inter": 1024, "experts": 512, "top_k": 4, "shared_experts": 1, "bits": 4, "group": 64,
+        "batch": 1, "layer_copies": layers,
+        "l2": f"inputs larger than L2: rotation over {layers} resident layers ({layers * 43.8:.0f} MB of weights per rotation)",
+    }
+
+
+def measured_peak():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(path) as f:
+            d = json.load(f)
+        return float(d["hbm_gbs"]), "measured"
+    except Exception:
+        return FALLBACK_HBM_GBS, "fallback"
+
+
+# ----------------------------------------------------------------- clocks --
+class ClockSampler:
+    REASONS = {0x4: "sw_power_cap", 0x8: "hw_slowdown", 0x20: "sw_thermal_slowdown",
+               0x40: "hw_thermal_slowdown", 0x80: "hw_power_brake_slowdown", 0x2: "applications_clocks_setting"}
+
+    def __init__(self, device_index: int, period: float = 0.01):
+        self.ok = False
+        self.samples = []
+        self.reasons = set()
+        self.period = period
+        try:
+            import pynvml
+            pynvml.nvmlInit()
+            self.nv = pynvml
+            try:
+                import torch
+                p = torch.cuda.get_device_properties(device_index)
+                bus = f"{p.pci_domain_id:08x}:{p.pci_bus_id:02x}:{p.pci_device_id:02x}.0"
+                self.h = pynvml.nvmlDeviceGetHandleByPciBusId(bus.encode())
+            except Exception:
+                self.h = pynvml.nvmlDeviceGetHandleByIndex(device_index)
+            self.max_mhz = pynvml.nvmlDeviceGetMaxClockInfo(self.h, pynvml.NVML_CLOCK_SM)
+            self.ok = True
+        except Exception:
+            self.max_mhz = None
+
+    def _sample(self):
+        nv = self.nv
+        self.samples.append(nv.nvmlDeviceGetClockInfo(self.h, nv.NVML_CLOCK_SM))
+        try:
+            r = nv.nvmlDeviceGetCurrentClocksEventReasons(self.h)
+        except Exception:
+            r = nv.nvmlDeviceGetCurrentClocksThrottleReasons(self.h)
+        for bit, name in self.REASONS.items():
+            if r & bit:
+                self.reasons.add(name)
+
+    def __enter__(self):
+        if self.ok:
+            self._stop = threading.Event()
+            self._sample()
+
+            def loop():
+                while not self._stop.wait(self.period):
+                    self._sample()
+            self._t = threading.Thread(target=loop, daemon=True)
+            self._t.start()
+        return self
+
+    def __exit__(self, *a):
+        if self.ok:
+            self._stop.set()
+            self._t.join()
+            self._sample()
+
+    def summary(self):
+        if not self.ok or not self.samples:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvml unavailable"]}
+        return {"sm_mhz": statistics.median(self.samples), "sm_max_mhz": self.max_mhz,
+                "reasons": sorted(self.reasons), "samples": len(self.samples)}
+
+
+# ------------------------------------------------------------ distributed --
+def dist_setup(n_gpus: int):
+    rank = int(os.environ.get("RANK", "0"))
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if world > 1:
+        import datetime
+        import torch
+        import torch.distributed as dist
+        torch.cuda.set_device(local)
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=600),
+                                device_id=torch.device("cuda", local))
+    return rank, world, local
+
+
+def barrier(world):
+    if world > 1:
+        import torch.distributed as dist
+        dist.barrier()
+
+
+def max_over_ranks(v: float, world: int) -> float:
+    if world == 1:
+        return v
+    import torch
+    import torch.distributed as dist
+    t = torch.tensor([v], dtype=torch.float64, device="cuda")
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+# ----------------------------------------------------------- CPU baseline --
+def oracle_layer_steps(max_steps: int, seconds: float, layers: int):
+    """Times the fp64 oracle, as it stands, on one host core: successive
+    single-token layer forwards of the benchmark workload through the layer
+    stack, until `max_steps` are done or `seconds` of oracle time are spent.
+    The selected experts are regenerated on demand; generation is not timed.
+    Returns (steps done, seconds spent in the oracle)."""
+    import numpy as np
+    import oracle
+    import synth
+    wl = synth.LAYER
+    done, spent = 0, 0.0
+    cache = {}
+    while done < max_steps and spent < seconds:
+        l = done % layers
+        if l not in cache:
+            cache[l] = oracle.LayerWeights(synth.router(wl, l), synth.shared_gate(wl, l), synth.norm_weight(wl, l), {})
+        lw = cache[l]
+        x = synth.tokens(wl, 1, stream=1000 + done)[0].astype(np.float64)
+        lg, _ = oracle.gemv_f32(lw.w_router, x)
+        ids, _, _ = oracle.topk_softmax(lg, wl.top_k)
+        lw.experts = {int(s): synth.expert(wl, l, int(s)) for s in list(ids) + [wl.n_experts]}
+        t0 = time.perf_counter()
+        oracle.layer_token(wl, lw, x, x)
+        spent += time.perf_counter() - t0
+        done += 1
+    return done, spent
+
+
+def cpu_baseline(seconds: float, layers: int) -> dict:
+    done, spent = oracle_layer_steps(10 ** 6, seconds, layers)
+    return {"value": done / spent, "unit": UNIT, "cores": 1, "kind": "oracle",
+            "sample": f"{done} single-token layer forwards of the benchmark workload (fp64 C oracle, one thread; "
+                      f"expert generation excluded), {spent:.1f} s"}
+
+
+def run_reference(args):
+    """The oracle as the reference arm: rank 0 alone times it on the host
+    cores (bounded sample: at most `steps` layer forwards or ~150 s)."""
+    rank = int(os.environ.get("RANK", "0"))
+    if rank != 0:
+        return
+    oracle_layer_steps(min(args.warmup, 1), 1e9, args.layers)
+    done, spent = oracle_layer_steps(max(1, args.steps), 150.0, args.layers)
+    value = done / spent
+    line = {"metric": METRIC, "value": value, "unit": UNIT, "n_gpus": args.gpus, "steps": done,
+            "warmup": args.warmup, "ms_per_step": 1e3 * spent / done, "higher_is_better": True, "scaling": "weak",
+            "vs_baseline": None, "dtype": "f64", "data": "synthetic", "config": workload_config(args.layers),
+            "impl": "reference",
+            "cpu_baseline": {"value": value, "unit": UNIT, "cores": 1, "kind": "oracle",
+                             "sample": f"{done} single-token layer forwards (fp64 C oracle, one thread; expert "
+                                       f"generation excluded), {spent:.1f} s of {max(1, args.steps)} requested steps"},
+            "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+    print(json.dumps(line), flush=True)
+
+
+# ------------------------------------------------------------------ ours --
+def run_ours(args):
+    import numpy as np
+    import torch
+
+    rank, world, local = dist_setup(args.gpus)
+    torch.cuda.set_device(local)
+    import quantized_expert_gemv_b200 as fm
+    import synth
+    from synth.device import upload_layer
+
+    wl = synth.LAYER
+    L = args.layers
+    scratch = {}
+    layers = [upload_layer(wl, l, scratch=scratch) for l in range(L)]
+    del scratch
+    torch.cuda.empty_cache()
+    desc = layers[0].desc
+    H = wl.hidden
+    ws = fm.alloc_workspace(desc, 1)
+    x0 = synth.tokens(wl, 1, stream=7 + rank)
+    h = torch.from_numpy(x0).cuda()
+    xn = h.clone()
+    stream = torch.cuda.Stream()
+    torch.cuda.synchronize()
+
+    # graphs: one per layer copy, and one for a whole rotation
+    graphs = []
+    with torch.cuda.stream(stream):
+        for l in range(L):  # eager warm-up of every layer once
+            fm.fmoe_layer_forward(layers[l], h, xn, ws, stream=stream)
+        stream.synchronize()
+        for l in range(L):
+            g = torch.cuda.CUDAGraph()
+            with torch.cuda.graph(g, stream=stream):
+                fm.fmoe_layer_forward(layers[l], h, xn, ws, stream=stream)
+            graphs.append(g)
+        g_all = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(g_all, stream=stream):
+            for l in range(L):
+                fm.fmoe_layer_forward(layers[l], h, xn, ws, stream=stream)
+    torch.cuda.synchronize()
+
+    def run_steps(n):
+        i = 0
+        while i + L <= n:
+            g_all.replay()
+            i += L
+        while i < n:
+            graphs[i % L].replay()
+            i += 1
+
+    with torch.cuda.stream(stream):
+        run_steps(args.warmup)
+    torch.cuda.synchronize()
+    barrier(world)
+    torch.cuda.synchronize()
+    ev0, ev1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    with ClockSampler(local) as clk:
+        with torch.cuda.stream(stream):
+            ev0.record(stream)
+            run_steps(args.steps)
+            ev1.record(stream)
+        ev1.synchronize()
+    torch.cuda.synchronize()
+    barrier(world)
+    ms = ev0.elapsed_time(ev1)
+    ms_max = max_over_ranks(ms, world)
+    st = fm.fmoe_read_status(clear=True)
+    if st:
+        raise RuntimeError(f"device status word {st:#x} after the timed region")
+
+    per_step_s = ms_max / 1e3 / args.steps
+    value = world * args.steps / (ms_max / 1e3)
+    rec = desc.record_bytes()
+    expert_bytes = (wl.top_k + 1) * rec
+    layer_bytes = expert_bytes + wl.n_experts * H * 4 + 2 * H * 4
+    peak, peak_kind = measured_peak()
+    achieved = layer_bytes / per_step_s / 1e9
+    roofline = {"bound": "hbm", "kernel": "one layer step (router, top-k, gate/up+SwiGLU, down, combine+RMSNorm)",
+                "achieved": achieved, "peak": peak, "peak_kind": peak_kind, "unit": "GB/s",
+                "frac": achieved / peak, "traffic": None,
+                "bytes_per_launch": layer_bytes}
+
+    # ---- end to end through the C ABI with host buffers (eager calls) ----
+    K2 = args.e2e_steps or min(args.steps, 2000)
+    xs = synth.tokens(wl, min(K2, 64), stream=500 + rank)
+    h_in = torch.from_numpy(np.ascontiguousarray(xs)).pin_memory()
+    out_h = torch.empty((min(K2, 64), H), dtype=torch.float32).pin_memory()
+    out_x = torch.empty((min(K2, 64), H), dtype=torch.float32).pin_memory()
+    nb = h_in.shape[0]
+
+    def e2e_steps(n):
+        for i in range(n):
+            j = i % nb
+            h.copy_(h_in[j:j + 1], non_blocking=True)
+            xn.copy_(h_in[j:j + 1], non_blocking=True)
+            fm.fmoe_layer_forward(layers[i % L], h, xn, ws, stream=stream)
+            out_h[j:j + 1].copy_(h, non_blocking=True)
+            out_x[j:j + 1].copy_(xn, non_blocking=True)
+
+    with torch.cuda.stream(stream):
+        e2e_steps(min(50, K2))
+    torch.cuda.synchronize()
+    barrier(world)
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    with torch.cuda.stream(stream):
+        e0.record(stream)
+        e2e_steps(K2)
+        e1.record(stream)
+    e1.synchronize()
+    e2e_ms = max_over_ranks(e0.elapsed_time(e1), world)
+    e2e = {"value": world * K2 / (e2e_ms / 1e3), "unit": UNIT, "h2d_bytes_per_step": 2 * H * 4,
+           "d2h_bytes_per_step": 2 * H * 4, "steps": K2,
+           "how": "per step: pinned host h, xn -> device, fmoe_layer_forward (eager C-ABI call), h', xn' -> pinned host"}
+
+    kernels_per_layer = 5
+    line = {"metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
+            "warmup": args.warmup, "ms_per_step": ms_max / args.steps, "higher_is_better": True,
+            "scaling": "weak", "vs_baseline": None, "dtype": "int4 codes x int16 fixed-point x, f32 accumulate",
+            "data": "synthetic (seeded generator, random-init weights of the layer shape)",
+            "config": workload_config(L),
+            "expert_weight_gbs": expert_bytes / per_step_s / 1e9,
+            "layer_gbs": achieved,
+            "pct_of_8tbs_expert_bytes": 100 * expert_bytes / per_step_s / 8e12,
+            "roofline": roofline, "e2e": e2e, "gpu_launches": kernels_per_layer * args.steps,
+            "clocks": clk.summary()}
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        line["cpu_baseline"] = cpu_baseline(args.cpu_seconds, L)
+    elif rank == 0:
+        line["cpu_baseline"] = None
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+    barrier(world)
+    del graphs, g_all
+    if world > 1:
+        import torch.distributed as dist
+        dist.destroy_process_group()
+
+
+def main():
+    args = parse()
+    if args.impl == "reference":
+        run_reference(args)
+    else:
+        run_ours(args)
+
+
+if __name__ == "__main__":
+    main()

@@ -1,0 +1,230 @@
+/*
+ * fmoe.h -- C ABI of the quantised MoE expert forward for B200 (sm_100a).
+ *
+ * One token's pass through a mixture-of-experts layer whose expert weights
+ * are group-affine 4-bit or 2-bit codes resident in HBM:
+ *   route   logits = W_r xn, top-k experts (k of E), softmax over the k
+ *           selected logits ("What is Flash-MoE?", section "Understanding
+ *           Mixture-of-Experts": 4 routed experts of 512 plus 1 shared)
+ *   expert  g = W_g xn, u = W_u xn, a = silu(g) u, y = W_d a for each selected
+ *           expert and the shared expert; every weight is code * scale + bias
+ *           with one bf16 scale/bias per 64 inputs ("What is Flash-MoE?",
+ *           sections "2. FMA-optimised dequantisation kernels" and
+ *           "3. Hand-tuned Metal compute shaders": 4-bit/2-bit matrix-vector
+ *           multiply, fused SwiGLU)
+ *   combine h' = h + sum_k p_k y_k + sigmoid(w_sg . xn) y_shared, then the
+ *           two-pass RMSNorm xn' = h' (mean(h'^2) + eps)^(-1/2) w
+ *           (same section: MoE combine + residual + sigmoid gating in one
+ *           pass; two-pass RMSNorm; the result feeds the next layer).
+ *
+ * Conventions (all entry points):
+ *   - Every call returns an int status (FMOE_OK == 0 on success).  Host-side
+ *     validation happens before anything is launched; on a validation error
+ *     nothing is launched and no output is touched.
+ *   - Pointers named d_* or documented "device" are device memory of the
+ *     current CUDA device; "host" pointers are ordinary host memory.  The
+ *     caller owns every buffer; no entry point allocates device memory.
+ *   - Device pointers must be 16-byte aligned.
+ *   - Device-side work is enqueued on the caller's stream and is
+ *     asynchronous: no entry point synchronises, except the packer, which
+ *     waits for its own host-to-device copy.
+ *   - Faults detected on the device (an expert id outside [0, E), a NaN
+ *     router logit, an exhausted wait) set bits of a sticky per-device
+ *     status word; kernels never trap.  Read and clear it with
+ *     fmoe_read_status().
+ *   - fp32 activations, row-major: a [T][H] array holds token t's hidden
+ *     vector at offset t * H.
+ */
+#ifndef FMOE_H_
+#define FMOE_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#include <cuda_runtime_api.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+/* ---------------------------------------------------------------- status -- */
+#define FMOE_OK 0
+#define FMOE_ERR_INVALID_ARG 1   /* null pointer, bad size, misaligned pointer */
+#define FMOE_ERR_UNSUPPORTED 2   /* a shape or bit width this build does not run */
+#define FMOE_ERR_CUDA 3          /* a CUDA runtime call failed */
+#define FMOE_ERR_DEVICE_STATUS 4 /* the device status word is non-zero */
+#define FMOE_ERR_BUFFER_TOO_SMALL 5
+
+/* bits of the device status word */
+#define FMOE_STATUS_BAD_EXPERT_ID 0x1u /* an id outside [0, E) was skipped */
+#define FMOE_STATUS_NAN_LOGIT 0x2u     /* a router logit was NaN (ordered below every number) */
+#define FMOE_STATUS_WAIT_TIMEOUT 0x4u  /* a bounded wait gave up; results are invalid */
+#define FMOE_STATUS_BAD_PACK_INPUT 0x8u /* device packer: a code out of range or a scale that cannot be pre-scaled exactly */
+
+/* Human-readable name of a status code (static string, never NULL). */
+const char* fmoe_error_string(int status);
+
+/* Reads the calling thread's current device's status word into *status
+ * (host pointer) after synchronising the device; clears it when clear != 0.
+ * Returns FMOE_OK or FMOE_ERR_CUDA. */
+int fmoe_read_status(uint32_t* status, int clear);
+
+/* ----------------------------------------------------------- the layer -- */
+typedef struct fmoe_layer_desc {
+  int hidden;      /* H: model width; a multiple of 64 with H/64 a power of two <= 32 or a multiple of 32 */
+  int inter;       /* I: expert intermediate width; same rule as H */
+  int n_experts;   /* E: routed experts, 1 .. 1024 */
+  int top_k;       /* k: routed experts per token, 1 .. 8, k <= E */
+  int bits;        /* code width of the routed experts: 4 or 2 */
+  int shared_bits; /* code width of the shared expert: 4 or 2 */
+  int group;       /* inputs per scale/bias group: must be 64 */
+  float eps;       /* RMSNorm epsilon (inside the square root) */
+} fmoe_layer_desc;
+
+typedef struct fmoe_layer_weights {
+  fmoe_layer_desc desc;
+  const void* experts;        /* device: E packed expert records, each fmoe_packed_bytes(bits, 1, H, I, 64) bytes, back to back */
+  const void* shared;         /* device: one packed record of the shared expert (shared_bits) */
+  const float* w_router;      /* device fp32 [E][H] */
+  const float* w_shared_gate; /* device fp32 [H]: the shared expert's output is scaled by sigmoid(w_shared_gate . xn) */
+  const float* norm_w;        /* device fp32 [H]: RMSNorm weight */
+} fmoe_layer_weights;
+
+/* ------------------------------------------------------------- packing -- */
+/* Logical expert layout (host input of the packer, output of the unpacker):
+ *   q      uint8 [3 * H * I] per expert: gate [I][H], up [I][H], down [H][I],
+ *          one code (0 .. 2^bits - 1) per byte, row-major;
+ *   scale, bias  uint16 bf16 bit patterns [3 * H * I / 64] per expert, one per
+ *          64 consecutive inputs of a row, same matrix order, row-major.
+ *   The weight of row r, input j is q * scale + bias of group j / 64.
+ * Experts follow one another: expert e starts at q + e * 3 * H * I, and at
+ * scale/bias + e * 3 * H * I / 64.
+ *
+ * Packed record (one per expert; all sections 16-byte aligned):
+ *   [gate/up codes][down codes][gate/up scale-bias][down scale-bias]
+ *   gate/up: I row pairs, gate row n then up row n; down: H rows.
+ *   A row of K inputs is split into segments of min(32, K/64) groups; within
+ *   a segment 4-bit codes store first the low halves (inputs 0..31) of all its
+ *   groups, 16 bytes each, then the high halves; 2-bit codes store each
+ *   group's 16 bytes in order.  Inside each 32-bit word the 8 (or 16) codes of
+ *   8 (16) consecutive inputs are permuted so that masking the word with
+ *   0x0F0F0F0F / 0xF0F0F0F0 (4-bit) or 0x03030303 .. 0xC0C0C0C0 (2-bit) yields
+ *   byte lanes that pair with consecutive inputs (field 2a+b, resp. 4a+b, of
+ *   the word holds input 4b+a).  Scale-bias: one 32-bit word per group,
+ *   bf16 scale * 2^-4 (4-bit) or * 2^-6 (2-bit) in the low half, bf16 bias in
+ *   the high half, row-major.
+ * Size per expert: 3 H I bits / 8 + 3 H I / 64 * 4 bytes (7,077,888 bytes =
+ * 6.75 MiB at H = 4096, I = 1024, 4-bit; 3,932,160 bytes at 2-bit). */
+
+/* Bytes of n_experts packed records.  Returns 0 for an unsupported shape. */
+size_t fmoe_packed_bytes(int bits, int n_experts, int hidden, int inter, int group);
+
+/* Packs n_experts logical experts (host arrays, layout above) into host
+ * memory h_packed (h_bytes >= fmoe_packed_bytes(...)).  Pure host code.
+ * Errors: FMOE_ERR_INVALID_ARG (null, code out of range, scale that cannot be
+ * pre-scaled exactly), FMOE_ERR_UNSUPPORTED (shape), FMOE_ERR_BUFFER_TOO_SMALL. */
+int fmoe_pack_experts_host(const uint8_t* q, const uint16_t* scale, const uint16_t* bias, int bits,
+                           int n_experts, int hidden, int inter, int group, void* h_packed,
+                           size_t h_bytes);
+
+/* Inverse of fmoe_pack_experts_host (host to host), for round-trip checks. */
+int fmoe_unpack_experts_host(const void* h_packed, int bits, int n_experts, int hidden, int inter,
+                             int group, uint8_t* q, uint16_t* scale, uint16_t* bias);
+
+/* Packs on the host and copies the records into device memory d_packed
+ * (d_bytes >= fmoe_packed_bytes(...)) on `stream`; returns after the copy
+ * has completed.  Not for the hot path (allocates a host staging buffer). */
+int fmoe_pack_experts(const uint8_t* q, const uint16_t* scale, const uint16_t* bias, int bits,
+                      int n_experts, int hidden, int inter, int group, void* d_packed,
+                      size_t d_bytes, cudaStream_t stream);
+
+/* As fmoe_pack_experts, with the logical arrays already in device memory
+ * (d_q, d_scale, d_bias, same layout as the host arrays; 16-byte aligned).
+ * Packs on `stream` without synchronising and without a host round trip.
+ * Invalid codes or scales are reported through FMOE_STATUS_BAD_PACK_INPUT in
+ * the device status word (the affected words are written as zero).
+ * Errors: FMOE_ERR_INVALID_ARG, FMOE_ERR_UNSUPPORTED, FMOE_ERR_BUFFER_TOO_SMALL,
+ * FMOE_ERR_CUDA. */
+int fmoe_pack_experts_device(const uint8_t* d_q, const uint16_t* d_scale, const uint16_t* d_bias,
+                             int bits, int n_experts, int hidden, int inter, int group,
+                             void* d_packed, size_t d_bytes, cudaStream_t stream);
+
+/* ----------------------------------------------------------- workspace -- */
+/* Device workspace for T tokens of a layer with descriptor d (bytes).  The
+ * workspace holds intermediates (router partial sums, logits, ids, gate
+ * weights, gamma, the SwiGLU outputs a and the expert outputs y) and a few
+ * counters; it must be zeroed once with fmoe_workspace_init before first use
+ * and is left re-usable by every call that completes. */
+size_t fmoe_workspace_bytes(const fmoe_layer_desc* d, int T);
+
+/* Zeroes a workspace (cudaMemsetAsync on `stream`). */
+int fmoe_workspace_init(void* d_ws, size_t ws_bytes, cudaStream_t stream);
+
+/* Offsets (bytes from the workspace start) of the intermediates that
+ * fmoe_layer_forward leaves behind: which = 0 logits fp32 [T][E],
+ * 1 ids int32 [T][k], 2 gate weights fp32 [T][k], 3 gamma fp32 [T],
+ * 4 a fp32 [T][k+1][I], 5 y fp32 [T][k+1][H].  Returns (size_t)-1 on error. */
+size_t fmoe_workspace_offset(const fmoe_layer_desc* d, int T, int which);
+
+/* --------------------------------------------------------- entry points -- */
+#define FMOE_LOGITS_GIVEN 0x1u /* route: logits are an input, skip the router product */
+
+/* Router product and top-k (section "Understanding Mixture-of-Experts").
+ *   d_xn       device fp32 [T][H] normed inputs
+ *   d_w_router device fp32 [E][H]
+ *   d_logits   device fp32 [T][E]: output, or input when flags has FMOE_LOGITS_GIVEN
+ *   d_ids      device int32 [T][k]: selected experts, largest logit first,
+ *              ties to the lower index, NaN below every number
+ *   d_weights  device fp32 [T][k]: softmax of the k selected logits
+ *   d_ws       device workspace of at least fmoe_workspace_bytes(d, T) bytes
+ *              for a descriptor with these H, E, k (only its router part is used)
+ * Errors: FMOE_ERR_INVALID_ARG, FMOE_ERR_UNSUPPORTED (k > 8, E > 1024), FMOE_ERR_CUDA. */
+int fmoe_route_topk(const float* d_xn, const float* d_w_router, int T, int H, int E, int k,
+                    unsigned flags, float* d_logits, int32_t* d_ids, float* d_weights, void* d_ws,
+                    size_t ws_bytes, cudaStream_t stream);
+
+/* Expert forward for T tokens: for each token t, the k experts d_ids[t][*]
+ * and the shared expert, on input d_xn[t]:
+ *   d_y     device fp32 [T][k+1][H]: y of each selected expert in the order of
+ *           d_ids, the shared expert last (not yet weighted)
+ *   d_gamma device fp32 [T]: sigmoid(w_shared_gate . xn)
+ * An id outside [0, E) contributes y = 0 and sets FMOE_STATUS_BAD_EXPERT_ID.
+ * Errors: FMOE_ERR_INVALID_ARG, FMOE_ERR_UNSUPPORTED, FMOE_ERR_CUDA. */
+int fmoe_expert_forward(const fmoe_layer_weights* lw, const float* d_xn, int T,
+                        const int32_t* d_ids, int k, float* d_y, float* d_gamma, void* d_ws,
+                        size_t ws_bytes, cudaStream_t stream);
+
+/* Combine + residual + shared gate, then RMSNorm, for T tokens:
+ *   h_out[t] = h[t] + sum_j weights[t][j] y[t][j] + gamma[t] y[t][k]
+ *   xn_out[t] = h_out[t] * (mean(h_out[t]^2) + eps)^(-1/2) * norm_w
+ * All device fp32; y [T][k+1][H]; h_out may alias h and xn_out may alias
+ * neither y nor h.  Errors: FMOE_ERR_INVALID_ARG, FMOE_ERR_CUDA. */
+int fmoe_combine_residual_rmsnorm(const float* d_y, const float* d_weights, const float* d_gamma,
+                                  const float* d_h, const float* d_norm_w, float eps, int T, int k,
+                                  int H, float* d_h_out, float* d_xn_out, cudaStream_t stream);
+
+/* One whole layer for T tokens, in place: reads the residual d_h [T][H] and
+ * the normed input d_xn [T][H], writes h' to d_h and xn' to d_xn.  All steps
+ * run on the device with no host round trip; the call is safe to capture in
+ * a CUDA graph.  The intermediates stay in the workspace (see
+ * fmoe_workspace_offset).  Errors: FMOE_ERR_INVALID_ARG, FMOE_ERR_UNSUPPORTED,
+ * FMOE_ERR_CUDA. */
+int fmoe_layer_forward(const fmoe_layer_weights* lw, float* d_h, float* d_xn, int T, void* d_ws,
+                       size_t ws_bytes, cudaStream_t stream);
+
+/* As fmoe_layer_forward, routing on given router logits d_logits [T][E]
+ * (device fp32) instead of the router product. */
+int fmoe_layer_forward_logits(const fmoe_layer_weights* lw, const float* d_logits, float* d_h,
+                              float* d_xn, int T, void* d_ws, size_t ws_bytes, cudaStream_t stream);
+
+/* A stack of n_layers layers (host array of weight descriptors, all with the
+ * same descriptor) for T tokens, in place on d_h / d_xn: layer l + 1 reads
+ * what layer l wrote.  Equivalent to n_layers calls of fmoe_layer_forward. */
+int fmoe_stack_forward(const fmoe_layer_weights* layers, int n_layers, float* d_h, float* d_xn,
+                       int T, void* d_ws, size_t ws_bytes, cudaStream_t stream);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* FMOE_H_ */

@@ -1,0 +1,297 @@
+"""Quantised MoE expert forward for B200 (sm_100a): Python binding of libfmoe.
+
+A thin ctypes layer over the C ABI declared in include/fmoe.h: it converts
+torch tensors / numpy arrays to pointers and checks status codes.  Every step
+of the computation runs in the library's CUDA kernels; there is no Python or
+CPU fallback.  If libfmoe.so has not been built, importing this package
+raises ImportError (build it with ``python -m quantized_expert_gemv_b200.build``
+or ``__graft_entry__.build()``).
+
+PyTorch is used only for device memory and streams: device arguments are
+CUDA tensors, and work is enqueued on ``torch.cuda.current_stream()`` unless
+a stream is given.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+from dataclasses import dataclass, field
+
+import numpy as np
+
+_PKG = os.path.dirname(os.path.abspath(__file__))
+_LIB_PATH = os.path.join(_PKG, "libfmoe.so")
+
+if not os.path.exists(_LIB_PATH):
+    raise ImportError(
+        f"{_LIB_PATH} is missing: the CUDA library has not been built "
+        "(run `python -m quantized_expert_gemv_b200.build`). There is no fallback.")
+
+_lib = ctypes.CDLL(_LIB_PATH)
+
+FMOE_OK = 0
+FMOE_ERR_INVALID_ARG = 1
+FMOE_ERR_UNSUPPORTED = 2
+FMOE_ERR_CUDA = 3
+FMOE_ERR_DEVICE_STATUS = 4
+FMOE_ERR_BUFFER_TOO_SMALL = 5
+
+FMOE_STATUS_BAD_EXPERT_ID = 0x1
+FMOE_STATUS_NAN_LOGIT = 0x2
+FMOE_STATUS_WAIT_TIMEOUT = 0x4
+FMOE_STATUS_BAD_PACK_INPUT = 0x8
+
+FMOE_LOGITS_GIVEN = 0x1
+
+WS_LOGITS, WS_IDS, WS_WEIGHTS, WS_GAMMA, WS_A, WS_Y = range(6)
+
+LIBRARY_PATH = _LIB_PATH
+
+
+class FmoeError(RuntimeError):
+    def __init__(self, status: int, where: str):
+        self.status = status
+        super().__init__(f"{where}: {fmoe_error_string(status)} (status {status})")
+
+
+class fmoe_layer_desc(ctypes.Structure):
+    _fields_ = [("hidden", ctypes.c_int), ("inter", ctypes.c_int), ("n_experts", ctypes.c_int),
+                ("top_k", ctypes.c_int), ("bits", ctypes.c_int), ("shared_bits", ctypes.c_int),
+                ("group", ctypes.c_int), ("eps", ctypes.c_float)]
+
+
+class fmoe_layer_weights(ctypes.Structure):
+    _fields_ = [("desc", fmoe_layer_desc), ("experts", ctypes.c_void_p), ("shared", ctypes.c_void_p),
+                ("w_router", ctypes.c_void_p), ("w_shared_gate", ctypes.c_void_p),
+                ("norm_w", ctypes.c_void_p)]
+
+
+_vp, _i32, _u32, _sz, _f32 = ctypes.c_void_p, ctypes.c_int, ctypes.c_uint, ctypes.c_size_t, ctypes.c_float
+_PDESC = ctypes.POINTER(fmoe_layer_desc)
+_PW = ctypes.POINTER(fmoe_layer_weights)
+
+_SIGS = {
+    "fmoe_error_string": (ctypes.c_char_p, [_i32]),
+    "fmoe_read_status": (_i32, [ctypes.POINTER(ctypes.c_uint32), _i32]),
+    "fmoe_packed_bytes": (_sz, [_i32, _i32, _i32, _i32, _i32]),
+    "fmoe_pack_experts_host": (_i32, [_vp, _vp, _vp, _i32, _i32, _i32, _i32, _i32, _vp, _sz]),
+    "fmoe_unpack_experts_host": (_i32, [_vp, _i32, _i32, _i32, _i32, _i32, _vp, _vp, _vp]),
+    "fmoe_pack_experts": (_i32, [_vp, _vp, _vp, _i32, _i32, _i32, _i32, _i32, _vp, _sz, _vp]),
+    "fmoe_pack_experts_device": (_i32, [_vp, _vp, _vp, _i32, _i32, _i32, _i32, _i32, _vp, _sz, _vp]),
+    "fmoe_workspace_bytes": (_sz, [_PDESC, _i32]),
+    "fmoe_workspace_init": (_i32, [_vp, _sz, _vp]),
+    "fmoe_workspace_offset": (_sz, [_PDESC, _i32, _i32]),
+    "fmoe_route_topk": (_i32, [_vp, _vp, _i32, _i32, _i32, _i32, _u32, _vp, _vp, _vp, _vp, _sz, _vp]),
+    "fmoe_expert_forward": (_i32, [_PW, _vp, _i32, _vp, _i32, _vp, _vp, _vp, _sz, _vp]),
+    "fmoe_combine_residual_rmsnorm": (_i32, [_vp, _vp, _vp, _vp, _vp, _f32, _i32, _i32, _i32, _vp, _vp, _vp]),
+    "fmoe_layer_forward": (_i32, [_PW, _vp, _vp, _i32, _vp, _sz, _vp]),
+    "fmoe_layer_forward_logits": (_i32, [_PW, _vp, _vp, _vp, _i32, _vp, _sz, _vp]),
+    "fmoe_stack_forward": (_i32, [_PW, _i32, _vp, _vp, _i32, _vp, _sz, _vp]),
+}
+for _name, (_res, _args) in _SIGS.items():
+    _fn = getattr(_lib, _name)
+    _fn.restype = _res
+    _fn.argtypes = _args
+
+EXPORTED = tuple(_SIGS)
+
+
+def _check(rc: int, where: str) -> None:
+    if rc != FMOE_OK:
+        raise FmoeError(rc, where)
+
+
+def _ptr(x):
+    """Device or host pointer of a torch tensor / numpy array (None -> NULL)."""
+    if x is None:
+        return None
+    if isinstance(x, np.ndarray):
+        assert x.flags["C_CONTIGUOUS"], "array must be contiguous"
+        return ctypes.c_void_p(x.ctypes.data)
+    if isinstance(x, int):
+        return ctypes.c_void_p(x)
+    assert x.is_contiguous(), "tensor must be contiguous"
+    return ctypes.c_void_p(x.data_ptr())
+
+
+def _stream(stream):
+    if stream is None:
+        import torch
+        return ctypes.c_void_p(torch.cuda.current_stream().cuda_stream)
+    if isinstance(stream, int):
+        return ctypes.c_void_p(stream)
+    return ctypes.c_void_p(stream.cuda_stream)
+
+
+def fmoe_error_string(status: int) -> str:
+    return _lib.fmoe_error_string(status).decode()
+
+
+def fmoe_read_status(clear: bool = True) -> int:
+    v = ctypes.c_uint32(0)
+    _check(_lib.fmoe_read_status(ctypes.byref(v), int(clear)), "fmoe_read_status")
+    return int(v.value)
+
+
+def fmoe_packed_bytes(bits: int, n_experts: int, hidden: int, inter: int, group: int = 64) -> int:
+    return int(_lib.fmoe_packed_bytes(bits, n_experts, hidden, inter, group))
+
+
+def fmoe_pack_experts_host(q: np.ndarray, scale: np.ndarray, bias: np.ndarray, bits: int, n_experts: int,
+                           hidden: int, inter: int, group: int = 64, out: np.ndarray | None = None) -> np.ndarray:
+    n = fmoe_packed_bytes(bits, n_experts, hidden, inter, group)
+    if out is None:
+        out = np.empty(max(n, 1), np.uint8)
+    rc = _lib.fmoe_pack_experts_host(_ptr(q), _ptr(scale), _ptr(bias), bits, n_experts, hidden, inter, group,
+                                     _ptr(out), out.nbytes)
+    _check(rc, "fmoe_pack_experts_host")
+    return out
+
+
+def fmoe_unpack_experts_host(packed: np.ndarray, bits: int, n_experts: int, hidden: int, inter: int,
+                             group: int = 64):
+    n = hidden * inter
+    q = np.empty(n_experts * 3 * n, np.uint8)
+    s = np.empty(n_experts * 3 * n // group, np.uint16)
+    b = np.empty_like(s)
+    rc = _lib.fmoe_unpack_experts_host(_ptr(packed), bits, n_experts, hidden, inter, group, _ptr(q), _ptr(s), _ptr(b))
+    _check(rc, "fmoe_unpack_experts_host")
+    return q, s, b
+
+
+def fmoe_pack_experts(q, scale, bias, bits: int, n_experts: int, hidden: int, inter: int, d_packed,
+                      group: int = 64, stream=None, byte_offset: int = 0) -> None:
+    """Packs host logical experts into the device tensor d_packed (at byte_offset)."""
+    dst = d_packed.data_ptr() + byte_offset
+    avail = d_packed.numel() * d_packed.element_size() - byte_offset
+    rc = _lib.fmoe_pack_experts(_ptr(q), _ptr(scale), _ptr(bias), bits, n_experts, hidden, inter, group,
+                                ctypes.c_void_p(dst), avail, _stream(stream))
+    _check(rc, "fmoe_pack_experts")
+
+
+def fmoe_pack_experts_device(d_q, d_scale, d_bias, bits: int, n_experts: int, hidden: int, inter: int, d_packed,
+                             group: int = 64, stream=None, byte_offset: int = 0) -> None:
+    """Packs logical experts already on the device into d_packed (at byte_offset)."""
+    dst = d_packed.data_ptr() + byte_offset
+    avail = d_packed.numel() * d_packed.element_size() - byte_offset
+    rc = _lib.fmoe_pack_experts_device(_ptr(d_q), _ptr(d_scale), _ptr(d_bias), bits, n_experts, hidden, inter,
+                                       group, ctypes.c_void_p(dst), avail, _stream(stream))
+    _check(rc, "fmoe_pack_experts_device")
+
+
+@dataclass
+class LayerDesc:
+    hidden: int = 4096
+    inter: int = 1024
+    n_experts: int = 512
+    top_k: int = 4
+    bits: int = 4
+    shared_bits: int = 4
+    group: int = 64
+    eps: float = 1e-6
+
+    def c(self) -> fmoe_layer_desc:
+        return fmoe_layer_desc(self.hidden, self.inter, self.n_experts, self.top_k, self.bits,
+                               self.shared_bits, self.group, self.eps)
+
+    def record_bytes(self, shared: bool = False) -> int:
+        return fmoe_packed_bytes(self.shared_bits if shared else self.bits, 1, self.hidden, self.inter, self.group)
+
+
+@dataclass
+class LayerWeights:
+    """Device tensors of one layer (kept alive here) and their C descriptor."""
+
+    desc: LayerDesc
+    experts: object        # uint8 CUDA tensor, E packed records
+    shared: object         # uint8 CUDA tensor, one packed record
+    w_router: object       # fp32 CUDA [E][H]
+    w_shared_gate: object  # fp32 CUDA [H]
+    norm_w: object         # fp32 CUDA [H]
+    _c: fmoe_layer_weights = field(default=None, repr=False)
+
+    def c(self) -> fmoe_layer_weights:
+        if self._c is None:
+            self._c = fmoe_layer_weights(self.desc.c(), self.experts.data_ptr(), self.shared.data_ptr(),
+                                         self.w_router.data_ptr(), self.w_shared_gate.data_ptr(),
+                                         self.norm_w.data_ptr())
+        return self._c
+
+
+def fmoe_workspace_bytes(desc: LayerDesc, T: int) -> int:
+    d = desc.c()
+    return int(_lib.fmoe_workspace_bytes(ctypes.byref(d), T))
+
+
+def fmoe_workspace_init(ws, stream=None) -> None:
+    _check(_lib.fmoe_workspace_init(_ptr(ws), ws.numel() * ws.element_size(), _stream(stream)), "fmoe_workspace_init")
+
+
+def fmoe_workspace_offset(desc: LayerDesc, T: int, which: int) -> int:
+    d = desc.c()
+    return int(_lib.fmoe_workspace_offset(ctypes.byref(d), T, which))
+
+
+def alloc_workspace(desc: LayerDesc, T: int, device="cuda"):
+    """A zero-initialised workspace tensor (uint8) for T tokens."""
+    import torch
+    n = fmoe_workspace_bytes(desc, T)
+    return torch.zeros(n, dtype=torch.uint8, device=device)
+
+
+def workspace_view(ws, desc: LayerDesc, T: int, which: int):
+    """Typed view of an intermediate that fmoe_layer_forward leaves in the workspace."""
+    import torch
+    k, H, I, E = desc.top_k, desc.hidden, desc.inter, desc.n_experts
+    off = fmoe_workspace_offset(desc, T, which)
+    shapes = {WS_LOGITS: ((T, E), torch.float32), WS_IDS: ((T, k), torch.int32),
+              WS_WEIGHTS: ((T, k), torch.float32), WS_GAMMA: ((T,), torch.float32),
+              WS_A: ((T, k + 1, I), torch.float32), WS_Y: ((T, k + 1, H), torch.float32)}
+    shape, dt = shapes[which]
+    n = int(np.prod(shape))
+    return ws[off:off + 4 * n].view(dt).view(*shape)
+
+
+def fmoe_route_topk(xn, w_router, k: int, logits, ids, weights, ws=None, flags: int = 0, stream=None) -> None:
+    T, E = logits.shape
+    H = w_router.shape[1] if w_router is not None else 64
+    nbytes = ws.numel() * ws.element_size() if ws is not None else 0
+    rc = _lib.fmoe_route_topk(_ptr(xn), _ptr(w_router), T, H, E, k, flags, _ptr(logits), _ptr(ids),
+                              _ptr(weights), _ptr(ws), nbytes, _stream(stream))
+    _check(rc, "fmoe_route_topk")
+
+
+def fmoe_expert_forward(lw: LayerWeights, xn, ids, y, gamma, ws, stream=None) -> None:
+    T = xn.shape[0]
+    c = lw.c()
+    rc = _lib.fmoe_expert_forward(ctypes.byref(c), _ptr(xn), T, _ptr(ids), lw.desc.top_k, _ptr(y), _ptr(gamma),
+                                  _ptr(ws), ws.numel() * ws.element_size(), _stream(stream))
+    _check(rc, "fmoe_expert_forward")
+
+
+def fmoe_combine_residual_rmsnorm(y, weights, gamma, h, norm_w, eps: float, h_out, xn_out, stream=None) -> None:
+    T, k1, H = y.shape
+    rc = _lib.fmoe_combine_residual_rmsnorm(_ptr(y), _ptr(weights), _ptr(gamma), _ptr(h), _ptr(norm_w), eps, T,
+                                            k1 - 1, H, _ptr(h_out), _ptr(xn_out), _stream(stream))
+    _check(rc, "fmoe_combine_residual_rmsnorm")
+
+
+def fmoe_layer_forward(lw: LayerWeights, h, xn, ws, stream=None) -> None:
+    c = lw.c()
+    rc = _lib.fmoe_layer_forward(ctypes.byref(c), _ptr(h), _ptr(xn), h.shape[0], _ptr(ws),
+                                 ws.numel() * ws.element_size(), _stream(stream))
+    _check(rc, "fmoe_layer_forward")
+
+
+def fmoe_layer_forward_logits(lw: LayerWeights, logits, h, xn, ws, stream=None) -> None:
+    c = lw.c()
+    rc = _lib.fmoe_layer_forward_logits(ctypes.byref(c), _ptr(logits), _ptr(h), _ptr(xn), h.shape[0], _ptr(ws),
+                                        ws.numel() * ws.element_size(), _stream(stream))
+    _check(rc, "fmoe_layer_forward_logits")
+
+
+def fmoe_stack_forward(layers, h, xn, ws, stream=None) -> None:
+    arr = (fmoe_layer_weights * len(layers))(*[lw.c() for lw in layers])
+    rc = _lib.fmoe_stack_forward(arr, len(layers), _ptr(h), _ptr(xn), h.shape[0], _ptr(ws),
+                                 ws.numel() * ws.element_size(), _stream(stream))
+    _check(rc, "fmoe_stack_forward")

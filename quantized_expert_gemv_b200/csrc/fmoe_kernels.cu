@@ -1,0 +1,746 @@
+// fmoe_kernels.cu -- sm_100a kernels and the C ABI of the quantised MoE
+// expert forward (see include/fmoe.h for the contract of every entry point).
+//
+// Kernels, in the order one layer runs them:
+//   router_partial_kernel  fp32 router rows x normed input, split along H
+//   topk_kernel            sums the splits, warp top-k, softmax of the k
+//                          selected logits, shared-expert sigmoid gate
+//   gateup_kernel          dequantising gate/up products of every selected
+//                          expert and the shared expert, fused SwiGLU
+//   down_kernel            dequantising down product
+//   combine_kernel         weighted combine + residual + shared gate, then the
+//                          two-pass RMSNorm
+// Source pages: "What is Flash-MoE?" (a2a-mcp.org), sections "Understanding
+// Mixture-of-Experts" (top-4 of 512 plus one shared expert),
+// "2. FMA-optimised dequantisation kernels" and "3. Hand-tuned Metal compute
+// shaders" (dequantising matrix-vector products, fused SwiGLU, MoE combine +
+// residual + sigmoid gating, two-pass RMSNorm feeding the next layer).
+#include <cstdint>
+#include <cstring>
+
+#include <cuda_runtime.h>
+
+#include "fmoe.h"
+#include "fmoe_device.cuh"
+#include "fmoe_layout.h"
+
+namespace fmoe {
+
+constexpr int kMaxK = 8;
+constexpr int kMaxE = 1024;
+constexpr int kRouterSplit = 4;  // router rows are split in 4 along H
+constexpr int kTokChunk = 8;     // tokens per router launch
+constexpr int kThreads = 256;
+constexpr int kWarps = kThreads / 32;
+
+// ------------------------------------------------------------ router ----
+// part[t][row][s] = sum over split s of W[row] . xn[t]; row E is the shared
+// expert's gate vector (skipped when w_sg is null).  One warp per (row, split).
+__global__ void __launch_bounds__(kThreads)
+router_partial_kernel(const float* __restrict__ xn, const float* __restrict__ w_router,
+                      const float* __restrict__ w_sg, int T, int H, int E,
+                      float* __restrict__ part) {
+  const int warp = (int)((blockIdx.x * blockDim.x + threadIdx.x) >> 5);
+  const int lane = threadIdx.x & 31;
+  if (warp >= (E + (w_sg ? 1 : 0)) * kRouterSplit) return;
+  const int row = warp / kRouterSplit, sp = warp % kRouterSplit;
+  const float* w = row < E ? w_router + (size_t)row * H : w_sg;
+  const int hs = H / kRouterSplit, c0 = sp * hs;
+  float acc[kTokChunk];
+#pragma unroll
+  for (int t = 0; t < kTokChunk; ++t) acc[t] = 0.f;
+#pragma unroll 4
+  for (int c = lane * 4; c < hs; c += 128) {
+    const float4 wv = ld_stream_f4(w + c0 + c);
+#pragma unroll
+    for (int t = 0; t < kTokChunk; ++t) {
+      if (t < T) {
+        const float4 xv = __ldg(reinterpret_cast<const float4*>(xn + (size_t)t * H + c0 + c));
+        acc[t] = fmaf(wv.x, xv.x, acc[t]);
+        acc[t] = fmaf(wv.y, xv.y, acc[t]);
+        acc[t] = fmaf(wv.z, xv.z, acc[t]);
+        acc[t] = fmaf(wv.w, xv.w, acc[t]);
+      }
+    }
+  }
+#pragma unroll
+  for (int t = 0; t < kTokChunk; ++t) {
+    if (t < T) {
+      const float v = warp_sum(acc[t]);
+      if (lane == 0) part[((size_t)t * (E + 1) + row) * kRouterSplit + sp] = v;
+    }
+  }
+}
+
+// Orders (value, index): larger value first, NaN below every number, equal
+// values (including +0 / -0) to the lower index; index < 0 marks "none".
+__device__ __forceinline__ bool route_better(float av, int ai, float bv, int bi) {
+  if (ai < 0) return false;
+  if (bi < 0) return true;
+  const bool an = isnan(av), bn = isnan(bv);
+  if (an || bn) return an && bn ? ai < bi : bn;
+  if (av != bv) return av > bv;
+  return ai < bi;
+}
+
+// One warp per token: logits (sum of the splits, or given), top-k, softmax
+// over the selected logits, and the shared gate sigmoid(z).
+__global__ void __launch_bounds__(128)
+topk_kernel(const float* __restrict__ part, const float* __restrict__ logits_in, int T, int E,
+            int k, float* __restrict__ logits, int32_t* __restrict__ ids,
+            float* __restrict__ weights, float* __restrict__ gamma) {
+  __shared__ float lg[4][kMaxE];
+  const int wi = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int t = blockIdx.x * 4 + wi;
+  if (t >= T) return;
+  bool nan_seen = false;
+  for (int e = lane; e < E; e += 32) {
+    float v;
+    if (part) {
+      const float* p = part + ((size_t)t * (E + 1) + e) * kRouterSplit;
+      v = p[0];
+#pragma unroll
+      for (int s = 1; s < kRouterSplit; ++s) v += p[s];
+      logits[(size_t)t * E + e] = v;
+    } else {
+      v = logits_in[(size_t)t * E + e];
+    }
+    nan_seen |= isnan(v);
+    lg[wi][e] = v;
+  }
+  if (part && gamma && lane == 0) {
+    const float* p = part + ((size_t)t * (E + 1) + E) * kRouterSplit;
+    float z = p[0];
+#pragma unroll
+    for (int s = 1; s < kRouterSplit; ++s) z += p[s];
+    gamma[t] = 1.f / (1.f + expf(-z));
+  }
+  if (__any_sync(0xffffffffu, nan_seen) && lane == 0) raise_status(FMOE_STATUS_NAN_LOGIT);
+  __syncwarp();
+  uint32_t taken = 0;  // bit i: element lane + 32 i already selected
+  float selv[kMaxK];
+  int seli[kMaxK];
+  for (int r = 0; r < k; ++r) {
+    float bv = 0.f;
+    int bi = -1;
+    for (int i = 0, e = lane; e < E; ++i, e += 32) {
+      if (taken & (1u << i)) continue;
+      const float v = lg[wi][e];
+      if (route_better(v, e, bv, bi)) { bv = v; bi = e; }
+    }
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) {
+      const float ov = __shfl_xor_sync(0xffffffffu, bv, o);
+      const int oi = __shfl_xor_sync(0xffffffffu, bi, o);
+      if (route_better(ov, oi, bv, bi)) { bv = ov; bi = oi; }
+    }
+    if (bi >= 0 && (bi & 31) == lane) taken |= 1u << (bi >> 5);
+    selv[r] = bv;
+    seli[r] = bi;
+  }
+  float m = -INFINITY;
+  for (int r = 0; r < k; ++r)
+    if (!isnan(selv[r])) m = fmaxf(m, selv[r]);
+  float p[kMaxK];
+  float z = 0.f;
+  for (int r = 0; r < k; ++r) {
+    p[r] = isnan(selv[r]) ? 0.f : expf(selv[r] - m);
+    z += p[r];
+  }
+  if (lane < k) {
+    float pv = 0.f;
+    int iv = 0;
+    for (int r = 0; r < k; ++r)
+      if (r == lane) { pv = p[r]; iv = seli[r]; }
+    ids[(size_t)t * k + lane] = iv;
+    weights[(size_t)t * k + lane] = z > 0.f ? pv / z : 0.f;
+  }
+}
+
+// ---------------------------------------------------------- experts ----
+struct ExpertSet {
+  const uint8_t* experts;  // E records
+  const uint8_t* shared;   // one record
+  size_t rec_bytes, shared_rec_bytes;
+  int bits, shared_bits;
+  int H, I, E, k;
+};
+
+// Resolves slot j of token t to a record; returns nullptr for a bad id.
+__device__ __forceinline__ const uint8_t* slot_record(const ExpertSet& es, const int32_t* ids,
+                                                      int t, int j, int* bits) {
+  if (j == es.k) {
+    *bits = es.shared_bits;
+    return es.shared;
+  }
+  const int id = ids[(size_t)t * es.k + j];
+  *bits = es.bits;
+  if (id < 0 || id >= es.E) return nullptr;
+  return es.experts + (size_t)id * es.rec_bytes;
+}
+
+// Gate/up rows of one record for one token: each warp owns units of
+// 32 / lanes_per_row row pairs; a lane owns whole groups of both the gate and
+// the up row of its pair, so the staged x it reads serves both.
+template <int BITS>
+__device__ __forceinline__ void gateup_rows(const uint8_t* rec, const ExpertSet& es,
+                                            const StagedX& sx, float* __restrict__ a_out,
+                                            int unit0, int unit1) {
+  const int H = es.H;
+  const int ng = H / 64;
+  const int lpr = ng < 32 ? ng : 32;  // lanes per row
+  const int gpl = ng / lpr;           // groups per lane
+  const int ppu = 32 / lpr;           // row pairs per unit
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  const int ps = lane / lpr, lg = lane % lpr;
+  const RecordLayout L = record_layout(BITS, H, es.I);
+  const uint8_t* codes = rec + L.gu_codes;
+  const uint32_t* sbw = reinterpret_cast<const uint32_t*>(rec + L.gu_sb);
+  for (int u = unit0 + warp; u < unit1; u += kWarps) {
+    const int n = u * ppu + ps;
+    const uint8_t* rg = codes + (size_t)(2 * n) * L.gu_row_bytes;
+    const uint8_t* ru = rg + L.gu_row_bytes;
+    float yg = 0.f, yu = 0.f;
+    for (int m = 0; m < gpl; ++m) {
+      const int g = lg + m * lpr;
+      const GroupCodes<BITS> cg = load_group<BITS>(rg, ng, g);
+      const GroupCodes<BITS> cu = load_group<BITS>(ru, ng, g);
+      const uint32_t sg = ld_stream_u32(sbw + (size_t)(2 * n) * ng + g);
+      const uint32_t su = ld_stream_u32(sbw + (size_t)(2 * n + 1) * ng + g);
+      uint4 xv[8];
+      load_xv(sx, ng, g, xv);
+      const float d = sx.delta[g], xs = sx.xsum[g];
+      yg = group_epilogue(yg, sg, group_dot<BITS>(cg, xv), d, xs);
+      yu = group_epilogue(yu, su, group_dot<BITS>(cu, xv), d, xs);
+    }
+    for (int o = lpr >> 1; o > 0; o >>= 1) {
+      yg += __shfl_xor_sync(0xffffffffu, yg, o);
+      yu += __shfl_xor_sync(0xffffffffu, yu, o);
+    }
+    if (lg == 0) a_out[n] = silu_mul(yg, yu);
+  }
+}
+
+// Down rows of one record: units of 32 / lanes_per_row rows.
+template <int BITS>
+__device__ __forceinline__ void down_rows(const uint8_t* rec, const ExpertSet& es,
+                                          const StagedX& sx, float* __restrict__ y_out, int unit0,
+                                          int unit1) {
+  const int I = es.I;
+  const int ng = I / 64;
+  const int lpr = ng < 32 ? ng : 32;
+  const int gpl = ng / lpr;
+  const int rpu = 32 / lpr;
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  const int rs = lane / lpr, lg = lane % lpr;
+  const RecordLayout L = record_layout(BITS, es.H, I);
+  const uint8_t* codes = rec + L.down_codes;
+  const uint32_t* sbw = reinterpret_cast<const uint32_t*>(rec + L.down_sb);
+  for (int u = unit0 + warp; u < unit1; u += kWarps) {
+    const int r = u * rpu + rs;
+    const uint8_t* row = codes + (size_t)r * L.down_row_bytes;
+    float y = 0.f;
+    for (int m = 0; m < gpl; ++m) {
+      const int g = lg + m * lpr;
+      const GroupCodes<BITS> c = load_group<BITS>(row, ng, g);
+      const uint32_t sb = ld_stream_u32(sbw + (size_t)r * ng + g);
+      uint4 xv[8];
+      load_xv(sx, ng, g, xv);
+      y = group_epilogue(y, sb, group_dot<BITS>(c, xv), sx.delta[g], sx.xsum[g]);
+    }
+    for (int o = lpr >> 1; o > 0; o >>= 1) y += __shfl_xor_sync(0xffffffffu, y, o);
+    if (lg == 0) y_out[r] = y;
+  }
+}
+
+__device__ __forceinline__ void unit_range(int n_units, int* u0, int* u1) {
+  const int per = (n_units + (int)gridDim.x - 1) / (int)gridDim.x;
+  *u0 = (int)blockIdx.x * per;
+  *u1 = min(n_units, *u0 + per);
+}
+
+// grid (row blocks, T * (k + 1) slots): slot = t * (k + 1) + j, j == k the shared expert.
+__global__ void __launch_bounds__(kThreads)
+gateup_kernel(ExpertSet es, const float* __restrict__ xn, const int32_t* __restrict__ ids,
+              float* __restrict__ a, const float* __restrict__ w_sg, float* __restrict__ gamma) {
+  extern __shared__ __align__(16) unsigned char smem[];
+  const int slot = blockIdx.y, t = slot / (es.k + 1), j = slot % (es.k + 1);
+  int bits;
+  const uint8_t* rec = slot_record(es, ids, t, j, &bits);
+  const int ng = es.H / 64, lpr = ng < 32 ? ng : 32;
+  int u0, u1;
+  unit_range(es.I / (32 / lpr), &u0, &u1);
+  float* a_out = a + (size_t)slot * es.I;
+  if (!rec) {
+    if (threadIdx.x == 0 && blockIdx.x == 0) raise_status(FMOE_STATUS_BAD_EXPERT_ID);
+    for (int i = u0 * (32 / lpr) + (int)threadIdx.x; i < u1 * (32 / lpr); i += blockDim.x) a_out[i] = 0.f;
+    return;
+  }
+  const StagedX sx = staged_x_at(smem, es.H);
+  stage_x(xn + (size_t)t * es.H, es.H, sx);
+  __syncthreads();
+  if (gamma && j == es.k && blockIdx.x == 0 && threadIdx.x < 32) {
+    const float* x = xn + (size_t)t * es.H;
+    float z = 0.f;
+    for (int c = threadIdx.x * 4; c < es.H; c += 128) {
+      const float4 w = __ldg(reinterpret_cast<const float4*>(w_sg + c));
+      const float4 v = __ldg(reinterpret_cast<const float4*>(x + c));
+      z = fmaf(w.x, v.x, z);
+      z = fmaf(w.y, v.y, z);
+      z = fmaf(w.z, v.z, z);
+      z = fmaf(w.w, v.w, z);
+    }
+    z = warp_sum(z);
+    if (threadIdx.x == 0) gamma[t] = 1.f / (1.f + expf(-z));
+  }
+  if (bits == 4)
+    gateup_rows<4>(rec, es, sx, a_out, u0, u1);
+  else
+    gateup_rows<2>(rec, es, sx, a_out, u0, u1);
+}
+
+__global__ void __launch_bounds__(kThreads)
+down_kernel(ExpertSet es, const int32_t* __restrict__ ids, const float* __restrict__ a,
+            float* __restrict__ y) {
+  extern __shared__ __align__(16) unsigned char smem[];
+  const int slot = blockIdx.y, t = slot / (es.k + 1), j = slot % (es.k + 1);
+  int bits;
+  const uint8_t* rec = slot_record(es, ids, t, j, &bits);
+  const int ng = es.I / 64, lpr = ng < 32 ? ng : 32;
+  int u0, u1;
+  unit_range(es.H / (32 / lpr), &u0, &u1);
+  float* y_out = y + (size_t)slot * es.H;
+  if (!rec) {
+    for (int i = u0 * (32 / lpr) + (int)threadIdx.x; i < u1 * (32 / lpr); i += blockDim.x) y_out[i] = 0.f;
+    return;
+  }
+  const StagedX sx = staged_x_at(smem, es.I);
+  stage_x(a + (size_t)slot * es.I, es.I, sx);
+  __syncthreads();
+  if (bits == 4)
+    down_rows<4>(rec, es, sx, y_out, u0, u1);
+  else
+    down_rows<2>(rec, es, sx, y_out, u0, u1);
+}
+
+// ---------------------------------------------------------- combine ----
+__device__ __forceinline__ float block_sum(float v, float* red) {
+  v = warp_sum(v);
+  const int w = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  __syncthreads();
+  if (lane == 0) red[w] = v;
+  __syncthreads();
+  float s = 0.f;
+  for (int i = 0; i < (int)(blockDim.x >> 5); ++i) s += red[i];
+  return s;
+}
+
+// One CTA per token.
+__global__ void __launch_bounds__(kThreads)
+combine_kernel(const float* __restrict__ y, const float* __restrict__ weights,
+               const float* __restrict__ gamma, const float* h, const float* __restrict__ norm_w,
+               float eps, int k, int H, float* h_out, float* __restrict__ xn_out) {
+  __shared__ float red[kWarps];
+  const int t = blockIdx.x;
+  const float* yt = y + (size_t)t * (k + 1) * H;
+  float p[kMaxK];
+  for (int j = 0; j < k; ++j) p[j] = weights[(size_t)t * k + j];
+  const float gm = gamma[t];
+  float ss = 0.f;
+  for (int i = threadIdx.x; i < H; i += blockDim.x) {
+    float v = h[(size_t)t * H + i];
+    for (int j = 0; j < k; ++j) v = fmaf(p[j], yt[(size_t)j * H + i], v);
+    v = fmaf(gm, yt[(size_t)k * H + i], v);
+    h_out[(size_t)t * H + i] = v;
+    ss = fmaf(v, v, ss);
+  }
+  ss = block_sum(ss, red);
+  const float r = 1.f / sqrtf(ss / (float)H + eps);
+  for (int i = threadIdx.x; i < H; i += blockDim.x)
+    xn_out[(size_t)t * H + i] = h_out[(size_t)t * H + i] * r * norm_w[i];
+}
+
+// ------------------------------------------------------- device packer ----
+// One thread per 16-byte code chunk of a packed row.  Packed row pr of an
+// expert: pr < 2I are the interleaved gate/up rows (pr = 2n + m: logical
+// matrix m, row n; H inputs), then H down rows (I inputs).
+template <int BITS>
+__global__ void pack_codes_kernel(const uint8_t* __restrict__ q, int n_experts, int H, int I,
+                                  uint8_t* __restrict__ out) {
+  const RecordLayout L = record_layout(BITS, H, I);
+  const size_t n = (size_t)H * I;
+  const int gu_chunks = H * BITS / 128, dn_chunks = I * BITS / 128;
+  const size_t per_expert = (size_t)2 * I * gu_chunks + (size_t)H * dn_chunks;
+  const size_t total = per_expert * n_experts;
+  for (size_t c = blockIdx.x * (size_t)blockDim.x + threadIdx.x; c < total; c += (size_t)gridDim.x * blockDim.x) {
+    const size_t e = c / per_expert;
+    size_t r = c % per_expert;
+    int K, p;
+    const uint8_t* src;
+    uint8_t* dst;
+    if (r < (size_t)2 * I * gu_chunks) {
+      const int pr = (int)(r / gu_chunks);
+      p = (int)(r % gu_chunks);
+      K = H;
+      src = q + e * 3 * n + (size_t)(pr & 1) * n + (size_t)(pr >> 1) * H;
+      dst = out + e * L.bytes + L.gu_codes + (size_t)pr * L.gu_row_bytes;
+    } else {
+      r -= (size_t)2 * I * gu_chunks;
+      const int row = (int)(r / dn_chunks);
+      p = (int)(r % dn_chunks);
+      K = I;
+      src = q + e * 3 * n + 2 * n + (size_t)row * I;
+      dst = out + e * L.bytes + L.down_codes + (size_t)row * L.down_row_bytes;
+    }
+    const int ng = K / 64;
+    int g, h;
+    if (BITS == 2) {
+      g = p;
+      h = 0;
+    } else {
+      const int seg = ng < 32 ? ng : 32;
+      const int s = p / (2 * seg), rem = p % (2 * seg);
+      h = rem / seg;
+      g = s * seg + rem % seg;
+    }
+    const uint8_t* in = src + g * 64 + h * 32;  // h is 0 for 2-bit
+    constexpr int per_word = 32 / BITS, per_byte = 8 / BITS;
+    uint32_t words[4];
+    bool bad = false;
+#pragma unroll
+    for (int w = 0; w < 4; ++w) {
+      uint32_t word = 0;
+#pragma unroll
+      for (int a = 0; a < 4; ++a)
+#pragma unroll
+        for (int b = 0; b < per_byte; ++b) {
+          const uint32_t v = in[w * per_word + 4 * b + a];
+          bad |= v >= (1u << BITS);
+          word |= (v & ((1u << BITS) - 1u)) << ((per_byte * a + b) * BITS);
+        }
+      words[w] = bad ? 0u : word;
+    }
+    if (bad) raise_status(FMOE_STATUS_BAD_PACK_INPUT);
+    *reinterpret_cast<uint4*>(dst + (size_t)p * 16) = make_uint4(words[0], words[1], words[2], words[3]);
+  }
+}
+
+// One thread per scale-bias word.
+__global__ void pack_sb_kernel(const uint16_t* __restrict__ scale, const uint16_t* __restrict__ bias,
+                               int bits, int n_experts, int H, int I, uint8_t* __restrict__ out) {
+  const RecordLayout L = record_layout(bits, H, I);
+  const size_t ng = (size_t)3 * H * I / 64;
+  const size_t gu = (size_t)2 * I * (H / 64);
+  const int shift = bits == 4 ? 4 : 6;
+  for (size_t c = blockIdx.x * (size_t)blockDim.x + threadIdx.x; c < ng * n_experts; c += (size_t)gridDim.x * blockDim.x) {
+    const size_t e = c / ng, r = c % ng;
+    size_t src;  // logical index within the expert
+    uint32_t* dst;
+    if (r < gu) {
+      const size_t gpr = H / 64, pr = r / gpr, g = r % gpr;
+      src = (pr & 1) * ((size_t)I * gpr) + (pr >> 1) * gpr + g;
+      dst = reinterpret_cast<uint32_t*>(out + e * L.bytes + L.gu_sb) + r;
+    } else {
+      src = r;
+      dst = reinterpret_cast<uint32_t*>(out + e * L.bytes + L.down_sb) + (r - gu);
+    }
+    const uint16_t sv = scale[e * ng + src], bv = bias[e * ng + src];
+    // exact scaling by 2^-shift of a bf16 value (normal, finite, no underflow)
+    const uint32_t ex = (sv >> 7) & 0xFFu;
+    uint16_t ps;
+    bool ok = true;
+    if ((sv & 0x7FFFu) == 0) ps = sv;
+    else if (ex == 0 || ex == 0xFFu || (int)ex - shift <= 0) { ps = 0; ok = false; }
+    else ps = (uint16_t)((sv & 0x807Fu) | ((ex - shift) << 7));
+    if (!ok) raise_status(FMOE_STATUS_BAD_PACK_INPUT);
+    *dst = ok ? ((uint32_t)ps | ((uint32_t)bv << 16)) : 0u;
+  }
+}
+
+// ------------------------------------------------------- host helpers ----
+struct WsLayout {
+  size_t part, logits, ids, weights, gamma, a, y, bytes;
+};
+
+static inline size_t align_up(size_t v, size_t a) { return (v + a - 1) / a * a; }
+
+static WsLayout ws_layout(int H, int I, int E, int k, int T) {
+  WsLayout w;
+  size_t o = 256;  // reserved
+  w.part = o;
+  o = align_up(o + (size_t)T * (E + 1) * kRouterSplit * 4, 256);
+  w.logits = o;
+  o = align_up(o + (size_t)T * E * 4, 256);
+  w.ids = o;
+  o = align_up(o + (size_t)T * k * 4, 256);
+  w.weights = o;
+  o = align_up(o + (size_t)T * k * 4, 256);
+  w.gamma = o;
+  o = align_up(o + (size_t)T * 4, 256);
+  w.a = o;
+  o = align_up(o + (size_t)T * (k + 1) * I * 4, 256);
+  w.y = o;
+  o = align_up(o + (size_t)T * (k + 1) * H * 4, 256);
+  w.bytes = o;
+  return w;
+}
+
+static inline bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+static bool desc_valid(const fmoe_layer_desc* d) {
+  return d && d->hidden > 0 && d->inter > 0 && d->n_experts >= 1 && d->n_experts <= kMaxE &&
+         d->top_k >= 1 && d->top_k <= kMaxK && d->top_k <= d->n_experts && d->eps >= 0.f;
+}
+
+static bool desc_supported(const fmoe_layer_desc* d) {
+  return shape_supported(d->bits, d->hidden, d->inter, d->group) &&
+         shape_supported(d->shared_bits, d->hidden, d->inter, d->group);
+}
+
+static int weights_check(const fmoe_layer_weights* lw) {
+  if (!lw || !desc_valid(&lw->desc)) return FMOE_ERR_INVALID_ARG;
+  if (!desc_supported(&lw->desc)) return FMOE_ERR_UNSUPPORTED;
+  const void* ps[] = {lw->experts, lw->shared, lw->w_router, lw->w_shared_gate, lw->norm_w};
+  for (const void* p : ps)
+    if (!p || !aligned16(p)) return FMOE_ERR_INVALID_ARG;
+  return FMOE_OK;
+}
+
+static ExpertSet expert_set(const fmoe_layer_weights* lw) {
+  const fmoe_layer_desc& d = lw->desc;
+  ExpertSet es;
+  es.experts = static_cast<const uint8_t*>(lw->experts);
+  es.shared = static_cast<const uint8_t*>(lw->shared);
+  es.rec_bytes = record_layout(d.bits, d.hidden, d.inter).bytes;
+  es.shared_rec_bytes = record_layout(d.shared_bits, d.hidden, d.inter).bytes;
+  es.bits = d.bits;
+  es.shared_bits = d.shared_bits;
+  es.H = d.hidden;
+  es.I = d.inter;
+  es.E = d.n_experts;
+  es.k = d.top_k;
+  return es;
+}
+
+static inline int cuda_rc(cudaError_t e) { return e == cudaSuccess ? FMOE_OK : FMOE_ERR_CUDA; }
+
+static int launch_router(const float* xn, const float* w_router, const float* w_sg, int T, int H,
+                         int E, float* part, cudaStream_t st) {
+  const int warps = (E + (w_sg ? 1 : 0)) * kRouterSplit;
+  const int blocks = (warps + kWarps - 1) / kWarps;
+  for (int t0 = 0; t0 < T; t0 += kTokChunk) {
+    const int nt = T - t0 < kTokChunk ? T - t0 : kTokChunk;
+    router_partial_kernel<<<blocks, kThreads, 0, st>>>(xn + (size_t)t0 * H, w_router, w_sg, nt, H, E,
+                                                      part + (size_t)t0 * (E + 1) * kRouterSplit);
+  }
+  return cuda_rc(cudaGetLastError());
+}
+
+static int launch_topk(const float* part, const float* logits_in, int T, int E, int k, float* logits,
+                       int32_t* ids, float* weights, float* gamma, cudaStream_t st) {
+  topk_kernel<<<(T + 3) / 4, 128, 0, st>>>(part, logits_in, T, E, k, logits, ids, weights, gamma);
+  return cuda_rc(cudaGetLastError());
+}
+
+static int launch_experts(const ExpertSet& es, const float* xn, const int32_t* ids, int T, float* a,
+                          float* y, const float* w_sg, float* gamma, cudaStream_t st) {
+  const int slots = T * (es.k + 1);
+  {
+    const int ng = es.H / 64, lpr = ng < 32 ? ng : 32;
+    const int units = es.I / (32 / lpr);
+    int blocks = (units + 2 * kWarps - 1) / (2 * kWarps);
+    const size_t smem = staged_x_bytes(es.H);
+    gateup_kernel<<<dim3(blocks, slots), kThreads, smem, st>>>(es, xn, ids, a, w_sg, gamma);
+  }
+  {
+    const int ng = es.I / 64, lpr = ng < 32 ? ng : 32;
+    const int units = es.H / (32 / lpr);
+    int blocks = (units + 4 * kWarps - 1) / (4 * kWarps);
+    const size_t smem = staged_x_bytes(es.I);
+    down_kernel<<<dim3(blocks, slots), kThreads, smem, st>>>(es, ids, a, y);
+  }
+  return cuda_rc(cudaGetLastError());
+}
+
+static int launch_combine(const float* y, const float* weights, const float* gamma, const float* h,
+                          const float* norm_w, float eps, int T, int k, int H, float* h_out,
+                          float* xn_out, cudaStream_t st) {
+  combine_kernel<<<T, kThreads, 0, st>>>(y, weights, gamma, h, norm_w, eps, k, H, h_out, xn_out);
+  return cuda_rc(cudaGetLastError());
+}
+
+static int layer_forward_impl(const fmoe_layer_weights* lw, const float* logits_in, float* h,
+                              float* xn, int T, void* ws, size_t ws_bytes, cudaStream_t st) {
+  int rc = weights_check(lw);
+  if (rc != FMOE_OK) return rc;
+  const fmoe_layer_desc& d = lw->desc;
+  if (T < 1 || !h || !xn || !ws || !aligned16(h) || !aligned16(xn) || !aligned16(ws))
+    return FMOE_ERR_INVALID_ARG;
+  if (logits_in && !aligned16(logits_in)) return FMOE_ERR_INVALID_ARG;
+  const WsLayout w = ws_layout(d.hidden, d.inter, d.n_experts, d.top_k, T);
+  if (ws_bytes < w.bytes) return FMOE_ERR_BUFFER_TOO_SMALL;
+  unsigned char* base = static_cast<unsigned char*>(ws);
+  float* part = reinterpret_cast<float*>(base + w.part);
+  float* logits = reinterpret_cast<float*>(base + w.logits);
+  int32_t* ids = reinterpret_cast<int32_t*>(base + w.ids);
+  float* weights = reinterpret_cast<float*>(base + w.weights);
+  float* gamma = reinterpret_cast<float*>(base + w.gamma);
+  float* a = reinterpret_cast<float*>(base + w.a);
+  float* y = reinterpret_cast<float*>(base + w.y);
+  const ExpertSet es = expert_set(lw);
+  if (logits_in) {
+    // given routing: top-k on the given logits; the shared gate is computed
+    // by the gate/up kernel
+    rc = cuda_rc(cudaMemcpyAsync(logits, logits_in, (size_t)T * d.n_experts * 4, cudaMemcpyDeviceToDevice, st));
+    if (rc == FMOE_OK) rc = launch_topk(nullptr, logits, T, d.n_experts, d.top_k, logits, ids, weights, nullptr, st);
+  } else {
+    rc = launch_router(xn, lw->w_router, lw->w_shared_gate, T, d.hidden, d.n_experts, part, st);
+    if (rc == FMOE_OK) rc = launch_topk(part, nullptr, T, d.n_experts, d.top_k, logits, ids, weights, gamma, st);
+  }
+  if (rc != FMOE_OK) return rc;
+  rc = launch_experts(es, xn, ids, T, a, y, lw->w_shared_gate, logits_in ? gamma : nullptr, st);
+  if (rc != FMOE_OK) return rc;
+  return launch_combine(y, weights, gamma, h, lw->norm_w, d.eps, T, d.top_k, d.hidden, h, xn, st);
+}
+
+}  // namespace fmoe
+
+using namespace fmoe;
+
+extern "C" const char* fmoe_error_string(int status) {
+  switch (status) {
+    case FMOE_OK: return "ok";
+    case FMOE_ERR_INVALID_ARG: return "invalid argument";
+    case FMOE_ERR_UNSUPPORTED: return "unsupported shape or bit width";
+    case FMOE_ERR_CUDA: return "CUDA runtime error";
+    case FMOE_ERR_DEVICE_STATUS: return "device status word set";
+    case FMOE_ERR_BUFFER_TOO_SMALL: return "buffer too small";
+    default: return "unknown status";
+  }
+}
+
+extern "C" int fmoe_read_status(uint32_t* status, int clear) {
+  if (!status) return FMOE_ERR_INVALID_ARG;
+  if (cudaDeviceSynchronize() != cudaSuccess) return FMOE_ERR_CUDA;
+  if (cudaMemcpyFromSymbol(status, g_status, sizeof(uint32_t)) != cudaSuccess) return FMOE_ERR_CUDA;
+  if (clear) {
+    const uint32_t zero = 0;
+    if (cudaMemcpyToSymbol(g_status, &zero, sizeof(uint32_t)) != cudaSuccess) return FMOE_ERR_CUDA;
+  }
+  return FMOE_OK;
+}
+
+extern "C" size_t fmoe_workspace_bytes(const fmoe_layer_desc* d, int T) {
+  if (!desc_valid(d) || T < 1) return 0;
+  return ws_layout(d->hidden, d->inter, d->n_experts, d->top_k, T).bytes;
+}
+
+extern "C" int fmoe_workspace_init(void* d_ws, size_t ws_bytes, cudaStream_t stream) {
+  if (!d_ws || !aligned16(d_ws)) return FMOE_ERR_INVALID_ARG;
+  return cuda_rc(cudaMemsetAsync(d_ws, 0, ws_bytes, stream));
+}
+
+extern "C" size_t fmoe_workspace_offset(const fmoe_layer_desc* d, int T, int which) {
+  if (!desc_valid(d) || T < 1) return (size_t)-1;
+  const WsLayout w = ws_layout(d->hidden, d->inter, d->n_experts, d->top_k, T);
+  switch (which) {
+    case 0: return w.logits;
+    case 1: return w.ids;
+    case 2: return w.weights;
+    case 3: return w.gamma;
+    case 4: return w.a;
+    case 5: return w.y;
+    default: return (size_t)-1;
+  }
+}
+
+extern "C" int fmoe_route_topk(const float* d_xn, const float* d_w_router, int T, int H, int E, int k,
+                               unsigned flags, float* d_logits, int32_t* d_ids, float* d_weights,
+                               void* d_ws, size_t ws_bytes, cudaStream_t stream) {
+  const bool given = (flags & FMOE_LOGITS_GIVEN) != 0;
+  if (T < 1 || H < 64 || H % 64 || E < 1 || k < 1 || k > E) return FMOE_ERR_INVALID_ARG;
+  if (k > kMaxK || E > kMaxE) return FMOE_ERR_UNSUPPORTED;
+  if (!d_logits || !d_ids || !d_weights || !aligned16(d_logits) || !aligned16(d_ids) || !aligned16(d_weights))
+    return FMOE_ERR_INVALID_ARG;
+  if (given) return launch_topk(nullptr, d_logits, T, E, k, d_logits, d_ids, d_weights, nullptr, stream);
+  if (!d_xn || !d_w_router || !d_ws || !aligned16(d_xn) || !aligned16(d_w_router) || !aligned16(d_ws))
+    return FMOE_ERR_INVALID_ARG;
+  const WsLayout w = ws_layout(H, 64, E, k, T);
+  if (ws_bytes < w.part + (size_t)T * (E + 1) * kRouterSplit * 4) return FMOE_ERR_BUFFER_TOO_SMALL;
+  float* part = reinterpret_cast<float*>(static_cast<unsigned char*>(d_ws) + w.part);
+  int rc = launch_router(d_xn, d_w_router, nullptr, T, H, E, part, stream);
+  if (rc != FMOE_OK) return rc;
+  return launch_topk(part, nullptr, T, E, k, d_logits, d_ids, d_weights, nullptr, stream);
+}
+
+extern "C" int fmoe_expert_forward(const fmoe_layer_weights* lw, const float* d_xn, int T,
+                                   const int32_t* d_ids, int k, float* d_y, float* d_gamma,
+                                   void* d_ws, size_t ws_bytes, cudaStream_t stream) {
+  int rc = weights_check(lw);
+  if (rc != FMOE_OK) return rc;
+  const fmoe_layer_desc& d = lw->desc;
+  if (T < 1 || k != d.top_k) return FMOE_ERR_INVALID_ARG;
+  const void* ps[] = {d_xn, d_ids, d_y, d_gamma, d_ws};
+  for (const void* p : ps)
+    if (!p || !aligned16(p)) return FMOE_ERR_INVALID_ARG;
+  const WsLayout w = ws_layout(d.hidden, d.inter, d.n_experts, d.top_k, T);
+  if (ws_bytes < w.bytes) return FMOE_ERR_BUFFER_TOO_SMALL;
+  float* a = reinterpret_cast<float*>(static_cast<unsigned char*>(d_ws) + w.a);
+  return launch_experts(expert_set(lw), d_xn, d_ids, T, a, d_y, lw->w_shared_gate, d_gamma, stream);
+}
+
+extern "C" int fmoe_combine_residual_rmsnorm(const float* d_y, const float* d_weights,
+                                             const float* d_gamma, const float* d_h,
+                                             const float* d_norm_w, float eps, int T, int k, int H,
+                                             float* d_h_out, float* d_xn_out, cudaStream_t stream) {
+  if (T < 1 || k < 1 || k > kMaxK || H < 1 || eps < 0.f) return FMOE_ERR_INVALID_ARG;
+  const void* ps[] = {d_y, d_weights, d_gamma, d_h, d_norm_w, d_h_out, d_xn_out};
+  for (const void* p : ps)
+    if (!p || !aligned16(p)) return FMOE_ERR_INVALID_ARG;
+  if (d_xn_out == d_h || d_xn_out == d_y) return FMOE_ERR_INVALID_ARG;
+  return launch_combine(d_y, d_weights, d_gamma, d_h, d_norm_w, eps, T, k, H, d_h_out, d_xn_out, stream);
+}
+
+extern "C" int fmoe_layer_forward(const fmoe_layer_weights* lw, float* d_h, float* d_xn, int T,
+                                  void* d_ws, size_t ws_bytes, cudaStream_t stream) {
+  return layer_forward_impl(lw, nullptr, d_h, d_xn, T, d_ws, ws_bytes, stream);
+}
+
+extern "C" int fmoe_layer_forward_logits(const fmoe_layer_weights* lw, const float* d_logits,
+                                         float* d_h, float* d_xn, int T, void* d_ws,
+                                         size_t ws_bytes, cudaStream_t stream) {
+  if (!d_logits) return FMOE_ERR_INVALID_ARG;
+  return layer_forward_impl(lw, d_logits, d_h, d_xn, T, d_ws, ws_bytes, stream);
+}
+
+extern "C" int fmoe_pack_experts_device(const uint8_t* d_q, const uint16_t* d_scale,
+                                        const uint16_t* d_bias, int bits, int n_experts, int hidden,
+                                        int inter, int group, void* d_packed, size_t d_bytes,
+                                        cudaStream_t stream) {
+  if (!d_q || !d_scale || !d_bias || !d_packed || n_experts < 1) return FMOE_ERR_INVALID_ARG;
+  const void* ps[] = {d_q, d_scale, d_bias, d_packed};
+  for (const void* p : ps)
+    if (!aligned16(p)) return FMOE_ERR_INVALID_ARG;
+  if (!shape_supported(bits, hidden, inter, group)) return FMOE_ERR_UNSUPPORTED;
+  const RecordLayout L = record_layout(bits, hidden, inter);
+  if (d_bytes < L.bytes * (size_t)n_experts) return FMOE_ERR_BUFFER_TOO_SMALL;
+  const unsigned blocks = 148u * 16u;
+  uint8_t* out = static_cast<uint8_t*>(d_packed);
+  if (bits == 4)
+    pack_codes_kernel<4><<<blocks, 256, 0, stream>>>(d_q, n_experts, hidden, inter, out);
+  else
+    pack_codes_kernel<2><<<blocks, 256, 0, stream>>>(d_q, n_experts, hidden, inter, out);
+  pack_sb_kernel<<<blocks, 256, 0, stream>>>(d_scale, d_bias, bits, n_experts, hidden, inter, out);
+  return cuda_rc(cudaGetLastError());
+}
+
+extern "C" int fmoe_stack_forward(const fmoe_layer_weights* layers, int n_layers, float* d_h,
+                                  float* d_xn, int T, void* d_ws, size_t ws_bytes,
+                                  cudaStream_t stream) {
+  if (!layers || n_layers < 1) return FMOE_ERR_INVALID_ARG;
+  for (int l = 0; l < n_layers; ++l) {
+    const int rc = fmoe_layer_forward(&layers[l], d_h, d_xn, T, d_ws, ws_bytes, stream);
+    if (rc != FMOE_OK) return rc;
+  }
+  return FMOE_OK;
+}

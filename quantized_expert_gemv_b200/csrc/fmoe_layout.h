@@ -1,0 +1,58 @@
+// fmoe_layout.h -- packed expert record geometry (host and device).
+//
+// One record per expert, sections 16-byte aligned:
+//   [gate/up codes: I row pairs x 2 rows x H*bits/8 bytes]
+//   [down codes:    H rows x I*bits/8 bytes]
+//   [gate/up scale-bias: I x 2 rows x H/64 words]
+//   [down scale-bias:    H rows x I/64 words]
+// The per-row chunk order and the code permutation inside a word are
+// described in include/fmoe.h.
+#pragma once
+
+#include <stddef.h>
+#include <stdint.h>
+
+#if defined(__CUDACC__)
+#define FMOE_HD __host__ __device__ __forceinline__
+#else
+#define FMOE_HD inline
+#endif
+
+namespace fmoe {
+
+struct RecordLayout {
+  size_t gu_row_bytes;    // bytes of one gate or up row (H codes)
+  size_t down_row_bytes;  // bytes of one down row (I codes)
+  size_t gu_codes;        // offsets of the four sections
+  size_t down_codes;
+  size_t gu_sb;
+  size_t down_sb;
+  size_t bytes;           // record size
+};
+
+FMOE_HD RecordLayout record_layout(int bits, int H, int I) {
+  RecordLayout L;
+  L.gu_row_bytes = (size_t)H * bits / 8;
+  L.down_row_bytes = (size_t)I * bits / 8;
+  L.gu_codes = 0;
+  L.down_codes = L.gu_codes + (size_t)I * 2 * L.gu_row_bytes;
+  L.gu_sb = L.down_codes + (size_t)H * L.down_row_bytes;
+  L.down_sb = L.gu_sb + (size_t)I * 2 * (H / 64) * 4;
+  L.bytes = L.down_sb + (size_t)H * (I / 64) * 4;
+  return L;
+}
+
+// A row of K inputs is handled by min(32, K/64) lanes, each owning whole
+// groups; so K/64 must be a power of two up to 32, or a multiple of 32.
+FMOE_HD bool width_supported(int K) {
+  if (K < 64 || K % 64) return false;
+  const int ng = K / 64;
+  if (ng >= 32) return ng % 32 == 0;
+  return (ng & (ng - 1)) == 0;
+}
+
+FMOE_HD bool shape_supported(int bits, int H, int I, int group) {
+  return (bits == 4 || bits == 2) && group == 64 && width_supported(H) && width_supported(I);
+}
+
+}  // namespace fmoe

@@ -47,14 +47,27 @@ K_GUMBEL = 15
 K_RESID = 16
 
 
-def build(force: bool = False) -> str:
-    """Compile libsynth.so with gcc (plain C, no GPU code)."""
+_DEV_LIB_PATH = os.path.join(_HERE, "libsynth_cuda.so")
+
+
+def build(force: bool = False, device: bool = True) -> str:
+    """Compile libsynth.so with gcc (plain C) and, when `device`, its CUDA twin
+    libsynth_cuda.so with nvcc (sm_100a)."""
     src = os.path.join(_HERE, "synth.c")
     if force or not os.path.exists(_LIB_PATH) or os.path.getmtime(_LIB_PATH) < os.path.getmtime(src):
         subprocess.check_call(
-            ["gcc", "-O2", "-fPIC", "-shared", "-std=c11", src, "-lm", "-o", _LIB_PATH + ".tmp"]
+            ["gcc", "-O2", "-fPIC", "-shared", "-std=c11", "-ffp-contract=off", src, "-lm",
+             "-o", _LIB_PATH + ".tmp"]
         )
         os.replace(_LIB_PATH + ".tmp", _LIB_PATH)
+    dsrc = os.path.join(_HERE, "synth_device.cu")
+    if device and (force or not os.path.exists(_DEV_LIB_PATH)
+                   or os.path.getmtime(_DEV_LIB_PATH) < os.path.getmtime(dsrc)):
+        nvcc = "/usr/local/cuda/bin/nvcc" if os.path.exists("/usr/local/cuda/bin/nvcc") else "nvcc"
+        subprocess.check_call([nvcc, "-gencode", "arch=compute_100a,code=sm_100a", "-O3", "-std=c++17",
+                               "--shared", "-Xcompiler", "-fPIC", "-fmad=false", dsrc,
+                               "-o", _DEV_LIB_PATH + ".tmp"])
+        os.replace(_DEV_LIB_PATH + ".tmp", _DEV_LIB_PATH)
     return _LIB_PATH
 
 
@@ -64,7 +77,7 @@ _lib = None
 def lib() -> ctypes.CDLL:
     global _lib
     if _lib is None:
-        build()
+        build(device=False)
         L = ctypes.CDLL(_LIB_PATH)
         u64, i32, dbl, vp = ctypes.c_uint64, ctypes.c_int, ctypes.c_double, ctypes.c_void_p
         L.synth_key.restype = u64

@@ -1,0 +1,166 @@
+"""C ABI: the library loads, exports what include/fmoe.h declares, packs and
+unpacks bit-exactly, and rejects bad arguments on the host before launching
+anything (none of these tests needs a GPU)."""
+import ctypes
+import os
+import re
+
+import numpy as np
+import pytest
+
+import synth
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+@pytest.fixture(scope="module")
+def fm():
+    from quantized_expert_gemv_b200 import build
+    build.build()
+    import quantized_expert_gemv_b200 as m
+    return m
+
+
+def declared_symbols():
+    out = set()
+    for name in os.listdir(os.path.join(ROOT, "include")):
+        if name.endswith(".h"):
+            src = open(os.path.join(ROOT, "include", name)).read()
+            src = re.sub(r"/\*.*?\*/", "", src, flags=re.S)
+            out |= set(re.findall(r"\b(fmoe_\w+)\s*\(", src))
+    return out
+
+
+def test_every_declared_symbol_is_exported(fm):
+    lib = ctypes.CDLL(fm.LIBRARY_PATH)
+    syms = declared_symbols()
+    assert len(syms) >= 15
+    for s in syms:
+        assert hasattr(lib, s), s
+    assert syms <= set(fm.EXPORTED) | {"fmoe_error_string"}
+
+
+def test_packed_bytes_closed_form(fm):
+    assert fm.fmoe_packed_bytes(4, 1, 4096, 1024) == 7_077_888  # 6.75 MiB
+    assert fm.fmoe_packed_bytes(2, 1, 4096, 1024) == 3_932_160  # 3.75 MiB
+    assert fm.fmoe_packed_bytes(4, 512, 4096, 1024) == 512 * 7_077_888
+    assert fm.fmoe_packed_bytes(4, 1, 256, 128) == 3 * 256 * 128 // 2 + 3 * 256 * 128 // 64 * 4
+    # unsupported: group != 64, width not a multiple of 64, 48 groups, bits 3
+    assert fm.fmoe_packed_bytes(4, 1, 4096, 1024, group=128) == 0
+    assert fm.fmoe_packed_bytes(4, 1, 4000, 1024) == 0
+    assert fm.fmoe_packed_bytes(4, 1, 3072, 1024) == 0
+    assert fm.fmoe_packed_bytes(3, 1, 4096, 1024) == 0
+
+
+@pytest.mark.parametrize("bits,H,I", [(4, 256, 128), (2, 256, 128), (4, 4096, 1024), (2, 4096, 1024),
+                                      (4, 64, 2048), (2, 128, 64)])
+def test_pack_unpack_round_trip(fm, bits, H, I):
+    wl = synth.Workload(hidden=H, inter=I, n_experts=3, bits=bits, seed=7 + bits)
+    exs = [synth.expert(wl, 1, e) for e in range(2)]
+    q = np.concatenate([e.q for e in exs])
+    s = np.concatenate([e.scale for e in exs])
+    b = np.concatenate([e.bias for e in exs])
+    packed = fm.fmoe_pack_experts_host(q, s, b, bits, 2, H, I)
+    assert packed.nbytes == fm.fmoe_packed_bytes(bits, 2, H, I)
+    q2, s2, b2 = fm.fmoe_unpack_experts_host(packed, bits, 2, H, I)
+    assert np.array_equal(q2, q) and np.array_equal(s2, s) and np.array_equal(b2, b)
+
+
+@pytest.mark.parametrize("bits", [4, 2])
+def test_pack_extreme_codes(fm, bits):
+    H, I = 128, 64
+    n, ng = 3 * H * I, 3 * H * I // 64
+    for fill in (0, (1 << bits) - 1):
+        q = np.full(n, fill, np.uint8)
+        s = np.full(ng, 0x3C00, np.uint16)  # 2^-7
+        b = np.full(ng, 0xBF80, np.uint16)  # -1
+        packed = fm.fmoe_pack_experts_host(q, s, b, bits, 1, H, I)
+        q2, s2, b2 = fm.fmoe_unpack_experts_host(packed, bits, 1, H, I)
+        assert np.array_equal(q2, q) and np.array_equal(s2, s) and np.array_equal(b2, b)
+
+
+def test_packed_word_permutation(fm):
+    """Inputs 0..7 of a 4-bit row land in the documented fields: field 2a+b
+    of the first word holds input 4b+a."""
+    H, I = 64, 64
+    n, ng = 3 * H * I, 3 * H * I // 64
+    q = np.zeros(n, np.uint8)
+    q[:8] = [1, 2, 3, 4, 5, 6, 7, 8]  # gate row 0, inputs 0..7
+    s = np.full(ng, 0x3F80, np.uint16)
+    b = np.zeros(ng, np.uint16)
+    packed = fm.fmoe_pack_experts_host(q, s, b, 4, 1, H, I)
+    word = int(packed[:4].view(np.uint32)[0])
+    fields = [(word >> (4 * p)) & 0xF for p in range(8)]
+    for a in range(4):
+        for bb in range(2):
+            assert fields[2 * a + bb] == q[4 * bb + a]
+    # scale is stored pre-multiplied by 2^-4: 1.0 -> 0x3D80
+    sb_off = 2 * 64 * H * 4 // 8 + H * I * 4 // 8
+    assert int(packed[sb_off:sb_off + 4].view(np.uint32)[0]) & 0xFFFF == 0x3D80
+
+
+def test_packer_rejects_bad_input(fm):
+    H, I = 64, 64
+    n, ng = 3 * H * I, 3 * H * I // 64
+    q = np.zeros(n, np.uint8)
+    s = np.full(ng, 0x3F80, np.uint16)
+    b = np.zeros(ng, np.uint16)
+    q[5] = 16  # out of range for 4-bit
+    with pytest.raises(fm.FmoeError) as e:
+        fm.fmoe_pack_experts_host(q, s, b, 4, 1, H, I)
+    assert e.value.status == fm.FMOE_ERR_INVALID_ARG
+    q[5] = 4
+    with pytest.raises(fm.FmoeError):
+        fm.fmoe_pack_experts_host(q, s, b, 2, 1, H, I)  # 4 > 3 for 2-bit
+    s[3] = 0x0001  # subnormal scale cannot be pre-scaled exactly
+    q[5] = 0
+    with pytest.raises(fm.FmoeError):
+        fm.fmoe_pack_experts_host(q, s, b, 4, 1, H, I)
+    with pytest.raises(fm.FmoeError) as e:
+        fm.fmoe_pack_experts_host(q, s, b, 4, 1, 96, 64)
+    assert e.value.status == fm.FMOE_ERR_UNSUPPORTED
+
+
+def test_host_validation_before_launch(fm):
+    """Bad arguments are refused on the host (no CUDA call is made, so this
+    runs without a GPU)."""
+    L = fm._lib
+    assert L.fmoe_layer_forward(None, None, None, 1, None, 0, None) == fm.FMOE_ERR_INVALID_ARG
+    d = fm.LayerDesc(hidden=256, inter=128, n_experts=16, top_k=4)
+    w = fm.fmoe_layer_weights(d.c(), 16, 16, 16, 16, 16)
+    # null activation pointers
+    assert L.fmoe_layer_forward(ctypes.byref(w), None, None, 1, 16, 1 << 30, None) == fm.FMOE_ERR_INVALID_ARG
+    # misaligned workspace
+    assert L.fmoe_layer_forward(ctypes.byref(w), 16, 16, 1, 17, 1 << 30, None) == fm.FMOE_ERR_INVALID_ARG
+    # workspace too small
+    assert L.fmoe_layer_forward(ctypes.byref(w), 16, 16, 1, 16, 64, None) == fm.FMOE_ERR_BUFFER_TOO_SMALL
+    # k > 8, k > E, E > 1024, T < 1
+    for bad in (dict(top_k=9, n_experts=16), dict(top_k=5, n_experts=4), dict(n_experts=2048)):
+        dd = fm.LayerDesc(hidden=256, inter=128, **{**dict(n_experts=16, top_k=4), **bad})
+        ww = fm.fmoe_layer_weights(dd.c(), 16, 16, 16, 16, 16)
+        assert L.fmoe_layer_forward(ctypes.byref(ww), 16, 16, 1, 16, 1 << 30, None) == fm.FMOE_ERR_INVALID_ARG
+    assert L.fmoe_layer_forward(ctypes.byref(w), 16, 16, 0, 16, 1 << 30, None) == fm.FMOE_ERR_INVALID_ARG
+    # unsupported shapes / bits
+    for bad in (dict(hidden=96), dict(inter=3072), dict(bits=3), dict(shared_bits=8), dict(group=32)):
+        dd = fm.LayerDesc(**{**dict(hidden=256, inter=128, n_experts=16, top_k=4), **bad})
+        ww = fm.fmoe_layer_weights(dd.c(), 16, 16, 16, 16, 16)
+        assert L.fmoe_layer_forward(ctypes.byref(ww), 16, 16, 1, 16, 1 << 30, None) == fm.FMOE_ERR_UNSUPPORTED
+    # expert forward: k mismatch
+    assert L.fmoe_expert_forward(ctypes.byref(w), 16, 1, 16, 3, 16, 16, 16, 1 << 30, None) == fm.FMOE_ERR_INVALID_ARG
+    # route: k > 8 unsupported, null outputs invalid
+    assert L.fmoe_route_topk(16, 16, 1, 256, 16, 9, 0, 16, 16, 16, 16, 1 << 20, None) == fm.FMOE_ERR_UNSUPPORTED
+    assert L.fmoe_route_topk(16, 16, 1, 256, 16, 4, 0, None, 16, 16, 16, 1 << 20, None) == fm.FMOE_ERR_INVALID_ARG
+    # combine: output aliasing its inputs
+    assert L.fmoe_combine_residual_rmsnorm(16, 16, 16, 32, 16, ctypes.c_float(1e-6), 1, 4, 256, 32, 32,
+                                           None) == fm.FMOE_ERR_INVALID_ARG
+    assert L.fmoe_stack_forward(None, 1, 16, 16, 1, 16, 1 << 30, None) == fm.FMOE_ERR_INVALID_ARG
+    assert fm.fmoe_error_string(fm.FMOE_ERR_UNSUPPORTED) == "unsupported shape or bit width"
+
+
+def test_workspace_layout(fm):
+    d = fm.LayerDesc()
+    n1, n64 = fm.fmoe_workspace_bytes(d, 1), fm.fmoe_workspace_bytes(d, 64)
+    assert 0 < n1 < n64
+    offs = [fm.fmoe_workspace_offset(d, 3, w) for w in range(6)]
+    assert offs == sorted(offs) and all(o % 256 == 0 for o in offs)
+    assert fm.fmoe_workspace_offset(d, 3, 6) == 2 ** 64 - 1

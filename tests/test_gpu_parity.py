@@ -1,0 +1,341 @@
+"""GPU parity: every C-ABI entry point against the fp64 CPU oracle.
+
+Inputs come from the seeded generator (synth); the oracle computes on the
+logical layout, the device on the packed layout through libfmoe.  Router
+top-k is compared bit-exactly on the device's own fp32 logits; every float
+output within |d - v| <= 1e-3 S + 1e-5 and relative L2 <= 2e-3 (tests/parity.py).
+"""
+import numpy as np
+import pytest
+import torch
+
+import oracle
+import synth
+from synth.device import layer_desc, upload_layer
+from tests.parity import check
+
+pytestmark = pytest.mark.gpu
+
+fm = pytest.importorskip("quantized_expert_gemv_b200")
+
+TINY2 = synth.Workload(hidden=256, inter=128, n_experts=16, bits=2)
+
+
+@pytest.fixture(scope="module", autouse=True)
+def _cuda():
+    if not torch.cuda.is_available():
+        pytest.skip("no CUDA device")
+    fm.fmoe_read_status(clear=True)
+    yield
+    torch.cuda.synchronize()
+
+
+def oracle_layer(wl, layer, slots=None):
+    lw = oracle.LayerWeights(synth.router(wl, layer), synth.shared_gate(wl, layer), synth.norm_weight(wl, layer), {})
+    slots = range(wl.n_experts + 1) if slots is None else slots
+    for s, ex in zip(slots, synth.experts(wl, layer, slots)):
+        lw.experts[int(s)] = ex
+    return lw
+
+
+def dev(a):
+    return torch.from_numpy(np.ascontiguousarray(a)).cuda()
+
+
+def host(t):
+    return t.detach().cpu().numpy()
+
+
+_layers = {}
+
+
+def device_layer(wl, layer=0):
+    key = (wl, layer)
+    if key not in _layers:
+        _layers[key] = upload_layer(wl, layer)
+    return _layers[key]
+
+
+def check_layer_token(wl, lw_o, ws, desc, T, t, h_in, xn_in, h_out, xn_out, label):
+    """Teacher-forced check of token t of one layer step: routing on the
+    device's fp32 logits, then y, h', xn' against the oracle."""
+    lg_d = host(fm.workspace_view(ws, desc, T, fm.WS_LOGITS))[t]
+    ids_d = host(fm.workspace_view(ws, desc, T, fm.WS_IDS))[t]
+    p_d = host(fm.workspace_view(ws, desc, T, fm.WS_WEIGHTS))[t]
+    y_d = host(fm.workspace_view(ws, desc, T, fm.WS_Y))[t]
+    gamma_d = host(fm.workspace_view(ws, desc, T, fm.WS_GAMMA))[t]
+    lg_o, S_l = oracle.gemv_f32(lw_o.w_router, xn_in.astype(np.float64))
+    check(lg_d, lg_o, S_l, f"{label} logits")
+    ref = oracle.layer_token(wl, lw_o, h_in.astype(np.float64), xn_in.astype(np.float64), logits_in=lg_d,
+                             expert_fn=lambda s: synth.expert(wl, lw_o.layer if hasattr(lw_o, "layer") else 0, s))
+    assert ref["ids"].tolist() == ids_d.tolist(), f"{label} ids {ids_d} vs oracle {ref['ids']}"
+    check(p_d, ref["p"], ref["p"], f"{label} gate weights")
+    check(gamma_d, ref["gamma"], ref["gamma"] + ref["S_gamma"], f"{label} gamma")
+    check(y_d, ref["y"], ref["S_y"], f"{label} y")
+    check(h_out, ref["h"], ref["S_h"], f"{label} h'")
+    check(xn_out, ref["xn"], ref["S_xn"], f"{label} xn'")
+    return ref
+
+
+# ------------------------------------------------------------------ routing --
+
+@pytest.mark.parametrize("E,k", [(16, 4), (512, 4), (1024, 8), (5, 5), (64, 1)])
+def test_route_topk_given_logits_exact(E, k):
+    rng = np.random.default_rng(E * 10 + k)
+    T = 7
+    lg = rng.normal(size=(T, E)).astype(np.float32)
+    lg[1] = 0.5                        # all tied
+    lg[2, ::3] = 2.0                   # many tied maxima
+    lg[3, 1:] = -np.arange(E - 1, dtype=np.float32)
+    lg[4, 0] = np.float32(-0.0)
+    lg[4, 1:] = 0.0                    # +0 / -0 tie
+    logits = dev(lg)
+    ids = torch.empty((T, k), dtype=torch.int32, device="cuda")
+    w = torch.empty((T, k), dtype=torch.float32, device="cuda")
+    fm.fmoe_route_topk(None, None, k, logits, ids, w, None, flags=fm.FMOE_LOGITS_GIVEN)
+    ids_h, w_h = host(ids), host(w)
+    for t in range(T):
+        ri, rp, _ = oracle.topk_softmax(lg[t].astype(np.float64), k)
+        assert ids_h[t].tolist() == ri.tolist(), (t, ids_h[t], ri)
+        check(w_h[t], rp, rp, f"weights t={t}")
+    assert fm.fmoe_read_status() == 0
+
+
+def test_route_topk_nan_logits_set_status():
+    E, k = 32, 4
+    lg = np.linspace(1, 0, E, dtype=np.float32)[None].repeat(2, 0)
+    lg[0, [0, 3]] = np.nan
+    logits = dev(lg)
+    ids = torch.empty((2, k), dtype=torch.int32, device="cuda")
+    w = torch.empty((2, k), dtype=torch.float32, device="cuda")
+    fm.fmoe_route_topk(None, None, k, logits, ids, w, None, flags=fm.FMOE_LOGITS_GIVEN)
+    st = fm.fmoe_read_status(clear=True)
+    assert st & fm.FMOE_STATUS_NAN_LOGIT
+    for t in range(2):
+        ri, rp, nan = oracle.topk_softmax(lg[t].astype(np.float64), k)
+        assert host(ids)[t].tolist() == ri.tolist()
+        check(host(w)[t], rp, rp, "weights")
+
+
+@pytest.mark.parametrize("wl", [synth.TINY, synth.LAYER], ids=["tiny", "layer"])
+def test_route_topk_router_product(wl):
+    T = 3
+    W = synth.router(wl, 2)
+    x = synth.tokens(wl, T, stream=5)
+    logits = torch.empty((T, wl.n_experts), device="cuda")
+    ids = torch.empty((T, wl.top_k), dtype=torch.int32, device="cuda")
+    w = torch.empty((T, wl.top_k), device="cuda")
+    ws = fm.alloc_workspace(layer_desc(wl), T)
+    fm.fmoe_route_topk(dev(x), dev(W), wl.top_k, logits, ids, w, ws)
+    lg_h = host(logits)
+    for t in range(T):
+        lo, S = oracle.gemv_f32(W, x[t].astype(np.float64))
+        check(lg_h[t], lo, S, "logits")
+        ri, rp, _ = oracle.topk_softmax(lg_h[t].astype(np.float64), wl.top_k)
+        assert host(ids)[t].tolist() == ri.tolist()
+        check(host(w)[t], rp, rp, "weights")
+
+
+# ------------------------------------------------------------ expert forward --
+
+@pytest.mark.parametrize("wl", [synth.TINY, TINY2,
+                                synth.Workload(n_experts=8), synth.Workload(n_experts=8, bits=2),
+                                synth.Workload(hidden=2048, inter=512, n_experts=6, bits=4),
+                                synth.Workload(hidden=128, inter=2048, n_experts=6, bits=4)],
+                         ids=["tiny4", "tiny2", "full4", "full2", "h2048", "i2048"])
+def test_expert_forward(wl):
+    T = 3
+    lw = device_layer(wl)
+    lw_o = oracle_layer(wl, 0)
+    rng = np.random.default_rng(1)
+    ids_h = np.stack([rng.choice(wl.n_experts, wl.top_k, replace=False) for _ in range(T)]).astype(np.int32)
+    ids_h[2, 1] = ids_h[2, 0]  # a duplicate selection is legal
+    x = synth.tokens(wl, T, stream=9)
+    y = torch.empty((T, wl.top_k + 1, wl.hidden), device="cuda")
+    gamma = torch.empty(T, device="cuda")
+    ws = fm.alloc_workspace(lw.desc, T)
+    fm.fmoe_expert_forward(lw, dev(x), dev(ids_h), y, gamma, ws)
+    y_h, g_h = host(y), host(gamma)
+    for t in range(T):
+        xd = x[t].astype(np.float64)
+        for j, slot in enumerate(list(ids_h[t]) + [wl.n_experts]):
+            ref = oracle.expert_ffn(lw_o.experts[int(slot)], wl.hidden, wl.inter, 64, xd)
+            check(y_h[t, j], ref["y"], ref["S_y"], f"y t={t} j={j}")
+        z, Sz = oracle.gemv_f32(lw_o.w_shared_gate[None], xd)
+        gm = oracle.sigmoid(z[0])
+        check(g_h[t], gm, gm + gm * (1 - gm) * Sz[0], "gamma")
+    assert fm.fmoe_read_status() == 0
+
+
+def test_expert_forward_bad_ids_set_status_and_zero_output():
+    wl = synth.TINY
+    lw = device_layer(wl)
+    lw_o = oracle_layer(wl, 0)
+    ids_h = np.array([[3, -1, wl.n_experts, 7]], np.int32)
+    x = synth.tokens(wl, 1, stream=11)
+    y = torch.full((1, 5, wl.hidden), 7.0, device="cuda")
+    gamma = torch.empty(1, device="cuda")
+    ws = fm.alloc_workspace(lw.desc, 1)
+    fm.fmoe_expert_forward(lw, dev(x), dev(ids_h), y, gamma, ws)
+    st = fm.fmoe_read_status(clear=True)
+    assert st & fm.FMOE_STATUS_BAD_EXPERT_ID
+    y_h = host(y)
+    assert np.all(y_h[0, 1] == 0) and np.all(y_h[0, 2] == 0)
+    for j, slot in ((0, 3), (3, 7), (4, wl.n_experts)):
+        ref = oracle.expert_ffn(lw_o.experts[slot], wl.hidden, wl.inter, 64, x[0].astype(np.float64))
+        check(y_h[0, j], ref["y"], ref["S_y"], f"y j={j}")
+
+
+# ------------------------------------------------------------------ combine --
+
+@pytest.mark.parametrize("H,k,T", [(256, 4, 3), (4096, 4, 2), (4096, 8, 1), (64, 1, 5)])
+def test_combine_residual_rmsnorm(H, k, T):
+    rng = np.random.default_rng(H + k)
+    y = rng.normal(size=(T, k + 1, H)).astype(np.float32) * 3
+    p = rng.dirichlet(np.ones(k), size=T).astype(np.float32)
+    gamma = rng.uniform(size=T).astype(np.float32)
+    h = rng.normal(size=(T, H)).astype(np.float32)
+    w = (1 + 0.1 * rng.normal(size=H)).astype(np.float32)
+    h_out = torch.empty((T, H), device="cuda")
+    xn_out = torch.empty((T, H), device="cuda")
+    fm.fmoe_combine_residual_rmsnorm(dev(y), dev(p), dev(gamma), dev(h), dev(w), 1e-6, h_out, xn_out)
+    for t in range(T):
+        ho, xo, Sh, Sx = oracle.combine_rmsnorm(y[t], p[t], gamma[t], h[t], w, 1e-6)
+        check(host(h_out)[t], ho, Sh, "h'")
+        check(host(xn_out)[t], xo, Sx, "xn'")
+
+
+def test_combine_in_place_residual():
+    H, k, T = 256, 4, 2
+    rng = np.random.default_rng(3)
+    y = rng.normal(size=(T, k + 1, H)).astype(np.float32)
+    p = rng.dirichlet(np.ones(k), size=T).astype(np.float32)
+    gamma = rng.uniform(size=T).astype(np.float32)
+    h = rng.normal(size=(T, H)).astype(np.float32)
+    w = np.ones(H, np.float32)
+    hd = dev(h)
+    xn_out = torch.empty((T, H), device="cuda")
+    fm.fmoe_combine_residual_rmsnorm(dev(y), dev(p), dev(gamma), hd, dev(w), 1e-6, hd, xn_out)
+    for t in range(T):
+        ho, xo, Sh, Sx = oracle.combine_rmsnorm(y[t], p[t], gamma[t], h[t], w, 1e-6)
+        check(host(hd)[t], ho, Sh, "h' in place")
+        check(host(xn_out)[t], xo, Sx, "xn'")
+
+
+# -------------------------------------------------------------- layer forward --
+
+@pytest.mark.parametrize("wl,T", [(synth.TINY, 1), (synth.TINY, 3), (TINY2, 2)], ids=["tiny-T1", "tiny-T3", "tiny2-T2"])
+def test_layer_forward_tiny(wl, T):
+    lw = device_layer(wl)
+    lw_o = oracle_layer(wl, 0)
+    x = synth.tokens(wl, T, stream=21)
+    h = dev(x)
+    xn = dev(x)
+    ws = fm.alloc_workspace(lw.desc, T)
+    fm.fmoe_layer_forward(lw, h, xn, ws)
+    for t in range(T):
+        check_layer_token(wl, lw_o, ws, lw.desc, T, t, x[t], x[t], host(h)[t], host(xn)[t], f"t={t}")
+    assert fm.fmoe_read_status() == 0
+
+
+@pytest.fixture(scope="module")
+def full_layer():
+    wl = synth.LAYER
+    return wl, device_layer(wl, 0), oracle_layer(wl, 0, slots=[wl.n_experts])
+
+
+def test_layer_forward_full_size(full_layer):
+    """One 4-bit layer at hidden 4096 / 512 experts, batch 1, every output checked."""
+    wl, lw, lw_o = full_layer
+    x = synth.tokens(wl, 1, stream=31)
+    h, xn = dev(x), dev(x)
+    ws = fm.alloc_workspace(lw.desc, 1)
+    fm.fmoe_layer_forward(lw, h, xn, ws)
+    check_layer_token(wl, lw_o, ws, lw.desc, 1, 0, x[0], x[0], host(h)[0], host(xn)[0], "full")
+    assert fm.fmoe_read_status() == 0
+
+
+def test_layer_forward_is_deterministic_and_graph_capturable(full_layer):
+    wl, lw, _ = full_layer
+    x = synth.tokens(wl, 1, stream=32)
+    ws = fm.alloc_workspace(lw.desc, 1)
+    outs = []
+    for _ in range(2):
+        h, xn = dev(x), dev(x)
+        fm.fmoe_layer_forward(lw, h, xn, ws)
+        outs.append((host(h), host(xn)))
+    assert np.array_equal(outs[0][0], outs[1][0]) and np.array_equal(outs[0][1], outs[1][1])
+    h, xn = dev(x), dev(x)
+    s = torch.cuda.Stream()
+    s.wait_stream(torch.cuda.current_stream())
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.stream(s):
+        with torch.cuda.graph(g, stream=s):
+            fm.fmoe_layer_forward(lw, h, xn, ws, stream=s)
+    torch.cuda.current_stream().wait_stream(s)
+    h.copy_(dev(x))
+    xn.copy_(dev(x))
+    g.replay()
+    torch.cuda.synchronize()
+    assert np.array_equal(host(h), outs[0][0]) and np.array_equal(host(xn), outs[0][1])
+
+
+def test_layer_forward_batched_zipf_routing(full_layer):
+    """64 tokens through one layer on Zipf(1)-popularity Gumbel-top-k routing
+    logits; 8 sampled tokens checked against the oracle."""
+    wl, lw, lw_o = full_layer
+    T = 64
+    lg, _ = synth.zipf_gumbel_logits(wl, 0, T)
+    x = synth.tokens(wl, T, stream=41)
+    h, xn = dev(x), dev(x)
+    ws = fm.alloc_workspace(lw.desc, T)
+    fm.fmoe_layer_forward_logits(lw, dev(lg), h, xn, ws)
+    ids_d = host(fm.workspace_view(ws, lw.desc, T, fm.WS_IDS))
+    counts = np.bincount(ids_d.ravel(), minlength=wl.n_experts)
+    assert counts.max() >= 16  # Zipf routing gives hot experts
+    for t in (0, 5, 17, 30, 42, 51, 60, 63):
+        ri, _, _ = oracle.topk_softmax(lg[t].astype(np.float64), wl.top_k)
+        assert ri.tolist() == ids_d[t].tolist()
+        check_layer_token(wl, lw_o, ws, lw.desc, T, t, x[t], x[t], host(h)[t], host(xn)[t], f"t={t}")
+
+
+# ------------------------------------------------------------------- chains --
+
+@pytest.mark.parametrize("wl", [synth.TINY, TINY2], ids=["int4", "int2"])
+def test_stack_chain_teacher_forced_and_free_running(wl):
+    """A 4-layer stack decoding 3 tokens: h, xn carried layer to layer, each
+    next token starting from the previous token's final xn'.  Each layer is
+    checked teacher-forced on the device's inputs; fmoe_stack_forward must
+    equal the layer-by-layer calls bit for bit; the free-running fp64 chain
+    must agree in relative L2."""
+    L, steps = 4, 3
+    lws = [device_layer(wl, l) for l in range(L)]
+    los = [oracle_layer(wl, l) for l in range(L)]
+    for l, lo in enumerate(los):
+        lo.layer = l
+    x0 = synth.tokens(wl, 1, stream=51)[0]
+    ws = fm.alloc_workspace(lws[0].desc, 1)
+    # layer by layer
+    tok = x0.copy()
+    h, xn = dev(tok[None]), dev(tok[None])
+    free_h = tok.astype(np.float64)
+    free_xn = tok.astype(np.float64)
+    for s in range(steps):
+        for l in range(L):
+            h_in, xn_in = host(h)[0], host(xn)[0]
+            fm.fmoe_layer_forward(lws[l], h, xn, ws)
+            check_layer_token(wl, los[l], ws, lws[l].desc, 1, 0, h_in, xn_in, host(h)[0], host(xn)[0],
+                              f"step {s} layer {l}")
+            ref = oracle.layer_token(wl, los[l], free_h, free_xn, expert_fn=lambda e, l=l: synth.expert(wl, l, e))
+            free_h, free_xn = ref["h"], ref["xn"]
+        h.copy_(xn)
+        free_h = free_xn.copy()
+    final_layered = host(xn)[0]
+    rel = np.linalg.norm(final_layered - free_xn) / np.linalg.norm(free_xn)
+    assert rel <= 2e-3, rel
+    # the stack entry point gives the same bits
+    h2, xn2 = dev(x0[None]), dev(x0[None])
+    for s in range(steps):
+        fm.fmoe_stack_forward(lws, h2, xn2, ws)
+        h2.copy_(xn2)
+    assert np.array_equal(host(xn2)[0], final_layered)
