@@ -217,11 +217,20 @@ int fmoe_layer_forward(const fmoe_layer_weights* lw, float* d_h, float* d_xn, in
 int fmoe_layer_forward_logits(const fmoe_layer_weights* lw, const float* d_logits, float* d_h,
                               float* d_xn, int T, void* d_ws, size_t ws_bytes, cudaStream_t stream);
 
-/* A stack of n_layers layers (host array of weight descriptors, all with the
- * same descriptor) for T tokens, in place on d_h / d_xn: layer l + 1 reads
- * what layer l wrote.  Equivalent to n_layers calls of fmoe_layer_forward. */
+/* A stack of n_layers layers (host array of weight descriptors) for T
+ * tokens, in place on d_h / d_xn: layer l + 1 reads what layer l wrote.
+ * Equivalent to n_layers calls of fmoe_layer_forward.  At T = 1 with one
+ * descriptor for all layers the whole stack runs as one persistent kernel
+ * (cooperative launch, one CTA per SM, up to 32 layers per launch).  If that
+ * kernel reports FMOE_STATUS_WAIT_TIMEOUT, re-initialise the workspace. */
 int fmoe_stack_forward(const fmoe_layer_weights* layers, int n_layers, float* d_h, float* d_xn,
                        int T, void* d_ws, size_t ws_bytes, cudaStream_t stream);
+
+/* Chooses the implementation of the T = 1 path: enable != 0 (the default)
+ * uses the persistent fused kernel wherever its shared-memory plan fits, 0
+ * the one-kernel-per-step path.  Both compute the same layer; process-wide
+ * setting, returns the previous value. */
+int fmoe_set_fused(int enable);
 
 #ifdef __cplusplus
 }

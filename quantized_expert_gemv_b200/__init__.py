@@ -87,6 +87,7 @@ _SIGS = {
     "fmoe_layer_forward": (_i32, [_PW, _vp, _vp, _i32, _vp, _sz, _vp]),
     "fmoe_layer_forward_logits": (_i32, [_PW, _vp, _vp, _vp, _i32, _vp, _sz, _vp]),
     "fmoe_stack_forward": (_i32, [_PW, _i32, _vp, _vp, _i32, _vp, _sz, _vp]),
+    "fmoe_set_fused": (_i32, [_i32]),
 }
 for _name, (_res, _args) in _SIGS.items():
     _fn = getattr(_lib, _name)
@@ -295,3 +296,9 @@ def fmoe_stack_forward(layers, h, xn, ws, stream=None) -> None:
     rc = _lib.fmoe_stack_forward(arr, len(layers), _ptr(h), _ptr(xn), h.shape[0], _ptr(ws),
                                  ws.numel() * ws.element_size(), _stream(stream))
     _check(rc, "fmoe_stack_forward")
+
+
+def fmoe_set_fused(enable: bool) -> bool:
+    """Selects the persistent fused kernel (True, default) or the one-kernel-per-step
+    path for T = 1; returns the previous setting."""
+    return bool(_lib.fmoe_set_fused(int(bool(enable))))

@@ -160,9 +160,11 @@ __device__ __forceinline__ StagedX staged_x_at(unsigned char* base, int K) {
   return s;
 }
 
-// Quantises x[0..K) (fp32, global) into `s`.  All threads of the block take
-// part; 8 consecutive threads share one group.  Caller syncs afterwards.
-__device__ __forceinline__ void stage_x(const float* __restrict__ x, int K, StagedX s) {
+// Quantises x[0..K) (fp32, global or shared) into `s`.  All threads of the
+// block take part; 8 consecutive threads share one group.  With `cg` the
+// loads bypass L1 (data written by other CTAs of a running kernel).  Caller
+// syncs afterwards.
+__device__ __forceinline__ void stage_x(const float* __restrict__ x, int K, StagedX s, bool cg = false) {
   const int ng = K / 64;
   const int nunits = ng * 8;
   // round the loop up to a multiple of 8 threads so that group shuffles stay converged
@@ -173,8 +175,9 @@ __device__ __forceinline__ void stage_x(const float* __restrict__ x, int K, Stag
     float v[8];
     float m = 0.f;
     if (active) {
-      const float4 a = *reinterpret_cast<const float4*>(x + (size_t)g * 64 + u * 8);
-      const float4 b = *reinterpret_cast<const float4*>(x + (size_t)g * 64 + u * 8 + 4);
+      const float4* src = reinterpret_cast<const float4*>(x + (size_t)g * 64 + u * 8);
+      const float4 a = cg ? __ldcg(src) : src[0];
+      const float4 b = cg ? __ldcg(src + 1) : src[1];
       v[0] = a.x; v[1] = a.y; v[2] = a.z; v[3] = a.w;
       v[4] = b.x; v[5] = b.y; v[6] = b.z; v[7] = b.w;
 #pragma unroll

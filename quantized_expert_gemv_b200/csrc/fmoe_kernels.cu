@@ -22,6 +22,7 @@
 
 #include "fmoe.h"
 #include "fmoe_device.cuh"
+#include "fmoe_fused.cuh"
 #include "fmoe_layout.h"
 
 namespace fmoe {
@@ -263,7 +264,7 @@ __device__ __forceinline__ void unit_range(int n_units, int* u0, int* u1) {
 __global__ void __launch_bounds__(kThreads)
 gateup_kernel(ExpertSet es, const float* __restrict__ xn, const int32_t* __restrict__ ids,
               float* __restrict__ a, const float* __restrict__ w_sg, float* __restrict__ gamma) {
-  extern __shared__ __align__(16) unsigned char smem[];
+  extern __shared__ __align__(128) unsigned char smem[];
   const int slot = blockIdx.y, t = slot / (es.k + 1), j = slot % (es.k + 1);
   int bits;
   const uint8_t* rec = slot_record(es, ids, t, j, &bits);
@@ -302,7 +303,7 @@ gateup_kernel(ExpertSet es, const float* __restrict__ xn, const int32_t* __restr
 __global__ void __launch_bounds__(kThreads)
 down_kernel(ExpertSet es, const int32_t* __restrict__ ids, const float* __restrict__ a,
             float* __restrict__ y) {
-  extern __shared__ __align__(16) unsigned char smem[];
+  extern __shared__ __align__(128) unsigned char smem[];
   const int slot = blockIdx.y, t = slot / (es.k + 1), j = slot % (es.k + 1);
   int bits;
   const uint8_t* rec = slot_record(es, ids, t, j, &bits);
@@ -459,14 +460,18 @@ __global__ void pack_sb_kernel(const uint16_t* __restrict__ scale, const uint16_
 
 // ------------------------------------------------------- host helpers ----
 struct WsLayout {
-  size_t part, logits, ids, weights, gamma, a, y, bytes;
+  size_t sync, ss, part, logits, ids, weights, gamma, a, y, bytes;
 };
 
 static inline size_t align_up(size_t v, size_t a) { return (v + a - 1) / a * a; }
 
+constexpr int kMaxSMs = 1024;
+
 static WsLayout ws_layout(int H, int I, int E, int k, int T) {
   WsLayout w;
-  size_t o = 256;  // reserved
+  w.sync = 0;    // grid-barrier counters of the fused kernel
+  w.ss = 256;    // per-CTA partial sums of h'^2
+  size_t o = 256 + (size_t)kMaxSMs * 4;
   w.part = o;
   o = align_up(o + (size_t)T * (E + 1) * kRouterSplit * 4, 256);
   w.logits = o;
@@ -569,6 +574,124 @@ static int launch_combine(const float* y, const float* weights, const float* gam
   return cuda_rc(cudaGetLastError());
 }
 
+// ----------------------------------------------------- fused batch-1 path --
+static int g_fused_enabled = 1;
+
+struct FusedConfig {
+  bool ok;
+  int n_sm;
+  FusedPlan plan;
+};
+
+static bool same_desc(const fmoe_layer_desc& a, const fmoe_layer_desc& b);
+
+// Per-device cache of the last configuration (shape checks and the
+// attribute / occupancy queries run once per shape, not per call).
+struct FusedCacheEntry {
+  bool valid;
+  fmoe_layer_desc desc;
+  FusedConfig fc;
+};
+static FusedCacheEntry g_fused_cache[64];
+
+static FusedConfig fused_config_uncached(const fmoe_layer_desc& d, int dev);
+
+static FusedConfig fused_config(const fmoe_layer_desc& d) {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return FusedConfig{};
+  FusedCacheEntry& e = g_fused_cache[dev];
+  if (e.valid && same_desc(e.desc, d)) return e.fc;
+  const FusedConfig fc = fused_config_uncached(d, dev);
+  e.desc = d;
+  e.fc = fc;
+  e.valid = true;
+  return fc;
+}
+
+static FusedConfig fused_config_uncached(const fmoe_layer_desc& d, int dev) {
+  FusedConfig fc{};
+  int n_sm = 0, optin = 0;
+  if (cudaDeviceGetAttribute(&n_sm, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess) return fc;
+  if (cudaDeviceGetAttribute(&optin, cudaDevAttrMaxSharedMemoryPerBlockOptin, dev) != cudaSuccess) return fc;
+  if (n_sm < 1 || n_sm > kMaxSMs) return fc;
+  const size_t max_dyn = optin > 2048 ? (size_t)optin - 1024 : 0;
+  if (!fused_plan(d.hidden, d.inter, d.n_experts, d.top_k, d.bits, d.shared_bits, n_sm, max_dyn, &fc.plan))
+    return fc;
+  if (cudaFuncSetAttribute(fused_stack_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                           (int)fc.plan.total) != cudaSuccess)
+    return fc;
+  int per_sm = 0;
+  if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, fused_stack_kernel, kFusedThreads,
+                                                    fc.plan.total) != cudaSuccess ||
+      per_sm < 1)
+    return fc;
+  fc.n_sm = n_sm;
+  fc.ok = true;
+  return fc;
+}
+
+static bool same_desc(const fmoe_layer_desc& a, const fmoe_layer_desc& b) {
+  return a.hidden == b.hidden && a.inter == b.inter && a.n_experts == b.n_experts && a.top_k == b.top_k &&
+         a.bits == b.bits && a.shared_bits == b.shared_bits && a.group == b.group && a.eps == b.eps;
+}
+
+// Runs n_layers layers (T = 1) with the persistent kernel.  Returns
+// FMOE_ERR_UNSUPPORTED when the configuration does not fit it.
+static int launch_fused(const fmoe_layer_weights* layers, int n_layers, float* h, float* xn, void* ws,
+                        size_t ws_bytes, cudaStream_t st) {
+  const fmoe_layer_desc& d = layers[0].desc;
+  const FusedConfig fc = fused_config(d);
+  if (!fc.ok) return FMOE_ERR_UNSUPPORTED;
+  const WsLayout w = ws_layout(d.hidden, d.inter, d.n_experts, d.top_k, 1);
+  if (ws_bytes < w.bytes) return FMOE_ERR_BUFFER_TOO_SMALL;
+  unsigned char* base = static_cast<unsigned char*>(ws);
+  FusedArgs args;
+  std::memset(&args, 0, sizeof(args));
+  args.H = d.hidden;
+  args.I = d.inter;
+  args.E = d.n_experts;
+  args.k = d.top_k;
+  args.bits = d.bits;
+  args.sbits = d.shared_bits;
+  args.eps = d.eps;
+  args.h = h;
+  args.xn = xn;
+  args.logits = reinterpret_cast<float*>(base + w.logits);
+  args.ids = reinterpret_cast<int32_t*>(base + w.ids);
+  args.weights = reinterpret_cast<float*>(base + w.weights);
+  args.gamma = reinterpret_cast<float*>(base + w.gamma);
+  args.a = reinterpret_cast<float*>(base + w.a);
+  args.y = reinterpret_cast<float*>(base + w.y);
+  args.ss_part = reinterpret_cast<float*>(base + w.ss);
+  args.sync = reinterpret_cast<unsigned*>(base + w.sync);
+  args.plan = fc.plan;
+  for (int l0 = 0; l0 < n_layers; l0 += kFusedMaxLayers) {
+    const int n = n_layers - l0 < kFusedMaxLayers ? n_layers - l0 : kFusedMaxLayers;
+    args.n_layers = n;
+    for (int l = 0; l < n; ++l) {
+      const fmoe_layer_weights& L = layers[l0 + l];
+      args.layers[l].experts = static_cast<const uint8_t*>(L.experts);
+      args.layers[l].shared = static_cast<const uint8_t*>(L.shared);
+      args.layers[l].w_router = L.w_router;
+      args.layers[l].w_sg = L.w_shared_gate;
+      args.layers[l].norm_w = L.norm_w;
+    }
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(fc.n_sm);
+    cfg.blockDim = dim3(kFusedThreads);
+    cfg.dynamicSmemBytes = fc.plan.total;
+    cfg.stream = st;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeCooperative;
+    attr[0].val.cooperative = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    const cudaError_t e = cudaLaunchKernelEx(&cfg, fused_stack_kernel, args);
+    if (e != cudaSuccess) return FMOE_ERR_CUDA;
+  }
+  return FMOE_OK;
+}
+
 static int layer_forward_impl(const fmoe_layer_weights* lw, const float* logits_in, float* h,
                               float* xn, int T, void* ws, size_t ws_bytes, cudaStream_t st) {
   int rc = weights_check(lw);
@@ -579,6 +702,10 @@ static int layer_forward_impl(const fmoe_layer_weights* lw, const float* logits_
   if (logits_in && !aligned16(logits_in)) return FMOE_ERR_INVALID_ARG;
   const WsLayout w = ws_layout(d.hidden, d.inter, d.n_experts, d.top_k, T);
   if (ws_bytes < w.bytes) return FMOE_ERR_BUFFER_TOO_SMALL;
+  if (T == 1 && !logits_in && g_fused_enabled) {
+    rc = launch_fused(lw, 1, h, xn, ws, ws_bytes, st);
+    if (rc != FMOE_ERR_UNSUPPORTED) return rc;
+  }
   unsigned char* base = static_cast<unsigned char*>(ws);
   float* part = reinterpret_cast<float*>(base + w.part);
   float* logits = reinterpret_cast<float*>(base + w.logits);
@@ -734,10 +861,30 @@ extern "C" int fmoe_pack_experts_device(const uint8_t* d_q, const uint16_t* d_sc
   return cuda_rc(cudaGetLastError());
 }
 
+extern "C" int fmoe_set_fused(int enable) {
+  const int prev = g_fused_enabled;
+  g_fused_enabled = enable ? 1 : 0;
+  return prev;
+}
+
 extern "C" int fmoe_stack_forward(const fmoe_layer_weights* layers, int n_layers, float* d_h,
                                   float* d_xn, int T, void* d_ws, size_t ws_bytes,
                                   cudaStream_t stream) {
   if (!layers || n_layers < 1) return FMOE_ERR_INVALID_ARG;
+  if (T == 1 && g_fused_enabled) {
+    bool uniform = true;
+    for (int l = 0; l < n_layers; ++l) {
+      const int rc = weights_check(&layers[l]);
+      if (rc != FMOE_OK) return rc;
+      uniform = uniform && same_desc(layers[l].desc, layers[0].desc);
+    }
+    if (!d_h || !d_xn || !d_ws || !aligned16(d_h) || !aligned16(d_xn) || !aligned16(d_ws))
+      return FMOE_ERR_INVALID_ARG;
+    if (uniform) {
+      const int rc = launch_fused(layers, n_layers, d_h, d_xn, d_ws, ws_bytes, stream);
+      if (rc != FMOE_ERR_UNSUPPORTED) return rc;
+    }
+  }
   for (int l = 0; l < n_layers; ++l) {
     const int rc = fmoe_layer_forward(&layers[l], d_h, d_xn, T, d_ws, ws_bytes, stream);
     if (rc != FMOE_OK) return rc;

@@ -19,6 +19,9 @@ pytestmark = pytest.mark.gpu
 fm = pytest.importorskip("quantized_expert_gemv_b200")
 
 TINY2 = synth.Workload(hidden=256, inter=128, n_experts=16, bits=2)
+# small shapes the persistent fused kernel accepts (inter a multiple of 256)
+SMALL = synth.Workload(hidden=256, inter=256, n_experts=16)
+SMALL2 = synth.Workload(hidden=256, inter=256, n_experts=16, bits=2)
 
 
 @pytest.fixture(scope="module", autouse=True)
@@ -56,18 +59,21 @@ def device_layer(wl, layer=0):
     return _layers[key]
 
 
-def check_layer_token(wl, lw_o, ws, desc, T, t, h_in, xn_in, h_out, xn_out, label):
+def check_layer_token(wl, lw_o, ws, desc, T, t, h_in, xn_in, h_out, xn_out, label, logits_given=False):
     """Teacher-forced check of token t of one layer step: routing on the
-    device's fp32 logits, then y, h', xn' against the oracle."""
+    device's fp32 logits (the router product is checked too unless the
+    logits were given), then y, h', xn' against the oracle."""
     lg_d = host(fm.workspace_view(ws, desc, T, fm.WS_LOGITS))[t]
     ids_d = host(fm.workspace_view(ws, desc, T, fm.WS_IDS))[t]
     p_d = host(fm.workspace_view(ws, desc, T, fm.WS_WEIGHTS))[t]
     y_d = host(fm.workspace_view(ws, desc, T, fm.WS_Y))[t]
     gamma_d = host(fm.workspace_view(ws, desc, T, fm.WS_GAMMA))[t]
-    lg_o, S_l = oracle.gemv_f32(lw_o.w_router, xn_in.astype(np.float64))
-    check(lg_d, lg_o, S_l, f"{label} logits")
+    if not logits_given:
+        lg_o, S_l = oracle.gemv_f32(lw_o.w_router, xn_in.astype(np.float64))
+        check(lg_d, lg_o, S_l, f"{label} logits")
+    layer = getattr(lw_o, "layer", 0)
     ref = oracle.layer_token(wl, lw_o, h_in.astype(np.float64), xn_in.astype(np.float64), logits_in=lg_d,
-                             expert_fn=lambda s: synth.expert(wl, lw_o.layer if hasattr(lw_o, "layer") else 0, s))
+                             expert_fn=lambda s: synth.expert(wl, layer, s))
     assert ref["ids"].tolist() == ids_d.tolist(), f"{label} ids {ids_d} vs oracle {ref['ids']}"
     check(p_d, ref["p"], ref["p"], f"{label} gate weights")
     check(gamma_d, ref["gamma"], ref["gamma"] + ref["S_gamma"], f"{label} gamma")
@@ -224,8 +230,17 @@ def test_combine_in_place_residual():
 
 # -------------------------------------------------------------- layer forward --
 
-@pytest.mark.parametrize("wl,T", [(synth.TINY, 1), (synth.TINY, 3), (TINY2, 2)], ids=["tiny-T1", "tiny-T3", "tiny2-T2"])
-def test_layer_forward_tiny(wl, T):
+@pytest.fixture(params=[True, False], ids=["fused", "per-step"])
+def path(request):
+    prev = fm.fmoe_set_fused(request.param)
+    yield request.param
+    fm.fmoe_set_fused(prev)
+
+
+@pytest.mark.parametrize("wl,T", [(synth.TINY, 1), (synth.TINY, 3), (TINY2, 1), (TINY2, 2), (SMALL, 1), (SMALL2, 1),
+                                  (SMALL, 2)],
+                         ids=["tiny-T1", "tiny-T3", "tiny2-T1", "tiny2-T2", "small-T1", "small2-T1", "small-T2"])
+def test_layer_forward_tiny(wl, T, path):
     lw = device_layer(wl)
     lw_o = oracle_layer(wl, 0)
     x = synth.tokens(wl, T, stream=21)
@@ -244,7 +259,7 @@ def full_layer():
     return wl, device_layer(wl, 0), oracle_layer(wl, 0, slots=[wl.n_experts])
 
 
-def test_layer_forward_full_size(full_layer):
+def test_layer_forward_full_size(full_layer, path):
     """One 4-bit layer at hidden 4096 / 512 experts, batch 1, every output checked."""
     wl, lw, lw_o = full_layer
     x = synth.tokens(wl, 1, stream=31)
@@ -253,6 +268,37 @@ def test_layer_forward_full_size(full_layer):
     fm.fmoe_layer_forward(lw, h, xn, ws)
     check_layer_token(wl, lw_o, ws, lw.desc, 1, 0, x[0], x[0], host(h)[0], host(xn)[0], "full")
     assert fm.fmoe_read_status() == 0
+
+
+@pytest.mark.parametrize("wl", [synth.Workload(n_experts=32, bits=2)], ids=["int2-32"])
+def test_layer_forward_full_size_int2(wl, path):
+    """hidden 4096 / inter 1024 with 2-bit routed experts (4-bit shared), batch 1."""
+    lw = device_layer(wl)
+    lw_o = oracle_layer(wl, 0, slots=[wl.n_experts])
+    for stream in (33, 34):
+        x = synth.tokens(wl, 1, stream=stream)
+        h, xn = dev(x), dev(x)
+        ws = fm.alloc_workspace(lw.desc, 1)
+        fm.fmoe_layer_forward(lw, h, xn, ws)
+        check_layer_token(wl, lw_o, ws, lw.desc, 1, 0, x[0], x[0], host(h)[0], host(xn)[0], f"int2 {stream}")
+    assert fm.fmoe_read_status() == 0
+
+
+def test_fused_and_per_step_paths_agree(full_layer):
+    wl, lw, _ = full_layer
+    x = synth.tokens(wl, 1, stream=35)
+    outs = {}
+    for fused in (True, False):
+        prev = fm.fmoe_set_fused(fused)
+        h, xn = dev(x), dev(x)
+        ws = fm.alloc_workspace(lw.desc, 1)
+        fm.fmoe_layer_forward(lw, h, xn, ws)
+        outs[fused] = (host(h)[0], host(xn)[0], host(fm.workspace_view(ws, lw.desc, 1, fm.WS_IDS))[0])
+        fm.fmoe_set_fused(prev)
+    assert outs[True][2].tolist() == outs[False][2].tolist()
+    for i in range(2):
+        a, b = outs[True][i], outs[False][i]
+        assert np.linalg.norm(a - b) / np.linalg.norm(b) < 1e-5
 
 
 def test_layer_forward_is_deterministic_and_graph_capturable(full_layer):
@@ -296,13 +342,14 @@ def test_layer_forward_batched_zipf_routing(full_layer):
     for t in (0, 5, 17, 30, 42, 51, 60, 63):
         ri, _, _ = oracle.topk_softmax(lg[t].astype(np.float64), wl.top_k)
         assert ri.tolist() == ids_d[t].tolist()
-        check_layer_token(wl, lw_o, ws, lw.desc, T, t, x[t], x[t], host(h)[t], host(xn)[t], f"t={t}")
+        check_layer_token(wl, lw_o, ws, lw.desc, T, t, x[t], x[t], host(h)[t], host(xn)[t], f"t={t}",
+                          logits_given=True)
 
 
 # ------------------------------------------------------------------- chains --
 
-@pytest.mark.parametrize("wl", [synth.TINY, TINY2], ids=["int4", "int2"])
-def test_stack_chain_teacher_forced_and_free_running(wl):
+@pytest.mark.parametrize("wl", [synth.TINY, TINY2, SMALL, SMALL2], ids=["tiny4", "tiny2", "small4", "small2"])
+def test_stack_chain_teacher_forced_and_free_running(wl, path):
     """A 4-layer stack decoding 3 tokens: h, xn carried layer to layer, each
     next token starting from the previous token's final xn'.  Each layer is
     checked teacher-forced on the device's inputs; fmoe_stack_forward must
