@@ -68,8 +68,10 @@ __device__ __forceinline__ int dp2a_hi(uint32_t a, uint32_t b, int c) {
 template <int BITS>
 __device__ __forceinline__ uint32_t chunk_off(int ng, int g, int h) {
   if (BITS == 2) return (uint32_t)g * 16u;
+  // segments hold min(32, ng) groups; ng is a power of two below 32
   const int seg = ng < 32 ? ng : 32;
-  return (uint32_t)((g / seg) * seg * 32 + h * seg * 16 + (g % seg) * 16);
+  const int sh = __ffs(seg) - 1;
+  return (uint32_t)(((g >> sh) << (sh + 5)) + (h << (sh + 4)) + ((g & (seg - 1)) << 4));
 }
 
 // Codes of one group of one row: 32 bytes (4-bit) or 16 bytes (2-bit).
@@ -213,6 +215,73 @@ __device__ __forceinline__ void stage_x(const float* __restrict__ x, int K, Stag
       if (u == 0) {
         s.delta[g] = delta;
         s.xsum[g] = delta * (float)sum;
+      }
+    }
+  }
+}
+
+// Stages nvec vectors of K inputs each (x + v * K, global, L1 bypassed) into
+// staged blocks at base + v * stride.  All loads of a thread are issued
+// before any of them is used (one memory round trip for up to 4 * blockDim.x
+// groups-of-8).  Caller syncs afterwards.
+__device__ __forceinline__ void stage_x_multi(const float* __restrict__ x, int K, int nvec,
+                                              unsigned char* base, size_t stride) {
+  constexpr int kMaxIt = 4;
+  const int upv = K / 8;  // units of 8 inputs per vector (a multiple of 8)
+  const int nunits = upv * nvec;
+  for (int base_u = 0; base_u < nunits; base_u += kMaxIt * (int)blockDim.x) {
+    float4 lo[kMaxIt], hi[kMaxIt];
+#pragma unroll
+    for (int it = 0; it < kMaxIt; ++it) {
+      const int idx = base_u + it * (int)blockDim.x + (int)threadIdx.x;
+      if (idx < nunits) {
+        const float4* src = reinterpret_cast<const float4*>(x + (size_t)idx * 8);
+        lo[it] = __ldcg(src);
+        hi[it] = __ldcg(src + 1);
+      } else {
+        lo[it] = make_float4(0.f, 0.f, 0.f, 0.f);
+        hi[it] = lo[it];
+      }
+    }
+#pragma unroll
+    for (int it = 0; it < kMaxIt; ++it) {
+      if (base_u + it * (int)blockDim.x >= nunits) break;  // uniform across the block
+      const int idx = base_u + it * (int)blockDim.x + (int)threadIdx.x;
+      const bool active = idx < nunits;
+      const int v = idx / upv, w = idx % upv, g = w >> 3, u = w & 7;
+      const float vals[8] = {lo[it].x, lo[it].y, lo[it].z, lo[it].w, hi[it].x, hi[it].y, hi[it].z, hi[it].w};
+      float m = 0.f;
+#pragma unroll
+      for (int i = 0; i < 8; ++i) m = fmaxf(m, fabsf(vals[i]));
+      m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, 1));
+      m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, 2));
+      m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, 4));
+      const float inv = m > 0.f ? 32767.f / m : 0.f;
+      const float delta = m * (1.f / 32767.f);
+      int q[8], sum = 0;
+#pragma unroll
+      for (int i = 0; i < 8; ++i) {
+        int t = __float2int_rn(vals[i] * inv);
+        t = t > 32767 ? 32767 : (t < -32767 ? -32767 : t);
+        q[i] = t;
+        sum += t;
+      }
+      sum += __shfl_xor_sync(0xffffffffu, sum, 1);
+      sum += __shfl_xor_sync(0xffffffffu, sum, 2);
+      sum += __shfl_xor_sync(0xffffffffu, sum, 4);
+      if (active) {
+        const StagedX s = staged_x_at(base + (size_t)v * stride, K);
+        const int ng = K / 64;
+        uint4 pk;
+        pk.x = (uint32_t)(q[0] & 0xFFFF) | ((uint32_t)q[1] << 16);
+        pk.y = (uint32_t)(q[2] & 0xFFFF) | ((uint32_t)q[3] << 16);
+        pk.z = (uint32_t)(q[4] & 0xFFFF) | ((uint32_t)q[5] << 16);
+        pk.w = (uint32_t)(q[6] & 0xFFFF) | ((uint32_t)q[7] << 16);
+        s.xs[u * ng + g] = pk;
+        if (u == 0) {
+          s.delta[g] = delta;
+          s.xsum[g] = delta * (float)sum;
+        }
       }
     }
   }

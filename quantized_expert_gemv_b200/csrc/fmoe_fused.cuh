@@ -44,13 +44,18 @@ constexpr int kFusedMaxRouterRows = 8;
 constexpr int kFusedMaxSharedPairs = 32;
 constexpr int kFusedMaxRoutedPairs = 96;
 constexpr int kFusedMaxK = 8;
+constexpr int kPairsPerChunk = 4;  // gate/up row pairs per bulk-copy chunk (one mbarrier)
 constexpr int kMbRouter = 0;
 constexpr int kMbSPair = kMbRouter + kFusedMaxRouterRows;
-constexpr int kMbSDown = kMbSPair + kFusedMaxSharedPairs;
+constexpr int kMbSDown = kMbSPair + kFusedMaxSharedPairs / kPairsPerChunk;
 constexpr int kMbRPair = kMbSDown + 1;
-constexpr int kMbRDown = kMbRPair + kFusedMaxRoutedPairs;
+constexpr int kMbRDown = kMbRPair + kFusedMaxRoutedPairs / kPairsPerChunk;
 constexpr int kMbCount = kMbRDown + kFusedMaxK;
 constexpr long long kWaitCycles = 4000000000LL;  // ~2 s at 2 GHz
+constexpr int kSyncGroups = 2;        // first per-group publication counter in FusedArgs::sync
+constexpr int kMaxGroupCounters = 1022;
+constexpr int kWStage = 144;          // per-warp staged a-group: 8 uint4 + delta + xsum (+pad)
+constexpr int kMaxSliceRows = 64;     // hidden rows per CTA in the down products (2 per lane)
 
 struct FusedLayer {
   const uint8_t* experts;
@@ -61,14 +66,23 @@ struct FusedLayer {
 };
 
 // Shared-memory plan (byte offsets), computed on the host.
+//   region A  P1: router rows, shared pairs' codes, shared pairs' scale-bias
+//             P2: routed pairs' codes, routed pairs' scale-bias
+//   region B  shared down rows, then routed down rows (fp32 x during P1)
+//   xq        staged int16 x (P1, P2), then the staged SwiGLU outputs (P3)
 struct FusedPlan {
-  uint32_t region_a;     // P1: router rows + shared pairs; P2: routed pairs; P3: staged a
-  uint32_t region_b;     // shared down rows, then routed down rows (x in fp32 during P1)
-  uint32_t xf;           // fp32 x (may alias the routed part of region B)
-  uint32_t xq;           // staged int16 x
-  uint32_t logit;        // fp32 [E]
-  uint32_t ypart;        // fp32 [(k+1)][down rows]
-  uint32_t rpart;        // fp32 [router rows][slices]
+  uint32_t region_a;
+  uint32_t region_b;
+  uint32_t xf;     // fp32 x (may alias the routed part of region B)
+  uint32_t xq;
+  uint32_t logit;  // fp32 [E]
+  uint32_t cand;   // top-k candidates: fp32 [warps][k] values, int32 [warps][k] ids
+  uint32_t ypart;  // fp32 [(k+1)][down rows]
+  uint32_t rpart;  // fp32 [router rows][slices]
+  uint32_t cons;   // inside region A, past the P1 data (free once the routed pairs are
+                   // consumed): per-warp staged a-groups, then per-warp partial down
+                   // sums fp32 [warps][2][kMaxSliceRows]
+  uint32_t prod;   // u32 [k * I / 64]: CTAs producing each routed a-group (static)
   uint32_t mbar;
   uint32_t total;
 };
@@ -87,7 +101,7 @@ struct FusedArgs {
   float* a;        // [(k+1)][I], shared expert last
   float* y;        // [(k+1)][H]
   float* ss_part;  // [gridDim.x]
-  unsigned* sync;  // [0] barrier arrivals, [1] exits
+  unsigned* sync;  // [0] barrier arrivals, [1] exits, [kSyncGroups + g] publications of a-group g
   FusedPlan plan;
 };
 
@@ -113,10 +127,12 @@ __device__ __forceinline__ void bulk_g2s(void* dst, const void* src, uint32_t by
       : "memory");
 }
 
+// One try_wait; the thread may be suspended (up to the hint, 20 us) until the
+// phase completes, so waiting warps do not compete for issue slots.
 __device__ __forceinline__ bool mbar_try(uint64_t* bar, uint32_t parity) {
   uint32_t done;
   asm volatile(
-      "{ .reg .pred p; mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2; selp.u32 %0, 1, 0, p; }"
+      "{ .reg .pred p; mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2, 20000; selp.u32 %0, 1, 0, p; }"
       : "=r"(done)
       : "r"(smem_u32(bar)), "r"(parity)
       : "memory");
@@ -165,14 +181,14 @@ __device__ __forceinline__ void lds_xv(const StagedX& s, int ng, int g, uint4* x
 // Dot products of gate and up row of a pair held in shared memory (codes of
 // both rows, then their scale-bias words), one lane group per pair.
 template <int BITS>
-__device__ __forceinline__ void pair_dot_smem(const uint8_t* slot, int H, const StagedX& sx, int lg,
-                                              int lpr, float* yg, float* yu) {
+__device__ __forceinline__ void pair_dot_smem(const uint8_t* codes, const uint32_t* sb, int H,
+                                              const StagedX& sx, int lg, int lpr, float* yg, float* yu) {
   const int ng = H / 64;
   const int rb = H * BITS / 8;
-  const uint8_t* rg = slot;
-  const uint8_t* ru = slot + rb;
-  const uint32_t* sbg = reinterpret_cast<const uint32_t*>(slot + 2 * rb);
-  const uint32_t* sbu = sbg + ng;
+  const uint8_t* rg = codes;
+  const uint8_t* ru = codes + rb;
+  const uint32_t* sbg = sb;
+  const uint32_t* sbu = sb + ng;
   float g = 0.f, u = 0.f;
   for (int gi = lg; gi < ng; gi += lpr) {
     const GroupCodes<BITS> cg = lds_group<BITS>(rg, ng, gi);
@@ -207,68 +223,66 @@ __device__ __forceinline__ float row_dot_smem(const uint8_t* codes, const uint32
   return y;
 }
 
-// Warp-level top-k over lg[0..E) (shared memory): lane r < k returns the
-// r-th selection in *id / *val.  Larger first, NaN last, ties to the lower index.
-__device__ __forceinline__ void warp_topk(const float* lg, int E, int k, int* id, float* val) {
-  const int lane = threadIdx.x & 31;
-  uint32_t taken = 0;
-  int my_id = 0;
-  float my_val = 0.f;
-  for (int r = 0; r < k; ++r) {
-    float bv = 0.f;
-    int bi = -1;
-    for (int i = 0, e = lane; e < E; ++i, e += 32) {
-      if (taken & (1u << i)) continue;
-      const float v = lg[e];
-      bool better;
-      if (bi < 0) better = true;
-      else {
-        const bool an = isnan(v), bn = isnan(bv);
-        better = (an || bn) ? (an && bn ? e < bi : bn) : (v != bv ? v > bv : e < bi);
-      }
-      if (better) { bv = v; bi = e; }
-    }
-#pragma unroll
-    for (int o = 16; o > 0; o >>= 1) {
-      const float ov = __shfl_xor_sync(0xffffffffu, bv, o);
-      const int oi = __shfl_xor_sync(0xffffffffu, bi, o);
-      bool better;
-      if (oi < 0) better = false;
-      else if (bi < 0) better = true;
-      else {
-        const bool an = isnan(ov), bn = isnan(bv);
-        better = (an || bn) ? (an && bn ? oi < bi : bn) : (ov != bv ? ov > bv : oi < bi);
-      }
-      if (better) { bv = ov; bi = oi; }
-    }
-    if (bi >= 0 && (bi & 31) == lane) taken |= 1u << (bi >> 5);
-    if (lane == r) { my_id = bi; my_val = bv; }
+// Routing key of logit v at index e: one 64-bit integer whose order is the
+// selection order -- larger value first, NaN after every number, +0 and -0
+// equal, then the lower index.  Key 0 never names a logit ("none").
+__device__ __forceinline__ uint64_t route_key(float v, int e) {
+  uint32_t k32;
+  if (isnan(v)) k32 = 0u;
+  else {
+    const uint32_t u = __float_as_uint(v == 0.f ? 0.f : v);
+    k32 = (u >> 31) ? ~u : (u | 0x80000000u);
   }
-  *id = my_id;
-  *val = my_val;
+  return ((uint64_t)k32 << 32) | (uint64_t)(0xFFFFFFFFu - (uint32_t)e);
+}
+
+__device__ __forceinline__ int key_index(uint64_t key) { return (int)(0xFFFFFFFFu - (uint32_t)key); }
+
+// Warp-wide selection of the k largest keys among the PER keys each lane
+// holds (0 = empty); the r-th selected key lands in lane r.  Two redux.sync
+// reductions per selection.
+template <int PER>
+__device__ __forceinline__ uint64_t warp_select_keys(uint64_t* key, int k) {
+  const int lane = threadIdx.x & 31;
+  uint64_t mine = 0;
+  for (int r = 0; r < k; ++r) {
+    uint64_t best = key[0];
+#pragma unroll
+    for (int i = 1; i < PER; ++i) best = key[i] > best ? key[i] : best;
+    const uint32_t hi = __reduce_max_sync(0xffffffffu, (uint32_t)(best >> 32));
+    const uint32_t lo = __reduce_max_sync(0xffffffffu, (uint32_t)(best >> 32) == hi ? (uint32_t)best : 0u);
+    const uint64_t win = ((uint64_t)hi << 32) | lo;
+#pragma unroll
+    for (int i = 0; i < PER; ++i)
+      if (key[i] == win) key[i] = 0;
+    if (lane == r) mine = win;
+  }
+  return mine;
 }
 
 // ------------------------------------------------------------ the kernel --
+template <int BITS, int SBITS>  // routed and shared code widths
 __global__ void __launch_bounds__(kFusedThreads, 1) fused_stack_kernel(const __grid_constant__ FusedArgs A) {
   extern __shared__ __align__(128) unsigned char smem[];
   __shared__ int s_abort;
   __shared__ int s_ids[kFusedMaxK];
   __shared__ float s_p[kFusedMaxK];
   __shared__ float s_red[kFusedWarps];
-  __shared__ float s_r;
 
   const int c = blockIdx.x, nC = gridDim.x;
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int H = A.H, I = A.I, E = A.E, k = A.k;
   const int ngH = H / 64, ngI = I / 64;
-  const int lprH = ngH < 32 ? ngH : 32, lprI = ngI < 32 ? ngI : 32;
+  const int lprH = ngH < 32 ? ngH : 32;
   const FusedPlan& P = A.plan;
   uint64_t* mbar = reinterpret_cast<uint64_t*>(smem + P.mbar);
   uint8_t* regA = smem + P.region_a;
   uint8_t* regB = smem + P.region_b;
   float* xf = reinterpret_cast<float*>(smem + P.xf);
-  const StagedX sxq = staged_x_at(smem + P.xq, H);
+  unsigned char* xq_base = smem + P.xq;
+  const StagedX sxq = staged_x_at(xq_base, H);
   float* slog = reinterpret_cast<float*>(smem + P.logit);
+  uint64_t* cand = reinterpret_cast<uint64_t*>(smem + P.cand);  // [warps][k] routing keys
   float* ypart = reinterpret_cast<float*>(smem + P.ypart);
   float* rpart = reinterpret_cast<float*>(smem + P.rpart);
 
@@ -284,15 +298,44 @@ __global__ void __launch_bounds__(kFusedThreads, 1) fused_stack_kernel(const __g
 
   const RecordLayout LR = record_layout(A.bits, H, I);   // routed records
   const RecordLayout LS = record_layout(A.sbits, H, I);  // shared record
-  const uint32_t pair_r = (uint32_t)(2 * LR.gu_row_bytes + 2 * ngH * 4);
-  const uint32_t pair_s = (uint32_t)(2 * LS.gu_row_bytes + 2 * ngH * 4);
+  const uint32_t pc_r = (uint32_t)(2 * LR.gu_row_bytes), pc_s = (uint32_t)(2 * LS.gu_row_bytes);  // pair codes
+  const uint32_t psb = (uint32_t)(2 * ngH * 4);                                                     // pair scale-bias
   const uint32_t drow_r = (uint32_t)(LR.down_row_bytes), drow_s = (uint32_t)(LS.down_row_bytes);
+  // region A
+  uint8_t* sc_codes = regA + (size_t)nr * H * 4;
+  uint8_t* sc_sb = sc_codes + (size_t)nsp * pc_s;
+  uint8_t* rc_codes = regA;
+  uint8_t* rc_sb = regA + (size_t)nq * pc_r;
   // region B: shared down [codes nd*drow_s][sb nd*ngI*4], then routed down per expert
   uint8_t* sd_codes = regB;
   uint32_t* sd_sb = reinterpret_cast<uint32_t*>(regB + (size_t)nd * drow_s);
   uint8_t* rd_base = regB + (size_t)nd * (drow_s + ngI * 4);
   const size_t rd_stride = (size_t)nd * (drow_r + ngI * 4);
+  uint8_t* cons = smem + P.cons;
+  float* cons_wy = reinterpret_cast<float*>(cons + kFusedWarps * kWStage);
+  // number of CTAs whose pair share touches a-group gg and publish it once per
+  // layer: gg < k I / 64 are the routed experts' groups (routed pairs shared
+  // out over k I pairs), the next I / 64 the shared expert's (I pairs)
+  auto producers = [&](int gg) -> unsigned {
+    const bool routed = gg < k * ngI;
+    const int T = routed ? k * I : I;
+    const int first = (routed ? gg : gg - k * ngI) * 64, last = first + 63;
+    const int c_lo = (int)((((long long)first + 1) * nC - 1) / T);
+    const int c_hi = (int)((((long long)last + 1) * nC - 1) / T);
+    unsigned cnt = 0;
+    for (int cc = c_lo; cc <= c_hi; ++cc) {
+      int a0, a1;
+      share(T, cc, nC, &a0, &a1);
+      if (a0 < a1) ++cnt;
+    }
+    return cnt;
+  };
 
+  // static tables: producers of each routed a-group; first/last expert of each warp's groups
+  unsigned* s_prod = reinterpret_cast<unsigned*>(smem + P.prod);
+  const int U = (k + 1) * ngI;                              // a-groups: k routed experts, then the shared one
+  const int per_warp = (U + kFusedWarps - 1) / kFusedWarps;  // a-groups per warp in the down products
+  for (int gg = tid; gg < U; gg += kFusedThreads) s_prod[gg] = producers(gg);
   if (tid == 0) {
     s_abort = 0;
     for (int i = 0; i < kMbCount; ++i) mbar_init(&mbar[i], 1);
@@ -301,32 +344,37 @@ __global__ void __launch_bounds__(kFusedThreads, 1) fused_stack_kernel(const __g
   __syncthreads();
 
   unsigned bar_target = 0;
-  uint32_t cur_par = 0;
-  // slots armed by this lane of warp 0 in the current layer (bulk copies are
-  // issued by the lanes of warp 0; each lane drains its own on abort)
-  uint32_t armed[(kMbCount + 31) / 32];
+  // per issuing thread (lane 0 of a warp): slots armed, by the parity of their
+  // latest arming (each issuer drains its own copies on abort)
+  constexpr int kMW = (kMbCount + 31) / 32;
+  uint32_t armed[2][kMW];
 #pragma unroll
-  for (int i = 0; i < (kMbCount + 31) / 32; ++i) armed[i] = 0;
-
-  auto arm = [&](int slot, uint32_t bytes) {
+  for (int p = 0; p < 2; ++p)
+#pragma unroll
+    for (int i = 0; i < kMW; ++i) armed[p][i] = 0;
+  auto arm = [&](int slot, uint32_t bytes, uint32_t parity) {
     mbar_expect_tx(&mbar[slot], bytes);
-    armed[slot >> 5] |= 1u << (slot & 31);
+    armed[parity][slot >> 5] |= 1u << (slot & 31);
+    armed[parity ^ 1][slot >> 5] &= ~(1u << (slot & 31));
   };
 
-  auto grid_sync = [&]() -> bool {
+  // split grid barrier: arrive once this CTA's results are written, do local
+  // work, then wait (release/acquire on one counter, bounded spin)
+  auto grid_arrive = [&]() {
     __syncthreads();
     bar_target += (unsigned)nC;
+    if (tid == 0) asm volatile("red.release.gpu.global.add.u32 [%0], 1;" ::"l"(A.sync) : "memory");
+  };
+  auto grid_wait = [&]() -> bool {
     if (tid == 0) {
-      __threadfence();
-      atomicAdd(&A.sync[0], 1u);
-      const long long t0 = clock64();
       bool ok = false;
+      const long long t0 = clock64();
       while (true) {
-        const unsigned v = *reinterpret_cast<volatile unsigned*>(&A.sync[0]);
+        unsigned v;
+        asm volatile("ld.acquire.gpu.global.u32 %0, [%1];" : "=r"(v) : "l"(A.sync) : "memory");
         if (v >= bar_target) { ok = true; break; }
         if (clock64() - t0 > kWaitCycles) break;
       }
-      __threadfence();
       if (!ok) {
         s_abort = 1;
         raise_status(FMOE_STATUS_WAIT_TIMEOUT);
@@ -343,56 +391,118 @@ __global__ void __launch_bounds__(kFusedThreads, 1) fused_stack_kernel(const __g
     return false;
   };
 
-  for (int l = 0; l < A.n_layers; ++l) {
+  // bulk copies, issued by lane 0 of several warps in parallel (each issue
+  // takes a few hundred cycles; spreading them keeps any one warp short) ---
+  // router rows and the shared expert's gate/up pairs of layer l (region A)
+  auto issue_p1 = [&](int l) {
     const FusedLayer& LY = A.layers[l];
     const uint32_t par = (uint32_t)(l & 1);
-    cur_par = par;
-    // ------------------------------------------------------------ P1 --
-    if (warp == 0) {
-#pragma unroll
-      for (int i = 0; i < (kMbCount + 31) / 32; ++i) armed[i] = 0;
+    if (lane != 0) return;
+    fence_proxy_async();
+    for (int r = warp; r < nr; r += kFusedWarps) {
+      const int row = r0 + r;
+      const float* src = row < E ? LY.w_router + (size_t)row * H : LY.w_sg;
+      arm(kMbRouter + r, (uint32_t)H * 4, par);
+      bulk_g2s(regA + (size_t)r * H * 4, src, (uint32_t)H * 4, &mbar[kMbRouter + r]);
+    }
+    const int nch = (nsp + kPairsPerChunk - 1) / kPairsPerChunk;
+    for (int ch = (warp + kFusedWarps - nr % kFusedWarps) % kFusedWarps; ch < nch; ch += kFusedWarps) {
+      const int pa = ch * kPairsPerChunk, pb = min(nsp, pa + kPairsPerChunk), n = s0 + pa;
+      arm(kMbSPair + ch, (uint32_t)(pb - pa) * (pc_s + psb), par);
+      bulk_g2s(sc_codes + (size_t)pa * pc_s, LY.shared + LS.gu_codes + (size_t)n * pc_s, (uint32_t)(pb - pa) * pc_s,
+               &mbar[kMbSPair + ch]);
+      bulk_g2s(sc_sb + (size_t)pa * psb, LY.shared + LS.gu_sb + (size_t)n * psb, (uint32_t)(pb - pa) * psb,
+               &mbar[kMbSPair + ch]);
+    }
+  };
+  // the shared expert's down rows of layer l (region B, shared part)
+  auto issue_sdown = [&](int l) {
+    const FusedLayer& LY = A.layers[l];
+    if (nd > 0 && lane == 0 && warp == kFusedWarps - 1) {
       fence_proxy_async();
-      for (int r = lane; r < nr; r += 32) {
-        const int row = r0 + r;
-        const float* src = row < E ? LY.w_router + (size_t)row * H : LY.w_sg;
-        arm(kMbRouter + r, (uint32_t)H * 4);
-        bulk_g2s(regA + (size_t)r * H * 4, src, (uint32_t)H * 4, &mbar[kMbRouter + r]);
-      }
-      uint8_t* sp_base = regA + (size_t)nr * H * 4;
-      for (int p = lane; p < nsp; p += 32) {
-        const int n = s0 + p;
-        uint8_t* dst = sp_base + (size_t)p * pair_s;
-        arm(kMbSPair + p, pair_s);
-        bulk_g2s(dst, LY.shared + LS.gu_codes + (size_t)(2 * n) * LS.gu_row_bytes,
-                 (uint32_t)(2 * LS.gu_row_bytes), &mbar[kMbSPair + p]);
-        bulk_g2s(dst + 2 * LS.gu_row_bytes, LY.shared + LS.gu_sb + (size_t)(2 * n) * ngH * 4,
-                 (uint32_t)(2 * ngH * 4), &mbar[kMbSPair + p]);
-      }
-      if (nd > 0 && lane == 31) {
-        arm(kMbSDown, (uint32_t)nd * (drow_s + ngI * 4));
-        bulk_g2s(sd_codes, LY.shared + LS.down_codes + (size_t)i0 * drow_s, (uint32_t)nd * drow_s,
-                 &mbar[kMbSDown]);
-        bulk_g2s(sd_sb, LY.shared + LS.down_sb + (size_t)i0 * ngI * 4, (uint32_t)nd * ngI * 4,
-                 &mbar[kMbSDown]);
+      arm(kMbSDown, (uint32_t)nd * (drow_s + ngI * 4), (uint32_t)(l & 1));
+      bulk_g2s(sd_codes, LY.shared + LS.down_codes + (size_t)i0 * drow_s, (uint32_t)nd * drow_s, &mbar[kMbSDown]);
+      bulk_g2s(sd_sb, LY.shared + LS.down_sb + (size_t)i0 * ngI * 4, (uint32_t)nd * ngI * 4, &mbar[kMbSDown]);
+    }
+  };
+  // the routed experts' gate/up pairs of this CTA's share and down rows of its slice
+  auto issue_routed = [&](int l) {
+    const FusedLayer& LY = A.layers[l];
+    const uint32_t par = (uint32_t)(l & 1);
+    if (lane != 0) return;
+    fence_proxy_async();
+    const int nch = (nq + kPairsPerChunk - 1) / kPairsPerChunk;
+    for (int ch = warp; ch < nch; ch += kFusedWarps) {
+      const int qa = ch * kPairsPerChunk, qb = min(nq, qa + kPairsPerChunk);
+      arm(kMbRPair + ch, (uint32_t)(qb - qa) * (pc_r + psb), par);
+      for (int q = qa; q < qb;) {  // runs within one expert
+        const int gq = q0 + q, j = gq / I, n = gq % I;
+        const int cnt = min(qb - q, I - n);
+        const uint8_t* rec = LY.experts + (size_t)s_ids[j] * LR.bytes;
+        bulk_g2s(rc_codes + (size_t)q * pc_r, rec + LR.gu_codes + (size_t)n * pc_r, (uint32_t)cnt * pc_r,
+                 &mbar[kMbRPair + ch]);
+        bulk_g2s(rc_sb + (size_t)q * psb, rec + LR.gu_sb + (size_t)n * psb, (uint32_t)cnt * psb, &mbar[kMbRPair + ch]);
+        q += cnt;
       }
     }
+    if (nd > 0) {
+      for (int j = (warp + kFusedWarps - nch % kFusedWarps) % kFusedWarps; j < k; j += kFusedWarps) {
+        const uint8_t* rec = LY.experts + (size_t)s_ids[j] * LR.bytes;
+        uint8_t* dst = rd_base + (size_t)j * rd_stride;
+        arm(kMbRDown + j, (uint32_t)nd * (drow_r + ngI * 4), par);
+        bulk_g2s(dst, rec + LR.down_codes + (size_t)i0 * drow_r, (uint32_t)nd * drow_r, &mbar[kMbRDown + j]);
+        bulk_g2s(dst + (size_t)nd * drow_r, rec + LR.down_sb + (size_t)i0 * ngI * 4, (uint32_t)nd * ngI * 4,
+                 &mbar[kMbRDown + j]);
+      }
+    }
+  };
+
+  // r = (sum of the CTAs' partial sums of h'^2 / H + eps)^(-1/2), the same
+  // summation order in every CTA; all threads take part
+  auto norm_scale = [&]() -> float {
+    float v = 0.f;
+    for (int i = tid; i < nC; i += kFusedThreads) v += ldcg_f(A.ss_part + i);
+    v = warp_sum(v);
+    if (lane == 0) s_red[warp] = v;
+    __syncthreads();
+    const float t = warp_sum(lane < kFusedWarps ? s_red[lane] : 0.f);  // same order in every warp
+    return 1.f / sqrtf(t / (float)H + A.eps);
+  };
+
+  if (A.n_layers > 0) {
+    issue_p1(0);
+    issue_sdown(0);
+  }
+
+  for (int l = 0; l < A.n_layers; ++l) {
+    const uint32_t par = (uint32_t)(l & 1);
+    // ------------------------------------------------------------ P1 --
     // x for this layer: the input (first layer) or h' r w of the previous layer
     if (l == 0) {
-      for (int j = tid; j < H; j += kFusedThreads) xf[j] = ldcg_f(A.xn + j);
+      for (int j = tid * 4; j < H; j += kFusedThreads * 4)
+        *reinterpret_cast<float4*>(xf + j) = __ldcg(reinterpret_cast<const float4*>(A.xn + j));
     } else {
-      if (warp == 0) {
-        float s = 0.f;
-        for (int i = lane; i < nC; i += 32) s += ldcg_f(A.ss_part + i);
-        s = warp_sum(s);
-        if (lane == 0) s_r = 1.f / sqrtf(s / (float)H + A.eps);
-      }
-      __syncthreads();
-      const float r = s_r;
+      constexpr int kMaxV = 4;  // float4 per thread (H <= 8192)
+      float4 hv[kMaxV], wv[kMaxV];
       const float* wprev = A.layers[l - 1].norm_w;
-      for (int j = tid; j < H; j += kFusedThreads) xf[j] = ldcg_f(A.h + j) * r * wprev[j];
+#pragma unroll
+      for (int it = 0; it < kMaxV; ++it) {
+        const int j = (it * kFusedThreads + tid) * 4;
+        if (j < H) {
+          hv[it] = __ldcg(reinterpret_cast<const float4*>(A.h + j));
+          wv[it] = __ldg(reinterpret_cast<const float4*>(wprev + j));
+        }
+      }
+      const float r = norm_scale();
+#pragma unroll
+      for (int it = 0; it < kMaxV; ++it) {
+        const int j = (it * kFusedThreads + tid) * 4;
+        if (j < H)
+          *reinterpret_cast<float4*>(xf + j) =
+              make_float4(hv[it].x * r * wv[it].x, hv[it].y * r * wv[it].y, hv[it].z * r * wv[it].z,
+                          hv[it].w * r * wv[it].w);
+      }
     }
-    __syncthreads();
-    stage_x(xf, H, sxq);
     __syncthreads();
     // router rows: units (row, slice)
     for (int u = warp; u < nr * nsl; u += kFusedWarps) {
@@ -412,25 +522,6 @@ __global__ void __launch_bounds__(kFusedThreads, 1) fused_stack_kernel(const __g
       acc = warp_sum(acc);
       if (lane == 0) rpart[r * nsl + sl] = acc;
     }
-    // shared expert gate/up pairs
-    {
-      const int ppu = 32 / lprH;  // pairs per warp unit
-      const int ps = lane / lprH, lg = lane % lprH;
-      const uint8_t* sp_base = regA + (size_t)nr * H * 4;
-      for (int u0 = warp * ppu; u0 < nsp; u0 += kFusedWarps * ppu) {
-        const int p = u0 + ps;
-        bool ok = true;
-        if (p < nsp) ok = wait_slot(kMbSPair + p, par);
-        if (!__all_sync(0xffffffffu, ok)) break;
-        float g = 0.f, uu = 0.f;
-        const int pp = p < nsp ? p : nsp - 1;
-        if (A.sbits == 4)
-          pair_dot_smem<4>(sp_base + (size_t)pp * pair_s, H, sxq, lg, lprH, &g, &uu);
-        else
-          pair_dot_smem<2>(sp_base + (size_t)pp * pair_s, H, sxq, lg, lprH, &g, &uu);
-        if (lg == 0 && p < nsp) A.a[(size_t)k * I + s0 + p] = silu_mul(g, uu);
-      }
-    }
     __syncthreads();
     if (tid < nr && !s_abort) {
       float v = rpart[tid * nsl];
@@ -439,60 +530,87 @@ __global__ void __launch_bounds__(kFusedThreads, 1) fused_stack_kernel(const __g
       if (row < E) A.logits[row] = v;
       else A.gamma[0] = 1.f / (1.f + expf(-v));
     }
-    if (s_abort || !grid_sync()) break;
-    // ------------------------------------------------------------ P2 --
-    if (warp == 0) {
-      bool nan_seen = false;
-      for (int e = lane; e < E; e += 32) {
-        const float v = ldcg_f(A.logits + e);
-        nan_seen |= isnan(v);
-        slog[e] = v;
+    if (s_abort) break;
+    grid_arrive();  // B1: logits written
+    // while the other CTAs finish: quantise x, run the shared expert's gate/up pairs
+    stage_x(xf, H, sxq);
+    __syncthreads();
+    {
+      const int ppu = 32 / lprH;  // pairs per warp unit
+      const int ps = lane / lprH, lg = lane % lprH;
+      for (int u0 = warp * ppu; u0 < nsp; u0 += kFusedWarps * ppu) {
+        const int p = u0 + ps;
+        bool ok = true;
+        if (p < nsp) ok = wait_slot(kMbSPair + p / kPairsPerChunk, par);
+        if (!__all_sync(0xffffffffu, ok)) break;
+        float g = 0.f, uu = 0.f;
+        const int pp = p < nsp ? p : nsp - 1;
+        const uint8_t* cp = sc_codes + (size_t)pp * pc_s;
+        const uint32_t* sp = reinterpret_cast<const uint32_t*>(sc_sb + (size_t)pp * psb);
+        pair_dot_smem<SBITS>(cp, sp, H, sxq, lg, lprH, &g, &uu);
+        if (lg == 0 && p < nsp) A.a[(size_t)k * I + s0 + p] = silu_mul(g, uu);
       }
-      __syncwarp();
-      int id;
-      float val;
-      warp_topk(slog, E, k, &id, &val);
-      float m = -INFINITY;
-      for (int r = 0; r < k; ++r) {
-        const float vr = __shfl_sync(0xffffffffu, val, r);
-        if (!isnan(vr)) m = fmaxf(m, vr);
-      }
-      const float pe = (lane < k && !isnan(val)) ? expf(val - m) : 0.f;
-      const float z = warp_sum(pe);
-      if (lane < k) {
-        s_ids[lane] = id;
-        s_p[lane] = z > 0.f ? pe / z : 0.f;
-        if (c == 0) {
-          A.ids[lane] = id;
-          A.weights[lane] = s_p[lane];
-        }
-      }
-      const bool any_nan = __any_sync(0xffffffffu, nan_seen);
-      if (c == 0 && lane == 0 && any_nan) raise_status(FMOE_STATUS_NAN_LOGIT);
     }
     __syncthreads();
-    if (warp == 0) {
-      fence_proxy_async();
-      for (int q = lane; q < nq; q += 32) {
-        const int gq = q0 + q, j = gq / I, n = gq % I;
-        const uint8_t* rec = LY.experts + (size_t)s_ids[j] * LR.bytes;
-        uint8_t* dst = regA + (size_t)q * pair_r;
-        arm(kMbRPair + q, pair_r);
-        bulk_g2s(dst, rec + LR.gu_codes + (size_t)(2 * n) * LR.gu_row_bytes, (uint32_t)(2 * LR.gu_row_bytes),
-                 &mbar[kMbRPair + q]);
-        bulk_g2s(dst + 2 * LR.gu_row_bytes, rec + LR.gu_sb + (size_t)(2 * n) * ngH * 4, (uint32_t)(2 * ngH * 4),
-                 &mbar[kMbRPair + q]);
+    // publish the shared expert's a-groups this CTA produced
+    if (nsp > 0 && tid <= (s1 - 1) / 64 - s0 / 64)
+      asm volatile("red.release.gpu.global.add.u32 [%0], 1;" ::"l"(A.sync + kSyncGroups + k * ngI + s0 / 64 + tid)
+                   : "memory");
+    if (s_abort || !grid_wait()) break;
+    // ------------------------------------------------------------ P2 --
+    {
+      // routing: every thread keys up to two logits; per-warp top-k, then one
+      // warp merges the warps' candidates
+      uint64_t key[2];
+      bool nan_seen = false;
+      float lv[2];
+#pragma unroll
+      for (int i = 0; i < 2; ++i) {
+        const int e = tid + i * kFusedThreads;
+        lv[i] = e < E ? ldcg_f(A.logits + e) : 0.f;
       }
-      if (nd > 0) {
-        for (int j = lane; j < k; j += 32) {
-          const uint8_t* rec = LY.experts + (size_t)s_ids[j] * LR.bytes;
-          uint8_t* dst = rd_base + (size_t)j * rd_stride;
-          arm(kMbRDown + j, (uint32_t)nd * (drow_r + ngI * 4));
-          bulk_g2s(dst, rec + LR.down_codes + (size_t)i0 * drow_r, (uint32_t)nd * drow_r, &mbar[kMbRDown + j]);
-          bulk_g2s(dst + (size_t)nd * drow_r, rec + LR.down_sb + (size_t)i0 * ngI * 4, (uint32_t)nd * ngI * 4,
-                   &mbar[kMbRDown + j]);
+#pragma unroll
+      for (int i = 0; i < 2; ++i) {
+        const int e = tid + i * kFusedThreads;
+        key[i] = 0;
+        if (e < E) {
+          nan_seen |= isnan(lv[i]);
+          slog[e] = lv[i];
+          key[i] = route_key(lv[i], e);
         }
       }
+      const uint64_t wk = warp_select_keys<2>(key, k);
+      if (lane < k) cand[warp * k + lane] = wk;
+      nan_seen = __syncthreads_or(nan_seen);
+      if (warp == 0) {
+        uint64_t kk[4];
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+          const int idx = lane + 32 * i;
+          kk[i] = idx < kFusedWarps * k ? cand[idx] : 0;
+        }
+        const uint64_t win = warp_select_keys<4>(kk, k);
+        const int sel = lane < k ? key_index(win) : 0;
+        const float val = lane < k ? slog[sel] : 0.f;
+        float m = -INFINITY;
+        for (int r = 0; r < k; ++r) {
+          const float vr = __shfl_sync(0xffffffffu, val, r);
+          if (!isnan(vr)) m = fmaxf(m, vr);
+        }
+        const float pe = (lane < k && !isnan(val)) ? expf(val - m) : 0.f;
+        const float z = warp_sum(pe);
+        if (lane < k) {
+          s_ids[lane] = sel;
+          s_p[lane] = z > 0.f ? pe / z : 0.f;
+          if (c == 0) {
+            A.ids[lane] = sel;
+            A.weights[lane] = s_p[lane];
+          }
+        }
+        if (c == 0 && lane == 0 && nan_seen) raise_status(FMOE_STATUS_NAN_LOGIT);
+      }
+      __syncthreads();
+      issue_routed(l);
     }
     {
       const int ppu = 32 / lprH;
@@ -500,53 +618,149 @@ __global__ void __launch_bounds__(kFusedThreads, 1) fused_stack_kernel(const __g
       for (int u0 = warp * ppu; u0 < nq; u0 += kFusedWarps * ppu) {
         const int q = u0 + ps;
         bool ok = true;
-        if (q < nq) ok = wait_slot(kMbRPair + q, par);
+        if (q < nq) ok = wait_slot(kMbRPair + q / kPairsPerChunk, par);
         if (!__all_sync(0xffffffffu, ok)) break;
         float g = 0.f, uu = 0.f;
         const int qq = q < nq ? q : nq - 1;
-        if (A.bits == 4)
-          pair_dot_smem<4>(regA + (size_t)qq * pair_r, H, sxq, lg, lprH, &g, &uu);
-        else
-          pair_dot_smem<2>(regA + (size_t)qq * pair_r, H, sxq, lg, lprH, &g, &uu);
-        if (lg == 0 && q < nq) {
-          const int gq = q0 + q;
-          A.a[gq] = silu_mul(g, uu);  // a[j][n] with gq = j * I + n
-        }
-      }
-    }
-    if (s_abort || !grid_sync()) break;
-    // ------------------------------------------------------------ P3 --
-    // stage a of the k routed experts and the shared one (region A is free)
-    const size_t sa_bytes = (staged_x_bytes(I) + 15) & ~(size_t)15;
-    for (int j = 0; j <= k; ++j) stage_x(A.a + (size_t)j * I, I, staged_x_at(regA + j * sa_bytes, I), true);
-    __syncthreads();
-    if (nd > 0) {
-      const int rpu = 32 / lprI;  // rows per warp unit
-      const int rs = lane / lprI, lg = lane % lprI;
-      const int units_per_expert = (nd + rpu - 1) / rpu;
-      for (int u = warp; u < (k + 1) * units_per_expert; u += kFusedWarps) {
-        const int j = u / units_per_expert, rr = (u % units_per_expert) * rpu + rs;
-        const bool shared = j == k;
-        bool ok = wait_slot(shared ? kMbSDown : kMbRDown + j, par);
-        if (!__all_sync(0xffffffffu, ok)) break;
-        const StagedX sa = staged_x_at(regA + j * sa_bytes, I);
-        const int row = rr < nd ? rr : nd - 1;
-        float v;
-        if (shared) {
-          const uint8_t* codes = sd_codes + (size_t)row * drow_s;
-          const uint32_t* sb = sd_sb + (size_t)row * ngI;
-          v = A.sbits == 4 ? row_dot_smem<4>(codes, sb, I, sa, lg, lprI) : row_dot_smem<2>(codes, sb, I, sa, lg, lprI);
-        } else {
-          const uint8_t* base = rd_base + (size_t)j * rd_stride;
-          const uint8_t* codes = base + (size_t)row * drow_r;
-          const uint32_t* sb = reinterpret_cast<const uint32_t*>(base + (size_t)nd * drow_r) + (size_t)row * ngI;
-          v = A.bits == 4 ? row_dot_smem<4>(codes, sb, I, sa, lg, lprI) : row_dot_smem<2>(codes, sb, I, sa, lg, lprI);
-        }
-        if (lg == 0 && rr < nd) ypart[j * nd + rr] = v;
+        const uint8_t* cp = rc_codes + (size_t)qq * pc_r;
+        const uint32_t* sp = reinterpret_cast<const uint32_t*>(rc_sb + (size_t)qq * psb);
+        pair_dot_smem<BITS>(cp, sp, H, sxq, lg, lprH, &g, &uu);
+        if (lg == 0 && q < nq) A.a[q0 + q] = silu_mul(g, uu);  // a[j][n], q0 + q = j * I + n
       }
     }
     __syncthreads();
     if (s_abort) break;
+    // this CTA's SwiGLU outputs are written: publish them, one counter per
+    // 64-wide group of a (release: the writes above are visible to whoever
+    // acquires the counter)
+    if (nq > 0 && tid <= (q1 - 1) / 64 - q0 / 64)
+      asm volatile("red.release.gpu.global.add.u32 [%0], 1;" ::"l"(A.sync + kSyncGroups + q0 / 64 + tid) : "memory");
+    // ---------------------------------------------- down products, dataflow --
+    // The routed experts' down rows of this CTA's hidden slice, one a-group at
+    // a time: each warp owns a contiguous run of a-groups, waits (one round of
+    // polls) until the CTAs producing them have published them, loads them
+    // (one round trip), then quantises each group and accumulates it, one
+    // hidden row per lane.  The warps' sums are added in warp order.
+    if (nd > 0) {
+      constexpr int kBatch = 6;
+      const int u_lo = min(U, warp * per_warp), u_hi = min(U, u_lo + per_warp);
+      uint8_t* wst = cons + warp * kWStage;
+      const uint4* wxs = reinterpret_cast<const uint4*>(wst);
+      float* wdx = reinterpret_cast<float*>(wst + 128);
+      float acc0 = 0.f, acc1 = 0.f;
+      const int j_first = u_lo < u_hi ? u_lo / ngI : -1;
+      int j_cur = -1;
+      bool ok = true;
+      for (int ub = u_lo; ub < u_hi && ok; ub += kBatch) {
+        const int nb = min(kBatch, u_hi - ub);
+        // 1. one round of polls for the batch
+        bool ready = lane >= nb;
+        const long long t0 = clock64();
+        while (true) {
+          if (!ready) {
+            unsigned v;
+            asm volatile("ld.acquire.gpu.global.u32 %0, [%1];" : "=r"(v) : "l"(A.sync + kSyncGroups + ub + lane)
+                         : "memory");
+            ready = v >= (unsigned)(l + 1) * s_prod[ub + lane];
+          }
+          if (__all_sync(0xffffffffu, ready)) break;
+          if (clock64() - t0 > kWaitCycles) {
+            if (lane == 0) {
+              s_abort = 1;
+              raise_status(FMOE_STATUS_WAIT_TIMEOUT);
+            }
+            ok = false;
+            break;
+          }
+        }
+        if (!ok) break;
+        // 2. one round of loads: lane holds inputs 2 lane, 2 lane + 1 of each group
+        float2 av[kBatch];
+#pragma unroll
+        for (int t = 0; t < kBatch; ++t)
+          if (t < nb) {
+            const int u = ub + t;
+            av[t] = __ldcg(reinterpret_cast<const float2*>(A.a + (size_t)(u / ngI) * I + (u % ngI) * 64) + lane);
+          }
+        // 3. quantise and accumulate each group
+#pragma unroll 1
+        for (int t = 0; t < nb; ++t) {
+          const int u = ub + t, j = u / ngI, g = u % ngI;
+          if (j != j_cur) {
+            if (j_cur >= 0) {  // flush the previous expert's sums
+              float* wy = cons_wy + (warp * 2 + (j_cur == j_first ? 0 : 1)) * kMaxSliceRows;
+              wy[lane] = acc0;
+              wy[lane + 32] = acc1;
+              acc0 = acc1 = 0.f;
+            }
+            ok = wait_slot(j == k ? kMbSDown : kMbRDown + j, par);
+            if (!__all_sync(0xffffffffu, ok)) { ok = false; break; }
+            j_cur = j;
+          }
+          float m = fmaxf(fabsf(av[t].x), fabsf(av[t].y));
+#pragma unroll
+          for (int o = 16; o > 0; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
+          const float inv = m > 0.f ? 32767.f / m : 0.f;
+          const float delta = m * (1.f / 32767.f);
+          int qa = __float2int_rn(av[t].x * inv), qb = __float2int_rn(av[t].y * inv);
+          qa = qa > 32767 ? 32767 : (qa < -32767 ? -32767 : qa);
+          qb = qb > 32767 ? 32767 : (qb < -32767 ? -32767 : qb);
+          int isum = qa + qb;
+#pragma unroll
+          for (int o = 16; o > 0; o >>= 1) isum += __shfl_xor_sync(0xffffffffu, isum, o);
+          __syncwarp();  // the previous group's staged values have been read
+          reinterpret_cast<uint32_t*>(wst)[lane] = (uint32_t)(qa & 0xFFFF) | ((uint32_t)qb << 16);
+          if (lane == 0) {
+            wdx[0] = delta;
+            wdx[1] = delta * (float)isum;
+          }
+          __syncwarp();
+          uint4 xv[8];
+#pragma unroll
+          for (int q = 0; q < 8; ++q) xv[q] = wxs[q];
+          const float dl = wdx[0], xsm = wdx[1];
+          const bool shd = j == k;
+          const uint8_t* base = shd ? sd_codes : rd_base + (size_t)j * rd_stride;
+          const uint32_t drow = shd ? drow_s : drow_r;
+          const uint32_t* sbb = reinterpret_cast<const uint32_t*>(base + (size_t)nd * drow);
+#pragma unroll 1
+          for (int half = 0; half < 2; ++half) {
+            const int rr = lane + 32 * half;
+            if (rr >= nd) break;
+            const uint8_t* cp = base + (size_t)rr * drow;
+            const int A32 = shd ? group_dot<SBITS>(lds_group<SBITS>(cp, ngI, g), xv)
+                                : group_dot<BITS>(lds_group<BITS>(cp, ngI, g), xv);
+            const float y = group_epilogue(half ? acc1 : acc0, sbb[rr * ngI + g], A32, dl, xsm);
+            if (half) acc1 = y;
+            else acc0 = y;
+          }
+        }
+      }
+      if (ok && j_cur >= 0) {
+        float* wy = cons_wy + (warp * 2 + (j_cur == j_first ? 0 : 1)) * kMaxSliceRows;
+        wy[lane] = acc0;
+        wy[lane + 32] = acc1;
+      }
+    }
+    __syncthreads();
+    if (s_abort) break;
+    // the routed down rows are consumed and the a-groups loaded: the next
+    // layer's router rows and shared pairs can stream now
+    if (l + 1 < A.n_layers) issue_p1(l + 1);
+    // y of each expert for this slice: the warps' sums in warp order
+    for (int idx = tid; idx < (k + 1) * nd; idx += kFusedThreads) {
+      const int j = idx / nd, rr = idx - j * nd;
+      float v = 0.f;
+      for (int w = 0; w < kFusedWarps; ++w) {
+        const int lo = w * per_warp;
+        if (lo >= U) break;
+        const int jf = lo / ngI, jl = (min(U, lo + per_warp) - 1) / ngI;
+        if (jf == j) v += cons_wy[(w * 2) * kMaxSliceRows + rr];
+        else if (jl == j) v += cons_wy[(w * 2 + 1) * kMaxSliceRows + rr];
+      }
+      ypart[j * nd + rr] = v;
+    }
+    __syncthreads();
     {
       const float gm = ldcg_f(A.gamma);
       float ss = 0.f;
@@ -568,35 +782,31 @@ __global__ void __launch_bounds__(kFusedThreads, 1) fused_stack_kernel(const __g
         A.ss_part[c] = t;
       }
     }
-    if (!grid_sync()) break;
+    grid_arrive();  // B3: h' and the partial sums written
+    // the shared down rows are consumed: the next layer's can stream now
+    if (l + 1 < A.n_layers) issue_sdown(l + 1);
+    if (!grid_wait()) break;
   }
 
   if (!s_abort) {
     // epilogue: xn' of the last layer for this CTA's rows
-    if (warp == 0) {
-      float s = 0.f;
-      for (int i = lane; i < nC; i += 32) s += ldcg_f(A.ss_part + i);
-      s = warp_sum(s);
-      if (lane == 0) s_r = 1.f / sqrtf(s / (float)H + A.eps);
-    }
-    __syncthreads();
-    const float r = s_r;
+    const float r = norm_scale();
     const float* w = A.layers[A.n_layers - 1].norm_w;
     for (int i = i0 + tid; i < i1; i += kFusedThreads) A.xn[i] = ldcg_f(A.h + i) * r * w[i];
     __syncthreads();
     if (tid == 0) {
       __threadfence();
       const unsigned prev = atomicAdd(&A.sync[1], 1u);
-      if (prev == (unsigned)nC - 1) {  // every CTA is past its last barrier
-        A.sync[0] = 0;
-        A.sync[1] = 0;
+      if (prev == (unsigned)nC - 1) {  // every CTA is past its last barrier and wait
+        for (int i = 0; i < kSyncGroups + (k + 1) * ngI; ++i) A.sync[i] = 0;
         __threadfence();
       }
     }
-  } else if (warp == 0) {
-    // drain: wait (bounded) for this lane's own copies still in flight
-    for (int s = 0; s < kMbCount; ++s)
-      if (armed[s >> 5] & (1u << (s & 31))) (void)mbar_wait(&mbar[s], cur_par);
+  } else if (lane == 0) {
+    // drain: wait (bounded) for this issuer's own copies still in flight
+    for (int p = 0; p < 2; ++p)
+      for (int s2 = 0; s2 < kMbCount; ++s2)
+        if (armed[p][s2 >> 5] & (1u << (s2 & 31))) (void)mbar_wait(&mbar[s2], (uint32_t)p);
   }
 }
 
@@ -607,32 +817,36 @@ inline bool fused_plan(int H, int I, int E, int k, int bits, int sbits, int n_ct
   // must be 16-byte aligned: a down row's scale-bias words (I/64 * 4 bytes)
   // and a pair's (2 * H/64 * 4 bytes) must come in multiples of 16 bytes
   if ((I / 64) % 4 != 0 || (H / 64) % 2 != 0) return false;
+  if (E > 2 * kFusedThreads || k > kFusedMaxK) return false;
   auto cdiv = [](long long a, long long b) { return (a + b - 1) / b; };
   const long long nr = cdiv(E + 1, n_ctas), nsp = cdiv(I, n_ctas), nq = cdiv((long long)k * I, n_ctas),
                   nd = cdiv(H, n_ctas);
-  if (nr > kFusedMaxRouterRows || nsp > kFusedMaxSharedPairs || nq > kFusedMaxRoutedPairs || k > kFusedMaxK)
-    return false;
+  if (nr > kFusedMaxRouterRows || nsp > kFusedMaxSharedPairs || nq > kFusedMaxRoutedPairs) return false;
   const RecordLayout LR = record_layout(bits, H, I), LS = record_layout(sbits, H, I);
   const int ngH = H / 64, ngI = I / 64;
-  const long long pair_r = 2 * (long long)LR.gu_row_bytes + 2 * ngH * 4;
-  const long long pair_s = 2 * (long long)LS.gu_row_bytes + 2 * ngH * 4;
+  const long long psb = 2LL * ngH * 4;
+  const long long pair_r = 2 * (long long)LR.gu_row_bytes + psb;
+  const long long pair_s = 2 * (long long)LS.gu_row_bytes + psb;
   const long long sa = ((long long)staged_x_bytes(I) + 15) & ~15LL;
   auto al = [](long long v) { return (v + 127) & ~127LL; };
+  if (nd > kMaxSliceRows || (long long)(k + 1) * ngI > kMaxGroupCounters) return false;
   const long long a_p1 = nr * H * 4 + nsp * pair_s;
   const long long a_p2 = nq * pair_r;
-  const long long a_p3 = (k + 1) * sa;
-  long long regA = a_p1 > a_p2 ? a_p1 : a_p2;
-  regA = regA > a_p3 ? regA : a_p3;
+  const long long cons_off = (a_p1 + 127) & ~127LL;
+  const long long cons_bytes = (long long)kFusedWarps * kWStage + (long long)kFusedWarps * 2 * kMaxSliceRows * 4;
+  const long long regA = a_p2 > cons_off + cons_bytes ? a_p2 : cons_off + cons_bytes;
   const long long sdown = nd * ((long long)LS.down_row_bytes + ngI * 4);
   const long long rdown = k * nd * ((long long)LR.down_row_bytes + ngI * 4);
+  const long long xq = (long long)staged_x_bytes(H);
   FusedPlan p;
   long long o = 0;
   p.region_a = (uint32_t)o;
+  p.cons = (uint32_t)(o + cons_off);
   o = al(o + regA);
   p.region_b = (uint32_t)o;
-  const long long xf_bytes = (long long)(H > I ? H : I) * 4;
+  const long long xf_bytes = (long long)H * 4;
   if (rdown >= xf_bytes) {
-    p.xf = (uint32_t)(o + sdown);  // aliases the routed down rows (P1 / P3 staging only)
+    p.xf = (uint32_t)(o + sdown);  // aliases the routed down rows (P1 only)
     o = al(o + sdown + rdown);
   } else {
     o = al(o + sdown + rdown);
@@ -640,13 +854,17 @@ inline bool fused_plan(int H, int I, int E, int k, int bits, int sbits, int n_ct
     o = al(o + xf_bytes);
   }
   p.xq = (uint32_t)o;
-  o = al(o + (long long)staged_x_bytes(H));
+  o = al(o + xq);
   p.logit = (uint32_t)o;
   o = al(o + (long long)E * 4);
+  p.cand = (uint32_t)o;
+  o = al(o + 2LL * kFusedWarps * kFusedMaxK * 4);
   p.ypart = (uint32_t)o;
   o = al(o + (k + 1) * nd * 4);
   p.rpart = (uint32_t)o;
   o = al(o + nr * (H >= 512 ? H / 512 : 1) * 4);
+  p.prod = (uint32_t)o;
+  o = al(o + 4LL * (k + 1) * ngI);
   p.mbar = (uint32_t)o;
   o = al(o + kMbCount * 8);
   p.total = (uint32_t)o;

@@ -469,9 +469,9 @@ constexpr int kMaxSMs = 1024;
 
 static WsLayout ws_layout(int H, int I, int E, int k, int T) {
   WsLayout w;
-  w.sync = 0;    // grid-barrier counters of the fused kernel
-  w.ss = 256;    // per-CTA partial sums of h'^2
-  size_t o = 256 + (size_t)kMaxSMs * 4;
+  w.sync = 0;    // grid-barrier and a-group publication counters of the fused kernel (1024 words)
+  w.ss = 4096;   // per-CTA partial sums of h'^2
+  size_t o = 4096 + (size_t)kMaxSMs * 4;
   w.part = o;
   o = align_up(o + (size_t)T * (E + 1) * kRouterSplit * 4, 256);
   w.logits = o;
@@ -608,6 +608,15 @@ static FusedConfig fused_config(const fmoe_layer_desc& d) {
   return fc;
 }
 
+// The fused kernel instantiation for a pair of code widths.
+static const void* fused_kernel_for(int bits, int sbits) {
+  if (bits == 4 && sbits == 4) return reinterpret_cast<const void*>(&fused_stack_kernel<4, 4>);
+  if (bits == 2 && sbits == 4) return reinterpret_cast<const void*>(&fused_stack_kernel<2, 4>);
+  if (bits == 2 && sbits == 2) return reinterpret_cast<const void*>(&fused_stack_kernel<2, 2>);
+  if (bits == 4 && sbits == 2) return reinterpret_cast<const void*>(&fused_stack_kernel<4, 2>);
+  return nullptr;
+}
+
 static FusedConfig fused_config_uncached(const fmoe_layer_desc& d, int dev) {
   FusedConfig fc{};
   int n_sm = 0, optin = 0;
@@ -617,12 +626,12 @@ static FusedConfig fused_config_uncached(const fmoe_layer_desc& d, int dev) {
   const size_t max_dyn = optin > 2048 ? (size_t)optin - 1024 : 0;
   if (!fused_plan(d.hidden, d.inter, d.n_experts, d.top_k, d.bits, d.shared_bits, n_sm, max_dyn, &fc.plan))
     return fc;
-  if (cudaFuncSetAttribute(fused_stack_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                           (int)fc.plan.total) != cudaSuccess)
+  const void* kfn = fused_kernel_for(d.bits, d.shared_bits);
+  if (!kfn) return fc;
+  if (cudaFuncSetAttribute(kfn, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)fc.plan.total) != cudaSuccess)
     return fc;
   int per_sm = 0;
-  if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, fused_stack_kernel, kFusedThreads,
-                                                    fc.plan.total) != cudaSuccess ||
+  if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kfn, kFusedThreads, fc.plan.total) != cudaSuccess ||
       per_sm < 1)
     return fc;
   fc.n_sm = n_sm;
@@ -686,7 +695,8 @@ static int launch_fused(const fmoe_layer_weights* layers, int n_layers, float* h
     attr[0].val.cooperative = 1;
     cfg.attrs = attr;
     cfg.numAttrs = 1;
-    const cudaError_t e = cudaLaunchKernelEx(&cfg, fused_stack_kernel, args);
+    void* kargs[] = {&args};
+    const cudaError_t e = cudaLaunchKernelExC(&cfg, fused_kernel_for(d.bits, d.shared_bits), kargs);
     if (e != cudaSuccess) return FMOE_ERR_CUDA;
   }
   return FMOE_OK;
