@@ -95,7 +95,7 @@ __device__ __forceinline__ GroupCodes<BITS> load_group(const uint8_t* row, int n
 template <int BITS>
 __device__ __forceinline__ int group_dot(const GroupCodes<BITS>& gc, const uint4* xv) {
   if (BITS == 4) {
-    int lo = 0, hi = 0;
+    int lo[2] = {0, 0}, hi[2] = {0, 0};  // two accumulators each: shorter dependency chains
 #pragma unroll
     for (int h = 0; h < 2; ++h) {
       const uint32_t w[4] = {gc.c[h].x, gc.c[h].y, gc.c[h].z, gc.c[h].w};
@@ -103,13 +103,13 @@ __device__ __forceinline__ int group_dot(const GroupCodes<BITS>& gc, const uint4
       for (int i = 0; i < 4; ++i) {
         const uint4 x = xv[4 * h + i];
         const uint32_t l = w[i] & 0x0F0F0F0Fu, u = w[i] & 0xF0F0F0F0u;
-        lo = dp2a_lo(x.x, l, lo);
-        lo = dp2a_hi(x.y, l, lo);
-        hi = dp2a_lo(x.z, u, hi);
-        hi = dp2a_hi(x.w, u, hi);
+        lo[i & 1] = dp2a_lo(x.x, l, lo[i & 1]);
+        lo[i & 1] = dp2a_hi(x.y, l, lo[i & 1]);
+        hi[i & 1] = dp2a_lo(x.z, u, hi[i & 1]);
+        hi[i & 1] = dp2a_hi(x.w, u, hi[i & 1]);
       }
     }
-    return 16 * lo + hi;
+    return 16 * (lo[0] + lo[1]) + (hi[0] + hi[1]);
   } else {
     int a0 = 0, a1 = 0, a2 = 0, a3 = 0;
     const uint32_t w[4] = {gc.c[0].x, gc.c[0].y, gc.c[0].z, gc.c[0].w};

@@ -31,6 +31,8 @@
 
 #include <cstdint>
 
+#include <cuda.h>  // CUtensorMap
+
 #include "fmoe.h"
 #include "fmoe_device.cuh"
 #include "fmoe_layout.h"
@@ -56,6 +58,12 @@ constexpr int kSyncGroups = 2;        // first per-group publication counter in 
 constexpr int kMaxGroupCounters = 1022;
 constexpr int kWStage = 144;          // per-warp staged a-group: 8 uint4 + delta + xsum (+pad)
 constexpr int kMaxSliceRows = 64;     // hidden rows per CTA in the down products (2 per lane)
+// Down rows reach shared memory through 3-D tensor copies whose box is
+// kRowPadWords wider than a row: the tensor engine zero-fills the excess, so
+// consecutive rows land 16 bytes off the 128-byte bank period and lanes
+// reading one row each do not collide on banks.
+constexpr int kRowPadWords = 4;
+enum { kTmRoutedCodes = 0, kTmRoutedSb = 1, kTmSharedCodes = 2, kTmSharedSb = 3, kTmPerLayer = 4 };
 
 struct FusedLayer {
   const uint8_t* experts;
@@ -84,10 +92,16 @@ struct FusedPlan {
                    // sums fp32 [warps][2][kMaxSliceRows]
   uint32_t prod;   // u32 [k * I / 64]: CTAs producing each routed a-group (static)
   uint32_t mbar;
+  uint32_t nd_box;     // rows of every down-row tensor copy (the largest hidden slice)
+  uint32_t sd_codes, sd_sb;         // offsets of the shared expert's padded down rows
+  uint32_t rd_slot;                 // offset of the first routed expert's padded down rows
+  uint32_t rd_stride;               // bytes per routed expert (codes then scale-bias)
+  uint32_t rd_sb;                   // offset of the scale-bias rows inside a routed slot
   uint32_t total;
 };
 
-struct FusedArgs {
+struct alignas(64) FusedArgs {
+  CUtensorMap tm[kFusedMaxLayers][kTmPerLayer];  // down rows (codes, scale-bias) of the routed / shared records
   FusedLayer layers[kFusedMaxLayers];
   int n_layers;
   int H, I, E, k, bits, sbits;
@@ -129,6 +143,16 @@ __device__ __forceinline__ void bulk_g2s(void* dst, const void* src, uint32_t by
 
 // One try_wait; the thread may be suspended (up to the hint, 20 us) until the
 // phase completes, so waiting warps do not compete for issue slots.
+// 3-D tensor copy global -> shared (box of `map` at coordinates c0, c1, c2).
+__device__ __forceinline__ void tma_load_3d(void* dst, const CUtensorMap* map, int c0, int c1, int c2,
+                                            uint64_t* bar) {
+  asm volatile(
+      "cp.async.bulk.tensor.3d.shared::cluster.global.tile.mbarrier::complete_tx::bytes [%0], [%1, {%2, %3, %4}], "
+      "[%5];" ::"r"(smem_u32(dst)),
+      "l"(map), "r"(c0), "r"(c1), "r"(c2), "r"(smem_u32(bar))
+      : "memory");
+}
+
 __device__ __forceinline__ bool mbar_try(uint64_t* bar, uint32_t parity) {
   uint32_t done;
   asm volatile(
@@ -306,11 +330,18 @@ __global__ void __launch_bounds__(kFusedThreads, 1) fused_stack_kernel(const __g
   uint8_t* sc_sb = sc_codes + (size_t)nsp * pc_s;
   uint8_t* rc_codes = regA;
   uint8_t* rc_sb = regA + (size_t)nq * pc_r;
-  // region B: shared down [codes nd*drow_s][sb nd*ngI*4], then routed down per expert
-  uint8_t* sd_codes = regB;
-  uint32_t* sd_sb = reinterpret_cast<uint32_t*>(regB + (size_t)nd * drow_s);
-  uint8_t* rd_base = regB + (size_t)nd * (drow_s + ngI * 4);
-  const size_t rd_stride = (size_t)nd * (drow_r + ngI * 4);
+  // region B: the shared expert's padded down rows, then the routed experts'
+  // (each: codes rows of drow + 16 bytes, then scale-bias rows of (I/64 + 4) words)
+  (void)regB;
+  uint8_t* sd_codes = smem + P.sd_codes;
+  const uint32_t* sd_sb = reinterpret_cast<const uint32_t*>(smem + P.sd_sb);
+  uint8_t* rd_base = smem + P.rd_slot;
+  const size_t rd_stride = P.rd_stride;
+  const uint32_t rd_sb_off = P.rd_sb;
+  const uint32_t prow_r = drow_r + 4 * kRowPadWords, prow_s = drow_s + 4 * kRowPadWords;  // padded code rows
+  const uint32_t psbrow = (uint32_t)(ngI + kRowPadWords);                                  // padded sb row, words
+  const uint32_t box_r = P.nd_box * prow_r + P.nd_box * psbrow * 4;  // bytes of one routed expert's copies
+  const uint32_t box_s = P.nd_box * prow_s + P.nd_box * psbrow * 4;
   uint8_t* cons = smem + P.cons;
   float* cons_wy = reinterpret_cast<float*>(cons + kFusedWarps * kWStage);
   // number of CTAs whose pair share touches a-group gg and publish it once per
@@ -417,12 +448,11 @@ __global__ void __launch_bounds__(kFusedThreads, 1) fused_stack_kernel(const __g
   };
   // the shared expert's down rows of layer l (region B, shared part)
   auto issue_sdown = [&](int l) {
-    const FusedLayer& LY = A.layers[l];
     if (nd > 0 && lane == 0 && warp == kFusedWarps - 1) {
       fence_proxy_async();
-      arm(kMbSDown, (uint32_t)nd * (drow_s + ngI * 4), (uint32_t)(l & 1));
-      bulk_g2s(sd_codes, LY.shared + LS.down_codes + (size_t)i0 * drow_s, (uint32_t)nd * drow_s, &mbar[kMbSDown]);
-      bulk_g2s(sd_sb, LY.shared + LS.down_sb + (size_t)i0 * ngI * 4, (uint32_t)nd * ngI * 4, &mbar[kMbSDown]);
+      arm(kMbSDown, box_s, (uint32_t)(l & 1));
+      tma_load_3d(sd_codes, &A.tm[l][kTmSharedCodes], 0, i0, 0, &mbar[kMbSDown]);
+      tma_load_3d(const_cast<uint32_t*>(sd_sb), &A.tm[l][kTmSharedSb], 0, i0, 0, &mbar[kMbSDown]);
     }
   };
   // the routed experts' gate/up pairs of this CTA's share and down rows of its slice
@@ -447,12 +477,10 @@ __global__ void __launch_bounds__(kFusedThreads, 1) fused_stack_kernel(const __g
     }
     if (nd > 0) {
       for (int j = (warp + kFusedWarps - nch % kFusedWarps) % kFusedWarps; j < k; j += kFusedWarps) {
-        const uint8_t* rec = LY.experts + (size_t)s_ids[j] * LR.bytes;
         uint8_t* dst = rd_base + (size_t)j * rd_stride;
-        arm(kMbRDown + j, (uint32_t)nd * (drow_r + ngI * 4), par);
-        bulk_g2s(dst, rec + LR.down_codes + (size_t)i0 * drow_r, (uint32_t)nd * drow_r, &mbar[kMbRDown + j]);
-        bulk_g2s(dst + (size_t)nd * drow_r, rec + LR.down_sb + (size_t)i0 * ngI * 4, (uint32_t)nd * ngI * 4,
-                 &mbar[kMbRDown + j]);
+        arm(kMbRDown + j, box_r, par);
+        tma_load_3d(dst, &A.tm[l][kTmRoutedCodes], 0, i0, s_ids[j], &mbar[kMbRDown + j]);
+        tma_load_3d(dst + rd_sb_off, &A.tm[l][kTmRoutedSb], 0, i0, s_ids[j], &mbar[kMbRDown + j]);
       }
     }
   };
@@ -697,17 +725,15 @@ __global__ void __launch_bounds__(kFusedThreads, 1) fused_stack_kernel(const __g
             if (!__all_sync(0xffffffffu, ok)) { ok = false; break; }
             j_cur = j;
           }
-          float m = fmaxf(fabsf(av[t].x), fabsf(av[t].y));
-#pragma unroll
-          for (int o = 16; o > 0; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
+          // group max of |a| in one redux (the bits of a non-negative float order as integers)
+          const float m = __uint_as_float(
+              __reduce_max_sync(0xffffffffu, __float_as_uint(fmaxf(fabsf(av[t].x), fabsf(av[t].y)))));
           const float inv = m > 0.f ? 32767.f / m : 0.f;
           const float delta = m * (1.f / 32767.f);
           int qa = __float2int_rn(av[t].x * inv), qb = __float2int_rn(av[t].y * inv);
           qa = qa > 32767 ? 32767 : (qa < -32767 ? -32767 : qa);
           qb = qb > 32767 ? 32767 : (qb < -32767 ? -32767 : qb);
-          int isum = qa + qb;
-#pragma unroll
-          for (int o = 16; o > 0; o >>= 1) isum += __shfl_xor_sync(0xffffffffu, isum, o);
+          const int isum = __reduce_add_sync(0xffffffffu, qa + qb);
           __syncwarp();  // the previous group's staged values have been read
           reinterpret_cast<uint32_t*>(wst)[lane] = (uint32_t)(qa & 0xFFFF) | ((uint32_t)qb << 16);
           if (lane == 0) {
@@ -721,8 +747,8 @@ __global__ void __launch_bounds__(kFusedThreads, 1) fused_stack_kernel(const __g
           const float dl = wdx[0], xsm = wdx[1];
           const bool shd = j == k;
           const uint8_t* base = shd ? sd_codes : rd_base + (size_t)j * rd_stride;
-          const uint32_t drow = shd ? drow_s : drow_r;
-          const uint32_t* sbb = reinterpret_cast<const uint32_t*>(base + (size_t)nd * drow);
+          const uint32_t drow = shd ? prow_s : prow_r;
+          const uint32_t* sbb = shd ? sd_sb : reinterpret_cast<const uint32_t*>(base + rd_sb_off);
 #pragma unroll 1
           for (int half = 0; half < 2; ++half) {
             const int rr = lane + 32 * half;
@@ -730,7 +756,7 @@ __global__ void __launch_bounds__(kFusedThreads, 1) fused_stack_kernel(const __g
             const uint8_t* cp = base + (size_t)rr * drow;
             const int A32 = shd ? group_dot<SBITS>(lds_group<SBITS>(cp, ngI, g), xv)
                                 : group_dot<BITS>(lds_group<BITS>(cp, ngI, g), xv);
-            const float y = group_epilogue(half ? acc1 : acc0, sbb[rr * ngI + g], A32, dl, xsm);
+            const float y = group_epilogue(half ? acc1 : acc0, sbb[rr * psbrow + g], A32, dl, xsm);
             if (half) acc1 = y;
             else acc0 = y;
           }
@@ -835,8 +861,14 @@ inline bool fused_plan(int H, int I, int E, int k, int bits, int sbits, int n_ct
   const long long cons_off = (a_p1 + 127) & ~127LL;
   const long long cons_bytes = (long long)kFusedWarps * kWStage + (long long)kFusedWarps * 2 * kMaxSliceRows * 4;
   const long long regA = a_p2 > cons_off + cons_bytes ? a_p2 : cons_off + cons_bytes;
-  const long long sdown = nd * ((long long)LS.down_row_bytes + ngI * 4);
-  const long long rdown = k * nd * ((long long)LR.down_row_bytes + ngI * 4);
+  // padded down-row boxes (tensor copies of nd rows, each kRowPadWords wider than a row)
+  const long long dw_r = (long long)LR.down_row_bytes / 4, dw_s = (long long)LS.down_row_bytes / 4;
+  if (dw_r + kRowPadWords > 256 || dw_s + kRowPadWords > 256 || ngI + kRowPadWords > 256 || nd > 256) return false;
+  const long long c_r = al(nd * (dw_r + kRowPadWords) * 4), c_s = al(nd * (dw_s + kRowPadWords) * 4);
+  const long long sbb = al(nd * (ngI + kRowPadWords) * 4);
+  const long long sdown = c_s + sbb;
+  const long long rstride = c_r + sbb;
+  const long long rdown = k * rstride;
   const long long xq = (long long)staged_x_bytes(H);
   FusedPlan p;
   long long o = 0;
@@ -844,6 +876,12 @@ inline bool fused_plan(int H, int I, int E, int k, int bits, int sbits, int n_ct
   p.cons = (uint32_t)(o + cons_off);
   o = al(o + regA);
   p.region_b = (uint32_t)o;
+  p.nd_box = (uint32_t)nd;
+  p.sd_codes = (uint32_t)o;
+  p.sd_sb = (uint32_t)(o + c_s);
+  p.rd_slot = (uint32_t)(o + sdown);
+  p.rd_stride = (uint32_t)rstride;
+  p.rd_sb = (uint32_t)c_r;
   const long long xf_bytes = (long long)H * 4;
   if (rdown >= xf_bytes) {
     p.xf = (uint32_t)(o + sdown);  // aliases the routed down rows (P1 only)

@@ -18,6 +18,8 @@
 #include <cstdint>
 #include <cstring>
 
+#include <cuda.h>
+#include <cudaTypedefs.h>
 #include <cuda_runtime.h>
 
 #include "fmoe.h"
@@ -644,6 +646,58 @@ static bool same_desc(const fmoe_layer_desc& a, const fmoe_layer_desc& b) {
          a.bits == b.bits && a.shared_bits == b.shared_bits && a.group == b.group && a.eps == b.eps;
 }
 
+// cuTensorMapEncodeTiled, fetched once through the runtime (no link-time
+// dependency on the driver library).
+static PFN_cuTensorMapEncodeTiled_v12000 tensor_map_encoder() {
+  static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
+  static bool tried = false;
+  if (!tried) {
+    tried = true;
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(p);
+  }
+  return fn;
+}
+
+// Tensor map over [n_mats][rows][words] 32-bit words (row stride row_bytes,
+// matrix stride mat_bytes) whose box is box_words x box_rows x 1: a box wider
+// than a row is zero-filled past the row end.
+static bool encode_rows(CUtensorMap* m, const void* base, uint64_t words, uint64_t rows, uint64_t row_bytes,
+                        uint64_t n_mats, uint64_t mat_bytes, uint32_t box_words, uint32_t box_rows) {
+  PFN_cuTensorMapEncodeTiled_v12000 enc = tensor_map_encoder();
+  if (!enc) return false;
+  const cuuint64_t dims[3] = {words, rows, n_mats};
+  const cuuint64_t strides[2] = {row_bytes, mat_bytes};
+  const cuuint32_t box[3] = {box_words, box_rows, 1};
+  const cuuint32_t es[3] = {1, 1, 1};
+  return enc(m, CU_TENSOR_MAP_DATA_TYPE_UINT32, 3, const_cast<void*>(base), dims, strides, box, es,
+             CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_NONE,
+             CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+// The four down-row tensor maps of one layer (routed codes / scale-bias,
+// shared codes / scale-bias).
+static bool encode_layer_maps(const fmoe_layer_weights& L, const FusedPlan& plan, CUtensorMap* tm) {
+  const fmoe_layer_desc& d = L.desc;
+  const RecordLayout LR = record_layout(d.bits, d.hidden, d.inter);
+  const RecordLayout LS = record_layout(d.shared_bits, d.hidden, d.inter);
+  const uint32_t ngI = (uint32_t)d.inter / 64, rows = plan.nd_box;
+  const uint8_t* ex = static_cast<const uint8_t*>(L.experts);
+  const uint8_t* sh = static_cast<const uint8_t*>(L.shared);
+  return encode_rows(&tm[kTmRoutedCodes], ex + LR.down_codes, LR.down_row_bytes / 4, (uint64_t)d.hidden,
+                     LR.down_row_bytes, (uint64_t)d.n_experts, LR.bytes,
+                     (uint32_t)(LR.down_row_bytes / 4 + kRowPadWords), rows) &&
+         encode_rows(&tm[kTmRoutedSb], ex + LR.down_sb, ngI, (uint64_t)d.hidden, (uint64_t)ngI * 4,
+                     (uint64_t)d.n_experts, LR.bytes, ngI + kRowPadWords, rows) &&
+         encode_rows(&tm[kTmSharedCodes], sh + LS.down_codes, LS.down_row_bytes / 4, (uint64_t)d.hidden,
+                     LS.down_row_bytes, 1, LS.bytes, (uint32_t)(LS.down_row_bytes / 4 + kRowPadWords), rows) &&
+         encode_rows(&tm[kTmSharedSb], sh + LS.down_sb, ngI, (uint64_t)d.hidden, (uint64_t)ngI * 4, 1, LS.bytes,
+                     ngI + kRowPadWords, rows);
+}
+
 // Runs n_layers layers (T = 1) with the persistent kernel.  Returns
 // FMOE_ERR_UNSUPPORTED when the configuration does not fit it.
 static int launch_fused(const fmoe_layer_weights* layers, int n_layers, float* h, float* xn, void* ws,
@@ -654,7 +708,7 @@ static int launch_fused(const fmoe_layer_weights* layers, int n_layers, float* h
   const WsLayout w = ws_layout(d.hidden, d.inter, d.n_experts, d.top_k, 1);
   if (ws_bytes < w.bytes) return FMOE_ERR_BUFFER_TOO_SMALL;
   unsigned char* base = static_cast<unsigned char*>(ws);
-  FusedArgs args;
+  thread_local FusedArgs args;  // 16 KB of tensor maps: not on the stack
   std::memset(&args, 0, sizeof(args));
   args.H = d.hidden;
   args.I = d.inter;
@@ -684,6 +738,7 @@ static int launch_fused(const fmoe_layer_weights* layers, int n_layers, float* h
       args.layers[l].w_router = L.w_router;
       args.layers[l].w_sg = L.w_shared_gate;
       args.layers[l].norm_w = L.norm_w;
+      if (!encode_layer_maps(L, fc.plan, args.tm[l])) return FMOE_ERR_UNSUPPORTED;
     }
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = dim3(fc.n_sm);
