@@ -232,6 +232,38 @@ int fmoe_stack_forward(const fmoe_layer_weights* layers, int n_layers, float* d_
  * setting, returns the previous value. */
 int fmoe_set_fused(int enable);
 
+/* ------------------------------------------- without caller workspace -- */
+/* fmoe_layer_forward for callers that cannot hand over a workspace.  The
+ * Flash-MoE pages have no counterpart to this call: it exists for hosts that
+ * must not reserve device memory on the path -- an engine whose device pool
+ * already owns all free memory, a latency-critical loop in which an
+ * allocation (with the device-wide synchronisation cudaMalloc/cudaFree can
+ * imply) is not acceptable, or a plain C program with no tensor library to
+ * manage a workspace.  It computes exactly what fmoe_layer_forward computes,
+ * through the same kernels, and allocates nothing: its workspace is an 8 MiB
+ * array in the library's device memory, one per device, set aside when the
+ * library's module is loaded on that device.
+ *   lw, d_h, d_xn, T, stream  as for fmoe_layer_forward.
+ * Limit: fmoe_workspace_bytes(&lw->desc, T) must not exceed 8 MiB (8388608
+ * bytes), which admits up to T = 74 tokens at hidden 4096 / inter 1024 /
+ * 512 experts / top-4; a larger request returns FMOE_ERR_BUFFER_TOO_SMALL
+ * before anything is launched.
+ * First call on each device: it looks up the array's device address and
+ * enqueues, on `stream`, a zeroing of the counter words at the array's start
+ * (the grid-barrier and publication counters of the persistent kernel); every
+ * completed call leaves them at zero again.  Make this first call on each
+ * device before any stream capture begins.
+ * One array per device: calls that can overlap on the device (different
+ * streams, or different host threads, without ordering between them) race on
+ * it and corrupt each other's results; order them, e.g. on one stream.  The
+ * intermediates are not exposed.  If the device status reports
+ * FMOE_STATUS_WAIT_TIMEOUT, the counters may be left non-zero and this entry
+ * point must not be used again on that device in this process.
+ * Errors: as fmoe_layer_forward, plus FMOE_ERR_BUFFER_TOO_SMALL above the
+ * limit and FMOE_ERR_UNSUPPORTED for a device ordinal of 64 or more. */
+int fmoe_layer_forward_noalloc(const fmoe_layer_weights* lw, float* d_h, float* d_xn, int T,
+                               cudaStream_t stream);
+
 #ifdef __cplusplus
 }
 #endif

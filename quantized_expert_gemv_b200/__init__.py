@@ -88,6 +88,7 @@ _SIGS = {
     "fmoe_layer_forward_logits": (_i32, [_PW, _vp, _vp, _vp, _i32, _vp, _sz, _vp]),
     "fmoe_stack_forward": (_i32, [_PW, _i32, _vp, _vp, _i32, _vp, _sz, _vp]),
     "fmoe_set_fused": (_i32, [_i32]),
+    "fmoe_layer_forward_noalloc": (_i32, [_PW, _vp, _vp, _i32, _vp]),
 }
 for _name, (_res, _args) in _SIGS.items():
     _fn = getattr(_lib, _name)
@@ -296,6 +297,14 @@ def fmoe_stack_forward(layers, h, xn, ws, stream=None) -> None:
     rc = _lib.fmoe_stack_forward(arr, len(layers), _ptr(h), _ptr(xn), h.shape[0], _ptr(ws),
                                  ws.numel() * ws.element_size(), _stream(stream))
     _check(rc, "fmoe_stack_forward")
+
+
+def fmoe_layer_forward_noalloc(lw: LayerWeights, h, xn, stream=None) -> None:
+    """fmoe_layer_forward with the library's fixed per-device scratch instead of a
+    caller workspace (nothing is allocated; calls on one device must not overlap)."""
+    c = lw.c()
+    rc = _lib.fmoe_layer_forward_noalloc(ctypes.byref(c), _ptr(h), _ptr(xn), h.shape[0], _stream(stream))
+    _check(rc, "fmoe_layer_forward_noalloc")
 
 
 def fmoe_set_fused(enable: bool) -> bool:

@@ -17,6 +17,7 @@
 // residual + sigmoid gating, two-pass RMSNorm feeding the next layer).
 #include <cstdint>
 #include <cstring>
+#include <mutex>
 
 #include <cuda.h>
 #include <cudaTypedefs.h>
@@ -955,4 +956,50 @@ extern "C" int fmoe_stack_forward(const fmoe_layer_weights* layers, int n_layers
     if (rc != FMOE_OK) return rc;
   }
   return FMOE_OK;
+}
+
+// --------------------------------------------- fixed device scratch ----
+// Workspace of fmoe_layer_forward_noalloc: one array per device, set aside
+// when the module loads, so that the call itself reserves no memory.
+namespace fmoe {
+
+constexpr size_t kStaticScratchBytes = size_t(8) << 20;  // 8 MiB: T <= 74 at 4096 x 1024 x 512 experts, top-4
+constexpr size_t kStaticCounterBytes = 4096;             // the counter words at the start of the layout
+constexpr int kStaticMaxDevices = 64;
+
+static __device__ __align__(256) unsigned char g_static_scratch[kStaticScratchBytes];
+
+static std::mutex g_static_scratch_mu;
+static void* g_static_scratch_ptr[kStaticMaxDevices];
+
+// Address of the current device's scratch.  The first call on a device looks
+// the symbol up and zeroes its counter words on `st`; later calls only read
+// the cached address.
+static int static_scratch(cudaStream_t st, void** out) {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return FMOE_ERR_CUDA;
+  if (dev < 0 || dev >= kStaticMaxDevices) return FMOE_ERR_UNSUPPORTED;
+  std::lock_guard<std::mutex> lock(g_static_scratch_mu);
+  if (!g_static_scratch_ptr[dev]) {
+    void* p = nullptr;
+    if (cudaGetSymbolAddress(&p, g_static_scratch) != cudaSuccess || !p) return FMOE_ERR_CUDA;
+    if (cudaMemsetAsync(p, 0, kStaticCounterBytes, st) != cudaSuccess) return FMOE_ERR_CUDA;
+    g_static_scratch_ptr[dev] = p;
+  }
+  *out = g_static_scratch_ptr[dev];
+  return FMOE_OK;
+}
+
+}  // namespace fmoe
+
+extern "C" int fmoe_layer_forward_noalloc(const fmoe_layer_weights* lw, float* d_h, float* d_xn, int T,
+                                          cudaStream_t stream) {
+  if (!lw || !desc_valid(&lw->desc) || T < 1) return FMOE_ERR_INVALID_ARG;
+  const fmoe_layer_desc& d = lw->desc;
+  if (ws_layout(d.hidden, d.inter, d.n_experts, d.top_k, T).bytes > kStaticScratchBytes)
+    return FMOE_ERR_BUFFER_TOO_SMALL;
+  void* ws = nullptr;
+  const int rc = static_scratch(stream, &ws);
+  if (rc != FMOE_OK) return rc;
+  return layer_forward_impl(lw, nullptr, d_h, d_xn, T, ws, kStaticScratchBytes, stream);
 }
