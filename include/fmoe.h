@@ -102,17 +102,23 @@ typedef struct fmoe_layer_weights {
  *
  * Packed record (one per expert; all sections 16-byte aligned):
  *   [gate/up codes][down codes][gate/up scale-bias][down scale-bias]
- *   gate/up: I row pairs, gate row n then up row n; down: H rows.
- *   A row of K inputs is split into segments of min(32, K/64) groups; within
- *   a segment 4-bit codes store first the low halves (inputs 0..31) of all its
- *   groups, 16 bytes each, then the high halves; 2-bit codes store each
- *   group's 16 bytes in order.  Inside each 32-bit word the 8 (or 16) codes of
- *   8 (16) consecutive inputs are permuted so that masking the word with
- *   0x0F0F0F0F / 0xF0F0F0F0 (4-bit) or 0x03030303 .. 0xC0C0C0C0 (2-bit) yields
- *   byte lanes that pair with consecutive inputs (field 2a+b, resp. 4a+b, of
- *   the word holds input 4b+a).  Scale-bias: one 32-bit word per group,
- *   bf16 scale * 2^-4 (4-bit) or * 2^-6 (2-bit) in the low half, bf16 bias in
- *   the high half, row-major.
+ *   gate/up: I row pairs, gate row n then up row n, row by row.  A row of K
+ *   inputs is split into segments of min(32, K/64) groups; within a segment
+ *   4-bit codes store first the low halves (inputs 0..31) of all its groups,
+ *   16 bytes each, then the high halves; 2-bit codes store each group's 16
+ *   bytes in order.
+ *   down: column blocks of w = 8 (4-bit) or 16 (2-bit) consecutive inputs;
+ *   block nb holds, for hidden rows 0 .. H-1 in order, one 32-bit word with
+ *   the codes of inputs nb*w .. nb*w + w - 1 of that row (word (nb, r) at
+ *   byte 4 * (nb * H + r) of the section).
+ *   Inside every 32-bit word the 8 (or 16) codes of 8 (16) consecutive
+ *   inputs are permuted so that masking the word with 0x0F0F0F0F /
+ *   0xF0F0F0F0 (4-bit) or 0x03030303 .. 0xC0C0C0C0 (2-bit) yields byte lanes
+ *   that pair with consecutive inputs (field 2a+b, resp. 4a+b, of the word
+ *   holds input 4b+a).  Scale-bias: one 32-bit word per group, bf16
+ *   scale * 2^-4 (4-bit) or * 2^-6 (2-bit) in the low half, bf16 bias in the
+ *   high half; gate/up row-major (row pr, group g at pr * H/64 + g), down
+ *   group-major (group g, row r at g * H + r).
  * Size per expert: 3 H I bits / 8 + 3 H I / 64 * 4 bytes (7,077,888 bytes =
  * 6.75 MiB at H = 4096, I = 1024, 4-bit; 3,932,160 bytes at 2-bit). */
 
@@ -142,7 +148,8 @@ int fmoe_pack_experts(const uint8_t* q, const uint16_t* scale, const uint16_t* b
  * (d_q, d_scale, d_bias, same layout as the host arrays; 16-byte aligned).
  * Packs on `stream` without synchronising and without a host round trip.
  * Invalid codes or scales are reported through FMOE_STATUS_BAD_PACK_INPUT in
- * the device status word (the affected words are written as zero).
+ * the device status word (the 16-byte code chunks or scale-bias words that
+ * hold them are written as zero).
  * Errors: FMOE_ERR_INVALID_ARG, FMOE_ERR_UNSUPPORTED, FMOE_ERR_BUFFER_TOO_SMALL,
  * FMOE_ERR_CUDA. */
 int fmoe_pack_experts_device(const uint8_t* d_q, const uint16_t* d_scale, const uint16_t* d_bias,
@@ -232,6 +239,12 @@ int fmoe_stack_forward(const fmoe_layer_weights* layers, int n_layers, float* d_
  * setting, returns the previous value. */
 int fmoe_set_fused(int enable);
 
+/* 1 if the persistent kernel runs layers of descriptor d at T = 1 on the
+ * current device (shape and shared-memory plan fit), else 0 (also on any
+ * error).  The persistent kernel leaves the gate/up outputs a in the
+ * workspace but not the per-expert down outputs y: it sums them on the fly. */
+int fmoe_fused_supported(const fmoe_layer_desc* d);
+
 /* ------------------------------------------- without caller workspace -- */
 /* fmoe_layer_forward for callers that cannot hand over a workspace.  The
  * Flash-MoE pages have no counterpart to this call: it exists for hosts that
@@ -240,14 +253,14 @@ int fmoe_set_fused(int enable);
  * allocation (with the device-wide synchronisation cudaMalloc/cudaFree can
  * imply) is not acceptable, or a plain C program with no tensor library to
  * manage a workspace.  It computes exactly what fmoe_layer_forward computes,
- * through the same kernels, and allocates nothing: its workspace is an 8 MiB
+ * through the same kernels, and allocates nothing: its workspace is a 12 MiB
  * array in the library's device memory, one per device, set aside when the
  * library's module is loaded on that device.
  *   lw, d_h, d_xn, T, stream  as for fmoe_layer_forward.
- * Limit: fmoe_workspace_bytes(&lw->desc, T) must not exceed 8 MiB (8388608
- * bytes), which admits up to T = 74 tokens at hidden 4096 / inter 1024 /
- * 512 experts / top-4; a larger request returns FMOE_ERR_BUFFER_TOO_SMALL
- * before anything is launched.
+ * Limit: fmoe_workspace_bytes(&lw->desc, T) must not exceed 12 MiB
+ * (12582912 bytes), which admits up to T = 88 tokens at hidden 4096 /
+ * inter 1024 / 512 experts / top-4; a larger request returns
+ * FMOE_ERR_BUFFER_TOO_SMALL before anything is launched.
  * First call on each device: it looks up the array's device address and
  * enqueues, on `stream`, a zeroing of the counter words at the array's start
  * (the grid-barrier and publication counters of the persistent kernel); every

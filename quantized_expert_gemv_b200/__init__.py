@@ -88,6 +88,7 @@ _SIGS = {
     "fmoe_layer_forward_logits": (_i32, [_PW, _vp, _vp, _vp, _i32, _vp, _sz, _vp]),
     "fmoe_stack_forward": (_i32, [_PW, _i32, _vp, _vp, _i32, _vp, _sz, _vp]),
     "fmoe_set_fused": (_i32, [_i32]),
+    "fmoe_fused_supported": (_i32, [_PDESC]),
     "fmoe_layer_forward_noalloc": (_i32, [_PW, _vp, _vp, _i32, _vp]),
 }
 for _name, (_res, _args) in _SIGS.items():
@@ -305,6 +306,12 @@ def fmoe_layer_forward_noalloc(lw: LayerWeights, h, xn, stream=None) -> None:
     c = lw.c()
     rc = _lib.fmoe_layer_forward_noalloc(ctypes.byref(c), _ptr(h), _ptr(xn), h.shape[0], _stream(stream))
     _check(rc, "fmoe_layer_forward_noalloc")
+
+
+def fmoe_fused_supported(desc: LayerDesc) -> bool:
+    """True if the persistent kernel runs layers of this shape at T = 1 on the current device."""
+    c = desc.c() if hasattr(desc, "c") else desc
+    return bool(_lib.fmoe_fused_supported(ctypes.byref(c)))
 
 
 def fmoe_set_fused(enable: bool) -> bool:

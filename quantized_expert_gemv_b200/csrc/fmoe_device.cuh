@@ -131,6 +131,27 @@ __device__ __forceinline__ int group_dot(const GroupCodes<BITS>& gc, const uint4
   }
 }
 
+// Integer dot product of one 32-bit word of 4-bit codes (8 inputs) with its
+// 8 staged inputs x (int16 pairs).  Returns 16 * sum q x, like group_dot.
+__device__ __forceinline__ int word_dot4(uint32_t w, uint4 x) {
+  const uint32_t l = w & 0x0F0F0F0Fu, u = w & 0xF0F0F0F0u;
+  const int lo = dp2a_hi(x.y, l, dp2a_lo(x.x, l, 0));
+  const int hi = dp2a_hi(x.w, u, dp2a_lo(x.z, u, 0));
+  return 16 * lo + hi;
+}
+
+// One word of 2-bit codes (16 inputs) with its staged inputs x0 (inputs
+// 0..7) and x1 (8..15).  Returns 64 * sum q x.
+__device__ __forceinline__ int word_dot2(uint32_t w, uint4 x0, uint4 x1) {
+  const uint32_t m0 = w & 0x03030303u, m1 = w & 0x0C0C0C0Cu;
+  const uint32_t m2 = w & 0x30303030u, m3 = w & 0xC0C0C0C0u;
+  const int a0 = dp2a_hi(x0.y, m0, dp2a_lo(x0.x, m0, 0));
+  const int a1 = dp2a_hi(x0.w, m1, dp2a_lo(x0.z, m1, 0));
+  const int a2 = dp2a_hi(x1.y, m2, dp2a_lo(x1.x, m2, 0));
+  const int a3 = dp2a_hi(x1.w, m3, dp2a_lo(x1.z, m3, 0));
+  return 64 * a0 + 16 * a1 + 4 * a2 + a3;
+}
+
 // fp32 epilogue of one group: y + (s * delta) * A + b * xsum, with the packed
 // scale-bias word (bf16 scale in the low half, bf16 bias in the high half).
 __device__ __forceinline__ float group_epilogue(float y, uint32_t sb, int A, float delta, float xsum) {

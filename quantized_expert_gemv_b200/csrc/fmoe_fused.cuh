@@ -1,37 +1,43 @@
 // fmoe_fused.cuh -- one persistent kernel for a stack of MoE layers, batch 1.
 //
 // One CTA per SM, launched cooperatively so that every CTA is resident and
-// grid-wide barriers are safe.  Each layer runs in three phases separated by
-// grid barriers -- the three global dependencies of the layer:
-//   P1  router rows and the shared expert's gate/up rows (neither depends on
-//       routing) -> logits, gamma, the shared expert's SwiGLU outputs
-//   --  barrier: all logits written
-//   P2  every CTA takes the top-k of the logits itself, then streams its
-//       share of the routed experts' gate/up rows -> SwiGLU outputs a, while
-//       the routed experts' down rows it will need are already on the way
-//   --  barrier: every a written
-//   P3  down rows (already in shared memory) of all k + 1 experts for this
-//       CTA's slice of the hidden dimension -> y; weighted combine +
-//       residual -> h', and this CTA's part of sum(h'^2)
-//   --  barrier: every h' and partial sum written
-// The next layer (or the epilogue) turns h' into xn' = h' r w with
-// r = (sum h'^2 / H + eps)^(-1/2), every CTA for the whole vector.
+// grid-wide barriers are safe.  The experts' intermediate dimension is cut
+// into column blocks of w = 8 (4-bit) or 16 (2-bit) units: a block is w
+// gate/up row pairs plus the matching w columns of the down matrix, one
+// 32-bit word of codes per hidden row (the packed record stores the down
+// matrix column block by column block).  A CTA that owns a block computes
+// its w SwiGLU outputs and, from them, the block's contribution to all H
+// outputs of the down product -- no other CTA's data is needed until the
+// partial outputs are summed.  Per layer:
+//   A  xn = h' r w (every CTA, whole vector) and this CTA's router rows
+//      (fp32, the shared gate vector as row E) -> logits
+//   -- barrier B1 (all logits written); while it completes, the CTA runs
+//      its block of the shared expert
+//   D  every CTA takes the top-k of all logits itself and fetches its run of
+//      routed blocks (each block's bytes are contiguous in the record)
+//   E  routed blocks: gate/up -> a -> weighted down contribution, held in
+//      registers (each thread owns H / 512 hidden rows)
+//   F  the CTA's partial output sum_j p_j y_j + gamma y_s for all H rows ->
+//      global; barrier B2
+//   G  each CTA sums the partials of its slice of rows in a fixed order,
+//      adds the residual -> h', and its part of sum(h'^2); barrier B3
 // Source pages: "What is Flash-MoE?" (a2a-mcp.org), sections
 // "Understanding Mixture-of-Experts", "2. FMA-optimised dequantisation
 // kernels" and "3. Hand-tuned Metal compute shaders" (deferred command-buffer
 // submission there plays the role the persistent kernel plays here: no host
 // round trip between the steps or between layers).
 //
-// Weight bytes move global -> shared with cp.async.bulk (the bulk-copy
-// engine), completion tracked by mbarriers; every weight byte is read from
-// HBM exactly once per layer.  Every wait (mbarrier or grid barrier) is
-// bounded: on expiry the CTA sets FMOE_STATUS_WAIT_TIMEOUT, waits (bounded)
-// for its own copies in flight, and returns.
+// Weight bytes move global -> shared with cp.async.bulk into three block
+// slots and two scale-bias entries (mbarrier completion).  At the top-k the
+// CTA requests its first three routed blocks and asks the L2 to prefetch
+// the rest and the next layer's router rows and shared block, so HBM keeps
+// streaming while the slots turn over.  Every weight byte is read from HBM
+// once per layer.  Every wait (mbarrier or grid barrier) is bounded: on
+// expiry the CTA sets FMOE_STATUS_WAIT_TIMEOUT, waits (bounded) for its own
+// copies in flight, and returns.
 #pragma once
 
 #include <cstdint>
-
-#include <cuda.h>  // CUtensorMap
 
 #include "fmoe.h"
 #include "fmoe_device.cuh"
@@ -42,28 +48,16 @@ namespace fmoe {
 constexpr int kFusedThreads = 512;
 constexpr int kFusedWarps = kFusedThreads / 32;
 constexpr int kFusedMaxLayers = 32;
-constexpr int kFusedMaxRouterRows = 8;
-constexpr int kFusedMaxSharedPairs = 32;
-constexpr int kFusedMaxRoutedPairs = 96;
 constexpr int kFusedMaxK = 8;
-constexpr int kPairsPerChunk = 4;  // gate/up row pairs per bulk-copy chunk (one mbarrier)
-constexpr int kMbRouter = 0;
-constexpr int kMbSPair = kMbRouter + kFusedMaxRouterRows;
-constexpr int kMbSDown = kMbSPair + kFusedMaxSharedPairs / kPairsPerChunk;
-constexpr int kMbRPair = kMbSDown + 1;
-constexpr int kMbRDown = kMbRPair + kFusedMaxRoutedPairs / kPairsPerChunk;
-constexpr int kMbCount = kMbRDown + kFusedMaxK;
+constexpr int kFusedMaxCtas = 160;      // partial outputs in the workspace: [kFusedMaxCtas][H]
+constexpr int kFusedMaxRouterRows = 4;  // router rows (E experts + the shared gate) per CTA
+constexpr int kFusedRowsPerThread = 8;  // hidden rows per thread in the down products: H <= 4096
+constexpr int kFusedMaxRouted = 16;     // routed blocks per CTA
+constexpr int kSlots = 3;
+constexpr int kSbEntries = 2;
+constexpr int kMbSb = kSlots;  // mbarriers: the slots, then the scale-bias entries
+constexpr int kMbCount = kSlots + kSbEntries;
 constexpr long long kWaitCycles = 4000000000LL;  // ~2 s at 2 GHz
-constexpr int kSyncGroups = 2;        // first per-group publication counter in FusedArgs::sync
-constexpr int kMaxGroupCounters = 1022;
-constexpr int kWStage = 144;          // per-warp staged a-group: 8 uint4 + delta + xsum (+pad)
-constexpr int kMaxSliceRows = 64;     // hidden rows per CTA in the down products (2 per lane)
-// Down rows reach shared memory through 3-D tensor copies whose box is
-// kRowPadWords wider than a row: the tensor engine zero-fills the excess, so
-// consecutive rows land 16 bytes off the 128-byte bank period and lanes
-// reading one row each do not collide on banks.
-constexpr int kRowPadWords = 4;
-enum { kTmRoutedCodes = 0, kTmRoutedSb = 1, kTmSharedCodes = 2, kTmSharedSb = 3, kTmPerLayer = 4 };
 
 struct FusedLayer {
   const uint8_t* experts;
@@ -73,38 +67,25 @@ struct FusedLayer {
   const float* norm_w;
 };
 
-// Shared-memory plan (byte offsets), computed on the host.
-//   region A  P1: router rows, shared pairs' codes, shared pairs' scale-bias
-//             P2: routed pairs' codes, routed pairs' scale-bias
-//   region B  shared down rows, then routed down rows (fp32 x during P1)
-//   xq        staged int16 x (P1, P2), then the staged SwiGLU outputs (P3)
+// Shared-memory plan (byte offsets), computed on the host.  A slot holds
+// one column block: [gate/up codes, 8 H bytes][down codes, 4 H bytes]
+// [gate/up scale-bias, w H / 8 bytes]; an entry holds the down scale-bias
+// words of one 64-group of one expert (4 H bytes).
 struct FusedPlan {
-  uint32_t region_a;
-  uint32_t region_b;
-  uint32_t xf;     // fp32 x (may alias the routed part of region B)
-  uint32_t xq;
+  uint32_t slot[kSlots];
+  uint32_t sbe[kSbEntries];
+  uint32_t xs;     // staged int16 x of the layer
   uint32_t logit;  // fp32 [E]
-  uint32_t cand;   // top-k candidates: fp32 [warps][k] values, int32 [warps][k] ids
-  uint32_t ypart;  // fp32 [(k+1)][down rows]
-  uint32_t rpart;  // fp32 [router rows][slices]
-  uint32_t cons;   // inside region A, past the P1 data (free once the routed pairs are
-                   // consumed): per-warp staged a-groups, then per-warp partial down
-                   // sums fp32 [warps][2][kMaxSliceRows]
-  uint32_t prod;   // u32 [k * I / 64]: CTAs producing each routed a-group (static)
+  uint32_t cand;   // top-k candidates: u64 [warps][k]
+  uint32_t red;    // fp32 [kFusedThreads]: partial sums of the row reduction
   uint32_t mbar;
-  uint32_t nd_box;     // rows of every down-row tensor copy (the largest hidden slice)
-  uint32_t sd_codes, sd_sb;         // offsets of the shared expert's padded down rows
-  uint32_t rd_slot;                 // offset of the first routed expert's padded down rows
-  uint32_t rd_stride;               // bytes per routed expert (codes then scale-bias)
-  uint32_t rd_sb;                   // offset of the scale-bias rows inside a routed slot
   uint32_t total;
 };
 
-struct alignas(64) FusedArgs {
-  CUtensorMap tm[kFusedMaxLayers][kTmPerLayer];  // down rows (codes, scale-bias) of the routed / shared records
+struct FusedArgs {
   FusedLayer layers[kFusedMaxLayers];
   int n_layers;
-  int H, I, E, k, bits, sbits;
+  int H, I, E, k;
   float eps;
   float* h;
   float* xn;
@@ -113,9 +94,9 @@ struct alignas(64) FusedArgs {
   float* weights;
   float* gamma;
   float* a;        // [(k+1)][I], shared expert last
-  float* y;        // [(k+1)][H]
   float* ss_part;  // [gridDim.x]
-  unsigned* sync;  // [0] barrier arrivals, [1] exits, [kSyncGroups + g] publications of a-group g
+  float* part;     // [gridDim.x][H] partial outputs
+  unsigned* sync;  // [0] barrier arrivals, [1] exits
   FusedPlan plan;
 };
 
@@ -141,18 +122,13 @@ __device__ __forceinline__ void bulk_g2s(void* dst, const void* src, uint32_t by
       : "memory");
 }
 
-// One try_wait; the thread may be suspended (up to the hint, 20 us) until the
-// phase completes, so waiting warps do not compete for issue slots.
-// 3-D tensor copy global -> shared (box of `map` at coordinates c0, c1, c2).
-__device__ __forceinline__ void tma_load_3d(void* dst, const CUtensorMap* map, int c0, int c1, int c2,
-                                            uint64_t* bar) {
-  asm volatile(
-      "cp.async.bulk.tensor.3d.shared::cluster.global.tile.mbarrier::complete_tx::bytes [%0], [%1, {%2, %3, %4}], "
-      "[%5];" ::"r"(smem_u32(dst)),
-      "l"(map), "r"(c0), "r"(c1), "r"(c2), "r"(smem_u32(bar))
-      : "memory");
+// Asks the L2 to fetch [p, p + bytes) from HBM (no shared memory involved).
+__device__ __forceinline__ void prefetch_l2(const void* p, uint32_t bytes) {
+  asm volatile("cp.async.bulk.prefetch.L2.global [%0], %1;" ::"l"(p), "r"(bytes) : "memory");
 }
 
+// One try_wait; the thread may be suspended (up to the hint, 20 us) until the
+// phase completes, so waiting warps do not compete for issue slots.
 __device__ __forceinline__ bool mbar_try(uint64_t* bar, uint32_t parity) {
   uint32_t done;
   asm volatile(
@@ -182,13 +158,16 @@ __device__ __forceinline__ uint4 lds128(const void* p) { return *reinterpret_cas
 
 __device__ __forceinline__ float ldcg_f(const float* p) { return __ldcg(p); }
 
+__device__ __forceinline__ float4 as_float4(uint4 v) {
+  return make_float4(__uint_as_float(v.x), __uint_as_float(v.y), __uint_as_float(v.z), __uint_as_float(v.w));
+}
+
 // [lo, hi) share of `total` items for part `c` of `n`
-__device__ __forceinline__ void share(int total, int c, int n, int* lo, int* hi) {
+__host__ __device__ __forceinline__ void share(int total, int c, int n, int* lo, int* hi) {
   *lo = (int)(((long long)total * c) / n);
   *hi = (int)(((long long)total * (c + 1)) / n);
 }
 
-// ------------------------------------------------------ GEMV from smem --
 template <int BITS>
 __device__ __forceinline__ GroupCodes<BITS> lds_group(const uint8_t* row, int ng, int g) {
   GroupCodes<BITS> gc;
@@ -200,51 +179,6 @@ __device__ __forceinline__ GroupCodes<BITS> lds_group(const uint8_t* row, int ng
 __device__ __forceinline__ void lds_xv(const StagedX& s, int ng, int g, uint4* xv) {
 #pragma unroll
   for (int u = 0; u < 8; ++u) xv[u] = lds128(s.xs + u * ng + g);
-}
-
-// Dot products of gate and up row of a pair held in shared memory (codes of
-// both rows, then their scale-bias words), one lane group per pair.
-template <int BITS>
-__device__ __forceinline__ void pair_dot_smem(const uint8_t* codes, const uint32_t* sb, int H,
-                                              const StagedX& sx, int lg, int lpr, float* yg, float* yu) {
-  const int ng = H / 64;
-  const int rb = H * BITS / 8;
-  const uint8_t* rg = codes;
-  const uint8_t* ru = codes + rb;
-  const uint32_t* sbg = sb;
-  const uint32_t* sbu = sb + ng;
-  float g = 0.f, u = 0.f;
-  for (int gi = lg; gi < ng; gi += lpr) {
-    const GroupCodes<BITS> cg = lds_group<BITS>(rg, ng, gi);
-    const GroupCodes<BITS> cu = lds_group<BITS>(ru, ng, gi);
-    uint4 xv[8];
-    lds_xv(sx, ng, gi, xv);
-    const float d = sx.delta[gi], xs = sx.xsum[gi];
-    g = group_epilogue(g, sbg[gi], group_dot<BITS>(cg, xv), d, xs);
-    u = group_epilogue(u, sbu[gi], group_dot<BITS>(cu, xv), d, xs);
-  }
-  for (int o = lpr >> 1; o > 0; o >>= 1) {
-    g += __shfl_xor_sync(0xffffffffu, g, o);
-    u += __shfl_xor_sync(0xffffffffu, u, o);
-  }
-  *yg = g;
-  *yu = u;
-}
-
-// Dot product of one down row held in shared memory (codes block, scale-bias block).
-template <int BITS>
-__device__ __forceinline__ float row_dot_smem(const uint8_t* codes, const uint32_t* sb, int I,
-                                              const StagedX& sx, int lg, int lpr) {
-  const int ng = I / 64;
-  float y = 0.f;
-  for (int gi = lg; gi < ng; gi += lpr) {
-    const GroupCodes<BITS> c = lds_group<BITS>(codes, ng, gi);
-    uint4 xv[8];
-    lds_xv(sx, ng, gi, xv);
-    y = group_epilogue(y, sb[gi], group_dot<BITS>(c, xv), sx.delta[gi], sx.xsum[gi]);
-  }
-  for (int o = lpr >> 1; o > 0; o >>= 1) y += __shfl_xor_sync(0xffffffffu, y, o);
-  return y;
 }
 
 // Routing key of logit v at index e: one 64-bit integer whose order is the
@@ -284,89 +218,146 @@ __device__ __forceinline__ uint64_t warp_select_keys(uint64_t* key, int k) {
   return mine;
 }
 
+// Geometry of a column block of an expert with BITS-bit codes.
+template <int BITS>
+struct BlockGeo {
+  static constexpr int kW = 32 / BITS;             // intermediate units per block
+  static constexpr int kPerGroup = 64 / kW;        // blocks per 64-group
+  static constexpr int kTpp = kFusedThreads / kW;  // threads per gate/up row pair
+  __host__ __device__ static uint32_t gu_codes(int H) { return 8u * (uint32_t)H; }
+  __host__ __device__ static uint32_t dn_codes(int H) { return 4u * (uint32_t)H; }
+  __host__ __device__ static uint32_t gu_sb(int H) { return (uint32_t)kW * 2u * (uint32_t)(H / 64) * 4u; }
+};
+
+// Block state shared by the threads of a CTA.
+struct BlockShared {
+  float gu[kFusedWarps][2];  // per-warp partial gate / up sums
+  uint32_t xi[8];            // the block's SwiGLU outputs as int16 pairs
+  float dq[2];               // weight * delta, weight * delta * sum(xi)
+};
+
+// One column block held in `slot`: gate/up of its w row pairs (x staged in
+// sx), SwiGLU, the w outputs quantised to 16-bit fixed point, then the
+// block's down columns for every hidden row this thread owns, scaled by
+// `weight` and added to y.  a_out (global) receives the w SwiGLU outputs.
+// Three block-wide barriers; the slot may be refilled after the last.
+template <int B>
+__device__ __forceinline__ void run_block(const uint8_t* slot, const uint32_t* dsb, int H, const StagedX& sx,
+                                          float weight, float* __restrict__ a_out, BlockShared& bs,
+                                          float (&y)[kFusedRowsPerThread]) {
+  using G = BlockGeo<B>;
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  const int ngH = H / 64;
+  {
+    const int p = tid / G::kTpp, lp = tid % G::kTpp;
+    const uint32_t rb = (uint32_t)H * B / 8;
+    const uint8_t* rg = slot + (size_t)(2 * p) * rb;
+    const uint8_t* ru = rg + rb;
+    const uint32_t* sbg = reinterpret_cast<const uint32_t*>(slot + G::gu_codes(H) + G::dn_codes(H)) + 2 * p * ngH;
+    const uint32_t* sbu = sbg + ngH;
+    float g = 0.f, u = 0.f;
+    for (int gi = lp; gi < ngH; gi += G::kTpp) {
+      const GroupCodes<B> cg = lds_group<B>(rg, ngH, gi);
+      const GroupCodes<B> cu = lds_group<B>(ru, ngH, gi);
+      uint4 xv[8];
+      lds_xv(sx, ngH, gi, xv);
+      const float d = sx.delta[gi], xsm = sx.xsum[gi];
+      g = group_epilogue(g, sbg[gi], group_dot<B>(cg, xv), d, xsm);
+      u = group_epilogue(u, sbu[gi], group_dot<B>(cu, xv), d, xsm);
+    }
+    g = warp_sum(g);
+    u = warp_sum(u);
+    if (lane == 0) {
+      bs.gu[warp][0] = g;
+      bs.gu[warp][1] = u;
+    }
+  }
+  __syncthreads();
+  if (warp == 0) {
+    // SwiGLU of the block's w pairs (pair p's sums come from warps
+    // p * kTpp / 32 ..), then one fixed-point step for the block
+    constexpr int kWpp = G::kTpp / 32;
+    float a = 0.f;
+    if (lane < G::kW) {
+      float gg = 0.f, uu = 0.f;
+#pragma unroll
+      for (int w = 0; w < kWpp; ++w) {
+        gg += bs.gu[lane * kWpp + w][0];
+        uu += bs.gu[lane * kWpp + w][1];
+      }
+      a = silu_mul(gg, uu);
+      a_out[lane] = a;
+    }
+    const float m = __uint_as_float(__reduce_max_sync(0xffffffffu, __float_as_uint(fabsf(a))));
+    const float inv = m > 0.f ? 32767.f / m : 0.f;
+    const float delta = m * (1.f / 32767.f);
+    int q = __float2int_rn(a * inv);
+    q = q > 32767 ? 32767 : (q < -32767 ? -32767 : q);
+    const int qsum = __reduce_add_sync(0xffffffffu, q);
+    const int q_hi = __shfl_down_sync(0xffffffffu, q, 1);
+    if (lane < G::kW && (lane & 1) == 0) bs.xi[lane >> 1] = (uint32_t)(q & 0xFFFF) | ((uint32_t)q_hi << 16);
+    if (lane == 0) {
+      bs.dq[0] = weight * delta;
+      bs.dq[1] = weight * delta * (float)qsum;
+    }
+  }
+  __syncthreads();
+  {
+    const uint4 x0 = make_uint4(bs.xi[0], bs.xi[1], bs.xi[2], bs.xi[3]);
+    const uint4 x1 = make_uint4(bs.xi[4], bs.xi[5], bs.xi[6], bs.xi[7]);
+    const float p1 = bs.dq[0], p2 = bs.dq[1];
+    const uint32_t* dc = reinterpret_cast<const uint32_t*>(slot + G::gu_codes(H));
+#pragma unroll
+    for (int m = 0; m < kFusedRowsPerThread; ++m) {
+      const int i = tid + m * kFusedThreads;
+      if (i < H) {
+        const uint32_t w = dc[i], sbw = dsb[i];
+        const int acc = B == 4 ? word_dot4(w, x0) : word_dot2(w, x0, x1);
+        const float s = __uint_as_float(sbw << 16), b = __uint_as_float(sbw & 0xFFFF0000u);
+        y[m] = fmaf(s, p1 * (float)acc, fmaf(b, p2, y[m]));
+      }
+    }
+  }
+  __syncthreads();
+}
+
 // ------------------------------------------------------------ the kernel --
 template <int BITS, int SBITS>  // routed and shared code widths
 __global__ void __launch_bounds__(kFusedThreads, 1) fused_stack_kernel(const __grid_constant__ FusedArgs A) {
+  using GR = BlockGeo<BITS>;
+  using GS = BlockGeo<SBITS>;
   extern __shared__ __align__(128) unsigned char smem[];
   __shared__ int s_abort;
   __shared__ int s_ids[kFusedMaxK];
   __shared__ float s_p[kFusedMaxK];
+  __shared__ float s_gamma;
+  __shared__ float s_rp[kFusedWarps][kFusedMaxRouterRows];
   __shared__ float s_red[kFusedWarps];
+  __shared__ BlockShared s_blk;
 
   const int c = blockIdx.x, nC = gridDim.x;
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int H = A.H, I = A.I, E = A.E, k = A.k;
-  const int ngH = H / 64, ngI = I / 64;
-  const int lprH = ngH < 32 ? ngH : 32;
+  const int ngH = H / 64;
   const FusedPlan& P = A.plan;
   uint64_t* mbar = reinterpret_cast<uint64_t*>(smem + P.mbar);
-  uint8_t* regA = smem + P.region_a;
-  uint8_t* regB = smem + P.region_b;
-  float* xf = reinterpret_cast<float*>(smem + P.xf);
-  unsigned char* xq_base = smem + P.xq;
-  const StagedX sxq = staged_x_at(xq_base, H);
+  const StagedX sx = staged_x_at(smem + P.xs, H);
   float* slog = reinterpret_cast<float*>(smem + P.logit);
-  uint64_t* cand = reinterpret_cast<uint64_t*>(smem + P.cand);  // [warps][k] routing keys
-  float* ypart = reinterpret_cast<float*>(smem + P.ypart);
-  float* rpart = reinterpret_cast<float*>(smem + P.rpart);
+  uint64_t* cand = reinterpret_cast<uint64_t*>(smem + P.cand);
+  float* sred = reinterpret_cast<float*>(smem + P.red);
 
-  // static work shares of this CTA
-  int r0, r1, s0, s1, q0, q1, i0, i1;
-  share(E + 1, c, nC, &r0, &r1);  // router rows; row E is the shared gate vector
-  share(I, c, nC, &s0, &s1);      // shared expert gate/up pairs
-  share(k * I, c, nC, &q0, &q1);  // routed gate/up pairs, expert-major
-  share(H, c, nC, &i0, &i1);      // hidden rows of the down products and the combine
-  const int nr = r1 - r0, nsp = s1 - s0, nq = q1 - q0, nd = i1 - i0;
-  const int nsl = H >= 512 ? H / 512 : 1;  // router slices per row
-  const int sl_len = H / nsl;
+  // static work of this CTA
+  const int nr = c <= E ? (E - c) / nC + 1 : 0;  // router rows c, c + nC, ... <= E (row E: shared gate)
+  const int NBr = I * BITS / 32, NBs = I * SBITS / 32;
+  const bool has_shared = c < NBs;  // shared block c
+  int q0, q1, i0, i1;
+  share(k * NBr, c, nC, &q0, &q1);  // routed blocks, expert-major
+  share(H, c, nC, &i0, &i1);        // hidden rows of the final sums
+  const int nq = q1 - q0, nd = i1 - i0;
+  const RecordLayout LR = record_layout(BITS, H, I);
+  const RecordLayout LS = record_layout(SBITS, H, I);
+  const bool xthr = tid * 8 < H;  // this thread holds inputs 8 tid .. 8 tid + 7
 
-  const RecordLayout LR = record_layout(A.bits, H, I);   // routed records
-  const RecordLayout LS = record_layout(A.sbits, H, I);  // shared record
-  const uint32_t pc_r = (uint32_t)(2 * LR.gu_row_bytes), pc_s = (uint32_t)(2 * LS.gu_row_bytes);  // pair codes
-  const uint32_t psb = (uint32_t)(2 * ngH * 4);                                                     // pair scale-bias
-  const uint32_t drow_r = (uint32_t)(LR.down_row_bytes), drow_s = (uint32_t)(LS.down_row_bytes);
-  // region A
-  uint8_t* sc_codes = regA + (size_t)nr * H * 4;
-  uint8_t* sc_sb = sc_codes + (size_t)nsp * pc_s;
-  uint8_t* rc_codes = regA;
-  uint8_t* rc_sb = regA + (size_t)nq * pc_r;
-  // region B: the shared expert's padded down rows, then the routed experts'
-  // (each: codes rows of drow + 16 bytes, then scale-bias rows of (I/64 + 4) words)
-  (void)regB;
-  uint8_t* sd_codes = smem + P.sd_codes;
-  const uint32_t* sd_sb = reinterpret_cast<const uint32_t*>(smem + P.sd_sb);
-  uint8_t* rd_base = smem + P.rd_slot;
-  const size_t rd_stride = P.rd_stride;
-  const uint32_t rd_sb_off = P.rd_sb;
-  const uint32_t prow_r = drow_r + 4 * kRowPadWords, prow_s = drow_s + 4 * kRowPadWords;  // padded code rows
-  const uint32_t psbrow = (uint32_t)(ngI + kRowPadWords);                                  // padded sb row, words
-  const uint32_t box_r = P.nd_box * prow_r + P.nd_box * psbrow * 4;  // bytes of one routed expert's copies
-  const uint32_t box_s = P.nd_box * prow_s + P.nd_box * psbrow * 4;
-  uint8_t* cons = smem + P.cons;
-  float* cons_wy = reinterpret_cast<float*>(cons + kFusedWarps * kWStage);
-  // number of CTAs whose pair share touches a-group gg and publish it once per
-  // layer: gg < k I / 64 are the routed experts' groups (routed pairs shared
-  // out over k I pairs), the next I / 64 the shared expert's (I pairs)
-  auto producers = [&](int gg) -> unsigned {
-    const bool routed = gg < k * ngI;
-    const int T = routed ? k * I : I;
-    const int first = (routed ? gg : gg - k * ngI) * 64, last = first + 63;
-    const int c_lo = (int)((((long long)first + 1) * nC - 1) / T);
-    const int c_hi = (int)((((long long)last + 1) * nC - 1) / T);
-    unsigned cnt = 0;
-    for (int cc = c_lo; cc <= c_hi; ++cc) {
-      int a0, a1;
-      share(T, cc, nC, &a0, &a1);
-      if (a0 < a1) ++cnt;
-    }
-    return cnt;
-  };
-
-  // static tables: producers of each routed a-group; first/last expert of each warp's groups
-  unsigned* s_prod = reinterpret_cast<unsigned*>(smem + P.prod);
-  const int U = (k + 1) * ngI;                              // a-groups: k routed experts, then the shared one
-  const int per_warp = (U + kFusedWarps - 1) / kFusedWarps;  // a-groups per warp in the down products
-  for (int gg = tid; gg < U; gg += kFusedThreads) s_prod[gg] = producers(gg);
   if (tid == 0) {
     s_abort = 0;
     for (int i = 0; i < kMbCount; ++i) mbar_init(&mbar[i], 1);
@@ -375,18 +366,53 @@ __global__ void __launch_bounds__(kFusedThreads, 1) fused_stack_kernel(const __g
   __syncthreads();
 
   unsigned bar_target = 0;
-  // per issuing thread (lane 0 of a warp): slots armed, by the parity of their
-  // latest arming (each issuer drains its own copies on abort)
-  constexpr int kMW = (kMbCount + 31) / 32;
-  uint32_t armed[2][kMW];
-#pragma unroll
-  for (int p = 0; p < 2; ++p)
-#pragma unroll
-    for (int i = 0; i < kMW; ++i) armed[p][i] = 0;
-  auto arm = [&](int slot, uint32_t bytes, uint32_t parity) {
-    mbar_expect_tx(&mbar[slot], bytes);
-    armed[parity][slot >> 5] |= 1u << (slot & 31);
-    armed[parity ^ 1][slot >> 5] &= ~(1u << (slot & 31));
+  uint32_t phase = 0;  // per mbarrier: parity of its next completion (same in every thread)
+  uint32_t armed = 0;  // thread 0: mbarriers with copies in flight
+
+  // ---- copies (thread 0 only) ----
+  auto arm = [&](int mb, uint32_t bytes) {
+    mbar_expect_tx(&mbar[mb], bytes);
+    armed |= 1u << mb;
+  };
+  // column block nb of the record `rec` into slot s
+  auto issue_block = [&](int s, const uint8_t* rec, const RecordLayout& L, int nb, uint32_t gu_sb_bytes) {
+    uint8_t* dst = smem + P.slot[s];
+    const uint32_t gub = 8u * (uint32_t)H, dnb = 4u * (uint32_t)H;
+    arm(s, gub + dnb + gu_sb_bytes);
+    bulk_g2s(dst, rec + L.gu_codes + (size_t)nb * gub, gub, &mbar[s]);
+    bulk_g2s(dst + gub, rec + L.down_codes + (size_t)nb * dnb, dnb, &mbar[s]);
+    bulk_g2s(dst + gub + dnb, rec + L.gu_sb + (size_t)nb * gu_sb_bytes, gu_sb_bytes, &mbar[s]);
+  };
+  auto prefetch_block = [&](const uint8_t* rec, const RecordLayout& L, int nb, uint32_t gu_sb_bytes) {
+    const uint32_t gub = 8u * (uint32_t)H, dnb = 4u * (uint32_t)H;
+    prefetch_l2(rec + L.gu_codes + (size_t)nb * gub, gub);
+    prefetch_l2(rec + L.down_codes + (size_t)nb * dnb, dnb);
+    prefetch_l2(rec + L.gu_sb + (size_t)nb * gu_sb_bytes, gu_sb_bytes);
+  };
+  // down scale-bias words of 64-group g of a record into entry e
+  auto issue_sb = [&](int e, const uint8_t* rec, const RecordLayout& L, int g) {
+    arm(kMbSb + e, 4u * (uint32_t)H);
+    bulk_g2s(smem + P.sbe[e], rec + L.down_sb + (size_t)g * H * 4, 4u * (uint32_t)H, &mbar[kMbSb + e]);
+  };
+  auto issue_shared = [&](int l) {  // layer l's shared block -> slot 1, its scale-bias -> entry 0
+    if (!has_shared) return;
+    fence_proxy_async();
+    const uint8_t* rec = A.layers[l].shared;
+    issue_block(1, rec, LS, c, GS::gu_sb(H));
+    issue_sb(0, rec, LS, c / GS::kPerGroup);
+  };
+
+  // ---- waits (all threads; the outcome is agreed block-wide) ----
+  auto wait_mb = [&](int mb) -> bool {
+    const bool ok = mbar_wait(&mbar[mb], (phase >> mb) & 1u);
+    phase ^= 1u << mb;
+    if (tid == 0 && ok) armed &= ~(1u << mb);
+    if (__syncthreads_and(ok)) return true;
+    if (tid == 0) {
+      s_abort = 1;
+      raise_status(FMOE_STATUS_WAIT_TIMEOUT);
+    }
+    return false;
   };
 
   // split grid barrier: arrive once this CTA's results are written, do local
@@ -415,177 +441,130 @@ __global__ void __launch_bounds__(kFusedThreads, 1) fused_stack_kernel(const __g
     return !s_abort;
   };
 
-  auto wait_slot = [&](int slot, uint32_t parity) -> bool {
-    if (mbar_wait(&mbar[slot], parity)) return true;
-    s_abort = 1;
-    raise_status(FMOE_STATUS_WAIT_TIMEOUT);
-    return false;
-  };
-
-  // bulk copies, issued by lane 0 of several warps in parallel (each issue
-  // takes a few hundred cycles; spreading them keeps any one warp short) ---
-  // router rows and the shared expert's gate/up pairs of layer l (region A)
-  auto issue_p1 = [&](int l) {
-    const FusedLayer& LY = A.layers[l];
-    const uint32_t par = (uint32_t)(l & 1);
-    if (lane != 0) return;
-    fence_proxy_async();
-    for (int r = warp; r < nr; r += kFusedWarps) {
-      const int row = r0 + r;
-      const float* src = row < E ? LY.w_router + (size_t)row * H : LY.w_sg;
-      arm(kMbRouter + r, (uint32_t)H * 4, par);
-      bulk_g2s(regA + (size_t)r * H * 4, src, (uint32_t)H * 4, &mbar[kMbRouter + r]);
-    }
-    const int nch = (nsp + kPairsPerChunk - 1) / kPairsPerChunk;
-    for (int ch = (warp + kFusedWarps - nr % kFusedWarps) % kFusedWarps; ch < nch; ch += kFusedWarps) {
-      const int pa = ch * kPairsPerChunk, pb = min(nsp, pa + kPairsPerChunk), n = s0 + pa;
-      arm(kMbSPair + ch, (uint32_t)(pb - pa) * (pc_s + psb), par);
-      bulk_g2s(sc_codes + (size_t)pa * pc_s, LY.shared + LS.gu_codes + (size_t)n * pc_s, (uint32_t)(pb - pa) * pc_s,
-               &mbar[kMbSPair + ch]);
-      bulk_g2s(sc_sb + (size_t)pa * psb, LY.shared + LS.gu_sb + (size_t)n * psb, (uint32_t)(pb - pa) * psb,
-               &mbar[kMbSPair + ch]);
-    }
-  };
-  // the shared expert's down rows of layer l (region B, shared part)
-  auto issue_sdown = [&](int l) {
-    if (nd > 0 && lane == 0 && warp == kFusedWarps - 1) {
-      fence_proxy_async();
-      arm(kMbSDown, box_s, (uint32_t)(l & 1));
-      tma_load_3d(sd_codes, &A.tm[l][kTmSharedCodes], 0, i0, 0, &mbar[kMbSDown]);
-      tma_load_3d(const_cast<uint32_t*>(sd_sb), &A.tm[l][kTmSharedSb], 0, i0, 0, &mbar[kMbSDown]);
-    }
-  };
-  // the routed experts' gate/up pairs of this CTA's share and down rows of its slice
-  auto issue_routed = [&](int l) {
-    const FusedLayer& LY = A.layers[l];
-    const uint32_t par = (uint32_t)(l & 1);
-    if (lane != 0) return;
-    fence_proxy_async();
-    const int nch = (nq + kPairsPerChunk - 1) / kPairsPerChunk;
-    for (int ch = warp; ch < nch; ch += kFusedWarps) {
-      const int qa = ch * kPairsPerChunk, qb = min(nq, qa + kPairsPerChunk);
-      arm(kMbRPair + ch, (uint32_t)(qb - qa) * (pc_r + psb), par);
-      for (int q = qa; q < qb;) {  // runs within one expert
-        const int gq = q0 + q, j = gq / I, n = gq % I;
-        const int cnt = min(qb - q, I - n);
-        const uint8_t* rec = LY.experts + (size_t)s_ids[j] * LR.bytes;
-        bulk_g2s(rc_codes + (size_t)q * pc_r, rec + LR.gu_codes + (size_t)n * pc_r, (uint32_t)cnt * pc_r,
-                 &mbar[kMbRPair + ch]);
-        bulk_g2s(rc_sb + (size_t)q * psb, rec + LR.gu_sb + (size_t)n * psb, (uint32_t)cnt * psb, &mbar[kMbRPair + ch]);
-        q += cnt;
-      }
-    }
-    if (nd > 0) {
-      for (int j = (warp + kFusedWarps - nch % kFusedWarps) % kFusedWarps; j < k; j += kFusedWarps) {
-        uint8_t* dst = rd_base + (size_t)j * rd_stride;
-        arm(kMbRDown + j, box_r, par);
-        tma_load_3d(dst, &A.tm[l][kTmRoutedCodes], 0, i0, s_ids[j], &mbar[kMbRDown + j]);
-        tma_load_3d(dst + rd_sb_off, &A.tm[l][kTmRoutedSb], 0, i0, s_ids[j], &mbar[kMbRDown + j]);
-      }
-    }
-  };
-
   // r = (sum of the CTAs' partial sums of h'^2 / H + eps)^(-1/2), the same
   // summation order in every CTA; all threads take part
   auto norm_scale = [&]() -> float {
-    float v = 0.f;
-    for (int i = tid; i < nC; i += kFusedThreads) v += ldcg_f(A.ss_part + i);
+    float v = tid < nC ? ldcg_f(A.ss_part + tid) : 0.f;
     v = warp_sum(v);
     if (lane == 0) s_red[warp] = v;
     __syncthreads();
-    const float t = warp_sum(lane < kFusedWarps ? s_red[lane] : 0.f);  // same order in every warp
+    float t = 0.f;
+#pragma unroll
+    for (int w = 0; w < kFusedWarps; ++w) t += s_red[w];
+    __syncthreads();
     return 1.f / sqrtf(t / (float)H + A.eps);
   };
 
-  if (A.n_layers > 0) {
-    issue_p1(0);
-    issue_sdown(0);
-  }
+  if (tid == 0 && A.n_layers > 0) issue_shared(0);
 
+  float yr[kFusedRowsPerThread], ys[kFusedRowsPerThread];
+  bool aborted = false;
   for (int l = 0; l < A.n_layers; ++l) {
-    const uint32_t par = (uint32_t)(l & 1);
-    // ------------------------------------------------------------ P1 --
-    // x for this layer: the input (first layer) or h' r w of the previous layer
-    if (l == 0) {
-      for (int j = tid * 4; j < H; j += kFusedThreads * 4)
-        *reinterpret_cast<float4*>(xf + j) = __ldcg(reinterpret_cast<const float4*>(A.xn + j));
-    } else {
-      constexpr int kMaxV = 4;  // float4 per thread (H <= 8192)
-      float4 hv[kMaxV], wv[kMaxV];
-      const float* wprev = A.layers[l - 1].norm_w;
+    const FusedLayer& LY = A.layers[l];
 #pragma unroll
-      for (int it = 0; it < kMaxV; ++it) {
-        const int j = (it * kFusedThreads + tid) * 4;
-        if (j < H) {
-          hv[it] = __ldcg(reinterpret_cast<const float4*>(A.h + j));
-          wv[it] = __ldg(reinterpret_cast<const float4*>(wprev + j));
-        }
+    for (int m = 0; m < kFusedRowsPerThread; ++m) yr[m] = ys[m] = 0.f;
+    // ------------------------------------------------------------- A --
+    // router rows (requested before anything they do not depend on)
+    float4 wr[kFusedMaxRouterRows][2];
+#pragma unroll
+    for (int m = 0; m < kFusedMaxRouterRows; ++m) {
+      const int row = c + m * nC;
+      if (m < nr && xthr) {
+        const float* src = (row < E ? LY.w_router + (size_t)row * H : LY.w_sg) + tid * 8;
+        wr[m][0] = as_float4(ld_stream(src));
+        wr[m][1] = as_float4(ld_stream(src + 4));
+      } else {
+        wr[m][0] = wr[m][1] = make_float4(0.f, 0.f, 0.f, 0.f);
+      }
+    }
+    float xv[8];
+    if (l == 0) {
+      float4 v0 = make_float4(0.f, 0.f, 0.f, 0.f), v1 = v0;
+      if (xthr) {
+        v0 = __ldcg(reinterpret_cast<const float4*>(A.xn + tid * 8));
+        v1 = __ldcg(reinterpret_cast<const float4*>(A.xn + tid * 8 + 4));
+      }
+      xv[0] = v0.x; xv[1] = v0.y; xv[2] = v0.z; xv[3] = v0.w;
+      xv[4] = v1.x; xv[5] = v1.y; xv[6] = v1.z; xv[7] = v1.w;
+    } else {
+      if (!grid_wait()) { aborted = true; break; }  // B3 of the previous layer
+      float4 h0 = make_float4(0.f, 0.f, 0.f, 0.f), h1 = h0, w0 = h0, w1 = h0;
+      const float* wprev = A.layers[l - 1].norm_w;
+      if (xthr) {
+        h0 = __ldcg(reinterpret_cast<const float4*>(A.h + tid * 8));
+        h1 = __ldcg(reinterpret_cast<const float4*>(A.h + tid * 8 + 4));
+        w0 = __ldg(reinterpret_cast<const float4*>(wprev + tid * 8));
+        w1 = __ldg(reinterpret_cast<const float4*>(wprev + tid * 8 + 4));
       }
       const float r = norm_scale();
+      xv[0] = h0.x * r * w0.x; xv[1] = h0.y * r * w0.y; xv[2] = h0.z * r * w0.z; xv[3] = h0.w * r * w0.w;
+      xv[4] = h1.x * r * w1.x; xv[5] = h1.y * r * w1.y; xv[6] = h1.z * r * w1.z; xv[7] = h1.w * r * w1.w;
+    }
+    // stage x: 8 consecutive threads share one 64-group
+    {
+      float m = 0.f;
 #pragma unroll
-      for (int it = 0; it < kMaxV; ++it) {
-        const int j = (it * kFusedThreads + tid) * 4;
-        if (j < H)
-          *reinterpret_cast<float4*>(xf + j) =
-              make_float4(hv[it].x * r * wv[it].x, hv[it].y * r * wv[it].y, hv[it].z * r * wv[it].z,
-                          hv[it].w * r * wv[it].w);
+      for (int i = 0; i < 8; ++i) m = fmaxf(m, fabsf(xv[i]));
+      m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, 1));
+      m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, 2));
+      m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, 4));
+      const float inv = m > 0.f ? 32767.f / m : 0.f;
+      const float delta = m * (1.f / 32767.f);
+      int q[8], sum = 0;
+#pragma unroll
+      for (int i = 0; i < 8; ++i) {
+        int t = __float2int_rn(xv[i] * inv);
+        t = t > 32767 ? 32767 : (t < -32767 ? -32767 : t);
+        q[i] = t;
+        sum += t;
+      }
+      sum += __shfl_xor_sync(0xffffffffu, sum, 1);
+      sum += __shfl_xor_sync(0xffffffffu, sum, 2);
+      sum += __shfl_xor_sync(0xffffffffu, sum, 4);
+      if (xthr) {
+        const int g = tid >> 3, u = tid & 7;
+        sx.xs[u * ngH + g] = make_uint4((uint32_t)(q[0] & 0xFFFF) | ((uint32_t)q[1] << 16),
+                                        (uint32_t)(q[2] & 0xFFFF) | ((uint32_t)q[3] << 16),
+                                        (uint32_t)(q[4] & 0xFFFF) | ((uint32_t)q[5] << 16),
+                                        (uint32_t)(q[6] & 0xFFFF) | ((uint32_t)q[7] << 16));
+        if (u == 0) {
+          sx.delta[g] = delta;
+          sx.xsum[g] = delta * (float)sum;
+        }
       }
     }
-    __syncthreads();
-    // router rows: units (row, slice)
-    for (int u = warp; u < nr * nsl; u += kFusedWarps) {
-      const int r = u / nsl, sl = u % nsl;
-      if (!wait_slot(kMbRouter + r, par)) break;
-      const float* w = reinterpret_cast<const float*>(regA) + (size_t)r * H + sl * sl_len;
-      const float* x = xf + sl * sl_len;
-      float acc = 0.f;
-      for (int cc = lane * 4; cc < sl_len; cc += 128) {
-        const float4 wv = *reinterpret_cast<const float4*>(w + cc);
-        const float4 xv = *reinterpret_cast<const float4*>(x + cc);
-        acc = fmaf(wv.x, xv.x, acc);
-        acc = fmaf(wv.y, xv.y, acc);
-        acc = fmaf(wv.z, xv.z, acc);
-        acc = fmaf(wv.w, xv.w, acc);
-      }
-      acc = warp_sum(acc);
-      if (lane == 0) rpart[r * nsl + sl] = acc;
+    // router partial dot products, reduced in warp order
+#pragma unroll
+    for (int m = 0; m < kFusedMaxRouterRows; ++m) {
+      float d = wr[m][0].x * xv[0];
+      d = fmaf(wr[m][0].y, xv[1], d);
+      d = fmaf(wr[m][0].z, xv[2], d);
+      d = fmaf(wr[m][0].w, xv[3], d);
+      d = fmaf(wr[m][1].x, xv[4], d);
+      d = fmaf(wr[m][1].y, xv[5], d);
+      d = fmaf(wr[m][1].z, xv[6], d);
+      d = fmaf(wr[m][1].w, xv[7], d);
+      d = warp_sum(d);
+      if (lane == 0) s_rp[warp][m] = d;
     }
     __syncthreads();
-    if (tid < nr && !s_abort) {
-      float v = rpart[tid * nsl];
-      for (int sl = 1; sl < nsl; ++sl) v += rpart[tid * nsl + sl];
-      const int row = r0 + tid;
+    if (tid < nr) {
+      float v = 0.f;
+      for (int w = 0; w < kFusedWarps; ++w) v += s_rp[w][tid];
+      const int row = c + tid * nC;
       if (row < E) A.logits[row] = v;
       else A.gamma[0] = 1.f / (1.f + expf(-v));
     }
-    if (s_abort) break;
     grid_arrive();  // B1: logits written
-    // while the other CTAs finish: quantise x, run the shared expert's gate/up pairs
-    stage_x(xf, H, sxq);
-    __syncthreads();
-    {
-      const int ppu = 32 / lprH;  // pairs per warp unit
-      const int ps = lane / lprH, lg = lane % lprH;
-      for (int u0 = warp * ppu; u0 < nsp; u0 += kFusedWarps * ppu) {
-        const int p = u0 + ps;
-        bool ok = true;
-        if (p < nsp) ok = wait_slot(kMbSPair + p / kPairsPerChunk, par);
-        if (!__all_sync(0xffffffffu, ok)) break;
-        float g = 0.f, uu = 0.f;
-        const int pp = p < nsp ? p : nsp - 1;
-        const uint8_t* cp = sc_codes + (size_t)pp * pc_s;
-        const uint32_t* sp = reinterpret_cast<const uint32_t*>(sc_sb + (size_t)pp * psb);
-        pair_dot_smem<SBITS>(cp, sp, H, sxq, lg, lprH, &g, &uu);
-        if (lg == 0 && p < nsp) A.a[(size_t)k * I + s0 + p] = silu_mul(g, uu);
-      }
+    // ------------------------------------------------------------- C --
+    // while the other CTAs finish: this CTA's block of the shared expert
+    if (has_shared) {
+      if (!wait_mb(1) || !wait_mb(kMbSb + 0)) { aborted = true; break; }
+      run_block<SBITS>(smem + P.slot[1], reinterpret_cast<const uint32_t*>(smem + P.sbe[0]), H, sx, 1.f,
+                       A.a + (size_t)k * I + (size_t)c * GS::kW, s_blk, ys);
     }
-    __syncthreads();
-    // publish the shared expert's a-groups this CTA produced
-    if (nsp > 0 && tid <= (s1 - 1) / 64 - s0 / 64)
-      asm volatile("red.release.gpu.global.add.u32 [%0], 1;" ::"l"(A.sync + kSyncGroups + k * ngI + s0 / 64 + tid)
-                   : "memory");
-    if (s_abort || !grid_wait()) break;
-    // ------------------------------------------------------------ P2 --
+    if (!grid_wait()) { aborted = true; break; }
+    // ------------------------------------------------------------- D --
     {
       // routing: every thread keys up to two logits; per-warp top-k, then one
       // warp merges the warps' candidates
@@ -635,186 +614,102 @@ __global__ void __launch_bounds__(kFusedThreads, 1) fused_stack_kernel(const __g
             A.weights[lane] = s_p[lane];
           }
         }
+        if (lane == 0) s_gamma = ldcg_f(A.gamma);
         if (c == 0 && lane == 0 && nan_seen) raise_status(FMOE_STATUS_NAN_LOGIT);
       }
       __syncthreads();
-      issue_routed(l);
     }
-    {
-      const int ppu = 32 / lprH;
-      const int ps = lane / lprH, lg = lane % lprH;
-      for (int u0 = warp * ppu; u0 < nq; u0 += kFusedWarps * ppu) {
-        const int q = u0 + ps;
-        bool ok = true;
-        if (q < nq) ok = wait_slot(kMbRPair + q / kPairsPerChunk, par);
-        if (!__all_sync(0xffffffffu, ok)) break;
-        float g = 0.f, uu = 0.f;
-        const int qq = q < nq ? q : nq - 1;
-        const uint8_t* cp = rc_codes + (size_t)qq * pc_r;
-        const uint32_t* sp = reinterpret_cast<const uint32_t*>(rc_sb + (size_t)qq * psb);
-        pair_dot_smem<BITS>(cp, sp, H, sxq, lg, lprH, &g, &uu);
-        if (lg == 0 && q < nq) A.a[q0 + q] = silu_mul(g, uu);  // a[j][n], q0 + q = j * I + n
+    // requests: the first routed blocks into the slots, the down scale-bias
+    // of their (at most two) 64-groups, L2 prefetches of the remaining
+    // blocks and of the next layer's router rows and shared block.  A routed
+    // block q (= j * NBr + nb) lies in 64-group q / kPerGroup of the
+    // concatenated experts.
+    const int key0 = q0 / GR::kPerGroup;
+    if (tid == 0) {
+      fence_proxy_async();
+      for (int b = 0; b < nq; ++b) {
+        const int q = q0 + b, j = q / NBr, nb = q % NBr;
+        const uint8_t* rec = LY.experts + (size_t)s_ids[j] * LR.bytes;
+        if (b < kSlots) issue_block(b, rec, LR, nb, GR::gu_sb(H));
+        else prefetch_block(rec, LR, nb, GR::gu_sb(H));
+        if (b == 0 || q / GR::kPerGroup != (q - 1) / GR::kPerGroup)
+          issue_sb(q / GR::kPerGroup == key0 ? 0 : 1, rec, LR, nb / GR::kPerGroup);
       }
-    }
-    __syncthreads();
-    if (s_abort) break;
-    // this CTA's SwiGLU outputs are written: publish them, one counter per
-    // 64-wide group of a (release: the writes above are visible to whoever
-    // acquires the counter)
-    if (nq > 0 && tid <= (q1 - 1) / 64 - q0 / 64)
-      asm volatile("red.release.gpu.global.add.u32 [%0], 1;" ::"l"(A.sync + kSyncGroups + q0 / 64 + tid) : "memory");
-    // ---------------------------------------------- down products, dataflow --
-    // The routed experts' down rows of this CTA's hidden slice, one a-group at
-    // a time: each warp owns a contiguous run of a-groups, waits (one round of
-    // polls) until the CTAs producing them have published them, loads them
-    // (one round trip), then quantises each group and accumulates it, one
-    // hidden row per lane.  The warps' sums are added in warp order.
-    if (nd > 0) {
-      constexpr int kBatch = 6;
-      const int u_lo = min(U, warp * per_warp), u_hi = min(U, u_lo + per_warp);
-      uint8_t* wst = cons + warp * kWStage;
-      const uint4* wxs = reinterpret_cast<const uint4*>(wst);
-      float* wdx = reinterpret_cast<float*>(wst + 128);
-      float acc0 = 0.f, acc1 = 0.f;
-      const int j_first = u_lo < u_hi ? u_lo / ngI : -1;
-      int j_cur = -1;
-      bool ok = true;
-      for (int ub = u_lo; ub < u_hi && ok; ub += kBatch) {
-        const int nb = min(kBatch, u_hi - ub);
-        // 1. one round of polls for the batch
-        bool ready = lane >= nb;
-        const long long t0 = clock64();
-        while (true) {
-          if (!ready) {
-            unsigned v;
-            asm volatile("ld.acquire.gpu.global.u32 %0, [%1];" : "=r"(v) : "l"(A.sync + kSyncGroups + ub + lane)
-                         : "memory");
-            ready = v >= (unsigned)(l + 1) * s_prod[ub + lane];
-          }
-          if (__all_sync(0xffffffffu, ready)) break;
-          if (clock64() - t0 > kWaitCycles) {
-            if (lane == 0) {
-              s_abort = 1;
-              raise_status(FMOE_STATUS_WAIT_TIMEOUT);
-            }
-            ok = false;
-            break;
-          }
+      if (l + 1 < A.n_layers) {
+        const FusedLayer& NX = A.layers[l + 1];
+        for (int m = 0; m < nr; ++m) {
+          const int row = c + m * nC;
+          prefetch_l2(row < E ? NX.w_router + (size_t)row * H : NX.w_sg, 4u * (uint32_t)H);
         }
-        if (!ok) break;
-        // 2. one round of loads: lane holds inputs 2 lane, 2 lane + 1 of each group
-        float2 av[kBatch];
-#pragma unroll
-        for (int t = 0; t < kBatch; ++t)
-          if (t < nb) {
-            const int u = ub + t;
-            av[t] = __ldcg(reinterpret_cast<const float2*>(A.a + (size_t)(u / ngI) * I + (u % ngI) * 64) + lane);
-          }
-        // 3. quantise and accumulate each group
-#pragma unroll 1
-        for (int t = 0; t < nb; ++t) {
-          const int u = ub + t, j = u / ngI, g = u % ngI;
-          if (j != j_cur) {
-            if (j_cur >= 0) {  // flush the previous expert's sums
-              float* wy = cons_wy + (warp * 2 + (j_cur == j_first ? 0 : 1)) * kMaxSliceRows;
-              wy[lane] = acc0;
-              wy[lane + 32] = acc1;
-              acc0 = acc1 = 0.f;
-            }
-            ok = wait_slot(j == k ? kMbSDown : kMbRDown + j, par);
-            if (!__all_sync(0xffffffffu, ok)) { ok = false; break; }
-            j_cur = j;
-          }
-          // group max of |a| in one redux (the bits of a non-negative float order as integers)
-          const float m = __uint_as_float(
-              __reduce_max_sync(0xffffffffu, __float_as_uint(fmaxf(fabsf(av[t].x), fabsf(av[t].y)))));
-          const float inv = m > 0.f ? 32767.f / m : 0.f;
-          const float delta = m * (1.f / 32767.f);
-          int qa = __float2int_rn(av[t].x * inv), qb = __float2int_rn(av[t].y * inv);
-          qa = qa > 32767 ? 32767 : (qa < -32767 ? -32767 : qa);
-          qb = qb > 32767 ? 32767 : (qb < -32767 ? -32767 : qb);
-          const int isum = __reduce_add_sync(0xffffffffu, qa + qb);
-          __syncwarp();  // the previous group's staged values have been read
-          reinterpret_cast<uint32_t*>(wst)[lane] = (uint32_t)(qa & 0xFFFF) | ((uint32_t)qb << 16);
-          if (lane == 0) {
-            wdx[0] = delta;
-            wdx[1] = delta * (float)isum;
-          }
-          __syncwarp();
-          uint4 xv[8];
-#pragma unroll
-          for (int q = 0; q < 8; ++q) xv[q] = wxs[q];
-          const float dl = wdx[0], xsm = wdx[1];
-          const bool shd = j == k;
-          const uint8_t* base = shd ? sd_codes : rd_base + (size_t)j * rd_stride;
-          const uint32_t drow = shd ? prow_s : prow_r;
-          const uint32_t* sbb = shd ? sd_sb : reinterpret_cast<const uint32_t*>(base + rd_sb_off);
-#pragma unroll 1
-          for (int half = 0; half < 2; ++half) {
-            const int rr = lane + 32 * half;
-            if (rr >= nd) break;
-            const uint8_t* cp = base + (size_t)rr * drow;
-            const int A32 = shd ? group_dot<SBITS>(lds_group<SBITS>(cp, ngI, g), xv)
-                                : group_dot<BITS>(lds_group<BITS>(cp, ngI, g), xv);
-            const float y = group_epilogue(half ? acc1 : acc0, sbb[rr * psbrow + g], A32, dl, xsm);
-            if (half) acc1 = y;
-            else acc0 = y;
-          }
+        if (has_shared) {
+          prefetch_block(NX.shared, LS, c, GS::gu_sb(H));
+          prefetch_l2(NX.shared + LS.down_sb + (size_t)(c / GS::kPerGroup) * H * 4, 4u * (uint32_t)H);
         }
       }
-      if (ok && j_cur >= 0) {
-        float* wy = cons_wy + (warp * 2 + (j_cur == j_first ? 0 : 1)) * kMaxSliceRows;
-        wy[lane] = acc0;
-        wy[lane + 32] = acc1;
-      }
     }
-    __syncthreads();
-    if (s_abort) break;
-    // the routed down rows are consumed and the a-groups loaded: the next
-    // layer's router rows and shared pairs can stream now
-    if (l + 1 < A.n_layers) issue_p1(l + 1);
-    // y of each expert for this slice: the warps' sums in warp order
-    for (int idx = tid; idx < (k + 1) * nd; idx += kFusedThreads) {
-      const int j = idx / nd, rr = idx - j * nd;
-      float v = 0.f;
-      for (int w = 0; w < kFusedWarps; ++w) {
-        const int lo = w * per_warp;
-        if (lo >= U) break;
-        const int jf = lo / ngI, jl = (min(U, lo + per_warp) - 1) / ngI;
-        if (jf == j) v += cons_wy[(w * 2) * kMaxSliceRows + rr];
-        else if (jl == j) v += cons_wy[(w * 2 + 1) * kMaxSliceRows + rr];
-      }
-      ypart[j * nd + rr] = v;
-    }
-    __syncthreads();
+    // ------------------------------------------------------------- E --
     {
-      const float gm = ldcg_f(A.gamma);
-      float ss = 0.f;
-      for (int rr = tid; rr < nd; rr += kFusedThreads) {
-        const int i = i0 + rr;
-        float v = ldcg_f(A.h + i);
-        for (int j = 0; j < k; ++j) v = fmaf(s_p[j], ypart[j * nd + rr], v);
-        v = fmaf(gm, ypart[k * nd + rr], v);
-        A.h[i] = v;
-        for (int j = 0; j <= k; ++j) A.y[(size_t)j * H + i] = ypart[j * nd + rr];
-        ss = fmaf(v, v, ss);
+      bool sb_ready[kSbEntries] = {false, false};
+      for (int b = 0; b < nq; ++b) {
+        const int q = q0 + b, j = q / NBr, nb = q % NBr;
+        const int s = b % kSlots, e = q / GR::kPerGroup == key0 ? 0 : 1;
+        if (!wait_mb(s)) { aborted = true; break; }
+        if (!sb_ready[e]) {
+          if (!wait_mb(kMbSb + e)) { aborted = true; break; }
+          sb_ready[e] = true;
+        }
+        run_block<BITS>(smem + P.slot[s], reinterpret_cast<const uint32_t*>(smem + P.sbe[e]), H, sx, s_p[j],
+                        A.a + (size_t)j * I + (size_t)nb * GR::kW, s_blk, yr);
+        if (tid == 0 && b + kSlots < nq) {  // the slot is free: its next block
+          const int q2 = q + kSlots, j2 = q2 / NBr, nb2 = q2 % NBr;
+          fence_proxy_async();
+          issue_block(s, LY.experts + (size_t)s_ids[j2] * LR.bytes, LR, nb2, GR::gu_sb(H));
+        }
       }
-      ss = warp_sum(ss);
-      if (lane == 0) s_red[warp] = ss;
+      if (aborted) break;
+    }
+    // every slot and entry is consumed: the next layer's shared block can come in
+    if (tid == 0 && l + 1 < A.n_layers) issue_shared(l + 1);
+    // ------------------------------------------------------------- F --
+    {
+      const float gm = s_gamma;
+      float* part = A.part + (size_t)c * H;
+#pragma unroll
+      for (int m = 0; m < kFusedRowsPerThread; ++m) {
+        const int i = tid + m * kFusedThreads;
+        if (i < H) part[i] = fmaf(gm, ys[m], yr[m]);
+      }
+    }
+    grid_arrive();  // B2: partial outputs written
+    if (!grid_wait()) { aborted = true; break; }
+    // ------------------------------------------------------------- G --
+    {
+      // rows i0 + r, r < nd: ngr threads per row each sum every ngr-th CTA's
+      // partial; then one thread per row adds those sums in order
+      const int ngr = nd > 0 ? kFusedThreads / nd : 0;
+      const int r = nd > 0 ? tid % nd : 0, pg = nd > 0 ? tid / nd : kFusedThreads;
+      if (pg < ngr) {
+        float v = 0.f;
+        for (int p = pg; p < nC; p += ngr) v += ldcg_f(A.part + (size_t)p * H + i0 + r);
+        sred[pg * nd + r] = v;
+      }
       __syncthreads();
-      if (tid == 0) {
-        float t = 0.f;
-        for (int w = 0; w < kFusedWarps; ++w) t += s_red[w];
-        A.ss_part[c] = t;
+      float ss = 0.f;
+      if (tid < nd) {
+        float v = ldcg_f(A.h + i0 + tid);
+        for (int g = 0; g < ngr; ++g) v += sred[g * nd + tid];
+        A.h[i0 + tid] = v;
+        ss = v * v;
+      }
+      if (warp == 0) {
+        ss = warp_sum(ss);
+        if (lane == 0) A.ss_part[c] = ss;
       }
     }
     grid_arrive();  // B3: h' and the partial sums written
-    // the shared down rows are consumed: the next layer's can stream now
-    if (l + 1 < A.n_layers) issue_sdown(l + 1);
-    if (!grid_wait()) break;
   }
 
-  if (!s_abort) {
+  if (!aborted && A.n_layers > 0 && grid_wait()) {
     // epilogue: xn' of the last layer for this CTA's rows
     const float r = norm_scale();
     const float* w = A.layers[A.n_layers - 1].norm_w;
@@ -824,87 +719,56 @@ __global__ void __launch_bounds__(kFusedThreads, 1) fused_stack_kernel(const __g
       __threadfence();
       const unsigned prev = atomicAdd(&A.sync[1], 1u);
       if (prev == (unsigned)nC - 1) {  // every CTA is past its last barrier and wait
-        for (int i = 0; i < kSyncGroups + (k + 1) * ngI; ++i) A.sync[i] = 0;
+        A.sync[0] = 0;
+        A.sync[1] = 0;
         __threadfence();
       }
     }
-  } else if (lane == 0) {
-    // drain: wait (bounded) for this issuer's own copies still in flight
-    for (int p = 0; p < 2; ++p)
-      for (int s2 = 0; s2 < kMbCount; ++s2)
-        if (armed[p][s2 >> 5] & (1u << (s2 & 31))) (void)mbar_wait(&mbar[s2], (uint32_t)p);
+  } else if (tid == 0) {
+    // drain: wait (bounded) for this CTA's copies still in flight
+    for (int mb = 0; mb < kMbCount; ++mb)
+      if (armed & (1u << mb)) (void)mbar_wait(&mbar[mb], (phase >> mb) & 1u);
   }
 }
 
-// Host-side plan: shared-memory layout for n_ctas CTAs; false if it does not fit.
+// Host-side plan: shared-memory layout for n_ctas CTAs; false if the shape
+// does not fit the kernel.
 inline bool fused_plan(int H, int I, int E, int k, int bits, int sbits, int n_ctas, size_t max_smem,
                        FusedPlan* out) {
-  // every per-CTA block moved by cp.async.bulk and every 16-byte shared load
-  // must be 16-byte aligned: a down row's scale-bias words (I/64 * 4 bytes)
-  // and a pair's (2 * H/64 * 4 bytes) must come in multiples of 16 bytes
-  if ((I / 64) % 4 != 0 || (H / 64) % 2 != 0) return false;
-  if (E > 2 * kFusedThreads || k > kFusedMaxK) return false;
-  auto cdiv = [](long long a, long long b) { return (a + b - 1) / b; };
-  const long long nr = cdiv(E + 1, n_ctas), nsp = cdiv(I, n_ctas), nq = cdiv((long long)k * I, n_ctas),
-                  nd = cdiv(H, n_ctas);
-  if (nr > kFusedMaxRouterRows || nsp > kFusedMaxSharedPairs || nq > kFusedMaxRoutedPairs) return false;
-  const RecordLayout LR = record_layout(bits, H, I), LS = record_layout(sbits, H, I);
-  const int ngH = H / 64, ngI = I / 64;
-  const long long psb = 2LL * ngH * 4;
-  const long long pair_r = 2 * (long long)LR.gu_row_bytes + psb;
-  const long long pair_s = 2 * (long long)LS.gu_row_bytes + psb;
-  const long long sa = ((long long)staged_x_bytes(I) + 15) & ~15LL;
+  if (H < 64 || H % 64 || I < 64 || I % 64 || H > kFusedThreads * kFusedRowsPerThread) return false;
+  if (E < 1 || E > 2 * kFusedThreads || k < 1 || k > kFusedMaxK || k > E) return false;
+  if (n_ctas < 1 || n_ctas > kFusedMaxCtas) return false;
+  if (E + 1 > kFusedMaxRouterRows * n_ctas) return false;
+  auto wn = [](int b) { return 32 / b; };
+  const int nbr = I / wn(bits), nbs = I / wn(sbits);
+  if (nbs > n_ctas) return false;  // one shared block per CTA at most
+  // routed blocks per CTA; a CTA's run spans at most two 64-groups
+  const int per_cta = (k * nbr + n_ctas - 1) / n_ctas;
+  if (per_cta > kFusedMaxRouted || per_cta > 64 / wn(bits) + 1) return false;
+  if ((H + n_ctas - 1) / n_ctas > 32) return false;  // rows per CTA in the final sums: one warp
+  auto blk = [&](int b) -> long long { return 12LL * H + (long long)wn(b) * 2 * (H / 64) * 4; };
+  const long long slot = blk(bits) > blk(sbits) ? blk(bits) : blk(sbits);
   auto al = [](long long v) { return (v + 127) & ~127LL; };
-  if (nd > kMaxSliceRows || (long long)(k + 1) * ngI > kMaxGroupCounters) return false;
-  const long long a_p1 = nr * H * 4 + nsp * pair_s;
-  const long long a_p2 = nq * pair_r;
-  const long long cons_off = (a_p1 + 127) & ~127LL;
-  const long long cons_bytes = (long long)kFusedWarps * kWStage + (long long)kFusedWarps * 2 * kMaxSliceRows * 4;
-  const long long regA = a_p2 > cons_off + cons_bytes ? a_p2 : cons_off + cons_bytes;
-  // padded down-row boxes (tensor copies of nd rows, each kRowPadWords wider than a row)
-  const long long dw_r = (long long)LR.down_row_bytes / 4, dw_s = (long long)LS.down_row_bytes / 4;
-  if (dw_r + kRowPadWords > 256 || dw_s + kRowPadWords > 256 || ngI + kRowPadWords > 256 || nd > 256) return false;
-  const long long c_r = al(nd * (dw_r + kRowPadWords) * 4), c_s = al(nd * (dw_s + kRowPadWords) * 4);
-  const long long sbb = al(nd * (ngI + kRowPadWords) * 4);
-  const long long sdown = c_s + sbb;
-  const long long rstride = c_r + sbb;
-  const long long rdown = k * rstride;
-  const long long xq = (long long)staged_x_bytes(H);
   FusedPlan p;
   long long o = 0;
-  p.region_a = (uint32_t)o;
-  p.cons = (uint32_t)(o + cons_off);
-  o = al(o + regA);
-  p.region_b = (uint32_t)o;
-  p.nd_box = (uint32_t)nd;
-  p.sd_codes = (uint32_t)o;
-  p.sd_sb = (uint32_t)(o + c_s);
-  p.rd_slot = (uint32_t)(o + sdown);
-  p.rd_stride = (uint32_t)rstride;
-  p.rd_sb = (uint32_t)c_r;
-  const long long xf_bytes = (long long)H * 4;
-  if (rdown >= xf_bytes) {
-    p.xf = (uint32_t)(o + sdown);  // aliases the routed down rows (P1 only)
-    o = al(o + sdown + rdown);
-  } else {
-    o = al(o + sdown + rdown);
-    p.xf = (uint32_t)o;
-    o = al(o + xf_bytes);
+  for (int s = 0; s < kSlots; ++s) {
+    p.slot[s] = (uint32_t)o;
+    o = al(o + slot);
   }
-  p.xq = (uint32_t)o;
-  o = al(o + xq);
+  for (int e = 0; e < kSbEntries; ++e) {
+    p.sbe[e] = (uint32_t)o;
+    o = al(o + 4LL * H);
+  }
+  p.xs = (uint32_t)o;
+  o = al(o + (long long)staged_x_bytes(H));
   p.logit = (uint32_t)o;
-  o = al(o + (long long)E * 4);
+  o = al(o + 4LL * E);
   p.cand = (uint32_t)o;
-  o = al(o + 2LL * kFusedWarps * kFusedMaxK * 4);
-  p.ypart = (uint32_t)o;
-  o = al(o + (k + 1) * nd * 4);
-  p.rpart = (uint32_t)o;
-  o = al(o + nr * (H >= 512 ? H / 512 : 1) * 4);
-  p.prod = (uint32_t)o;
-  o = al(o + 4LL * (k + 1) * ngI);
+  o = al(o + 8LL * kFusedWarps * kFusedMaxK);
+  p.red = (uint32_t)o;
+  o = al(o + 4LL * kFusedThreads);
   p.mbar = (uint32_t)o;
-  o = al(o + kMbCount * 8);
+  o = al(o + 8LL * kMbCount);
   p.total = (uint32_t)o;
   if ((size_t)o > max_smem) return false;
   *out = p;

@@ -19,8 +19,6 @@
 #include <cstring>
 #include <mutex>
 
-#include <cuda.h>
-#include <cudaTypedefs.h>
 #include <cuda_runtime.h>
 
 #include "fmoe.h"
@@ -225,36 +223,34 @@ __device__ __forceinline__ void gateup_rows(const uint8_t* rec, const ExpertSet&
   }
 }
 
-// Down rows of one record: units of 32 / lanes_per_row rows.
+// Down product of one record for one hidden row: the column blocks of each
+// 64-group of the intermediate dimension (8 words of 4-bit codes or 4 of
+// 2-bit codes, one per block), accumulated exactly in int32 and scaled once
+// per group.  Consecutive threads take consecutive rows, so every load of a
+// warp is one contiguous 128-byte line.
 template <int BITS>
-__device__ __forceinline__ void down_rows(const uint8_t* rec, const ExpertSet& es,
-                                          const StagedX& sx, float* __restrict__ y_out, int unit0,
-                                          int unit1) {
-  const int I = es.I;
-  const int ng = I / 64;
-  const int lpr = ng < 32 ? ng : 32;
-  const int gpl = ng / lpr;
-  const int rpu = 32 / lpr;
-  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
-  const int rs = lane / lpr, lg = lane % lpr;
-  const RecordLayout L = record_layout(BITS, es.H, I);
-  const uint8_t* codes = rec + L.down_codes;
-  const uint32_t* sbw = reinterpret_cast<const uint32_t*>(rec + L.down_sb);
-  for (int u = unit0 + warp; u < unit1; u += kWarps) {
-    const int r = u * rpu + rs;
-    const uint8_t* row = codes + (size_t)r * L.down_row_bytes;
-    float y = 0.f;
-    for (int m = 0; m < gpl; ++m) {
-      const int g = lg + m * lpr;
-      const GroupCodes<BITS> c = load_group<BITS>(row, ng, g);
-      const uint32_t sb = ld_stream_u32(sbw + (size_t)r * ng + g);
-      uint4 xv[8];
-      load_xv(sx, ng, g, xv);
-      y = group_epilogue(y, sb, group_dot<BITS>(c, xv), sx.delta[g], sx.xsum[g]);
+__device__ __forceinline__ float down_row_cols(const uint8_t* rec, const ExpertSet& es, const StagedX& sx,
+                                               int row) {
+  const int H = es.H, I = es.I, ngI = I / 64;
+  constexpr int kWpg = BITS == 4 ? 8 : 4;  // column blocks (words) per group
+  const RecordLayout L = record_layout(BITS, H, I);
+  const uint32_t* codes = reinterpret_cast<const uint32_t*>(rec + L.down_codes) + row;
+  const uint32_t* sbw = reinterpret_cast<const uint32_t*>(rec + L.down_sb) + row;
+  float y = 0.f;
+  for (int g = 0; g < ngI; ++g) {
+    uint32_t w[kWpg];
+#pragma unroll
+    for (int b = 0; b < kWpg; ++b) w[b] = ld_stream_u32(codes + (size_t)(g * kWpg + b) * H);
+    const uint32_t sb = ld_stream_u32(sbw + (size_t)g * H);
+    int acc = 0;
+#pragma unroll
+    for (int b = 0; b < kWpg; ++b) {
+      if (BITS == 4) acc += word_dot4(w[b], sx.xs[b * ngI + g]);
+      else acc += word_dot2(w[b], sx.xs[(2 * b) * ngI + g], sx.xs[(2 * b + 1) * ngI + g]);
     }
-    for (int o = lpr >> 1; o > 0; o >>= 1) y += __shfl_xor_sync(0xffffffffu, y, o);
-    if (lg == 0) y_out[r] = y;
+    y = group_epilogue(y, sb, acc, sx.delta[g], sx.xsum[g]);
   }
+  return y;
 }
 
 __device__ __forceinline__ void unit_range(int n_units, int* u0, int* u1) {
@@ -303,28 +299,26 @@ gateup_kernel(ExpertSet es, const float* __restrict__ xn, const int32_t* __restr
     gateup_rows<2>(rec, es, sx, a_out, u0, u1);
 }
 
-__global__ void __launch_bounds__(kThreads)
+// grid (H / kDownThreads, T * (k + 1) slots); one hidden row per thread.
+constexpr int kDownThreads = 128;
+__global__ void __launch_bounds__(kDownThreads)
 down_kernel(ExpertSet es, const int32_t* __restrict__ ids, const float* __restrict__ a,
             float* __restrict__ y) {
   extern __shared__ __align__(128) unsigned char smem[];
   const int slot = blockIdx.y, t = slot / (es.k + 1), j = slot % (es.k + 1);
   int bits;
   const uint8_t* rec = slot_record(es, ids, t, j, &bits);
-  const int ng = es.I / 64, lpr = ng < 32 ? ng : 32;
-  int u0, u1;
-  unit_range(es.H / (32 / lpr), &u0, &u1);
+  const int row = (int)blockIdx.x * kDownThreads + (int)threadIdx.x;
   float* y_out = y + (size_t)slot * es.H;
   if (!rec) {
-    for (int i = u0 * (32 / lpr) + (int)threadIdx.x; i < u1 * (32 / lpr); i += blockDim.x) y_out[i] = 0.f;
+    if (row < es.H) y_out[row] = 0.f;
     return;
   }
   const StagedX sx = staged_x_at(smem, es.I);
   stage_x(a + (size_t)slot * es.I, es.I, sx);
   __syncthreads();
-  if (bits == 4)
-    down_rows<4>(rec, es, sx, y_out, u0, u1);
-  else
-    down_rows<2>(rec, es, sx, y_out, u0, u1);
+  if (row >= es.H) return;
+  y_out[row] = bits == 4 ? down_row_cols<4>(rec, es, sx, row) : down_row_cols<2>(rec, es, sx, row);
 }
 
 // ---------------------------------------------------------- combine ----
@@ -365,50 +359,49 @@ combine_kernel(const float* __restrict__ y, const float* __restrict__ weights,
 }
 
 // ------------------------------------------------------- device packer ----
-// One thread per 16-byte code chunk of a packed row.  Packed row pr of an
-// expert: pr < 2I are the interleaved gate/up rows (pr = 2n + m: logical
-// matrix m, row n; H inputs), then H down rows (I inputs).
+// One thread per 16-byte chunk of packed codes.  Gate/up: packed row pr of
+// an expert (pr = 2n + m: logical matrix m, row n; H inputs), chunk p of the
+// row.  Down: column block nb, rows 4j .. 4j + 3 (one word each).
 template <int BITS>
 __global__ void pack_codes_kernel(const uint8_t* __restrict__ q, int n_experts, int H, int I,
                                   uint8_t* __restrict__ out) {
   const RecordLayout L = record_layout(BITS, H, I);
   const size_t n = (size_t)H * I;
-  const int gu_chunks = H * BITS / 128, dn_chunks = I * BITS / 128;
-  const size_t per_expert = (size_t)2 * I * gu_chunks + (size_t)H * dn_chunks;
+  const int gu_chunks = H * BITS / 128;
+  constexpr int per_word = 32 / BITS, per_byte = 8 / BITS;
+  const size_t gu_total = (size_t)2 * I * gu_chunks;
+  const size_t per_expert = gu_total + (size_t)(I / per_word) * (H / 4);
   const size_t total = per_expert * n_experts;
   for (size_t c = blockIdx.x * (size_t)blockDim.x + threadIdx.x; c < total; c += (size_t)gridDim.x * blockDim.x) {
     const size_t e = c / per_expert;
     size_t r = c % per_expert;
-    int K, p;
-    const uint8_t* src;
+    const uint8_t* in[4];  // the 32 / BITS inputs of each of the four words
     uint8_t* dst;
-    if (r < (size_t)2 * I * gu_chunks) {
+    if (r < gu_total) {
       const int pr = (int)(r / gu_chunks);
-      p = (int)(r % gu_chunks);
-      K = H;
-      src = q + e * 3 * n + (size_t)(pr & 1) * n + (size_t)(pr >> 1) * H;
-      dst = out + e * L.bytes + L.gu_codes + (size_t)pr * L.gu_row_bytes;
+      const int p = (int)(r % gu_chunks);
+      const uint8_t* src = q + e * 3 * n + (size_t)(pr & 1) * n + (size_t)(pr >> 1) * H;
+      dst = out + e * L.bytes + L.gu_codes + (size_t)pr * L.gu_row_bytes + (size_t)p * 16;
+      const int ng = H / 64;
+      int g, h;
+      if (BITS == 2) {
+        g = p;
+        h = 0;
+      } else {
+        const int seg = ng < 32 ? ng : 32;
+        const int s = p / (2 * seg), rem = p % (2 * seg);
+        h = rem / seg;
+        g = s * seg + rem % seg;
+      }
+#pragma unroll
+      for (int w = 0; w < 4; ++w) in[w] = src + g * 64 + h * 32 + w * per_word;  // h is 0 for 2-bit
     } else {
-      r -= (size_t)2 * I * gu_chunks;
-      const int row = (int)(r / dn_chunks);
-      p = (int)(r % dn_chunks);
-      K = I;
-      src = q + e * 3 * n + 2 * n + (size_t)row * I;
-      dst = out + e * L.bytes + L.down_codes + (size_t)row * L.down_row_bytes;
+      r -= gu_total;
+      const int nb = (int)(r / (H / 4)), row0 = (int)(r % (H / 4)) * 4;
+      dst = out + e * L.bytes + L.down_codes + ((size_t)nb * H + row0) * 4;
+#pragma unroll
+      for (int w = 0; w < 4; ++w) in[w] = q + e * 3 * n + 2 * n + (size_t)(row0 + w) * I + (size_t)nb * per_word;
     }
-    const int ng = K / 64;
-    int g, h;
-    if (BITS == 2) {
-      g = p;
-      h = 0;
-    } else {
-      const int seg = ng < 32 ? ng : 32;
-      const int s = p / (2 * seg), rem = p % (2 * seg);
-      h = rem / seg;
-      g = s * seg + rem % seg;
-    }
-    const uint8_t* in = src + g * 64 + h * 32;  // h is 0 for 2-bit
-    constexpr int per_word = 32 / BITS, per_byte = 8 / BITS;
     uint32_t words[4];
     bool bad = false;
 #pragma unroll
@@ -418,14 +411,17 @@ __global__ void pack_codes_kernel(const uint8_t* __restrict__ q, int n_experts, 
       for (int a = 0; a < 4; ++a)
 #pragma unroll
         for (int b = 0; b < per_byte; ++b) {
-          const uint32_t v = in[w * per_word + 4 * b + a];
+          const uint32_t v = in[w][4 * b + a];
           bad |= v >= (1u << BITS);
           word |= (v & ((1u << BITS) - 1u)) << ((per_byte * a + b) * BITS);
         }
-      words[w] = bad ? 0u : word;
+      words[w] = word;
     }
-    if (bad) raise_status(FMOE_STATUS_BAD_PACK_INPUT);
-    *reinterpret_cast<uint4*>(dst + (size_t)p * 16) = make_uint4(words[0], words[1], words[2], words[3]);
+    if (bad) {
+      raise_status(FMOE_STATUS_BAD_PACK_INPUT);
+      words[0] = words[1] = words[2] = words[3] = 0u;
+    }
+    *reinterpret_cast<uint4*>(dst) = make_uint4(words[0], words[1], words[2], words[3]);
   }
 }
 
@@ -446,7 +442,8 @@ __global__ void pack_sb_kernel(const uint16_t* __restrict__ scale, const uint16_
       dst = reinterpret_cast<uint32_t*>(out + e * L.bytes + L.gu_sb) + r;
     } else {
       src = r;
-      dst = reinterpret_cast<uint32_t*>(out + e * L.bytes + L.down_sb) + (r - gu);
+      const size_t gpr = I / 64, rr = r - gu, row = rr / gpr, g = rr % gpr;
+      dst = reinterpret_cast<uint32_t*>(out + e * L.bytes + L.down_sb) + g * H + row;
     }
     const uint16_t sv = scale[e * ng + src], bv = bias[e * ng + src];
     // exact scaling by 2^-shift of a bf16 value (normal, finite, no underflow)
@@ -463,7 +460,7 @@ __global__ void pack_sb_kernel(const uint16_t* __restrict__ scale, const uint16_
 
 // ------------------------------------------------------- host helpers ----
 struct WsLayout {
-  size_t sync, ss, part, logits, ids, weights, gamma, a, y, bytes;
+  size_t sync, ss, fpart, part, logits, ids, weights, gamma, a, y, bytes;
 };
 
 static inline size_t align_up(size_t v, size_t a) { return (v + a - 1) / a * a; }
@@ -472,9 +469,11 @@ constexpr int kMaxSMs = 1024;
 
 static WsLayout ws_layout(int H, int I, int E, int k, int T) {
   WsLayout w;
-  w.sync = 0;    // grid-barrier and a-group publication counters of the fused kernel (1024 words)
+  w.sync = 0;    // grid-barrier counters of the fused kernel
   w.ss = 4096;   // per-CTA partial sums of h'^2
   size_t o = 4096 + (size_t)kMaxSMs * 4;
+  w.fpart = o;   // per-CTA partial outputs of the fused kernel [kFusedMaxCtas][H]
+  o = align_up(o + (size_t)kFusedMaxCtas * H * 4, 256);
   w.part = o;
   o = align_up(o + (size_t)T * (E + 1) * kRouterSplit * 4, 256);
   w.logits = o;
@@ -561,11 +560,9 @@ static int launch_experts(const ExpertSet& es, const float* xn, const int32_t* i
     gateup_kernel<<<dim3(blocks, slots), kThreads, smem, st>>>(es, xn, ids, a, w_sg, gamma);
   }
   {
-    const int ng = es.I / 64, lpr = ng < 32 ? ng : 32;
-    const int units = es.H / (32 / lpr);
-    int blocks = (units + 4 * kWarps - 1) / (4 * kWarps);
+    const int blocks = (es.H + kDownThreads - 1) / kDownThreads;
     const size_t smem = staged_x_bytes(es.I);
-    down_kernel<<<dim3(blocks, slots), kThreads, smem, st>>>(es, ids, a, y);
+    down_kernel<<<dim3(blocks, slots), kDownThreads, smem, st>>>(es, ids, a, y);
   }
   return cuda_rc(cudaGetLastError());
 }
@@ -625,7 +622,8 @@ static FusedConfig fused_config_uncached(const fmoe_layer_desc& d, int dev) {
   int n_sm = 0, optin = 0;
   if (cudaDeviceGetAttribute(&n_sm, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess) return fc;
   if (cudaDeviceGetAttribute(&optin, cudaDevAttrMaxSharedMemoryPerBlockOptin, dev) != cudaSuccess) return fc;
-  if (n_sm < 1 || n_sm > kMaxSMs) return fc;
+  if (n_sm < 1) return fc;
+  if (n_sm > kFusedMaxCtas) n_sm = kFusedMaxCtas;  // one CTA per SM, at most kFusedMaxCtas of them
   const size_t max_dyn = optin > 2048 ? (size_t)optin - 1024 : 0;
   if (!fused_plan(d.hidden, d.inter, d.n_experts, d.top_k, d.bits, d.shared_bits, n_sm, max_dyn, &fc.plan))
     return fc;
@@ -647,58 +645,6 @@ static bool same_desc(const fmoe_layer_desc& a, const fmoe_layer_desc& b) {
          a.bits == b.bits && a.shared_bits == b.shared_bits && a.group == b.group && a.eps == b.eps;
 }
 
-// cuTensorMapEncodeTiled, fetched once through the runtime (no link-time
-// dependency on the driver library).
-static PFN_cuTensorMapEncodeTiled_v12000 tensor_map_encoder() {
-  static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
-  static bool tried = false;
-  if (!tried) {
-    tried = true;
-    void* p = nullptr;
-    cudaDriverEntryPointQueryResult q;
-    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) == cudaSuccess &&
-        q == cudaDriverEntryPointSuccess)
-      fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(p);
-  }
-  return fn;
-}
-
-// Tensor map over [n_mats][rows][words] 32-bit words (row stride row_bytes,
-// matrix stride mat_bytes) whose box is box_words x box_rows x 1: a box wider
-// than a row is zero-filled past the row end.
-static bool encode_rows(CUtensorMap* m, const void* base, uint64_t words, uint64_t rows, uint64_t row_bytes,
-                        uint64_t n_mats, uint64_t mat_bytes, uint32_t box_words, uint32_t box_rows) {
-  PFN_cuTensorMapEncodeTiled_v12000 enc = tensor_map_encoder();
-  if (!enc) return false;
-  const cuuint64_t dims[3] = {words, rows, n_mats};
-  const cuuint64_t strides[2] = {row_bytes, mat_bytes};
-  const cuuint32_t box[3] = {box_words, box_rows, 1};
-  const cuuint32_t es[3] = {1, 1, 1};
-  return enc(m, CU_TENSOR_MAP_DATA_TYPE_UINT32, 3, const_cast<void*>(base), dims, strides, box, es,
-             CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_NONE,
-             CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
-}
-
-// The four down-row tensor maps of one layer (routed codes / scale-bias,
-// shared codes / scale-bias).
-static bool encode_layer_maps(const fmoe_layer_weights& L, const FusedPlan& plan, CUtensorMap* tm) {
-  const fmoe_layer_desc& d = L.desc;
-  const RecordLayout LR = record_layout(d.bits, d.hidden, d.inter);
-  const RecordLayout LS = record_layout(d.shared_bits, d.hidden, d.inter);
-  const uint32_t ngI = (uint32_t)d.inter / 64, rows = plan.nd_box;
-  const uint8_t* ex = static_cast<const uint8_t*>(L.experts);
-  const uint8_t* sh = static_cast<const uint8_t*>(L.shared);
-  return encode_rows(&tm[kTmRoutedCodes], ex + LR.down_codes, LR.down_row_bytes / 4, (uint64_t)d.hidden,
-                     LR.down_row_bytes, (uint64_t)d.n_experts, LR.bytes,
-                     (uint32_t)(LR.down_row_bytes / 4 + kRowPadWords), rows) &&
-         encode_rows(&tm[kTmRoutedSb], ex + LR.down_sb, ngI, (uint64_t)d.hidden, (uint64_t)ngI * 4,
-                     (uint64_t)d.n_experts, LR.bytes, ngI + kRowPadWords, rows) &&
-         encode_rows(&tm[kTmSharedCodes], sh + LS.down_codes, LS.down_row_bytes / 4, (uint64_t)d.hidden,
-                     LS.down_row_bytes, 1, LS.bytes, (uint32_t)(LS.down_row_bytes / 4 + kRowPadWords), rows) &&
-         encode_rows(&tm[kTmSharedSb], sh + LS.down_sb, ngI, (uint64_t)d.hidden, (uint64_t)ngI * 4, 1, LS.bytes,
-                     ngI + kRowPadWords, rows);
-}
-
 // Runs n_layers layers (T = 1) with the persistent kernel.  Returns
 // FMOE_ERR_UNSUPPORTED when the configuration does not fit it.
 static int launch_fused(const fmoe_layer_weights* layers, int n_layers, float* h, float* xn, void* ws,
@@ -709,14 +655,12 @@ static int launch_fused(const fmoe_layer_weights* layers, int n_layers, float* h
   const WsLayout w = ws_layout(d.hidden, d.inter, d.n_experts, d.top_k, 1);
   if (ws_bytes < w.bytes) return FMOE_ERR_BUFFER_TOO_SMALL;
   unsigned char* base = static_cast<unsigned char*>(ws);
-  thread_local FusedArgs args;  // 16 KB of tensor maps: not on the stack
+  FusedArgs args;
   std::memset(&args, 0, sizeof(args));
   args.H = d.hidden;
   args.I = d.inter;
   args.E = d.n_experts;
   args.k = d.top_k;
-  args.bits = d.bits;
-  args.sbits = d.shared_bits;
   args.eps = d.eps;
   args.h = h;
   args.xn = xn;
@@ -725,8 +669,8 @@ static int launch_fused(const fmoe_layer_weights* layers, int n_layers, float* h
   args.weights = reinterpret_cast<float*>(base + w.weights);
   args.gamma = reinterpret_cast<float*>(base + w.gamma);
   args.a = reinterpret_cast<float*>(base + w.a);
-  args.y = reinterpret_cast<float*>(base + w.y);
   args.ss_part = reinterpret_cast<float*>(base + w.ss);
+  args.part = reinterpret_cast<float*>(base + w.fpart);
   args.sync = reinterpret_cast<unsigned*>(base + w.sync);
   args.plan = fc.plan;
   for (int l0 = 0; l0 < n_layers; l0 += kFusedMaxLayers) {
@@ -739,7 +683,6 @@ static int launch_fused(const fmoe_layer_weights* layers, int n_layers, float* h
       args.layers[l].w_router = L.w_router;
       args.layers[l].w_sg = L.w_shared_gate;
       args.layers[l].norm_w = L.norm_w;
-      if (!encode_layer_maps(L, fc.plan, args.tm[l])) return FMOE_ERR_UNSUPPORTED;
     }
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = dim3(fc.n_sm);
@@ -927,6 +870,11 @@ extern "C" int fmoe_pack_experts_device(const uint8_t* d_q, const uint16_t* d_sc
   return cuda_rc(cudaGetLastError());
 }
 
+extern "C" int fmoe_fused_supported(const fmoe_layer_desc* d) {
+  if (!desc_valid(d) || !desc_supported(d)) return 0;
+  return fused_config(*d).ok ? 1 : 0;
+}
+
 extern "C" int fmoe_set_fused(int enable) {
   const int prev = g_fused_enabled;
   g_fused_enabled = enable ? 1 : 0;
@@ -963,7 +911,7 @@ extern "C" int fmoe_stack_forward(const fmoe_layer_weights* layers, int n_layers
 // when the module loads, so that the call itself reserves no memory.
 namespace fmoe {
 
-constexpr size_t kStaticScratchBytes = size_t(8) << 20;  // 8 MiB: T <= 74 at 4096 x 1024 x 512 experts, top-4
+constexpr size_t kStaticScratchBytes = size_t(12) << 20;  // 12 MiB: T <= 88 at 4096 x 1024 x 512 experts, top-4
 constexpr size_t kStaticCounterBytes = 4096;             // the counter words at the start of the layout
 constexpr int kStaticMaxDevices = 64;
 

@@ -2,11 +2,14 @@
 //
 // One record per expert, sections 16-byte aligned:
 //   [gate/up codes: I row pairs x 2 rows x H*bits/8 bytes]
-//   [down codes:    H rows x I*bits/8 bytes]
+//   [down codes:    I*bits/32 column blocks x H rows x one 32-bit word]
 //   [gate/up scale-bias: I x 2 rows x H/64 words]
-//   [down scale-bias:    H rows x I/64 words]
-// The per-row chunk order and the code permutation inside a word are
-// described in include/fmoe.h.
+//   [down scale-bias:    I/64 groups x H rows x one word]
+// Gate/up rows are stored row by row (one row pair gives g_n and u_n); the
+// down matrix column block by column block, so that the codes of any run of
+// 8 (4-bit) or 16 (2-bit) consecutive intermediate units for every hidden
+// row are one contiguous range.  The per-row chunk order and the code
+// permutation inside a word are described in include/fmoe.h.
 #pragma once
 
 #include <stddef.h>
@@ -22,7 +25,7 @@ namespace fmoe {
 
 struct RecordLayout {
   size_t gu_row_bytes;    // bytes of one gate or up row (H codes)
-  size_t down_row_bytes;  // bytes of one down row (I codes)
+  size_t down_row_bytes;  // bytes of one down row's codes (I codes), spread over the column blocks
   size_t gu_codes;        // offsets of the four sections
   size_t down_codes;
   size_t gu_sb;

@@ -54,26 +54,34 @@ static inline size_t chunk_offset(int bits, int K, int g, int half) {
   return (size_t)s * seg * 32 + (size_t)half * seg * 16 + (size_t)gi * 16;
 }
 
+// One 32-bit word of codes for 32 / bits consecutive inputs src[0 ..):
+// field per_byte * a + b (bits wide) holds input 4 b + a, so that masking the
+// word leaves byte lanes that pair with consecutive inputs.
+static uint32_t pack_word(int bits, const uint8_t* src) {
+  const int per_byte = 8 / bits;  // 2 or 4
+  uint32_t word = 0;
+  for (int a = 0; a < 4; ++a)
+    for (int b = 0; b < per_byte; ++b) word |= (uint32_t)src[4 * b + a] << ((per_byte * a + b) * bits);
+  return word;
+}
+
+static void unpack_word(int bits, uint32_t word, uint8_t* out) {
+  const int per_byte = 8 / bits;
+  const uint32_t mask = (1u << bits) - 1u;
+  for (int a = 0; a < 4; ++a)
+    for (int b = 0; b < per_byte; ++b) out[4 * b + a] = (uint8_t)((word >> ((per_byte * a + b) * bits)) & mask);
+}
+
 // Packs one logical row (K codes) into `dst` (K * bits / 8 bytes).
 static void pack_row(int bits, int K, const uint8_t* q, uint8_t* dst) {
   const int ng = K / 64;
   const int per_chunk = 128 / bits;   // inputs per 16-byte chunk: 32 or 64
   const int per_word = 32 / bits;     // inputs per 32-bit word: 8 or 16
-  const int per_byte = 8 / bits;      // 2 or 4
   for (int g = 0; g < ng; ++g) {
     for (int half = 0; half < 64 / per_chunk; ++half) {
       uint32_t words[4];
       const uint8_t* src = q + (size_t)g * 64 + (size_t)half * per_chunk;
-      for (int w = 0; w < 4; ++w) {
-        uint32_t word = 0;
-        for (int a = 0; a < 4; ++a)
-          for (int b = 0; b < per_byte; ++b) {
-            const int field = per_byte * a + b;  // bit position field * bits
-            const int input = 4 * b + a;         // input index within the word
-            word |= (uint32_t)src[w * per_word + input] << (field * bits);
-          }
-        words[w] = word;
-      }
+      for (int w = 0; w < 4; ++w) words[w] = pack_word(bits, src + w * per_word);
       std::memcpy(dst + chunk_offset(bits, K, g, half), words, 16);
     }
   }
@@ -81,19 +89,13 @@ static void pack_row(int bits, int K, const uint8_t* q, uint8_t* dst) {
 
 static void unpack_row(int bits, int K, const uint8_t* src, uint8_t* q) {
   const int ng = K / 64;
-  const int per_chunk = 128 / bits, per_word = 32 / bits, per_byte = 8 / bits;
-  const uint32_t mask = (1u << bits) - 1u;
+  const int per_chunk = 128 / bits, per_word = 32 / bits;
   for (int g = 0; g < ng; ++g)
     for (int half = 0; half < 64 / per_chunk; ++half) {
       uint32_t words[4];
       std::memcpy(words, src + chunk_offset(bits, K, g, half), 16);
       uint8_t* out = q + (size_t)g * 64 + (size_t)half * per_chunk;
-      for (int w = 0; w < 4; ++w)
-        for (int a = 0; a < 4; ++a)
-          for (int b = 0; b < per_byte; ++b) {
-            const int field = per_byte * a + b;
-            out[w * per_word + 4 * b + a] = (uint8_t)((words[w] >> (field * bits)) & mask);
-          }
+      for (int w = 0; w < 4; ++w) unpack_word(bits, words[w], out + w * per_word);
     }
 }
 
@@ -118,14 +120,19 @@ static int pack_expert(int bits, int H, int I, const uint8_t* q, const uint16_t*
         sb[g] = (uint32_t)s | ((uint32_t)bi[m * ng + (size_t)r * gpr + g] << 16);
       }
     }
+  // down matrix, column-block major: word (nb, r) holds inputs
+  // [nb * per_word, (nb + 1) * per_word) of row r; scale-bias word (g, r)
+  const int per_word = 32 / bits;
+  uint32_t* dw = reinterpret_cast<uint32_t*>(dst + L.down_codes);
+  uint32_t* dsb = reinterpret_cast<uint32_t*>(dst + L.down_sb);
+  const size_t gpr = (size_t)I / 64;
   for (int r = 0; r < H; ++r) {
-    pack_row(bits, I, q + 2 * n + (size_t)r * I, dst + L.down_codes + (size_t)r * L.down_row_bytes);
-    const size_t gpr = (size_t)I / 64;
-    uint32_t* sb = reinterpret_cast<uint32_t*>(dst + L.down_sb) + (size_t)r * gpr;
+    const uint8_t* qr = q + 2 * n + (size_t)r * I;
+    for (int nb = 0; nb < I / per_word; ++nb) dw[(size_t)nb * H + r] = pack_word(bits, qr + (size_t)nb * per_word);
     for (size_t g = 0; g < gpr; ++g) {
       uint16_t s;
       if (!bf16_scale_pow2(sc[2 * ng + (size_t)r * gpr + g], shift, &s)) return FMOE_ERR_INVALID_ARG;
-      sb[g] = (uint32_t)s | ((uint32_t)bi[2 * ng + (size_t)r * gpr + g] << 16);
+      dsb[g * H + r] = (uint32_t)s | ((uint32_t)bi[2 * ng + (size_t)r * gpr + g] << 16);
     }
   }
   return FMOE_OK;
@@ -147,14 +154,18 @@ static int unpack_expert(int bits, int H, int I, const uint8_t* src, uint8_t* q,
         bi[m * ng + (size_t)r * gpr + g] = (uint16_t)(sb[g] >> 16);
       }
     }
+  const int per_word = 32 / bits;
+  const uint32_t* dw = reinterpret_cast<const uint32_t*>(src + L.down_codes);
+  const uint32_t* dsb = reinterpret_cast<const uint32_t*>(src + L.down_sb);
+  const size_t gpr = (size_t)I / 64;
   for (int r = 0; r < H; ++r) {
-    unpack_row(bits, I, src + L.down_codes + (size_t)r * L.down_row_bytes, q + 2 * n + (size_t)r * I);
-    const size_t gpr = (size_t)I / 64;
-    const uint32_t* sb = reinterpret_cast<const uint32_t*>(src + L.down_sb) + (size_t)r * gpr;
+    uint8_t* qr = q + 2 * n + (size_t)r * I;
+    for (int nb = 0; nb < I / per_word; ++nb) unpack_word(bits, dw[(size_t)nb * H + r], qr + (size_t)nb * per_word);
     for (size_t g = 0; g < gpr; ++g) {
-      if (!bf16_unscale_pow2((uint16_t)(sb[g] & 0xFFFFu), shift, &sc[2 * ng + (size_t)r * gpr + g]))
+      const uint32_t w = dsb[g * H + r];
+      if (!bf16_unscale_pow2((uint16_t)(w & 0xFFFFu), shift, &sc[2 * ng + (size_t)r * gpr + g]))
         return FMOE_ERR_INVALID_ARG;
-      bi[2 * ng + (size_t)r * gpr + g] = (uint16_t)(sb[g] >> 16);
+      bi[2 * ng + (size_t)r * gpr + g] = (uint16_t)(w >> 16);
     }
   }
   return FMOE_OK;

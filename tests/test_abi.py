@@ -99,6 +99,35 @@ def test_packed_word_permutation(fm):
     assert int(packed[sb_off:sb_off + 4].view(np.uint32)[0]) & 0xFFFF == 0x3D80
 
 
+@pytest.mark.parametrize("bits", [4, 2])
+def test_packed_down_column_blocks(fm, bits):
+    """Down codes are stored column block by column block: the word at
+    (block nb, row r) holds inputs nb*w .. nb*w + w - 1 of down row r (w = 32 /
+    bits) in the documented field order; down scale-bias words are group-major."""
+    H, I = 128, 128
+    n, ng = H * I, H * I // 64
+    rng = np.random.default_rng(bits)
+    q = rng.integers(0, 1 << bits, size=3 * n, dtype=np.uint8)
+    s = np.full(3 * ng, 0x3F80, np.uint16)
+    b = rng.integers(0, 1 << 15, size=3 * ng).astype(np.uint16)
+    packed = fm.fmoe_pack_experts_host(q, s, b, bits, 1, H, I)
+    w, per_byte = 32 // bits, 8 // bits
+    down_codes = 2 * I * H * bits // 8
+    words = packed[down_codes:down_codes + H * I * bits // 8].view(np.uint32)
+    qd = q[2 * n:].reshape(H, I)
+    for nb, r in [(0, 0), (1, 5), (I // w - 1, H - 1), (3, 77)]:
+        word = int(words[nb * H + r])
+        for a in range(4):
+            for bb in range(per_byte):
+                field = (word >> (bits * (per_byte * a + bb))) & ((1 << bits) - 1)
+                assert field == qd[r, nb * w + 4 * bb + a]
+    sb_off = down_codes + H * I * bits // 8 + 2 * I * (H // 64) * 4
+    sbw = packed[sb_off:sb_off + H * (I // 64) * 4].view(np.uint32)
+    bd = b[2 * ng:].reshape(H, I // 64)
+    for g, r in [(0, 0), (1, 3), (I // 64 - 1, H - 1)]:
+        assert int(sbw[g * H + r]) >> 16 == bd[r, g]
+
+
 def test_packer_rejects_bad_input(fm):
     H, I = 64, 64
     n, ng = 3 * H * I, 3 * H * I // 64

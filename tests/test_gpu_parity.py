@@ -59,13 +59,24 @@ def device_layer(wl, layer=0):
     return _layers[key]
 
 
+def fused_on():
+    prev = fm.fmoe_set_fused(True)
+    fm.fmoe_set_fused(prev)
+    return prev
+
+
 def check_layer_token(wl, lw_o, ws, desc, T, t, h_in, xn_in, h_out, xn_out, label, logits_given=False):
     """Teacher-forced check of token t of one layer step: routing on the
     device's fp32 logits (the router product is checked too unless the
-    logits were given), then y, h', xn' against the oracle."""
+    logits were given), then each expert's SwiGLU outputs a, the expert
+    outputs y (left in the workspace by the one-kernel-per-step path only;
+    the persistent kernel sums them on the fly), h' and xn' against the
+    oracle."""
+    fused = T == 1 and not logits_given and fused_on() and fm.fmoe_fused_supported(desc)
     lg_d = host(fm.workspace_view(ws, desc, T, fm.WS_LOGITS))[t]
     ids_d = host(fm.workspace_view(ws, desc, T, fm.WS_IDS))[t]
     p_d = host(fm.workspace_view(ws, desc, T, fm.WS_WEIGHTS))[t]
+    a_d = host(fm.workspace_view(ws, desc, T, fm.WS_A))[t]
     y_d = host(fm.workspace_view(ws, desc, T, fm.WS_Y))[t]
     gamma_d = host(fm.workspace_view(ws, desc, T, fm.WS_GAMMA))[t]
     if not logits_given:
@@ -77,7 +88,11 @@ def check_layer_token(wl, lw_o, ws, desc, T, t, h_in, xn_in, h_out, xn_out, labe
     assert ref["ids"].tolist() == ids_d.tolist(), f"{label} ids {ids_d} vs oracle {ref['ids']}"
     check(p_d, ref["p"], ref["p"], f"{label} gate weights")
     check(gamma_d, ref["gamma"], ref["gamma"] + ref["S_gamma"], f"{label} gamma")
-    check(y_d, ref["y"], ref["S_y"], f"{label} y")
+    for j, slot in enumerate(list(ids_d) + [wl.n_experts]):
+        e = oracle.expert_ffn(lw_o.experts[int(slot)], wl.hidden, wl.inter, wl.group, xn_in)
+        check(a_d[j], e["a"], e["S_a"], f"{label} a[{j}]")
+    if not fused:
+        check(y_d, ref["y"], ref["S_y"], f"{label} y")
     check(h_out, ref["h"], ref["S_h"], f"{label} h'")
     check(xn_out, ref["xn"], ref["S_xn"], f"{label} xn'")
     return ref
@@ -285,6 +300,11 @@ def test_layer_forward_full_size_int2(wl, path):
 
 
 def test_fused_and_per_step_paths_agree(full_layer):
+    """The persistent kernel and the one-kernel-per-step path route alike and
+    agree to well inside the oracle tolerance.  They are not bit-identical:
+    the persistent kernel rounds the SwiGLU outputs to 16-bit fixed point
+    per column block of 8 units, the per-step path per 64-group, and it sums
+    the expert outputs in another order."""
     wl, lw, _ = full_layer
     x = synth.tokens(wl, 1, stream=35)
     outs = {}
@@ -293,12 +313,13 @@ def test_fused_and_per_step_paths_agree(full_layer):
         h, xn = dev(x), dev(x)
         ws = fm.alloc_workspace(lw.desc, 1)
         fm.fmoe_layer_forward(lw, h, xn, ws)
-        outs[fused] = (host(h)[0], host(xn)[0], host(fm.workspace_view(ws, lw.desc, 1, fm.WS_IDS))[0])
+        outs[fused] = (host(h)[0], host(xn)[0], host(fm.workspace_view(ws, lw.desc, 1, fm.WS_A))[0],
+                       host(fm.workspace_view(ws, lw.desc, 1, fm.WS_IDS))[0])
         fm.fmoe_set_fused(prev)
-    assert outs[True][2].tolist() == outs[False][2].tolist()
-    for i in range(2):
+    assert outs[True][3].tolist() == outs[False][3].tolist()
+    for i in range(3):
         a, b = outs[True][i], outs[False][i]
-        assert np.linalg.norm(a - b) / np.linalg.norm(b) < 1e-5
+        assert np.linalg.norm(a - b) / np.linalg.norm(b) < 2e-4, i
 
 
 def test_layer_forward_is_deterministic_and_graph_capturable(full_layer):
