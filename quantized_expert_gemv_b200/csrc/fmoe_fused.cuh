@@ -231,90 +231,133 @@ struct BlockGeo {
 
 // Block state shared by the threads of a CTA.
 struct BlockShared {
-  float gu[kFusedWarps][2];  // per-warp partial gate / up sums
-  uint32_t xi[8];            // the block's SwiGLU outputs as int16 pairs
-  float dq[2];               // weight * delta, weight * delta * sum(xi)
+  float gu[kFusedWarps][4][2];  // per warp, per pair of the thread set: partial gate / up sums
 };
 
-// One column block held in `slot`: gate/up of its w row pairs (x staged in
-// sx), SwiGLU, the w outputs quantised to 16-bit fixed point, then the
-// block's down columns for every hidden row this thread owns, scaled by
-// `weight` and added to y.  a_out (global) receives the w SwiGLU outputs.
-// Three block-wide barriers; the slot may be refilled after the last.
-template <int B>
-__device__ __forceinline__ void run_block(const uint8_t* slot, const uint32_t* dsb, int H, const StagedX& sx,
-                                          float weight, float* __restrict__ a_out, BlockShared& bs,
-                                          float (&y)[kFusedRowsPerThread]) {
+// The staged inputs of one 64-group, kept in registers for the whole layer:
+// thread t serves group t % 64 of every gate/up row it touches.
+struct XGroup {
+  uint4 xv[8];
+  float delta, xsum;
+};
+
+__device__ __forceinline__ XGroup load_xgroup(const StagedX& sx, int ngH) {
+  XGroup x;
+  const int g = threadIdx.x & 63;
+  if (g < ngH) {
+    lds_xv(sx, ngH, g, x.xv);
+    x.delta = sx.delta[g];
+    x.xsum = sx.xsum[g];
+  } else {
+#pragma unroll
+    for (int u = 0; u < 8; ++u) x.xv[u] = make_uint4(0u, 0u, 0u, 0u);
+    x.delta = x.xsum = 0.f;
+  }
+  return x;
+}
+
+// One or two column blocks (NB), block n held in slots[n]: gate/up of
+// their w row pairs each, SwiGLU, each block's w outputs rounded to 16-bit
+// fixed point with its own step, then the blocks' down columns for every
+// hidden row this thread owns, block n scaled by weight[n], added to y.
+// Thread t works on group t % 64 of pairs t / 64 + 8 i (pair p = block
+// p / w, row pair p % w of it); every warp then forms all the blocks'
+// outputs itself from the per-warp sums, so one block-wide barrier separates
+// the two halves.  a_out[n] (global) receives block n's w SwiGLU outputs.
+// The slots may be refilled after the closing barrier.
+template <int B, int NB>
+__device__ __forceinline__ void run_blocks(const uint8_t* const (&slots)[2], const uint32_t* const (&dsb)[2], int H,
+                                           const XGroup& xg, const float (&weight)[2], float* const (&a_out)[2],
+                                           BlockShared& bs, float (&y)[kFusedRowsPerThread]) {
   using G = BlockGeo<B>;
+  constexpr int kW = G::kW;
+  constexpr int kNP = NB * kW;   // row pairs: 8, 16 or 32
+  constexpr int kPP = kNP / 8;   // pairs per thread
+  static_assert(kNP <= 32 && kPP <= 4, "one warp forms all outputs");
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   const int ngH = H / 64;
+  const int g = tid & 63, ps = tid >> 6;
   {
-    const int p = tid / G::kTpp, lp = tid % G::kTpp;
     const uint32_t rb = (uint32_t)H * B / 8;
-    const uint8_t* rg = slot + (size_t)(2 * p) * rb;
-    const uint8_t* ru = rg + rb;
-    const uint32_t* sbg = reinterpret_cast<const uint32_t*>(slot + G::gu_codes(H) + G::dn_codes(H)) + 2 * p * ngH;
-    const uint32_t* sbu = sbg + ngH;
-    float g = 0.f, u = 0.f;
-    for (int gi = lp; gi < ngH; gi += G::kTpp) {
-      const GroupCodes<B> cg = lds_group<B>(rg, ngH, gi);
-      const GroupCodes<B> cu = lds_group<B>(ru, ngH, gi);
-      uint4 xv[8];
-      lds_xv(sx, ngH, gi, xv);
-      const float d = sx.delta[gi], xsm = sx.xsum[gi];
-      g = group_epilogue(g, sbg[gi], group_dot<B>(cg, xv), d, xsm);
-      u = group_epilogue(u, sbu[gi], group_dot<B>(cu, xv), d, xsm);
-    }
-    g = warp_sum(g);
-    u = warp_sum(u);
-    if (lane == 0) {
-      bs.gu[warp][0] = g;
-      bs.gu[warp][1] = u;
-    }
-  }
-  __syncthreads();
-  if (warp == 0) {
-    // SwiGLU of the block's w pairs (pair p's sums come from warps
-    // p * kTpp / 32 ..), then one fixed-point step for the block
-    constexpr int kWpp = G::kTpp / 32;
-    float a = 0.f;
-    if (lane < G::kW) {
-      float gg = 0.f, uu = 0.f;
+    float gs[kPP], us[kPP];
 #pragma unroll
-      for (int w = 0; w < kWpp; ++w) {
-        gg += bs.gu[lane * kWpp + w][0];
-        uu += bs.gu[lane * kWpp + w][1];
+    for (int pp = 0; pp < kPP; ++pp) {
+      // pair ps + 8 pp: block (8 pp) / w and row pair ps + 8 (pp % (w / 8)) of it (ps < 8)
+      constexpr int kSub = kW / 8;
+      const int n = (8 * pp) / kW, pl = ps + 8 * (pp % kSub);
+      gs[pp] = us[pp] = 0.f;
+      if (g < ngH) {
+        const uint8_t* rg = slots[n] + (size_t)(2 * pl) * rb;
+        const uint32_t* sbg = reinterpret_cast<const uint32_t*>(slots[n] + G::gu_codes(H) + G::dn_codes(H)) +
+                              2 * pl * ngH;
+        const GroupCodes<B> cg = lds_group<B>(rg, ngH, g);
+        const GroupCodes<B> cu = lds_group<B>(rg + rb, ngH, g);
+        gs[pp] = group_epilogue(0.f, sbg[g], group_dot<B>(cg, xg.xv), xg.delta, xg.xsum);
+        us[pp] = group_epilogue(0.f, sbg[ngH + g], group_dot<B>(cu, xg.xv), xg.delta, xg.xsum);
       }
-      a = silu_mul(gg, uu);
-      a_out[lane] = a;
     }
-    const float m = __uint_as_float(__reduce_max_sync(0xffffffffu, __float_as_uint(fabsf(a))));
-    const float inv = m > 0.f ? 32767.f / m : 0.f;
-    const float delta = m * (1.f / 32767.f);
-    int q = __float2int_rn(a * inv);
-    q = q > 32767 ? 32767 : (q < -32767 ? -32767 : q);
-    const int qsum = __reduce_add_sync(0xffffffffu, q);
-    const int q_hi = __shfl_down_sync(0xffffffffu, q, 1);
-    if (lane < G::kW && (lane & 1) == 0) bs.xi[lane >> 1] = (uint32_t)(q & 0xFFFF) | ((uint32_t)q_hi << 16);
-    if (lane == 0) {
-      bs.dq[0] = weight * delta;
-      bs.dq[1] = weight * delta * (float)qsum;
+#pragma unroll
+    for (int pp = 0; pp < kPP; ++pp) {
+      const float gsum = warp_sum(gs[pp]), usum = warp_sum(us[pp]);
+      if (lane == 0) {
+        bs.gu[warp][pp][0] = gsum;
+        bs.gu[warp][pp][1] = usum;
+      }
     }
   }
   __syncthreads();
+  // every warp: SwiGLU of all pairs (lane l < kNP: pair l, whose sums sit in
+  // warps 2 (l % 8), 2 (l % 8) + 1, slot l / 8), one fixed-point step per
+  // block, the int16 pairs of every block spread to all lanes
+  uint32_t xw[NB][8];
+  float p1[NB], p2[NB];
   {
-    const uint4 x0 = make_uint4(bs.xi[0], bs.xi[1], bs.xi[2], bs.xi[3]);
-    const uint4 x1 = make_uint4(bs.xi[4], bs.xi[5], bs.xi[6], bs.xi[7]);
-    const float p1 = bs.dq[0], p2 = bs.dq[1];
-    const uint32_t* dc = reinterpret_cast<const uint32_t*>(slot + G::gu_codes(H));
+    float a = 0.f;
+    if (lane < kNP) {
+      const int pw = 2 * (lane & 7), pp = lane >> 3;
+      a = silu_mul(bs.gu[pw][pp][0] + bs.gu[pw + 1][pp][0], bs.gu[pw][pp][1] + bs.gu[pw + 1][pp][1]);
+      if (warp == 0) (NB == 2 && lane >= kW ? a_out[NB - 1] : a_out[0])[lane % kW] = a;
+    }
+    const int mine = lane / kW;  // this lane's block (>= NB: none)
+    float delta_m = 0.f;
+#pragma unroll
+    for (int n = 0; n < NB; ++n) {
+      const float m = __uint_as_float(__reduce_max_sync(0xffffffffu, mine == n ? __float_as_uint(fabsf(a)) : 0u));
+      const float delta = m * (1.f / 32767.f);
+      if (mine == n) delta_m = m > 0.f ? 32767.f / m : 0.f;
+      p1[n] = weight[n] * delta;
+    }
+    int q = __float2int_rn(a * delta_m);
+    q = q > 32767 ? 32767 : (q < -32767 ? -32767 : q);
+#pragma unroll
+    for (int n = 0; n < NB; ++n) p2[n] = p1[n] * (float)__reduce_add_sync(0xffffffffu, mine == n ? q : 0);
+    const int q_hi = __shfl_down_sync(0xffffffffu, q, 1);
+    const uint32_t word = (uint32_t)(q & 0xFFFF) | ((uint32_t)q_hi << 16);
+#pragma unroll
+    for (int n = 0; n < NB; ++n) {
+#pragma unroll
+      for (int i = 0; i < 8; ++i) xw[n][i] = i < kW / 2 ? __shfl_sync(0xffffffffu, word, n * kW + 2 * i) : 0u;
+    }
+  }
+  {
+    const uint32_t* dc[NB];
+#pragma unroll
+    for (int n = 0; n < NB; ++n) dc[n] = reinterpret_cast<const uint32_t*>(slots[n] + G::gu_codes(H));
 #pragma unroll
     for (int m = 0; m < kFusedRowsPerThread; ++m) {
       const int i = tid + m * kFusedThreads;
       if (i < H) {
-        const uint32_t w = dc[i], sbw = dsb[i];
-        const int acc = B == 4 ? word_dot4(w, x0) : word_dot2(w, x0, x1);
-        const float s = __uint_as_float(sbw << 16), b = __uint_as_float(sbw & 0xFFFF0000u);
-        y[m] = fmaf(s, p1 * (float)acc, fmaf(b, p2, y[m]));
+        float v = y[m];
+#pragma unroll
+        for (int n = 0; n < NB; ++n) {
+          const uint32_t w = dc[n][i], sbw = dsb[n][i];
+          const int acc = B == 4 ? word_dot4(w, make_uint4(xw[n][0], xw[n][1], xw[n][2], xw[n][3]))
+                                 : word_dot2(w, make_uint4(xw[n][0], xw[n][1], xw[n][2], xw[n][3]),
+                                             make_uint4(xw[n][4], xw[n][5], xw[n][6], xw[n][7]));
+          const float sc = __uint_as_float(sbw << 16), bi = __uint_as_float(sbw & 0xFFFF0000u);
+          v = fmaf(sc, p1[n] * (float)acc, fmaf(bi, p2[n], v));
+        }
+        y[m] = v;
       }
     }
   }
@@ -367,9 +410,10 @@ __global__ void __launch_bounds__(kFusedThreads, 1) fused_stack_kernel(const __g
 
   unsigned bar_target = 0;
   uint32_t phase = 0;  // per mbarrier: parity of its next completion (same in every thread)
-  uint32_t armed = 0;  // thread 0: mbarriers with copies in flight
+  uint32_t armed = 0;  // lane 0 of an issuing warp: its mbarriers with copies in flight
 
-  // ---- copies (thread 0 only) ----
+  // ---- copies (lane 0 of one warp per mbarrier: slot s <- warp s, entry e
+  // <- warp kSlots + e, so each issuer drains its own copies on abort) ----
   auto arm = [&](int mb, uint32_t bytes) {
     mbar_expect_tx(&mbar[mb], bytes);
     armed |= 1u << mb;
@@ -394,19 +438,37 @@ __global__ void __launch_bounds__(kFusedThreads, 1) fused_stack_kernel(const __g
     arm(kMbSb + e, 4u * (uint32_t)H);
     bulk_g2s(smem + P.sbe[e], rec + L.down_sb + (size_t)g * H * 4, 4u * (uint32_t)H, &mbar[kMbSb + e]);
   };
-  auto issue_shared = [&](int l) {  // layer l's shared block -> slot 1, its scale-bias -> entry 0
+  // layer l's shared block -> slot 1 (warp 1), its scale-bias -> entry 0 (warp kSlots); lane 0 only
+  auto issue_shared = [&](int l) {
     if (!has_shared) return;
-    fence_proxy_async();
     const uint8_t* rec = A.layers[l].shared;
-    issue_block(1, rec, LS, c, GS::gu_sb(H));
-    issue_sb(0, rec, LS, c / GS::kPerGroup);
+    if (warp == 1) {
+      fence_proxy_async();
+      issue_block(1, rec, LS, c, GS::gu_sb(H));
+    } else if (warp == kSlots) {
+      fence_proxy_async();
+      issue_sb(0, rec, LS, c / GS::kPerGroup);
+    }
+  };
+
+  // L2 prefetch of layer l's router rows and shared block (any one thread)
+  auto prefetch_next = [&](int l) {
+    const FusedLayer& NX = A.layers[l];
+    for (int m = 0; m < nr; ++m) {
+      const int row = c + m * nC;
+      prefetch_l2(row < E ? NX.w_router + (size_t)row * H : NX.w_sg, 4u * (uint32_t)H);
+    }
+    if (has_shared) {
+      prefetch_block(NX.shared, LS, c, GS::gu_sb(H));
+      prefetch_l2(NX.shared + LS.down_sb + (size_t)(c / GS::kPerGroup) * H * 4, 4u * (uint32_t)H);
+    }
   };
 
   // ---- waits (all threads; the outcome is agreed block-wide) ----
   auto wait_mb = [&](int mb) -> bool {
     const bool ok = mbar_wait(&mbar[mb], (phase >> mb) & 1u);
     phase ^= 1u << mb;
-    if (tid == 0 && ok) armed &= ~(1u << mb);
+    if (lane == 0 && ok) armed &= ~(1u << mb);
     if (__syncthreads_and(ok)) return true;
     if (tid == 0) {
       s_abort = 1;
@@ -455,7 +517,7 @@ __global__ void __launch_bounds__(kFusedThreads, 1) fused_stack_kernel(const __g
     return 1.f / sqrtf(t / (float)H + A.eps);
   };
 
-  if (tid == 0 && A.n_layers > 0) issue_shared(0);
+  if (lane == 0 && A.n_layers > 0) issue_shared(0);
 
   float yr[kFusedRowsPerThread], ys[kFusedRowsPerThread];
   bool aborted = false;
@@ -556,12 +618,16 @@ __global__ void __launch_bounds__(kFusedThreads, 1) fused_stack_kernel(const __g
       else A.gamma[0] = 1.f / (1.f + expf(-v));
     }
     grid_arrive();  // B1: logits written
+    const XGroup xg = load_xgroup(sx, ngH);
     // ------------------------------------------------------------- C --
     // while the other CTAs finish: this CTA's block of the shared expert
     if (has_shared) {
       if (!wait_mb(1) || !wait_mb(kMbSb + 0)) { aborted = true; break; }
-      run_block<SBITS>(smem + P.slot[1], reinterpret_cast<const uint32_t*>(smem + P.sbe[0]), H, sx, 1.f,
-                       A.a + (size_t)k * I + (size_t)c * GS::kW, s_blk, ys);
+      const uint8_t* const sl[2] = {smem + P.slot[1], nullptr};
+      const uint32_t* const sb[2] = {reinterpret_cast<const uint32_t*>(smem + P.sbe[0]), nullptr};
+      const float wt[2] = {1.f, 0.f};
+      float* const ao[2] = {A.a + (size_t)k * I + (size_t)c * GS::kW, nullptr};
+      run_blocks<SBITS, 1>(sl, sb, H, xg, wt, ao, s_blk, ys);
     }
     if (!grid_wait()) { aborted = true; break; }
     // ------------------------------------------------------------- D --
@@ -571,11 +637,13 @@ __global__ void __launch_bounds__(kFusedThreads, 1) fused_stack_kernel(const __g
       uint64_t key[2];
       bool nan_seen = false;
       float lv[2];
+      const float gv = tid == 0 ? ldcg_f(A.gamma) : 0.f;
 #pragma unroll
       for (int i = 0; i < 2; ++i) {
         const int e = tid + i * kFusedThreads;
         lv[i] = e < E ? ldcg_f(A.logits + e) : 0.f;
       }
+      if (tid == 0) s_gamma = gv;
 #pragma unroll
       for (int i = 0; i < 2; ++i) {
         const int e = tid + i * kFusedThreads;
@@ -614,7 +682,6 @@ __global__ void __launch_bounds__(kFusedThreads, 1) fused_stack_kernel(const __g
             A.weights[lane] = s_p[lane];
           }
         }
-        if (lane == 0) s_gamma = ldcg_f(A.gamma);
         if (c == 0 && lane == 0 && nan_seen) raise_status(FMOE_STATUS_NAN_LOGIT);
       }
       __syncthreads();
@@ -624,52 +691,85 @@ __global__ void __launch_bounds__(kFusedThreads, 1) fused_stack_kernel(const __g
     // blocks and of the next layer's router rows and shared block.  A routed
     // block q (= j * NBr + nb) lies in 64-group q / kPerGroup of the
     // concatenated experts.
-    const int key0 = q0 / GR::kPerGroup;
-    if (tid == 0) {
-      fence_proxy_async();
-      for (int b = 0; b < nq; ++b) {
-        const int q = q0 + b, j = q / NBr, nb = q % NBr;
-        const uint8_t* rec = LY.experts + (size_t)s_ids[j] * LR.bytes;
-        if (b < kSlots) issue_block(b, rec, LR, nb, GR::gu_sb(H));
-        else prefetch_block(rec, LR, nb, GR::gu_sb(H));
-        if (b == 0 || q / GR::kPerGroup != (q - 1) / GR::kPerGroup)
-          issue_sb(q / GR::kPerGroup == key0 ? 0 : 1, rec, LR, nb / GR::kPerGroup);
-      }
-      if (l + 1 < A.n_layers) {
-        const FusedLayer& NX = A.layers[l + 1];
-        for (int m = 0; m < nr; ++m) {
-          const int row = c + m * nC;
-          prefetch_l2(row < E ? NX.w_router + (size_t)row * H : NX.w_sg, 4u * (uint32_t)H);
+    // Jobs are spread over the warps' lane 0 so they go out in parallel:
+    // block b < kSlots <- warp b, entry e <- warp kSlots + e, L2 prefetch of
+    // the blocks b >= kSlots <- the following warps.
+    const int key0 = q0 / GR::kPerGroup, key1 = (q1 - 1) / GR::kPerGroup;
+    const int ngI = I / 64;
+    if (lane == 0) {
+      if (warp < kSlots) {
+        if (warp < nq) {
+          const int q = q0 + warp;
+          fence_proxy_async();
+          issue_block(warp, LY.experts + (size_t)s_ids[q / NBr] * LR.bytes, LR, q % NBr, GR::gu_sb(H));
         }
-        if (has_shared) {
-          prefetch_block(NX.shared, LS, c, GS::gu_sb(H));
-          prefetch_l2(NX.shared + LS.down_sb + (size_t)(c / GS::kPerGroup) * H * 4, 4u * (uint32_t)H);
+      } else if (warp < kSlots + kSbEntries) {
+        const int e = warp - kSlots;
+        if (nq > 0 && (e == 0 || key1 != key0)) {
+          const int key = e == 0 ? key0 : key1;
+          fence_proxy_async();
+          issue_sb(e, LY.experts + (size_t)s_ids[key / ngI] * LR.bytes, LR, key % ngI);
+        }
+      } else {
+        for (int b = kSlots + (warp - kSlots - kSbEntries); b < nq; b += kFusedWarps - kSlots - kSbEntries) {
+          const int q = q0 + b;
+          prefetch_block(LY.experts + (size_t)s_ids[q / NBr] * LR.bytes, LR, q % NBr, GR::gu_sb(H));
         }
       }
     }
     // ------------------------------------------------------------- E --
+    // routed blocks two at a time (block b in slot b % kSlots); a freed slot
+    // takes block b + kSlots at once
     {
-      bool sb_ready[kSbEntries] = {false, false};
-      for (int b = 0; b < nq; ++b) {
-        const int q = q0 + b, j = q / NBr, nb = q % NBr;
-        const int s = b % kSlots, e = q / GR::kPerGroup == key0 ? 0 : 1;
-        if (!wait_mb(s)) { aborted = true; break; }
-        if (!sb_ready[e]) {
-          if (!wait_mb(kMbSb + e)) { aborted = true; break; }
-          sb_ready[e] = true;
+      unsigned sb_ready = 0;  // bit e: entry e waited for in this layer
+      for (int b = 0; b < nq; b += 2) {
+        const int nb_round = nq - b >= 2 ? 2 : 1;
+        const uint8_t* sl[2] = {nullptr, nullptr};
+        const uint32_t* sb[2] = {nullptr, nullptr};
+        float wt[2] = {0.f, 0.f};
+        float* ao[2] = {nullptr, nullptr};
+#pragma unroll
+        for (int n = 0; n < 2; ++n) {
+          if (n >= nb_round) break;
+          const int q = q0 + b + n, j = q / NBr, nbk = q % NBr;
+          const int s = (b + n) % kSlots, e = q / GR::kPerGroup == key0 ? 0 : 1;
+          if (!wait_mb(s)) { aborted = true; break; }
+          if (!(sb_ready & (1u << e))) {
+            if (!wait_mb(kMbSb + e)) { aborted = true; break; }
+            sb_ready |= 1u << e;
+          }
+          sl[n] = smem + P.slot[s];
+          sb[n] = reinterpret_cast<const uint32_t*>(smem + P.sbe[e]);
+          wt[n] = s_p[j];
+          ao[n] = A.a + (size_t)j * I + (size_t)nbk * GR::kW;
         }
-        run_block<BITS>(smem + P.slot[s], reinterpret_cast<const uint32_t*>(smem + P.sbe[e]), H, sx, s_p[j],
-                        A.a + (size_t)j * I + (size_t)nb * GR::kW, s_blk, yr);
-        if (tid == 0 && b + kSlots < nq) {  // the slot is free: its next block
-          const int q2 = q + kSlots, j2 = q2 / NBr, nb2 = q2 % NBr;
-          fence_proxy_async();
-          issue_block(s, LY.experts + (size_t)s_ids[j2] * LR.bytes, LR, nb2, GR::gu_sb(H));
+        if (aborted) break;
+        const uint8_t* const slc[2] = {sl[0], sl[1]};
+        const uint32_t* const sbc[2] = {sb[0], sb[1]};
+        const float wtc[2] = {wt[0], wt[1]};
+        float* const aoc[2] = {ao[0], ao[1]};
+        if (nb_round == 2) run_blocks<BITS, 2>(slc, sbc, H, xg, wtc, aoc, s_blk, yr);
+        else run_blocks<BITS, 1>(slc, sbc, H, xg, wtc, aoc, s_blk, yr);
+        // the freed slots take their next blocks
+#pragma unroll
+        for (int n = 0; n < 2; ++n) {
+          if (n >= nb_round) break;
+          const int bb = b + n, s = bb % kSlots;
+          if (warp == s && lane == 0 && bb + kSlots < nq) {
+            const int q2 = q0 + bb + kSlots;
+            fence_proxy_async();
+            issue_block(s, LY.experts + (size_t)s_ids[q2 / NBr] * LR.bytes, LR, q2 % NBr, GR::gu_sb(H));
+          }
         }
+        // once the first round is done, the next layer's router rows and
+        // shared block may compete for HBM
+        if (b == 0 && warp == kFusedWarps - 1 && lane == 0 && l + 1 < A.n_layers) prefetch_next(l + 1);
       }
       if (aborted) break;
+      if (nq == 0 && warp == kFusedWarps - 1 && lane == 0 && l + 1 < A.n_layers) prefetch_next(l + 1);
     }
     // every slot and entry is consumed: the next layer's shared block can come in
-    if (tid == 0 && l + 1 < A.n_layers) issue_shared(l + 1);
+    if (lane == 0 && l + 1 < A.n_layers) issue_shared(l + 1);
     // ------------------------------------------------------------- F --
     {
       const float gm = s_gamma;
@@ -689,9 +789,17 @@ __global__ void __launch_bounds__(kFusedThreads, 1) fused_stack_kernel(const __g
       const int ngr = nd > 0 ? kFusedThreads / nd : 0;
       const int r = nd > 0 ? tid % nd : 0, pg = nd > 0 ? tid / nd : kFusedThreads;
       if (pg < ngr) {
-        float v = 0.f;
-        for (int p = pg; p < nC; p += ngr) v += ldcg_f(A.part + (size_t)p * H + i0 + r);
-        sred[pg * nd + r] = v;
+        constexpr int kLoads = (kFusedMaxCtas * 32 + kFusedThreads - 1) / kFusedThreads;  // ngr >= 512 / 32
+        float v[kLoads];
+#pragma unroll
+        for (int t2 = 0; t2 < kLoads; ++t2) {
+          const int p = pg + t2 * ngr;
+          v[t2] = p < nC ? ldcg_f(A.part + (size_t)p * H + i0 + r) : 0.f;
+        }
+        float acc = 0.f;
+#pragma unroll
+        for (int t2 = 0; t2 < kLoads; ++t2) acc += v[t2];
+        sred[pg * nd + r] = acc;
       }
       __syncthreads();
       float ss = 0.f;
@@ -724,8 +832,8 @@ __global__ void __launch_bounds__(kFusedThreads, 1) fused_stack_kernel(const __g
         __threadfence();
       }
     }
-  } else if (tid == 0) {
-    // drain: wait (bounded) for this CTA's copies still in flight
+  } else if (lane == 0) {
+    // drain: wait (bounded) for this issuer's copies still in flight
     for (int mb = 0; mb < kMbCount; ++mb)
       if (armed & (1u << mb)) (void)mbar_wait(&mbar[mb], (phase >> mb) & 1u);
   }
