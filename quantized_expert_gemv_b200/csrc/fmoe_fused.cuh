@@ -54,6 +54,7 @@ constexpr int kFusedMaxRouterRows = 4;  // router rows (E experts + the shared g
 constexpr int kFusedRowsPerThread = 8;  // hidden rows per thread in the down products: H <= 4096
 constexpr int kFusedMaxRouted = 16;     // routed blocks per CTA
 constexpr int kSlots = 3;
+constexpr int kFirstWave = 2;  // routed blocks requested at the top-k; the rest after they land
 constexpr int kSbEntries = 2;
 constexpr int kMbSb = kSlots;  // mbarriers: the slots, then the scale-bias entries
 constexpr int kMbCount = kSlots + kSbEntries;
@@ -93,10 +94,14 @@ struct FusedArgs {
   int32_t* ids;
   float* weights;
   float* gamma;
-  float* a;        // [(k+1)][I], shared expert last
-  float* ss_part;  // [gridDim.x]
-  float* part;     // [gridDim.x][H] partial outputs
-  unsigned* sync;  // [0] barrier arrivals, [1] exits
+  float* a;          // [(k+1)][I], shared expert last
+  // exchange words between CTAs: (epoch << 32) | fp32 bits, written and read
+  // as single 64-bit accesses, so a reader that sees the epoch it waits for
+  // holds the value that came with it (no separate flag or barrier)
+  uint64_t* x_logit;  // [E + 1]: router logits, then sigmoid(w_sg . xn)
+  uint64_t* x_part;   // [gridDim.x][H]: partial outputs
+  float* ss_part;     // [gridDim.x]: partial sums of h'^2 (behind the grid barrier)
+  unsigned* sync;     // [0] grid-barrier arrivals, [1] exits, [2] epoch of the last launch
   FusedPlan plan;
 };
 
@@ -160,6 +165,58 @@ __device__ __forceinline__ float ldcg_f(const float* p) { return __ldcg(p); }
 
 __device__ __forceinline__ float4 as_float4(uint4 v) {
   return make_float4(__uint_as_float(v.x), __uint_as_float(v.y), __uint_as_float(v.z), __uint_as_float(v.w));
+}
+
+__device__ __forceinline__ uint64_t ld_relaxed64(const uint64_t* p) {
+  uint64_t v;
+  asm volatile("ld.relaxed.gpu.global.b64 %0, [%1];" : "=l"(v) : "l"(p) : "memory");
+  return v;
+}
+
+__device__ __forceinline__ void st_relaxed64(uint64_t* p, uint64_t v) {
+  asm volatile("st.relaxed.gpu.global.b64 [%0], %1;" ::"l"(p), "l"(v) : "memory");
+}
+
+__device__ __forceinline__ uint64_t x_word(uint32_t epoch, float v) {
+  return ((uint64_t)epoch << 32) | __float_as_uint(v);
+}
+
+__device__ __forceinline__ bool x_ready(uint64_t w, uint32_t epoch) { return (uint32_t)(w >> 32) == epoch; }
+
+// Re-reads *p until it carries `epoch` (bounded); false on expiry.
+__device__ __forceinline__ bool x_spin(const uint64_t* p, uint32_t epoch, uint64_t* w) {
+  if (x_ready(*w, epoch)) return true;
+  const long long t0 = clock64();
+  while (clock64() - t0 < kWaitCycles) {
+    *w = ld_relaxed64(p);
+    if (x_ready(*w, epoch)) return true;
+  }
+  return false;
+}
+
+// N exchange words at p(i) (those with valid(i)): re-reads, all in one round
+// trip per pass, the ones that do not yet carry `epoch` (bounded).
+// While words are missing, only the first missing one is polled; once it
+// has arrived, the others are re-read together.
+template <int N, class Addr, class Valid>
+__device__ __forceinline__ bool x_spin_all(uint64_t (&w)[N], uint32_t epoch, Addr p, Valid valid) {
+  const long long t0 = clock64();
+  while (true) {
+    int miss = -1;
+#pragma unroll
+    for (int i = N - 1; i >= 0; --i)
+      if (valid(i) && !x_ready(w[i], epoch)) miss = i;
+    if (miss < 0) return true;
+    if (clock64() - t0 > kWaitCycles) return false;
+    uint64_t v = ld_relaxed64(p(miss));
+    while (!x_ready(v, epoch)) {
+      if (clock64() - t0 > kWaitCycles) return false;
+      v = ld_relaxed64(p(miss));
+    }
+#pragma unroll
+    for (int i = 0; i < N; ++i)
+      if (valid(i) && !x_ready(w[i], epoch)) w[i] = i == miss ? v : ld_relaxed64(p(i));
+  }
 }
 
 // [lo, hi) share of `total` items for part `c` of `n`
@@ -370,7 +427,6 @@ __global__ void __launch_bounds__(kFusedThreads, 1) fused_stack_kernel(const __g
   using GR = BlockGeo<BITS>;
   using GS = BlockGeo<SBITS>;
   extern __shared__ __align__(128) unsigned char smem[];
-  __shared__ int s_abort;
   __shared__ int s_ids[kFusedMaxK];
   __shared__ float s_p[kFusedMaxK];
   __shared__ float s_gamma;
@@ -402,13 +458,11 @@ __global__ void __launch_bounds__(kFusedThreads, 1) fused_stack_kernel(const __g
   const bool xthr = tid * 8 < H;  // this thread holds inputs 8 tid .. 8 tid + 7
 
   if (tid == 0) {
-    s_abort = 0;
     for (int i = 0; i < kMbCount; ++i) mbar_init(&mbar[i], 1);
     asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
   }
   __syncthreads();
 
-  unsigned bar_target = 0;
   uint32_t phase = 0;  // per mbarrier: parity of its next completion (same in every thread)
   uint32_t armed = 0;  // lane 0 of an issuing warp: its mbarriers with copies in flight
 
@@ -470,23 +524,29 @@ __global__ void __launch_bounds__(kFusedThreads, 1) fused_stack_kernel(const __g
     phase ^= 1u << mb;
     if (lane == 0 && ok) armed &= ~(1u << mb);
     if (__syncthreads_and(ok)) return true;
-    if (tid == 0) {
-      s_abort = 1;
-      raise_status(FMOE_STATUS_WAIT_TIMEOUT);
-    }
+    if (tid == 0) raise_status(FMOE_STATUS_WAIT_TIMEOUT);
     return false;
   };
 
-  // split grid barrier: arrive once this CTA's results are written, do local
-  // work, then wait (release/acquire on one counter, bounded spin)
+  // block-wide agreement after a round of exchange reads
+  auto x_agree = [&](bool ok) -> bool {
+    if (__syncthreads_and(ok)) return true;
+    if (tid == 0) raise_status(FMOE_STATUS_WAIT_TIMEOUT);
+    return false;
+  };
+  // grid barrier after h' (every CTA needs all of it): arrive once this
+  // CTA's rows are written, wait at the start of the next layer
+  // (release/acquire on one counter, bounded spin)
+  unsigned bar_target = 0;
   auto grid_arrive = [&]() {
     __syncthreads();
     bar_target += (unsigned)nC;
     if (tid == 0) asm volatile("red.release.gpu.global.add.u32 [%0], 1;" ::"l"(A.sync) : "memory");
   };
   auto grid_wait = [&]() -> bool {
+    bool ok = true;
     if (tid == 0) {
-      bool ok = false;
+      ok = false;
       const long long t0 = clock64();
       while (true) {
         unsigned v;
@@ -494,17 +554,11 @@ __global__ void __launch_bounds__(kFusedThreads, 1) fused_stack_kernel(const __g
         if (v >= bar_target) { ok = true; break; }
         if (clock64() - t0 > kWaitCycles) break;
       }
-      if (!ok) {
-        s_abort = 1;
-        raise_status(FMOE_STATUS_WAIT_TIMEOUT);
-      }
     }
-    __syncthreads();
-    return !s_abort;
+    return x_agree(ok);
   };
-
-  // r = (sum of the CTAs' partial sums of h'^2 / H + eps)^(-1/2), the same
-  // summation order in every CTA; all threads take part
+  // r = (sum of the CTAs' partial sums of h'^2 / H + eps)^(-1/2), summed in
+  // the same order in every CTA (after the grid barrier)
   auto norm_scale = [&]() -> float {
     float v = tid < nC ? ldcg_f(A.ss_part + tid) : 0.f;
     v = warp_sum(v);
@@ -512,11 +566,12 @@ __global__ void __launch_bounds__(kFusedThreads, 1) fused_stack_kernel(const __g
     __syncthreads();
     float t = 0.f;
 #pragma unroll
-    for (int w = 0; w < kFusedWarps; ++w) t += s_red[w];
+    for (int wi = 0; wi < kFusedWarps; ++wi) t += s_red[wi];
     __syncthreads();
     return 1.f / sqrtf(t / (float)H + A.eps);
   };
 
+  const uint32_t base = __ldcg(A.sync + 2);  // epochs of this launch: base + 2 l + 1, base + 2 l + 2
   if (lane == 0 && A.n_layers > 0) issue_shared(0);
 
   float yr[kFusedRowsPerThread], ys[kFusedRowsPerThread];
@@ -549,7 +604,7 @@ __global__ void __launch_bounds__(kFusedThreads, 1) fused_stack_kernel(const __g
       xv[0] = v0.x; xv[1] = v0.y; xv[2] = v0.z; xv[3] = v0.w;
       xv[4] = v1.x; xv[5] = v1.y; xv[6] = v1.z; xv[7] = v1.w;
     } else {
-      if (!grid_wait()) { aborted = true; break; }  // B3 of the previous layer
+      if (!grid_wait()) { aborted = true; break; }  // h' of the previous layer written
       float4 h0 = make_float4(0.f, 0.f, 0.f, 0.f), h1 = h0, w0 = h0, w1 = h0;
       const float* wprev = A.layers[l - 1].norm_w;
       if (xthr) {
@@ -562,6 +617,7 @@ __global__ void __launch_bounds__(kFusedThreads, 1) fused_stack_kernel(const __g
       xv[0] = h0.x * r * w0.x; xv[1] = h0.y * r * w0.y; xv[2] = h0.z * r * w0.z; xv[3] = h0.w * r * w0.w;
       xv[4] = h1.x * r * w1.x; xv[5] = h1.y * r * w1.y; xv[6] = h1.z * r * w1.z; xv[7] = h1.w * r * w1.w;
     }
+    const uint32_t e_logit = base + 2u * (uint32_t)l + 1u, e_part = e_logit + 1u;
     // stage x: 8 consecutive threads share one 64-group
     {
       float m = 0.f;
@@ -615,9 +671,9 @@ __global__ void __launch_bounds__(kFusedThreads, 1) fused_stack_kernel(const __g
       for (int w = 0; w < kFusedWarps; ++w) v += s_rp[w][tid];
       const int row = c + tid * nC;
       if (row < E) A.logits[row] = v;
-      else A.gamma[0] = 1.f / (1.f + expf(-v));
+      else A.gamma[0] = v = 1.f / (1.f + expf(-v));
+      st_relaxed64(A.x_logit + row, x_word(e_logit, v));
     }
-    grid_arrive();  // B1: logits written
     const XGroup xg = load_xgroup(sx, ngH);
     // ------------------------------------------------------------- C --
     // while the other CTAs finish: this CTA's block of the shared expert
@@ -629,7 +685,6 @@ __global__ void __launch_bounds__(kFusedThreads, 1) fused_stack_kernel(const __g
       float* const ao[2] = {A.a + (size_t)k * I + (size_t)c * GS::kW, nullptr};
       run_blocks<SBITS, 1>(sl, sb, H, xg, wt, ao, s_blk, ys);
     }
-    if (!grid_wait()) { aborted = true; break; }
     // ------------------------------------------------------------- D --
     {
       // routing: every thread keys up to two logits; per-warp top-k, then one
@@ -637,13 +692,28 @@ __global__ void __launch_bounds__(kFusedThreads, 1) fused_stack_kernel(const __g
       uint64_t key[2];
       bool nan_seen = false;
       float lv[2];
-      const float gv = tid == 0 ? ldcg_f(A.gamma) : 0.f;
+      {
+        uint64_t lw[2], gw = 0;
+        bool ok = true;
+        if (tid == 0) gw = ld_relaxed64(A.x_logit + E);
 #pragma unroll
-      for (int i = 0; i < 2; ++i) {
-        const int e = tid + i * kFusedThreads;
-        lv[i] = e < E ? ldcg_f(A.logits + e) : 0.f;
+        for (int i = 0; i < 2; ++i) {
+          const int e = tid + i * kFusedThreads;
+          lw[i] = e < E ? ld_relaxed64(A.x_logit + e) : 0;
+        }
+        {
+          uint64_t all3[3] = {lw[0], lw[1], gw};
+          ok = x_spin_all(all3, e_logit, [&](int i) { return A.x_logit + (i < 2 ? tid + i * kFusedThreads : E); },
+                          [&](int i) { return i < 2 ? tid + i * kFusedThreads < E : tid == 0; });
+          lw[0] = all3[0];
+          lw[1] = all3[1];
+          gw = all3[2];
+        }
+#pragma unroll
+        for (int i = 0; i < 2; ++i) lv[i] = __uint_as_float((uint32_t)lw[i]);
+        if (tid == 0) s_gamma = __uint_as_float((uint32_t)gw);
+        if (!x_agree(ok)) { aborted = true; break; }
       }
-      if (tid == 0) s_gamma = gv;
 #pragma unroll
       for (int i = 0; i < 2; ++i) {
         const int e = tid + i * kFusedThreads;
@@ -697,26 +767,39 @@ __global__ void __launch_bounds__(kFusedThreads, 1) fused_stack_kernel(const __g
     const int key0 = q0 / GR::kPerGroup, key1 = (q1 - 1) / GR::kPerGroup;
     const int ngI = I / 64;
     if (lane == 0) {
-      if (warp < kSlots) {
+      if (warp < kFirstWave) {
         if (warp < nq) {
           const int q = q0 + warp;
           fence_proxy_async();
           issue_block(warp, LY.experts + (size_t)s_ids[q / NBr] * LR.bytes, LR, q % NBr, GR::gu_sb(H));
         }
-      } else if (warp < kSlots + kSbEntries) {
+      } else if (warp >= kSlots && warp < kSlots + kSbEntries) {
         const int e = warp - kSlots;
         if (nq > 0 && (e == 0 || key1 != key0)) {
           const int key = e == 0 ? key0 : key1;
           fence_proxy_async();
           issue_sb(e, LY.experts + (size_t)s_ids[key / ngI] * LR.bytes, LR, key % ngI);
         }
-      } else {
+      }
+    }
+    // the second wave (the other slots, L2 prefetch of the later blocks) goes
+    // out once the first wave has landed, so that the first blocks are not
+    // slowed by requests for the later ones
+    auto second_wave = [&]() {
+      if (lane != 0) return;
+      if (warp >= kFirstWave && warp < kSlots) {
+        if (warp < nq) {
+          const int q = q0 + warp;
+          fence_proxy_async();
+          issue_block(warp, LY.experts + (size_t)s_ids[q / NBr] * LR.bytes, LR, q % NBr, GR::gu_sb(H));
+        }
+      } else if (warp >= kSlots + kSbEntries) {
         for (int b = kSlots + (warp - kSlots - kSbEntries); b < nq; b += kFusedWarps - kSlots - kSbEntries) {
           const int q = q0 + b;
           prefetch_block(LY.experts + (size_t)s_ids[q / NBr] * LR.bytes, LR, q % NBr, GR::gu_sb(H));
         }
       }
-    }
+    };
     // ------------------------------------------------------------- E --
     // routed blocks two at a time (block b in slot b % kSlots); a freed slot
     // takes block b + kSlots at once
@@ -744,6 +827,7 @@ __global__ void __launch_bounds__(kFusedThreads, 1) fused_stack_kernel(const __g
           ao[n] = A.a + (size_t)j * I + (size_t)nbk * GR::kW;
         }
         if (aborted) break;
+        if (b == 0) second_wave();
         const uint8_t* const slc[2] = {sl[0], sl[1]};
         const uint32_t* const sbc[2] = {sb[0], sb[1]};
         const float wtc[2] = {wt[0], wt[1]};
@@ -773,38 +857,40 @@ __global__ void __launch_bounds__(kFusedThreads, 1) fused_stack_kernel(const __g
     // ------------------------------------------------------------- F --
     {
       const float gm = s_gamma;
-      float* part = A.part + (size_t)c * H;
+      uint64_t* part = A.x_part + (size_t)c * H;
 #pragma unroll
       for (int m = 0; m < kFusedRowsPerThread; ++m) {
         const int i = tid + m * kFusedThreads;
-        if (i < H) part[i] = fmaf(gm, ys[m], yr[m]);
+        if (i < H) st_relaxed64(part + i, x_word(e_part, fmaf(gm, ys[m], yr[m])));
       }
     }
-    grid_arrive();  // B2: partial outputs written
-    if (!grid_wait()) { aborted = true; break; }
     // ------------------------------------------------------------- G --
     {
       // rows i0 + r, r < nd: ngr threads per row each sum every ngr-th CTA's
       // partial; then one thread per row adds those sums in order
       const int ngr = nd > 0 ? kFusedThreads / nd : 0;
       const int r = nd > 0 ? tid % nd : 0, pg = nd > 0 ? tid / nd : kFusedThreads;
+      const float hres = tid < nd ? A.h[i0 + tid] : 0.f;  // this CTA's own rows
+      bool ok = true;
       if (pg < ngr) {
         constexpr int kLoads = (kFusedMaxCtas * 32 + kFusedThreads - 1) / kFusedThreads;  // ngr >= 512 / 32
-        float v[kLoads];
+        uint64_t v[kLoads];
 #pragma unroll
         for (int t2 = 0; t2 < kLoads; ++t2) {
           const int p = pg + t2 * ngr;
-          v[t2] = p < nC ? ldcg_f(A.part + (size_t)p * H + i0 + r) : 0.f;
+          v[t2] = p < nC ? ld_relaxed64(A.x_part + (size_t)p * H + i0 + r) : x_word(e_part, 0.f);
         }
+        ok = x_spin_all(v, e_part, [&](int t2) { return A.x_part + (size_t)(pg + t2 * ngr) * H + i0 + r; },
+                        [&](int t2) { return pg + t2 * ngr < nC; });
         float acc = 0.f;
 #pragma unroll
-        for (int t2 = 0; t2 < kLoads; ++t2) acc += v[t2];
+        for (int t2 = 0; t2 < kLoads; ++t2) acc += __uint_as_float((uint32_t)v[t2]);
         sred[pg * nd + r] = acc;
       }
-      __syncthreads();
+      if (!x_agree(ok)) { aborted = true; break; }
       float ss = 0.f;
       if (tid < nd) {
-        float v = ldcg_f(A.h + i0 + tid);
+        float v = hres;
         for (int g = 0; g < ngr; ++g) v += sred[g * nd + tid];
         A.h[i0 + tid] = v;
         ss = v * v;
@@ -814,19 +900,20 @@ __global__ void __launch_bounds__(kFusedThreads, 1) fused_stack_kernel(const __g
         if (lane == 0) A.ss_part[c] = ss;
       }
     }
-    grid_arrive();  // B3: h' and the partial sums written
+    grid_arrive();  // h' and the partial sums written
   }
 
   if (!aborted && A.n_layers > 0 && grid_wait()) {
-    // epilogue: xn' of the last layer for this CTA's rows
-    const float r = norm_scale();
+    // epilogue: xn' of the last layer for this CTA's rows (h' written by this thread)
+    const float r_last = norm_scale();
     const float* w = A.layers[A.n_layers - 1].norm_w;
-    for (int i = i0 + tid; i < i1; i += kFusedThreads) A.xn[i] = ldcg_f(A.h + i) * r * w[i];
+    if (tid < nd) A.xn[i0 + tid] = A.h[i0 + tid] * r_last * w[i0 + tid];
     __syncthreads();
     if (tid == 0) {
       __threadfence();
       const unsigned prev = atomicAdd(&A.sync[1], 1u);
-      if (prev == (unsigned)nC - 1) {  // every CTA is past its last barrier and wait
+      if (prev == (unsigned)nC - 1) {  // every CTA has read the epoch base and is past its last exchange
+        A.sync[2] = base + 2u * (uint32_t)A.n_layers + 2u;
         A.sync[0] = 0;
         A.sync[1] = 0;
         __threadfence();

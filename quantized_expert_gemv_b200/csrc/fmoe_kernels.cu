@@ -460,7 +460,7 @@ __global__ void pack_sb_kernel(const uint16_t* __restrict__ scale, const uint16_
 
 // ------------------------------------------------------- host helpers ----
 struct WsLayout {
-  size_t sync, ss, fpart, part, logits, ids, weights, gamma, a, y, bytes;
+  size_t sync, ss, x_logit, x_part, part, logits, ids, weights, gamma, a, y, bytes;
 };
 
 static inline size_t align_up(size_t v, size_t a) { return (v + a - 1) / a * a; }
@@ -469,11 +469,14 @@ constexpr int kMaxSMs = 1024;
 
 static WsLayout ws_layout(int H, int I, int E, int k, int T) {
   WsLayout w;
-  w.sync = 0;    // grid-barrier counters of the fused kernel
-  w.ss = 4096;   // per-CTA partial sums of h'^2
+  w.sync = 0;    // grid-barrier counter, exit counter and epoch of the fused kernel
+  w.ss = 4096;   // per-CTA partial sums of h'^2 of the fused kernel
   size_t o = 4096 + (size_t)kMaxSMs * 4;
-  w.fpart = o;   // per-CTA partial outputs of the fused kernel [kFusedMaxCtas][H]
-  o = align_up(o + (size_t)kFusedMaxCtas * H * 4, 256);
+  // exchange words of the fused kernel (8 bytes each)
+  w.x_logit = o;
+  o = align_up(o + (size_t)(E + 1) * 8, 256);
+  w.x_part = o;
+  o = align_up(o + (size_t)kFusedMaxCtas * H * 8, 256);
   w.part = o;
   o = align_up(o + (size_t)T * (E + 1) * kRouterSplit * 4, 256);
   w.logits = o;
@@ -669,8 +672,9 @@ static int launch_fused(const fmoe_layer_weights* layers, int n_layers, float* h
   args.weights = reinterpret_cast<float*>(base + w.weights);
   args.gamma = reinterpret_cast<float*>(base + w.gamma);
   args.a = reinterpret_cast<float*>(base + w.a);
+  args.x_logit = reinterpret_cast<uint64_t*>(base + w.x_logit);
+  args.x_part = reinterpret_cast<uint64_t*>(base + w.x_part);
   args.ss_part = reinterpret_cast<float*>(base + w.ss);
-  args.part = reinterpret_cast<float*>(base + w.fpart);
   args.sync = reinterpret_cast<unsigned*>(base + w.sync);
   args.plan = fc.plan;
   for (int l0 = 0; l0 < n_layers; l0 += kFusedMaxLayers) {
