@@ -1,0 +1,292 @@
+// fmoe_batched.cuh -- the expert forward for T > 1 tokens, grouped by expert.
+//
+// With T tokens and k routed experts each, the T k routed slots and the T
+// shared-expert slots are sorted by expert (group_kernel, in token order
+// within an expert, so every result is deterministic).  Each expert's
+// weights are then read once per step for all of its tokens:
+//   - groups with fewer than kTcMinTokens tokens, in work items of up to
+//     kGrpMaxM tokens, go through the integer-dot GEMV (gateup_group_kernel,
+//     down_group_kernel): one load of a weight row serves every token of the
+//     item;
+//   - groups with at least kTcMinTokens tokens are dense enough for the
+//     tensor cores (fmoe_tc.cuh): their items are listed separately.
+// Slot s = t (k + 1) + j addresses a [T][k+1][I] and y [T][k+1][H] exactly as
+// on the one-kernel-per-slot path, so the combine kernel is shared.
+// Source pages: "What is Flash-MoE?" (a2a-mcp.org), section "2. FMA-optimised
+// dequantisation kernels" (the pages run one token at a time; grouping the
+// batch by expert is this implementation's addition for T > 1).
+#pragma once
+
+#include <cstdint>
+
+#include "fmoe.h"
+#include "fmoe_device.cuh"
+#include "fmoe_layout.h"
+
+namespace fmoe {
+
+constexpr int kGrpMaxM = 16;      // tokens per GEMV work item
+constexpr int kGrpThreads = 256;
+constexpr int kGuSplit = 16;      // CTAs per item over the gate/up row pairs
+constexpr int kDnRows = 128;      // hidden rows per CTA of the grouped down product
+
+// Device lists built by group_kernel.  Group g < E is routed expert g, group
+// E the shared expert.
+struct GroupWork {
+  int* count;   // [E + 1] slots per group
+  int* offset;  // [E + 2] first slot of each group in `slots`
+  int* slots;   // [T (k + 1)] slot indices, grouped, in token order
+  int* n_items; // [2] GEMV work items, tensor-core work items
+  int4* items;  // [max_items] (group, first slot within the group, tokens, 0)
+  int4* tc;     // [max_tc]    (group, first, tokens, 0)
+};
+
+__host__ __device__ constexpr int group_max_items(int T, int k, int E) {
+  // one item per non-empty group plus one per further kGrpMaxM slots
+  return (T * k < E ? T * k : E) + 1 + (T * (k + 1)) / kGrpMaxM + 1;
+}
+
+// One CTA.  Sorts the T (k + 1) slots by group (stable), builds the work
+// items (groups with >= tc_min tokens go to the tensor-core list when
+// tc_min > 0), and zeroes a / y of slots whose expert id is out of range.
+__global__ void __launch_bounds__(1024) group_kernel(const int32_t* __restrict__ ids, int T, int k, int E, int I,
+                                                     int H, int tc_min, GroupWork w, float* __restrict__ a,
+                                                     float* __restrict__ y) {
+  extern __shared__ int gsm[];
+  int* cnt = gsm;             // [E + 1]
+  int* off = cnt + (E + 1);   // [E + 2]
+  int* nit = off + (E + 2);   // [E + 2]: items per group, then their exclusive scan
+  const int S = T * (k + 1);
+  const int tid = threadIdx.x, nt = blockDim.x;
+  for (int g = tid; g <= E; g += nt) cnt[g] = 0;
+  __syncthreads();
+  auto group_of = [&](int s) -> int {
+    const int t = s / (k + 1), j = s % (k + 1);
+    if (j == k) return E;
+    const int id = ids[(size_t)t * k + j];
+    return (id >= 0 && id < E) ? id : -1;
+  };
+  bool bad = false;
+  for (int s = tid; s < S; s += nt) {
+    const int g = group_of(s);
+    if (g >= 0) atomicAdd(&cnt[g], 1);
+    else {
+      bad = true;
+      for (int i = 0; i < I; ++i) a[(size_t)s * I + i] = 0.f;
+      for (int i = 0; i < H; ++i) y[(size_t)s * H + i] = 0.f;
+    }
+  }
+  if (__syncthreads_or(bad) && tid == 0) raise_status(FMOE_STATUS_BAD_EXPERT_ID);
+  if (tid == 0) {  // exclusive scans (E + 1 <= 1025 entries)
+    int o = 0, it = 0;
+    for (int g = 0; g <= E; ++g) {
+      off[g] = o;
+      o += cnt[g];
+      const int c = cnt[g];
+      const int n = c == 0 ? 0 : (tc_min > 0 && c >= tc_min ? 0 : (c + kGrpMaxM - 1) / kGrpMaxM);
+      nit[g] = it;
+      it += n;
+    }
+    off[E + 1] = o;
+    nit[E + 1] = it;
+    int ntc = 0;
+    for (int g = 0; g <= E; ++g)
+      if (tc_min > 0 && cnt[g] >= tc_min) w.tc[ntc++] = make_int4(g, 0, cnt[g], 0);
+    w.n_items[0] = it;
+    w.n_items[1] = ntc;
+  }
+  __syncthreads();
+  for (int g = tid; g <= E + 1; g += nt) w.offset[g] = off[g];
+  for (int g = tid; g <= E; g += nt) {
+    w.count[g] = cnt[g];
+    const int c = cnt[g];
+    if (c > 0 && !(tc_min > 0 && c >= tc_min))
+      for (int i = 0; i * kGrpMaxM < c; ++i)
+        w.items[nit[g] + i] = make_int4(g, i * kGrpMaxM, min(kGrpMaxM, c - i * kGrpMaxM), 0);
+  }
+  // stable placement: rank of s = earlier slots of the same group
+  for (int s = tid; s < S; s += nt) {
+    const int g = group_of(s);
+    if (g < 0) continue;
+    int r = 0;
+    for (int s2 = 0; s2 < s; ++s2) r += group_of(s2) == g;
+    w.slots[off[g] + r] = s;
+  }
+}
+
+__device__ __forceinline__ const uint8_t* group_record(const ExpertSet& es, int g, int* bits) {
+  if (g == es.E) {
+    *bits = es.shared_bits;
+    return es.shared;
+  }
+  *bits = es.bits;
+  return es.experts + (size_t)g * es.rec_bytes;
+}
+
+// Token i's staged vector: K inputs at base + i * stride.
+__device__ __forceinline__ StagedX staged_i(unsigned char* base, size_t stride, int i, int K) {
+  return staged_x_at(base + (size_t)i * stride, K);
+}
+
+// Gate/up row pairs [p0, p1) of one record for the m tokens staged at sxb:
+// each warp takes row pairs; a lane owns whole groups of both rows of a
+// pair, loads their codes once and applies them to every token.
+
+template <int BITS>
+__device__ __forceinline__ void gateup_rows_multi(const uint8_t* rec, const ExpertSet& es, unsigned char* sxb,
+                                                  size_t sxs, int m, float* __restrict__ a, const int* slot_of,
+                                                  int p0, int p1) {
+  const int H = es.H, ng = H / 64;
+  const int lpr = ng < 32 ? ng : 32, gpl = ng / lpr, ppu = 32 / lpr;
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5, nw = blockDim.x >> 5;
+  const int ps = lane / lpr, lg = lane % lpr;
+  const RecordLayout L = record_layout(BITS, H, es.I);
+  const uint8_t* codes = rec + L.gu_codes;
+  const uint32_t* sbw = reinterpret_cast<const uint32_t*>(rec + L.gu_sb);
+  for (int u = p0 / ppu + warp; u * ppu < p1; u += nw) {
+    const int n = u * ppu + ps;
+    const bool live = n < p1;
+    const int nn = live ? n : p1 - 1;
+    const uint8_t* rg = codes + (size_t)(2 * nn) * L.gu_row_bytes;
+    const uint8_t* ru = rg + L.gu_row_bytes;
+    float yg[kGrpMaxM], yu[kGrpMaxM];
+#pragma unroll
+    for (int i = 0; i < kGrpMaxM; ++i) yg[i] = yu[i] = 0.f;
+    for (int mm = 0; mm < gpl; ++mm) {
+      const int g = lg + mm * lpr;
+      const GroupCodes<BITS> cg = load_group<BITS>(rg, ng, g);
+      const GroupCodes<BITS> cu = load_group<BITS>(ru, ng, g);
+      const uint32_t sg = ld_stream_u32(sbw + (size_t)(2 * nn) * ng + g);
+      const uint32_t su = ld_stream_u32(sbw + (size_t)(2 * nn + 1) * ng + g);
+#pragma unroll
+      for (int i = 0; i < kGrpMaxM; ++i) {
+        if (i < m) {
+          const StagedX sx = staged_i(sxb, sxs, i, H);
+          uint4 xv[8];
+          load_xv(sx, ng, g, xv);
+          const float d = sx.delta[g], xs = sx.xsum[g];
+          yg[i] = group_epilogue(yg[i], sg, group_dot<BITS>(cg, xv), d, xs);
+          yu[i] = group_epilogue(yu[i], su, group_dot<BITS>(cu, xv), d, xs);
+        }
+      }
+    }
+#pragma unroll
+    for (int i = 0; i < kGrpMaxM; ++i) {
+      if (i < m) {
+        float g = yg[i], v = yu[i];
+        for (int o = lpr >> 1; o > 0; o >>= 1) {
+          g += __shfl_xor_sync(0xffffffffu, g, o);
+          v += __shfl_xor_sync(0xffffffffu, v, o);
+        }
+        if (lg == 0 && live) a[(size_t)slot_of[i] * es.I + n] = silu_mul(g, v);
+      }
+    }
+  }
+}
+
+// grid (max items, kGuSplit).  Item (group, first, m): the group's slots
+// first .. first + m - 1.  Also computes gamma[t] = sigmoid(w_sg . xn[t])
+// for the shared expert's tokens when gamma is given.
+__global__ void __launch_bounds__(kGrpThreads)
+gateup_group_kernel(ExpertSet es, GroupWork w, const float* __restrict__ xn, float* __restrict__ a,
+                    const float* __restrict__ w_sg, float* __restrict__ gamma) {
+  extern __shared__ __align__(128) unsigned char smem[];
+  __shared__ int s_slot[kGrpMaxM];
+  if ((int)blockIdx.x >= w.n_items[0]) return;
+  const int4 it = w.items[blockIdx.x];
+  const int g = it.x, m = it.z, k1 = es.k + 1;
+  if (threadIdx.x < m) s_slot[threadIdx.x] = w.slots[w.offset[g] + it.y + threadIdx.x];
+  __syncthreads();
+  const size_t sxs = (staged_x_bytes(es.H) + 15) & ~(size_t)15;
+  for (int i = 0; i < m; ++i) stage_x(xn + (size_t)(s_slot[i] / k1) * es.H, es.H, staged_i(smem, sxs, i, es.H));
+  __syncthreads();
+  if (gamma && g == es.E && blockIdx.y == 0) {
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    for (int i = warp; i < m; i += kGrpThreads / 32) {
+      const float* x = xn + (size_t)(s_slot[i] / k1) * es.H;
+      float z = 0.f;
+      for (int c = lane * 4; c < es.H; c += 128) {
+        const float4 wv = __ldg(reinterpret_cast<const float4*>(w_sg + c));
+        const float4 v = __ldg(reinterpret_cast<const float4*>(x + c));
+        z = fmaf(wv.x, v.x, z);
+        z = fmaf(wv.y, v.y, z);
+        z = fmaf(wv.z, v.z, z);
+        z = fmaf(wv.w, v.w, z);
+      }
+      z = warp_sum(z);
+      if (lane == 0) gamma[s_slot[i] / k1] = 1.f / (1.f + expf(-z));
+    }
+  }
+  int p0, p1;
+  {
+    const int ng = es.H / 64, ppu = 32 / (ng < 32 ? ng : 32);  // row pairs per warp unit
+    const int per = ((es.I + kGuSplit - 1) / kGuSplit + ppu - 1) / ppu * ppu;
+    p0 = min(es.I, (int)blockIdx.y * per);
+    p1 = min(es.I, p0 + per);
+  }
+  int bits;
+  const uint8_t* rec = group_record(es, g, &bits);
+  if (bits == 4) gateup_rows_multi<4>(rec, es, smem, sxs, m, a, s_slot, p0, p1);
+  else gateup_rows_multi<2>(rec, es, smem, sxs, m, a, s_slot, p0, p1);
+}
+
+// Down product of one record for one hidden row and the m tokens staged at
+// sx[0..m) (their SwiGLU outputs): the group's column-block words are loaded
+// once and applied to every token.
+template <int BITS>
+__device__ __forceinline__ void down_row_multi(const uint8_t* rec, const ExpertSet& es, unsigned char* sab,
+                                               size_t sas, int m, int row, float (&yv)[kGrpMaxM]) {
+  const int H = es.H, I = es.I, ngI = I / 64;
+  constexpr int kWpg = BITS == 4 ? 8 : 4;
+  const RecordLayout L = record_layout(BITS, H, I);
+  const uint32_t* codes = reinterpret_cast<const uint32_t*>(rec + L.down_codes) + row;
+  const uint32_t* sbw = reinterpret_cast<const uint32_t*>(rec + L.down_sb) + row;
+  for (int g = 0; g < ngI; ++g) {
+    uint32_t wd[kWpg];
+#pragma unroll
+    for (int b = 0; b < kWpg; ++b) wd[b] = ld_stream_u32(codes + (size_t)(g * kWpg + b) * H);
+    const uint32_t sb = ld_stream_u32(sbw + (size_t)g * H);
+#pragma unroll
+    for (int i = 0; i < kGrpMaxM; ++i) {
+      if (i < m) {
+        const StagedX sx = staged_i(sab, sas, i, I);
+        int acc = 0;
+#pragma unroll
+        for (int b = 0; b < kWpg; ++b) {
+          if (BITS == 4) acc += word_dot4(wd[b], sx.xs[b * ngI + g]);
+          else acc += word_dot2(wd[b], sx.xs[(2 * b) * ngI + g], sx.xs[(2 * b + 1) * ngI + g]);
+        }
+        yv[i] = group_epilogue(yv[i], sb, acc, sx.delta[g], sx.xsum[g]);
+      }
+    }
+  }
+}
+
+// grid (max items, H / kDnRows); one hidden row per thread.
+__global__ void __launch_bounds__(kDnRows)
+down_group_kernel(ExpertSet es, GroupWork w, const float* __restrict__ a, float* __restrict__ y) {
+  extern __shared__ __align__(128) unsigned char smem[];
+  __shared__ int s_slot[kGrpMaxM];
+  if ((int)blockIdx.x >= w.n_items[0]) return;
+  const int4 it = w.items[blockIdx.x];
+  const int g = it.x, m = it.z;
+  if (threadIdx.x < m) s_slot[threadIdx.x] = w.slots[w.offset[g] + it.y + threadIdx.x];
+  __syncthreads();
+  const size_t sas = (staged_x_bytes(es.I) + 15) & ~(size_t)15;
+  for (int i = 0; i < m; ++i) stage_x(a + (size_t)s_slot[i] * es.I, es.I, staged_i(smem, sas, i, es.I));
+  __syncthreads();
+  const int row = (int)blockIdx.y * kDnRows + (int)threadIdx.x;
+  if (row >= es.H) return;
+  float yv[kGrpMaxM];
+#pragma unroll
+  for (int i = 0; i < kGrpMaxM; ++i) yv[i] = 0.f;
+  int bits;
+  const uint8_t* rec = group_record(es, g, &bits);
+  if (bits == 4) down_row_multi<4>(rec, es, smem, sas, m, row, yv);
+  else down_row_multi<2>(rec, es, smem, sas, m, row, yv);
+#pragma unroll
+  for (int i = 0; i < kGrpMaxM; ++i)
+    if (i < m) y[(size_t)s_slot[i] * es.H + row] = yv[i];
+}
+
+}  // namespace fmoe

@@ -321,6 +321,12 @@ down_kernel(ExpertSet es, const int32_t* __restrict__ ids, const float* __restri
   y_out[row] = bits == 4 ? down_row_cols<4>(rec, es, sx, row) : down_row_cols<2>(rec, es, sx, row);
 }
 
+}  // namespace fmoe
+
+#include "fmoe_batched.cuh"
+
+namespace fmoe {
+
 // ---------------------------------------------------------- combine ----
 __device__ __forceinline__ float block_sum(float v, float* red) {
   v = warp_sum(v);
@@ -460,7 +466,8 @@ __global__ void pack_sb_kernel(const uint16_t* __restrict__ scale, const uint16_
 
 // ------------------------------------------------------- host helpers ----
 struct WsLayout {
-  size_t sync, ss, x_logit, x_part, part, logits, ids, weights, gamma, a, y, bytes;
+  size_t sync, ss, x_logit, x_part, grp, part, logits, ids, weights, gamma, a, y, bytes;
+  size_t g_count, g_offset, g_slots, g_nitems, g_items, g_tc;  // inside grp
 };
 
 static inline size_t align_up(size_t v, size_t a) { return (v + a - 1) / a * a; }
@@ -477,6 +484,20 @@ static WsLayout ws_layout(int H, int I, int E, int k, int T) {
   o = align_up(o + (size_t)(E + 1) * 8, 256);
   w.x_part = o;
   o = align_up(o + (size_t)kFusedMaxCtas * H * 8, 256);
+  // expert groups of the T > 1 path
+  w.grp = o;
+  w.g_count = o;
+  o = align_up(o + (size_t)(E + 1) * 4, 16);
+  w.g_offset = o;
+  o = align_up(o + (size_t)(E + 2) * 4, 16);
+  w.g_slots = o;
+  o = align_up(o + (size_t)T * (k + 1) * 4, 16);
+  w.g_nitems = o;
+  o = align_up(o + 16, 16);
+  w.g_items = o;
+  o = align_up(o + (size_t)group_max_items(T, k, E) * 16, 16);
+  w.g_tc = o;
+  o = align_up(o + (size_t)(E + 1) * 16, 256);
   w.part = o;
   o = align_up(o + (size_t)T * (E + 1) * kRouterSplit * 4, 256);
   w.logits = o;
@@ -552,9 +573,37 @@ static int launch_topk(const float* part, const float* logits_in, int T, int E, 
   return cuda_rc(cudaGetLastError());
 }
 
+// Dynamic shared memory above the default 48 KB for a kernel, set once per device.
+static bool smem_optin(const void* fn, size_t bytes, int slot) {
+  static size_t done[64][8];
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return false;
+  if (done[dev][slot] >= bytes) return true;
+  if (cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)bytes) != cudaSuccess) return false;
+  done[dev][slot] = bytes;
+  return true;
+}
+
+// Expert forward of T tokens.  With T >= 2 and a group workspace the slots
+// are grouped by expert first (each expert's weights read once per step);
+// otherwise one CTA column per slot.
 static int launch_experts(const ExpertSet& es, const float* xn, const int32_t* ids, int T, float* a,
-                          float* y, const float* w_sg, float* gamma, cudaStream_t st) {
+                          float* y, const float* w_sg, float* gamma, const GroupWork* gw, cudaStream_t st) {
   const int slots = T * (es.k + 1);
+  if (T >= 2 && gw) {
+    const size_t sxs = (staged_x_bytes(es.H) + 15) & ~(size_t)15, sas = (staged_x_bytes(es.I) + 15) & ~(size_t)15;
+    const size_t gu_smem = kGrpMaxM * sxs, dn_smem = kGrpMaxM * sas;
+    const size_t grp_smem = (size_t)(3 * es.E + 5) * 4;
+    if (gu_smem <= 200 * 1024 && dn_smem <= 200 * 1024 &&
+        smem_optin(reinterpret_cast<const void*>(&gateup_group_kernel), gu_smem, 0) &&
+        smem_optin(reinterpret_cast<const void*>(&down_group_kernel), dn_smem, 1)) {
+      const int items = group_max_items(T, es.k, es.E);
+      group_kernel<<<1, 1024, grp_smem, st>>>(ids, T, es.k, es.E, es.I, es.H, 0, *gw, a, y);
+      gateup_group_kernel<<<dim3(items, kGuSplit), kGrpThreads, gu_smem, st>>>(es, *gw, xn, a, w_sg, gamma);
+      down_group_kernel<<<dim3(items, (es.H + kDnRows - 1) / kDnRows), kDnRows, dn_smem, st>>>(es, *gw, a, y);
+      return cuda_rc(cudaGetLastError());
+    }
+  }
   {
     const int ng = es.H / 64, lpr = ng < 32 ? ng : 32;
     const int units = es.I / (32 / lpr);
@@ -705,6 +754,17 @@ static int launch_fused(const fmoe_layer_weights* layers, int n_layers, float* h
   return FMOE_OK;
 }
 
+static GroupWork group_work(unsigned char* base, const WsLayout& w) {
+  GroupWork g;
+  g.count = reinterpret_cast<int*>(base + w.g_count);
+  g.offset = reinterpret_cast<int*>(base + w.g_offset);
+  g.slots = reinterpret_cast<int*>(base + w.g_slots);
+  g.n_items = reinterpret_cast<int*>(base + w.g_nitems);
+  g.items = reinterpret_cast<int4*>(base + w.g_items);
+  g.tc = reinterpret_cast<int4*>(base + w.g_tc);
+  return g;
+}
+
 static int layer_forward_impl(const fmoe_layer_weights* lw, const float* logits_in, float* h,
                               float* xn, int T, void* ws, size_t ws_bytes, cudaStream_t st) {
   int rc = weights_check(lw);
@@ -738,7 +798,8 @@ static int layer_forward_impl(const fmoe_layer_weights* lw, const float* logits_
     if (rc == FMOE_OK) rc = launch_topk(part, nullptr, T, d.n_experts, d.top_k, logits, ids, weights, gamma, st);
   }
   if (rc != FMOE_OK) return rc;
-  rc = launch_experts(es, xn, ids, T, a, y, lw->w_shared_gate, logits_in ? gamma : nullptr, st);
+  const GroupWork gw = group_work(base, w);
+  rc = launch_experts(es, xn, ids, T, a, y, lw->w_shared_gate, logits_in ? gamma : nullptr, &gw, st);
   if (rc != FMOE_OK) return rc;
   return launch_combine(y, weights, gamma, h, lw->norm_w, d.eps, T, d.top_k, d.hidden, h, xn, st);
 }
@@ -826,7 +887,8 @@ extern "C" int fmoe_expert_forward(const fmoe_layer_weights* lw, const float* d_
   const WsLayout w = ws_layout(d.hidden, d.inter, d.n_experts, d.top_k, T);
   if (ws_bytes < w.bytes) return FMOE_ERR_BUFFER_TOO_SMALL;
   float* a = reinterpret_cast<float*>(static_cast<unsigned char*>(d_ws) + w.a);
-  return launch_experts(expert_set(lw), d_xn, d_ids, T, a, d_y, lw->w_shared_gate, d_gamma, stream);
+  const GroupWork gw = group_work(static_cast<unsigned char*>(d_ws), w);
+  return launch_experts(expert_set(lw), d_xn, d_ids, T, a, d_y, lw->w_shared_gate, d_gamma, &gw, stream);
 }
 
 extern "C" int fmoe_combine_residual_rmsnorm(const float* d_y, const float* d_weights,

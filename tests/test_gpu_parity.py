@@ -367,6 +367,27 @@ def test_layer_forward_batched_zipf_routing(full_layer):
                           logits_given=True)
 
 
+@pytest.mark.parametrize("wl", [SMALL, SMALL2], ids=["small4", "small2"])
+def test_grouped_experts_many_tokens_per_expert(wl):
+    """40 tokens all routed to the same four experts (given logits): every
+    group holds 40 slots, so the grouped path splits them into work items of
+    up to 16 tokens.  Tokens from each item, and the last one, are checked
+    against the oracle."""
+    T = 40
+    lw = device_layer(wl)
+    lw_o = oracle_layer(wl, 0)
+    lg = np.zeros((T, wl.n_experts), np.float32)
+    lg[:, [3, 7, 11, 15]] = [4.0, 3.0, 2.0, 1.0]
+    x = synth.tokens(wl, T, stream=43)
+    h, xn = dev(x), dev(x)
+    ws = fm.alloc_workspace(lw.desc, T)
+    fm.fmoe_layer_forward_logits(lw, dev(lg), h, xn, ws)
+    for t in (0, 15, 16, 31, 32, 39):
+        check_layer_token(wl, lw_o, ws, lw.desc, T, t, x[t], x[t], host(h)[t], host(xn)[t], f"t={t}",
+                          logits_given=True)
+    assert fm.fmoe_read_status() == 0
+
+
 # ------------------------------------------------------------------- chains --
 
 @pytest.mark.parametrize("wl", [synth.TINY, TINY2, SMALL, SMALL2], ids=["tiny4", "tiny2", "small4", "small2"])
