@@ -239,6 +239,15 @@ int fmoe_stack_forward(const fmoe_layer_weights* layers, int n_layers, float* d_
  * setting, returns the previous value. */
 int fmoe_set_fused(int enable);
 
+/* Chooses the expert products of the T > 1 path for experts that receive at
+ * least 16 tokens in a step (and the shared expert when T >= 16): enable != 0
+ * (the default) runs them as tcgen05 tensor-core matrix products on
+ * dequantised fp16 weights (inputs kept to ~22 bits as an fp16 hi / lo
+ * pair), 0 as the integer-dot matrix-vector path in batches of 16 tokens.
+ * Both compute the same products within the tolerance; process-wide
+ * setting, returns the previous value. */
+int fmoe_set_tensor_cores(int enable);
+
 /* 1 if the persistent kernel runs layers of descriptor d at T = 1 on the
  * current device (shape and shared-memory plan fit), else 0 (also on any
  * error).  The persistent kernel leaves the gate/up outputs a in the

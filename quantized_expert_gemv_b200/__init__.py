@@ -89,6 +89,7 @@ _SIGS = {
     "fmoe_stack_forward": (_i32, [_PW, _i32, _vp, _vp, _i32, _vp, _sz, _vp]),
     "fmoe_set_fused": (_i32, [_i32]),
     "fmoe_fused_supported": (_i32, [_PDESC]),
+    "fmoe_set_tensor_cores": (_i32, [_i32]),
     "fmoe_layer_forward_noalloc": (_i32, [_PW, _vp, _vp, _i32, _vp]),
 }
 for _name, (_res, _args) in _SIGS.items():
@@ -312,6 +313,12 @@ def fmoe_fused_supported(desc: LayerDesc) -> bool:
     """True if the persistent kernel runs layers of this shape at T = 1 on the current device."""
     c = desc.c() if hasattr(desc, "c") else desc
     return bool(_lib.fmoe_fused_supported(ctypes.byref(c)))
+
+
+def fmoe_set_tensor_cores(enable: bool) -> bool:
+    """Selects tensor-core products (True, default) or the integer-dot path for the
+    heavily routed experts of the T > 1 path; returns the previous setting."""
+    return bool(_lib.fmoe_set_tensor_cores(int(bool(enable))))
 
 
 def fmoe_set_fused(enable: bool) -> bool:

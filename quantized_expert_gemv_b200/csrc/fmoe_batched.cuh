@@ -26,6 +26,7 @@
 namespace fmoe {
 
 constexpr int kGrpMaxM = 16;      // tokens per GEMV work item
+constexpr int kTcItemMax = 128;   // tokens per tensor-core work item
 constexpr int kGrpThreads = 256;
 constexpr int kGuSplit = 16;      // CTAs per item over the gate/up row pairs
 constexpr int kDnRows = 128;      // hidden rows per CTA of the grouped down product
@@ -38,8 +39,12 @@ struct GroupWork {
   int* slots;   // [T (k + 1)] slot indices, grouped, in token order
   int* n_items; // [2] GEMV work items, tensor-core work items
   int4* items;  // [max_items] (group, first slot within the group, tokens, 0)
-  int4* tc;     // [max_tc]    (group, first, tokens, 0)
+  int4* tc;     // [max_tc]    (group, first, tokens, running sum of the items' tokens rounded up to 8)
 };
+
+__host__ __device__ constexpr int group_max_tc(int T, int k, int min_tokens) {
+  return T * (k + 1) / min_tokens + T * (k + 1) / kTcItemMax + 2;
+}
 
 __host__ __device__ constexpr int group_max_items(int T, int k, int E) {
   // one item per non-empty group plus one per further kGrpMaxM slots
@@ -89,9 +94,14 @@ __global__ void __launch_bounds__(1024) group_kernel(const int32_t* __restrict__
     }
     off[E + 1] = o;
     nit[E + 1] = it;
-    int ntc = 0;
+    int ntc = 0, np_sum = 0;
     for (int g = 0; g <= E; ++g)
-      if (tc_min > 0 && cnt[g] >= tc_min) w.tc[ntc++] = make_int4(g, 0, cnt[g], 0);
+      if (tc_min > 0 && cnt[g] >= tc_min)
+        for (int f = 0; f < cnt[g]; f += kTcItemMax) {
+          const int mm = min(kTcItemMax, cnt[g] - f);
+          w.tc[ntc++] = make_int4(g, f, mm, np_sum);
+          np_sum += (mm + 7) / 8 * 8;
+        }
     w.n_items[0] = it;
     w.n_items[1] = ntc;
   }

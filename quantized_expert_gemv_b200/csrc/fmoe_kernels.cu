@@ -324,6 +324,7 @@ down_kernel(ExpertSet es, const int32_t* __restrict__ ids, const float* __restri
 }  // namespace fmoe
 
 #include "fmoe_batched.cuh"
+#include "fmoe_tc.cuh"
 
 namespace fmoe {
 
@@ -468,7 +469,14 @@ __global__ void pack_sb_kernel(const uint16_t* __restrict__ scale, const uint16_
 struct WsLayout {
   size_t sync, ss, x_logit, x_part, grp, part, logits, ids, weights, gamma, a, y, bytes;
   size_t g_count, g_offset, g_slots, g_nitems, g_items, g_tc;  // inside grp
+  size_t tcx, tca;  // staged fp16 inputs of the tensor-core items (0 bytes when T < kTcMinTokens)
 };
+
+// Upper bound of the tensor-core items' token rows (sum of tokens rounded up to 8).
+static size_t tc_np_bound(int T, int k) {
+  if (T < kTcMinTokens) return 0;
+  return (size_t)T * (k + 1) + 8 * (size_t)group_max_tc(T, k, kTcMinTokens);
+}
 
 static inline size_t align_up(size_t v, size_t a) { return (v + a - 1) / a * a; }
 
@@ -497,7 +505,11 @@ static WsLayout ws_layout(int H, int I, int E, int k, int T) {
   w.g_items = o;
   o = align_up(o + (size_t)group_max_items(T, k, E) * 16, 16);
   w.g_tc = o;
-  o = align_up(o + (size_t)(E + 1) * 16, 256);
+  o = align_up(o + (size_t)group_max_tc(T, k, kTcMinTokens) * 16, 256);
+  w.tcx = o;
+  o = align_up(o + tc_np_bound(T, k) * 4 * H, 256);
+  w.tca = o;
+  o = align_up(o + tc_np_bound(T, k) * 4 * I, 256);
   w.part = o;
   o = align_up(o + (size_t)T * (E + 1) * kRouterSplit * 4, 256);
   w.logits = o;
@@ -573,6 +585,8 @@ static int launch_topk(const float* part, const float* logits_in, int T, int E, 
   return cuda_rc(cudaGetLastError());
 }
 
+static int g_tc_enabled = 1;  // tensor-core products for groups of >= kTcMinTokens tokens
+
 // Dynamic shared memory above the default 48 KB for a kernel, set once per device.
 static bool smem_optin(const void* fn, size_t bytes, int slot) {
   static size_t done[64][8];
@@ -588,7 +602,8 @@ static bool smem_optin(const void* fn, size_t bytes, int slot) {
 // are grouped by expert first (each expert's weights read once per step);
 // otherwise one CTA column per slot.
 static int launch_experts(const ExpertSet& es, const float* xn, const int32_t* ids, int T, float* a,
-                          float* y, const float* w_sg, float* gamma, const GroupWork* gw, cudaStream_t st) {
+                          float* y, const float* w_sg, float* gamma, const GroupWork* gw, uint8_t* tcx,
+                          uint8_t* tca, cudaStream_t st) {
   const int slots = T * (es.k + 1);
   if (T >= 2 && gw) {
     const size_t sxs = (staged_x_bytes(es.H) + 15) & ~(size_t)15, sas = (staged_x_bytes(es.I) + 15) & ~(size_t)15;
@@ -598,9 +613,25 @@ static int launch_experts(const ExpertSet& es, const float* xn, const int32_t* i
         smem_optin(reinterpret_cast<const void*>(&gateup_group_kernel), gu_smem, 0) &&
         smem_optin(reinterpret_cast<const void*>(&down_group_kernel), dn_smem, 1)) {
       const int items = group_max_items(T, es.k, es.E);
-      group_kernel<<<1, 1024, grp_smem, st>>>(ids, T, es.k, es.E, es.I, es.H, 0, *gw, a, y);
+      // groups of >= kTcMinTokens tokens go to the tensor cores when the shape tiles
+      const bool tc = g_tc_enabled && T >= kTcMinTokens && tcx && tca && es.H % kTcRows == 0 &&
+                      (2 * es.I) % kTcRows == 0 &&
+                      smem_optin(reinterpret_cast<const void*>(&tc_gemm_kernel<0>), tc_smem_bytes(), 2) &&
+                      smem_optin(reinterpret_cast<const void*>(&tc_gemm_kernel<1>), tc_smem_bytes(), 3);
+      const int max_tc = group_max_tc(T, es.k, kTcMinTokens);
+      group_kernel<<<1, 1024, grp_smem, st>>>(ids, T, es.k, es.E, es.I, es.H, tc ? kTcMinTokens : 0, *gw, a, y);
       gateup_group_kernel<<<dim3(items, kGuSplit), kGrpThreads, gu_smem, st>>>(es, *gw, xn, a, w_sg, gamma);
+      if (tc) {
+        tc_stage_kernel<<<dim3(max_tc, es.H / 64), kTcThreads, 0, st>>>(*gw, xn, es.H, es.k + 1, 0, tcx, es.E, w_sg,
+                                                                      gamma);
+        tc_gemm_kernel<0><<<dim3(max_tc, 2 * es.I / kTcRows), kTcThreads, tc_smem_bytes(), st>>>(es, *gw, tcx, a);
+      }
       down_group_kernel<<<dim3(items, (es.H + kDnRows - 1) / kDnRows), kDnRows, dn_smem, st>>>(es, *gw, a, y);
+      if (tc) {
+        tc_stage_kernel<<<dim3(max_tc, es.I / 64), kTcThreads, 0, st>>>(*gw, a, es.I, es.k + 1, 1, tca, es.E, nullptr,
+                                                                      nullptr);
+        tc_gemm_kernel<1><<<dim3(max_tc, es.H / kTcRows), kTcThreads, tc_smem_bytes(), st>>>(es, *gw, tca, y);
+      }
       return cuda_rc(cudaGetLastError());
     }
   }
@@ -799,7 +830,8 @@ static int layer_forward_impl(const fmoe_layer_weights* lw, const float* logits_
   }
   if (rc != FMOE_OK) return rc;
   const GroupWork gw = group_work(base, w);
-  rc = launch_experts(es, xn, ids, T, a, y, lw->w_shared_gate, logits_in ? gamma : nullptr, &gw, st);
+  rc = launch_experts(es, xn, ids, T, a, y, lw->w_shared_gate, logits_in ? gamma : nullptr, &gw, base + w.tcx,
+                      base + w.tca, st);
   if (rc != FMOE_OK) return rc;
   return launch_combine(y, weights, gamma, h, lw->norm_w, d.eps, T, d.top_k, d.hidden, h, xn, st);
 }
@@ -887,8 +919,10 @@ extern "C" int fmoe_expert_forward(const fmoe_layer_weights* lw, const float* d_
   const WsLayout w = ws_layout(d.hidden, d.inter, d.n_experts, d.top_k, T);
   if (ws_bytes < w.bytes) return FMOE_ERR_BUFFER_TOO_SMALL;
   float* a = reinterpret_cast<float*>(static_cast<unsigned char*>(d_ws) + w.a);
-  const GroupWork gw = group_work(static_cast<unsigned char*>(d_ws), w);
-  return launch_experts(expert_set(lw), d_xn, d_ids, T, a, d_y, lw->w_shared_gate, d_gamma, &gw, stream);
+  unsigned char* base = static_cast<unsigned char*>(d_ws);
+  const GroupWork gw = group_work(base, w);
+  return launch_experts(expert_set(lw), d_xn, d_ids, T, a, d_y, lw->w_shared_gate, d_gamma, &gw, base + w.tcx,
+                        base + w.tca, stream);
 }
 
 extern "C" int fmoe_combine_residual_rmsnorm(const float* d_y, const float* d_weights,
@@ -939,6 +973,12 @@ extern "C" int fmoe_pack_experts_device(const uint8_t* d_q, const uint16_t* d_sc
 extern "C" int fmoe_fused_supported(const fmoe_layer_desc* d) {
   if (!desc_valid(d) || !desc_supported(d)) return 0;
   return fused_config(*d).ok ? 1 : 0;
+}
+
+extern "C" int fmoe_set_tensor_cores(int enable) {
+  const int prev = g_tc_enabled;
+  g_tc_enabled = enable ? 1 : 0;
+  return prev;
 }
 
 extern "C" int fmoe_set_fused(int enable) {

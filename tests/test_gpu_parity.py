@@ -347,9 +347,10 @@ def test_layer_forward_is_deterministic_and_graph_capturable(full_layer):
     assert np.array_equal(host(h), outs[0][0]) and np.array_equal(host(xn), outs[0][1])
 
 
-def test_layer_forward_batched_zipf_routing(full_layer):
+def test_layer_forward_batched_zipf_routing(full_layer, tc_path):
     """64 tokens through one layer on Zipf(1)-popularity Gumbel-top-k routing
-    logits; 8 sampled tokens checked against the oracle."""
+    logits; 8 sampled tokens checked against the oracle (hot experts and the
+    shared expert on the tensor cores, or all on the integer-dot path)."""
     wl, lw, lw_o = full_layer
     T = 64
     lg, _ = synth.zipf_gumbel_logits(wl, 0, T)
@@ -367,12 +368,19 @@ def test_layer_forward_batched_zipf_routing(full_layer):
                           logits_given=True)
 
 
+@pytest.fixture(params=[True, False], ids=["tensor-cores", "integer-dot"])
+def tc_path(request):
+    prev = fm.fmoe_set_tensor_cores(request.param)
+    yield request.param
+    fm.fmoe_set_tensor_cores(prev)
+
+
 @pytest.mark.parametrize("wl", [SMALL, SMALL2], ids=["small4", "small2"])
-def test_grouped_experts_many_tokens_per_expert(wl):
+def test_grouped_experts_many_tokens_per_expert(wl, tc_path):
     """40 tokens all routed to the same four experts (given logits): every
-    group holds 40 slots, so the grouped path splits them into work items of
-    up to 16 tokens.  Tokens from each item, and the last one, are checked
-    against the oracle."""
+    group holds 40 slots -- a dense product on the tensor cores, or work
+    items of up to 16 tokens on the integer-dot path.  Tokens from each
+    item, and the last one, are checked against the oracle."""
     T = 40
     lw = device_layer(wl)
     lw_o = oracle_layer(wl, 0)
@@ -386,6 +394,29 @@ def test_grouped_experts_many_tokens_per_expert(wl):
         check_layer_token(wl, lw_o, ws, lw.desc, T, t, x[t], x[t], host(h)[t], host(xn)[t], f"t={t}",
                           logits_given=True)
     assert fm.fmoe_read_status() == 0
+
+
+def test_tensor_core_and_integer_paths_differ_only_by_rounding():
+    """The two implementations of the grouped products both run (their
+    results are not bit-identical) and agree well inside the tolerance."""
+    wl = SMALL
+    T = 40
+    lw = device_layer(wl)
+    lg = np.zeros((T, wl.n_experts), np.float32)
+    lg[:, [2, 5, 9, 13]] = [4.0, 3.0, 2.0, 1.0]
+    x = synth.tokens(wl, T, stream=44)
+    outs = {}
+    for tc in (True, False):
+        prev = fm.fmoe_set_tensor_cores(tc)
+        h, xn = dev(x), dev(x)
+        ws = fm.alloc_workspace(lw.desc, T)
+        fm.fmoe_layer_forward_logits(lw, dev(lg), h, xn, ws)
+        outs[tc] = (host(fm.workspace_view(ws, lw.desc, T, fm.WS_A)), host(fm.workspace_view(ws, lw.desc, T, fm.WS_Y)))
+        fm.fmoe_set_tensor_cores(prev)
+    for i in range(2):
+        a, b = outs[True][i], outs[False][i]
+        assert not np.array_equal(a, b)
+        assert np.linalg.norm(a - b) / np.linalg.norm(b) < 1e-3
 
 
 # ------------------------------------------------------------------- chains --
