@@ -44,7 +44,90 @@ def parse():
     ap.add_argument("--e2e-steps", type=int, default=None)
     ap.add_argument("--cpu-seconds", type=float, default=15.0, help="budget of the oracle CPU baseline sample")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-extra", action="store_true", help="skip the batched and 2-bit chain measurements")
     return ap.parse_args()
+
+
+def batched_measure(fm, synth, np, torch, lw, wl, stream, steps=50, warmup=5, T=64):
+    """64 tokens per step through one layer, top-4 drawn from Zipf(1) expert
+    popularity (fresh Gumbel-top-k logits every step, given as router
+    logits): tokens/s and the expert bytes the steps touch."""
+    logits = [torch.from_numpy(synth.zipf_gumbel_logits(wl, s, T)[0]).cuda() for s in range(steps)]
+    hot = []
+    for lg in logits:
+        ids = torch.topk(lg, wl.top_k, dim=1).indices.cpu().numpy()
+        cnt = np.bincount(ids.ravel(), minlength=wl.n_experts)
+        hot.append(((cnt > 0).sum(), (cnt >= 16).sum()))
+    x = torch.from_numpy(synth.tokens(wl, T, stream=900)).cuda()
+    h, xn = x.clone(), x.clone()
+    ws = fm.alloc_workspace(lw.desc, T)
+    with torch.cuda.stream(stream):
+        for s in range(warmup):
+            fm.fmoe_layer_forward_logits(lw, logits[s % steps], h, xn, ws, stream=stream)
+    torch.cuda.synchronize()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    with torch.cuda.stream(stream):
+        e0.record(stream)
+        for s in range(steps):
+            fm.fmoe_layer_forward_logits(lw, logits[s], h, xn, ws, stream=stream)
+        e1.record(stream)
+    e1.synchronize()
+    ms = e0.elapsed_time(e1)
+    rec = lw.desc.record_bytes()
+    distinct = float(np.mean([d for d, _ in hot]))
+    bytes_step = (distinct + 1) * rec  # routed experts touched + the shared expert
+    return {"workload": f"moe_layer_int4_batch{T}_zipf: {T} tokens per step through one 512-expert layer, Zipf(1) "
+                        f"top-4 routing (fresh Gumbel-top-k logits each step, given), {steps} steps",
+            "tokens_per_s": T * steps / (ms / 1e3), "ms_per_step": ms / steps,
+            "distinct_experts_per_step": distinct, "tensor_core_experts_per_step": float(np.mean([t for _, t in hot])) + 1,
+            "expert_weight_gbs": bytes_step * steps / (ms / 1e3) / 1e9,
+            "timing": "CUDA events on the launching stream, 50 consecutive steps"}
+
+
+def int2_chain_measure(fm, synth, torch, stream, layers=20, steps=2000, warmup=100):
+    """The 2-bit variant of the layer stack (routed experts 2-bit, shared
+    expert 4-bit), one token carried through all layers: layers/s."""
+    wl = synth.LAYER_INT2
+    scratch = {}
+    lws = [synth_device_upload(synth, wl, l, scratch) for l in range(layers)]
+    del scratch
+    torch.cuda.empty_cache()
+    x = torch.from_numpy(synth.tokens(wl, 1, stream=901)).cuda()
+    h, xn = x.clone(), x.clone()
+    ws = fm.alloc_workspace(lws[0].desc, 1)
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.stream(stream):
+        fm.fmoe_stack_forward(lws, h, xn, ws, stream=stream)
+        stream.synchronize()
+        with torch.cuda.graph(g, stream=stream):
+            fm.fmoe_stack_forward(lws, h, xn, ws, stream=stream)
+    torch.cuda.synchronize()
+    with torch.cuda.stream(stream):
+        for _ in range(max(1, warmup // layers)):
+            g.replay()
+    torch.cuda.synchronize()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    n = max(1, steps // layers)
+    with torch.cuda.stream(stream):
+        e0.record(stream)
+        for _ in range(n):
+            g.replay()
+        e1.record(stream)
+    e1.synchronize()
+    ms = e0.elapsed_time(e1)
+    d = lws[0].desc
+    layer_bytes = 4 * d.record_bytes() + d.record_bytes(shared=True) + wl.n_experts * wl.hidden * 4 + 2 * wl.hidden * 4
+    per_layer_s = ms / 1e3 / (n * layers)
+    del g
+    return {"workload": f"moe_stack_int2_batch1: {layers} resident layers, 2-bit routed experts (3.75 MiB), 4-bit "
+                        f"shared expert, one token carried through the stack",
+            "layer_fwd_per_s": 1 / per_layer_s, "tokens_per_s": 1 / per_layer_s / layers,
+            "layer_gbs": layer_bytes / per_layer_s / 1e9, "bytes_per_layer": layer_bytes}
+
+
+def synth_device_upload(synth, wl, layer, scratch):
+    from synth.device import upload_layer
+    return upload_layer(wl, layer, scratch=scratch)
 
 
 def workload_config(layers: int, experts: int = 512) -> dict:
@@ -346,6 +429,13 @@ def run_ours(args):
             "pct_of_8tbs_expert_bytes": 100 * expert_bytes / per_step_s / 8e12,
             "roofline": roofline, "e2e": e2e, "gpu_launches": launches,
             "clocks": clk.summary()}
+    line["tokens_per_s"] = value / L  # one token through the L-layer stack
+    if not args.no_extra and wl.n_experts == 512:
+        line["batched"] = batched_measure(fm, synth, np, torch, layers[0], wl, stream)
+        del layers, graphs, g_all
+        graphs = g_all = None
+        torch.cuda.empty_cache()
+        line["int2_chain"] = int2_chain_measure(fm, synth, torch, stream)
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         line["cpu_baseline"] = cpu_baseline(args.cpu_seconds, L)
     elif rank == 0:
