@@ -61,16 +61,21 @@ __global__ void __launch_bounds__(1024) group_kernel(const int32_t* __restrict__
   int* cnt = gsm;             // [E + 1]
   int* off = cnt + (E + 1);   // [E + 2]
   int* nit = off + (E + 2);   // [E + 2]: items per group, then their exclusive scan
+  int* grp = nit + (E + 2);   // [S]: group of each slot (-1: bad id)
   const int S = T * (k + 1);
   const int tid = threadIdx.x, nt = blockDim.x;
   for (int g = tid; g <= E; g += nt) cnt[g] = 0;
-  __syncthreads();
-  auto group_of = [&](int s) -> int {
+  for (int s = tid; s < S; s += nt) {
     const int t = s / (k + 1), j = s % (k + 1);
-    if (j == k) return E;
-    const int id = ids[(size_t)t * k + j];
-    return (id >= 0 && id < E) ? id : -1;
-  };
+    int g = E;
+    if (j < k) {
+      const int id = ids[(size_t)t * k + j];
+      g = (id >= 0 && id < E) ? id : -1;
+    }
+    grp[s] = g;
+  }
+  __syncthreads();
+  auto group_of = [&](int s) -> int { return grp[s]; };
   bool bad = false;
   for (int s = tid; s < S; s += nt) {
     const int g = group_of(s);

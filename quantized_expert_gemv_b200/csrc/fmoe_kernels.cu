@@ -608,8 +608,9 @@ static int launch_experts(const ExpertSet& es, const float* xn, const int32_t* i
   if (T >= 2 && gw) {
     const size_t sxs = (staged_x_bytes(es.H) + 15) & ~(size_t)15, sas = (staged_x_bytes(es.I) + 15) & ~(size_t)15;
     const size_t gu_smem = kGrpMaxM * sxs, dn_smem = kGrpMaxM * sas;
-    const size_t grp_smem = (size_t)(3 * es.E + 5) * 4;
-    if (gu_smem <= 200 * 1024 && dn_smem <= 200 * 1024 &&
+    const size_t grp_smem = (size_t)(3 * es.E + 5 + slots) * 4;
+    if (gu_smem <= 200 * 1024 && dn_smem <= 200 * 1024 && grp_smem <= 200 * 1024 &&
+        smem_optin(reinterpret_cast<const void*>(&group_kernel), grp_smem, 4) &&
         smem_optin(reinterpret_cast<const void*>(&gateup_group_kernel), gu_smem, 0) &&
         smem_optin(reinterpret_cast<const void*>(&down_group_kernel), dn_smem, 1)) {
       const int items = group_max_items(T, es.k, es.E);

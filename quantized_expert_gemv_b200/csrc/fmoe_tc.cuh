@@ -12,8 +12,9 @@
 //     memory (fp16, K-major core matrices of 8 rows x 16 bytes);
 //   - the staged X tile of that group arrives by one bulk copy;
 //   - one thread issues the four 128 x N x 16 tcgen05.mma of the group and
-//     commits them to the stage's mbarrier (two stages, so dequantising the
-//     next group overlaps the tensor cores);
+//     commits them to the stage's mbarrier (a ring of three stages, so
+//     dequantising the next groups overlaps the tensor cores; the raw
+//     weight words are loaded four groups ahead);
 //   - the epilogue reads the accumulator with tcgen05.ld (warp w: tensor
 //     memory lanes 32 (w % 4) ..), adds the hi and lo columns, and writes
 //     SwiGLU outputs (gate/up) or expert outputs (down).
@@ -99,7 +100,7 @@ __host__ __device__ __forceinline__ int tc_np(int m) { return (m + 7) / 8 * 8; }
 // byte it.w * 4 K (it.w: the items' running sum of Np).
 //   mode 0: token vectors src + (slot / (k + 1)) K   (normed inputs xn)
 //   mode 1: slot vectors  src + slot K               (SwiGLU outputs a)
-// With mode 0 the CTA of step 0 also computes gamma for the shared expert.
+// With mode 0 the CTAs also compute gamma for the shared expert's tokens.
 __global__ void __launch_bounds__(kTcThreads)
 tc_stage_kernel(GroupWork w, const float* __restrict__ src, int K, int k1, int mode, uint8_t* __restrict__ dst,
                 int E, const float* __restrict__ w_sg, float* __restrict__ gamma) {
@@ -126,9 +127,9 @@ tc_stage_kernel(GroupWork w, const float* __restrict__ src, int K, int k1, int m
     }
     *reinterpret_cast<uint4*>(base + (size_t)kc * (2 * np / 8) * 128 + (size_t)(row >> 3) * 128 + (row & 7) * 16) = out;
   }
-  if (mode == 0 && g == E && s == 0 && gamma) {
-    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    for (int i = warp; i < m; i += kTcThreads / 32) {
+  if (mode == 0 && g == E && gamma) {  // token i's gate in the CTA of step i % steps, one warp each
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31, steps = K / 64;
+    for (int i = s + steps * warp; i < m; i += steps * (kTcThreads / 32)) {
       const int t = slots[i] / k1;
       const float* x = src + (size_t)t * K;
       float z = 0.f;
@@ -173,20 +174,53 @@ __device__ __forceinline__ void sb_true(uint32_t sbw, int bits, float* s, float*
   *b = __uint_as_float(sbw & 0xFFFF0000u);
 }
 
-// Tile rows [r0, r0 + 128) of the gate/up matrix (packed rows: gate n, up n
-// interleaved), 64-group gi -> A tile.  Thread t: row t / 2, inputs
-// 32 (t % 2) .. + 31.
-template <int BITS>
-__device__ __forceinline__ void dequant_gu(const uint8_t* rec, int H, int I, int r0, int gi, uint8_t* a_tile) {
+// Raw words of one thread's share of a tile step: 16 bytes of codes (up to
+// four 32-bit words) and the scale-bias word.
+struct TcRaw {
+  uint4 c;
+  uint32_t sb;
+};
+
+// Thread t's share of 64-group gi of tile rows [r0, r0 + 128): row t / 2,
+// inputs 32 (t % 2) .. + 31.  MODE 0: gate/up rows (packed rows: gate n, up
+// n interleaved, row-major codes); MODE 1: down rows (column-block codes).
+template <int MODE, int BITS>
+__device__ __forceinline__ TcRaw tc_load_raw(const uint8_t* rec, int H, int I, int r0, int gi) {
   const RecordLayout L = record_layout(BITS, H, I);
-  const int t = threadIdx.x, r = t >> 1, hh = t & 1, ng = H / 64;
-  const int pr = r0 + r;
-  const uint8_t* row = rec + L.gu_codes + (size_t)pr * L.gu_row_bytes;
+  const int t = threadIdx.x, r = t >> 1, hh = t & 1;
+  TcRaw w;
+  if (MODE == 0) {
+    const int ng = H / 64, pr = r0 + r;
+    const uint8_t* row = rec + L.gu_codes + (size_t)pr * L.gu_row_bytes;
+    w.c = ld_stream(row + (BITS == 4 ? chunk_off<4>(ng, gi, hh) : chunk_off<2>(ng, gi, 0)));
+    if (BITS == 2 && hh) w.c = make_uint4(w.c.z, w.c.w, 0u, 0u);
+    w.sb = ld_stream_u32(reinterpret_cast<const uint32_t*>(rec + L.gu_sb) + (size_t)pr * ng + gi);
+  } else {
+    const int row = r0 + r;
+    const uint32_t* codes = reinterpret_cast<const uint32_t*>(rec + L.down_codes) + row;
+    if (BITS == 4) {  // words 8 gi + 4 hh .. + 3
+      w.c.x = ld_stream_u32(codes + (size_t)(8 * gi + 4 * hh + 0) * H);
+      w.c.y = ld_stream_u32(codes + (size_t)(8 * gi + 4 * hh + 1) * H);
+      w.c.z = ld_stream_u32(codes + (size_t)(8 * gi + 4 * hh + 2) * H);
+      w.c.w = ld_stream_u32(codes + (size_t)(8 * gi + 4 * hh + 3) * H);
+    } else {  // words 4 gi + 2 hh .. + 1
+      w.c.x = ld_stream_u32(codes + (size_t)(4 * gi + 2 * hh + 0) * H);
+      w.c.y = ld_stream_u32(codes + (size_t)(4 * gi + 2 * hh + 1) * H);
+      w.c.z = w.c.w = 0u;
+    }
+    w.sb = ld_stream_u32(reinterpret_cast<const uint32_t*>(rec + L.down_sb) + (size_t)gi * H + row);
+  }
+  return w;
+}
+
+// Dequantises a thread's share into the fp16 A tile.
+template <int BITS>
+__device__ __forceinline__ void tc_dequant(const TcRaw& w, uint8_t* a_tile) {
+  const int t = threadIdx.x, r = t >> 1, hh = t & 1;
   float s, b;
-  sb_true(ld_stream_u32(reinterpret_cast<const uint32_t*>(rec + L.gu_sb) + (size_t)pr * ng + gi), BITS, &s, &b);
+  sb_true(w.sb, BITS, &s, &b);
   if (BITS == 4) {
-    const uint4 c = ld_stream(row + chunk_off<4>(ng, gi, hh));
-    const uint32_t wd[4] = {c.x, c.y, c.z, c.w};
+    const uint32_t wd[4] = {w.c.x, w.c.y, w.c.z, w.c.w};
 #pragma unroll
     for (int q = 0; q < 4; ++q) {
       float w8[8];
@@ -194,8 +228,7 @@ __device__ __forceinline__ void dequant_gu(const uint8_t* rec, int H, int I, int
       store_a8(a_tile, r, 4 * hh + q, w8);
     }
   } else {
-    const uint4 c = ld_stream(row + chunk_off<2>(ng, gi, 0));
-    const uint32_t wd[2] = {hh ? c.z : c.x, hh ? c.w : c.y};
+    const uint32_t wd[2] = {w.c.x, w.c.y};
 #pragma unroll
     for (int q = 0; q < 2; ++q) {
       float w16[16];
@@ -206,114 +239,79 @@ __device__ __forceinline__ void dequant_gu(const uint8_t* rec, int H, int I, int
   }
 }
 
-// Tile rows [r0, r0 + 128) of the down matrix (column-block layout),
-// 64-group gi of the intermediate dimension -> A tile.
-template <int BITS>
-__device__ __forceinline__ void dequant_dn(const uint8_t* rec, int H, int I, int r0, int gi, uint8_t* a_tile) {
-  const RecordLayout L = record_layout(BITS, H, I);
-  const int t = threadIdx.x, r = t >> 1, hh = t & 1;
-  const int row = r0 + r;
-  const uint32_t* codes = reinterpret_cast<const uint32_t*>(rec + L.down_codes) + row;
-  float s, b;
-  sb_true(ld_stream_u32(reinterpret_cast<const uint32_t*>(rec + L.down_sb) + (size_t)gi * H + row), BITS, &s, &b);
-  if (BITS == 4) {  // words 8 gi + 4 hh .. + 3, 8 inputs each
-#pragma unroll
-    for (int q = 0; q < 4; ++q) {
-      float w8[8];
-      dequant_word4(ld_stream_u32(codes + (size_t)(8 * gi + 4 * hh + q) * H), s, b, w8);
-      store_a8(a_tile, r, 4 * hh + q, w8);
-    }
-  } else {  // words 4 gi + 2 hh .. + 1, 16 inputs each
-#pragma unroll
-    for (int q = 0; q < 2; ++q) {
-      float w16[16];
-      dequant_word2(ld_stream_u32(codes + (size_t)(4 * gi + 2 * hh + q) * H), s, b, w16);
-      store_a8(a_tile, r, 4 * hh + 2 * q, w16);
-      store_a8(a_tile, r, 4 * hh + 2 * q + 1, w16 + 8);
-    }
-  }
+// ------------------------------------------------------------- the GEMM --
+constexpr int kTcStages = 3;  // shared-memory ring of A and B tiles
+constexpr int kTcAhead = 4;   // steps of raw weight words held in registers ahead of use
+
+template <int MODE, int BITS>
+__device__ __forceinline__ TcRaw tc_raw_or_zero(const uint8_t* rec, int H, int I, int r0, int gi, int steps) {
+  if (gi < steps) return tc_load_raw<MODE, BITS>(rec, H, I, r0, gi);
+  TcRaw z;
+  z.c = make_uint4(0u, 0u, 0u, 0u);
+  z.sb = 0u;
+  return z;
 }
 
-// ------------------------------------------------------------- the GEMM --
 // grid (max tensor-core items, M / 128).  MODE 0: gate/up (M = 2 I, K = H),
 // epilogue SwiGLU -> a[slot][n].  MODE 1: down (M = H, K = I) -> y[slot][row].
-// Bounded waits: on expiry the CTA sets FMOE_STATUS_WAIT_TIMEOUT, waits
-// (bounded) for its committed products, frees its tensor memory and returns.
-template <int MODE>
-__global__ void __launch_bounds__(kTcThreads)
-tc_gemm_kernel(ExpertSet es, GroupWork w, const uint8_t* __restrict__ staged, float* __restrict__ out) {
-  extern __shared__ __align__(1024) unsigned char tsm[];
-  __shared__ uint64_t bar_b[2], bar_m[2];
-  __shared__ uint32_t s_tmem;
-  __shared__ int s_slot[kTcMaxNp];
-  __shared__ int s_ok;
-  if ((int)blockIdx.x >= w.n_items[1]) return;
-  const int4 it = w.tc[blockIdx.x];
-  const int g = it.x, m = it.z, np = tc_np(m), N = 2 * np;
+// Step s (one 64-input group) uses ring stage s % 3; completion c of a
+// stage's mbarriers belongs to step stage + 3 c, so every wait's parity is
+// (s / 3) & 1.  The token tile of step s is copied two steps ahead, the raw
+// weight words four steps ahead.  Bounded waits: on expiry the CTA sets
+// FMOE_STATUS_WAIT_TIMEOUT, waits (bounded) for its committed products,
+// frees its tensor memory and returns.
+template <int MODE, int BITS>
+__device__ __forceinline__ void tc_gemm_body(const ExpertSet& es, const int4 it, const uint8_t* rec,
+                                             const uint8_t* __restrict__ staged, float* __restrict__ out,
+                                             unsigned char* tsm, uint64_t* bar_b, uint64_t* bar_m, uint32_t tmem,
+                                             const int* s_slot, int* s_ok) {
+  const int m = it.z, np = tc_np(m), N = 2 * np;
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int K = MODE == 0 ? es.H : es.I;
   const int steps = K / 64;
   const int r0 = (int)blockIdx.y * kTcRows;
   const uint32_t b_bytes = (uint32_t)N * 128;  // one 64-input step of the staged tokens
-  uint8_t* a_st[2] = {tsm, tsm + kTcATile};
-  uint8_t* b_st[2] = {tsm + 2 * kTcATile, tsm + 2 * kTcATile + (uint32_t)kTcMaxNp * 2 * 128};
   const uint8_t* bsrc = staged + (size_t)it.w * 4 * K;
-  uint32_t ncols = 32;
-  while ((int)ncols < N) ncols <<= 1;
-
-  for (int i = tid; i < m; i += kTcThreads) s_slot[i] = w.slots[w.offset[g] + it.y + i];
-  if (tid == 0) {
-    s_ok = 1;
-    for (int i = 0; i < 2; ++i) {
-      mbar_init(&bar_b[i], 1);
-      mbar_init(&bar_m[i], 1);
-    }
-    asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
-  }
-  if (warp == 0) {
-    asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(smem_u32(&s_tmem)),
-                 "r"(ncols)
-                 : "memory");
-    asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::: "memory");
-  }
-  tc_fence_before();
-  __syncthreads();
-  tc_fence_after();
-  const uint32_t tmem = s_tmem;
-  int bits;
-  const uint8_t* rec = group_record(es, g, &bits);
+  auto a_st = [&](int st) { return tsm + (size_t)st * kTcATile; };
+  auto b_st = [&](int st) { return tsm + (size_t)kTcStages * kTcATile + (size_t)st * kTcMaxNp * 2 * 128; };
   const uint32_t idesc = umma_idesc_f16(kTcRows, N);
-  uint32_t ph_b = 0, ph_m = 0;  // parity bits per stage
-  int committed = 0;            // thread 0: products committed and not yet waited for (per stage bit)
+  auto par = [](int s) { return (uint32_t)((s / kTcStages) & 1); };
+  int last_commit = -1;  // thread 0: last step whose products were committed
+  int b_issued = -1, b_waited = -1;  // thread 0: token tiles requested / waited for
+  auto issue_b = [&](int s) {
+    const int st = s % kTcStages;
+    b_issued = s;
+    fence_proxy_async();
+    mbar_expect_tx(&bar_b[st], b_bytes);
+    bulk_g2s(b_st(st), bsrc + (size_t)s * b_bytes, b_bytes, &bar_b[st]);
+  };
+  if (tid == 0) {
+    issue_b(0);
+    if (steps > 1) issue_b(1);
+  }
+  // raw words of steps s, s + 1, s + 2, s + 3 in four fixed registers sets;
+  // each set is refilled with step s + 4 right after its use (no register
+  // moves, so a load stays in flight until its own step)
+  TcRaw rw[kTcAhead];
+#pragma unroll
+  for (int i = 0; i < kTcAhead; ++i) rw[i] = tc_raw_or_zero<MODE, BITS>(rec, es.H, es.I, r0, i, steps);
   bool ok = true;
-  for (int s = 0; s < steps && ok; ++s) {
-    const int st = s & 1;
-    if (s >= 2) {  // the products that read this stage are done
-      const bool done = mbar_wait(&bar_m[st], (ph_m >> st) & 1u);
-      ph_m ^= 1u << st;
-      if (tid == 0 && done) committed &= ~(1 << st);
-      if (!__syncthreads_and(done)) { ok = false; break; }
+  auto step = [&](int s, TcRaw& raw) -> bool {
+    const int st = s % kTcStages;
+    if (s >= kTcStages) {  // the products of step s - 3 read this stage
+      const bool done = mbar_wait(&bar_m[st], par(s - kTcStages));
+      if (!__syncthreads_and(done)) return false;
     }
-    if (tid == 0) {
-      fence_proxy_async();
-      mbar_expect_tx(&bar_b[st], b_bytes);
-      bulk_g2s(b_st[st], bsrc + (size_t)s * b_bytes, b_bytes, &bar_b[st]);
-    }
-    if (MODE == 0) {
-      if (bits == 4) dequant_gu<4>(rec, es.H, es.I, r0, s, a_st[st]);
-      else dequant_gu<2>(rec, es.H, es.I, r0, s, a_st[st]);
-    } else {
-      if (bits == 4) dequant_dn<4>(rec, es.H, es.I, r0, s, a_st[st]);
-      else dequant_dn<2>(rec, es.H, es.I, r0, s, a_st[st]);
-    }
+    tc_dequant<BITS>(raw, a_st(st));
+    raw = tc_raw_or_zero<MODE, BITS>(rec, es.H, es.I, r0, s + kTcAhead, steps);
     fence_proxy_async();  // the generic-proxy A tile is read by the tensor cores
     __syncthreads();
     if (tid == 0) {
-      const bool got = mbar_wait(&bar_b[st], (ph_b >> st) & 1u);
-      if (!got) s_ok = 0;
+      if (!mbar_wait(&bar_b[st], par(s))) *s_ok = 0;
       else {
+        b_waited = s;
         tc_fence_after();
-        const uint32_t a0 = smem_u32(a_st[st]), b0 = smem_u32(b_st[st]);
+        const uint32_t a0 = smem_u32(a_st(st)), b0 = smem_u32(b_st(st));
 #pragma unroll
         for (int j = 0; j < 4; ++j) {  // K = 16 slices: two 8-input chunks each
           const uint64_t ad = umma_desc(a0 + (uint32_t)(2 * j) * (kTcRows / 8) * 128, (kTcRows / 8) * 128, 128);
@@ -321,21 +319,25 @@ tc_gemm_kernel(ExpertSet es, GroupWork w, const uint8_t* __restrict__ staged, fl
           umma_f16(tmem, ad, bd, idesc, s > 0 || j > 0);
         }
         umma_commit(&bar_m[st]);
-        committed |= 1 << st;
+        last_commit = s;
+        // token tile of step s + 2: its stage was read by the products of step s - 1
+        if (s + 2 < steps) {
+          if (s >= 1 && !mbar_wait(&bar_m[(s + 2) % kTcStages], par(s - 1))) *s_ok = 0;
+          else issue_b(s + 2);
+        }
       }
     }
-    ph_b ^= 1u << st;
-    if (!__syncthreads_and(s_ok != 0)) ok = false;
+    return __syncthreads_and(*s_ok != 0);
+  };
+  for (int s = 0; s < steps && ok; s += kTcAhead) {
+#pragma unroll
+    for (int i = 0; i < kTcAhead; ++i)
+      if (ok && s + i < steps) ok = step(s + i, rw[i]);
   }
-  // the last products (one per stage still pending)
+  // the last products
   if (ok) {
-    for (int q = steps - 2 < 0 ? 0 : steps - 2; q < steps; ++q) {
-      const int st = q & 1;
-      const bool done = mbar_wait(&bar_m[st], (ph_m >> st) & 1u);
-      ph_m ^= 1u << st;
-      if (tid == 0 && done) committed &= ~(1 << st);
-      if (!__syncthreads_and(done)) { ok = false; break; }
-    }
+    const bool done = mbar_wait(&bar_m[(steps - 1) % kTcStages], par(steps - 1));
+    if (!__syncthreads_and(done)) ok = false;
   }
   tc_fence_after();
   if (ok) {
@@ -361,13 +363,52 @@ tc_gemm_kernel(ExpertSet es, GroupWork w, const uint8_t* __restrict__ staged, fl
         }
       }
     }
-  } else {
-    if (tid == 0) {
-      raise_status(FMOE_STATUS_WAIT_TIMEOUT);
-      for (int st = 0; st < 2; ++st)  // bounded wait for this CTA's committed products
-        if (committed & (1 << st)) (void)mbar_wait(&bar_m[st], (ph_m >> st) & 1u);
-    }
+  } else if (tid == 0) {
+    raise_status(FMOE_STATUS_WAIT_TIMEOUT);
+    if (last_commit >= 0)  // products complete in order: the last one covers the rest
+      (void)mbar_wait(&bar_m[last_commit % kTcStages], par(last_commit));
+    for (int q = b_waited + 1; q <= b_issued; ++q)  // token tiles still in flight
+      (void)mbar_wait(&bar_b[q % kTcStages], par(q));
   }
+}
+
+template <int MODE>
+__global__ void __launch_bounds__(kTcThreads)
+tc_gemm_kernel(ExpertSet es, GroupWork w, const uint8_t* __restrict__ staged, float* __restrict__ out) {
+  extern __shared__ __align__(1024) unsigned char tsm[];
+  __shared__ uint64_t bar_b[kTcStages], bar_m[kTcStages];
+  __shared__ uint32_t s_tmem;
+  __shared__ int s_slot[kTcMaxNp];
+  __shared__ int s_ok;
+  if ((int)blockIdx.x >= w.n_items[1]) return;
+  const int4 it = w.tc[blockIdx.x];
+  const int g = it.x, m = it.z, N = 2 * tc_np(m);
+  const int tid = threadIdx.x, warp = tid >> 5;
+  uint32_t ncols = 32;
+  while ((int)ncols < N) ncols <<= 1;
+  for (int i = tid; i < m; i += kTcThreads) s_slot[i] = w.slots[w.offset[g] + it.y + i];
+  if (tid == 0) {
+    s_ok = 1;
+    for (int i = 0; i < kTcStages; ++i) {
+      mbar_init(&bar_b[i], 1);
+      mbar_init(&bar_m[i], 1);
+    }
+    asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+  }
+  if (warp == 0) {
+    asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(smem_u32(&s_tmem)),
+                 "r"(ncols)
+                 : "memory");
+    asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::: "memory");
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = s_tmem;
+  int bits;
+  const uint8_t* rec = group_record(es, g, &bits);
+  if (bits == 4) tc_gemm_body<MODE, 4>(es, it, rec, staged, out, tsm, bar_b, bar_m, tmem, s_slot, &s_ok);
+  else tc_gemm_body<MODE, 2>(es, it, rec, staged, out, tsm, bar_b, bar_m, tmem, s_slot, &s_ok);
   tc_fence_before();
   __syncthreads();
   if (warp == 0) {
@@ -376,7 +417,7 @@ tc_gemm_kernel(ExpertSet es, GroupWork w, const uint8_t* __restrict__ staged, fl
   }
 }
 
-// Dynamic shared memory of tc_gemm_kernel: two A stages and two B stages.
-constexpr size_t tc_smem_bytes() { return 2 * (size_t)kTcATile + 2 * (size_t)kTcMaxNp * 2 * 128; }
+// Dynamic shared memory of tc_gemm_kernel: the ring of A and B tiles.
+constexpr size_t tc_smem_bytes() { return kTcStages * ((size_t)kTcATile + (size_t)kTcMaxNp * 2 * 128); }
 
 }  // namespace fmoe
