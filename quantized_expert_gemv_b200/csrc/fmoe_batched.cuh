@@ -26,6 +26,7 @@
 namespace fmoe {
 
 constexpr int kGrpMaxM = 16;      // tokens per GEMV work item
+constexpr int kGrpBuckets = 4;    // GEMV items by size: <= 2, <= 4, <= 8, <= 16 tokens
 constexpr int kTcItemMax = 128;   // tokens per tensor-core work item
 constexpr int kGrpThreads = 256;
 constexpr int kGuSplit = 16;      // CTAs per item over the gate/up row pairs
@@ -37,14 +38,19 @@ struct GroupWork {
   int* count;   // [E + 1] slots per group
   int* offset;  // [E + 2] first slot of each group in `slots`
   int* slots;   // [T (k + 1)] slot indices, grouped, in token order
-  int* n_items; // [2] GEMV work items, tensor-core work items
-  int4* items;  // [max_items] (group, first slot within the group, tokens, 0)
+  int* n_items; // [2 + kGrpBuckets] GEMV items, tensor-core items, GEMV items per size bucket
+  int4* items;  // [max_items] (group, first slot within the group, tokens, 0), by group
+  int4* bitems; // [kGrpBuckets][max_items] the GEMV items of each size bucket
   int4* tc;     // [max_tc]    (group, first, tokens, running sum of the items' tokens rounded up to 8)
 };
 
 __host__ __device__ constexpr int group_max_tc(int T, int k, int min_tokens) {
   return T * (k + 1) / min_tokens + T * (k + 1) / kTcItemMax + 2;
 }
+
+__host__ __device__ constexpr int grp_bucket_max(int b) { return 2 << b; }
+
+__device__ __forceinline__ int grp_bucket(int m) { return m <= 2 ? 0 : (m <= 4 ? 1 : (m <= 8 ? 2 : 3)); }
 
 __host__ __device__ constexpr int group_max_items(int T, int k, int E) {
   // one item per non-empty group plus one per further kGrpMaxM slots
@@ -109,15 +115,22 @@ __global__ void __launch_bounds__(1024) group_kernel(const int32_t* __restrict__
         }
     w.n_items[0] = it;
     w.n_items[1] = ntc;
+    for (int b = 0; b < kGrpBuckets; ++b) w.n_items[2 + b] = 0;
   }
   __syncthreads();
+  const int max_items = group_max_items(T, k, E);
   for (int g = tid; g <= E + 1; g += nt) w.offset[g] = off[g];
   for (int g = tid; g <= E; g += nt) {
     w.count[g] = cnt[g];
     const int c = cnt[g];
     if (c > 0 && !(tc_min > 0 && c >= tc_min))
-      for (int i = 0; i * kGrpMaxM < c; ++i)
-        w.items[nit[g] + i] = make_int4(g, i * kGrpMaxM, min(kGrpMaxM, c - i * kGrpMaxM), 0);
+      for (int i = 0; i * kGrpMaxM < c; ++i) {
+        const int mm = min(kGrpMaxM, c - i * kGrpMaxM), b = grp_bucket(mm);
+        const int4 item = make_int4(g, i * kGrpMaxM, mm, 0);
+        w.items[nit[g] + i] = item;
+        // bucket order does not matter: every item writes its own slots
+        w.bitems[(size_t)b * max_items + atomicAdd(&w.n_items[2 + b], 1)] = item;
+      }
   }
   // stable placement: rank of s = earlier slots of the same group
   for (int s = tid; s < S; s += nt) {
@@ -143,11 +156,18 @@ __device__ __forceinline__ StagedX staged_i(unsigned char* base, size_t stride, 
   return staged_x_at(base + (size_t)i * stride, K);
 }
 
-// Gate/up row pairs [p0, p1) of one record for the m tokens staged at sxb:
-// each warp takes row pairs; a lane owns whole groups of both rows of a
-// pair, loads their codes once and applies them to every token.
+// Stages every token's normed input once per step (int16 groups, the
+// layout of StagedX) at xs + t * stride.  grid T.
+__global__ void __launch_bounds__(kGrpThreads)
+stage_tokens_kernel(const float* __restrict__ xn, int H, unsigned char* __restrict__ xs, size_t stride) {
+  stage_x(xn + (size_t)blockIdx.x * H, H, staged_x_at(xs + blockIdx.x * stride, H));
+}
 
-template <int BITS>
+// Gate/up row pairs [p0, p1) of one record for the m <= MB tokens staged at
+// sxb: each warp takes PAIRS row pairs at a time (their code loads in flight
+// together); a lane owns whole groups of both rows of a pair, loads their
+// codes once and applies them to every token.
+template <int BITS, int MB, int PAIRS>
 __device__ __forceinline__ void gateup_rows_multi(const uint8_t* rec, const ExpertSet& es, unsigned char* sxb,
                                                   size_t sxs, int m, float* __restrict__ a, const int* slot_of,
                                                   int p0, int p1) {
@@ -158,62 +178,82 @@ __device__ __forceinline__ void gateup_rows_multi(const uint8_t* rec, const Expe
   const RecordLayout L = record_layout(BITS, H, es.I);
   const uint8_t* codes = rec + L.gu_codes;
   const uint32_t* sbw = reinterpret_cast<const uint32_t*>(rec + L.gu_sb);
-  for (int u = p0 / ppu + warp; u * ppu < p1; u += nw) {
-    const int n = u * ppu + ps;
-    const bool live = n < p1;
-    const int nn = live ? n : p1 - 1;
-    const uint8_t* rg = codes + (size_t)(2 * nn) * L.gu_row_bytes;
-    const uint8_t* ru = rg + L.gu_row_bytes;
-    float yg[kGrpMaxM], yu[kGrpMaxM];
+  for (int u0 = p0 / ppu + warp; u0 * ppu < p1; u0 += nw * PAIRS) {
+    float yg[PAIRS][MB], yu[PAIRS][MB];
 #pragma unroll
-    for (int i = 0; i < kGrpMaxM; ++i) yg[i] = yu[i] = 0.f;
+    for (int q = 0; q < PAIRS; ++q)
+#pragma unroll
+      for (int i = 0; i < MB; ++i) yg[q][i] = yu[q][i] = 0.f;
     for (int mm = 0; mm < gpl; ++mm) {
       const int g = lg + mm * lpr;
-      const GroupCodes<BITS> cg = load_group<BITS>(rg, ng, g);
-      const GroupCodes<BITS> cu = load_group<BITS>(ru, ng, g);
-      const uint32_t sg = ld_stream_u32(sbw + (size_t)(2 * nn) * ng + g);
-      const uint32_t su = ld_stream_u32(sbw + (size_t)(2 * nn + 1) * ng + g);
+      GroupCodes<BITS> cg[PAIRS], cu[PAIRS];
+      uint32_t sg[PAIRS], su[PAIRS];
 #pragma unroll
-      for (int i = 0; i < kGrpMaxM; ++i) {
+      for (int q = 0; q < PAIRS; ++q) {  // all loads of the PAIRS pairs first
+        const int n = (u0 + q * nw) * ppu + ps;
+        const int nn = n < p1 ? n : p1 - 1;
+        const uint8_t* rg = codes + (size_t)(2 * nn) * L.gu_row_bytes;
+        cg[q] = load_group<BITS>(rg, ng, g);
+        cu[q] = load_group<BITS>(rg + L.gu_row_bytes, ng, g);
+        sg[q] = ld_stream_u32(sbw + (size_t)(2 * nn) * ng + g);
+        su[q] = ld_stream_u32(sbw + (size_t)(2 * nn + 1) * ng + g);
+      }
+#pragma unroll
+      for (int i = 0; i < MB; ++i) {
         if (i < m) {
           const StagedX sx = staged_i(sxb, sxs, i, H);
           uint4 xv[8];
           load_xv(sx, ng, g, xv);
           const float d = sx.delta[g], xs = sx.xsum[g];
-          yg[i] = group_epilogue(yg[i], sg, group_dot<BITS>(cg, xv), d, xs);
-          yu[i] = group_epilogue(yu[i], su, group_dot<BITS>(cu, xv), d, xs);
+#pragma unroll
+          for (int q = 0; q < PAIRS; ++q) {
+            yg[q][i] = group_epilogue(yg[q][i], sg[q], group_dot<BITS>(cg[q], xv), d, xs);
+            yu[q][i] = group_epilogue(yu[q][i], su[q], group_dot<BITS>(cu[q], xv), d, xs);
+          }
         }
       }
     }
 #pragma unroll
-    for (int i = 0; i < kGrpMaxM; ++i) {
-      if (i < m) {
-        float g = yg[i], v = yu[i];
-        for (int o = lpr >> 1; o > 0; o >>= 1) {
-          g += __shfl_xor_sync(0xffffffffu, g, o);
-          v += __shfl_xor_sync(0xffffffffu, v, o);
+    for (int q = 0; q < PAIRS; ++q) {
+      const int n = (u0 + q * nw) * ppu + ps;
+#pragma unroll
+      for (int i = 0; i < MB; ++i) {
+        if (i < m) {
+          float g = yg[q][i], v = yu[q][i];
+          for (int o = lpr >> 1; o > 0; o >>= 1) {
+            g += __shfl_xor_sync(0xffffffffu, g, o);
+            v += __shfl_xor_sync(0xffffffffu, v, o);
+          }
+          if (lg == 0 && n < p1) a[(size_t)slot_of[i] * es.I + n] = silu_mul(g, v);
         }
-        if (lg == 0 && live) a[(size_t)slot_of[i] * es.I + n] = silu_mul(g, v);
       }
     }
   }
 }
 
-// grid (max items, kGuSplit).  Item (group, first, m): the group's slots
-// first .. first + m - 1.  Also computes gamma[t] = sigmoid(w_sg . xn[t])
-// for the shared expert's tokens when gamma is given.
-__global__ void __launch_bounds__(kGrpThreads)
-gateup_group_kernel(ExpertSet es, GroupWork w, const float* __restrict__ xn, float* __restrict__ a,
-                    const float* __restrict__ w_sg, float* __restrict__ gamma) {
+// grid (max items, kGuSplit), one size bucket of GEMV items (m <= MB).
+// Item (group, first, m): the group's slots first .. first + m - 1; the
+// tokens' staged inputs are copied from xs (stage_tokens_kernel).  Also
+// computes gamma[t] = sigmoid(w_sg . xn[t]) for the shared expert's tokens
+// when gamma is given.
+template <int MB>
+__global__ void __launch_bounds__(kGrpThreads, MB <= 4 ? 2 : 1)
+gateup_group_kernel(ExpertSet es, GroupWork w, int bucket, int max_items, const float* __restrict__ xn,
+                    const unsigned char* __restrict__ xs, float* __restrict__ a, const float* __restrict__ w_sg,
+                    float* __restrict__ gamma) {
   extern __shared__ __align__(128) unsigned char smem[];
   __shared__ int s_slot[kGrpMaxM];
-  if ((int)blockIdx.x >= w.n_items[0]) return;
-  const int4 it = w.items[blockIdx.x];
+  if ((int)blockIdx.x >= w.n_items[2 + bucket]) return;
+  const int4 it = w.bitems[(size_t)bucket * max_items + blockIdx.x];
   const int g = it.x, m = it.z, k1 = es.k + 1;
   if (threadIdx.x < m) s_slot[threadIdx.x] = w.slots[w.offset[g] + it.y + threadIdx.x];
   __syncthreads();
   const size_t sxs = (staged_x_bytes(es.H) + 15) & ~(size_t)15;
-  for (int i = 0; i < m; ++i) stage_x(xn + (size_t)(s_slot[i] / k1) * es.H, es.H, staged_i(smem, sxs, i, es.H));
+  for (int i = 0; i < m; ++i) {
+    const uint4* src = reinterpret_cast<const uint4*>(xs + (size_t)(s_slot[i] / k1) * sxs);
+    uint4* dst = reinterpret_cast<uint4*>(smem + (size_t)i * sxs);
+    for (int j = threadIdx.x; j < (int)(sxs / 16); j += kGrpThreads) dst[j] = __ldcg(src + j);
+  }
   __syncthreads();
   if (gamma && g == es.E && blockIdx.y == 0) {
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -241,16 +281,17 @@ gateup_group_kernel(ExpertSet es, GroupWork w, const float* __restrict__ xn, flo
   }
   int bits;
   const uint8_t* rec = group_record(es, g, &bits);
-  if (bits == 4) gateup_rows_multi<4>(rec, es, smem, sxs, m, a, s_slot, p0, p1);
-  else gateup_rows_multi<2>(rec, es, smem, sxs, m, a, s_slot, p0, p1);
+  constexpr int kPairs = MB <= 4 ? 2 : 1;
+  if (bits == 4) gateup_rows_multi<4, MB, kPairs>(rec, es, smem, sxs, m, a, s_slot, p0, p1);
+  else gateup_rows_multi<2, MB, kPairs>(rec, es, smem, sxs, m, a, s_slot, p0, p1);
 }
 
 // Down product of one record for one hidden row and the m tokens staged at
 // sx[0..m) (their SwiGLU outputs): the group's column-block words are loaded
 // once and applied to every token.
-template <int BITS>
+template <int BITS, int MB>
 __device__ __forceinline__ void down_row_multi(const uint8_t* rec, const ExpertSet& es, unsigned char* sab,
-                                               size_t sas, int m, int row, float (&yv)[kGrpMaxM]) {
+                                               size_t sas, int m, int row, float (&yv)[MB]) {
   const int H = es.H, I = es.I, ngI = I / 64;
   constexpr int kWpg = BITS == 4 ? 8 : 4;
   const RecordLayout L = record_layout(BITS, H, I);
@@ -262,7 +303,7 @@ __device__ __forceinline__ void down_row_multi(const uint8_t* rec, const ExpertS
     for (int b = 0; b < kWpg; ++b) wd[b] = ld_stream_u32(codes + (size_t)(g * kWpg + b) * H);
     const uint32_t sb = ld_stream_u32(sbw + (size_t)g * H);
 #pragma unroll
-    for (int i = 0; i < kGrpMaxM; ++i) {
+    for (int i = 0; i < MB; ++i) {
       if (i < m) {
         const StagedX sx = staged_i(sab, sas, i, I);
         int acc = 0;
@@ -277,13 +318,16 @@ __device__ __forceinline__ void down_row_multi(const uint8_t* rec, const ExpertS
   }
 }
 
-// grid (max items, H / kDnRows); one hidden row per thread.
+// grid (max items, H / kDnRows), one size bucket of GEMV items (m <= MB);
+// one hidden row per thread.
+template <int MB>
 __global__ void __launch_bounds__(kDnRows)
-down_group_kernel(ExpertSet es, GroupWork w, const float* __restrict__ a, float* __restrict__ y) {
+down_group_kernel(ExpertSet es, GroupWork w, int bucket, int max_items, const float* __restrict__ a,
+                  float* __restrict__ y) {
   extern __shared__ __align__(128) unsigned char smem[];
   __shared__ int s_slot[kGrpMaxM];
-  if ((int)blockIdx.x >= w.n_items[0]) return;
-  const int4 it = w.items[blockIdx.x];
+  if ((int)blockIdx.x >= w.n_items[2 + bucket]) return;
+  const int4 it = w.bitems[(size_t)bucket * max_items + blockIdx.x];
   const int g = it.x, m = it.z;
   if (threadIdx.x < m) s_slot[threadIdx.x] = w.slots[w.offset[g] + it.y + threadIdx.x];
   __syncthreads();
@@ -292,15 +336,15 @@ down_group_kernel(ExpertSet es, GroupWork w, const float* __restrict__ a, float*
   __syncthreads();
   const int row = (int)blockIdx.y * kDnRows + (int)threadIdx.x;
   if (row >= es.H) return;
-  float yv[kGrpMaxM];
+  float yv[MB];
 #pragma unroll
-  for (int i = 0; i < kGrpMaxM; ++i) yv[i] = 0.f;
+  for (int i = 0; i < MB; ++i) yv[i] = 0.f;
   int bits;
   const uint8_t* rec = group_record(es, g, &bits);
-  if (bits == 4) down_row_multi<4>(rec, es, smem, sas, m, row, yv);
-  else down_row_multi<2>(rec, es, smem, sas, m, row, yv);
+  if (bits == 4) down_row_multi<4, MB>(rec, es, smem, sas, m, row, yv);
+  else down_row_multi<2, MB>(rec, es, smem, sas, m, row, yv);
 #pragma unroll
-  for (int i = 0; i < kGrpMaxM; ++i)
+  for (int i = 0; i < MB; ++i)
     if (i < m) y[(size_t)s_slot[i] * es.H + row] = yv[i];
 }
 

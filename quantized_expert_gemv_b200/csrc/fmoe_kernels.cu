@@ -468,7 +468,7 @@ __global__ void pack_sb_kernel(const uint16_t* __restrict__ scale, const uint16_
 // ------------------------------------------------------- host helpers ----
 struct WsLayout {
   size_t sync, ss, x_logit, x_part, grp, part, logits, ids, weights, gamma, a, y, bytes;
-  size_t g_count, g_offset, g_slots, g_nitems, g_items, g_tc;  // inside grp
+  size_t g_count, g_offset, g_slots, g_nitems, g_items, g_bitems, g_tc, g_xs;  // inside grp
   size_t tcx, tca;  // staged fp16 inputs of the tensor-core items (0 bytes when T < kTcMinTokens)
 };
 
@@ -501,9 +501,13 @@ static WsLayout ws_layout(int H, int I, int E, int k, int T) {
   w.g_slots = o;
   o = align_up(o + (size_t)T * (k + 1) * 4, 16);
   w.g_nitems = o;
-  o = align_up(o + 16, 16);
+  o = align_up(o + 4 * (2 + kGrpBuckets), 16);
   w.g_items = o;
   o = align_up(o + (size_t)group_max_items(T, k, E) * 16, 16);
+  w.g_bitems = o;
+  o = align_up(o + (size_t)kGrpBuckets * group_max_items(T, k, E) * 16, 16);
+  w.g_xs = o;  // every token's staged input (T > 1)
+  o = align_up(o + (T > 1 ? (size_t)T * ((staged_x_bytes(H) + 15) & ~(size_t)15) : 0), 16);
   w.g_tc = o;
   o = align_up(o + (size_t)group_max_tc(T, k, kTcMinTokens) * 16, 256);
   w.tcx = o;
@@ -601,18 +605,39 @@ static bool smem_optin(const void* fn, size_t bytes, int slot) {
 // Expert forward of T tokens.  With T >= 2 and a group workspace the slots
 // are grouped by expert first (each expert's weights read once per step);
 // otherwise one CTA column per slot.
+template <int MB>
+static bool grp_optin(size_t gu_smem, size_t dn_smem, int b) {
+  return smem_optin(reinterpret_cast<const void*>(&gateup_group_kernel<MB>), gu_smem, 8 + b) &&
+         smem_optin(reinterpret_cast<const void*>(&down_group_kernel<MB>), dn_smem, 12 + b);
+}
+
+template <int MB>
+static void grp_launch_gu(const ExpertSet& es, const GroupWork& gw, int b, int items, const float* xn,
+                          const unsigned char* xs, float* a, const float* w_sg, float* gamma, size_t sxs,
+                          cudaStream_t st) {
+  gateup_group_kernel<MB><<<dim3(items, kGuSplit), kGrpThreads, MB * sxs, st>>>(es, gw, b, items, xn, xs, a, w_sg,
+                                                                              gamma);
+}
+
+template <int MB>
+static void grp_launch_dn(const ExpertSet& es, const GroupWork& gw, int b, int items, const float* a, float* y,
+                          size_t sas, cudaStream_t st) {
+  down_group_kernel<MB><<<dim3(items, (es.H + kDnRows - 1) / kDnRows), kDnRows, MB * sas, st>>>(es, gw, b, items, a,
+                                                                                                  y);
+}
+
 static int launch_experts(const ExpertSet& es, const float* xn, const int32_t* ids, int T, float* a,
                           float* y, const float* w_sg, float* gamma, const GroupWork* gw, uint8_t* tcx,
-                          uint8_t* tca, cudaStream_t st) {
+                          uint8_t* tca, unsigned char* xs, cudaStream_t st) {
   const int slots = T * (es.k + 1);
   if (T >= 2 && gw) {
     const size_t sxs = (staged_x_bytes(es.H) + 15) & ~(size_t)15, sas = (staged_x_bytes(es.I) + 15) & ~(size_t)15;
     const size_t gu_smem = kGrpMaxM * sxs, dn_smem = kGrpMaxM * sas;
     const size_t grp_smem = (size_t)(3 * es.E + 5 + slots) * 4;
-    if (gu_smem <= 200 * 1024 && dn_smem <= 200 * 1024 && grp_smem <= 200 * 1024 &&
-        smem_optin(reinterpret_cast<const void*>(&group_kernel), grp_smem, 4) &&
-        smem_optin(reinterpret_cast<const void*>(&gateup_group_kernel), gu_smem, 0) &&
-        smem_optin(reinterpret_cast<const void*>(&down_group_kernel), dn_smem, 1)) {
+    if (xs && gu_smem <= 200 * 1024 && dn_smem <= 200 * 1024 && grp_smem <= 200 * 1024 &&
+        smem_optin(reinterpret_cast<const void*>(&group_kernel), grp_smem, 4) && grp_optin<2>(2 * sxs, 2 * sas, 0) &&
+        grp_optin<4>(4 * sxs, 4 * sas, 1) && grp_optin<8>(8 * sxs, 8 * sas, 2) &&
+        grp_optin<16>(16 * sxs, 16 * sas, 3)) {
       const int items = group_max_items(T, es.k, es.E);
       // groups of >= kTcMinTokens tokens go to the tensor cores when the shape tiles
       const bool tc = g_tc_enabled && T >= kTcMinTokens && tcx && tca && es.H % kTcRows == 0 &&
@@ -621,17 +646,24 @@ static int launch_experts(const ExpertSet& es, const float* xn, const int32_t* i
                       smem_optin(reinterpret_cast<const void*>(&tc_gemm_kernel<1>), tc_smem_bytes(), 3);
       const int max_tc = group_max_tc(T, es.k, kTcMinTokens);
       group_kernel<<<1, 1024, grp_smem, st>>>(ids, T, es.k, es.E, es.I, es.H, tc ? kTcMinTokens : 0, *gw, a, y);
-      gateup_group_kernel<<<dim3(items, kGuSplit), kGrpThreads, gu_smem, st>>>(es, *gw, xn, a, w_sg, gamma);
+      stage_tokens_kernel<<<T, kGrpThreads, 0, st>>>(xn, es.H, xs, sxs);
+      grp_launch_gu<2>(es, *gw, 0, items, xn, xs, a, w_sg, gamma, sxs, st);
+      grp_launch_gu<4>(es, *gw, 1, items, xn, xs, a, w_sg, gamma, sxs, st);
+      grp_launch_gu<8>(es, *gw, 2, items, xn, xs, a, w_sg, gamma, sxs, st);
+      grp_launch_gu<16>(es, *gw, 3, items, xn, xs, a, w_sg, gamma, sxs, st);
       if (tc) {
         tc_stage_kernel<<<dim3(max_tc, es.H / 64), kTcThreads, 0, st>>>(*gw, xn, es.H, es.k + 1, 0, tcx, es.E, w_sg,
                                                                       gamma);
-        tc_gemm_kernel<0><<<dim3(max_tc, 2 * es.I / kTcRows), kTcThreads, tc_smem_bytes(), st>>>(es, *gw, tcx, a);
+        tc_gemm_kernel<0><<<dim3(max_tc, 2 * es.I / kTcRows), kTcThreads + 32, tc_smem_bytes(), st>>>(es, *gw, tcx, a);
       }
-      down_group_kernel<<<dim3(items, (es.H + kDnRows - 1) / kDnRows), kDnRows, dn_smem, st>>>(es, *gw, a, y);
+      grp_launch_dn<2>(es, *gw, 0, items, a, y, sas, st);
+      grp_launch_dn<4>(es, *gw, 1, items, a, y, sas, st);
+      grp_launch_dn<8>(es, *gw, 2, items, a, y, sas, st);
+      grp_launch_dn<16>(es, *gw, 3, items, a, y, sas, st);
       if (tc) {
         tc_stage_kernel<<<dim3(max_tc, es.I / 64), kTcThreads, 0, st>>>(*gw, a, es.I, es.k + 1, 1, tca, es.E, nullptr,
                                                                       nullptr);
-        tc_gemm_kernel<1><<<dim3(max_tc, es.H / kTcRows), kTcThreads, tc_smem_bytes(), st>>>(es, *gw, tca, y);
+        tc_gemm_kernel<1><<<dim3(max_tc, es.H / kTcRows), kTcThreads + 32, tc_smem_bytes(), st>>>(es, *gw, tca, y);
       }
       return cuda_rc(cudaGetLastError());
     }
@@ -793,6 +825,7 @@ static GroupWork group_work(unsigned char* base, const WsLayout& w) {
   g.slots = reinterpret_cast<int*>(base + w.g_slots);
   g.n_items = reinterpret_cast<int*>(base + w.g_nitems);
   g.items = reinterpret_cast<int4*>(base + w.g_items);
+  g.bitems = reinterpret_cast<int4*>(base + w.g_bitems);
   g.tc = reinterpret_cast<int4*>(base + w.g_tc);
   return g;
 }
@@ -832,7 +865,7 @@ static int layer_forward_impl(const fmoe_layer_weights* lw, const float* logits_
   if (rc != FMOE_OK) return rc;
   const GroupWork gw = group_work(base, w);
   rc = launch_experts(es, xn, ids, T, a, y, lw->w_shared_gate, logits_in ? gamma : nullptr, &gw, base + w.tcx,
-                      base + w.tca, st);
+                      base + w.tca, T > 1 ? base + w.g_xs : nullptr, st);
   if (rc != FMOE_OK) return rc;
   return launch_combine(y, weights, gamma, h, lw->norm_w, d.eps, T, d.top_k, d.hidden, h, xn, st);
 }
@@ -923,7 +956,7 @@ extern "C" int fmoe_expert_forward(const fmoe_layer_weights* lw, const float* d_
   unsigned char* base = static_cast<unsigned char*>(d_ws);
   const GroupWork gw = group_work(base, w);
   return launch_experts(expert_set(lw), d_xn, d_ids, T, a, d_y, lw->w_shared_gate, d_gamma, &gw, base + w.tcx,
-                        base + w.tca, stream);
+                        base + w.tca, T > 1 ? base + w.g_xs : nullptr, stream);
 }
 
 extern "C" int fmoe_combine_residual_rmsnorm(const float* d_y, const float* d_weights,

@@ -252,19 +252,25 @@ __device__ __forceinline__ TcRaw tc_raw_or_zero(const uint8_t* rec, int H, int I
   return z;
 }
 
-// grid (max tensor-core items, M / 128).  MODE 0: gate/up (M = 2 I, K = H),
-// epilogue SwiGLU -> a[slot][n].  MODE 1: down (M = H, K = I) -> y[slot][row].
-// Step s (one 64-input group) uses ring stage s % 3; completion c of a
-// stage's mbarriers belongs to step stage + 3 c, so every wait's parity is
-// (s / 3) & 1.  The token tile of step s is copied two steps ahead, the raw
-// weight words four steps ahead.  Bounded waits: on expiry the CTA sets
-// FMOE_STATUS_WAIT_TIMEOUT, waits (bounded) for its committed products,
-// frees its tensor memory and returns.
+__device__ __forceinline__ void mbar_arrive(uint64_t* bar) {
+  asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(smem_u32(bar)) : "memory");
+}
+
+// grid (max tensor-core items, M / 128), kTcThreads + 32 threads.  MODE 0:
+// gate/up (M = 2 I, K = H), epilogue SwiGLU -> a[slot][n].  MODE 1: down
+// (M = H, K = I) -> y[slot][row].  Warps 0..7 dequantise step s (one
+// 64-input group) into ring stage s % 3 and arrive on full[stage]; warp 8
+// (one thread) waits for the stage's A and token tile, issues the four
+// products, commits them to done[stage] and requests the token tile of step
+// s + 2.  Completion c of a stage's mbarriers belongs to step stage + 3 c,
+// so every wait's parity is (s / 3) & 1.  Bounded waits: on expiry the CTA
+// sets FMOE_STATUS_WAIT_TIMEOUT, waits (bounded) for its committed products
+// and copies, frees its tensor memory and returns.
 template <int MODE, int BITS>
 __device__ __forceinline__ void tc_gemm_body(const ExpertSet& es, const int4 it, const uint8_t* rec,
                                              const uint8_t* __restrict__ staged, float* __restrict__ out,
-                                             unsigned char* tsm, uint64_t* bar_b, uint64_t* bar_m, uint32_t tmem,
-                                             const int* s_slot, int* s_ok) {
+                                             unsigned char* tsm, uint64_t* bar_b, uint64_t* bar_m, uint64_t* bar_f,
+                                             uint32_t tmem, const int* s_slot, int* s_ok) {
   const int m = it.z, np = tc_np(m), N = 2 * np;
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int K = MODE == 0 ? es.H : es.I;
@@ -274,73 +280,89 @@ __device__ __forceinline__ void tc_gemm_body(const ExpertSet& es, const int4 it,
   const uint8_t* bsrc = staged + (size_t)it.w * 4 * K;
   auto a_st = [&](int st) { return tsm + (size_t)st * kTcATile; };
   auto b_st = [&](int st) { return tsm + (size_t)kTcStages * kTcATile + (size_t)st * kTcMaxNp * 2 * 128; };
-  const uint32_t idesc = umma_idesc_f16(kTcRows, N);
   auto par = [](int s) { return (uint32_t)((s / kTcStages) & 1); };
-  int last_commit = -1;  // thread 0: last step whose products were committed
-  int b_issued = -1, b_waited = -1;  // thread 0: token tiles requested / waited for
-  auto issue_b = [&](int s) {
-    const int st = s % kTcStages;
-    b_issued = s;
-    fence_proxy_async();
-    mbar_expect_tx(&bar_b[st], b_bytes);
-    bulk_g2s(b_st(st), bsrc + (size_t)s * b_bytes, b_bytes, &bar_b[st]);
-  };
-  if (tid == 0) {
-    issue_b(0);
-    if (steps > 1) issue_b(1);
-  }
-  // raw words of steps s, s + 1, s + 2, s + 3 in four fixed registers sets;
-  // each set is refilled with step s + 4 right after its use (no register
-  // moves, so a load stays in flight until its own step)
-  TcRaw rw[kTcAhead];
+  if (warp < kTcThreads / 32) {
+    // ---- producers: raw words of steps s .. s + 3 in four fixed register
+    // sets, each refilled with step s + 4 right after its use
+    TcRaw rw[kTcAhead];
 #pragma unroll
-  for (int i = 0; i < kTcAhead; ++i) rw[i] = tc_raw_or_zero<MODE, BITS>(rec, es.H, es.I, r0, i, steps);
-  bool ok = true;
-  auto step = [&](int s, TcRaw& raw) -> bool {
-    const int st = s % kTcStages;
-    if (s >= kTcStages) {  // the products of step s - 3 read this stage
-      const bool done = mbar_wait(&bar_m[st], par(s - kTcStages));
-      if (!__syncthreads_and(done)) return false;
-    }
-    tc_dequant<BITS>(raw, a_st(st));
-    raw = tc_raw_or_zero<MODE, BITS>(rec, es.H, es.I, r0, s + kTcAhead, steps);
-    fence_proxy_async();  // the generic-proxy A tile is read by the tensor cores
-    __syncthreads();
-    if (tid == 0) {
-      if (!mbar_wait(&bar_b[st], par(s))) *s_ok = 0;
-      else {
-        b_waited = s;
-        tc_fence_after();
-        const uint32_t a0 = smem_u32(a_st(st)), b0 = smem_u32(b_st(st));
+    for (int i = 0; i < kTcAhead; ++i) rw[i] = tc_raw_or_zero<MODE, BITS>(rec, es.H, es.I, r0, i, steps);
+    bool ok = true;
+    for (int s0 = 0; s0 < steps && ok; s0 += kTcAhead) {
 #pragma unroll
-        for (int j = 0; j < 4; ++j) {  // K = 16 slices: two 8-input chunks each
-          const uint64_t ad = umma_desc(a0 + (uint32_t)(2 * j) * (kTcRows / 8) * 128, (kTcRows / 8) * 128, 128);
-          const uint64_t bd = umma_desc(b0 + (uint32_t)(2 * j) * (uint32_t)(N / 8) * 128, (uint32_t)(N / 8) * 128, 128);
-          umma_f16(tmem, ad, bd, idesc, s > 0 || j > 0);
+      for (int i = 0; i < kTcAhead; ++i) {
+        const int s = s0 + i;
+        if (!ok || s >= steps) break;
+        const int st = s % kTcStages;
+        if (s >= kTcStages && !mbar_wait(&bar_m[st], par(s - kTcStages))) {  // products of step s - 3 done
+          ok = false;
+          *s_ok = 0;
+          break;
         }
-        umma_commit(&bar_m[st]);
-        last_commit = s;
-        // token tile of step s + 2: its stage was read by the products of step s - 1
-        if (s + 2 < steps) {
-          if (s >= 1 && !mbar_wait(&bar_m[(s + 2) % kTcStages], par(s - 1))) *s_ok = 0;
-          else issue_b(s + 2);
-        }
+        tc_dequant<BITS>(rw[i], a_st(st));
+        rw[i] = tc_raw_or_zero<MODE, BITS>(rec, es.H, es.I, r0, s + kTcAhead, steps);
+        fence_proxy_async();  // the generic-proxy A tile is read by the tensor cores
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&bar_f[st]);
       }
     }
-    return __syncthreads_and(*s_ok != 0);
-  };
-  for (int s = 0; s < steps && ok; s += kTcAhead) {
+  } else if (lane == 0) {
+    // ---- issuer
+    const uint32_t idesc = umma_idesc_f16(kTcRows, N);
+    int last_commit = -1, b_issued = -1, b_waited = -1;
+    auto issue_b = [&](int s) {
+      const int st = s % kTcStages;
+      b_issued = s;
+      mbar_expect_tx(&bar_b[st], b_bytes);
+      bulk_g2s(b_st(st), bsrc + (size_t)s * b_bytes, b_bytes, &bar_b[st]);
+    };
+    issue_b(0);
+    if (steps > 1) issue_b(1);
+    bool ok = true;
+    for (int s = 0; s < steps; ++s) {
+      const int st = s % kTcStages;
+      if (!mbar_wait(&bar_f[st], par(s)) || !mbar_wait(&bar_b[st], par(s))) {
+        ok = false;
+        break;
+      }
+      b_waited = s;
+      tc_fence_after();
+      const uint32_t a0 = smem_u32(a_st(st)), b0 = smem_u32(b_st(st));
 #pragma unroll
-    for (int i = 0; i < kTcAhead; ++i)
-      if (ok && s + i < steps) ok = step(s + i, rw[i]);
+      for (int j = 0; j < 4; ++j) {  // K = 16 slices: two 8-input chunks each
+        const uint64_t ad = umma_desc(a0 + (uint32_t)(2 * j) * (kTcRows / 8) * 128, (kTcRows / 8) * 128, 128);
+        const uint64_t bd = umma_desc(b0 + (uint32_t)(2 * j) * (uint32_t)(N / 8) * 128, (uint32_t)(N / 8) * 128, 128);
+        umma_f16(tmem, ad, bd, idesc, s > 0 || j > 0);
+      }
+      umma_commit(&bar_m[st]);
+      last_commit = s;
+      // token tile of step s + 2: its stage was read by the products of step s - 1
+      if (s + 2 < steps) {
+        if (s >= 1 && !mbar_wait(&bar_m[(s + 2) % kTcStages], par(s - 1))) {
+          ok = false;
+          break;
+        }
+        issue_b(s + 2);
+      }
+    }
+    if (!ok) {
+      *s_ok = 0;
+      if (last_commit >= 0)  // products complete in order: the last one covers the rest
+        (void)mbar_wait(&bar_m[last_commit % kTcStages], par(last_commit));
+      for (int q = b_waited + 1; q <= b_issued; ++q)  // token tiles still in flight
+        (void)mbar_wait(&bar_b[q % kTcStages], par(q));
+    }
   }
-  // the last products
-  if (ok) {
+  __syncthreads();
+  bool ok = *s_ok != 0;
+  if (ok) {  // the last products
     const bool done = mbar_wait(&bar_m[(steps - 1) % kTcStages], par(steps - 1));
-    if (!__syncthreads_and(done)) ok = false;
+    ok = __syncthreads_and(done);
+  } else {
+    __syncthreads_and(false);
   }
   tc_fence_after();
-  if (ok) {
+  if (ok && warp < kTcThreads / 32) {
     // epilogue: warp w reads lanes 32 (w % 4) .. (tile rows), tokens split
     // between warps w and w + 4 in chunks of 8 columns
     const int q4 = warp & 3, half = warp >> 2;
@@ -363,20 +385,15 @@ __device__ __forceinline__ void tc_gemm_body(const ExpertSet& es, const int4 it,
         }
       }
     }
-  } else if (tid == 0) {
-    raise_status(FMOE_STATUS_WAIT_TIMEOUT);
-    if (last_commit >= 0)  // products complete in order: the last one covers the rest
-      (void)mbar_wait(&bar_m[last_commit % kTcStages], par(last_commit));
-    for (int q = b_waited + 1; q <= b_issued; ++q)  // token tiles still in flight
-      (void)mbar_wait(&bar_b[q % kTcStages], par(q));
   }
+  if (!ok && tid == 0) raise_status(FMOE_STATUS_WAIT_TIMEOUT);
 }
 
 template <int MODE>
-__global__ void __launch_bounds__(kTcThreads)
+__global__ void __launch_bounds__(kTcThreads + 32)
 tc_gemm_kernel(ExpertSet es, GroupWork w, const uint8_t* __restrict__ staged, float* __restrict__ out) {
   extern __shared__ __align__(1024) unsigned char tsm[];
-  __shared__ uint64_t bar_b[kTcStages], bar_m[kTcStages];
+  __shared__ uint64_t bar_b[kTcStages], bar_m[kTcStages], bar_f[kTcStages];
   __shared__ uint32_t s_tmem;
   __shared__ int s_slot[kTcMaxNp];
   __shared__ int s_ok;
@@ -386,12 +403,13 @@ tc_gemm_kernel(ExpertSet es, GroupWork w, const uint8_t* __restrict__ staged, fl
   const int tid = threadIdx.x, warp = tid >> 5;
   uint32_t ncols = 32;
   while ((int)ncols < N) ncols <<= 1;
-  for (int i = tid; i < m; i += kTcThreads) s_slot[i] = w.slots[w.offset[g] + it.y + i];
+  for (int i = tid; i < m; i += blockDim.x) s_slot[i] = w.slots[w.offset[g] + it.y + i];
   if (tid == 0) {
     s_ok = 1;
     for (int i = 0; i < kTcStages; ++i) {
       mbar_init(&bar_b[i], 1);
       mbar_init(&bar_m[i], 1);
+      mbar_init(&bar_f[i], kTcThreads / 32);
     }
     asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
   }
@@ -407,8 +425,8 @@ tc_gemm_kernel(ExpertSet es, GroupWork w, const uint8_t* __restrict__ staged, fl
   const uint32_t tmem = s_tmem;
   int bits;
   const uint8_t* rec = group_record(es, g, &bits);
-  if (bits == 4) tc_gemm_body<MODE, 4>(es, it, rec, staged, out, tsm, bar_b, bar_m, tmem, s_slot, &s_ok);
-  else tc_gemm_body<MODE, 2>(es, it, rec, staged, out, tsm, bar_b, bar_m, tmem, s_slot, &s_ok);
+  if (bits == 4) tc_gemm_body<MODE, 4>(es, it, rec, staged, out, tsm, bar_b, bar_m, bar_f, tmem, s_slot, &s_ok);
+  else tc_gemm_body<MODE, 2>(es, it, rec, staged, out, tsm, bar_b, bar_m, bar_f, tmem, s_slot, &s_ok);
   tc_fence_before();
   __syncthreads();
   if (warp == 0) {
