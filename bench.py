@@ -45,6 +45,7 @@ def parse():
     ap.add_argument("--cpu-seconds", type=float, default=15.0, help="budget of the oracle CPU baseline sample")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-extra", action="store_true", help="skip the batched and 2-bit chain measurements")
+    ap.add_argument("--int2-layers", type=int, default=20, help="resident 2-bit layers of the 2-bit chain (0: skip)")
     return ap.parse_args()
 
 
@@ -138,6 +139,24 @@ def workload_config(layers: int, experts: int = 512) -> dict:
         "batch": 1, "layer_copies": layers,
         "l2": f"inputs larger than L2: rotation over {layers} resident layers ({layers * 43.8:.0f} MB of weights per rotation)",
     }
+
+
+# DRAM bytes (read + write) of one full-size int4 layer of fused_stack_kernel,
+# from an ncu capture (profiles/fused_stack_kernel_int4_batch1.md), valid for
+# the kernel sources whose digest is given; any later change to them voids it.
+TRAFFIC_PER_LAYER = {"sources_sha256_16": "3cab5dcca312ed9a", "bytes": 43_963_392}
+TRAFFIC_SOURCES = ("fmoe_fused.cuh", "fmoe_device.cuh", "fmoe_layout.h")
+
+
+def measured_traffic(layers: int):
+    import hashlib
+    h = hashlib.sha256()
+    for f in TRAFFIC_SOURCES:
+        with open(os.path.join(ROOT, "quantized_expert_gemv_b200", "csrc", f), "rb") as fh:
+            h.update(fh.read())
+    if h.hexdigest()[:16] != TRAFFIC_PER_LAYER["sources_sha256_16"]:
+        return None
+    return TRAFFIC_PER_LAYER["bytes"] * layers
 
 
 def measured_peak():
@@ -383,7 +402,10 @@ def run_ours(args):
                 "kernel": f"fused_stack_kernel: whole layers (router, top-k, gate/up+SwiGLU, down, combine+RMSNorm), "
                           f"{L} layers per launch",
                 "achieved": achieved, "peak": peak, "peak_kind": peak_kind, "unit": "GB/s",
-                "frac": achieved / peak, "traffic": None,
+                "frac": achieved / peak,
+                "traffic": measured_traffic(L) if wl.n_experts == 512 else None,
+                "traffic_note": "ncu dram__bytes_read.sum + dram__bytes_write.sum of one full-size layer launch, "
+                                "times the layers per launch (per-layer traffic is additive)",
                 "bytes_per_layer": layer_bytes, "layers_per_launch": L,
                 "timing": "CUDA events on the launching stream around the timed replays"}
 
@@ -435,7 +457,8 @@ def run_ours(args):
         del layers, graphs, g_all
         graphs = g_all = None
         torch.cuda.empty_cache()
-        line["int2_chain"] = int2_chain_measure(fm, synth, torch, stream)
+        if args.int2_layers > 0:
+            line["int2_chain"] = int2_chain_measure(fm, synth, torch, stream, layers=args.int2_layers)
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         line["cpu_baseline"] = cpu_baseline(args.cpu_seconds, L)
     elif rank == 0:
