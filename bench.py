@@ -252,14 +252,22 @@ def barrier(world):
         dist.barrier()
 
 
-def max_over_ranks(v: float, world: int) -> float:
+def max_over_ranks(v: float, world: int, device: str = "cuda") -> float:
+    """The slowest rank's time (every rank takes part; `device` is where the
+    reduction runs: the rank's GPU under NCCL, "cpu" under gloo)."""
     if world == 1:
         return v
     import torch
     import torch.distributed as dist
-    t = torch.tensor([v], dtype=torch.float64, device="cuda")
+    t = torch.tensor([v], dtype=torch.float64, device=device)
     dist.all_reduce(t, op=dist.ReduceOp.MAX)
     return float(t.item())
+
+
+def job_rate(units_per_rank: int, world: int, ms_max: float) -> float:
+    """Whole-job throughput of `world` replicas that each processed
+    units_per_rank units, timed by the slowest rank."""
+    return world * units_per_rank / (ms_max / 1e3)
 
 
 # ----------------------------------------------------------- CPU baseline --
@@ -390,7 +398,7 @@ def run_ours(args):
         raise RuntimeError(f"device status word {st:#x} after the timed region")
 
     per_step_s = ms_max / 1e3 / args.steps
-    value = world * args.steps / (ms_max / 1e3)
+    value = job_rate(args.steps, world, ms_max)
     rec = desc.record_bytes()
     expert_bytes = (wl.top_k + 1) * rec
     layer_bytes = expert_bytes + wl.n_experts * H * 4 + 2 * H * 4
@@ -437,7 +445,7 @@ def run_ours(args):
         e1.record(stream)
     e1.synchronize()
     e2e_ms = max_over_ranks(e0.elapsed_time(e1), world)
-    e2e = {"value": world * K2 / (e2e_ms / 1e3), "unit": UNIT, "h2d_bytes_per_step": 2 * H * 4,
+    e2e = {"value": job_rate(K2, world, e2e_ms), "unit": UNIT, "h2d_bytes_per_step": 2 * H * 4,
            "d2h_bytes_per_step": 2 * H * 4, "steps": K2,
            "how": "per step: pinned host h, xn -> device, fmoe_layer_forward (eager C-ABI call), h', xn' -> pinned host"}
 
