@@ -29,7 +29,10 @@ constexpr int kGrpMaxM = 16;      // tokens per GEMV work item
 constexpr int kGrpBuckets = 4;    // GEMV items by size: <= 2, <= 4, <= 8, <= 16 tokens
 constexpr int kTcItemMax = 128;   // tokens per tensor-core work item
 constexpr int kGrpThreads = 256;
-constexpr int kGuSplit = 16;      // CTAs per item over the gate/up row pairs
+// CTAs per item over the gate/up row pairs for items of up to MB tokens:
+// the larger items are bound by the integer dot products rather than by
+// their weight bytes, so they are cut finer to keep every SM busy
+__host__ __device__ constexpr int gu_split(int MB) { return MB <= 4 ? 16 : 4 * MB; }
 constexpr int kDnRows = 128;      // hidden rows per CTA of the grouped down product
 
 // Device lists built by group_kernel.  Group g < E is routed expert g, group
@@ -57,20 +60,54 @@ __host__ __device__ constexpr int group_max_items(int T, int k, int E) {
   return (T * k < E ? T * k : E) + 1 + (T * (k + 1)) / kGrpMaxM + 1;
 }
 
-// One CTA.  Sorts the T (k + 1) slots by group (stable), builds the work
-// items (groups with >= tc_min tokens go to the tensor-core list when
-// tc_min > 0), and zeroes a / y of slots whose expert id is out of range.
+// Block-wide exclusive scan (component-wise) of v over the CTA's threads in
+// thread order; returns the scan, *total the sum.  blockDim.x <= 1024, a
+// multiple of 32; red: 32 int4 of shared memory.
+__device__ __forceinline__ int4 block_scan4(int4 v, int4* red, int4* total) {
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5, nw = blockDim.x >> 5;
+  int4 x = v;
+#pragma unroll
+  for (int o = 1; o < 32; o <<= 1) {
+    const int a = __shfl_up_sync(0xffffffffu, x.x, o), b = __shfl_up_sync(0xffffffffu, x.y, o);
+    const int c = __shfl_up_sync(0xffffffffu, x.z, o), d = __shfl_up_sync(0xffffffffu, x.w, o);
+    if (lane >= o) x = make_int4(x.x + a, x.y + b, x.z + c, x.w + d);
+  }
+  if (lane == 31) red[warp] = x;
+  __syncthreads();
+  if (warp == 0) {
+    int4 t = lane < nw ? red[lane] : make_int4(0, 0, 0, 0);
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      const int a = __shfl_up_sync(0xffffffffu, t.x, o), b = __shfl_up_sync(0xffffffffu, t.y, o);
+      const int c = __shfl_up_sync(0xffffffffu, t.z, o), d = __shfl_up_sync(0xffffffffu, t.w, o);
+      if (lane >= o) t = make_int4(t.x + a, t.y + b, t.z + c, t.w + d);
+    }
+    if (lane < nw) red[lane] = t;  // inclusive sums of the warps
+  }
+  __syncthreads();
+  const int4 before = warp > 0 ? red[warp - 1] : make_int4(0, 0, 0, 0);
+  *total = red[nw - 1];
+  __syncthreads();  // red may be reused
+  return make_int4(before.x + x.x - v.x, before.y + x.y - v.y, before.z + x.z - v.z, before.w + x.w - v.w);
+}
+
+// One CTA of 1024 threads.  Sorts the T (k + 1) slots by group (stable),
+// builds the work items (groups with >= tc_min tokens go to the tensor-core
+// list when tc_min > 0), and zeroes a / y of slots whose expert id is out of
+// range.  Groups are scanned two per thread (E + 1 <= 2048).
 __global__ void __launch_bounds__(1024) group_kernel(const int32_t* __restrict__ ids, int T, int k, int E, int I,
                                                      int H, int tc_min, GroupWork w, float* __restrict__ a,
                                                      float* __restrict__ y) {
   extern __shared__ int gsm[];
+  __shared__ int4 s_red[32];
   int* cnt = gsm;             // [E + 1]
   int* off = cnt + (E + 1);   // [E + 2]
-  int* nit = off + (E + 2);   // [E + 2]: items per group, then their exclusive scan
+  int* nit = off + (E + 2);   // [E + 2]: first GEMV item of each group
   int* grp = nit + (E + 2);   // [S]: group of each slot (-1: bad id)
   const int S = T * (k + 1);
   const int tid = threadIdx.x, nt = blockDim.x;
   for (int g = tid; g <= E; g += nt) cnt[g] = 0;
+  if (tid < kGrpBuckets) w.n_items[2 + tid] = 0;
   for (int s = tid; s < S; s += nt) {
     const int t = s / (k + 1), j = s % (k + 1);
     int g = E;
@@ -81,10 +118,9 @@ __global__ void __launch_bounds__(1024) group_kernel(const int32_t* __restrict__
     grp[s] = g;
   }
   __syncthreads();
-  auto group_of = [&](int s) -> int { return grp[s]; };
   bool bad = false;
   for (int s = tid; s < S; s += nt) {
-    const int g = group_of(s);
+    const int g = grp[s];
     if (g >= 0) atomicAdd(&cnt[g], 1);
     else {
       bad = true;
@@ -93,29 +129,42 @@ __global__ void __launch_bounds__(1024) group_kernel(const int32_t* __restrict__
     }
   }
   if (__syncthreads_or(bad) && tid == 0) raise_status(FMOE_STATUS_BAD_EXPERT_ID);
-  if (tid == 0) {  // exclusive scans (E + 1 <= 1025 entries)
-    int o = 0, it = 0;
-    for (int g = 0; g <= E; ++g) {
-      off[g] = o;
-      o += cnt[g];
-      const int c = cnt[g];
-      const int n = c == 0 ? 0 : (tc_min > 0 && c >= tc_min ? 0 : (c + kGrpMaxM - 1) / kGrpMaxM);
-      nit[g] = it;
-      it += n;
+  // per group: (slots, GEMV items, tensor-core items, their rounded tokens)
+  auto group_terms = [&](int g) -> int4 {
+    if (g > E) return make_int4(0, 0, 0, 0);
+    const int c = cnt[g];
+    if (c == 0) return make_int4(0, 0, 0, 0);
+    if (tc_min > 0 && c >= tc_min) {
+      const int full = c / kTcItemMax, rem = c % kTcItemMax;
+      return make_int4(c, 0, full + (rem > 0), full * kTcItemMax + (rem + 7) / 8 * 8);
     }
-    off[E + 1] = o;
-    nit[E + 1] = it;
-    int ntc = 0, np_sum = 0;
-    for (int g = 0; g <= E; ++g)
-      if (tc_min > 0 && cnt[g] >= tc_min)
-        for (int f = 0; f < cnt[g]; f += kTcItemMax) {
-          const int mm = min(kTcItemMax, cnt[g] - f);
-          w.tc[ntc++] = make_int4(g, f, mm, np_sum);
-          np_sum += (mm + 7) / 8 * 8;
-        }
-    w.n_items[0] = it;
-    w.n_items[1] = ntc;
-    for (int b = 0; b < kGrpBuckets; ++b) w.n_items[2 + b] = 0;
+    return make_int4(c, (c + kGrpMaxM - 1) / kGrpMaxM, 0, 0);
+  };
+  const int g0 = 2 * tid, g1 = g0 + 1;
+  const int4 v0 = group_terms(g0), v1 = group_terms(g1);
+  int4 tot;
+  const int4 e0 = block_scan4(make_int4(v0.x + v1.x, v0.y + v1.y, v0.z + v1.z, v0.w + v1.w), s_red, &tot);
+  const int4 e1 = make_int4(e0.x + v0.x, e0.y + v0.y, e0.z + v0.z, e0.w + v0.w);
+  if (g0 <= E) off[g0] = e0.x, nit[g0] = e0.y;
+  if (g1 <= E) off[g1] = e1.x, nit[g1] = e1.y;
+  if (tid == 0) {
+    off[E + 1] = tot.x;
+    nit[E + 1] = tot.y;
+    w.n_items[0] = tot.y;
+    w.n_items[1] = tot.z;
+  }
+  // tensor-core items of this thread's groups, in group order
+#pragma unroll
+  for (int h = 0; h < 2; ++h) {
+    const int g = h == 0 ? g0 : g1;
+    const int4 v = h == 0 ? v0 : v1;
+    const int4 e = h == 0 ? e0 : e1;
+    int idx = e.z, np_sum = e.w;
+    for (int f = 0; f < v.x && v.z > 0; f += kTcItemMax) {
+      const int mm = min(kTcItemMax, v.x - f);
+      w.tc[idx++] = make_int4(g, f, mm, np_sum);
+      np_sum += (mm + 7) / 8 * 8;
+    }
   }
   __syncthreads();
   const int max_items = group_max_items(T, k, E);
@@ -134,10 +183,11 @@ __global__ void __launch_bounds__(1024) group_kernel(const int32_t* __restrict__
   }
   // stable placement: rank of s = earlier slots of the same group
   for (int s = tid; s < S; s += nt) {
-    const int g = group_of(s);
+    const int g = grp[s];
     if (g < 0) continue;
     int r = 0;
-    for (int s2 = 0; s2 < s; ++s2) r += group_of(s2) == g;
+#pragma unroll 8
+    for (int s2 = 0; s2 < s; ++s2) r += grp[s2] == g;
     w.slots[off[g] + r] = s;
   }
 }
@@ -231,7 +281,7 @@ __device__ __forceinline__ void gateup_rows_multi(const uint8_t* rec, const Expe
   }
 }
 
-// grid (max items, kGuSplit), one size bucket of GEMV items (m <= MB).
+// grid (max items, gu_split(MB)), one size bucket of GEMV items (m <= MB).
 // Item (group, first, m): the group's slots first .. first + m - 1; the
 // tokens' staged inputs are copied from xs (stage_tokens_kernel).  Also
 // computes gamma[t] = sigmoid(w_sg . xn[t]) for the shared expert's tokens
@@ -275,7 +325,7 @@ gateup_group_kernel(ExpertSet es, GroupWork w, int bucket, int max_items, const 
   int p0, p1;
   {
     const int ng = es.H / 64, ppu = 32 / (ng < 32 ? ng : 32);  // row pairs per warp unit
-    const int per = ((es.I + kGuSplit - 1) / kGuSplit + ppu - 1) / ppu * ppu;
+    const int per = ((es.I + gu_split(MB) - 1) / gu_split(MB) + ppu - 1) / ppu * ppu;
     p0 = min(es.I, (int)blockIdx.y * per);
     p1 = min(es.I, p0 + per);
   }

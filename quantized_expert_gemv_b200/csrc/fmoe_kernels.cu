@@ -340,7 +340,10 @@ __device__ __forceinline__ float block_sum(float v, float* red) {
   return s;
 }
 
-// One CTA per token.
+// One CTA per token.  With H <= 4 kCombVec kThreads (and H % 4 == 0) each
+// thread keeps its h' values in registers: all of its loads go out at once
+// and the norm pass reads nothing back; otherwise a strided two-pass loop.
+constexpr int kCombVec = 4;
 __global__ void __launch_bounds__(kThreads)
 combine_kernel(const float* __restrict__ y, const float* __restrict__ weights,
                const float* __restrict__ gamma, const float* h, const float* __restrict__ norm_w,
@@ -349,9 +352,54 @@ combine_kernel(const float* __restrict__ y, const float* __restrict__ weights,
   const int t = blockIdx.x;
   const float* yt = y + (size_t)t * (k + 1) * H;
   float p[kMaxK];
-  for (int j = 0; j < k; ++j) p[j] = weights[(size_t)t * k + j];
+#pragma unroll
+  for (int j = 0; j < kMaxK; ++j) p[j] = j < k ? weights[(size_t)t * k + j] : 0.f;
   const float gm = gamma[t];
   float ss = 0.f;
+  if (H % 4 == 0 && H <= 4 * kCombVec * (int)blockDim.x) {
+    const int nv = H / 4;
+    float4 v[kCombVec];
+#pragma unroll
+    for (int u = 0; u < kCombVec; ++u) {
+      const int i4 = threadIdx.x + u * blockDim.x;
+      if (i4 < nv) {
+        float4 acc = reinterpret_cast<const float4*>(h + (size_t)t * H)[i4];
+        const float4 ys = __ldcg(reinterpret_cast<const float4*>(yt + (size_t)k * H) + i4);
+#pragma unroll
+        for (int j = 0; j < kMaxK; ++j) {
+          if (j < k) {
+            const float4 yj = __ldcg(reinterpret_cast<const float4*>(yt + (size_t)j * H) + i4);
+            acc.x = fmaf(p[j], yj.x, acc.x);
+            acc.y = fmaf(p[j], yj.y, acc.y);
+            acc.z = fmaf(p[j], yj.z, acc.z);
+            acc.w = fmaf(p[j], yj.w, acc.w);
+          }
+        }
+        acc.x = fmaf(gm, ys.x, acc.x);
+        acc.y = fmaf(gm, ys.y, acc.y);
+        acc.z = fmaf(gm, ys.z, acc.z);
+        acc.w = fmaf(gm, ys.w, acc.w);
+        v[u] = acc;
+        reinterpret_cast<float4*>(h_out + (size_t)t * H)[i4] = acc;
+        ss = fmaf(acc.x, acc.x, ss);
+        ss = fmaf(acc.y, acc.y, ss);
+        ss = fmaf(acc.z, acc.z, ss);
+        ss = fmaf(acc.w, acc.w, ss);
+      }
+    }
+    ss = block_sum(ss, red);
+    const float r = 1.f / sqrtf(ss / (float)H + eps);
+#pragma unroll
+    for (int u = 0; u < kCombVec; ++u) {
+      const int i4 = threadIdx.x + u * blockDim.x;
+      if (i4 < nv) {
+        const float4 nw = __ldg(reinterpret_cast<const float4*>(norm_w) + i4);
+        reinterpret_cast<float4*>(xn_out + (size_t)t * H)[i4] =
+            make_float4(v[u].x * r * nw.x, v[u].y * r * nw.y, v[u].z * r * nw.z, v[u].w * r * nw.w);
+      }
+    }
+    return;
+  }
   for (int i = threadIdx.x; i < H; i += blockDim.x) {
     float v = h[(size_t)t * H + i];
     for (int j = 0; j < k; ++j) v = fmaf(p[j], yt[(size_t)j * H + i], v);
@@ -615,7 +663,7 @@ template <int MB>
 static void grp_launch_gu(const ExpertSet& es, const GroupWork& gw, int b, int items, const float* xn,
                           const unsigned char* xs, float* a, const float* w_sg, float* gamma, size_t sxs,
                           cudaStream_t st) {
-  gateup_group_kernel<MB><<<dim3(items, kGuSplit), kGrpThreads, MB * sxs, st>>>(es, gw, b, items, xn, xs, a, w_sg,
+  gateup_group_kernel<MB><<<dim3(items, gu_split(MB)), kGrpThreads, MB * sxs, st>>>(es, gw, b, items, xn, xs, a, w_sg,
                                                                               gamma);
 }
 
