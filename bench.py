@@ -54,11 +54,11 @@ def batched_measure(fm, synth, np, torch, lw, wl, stream, steps=50, warmup=5, T=
     popularity (fresh Gumbel-top-k logits every step, given as router
     logits): tokens/s and the expert bytes the steps touch."""
     logits = [torch.from_numpy(synth.zipf_gumbel_logits(wl, s, T)[0]).cuda() for s in range(steps)]
-    hot = []
+    hot, tc_min = [], fm.fmoe_tc_min_tokens()
     for lg in logits:
         ids = torch.topk(lg, wl.top_k, dim=1).indices.cpu().numpy()
         cnt = np.bincount(ids.ravel(), minlength=wl.n_experts)
-        hot.append(((cnt > 0).sum(), (cnt >= 16).sum()))
+        hot.append(((cnt > 0).sum(), (cnt >= tc_min).sum()))
     x = torch.from_numpy(synth.tokens(wl, T, stream=900)).cuda()
     h, xn = x.clone(), x.clone()
     ws = fm.alloc_workspace(lw.desc, T)

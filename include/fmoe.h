@@ -240,13 +240,19 @@ int fmoe_stack_forward(const fmoe_layer_weights* layers, int n_layers, float* d_
 int fmoe_set_fused(int enable);
 
 /* Chooses the expert products of the T > 1 path for experts that receive at
- * least 16 tokens in a step (and the shared expert when T >= 16): enable != 0
- * (the default) runs them as tcgen05 tensor-core matrix products on
- * dequantised fp16 weights (inputs kept to ~22 bits as an fp16 hi / lo
- * pair), 0 as the integer-dot matrix-vector path in batches of 16 tokens.
- * Both compute the same products within the tolerance; process-wide
- * setting, returns the previous value. */
+ * least fmoe_tc_min_tokens() tokens in a step (and the shared expert when T
+ * reaches it): enable != 0 (the default) runs them as tcgen05 tensor-core
+ * matrix products on dequantised fp16 weights (inputs kept to ~22 bits as an
+ * fp16 hi / lo pair), 0 as the integer-dot matrix-vector path in batches of
+ * 16 tokens.  Both compute the same products within the tolerance;
+ * process-wide setting, returns the previous value. */
 int fmoe_set_tensor_cores(int enable);
+
+/* Tokens an expert needs in a step for its products to run on the tensor
+ * cores (when enabled): 5.  From about five tokens per expert the
+ * integer-dot matrix-vector path is bound by its dot products rather than by
+ * the expert's weight bytes. */
+int fmoe_tc_min_tokens(void);
 
 /* 1 if the persistent kernel runs layers of descriptor d at T = 1 on the
  * current device (shape and shared-memory plan fit), else 0 (also on any
@@ -267,8 +273,9 @@ int fmoe_fused_supported(const fmoe_layer_desc* d);
  * library's module is loaded on that device.
  *   lw, d_h, d_xn, T, stream  as for fmoe_layer_forward.
  * Limit: fmoe_workspace_bytes(&lw->desc, T) must not exceed 12 MiB
- * (12582912 bytes), which admits up to T = 88 tokens at hidden 4096 /
- * inter 1024 / 512 experts / top-4; a larger request returns
+ * (12582912 bytes), which admits up to T = 17 tokens at hidden 4096 /
+ * inter 1024 / 512 experts / top-4 (from T = 5 the workspace holds the
+ * tensor-core inputs, about 100 KB per token); a larger request returns
  * FMOE_ERR_BUFFER_TOO_SMALL before anything is launched.
  * First call on each device: it looks up the array's device address and
  * enqueues, on `stream`, a zeroing of the counter words at the array's start

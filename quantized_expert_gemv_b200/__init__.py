@@ -90,6 +90,7 @@ _SIGS = {
     "fmoe_set_fused": (_i32, [_i32]),
     "fmoe_fused_supported": (_i32, [_PDESC]),
     "fmoe_set_tensor_cores": (_i32, [_i32]),
+    "fmoe_tc_min_tokens": (_i32, []),
     "fmoe_layer_forward_noalloc": (_i32, [_PW, _vp, _vp, _i32, _vp]),
 }
 for _name, (_res, _args) in _SIGS.items():
@@ -319,6 +320,11 @@ def fmoe_set_tensor_cores(enable: bool) -> bool:
     """Selects tensor-core products (True, default) or the integer-dot path for the
     heavily routed experts of the T > 1 path; returns the previous setting."""
     return bool(_lib.fmoe_set_tensor_cores(int(bool(enable))))
+
+
+def fmoe_tc_min_tokens() -> int:
+    """Tokens an expert needs in a step for the tensor-core products."""
+    return int(_lib.fmoe_tc_min_tokens())
 
 
 def fmoe_set_fused(enable: bool) -> bool:

@@ -27,7 +27,7 @@ namespace fmoe {
 
 constexpr int kGrpMaxM = 16;      // tokens per GEMV work item
 constexpr int kGrpBuckets = 4;    // GEMV items by size: <= 2, <= 4, <= 8, <= 16 tokens
-constexpr int kTcItemMax = 128;   // tokens per tensor-core work item
+constexpr int kTcItemMax = 32;    // tokens per tensor-core work item (more CTAs, shorter products each)
 constexpr int kGrpThreads = 256;
 // CTAs per item over the gate/up row pairs for items of up to MB tokens:
 // the larger items are bound by the integer dot products rather than by
@@ -310,6 +310,7 @@ gateup_group_kernel(ExpertSet es, GroupWork w, int bucket, int max_items, const 
     for (int i = warp; i < m; i += kGrpThreads / 32) {
       const float* x = xn + (size_t)(s_slot[i] / k1) * es.H;
       float z = 0.f;
+#pragma unroll 8
       for (int c = lane * 4; c < es.H; c += 128) {
         const float4 wv = __ldg(reinterpret_cast<const float4*>(w_sg + c));
         const float4 v = __ldg(reinterpret_cast<const float4*>(x + c));

@@ -660,18 +660,39 @@ static bool grp_optin(size_t gu_smem, size_t dn_smem, int b) {
 }
 
 template <int MB>
-static void grp_launch_gu(const ExpertSet& es, const GroupWork& gw, int b, int items, const float* xn,
+static void grp_launch_gu(const ExpertSet& es, const GroupWork& gw, int b, int items, int grid, const float* xn,
                           const unsigned char* xs, float* a, const float* w_sg, float* gamma, size_t sxs,
                           cudaStream_t st) {
-  gateup_group_kernel<MB><<<dim3(items, gu_split(MB)), kGrpThreads, MB * sxs, st>>>(es, gw, b, items, xn, xs, a, w_sg,
-                                                                              gamma);
+  gateup_group_kernel<MB><<<dim3(grid, gu_split(MB)), kGrpThreads, MB * sxs, st>>>(es, gw, b, items, xn, xs, a, w_sg,
+                                                                             gamma);
 }
 
 template <int MB>
-static void grp_launch_dn(const ExpertSet& es, const GroupWork& gw, int b, int items, const float* a, float* y,
-                          size_t sas, cudaStream_t st) {
-  down_group_kernel<MB><<<dim3(items, (es.H + kDnRows - 1) / kDnRows), kDnRows, MB * sas, st>>>(es, gw, b, items, a,
-                                                                                                  y);
+static void grp_launch_dn(const ExpertSet& es, const GroupWork& gw, int b, int items, int grid, const float* a,
+                          float* y, size_t sas, cudaStream_t st) {
+  down_group_kernel<MB><<<dim3(grid, (es.H + kDnRows - 1) / kDnRows), kDnRows, MB * sas, st>>>(es, gw, b, items, a,
+                                                                                                 y);
+}
+
+// SMs of the current device (cached per device; 148 if the query fails).
+static int device_sms() {
+  static int cached[64];
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return 148;
+  if (cached[dev] == 0) {
+    int n = 0;
+    cached[dev] = cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) == cudaSuccess && n > 0 ? n : 148;
+  }
+  return cached[dev];
+}
+
+// Upper bound of the GEMV items of size bucket b (sizes (2^b, 2^(b+1)], the
+// first bucket from 1): no more than S / (smallest size) of them, and none
+// when the tensor cores take every group of that size.
+static int bucket_items_bound(int b, int S, int max_items, int tc_min) {
+  const int lo = b == 0 ? 1 : (1 << b) + 1;
+  if (tc_min > 0 && lo >= tc_min) return 0;
+  return S / lo < max_items ? S / lo : max_items;
 }
 
 static int launch_experts(const ExpertSet& es, const float* xn, const int32_t* ids, int T, float* a,
@@ -689,29 +710,37 @@ static int launch_experts(const ExpertSet& es, const float* xn, const int32_t* i
       const int items = group_max_items(T, es.k, es.E);
       // groups of >= kTcMinTokens tokens go to the tensor cores when the shape tiles
       const bool tc = g_tc_enabled && T >= kTcMinTokens && tcx && tca && es.H % kTcRows == 0 &&
-                      (2 * es.I) % kTcRows == 0 &&
+                      (2 * es.I) % kTcRows == 0 && (es.H / 64) % 4 == 0 && (es.I / 64) % 4 == 0 &&
                       smem_optin(reinterpret_cast<const void*>(&tc_gemm_kernel<0>), tc_smem_bytes(), 2) &&
                       smem_optin(reinterpret_cast<const void*>(&tc_gemm_kernel<1>), tc_smem_bytes(), 3);
       const int max_tc = group_max_tc(T, es.k, kTcMinTokens);
       group_kernel<<<1, 1024, grp_smem, st>>>(ids, T, es.k, es.E, es.I, es.H, tc ? kTcMinTokens : 0, *gw, a, y);
       stage_tokens_kernel<<<T, kGrpThreads, 0, st>>>(xn, es.H, xs, sxs);
-      grp_launch_gu<2>(es, *gw, 0, items, xn, xs, a, w_sg, gamma, sxs, st);
-      grp_launch_gu<4>(es, *gw, 1, items, xn, xs, a, w_sg, gamma, sxs, st);
-      grp_launch_gu<8>(es, *gw, 2, items, xn, xs, a, w_sg, gamma, sxs, st);
-      grp_launch_gu<16>(es, *gw, 3, items, xn, xs, a, w_sg, gamma, sxs, st);
+      // a bucket's grid covers at most the items it can hold (the kernels
+      // index the bucket lists with the full stride `items`)
+      int nb[kGrpBuckets];
+      for (int b = 0; b < kGrpBuckets; ++b) nb[b] = bucket_items_bound(b, slots, items, tc ? kTcMinTokens : 0);
+      if (nb[0]) grp_launch_gu<2>(es, *gw, 0, items, nb[0], xn, xs, a, w_sg, gamma, sxs, st);
+      if (nb[1]) grp_launch_gu<4>(es, *gw, 1, items, nb[1], xn, xs, a, w_sg, gamma, sxs, st);
+      if (nb[2]) grp_launch_gu<8>(es, *gw, 2, items, nb[2], xn, xs, a, w_sg, gamma, sxs, st);
+      if (nb[3]) grp_launch_gu<16>(es, *gw, 3, items, nb[3], xn, xs, a, w_sg, gamma, sxs, st);
       if (tc) {
         tc_stage_kernel<<<dim3(max_tc, es.H / 64), kTcThreads, 0, st>>>(*gw, xn, es.H, es.k + 1, 0, tcx, es.E, w_sg,
                                                                       gamma);
-        tc_gemm_kernel<0><<<dim3(max_tc, 2 * es.I / kTcRows), kTcThreads + 32, tc_smem_bytes(), st>>>(es, *gw, tcx, a);
+        const int n_sm = device_sms();
+        const int u0 = max_tc * (2 * es.I / kTcRows);
+        tc_gemm_kernel<0><<<u0 < n_sm ? u0 : n_sm, kTcThreads + 32, tc_smem_bytes(), st>>>(es, *gw, tcx, a);
       }
-      grp_launch_dn<2>(es, *gw, 0, items, a, y, sas, st);
-      grp_launch_dn<4>(es, *gw, 1, items, a, y, sas, st);
-      grp_launch_dn<8>(es, *gw, 2, items, a, y, sas, st);
-      grp_launch_dn<16>(es, *gw, 3, items, a, y, sas, st);
+      if (nb[0]) grp_launch_dn<2>(es, *gw, 0, items, nb[0], a, y, sas, st);
+      if (nb[1]) grp_launch_dn<4>(es, *gw, 1, items, nb[1], a, y, sas, st);
+      if (nb[2]) grp_launch_dn<8>(es, *gw, 2, items, nb[2], a, y, sas, st);
+      if (nb[3]) grp_launch_dn<16>(es, *gw, 3, items, nb[3], a, y, sas, st);
       if (tc) {
         tc_stage_kernel<<<dim3(max_tc, es.I / 64), kTcThreads, 0, st>>>(*gw, a, es.I, es.k + 1, 1, tca, es.E, nullptr,
                                                                       nullptr);
-        tc_gemm_kernel<1><<<dim3(max_tc, es.H / kTcRows), kTcThreads + 32, tc_smem_bytes(), st>>>(es, *gw, tca, y);
+        const int n_sm = device_sms();
+        const int u1 = max_tc * (es.H / kTcRows);
+        tc_gemm_kernel<1><<<u1 < n_sm ? u1 : n_sm, kTcThreads + 32, tc_smem_bytes(), st>>>(es, *gw, tca, y);
       }
       return cuda_rc(cudaGetLastError());
     }
@@ -1062,6 +1091,8 @@ extern "C" int fmoe_set_tensor_cores(int enable) {
   g_tc_enabled = enable ? 1 : 0;
   return prev;
 }
+
+extern "C" int fmoe_tc_min_tokens(void) { return kTcMinTokens; }
 
 extern "C" int fmoe_set_fused(int enable) {
   const int prev = g_fused_enabled;

@@ -38,8 +38,8 @@
 
 namespace fmoe {
 
-constexpr int kTcMinTokens = 16;  // a group this large goes to the tensor cores
-constexpr int kTcMaxNp = 128;     // tokens per tensor-core item (N = 2 Np <= 256)
+constexpr int kTcMinTokens = 5;   // from 5 tokens per expert the integer GEMV is bound by its dot products (measured)
+constexpr int kTcMaxNp = kTcItemMax;  // tokens per tensor-core item (N = 2 Np <= 64)
 constexpr int kTcThreads = 256;
 constexpr int kTcRows = 128;      // weight rows per CTA (the MMA's M)
 constexpr uint32_t kTcATile = kTcRows * 64 * 2;  // fp16 A tile of one 64-input group
@@ -133,6 +133,7 @@ tc_stage_kernel(GroupWork w, const float* __restrict__ src, int K, int k1, int m
       const int t = slots[i] / k1;
       const float* x = src + (size_t)t * K;
       float z = 0.f;
+#pragma unroll 8
       for (int c = lane * 4; c < K; c += 128) {
         const float4 wv = __ldg(reinterpret_cast<const float4*>(w_sg + c));
         const float4 v = __ldg(reinterpret_cast<const float4*>(x + c));
@@ -148,23 +149,41 @@ tc_stage_kernel(GroupWork w, const float* __restrict__ src, int K, int k1, int m
 }
 
 // ---------------------------------------------------------- dequantise --
-// Four 16-byte fp16 stores of 8 weights each into the A tile: row r, inputs
-// 8 c .. 8 c + 7 for c = c0 .. c0 + 3.
-__device__ __forceinline__ void store_a8(uint8_t* a_tile, int r, int c, const float* w8) {
-  *reinterpret_cast<uint4*>(a_tile + (size_t)c * (kTcRows / 8) * 128 + (r >> 3) * 128 + (r & 7) * 16) =
-      make_uint4(pack_h2(w8[0], w8[1]), pack_h2(w8[2], w8[3]), pack_h2(w8[4], w8[5]), pack_h2(w8[6], w8[7]));
+// Codes become fp16 pairs without integer-to-float conversions: a pair of
+// code fields is moved into the low mantissa bits of two fp16 values of
+// exponent 2^10 (1024 + field, exact), 1024 is subtracted (exact), and one
+// fused half2 multiply-add applies the group's scale and bias, so each
+// weight is rounded once to fp16.  A field that sits j bits up in its half
+// reads as 2^j code, so its pair takes the scale 2^-j s.
+__device__ __forceinline__ uint32_t deq_pair(uint32_t fields, __half2 s2, __half2 b2) {
+  const uint32_t v = fields | 0x64006400u, m = 0x64006400u;
+  const __half2 q = __hsub2(*reinterpret_cast<const __half2*>(&v), *reinterpret_cast<const __half2*>(&m));
+  const __half2 w = __hfma2(q, s2, b2);
+  return *reinterpret_cast<const uint32_t*>(&w);
 }
 
-// Weights of inputs 0..7 of a 4-bit word (field 2a+b holds input 4b+a).
-__device__ __forceinline__ void dequant_word4(uint32_t word, float s, float b, float* w8) {
-#pragma unroll
-  for (int i = 0; i < 8; ++i) w8[i] = fmaf((float)((word >> (4 * (2 * (i & 3) + (i >> 2)))) & 15u), s, b);
+// 16-byte fp16 store of inputs 8 c .. 8 c + 7 of row r into the A tile.
+__device__ __forceinline__ void store_a8h(uint8_t* a_tile, int r, int c, uint4 h) {
+  *reinterpret_cast<uint4*>(a_tile + (size_t)c * (kTcRows / 8) * 128 + (r >> 3) * 128 + (r & 7) * 16) = h;
 }
 
-// Weights of inputs 0..15 of a 2-bit word (field 4a+b holds input 4b+a).
-__device__ __forceinline__ void dequant_word2(uint32_t word, float s, float b, float* w16) {
-#pragma unroll
-  for (int i = 0; i < 16; ++i) w16[i] = fmaf((float)((word >> (2 * (4 * (i & 3) + (i >> 2)))) & 3u), s, b);
+// The eight weights of a 4-bit word (field 2a+b holds input 4b+a: byte j
+// holds inputs j and 4 + j), scales s (low fields) and s / 16 (high fields).
+__device__ __forceinline__ uint4 dequant_word4h(uint32_t word, __half2 s1, __half2 s16, __half2 b2) {
+  const uint32_t p01 = __byte_perm(word, 0u, 0x4140), p23 = __byte_perm(word, 0u, 0x4342);
+  return make_uint4(deq_pair(p01 & 0x000F000Fu, s1, b2), deq_pair(p23 & 0x000F000Fu, s1, b2),
+                    deq_pair(p01 & 0x00F000F0u, s16, b2), deq_pair(p23 & 0x00F000F0u, s16, b2));
+}
+
+// The sixteen weights of a 2-bit word (field 4a+b holds input 4b+a: byte j
+// holds inputs j, 4 + j, 8 + j, 12 + j), as two 8-input chunks; sc[i] = 4^-i s.
+__device__ __forceinline__ void dequant_word2h(uint32_t word, const __half2 (&sc)[4], __half2 b2, uint4* lo,
+                                               uint4* hi) {
+  const uint32_t p01 = __byte_perm(word, 0u, 0x4140), p23 = __byte_perm(word, 0u, 0x4342);
+  *lo = make_uint4(deq_pair(p01 & 0x00030003u, sc[0], b2), deq_pair(p23 & 0x00030003u, sc[0], b2),
+                   deq_pair(p01 & 0x000C000Cu, sc[1], b2), deq_pair(p23 & 0x000C000Cu, sc[1], b2));
+  *hi = make_uint4(deq_pair(p01 & 0x00300030u, sc[2], b2), deq_pair(p23 & 0x00300030u, sc[2], b2),
+                   deq_pair(p01 & 0x00C000C0u, sc[3], b2), deq_pair(p23 & 0x00C000C0u, sc[3], b2));
 }
 
 // True scale and bias of a packed scale-bias word (the scale is stored
@@ -174,6 +193,94 @@ __device__ __forceinline__ void sb_true(uint32_t sbw, int bits, float* s, float*
   *b = __uint_as_float(sbw & 0xFFFF0000u);
 }
 
+// ------------------------------------------------------ raw code ring --
+// The producers stream the tile's raw codes and scale-bias words into a
+// shared-memory ring of three "supersteps" of SG = 8 (or 4) 64-groups each,
+// two supersteps ahead of the one being dequantised.  A superstep's bytes
+// are copied in runs that are contiguous in global memory -- a row's SG
+// groups (gate/up codes: two 16 SG byte runs per row, one per half of the
+// 32-byte group), or 128 rows of one column-block word (down codes) -- so
+// every warp-wide cp.async covers whole 128-byte lines.  The shared-memory
+// copies are laid out so that the dequantising warps (lane l: rows l,
+// l + 32, l + 64, l + 96, one half of the group's inputs) read without bank
+// conflicts:
+//   gate/up codes  [128 rows][2 halves][SG groups][16 B], row stride 272 B
+//   gate/up s-b    [128 rows][SG words], row stride 48 B, at kRawSbOff
+//   down codes     [SG groups x words per group][128 rows] u32
+//   down s-b       [SG][128 rows] u32, at kRawDnSbOff
+constexpr int kTcStages = 4;                      // ring of A tiles
+constexpr int kTcBStages = 4;                     // ring of token tiles
+constexpr int kTcBLag = 2;                        // a token tile is refilled once the products 2 steps back are done
+constexpr uint32_t kTcBRing = kTcBStages * kTcMaxNp * 2 * 128;
+constexpr int kTcRawBufs = 3;                     // supersteps in the raw ring
+constexpr int kTcMaxSG = 8;                       // 64-groups per superstep
+constexpr uint32_t kRawRow = 272, kRawSbRow = 48;
+constexpr uint32_t kRawSbOff = 128 * kRawRow;                 // 34816
+constexpr uint32_t kRawDnSbOff = 8 * kTcMaxSG * 128 * 4;     // 32768
+constexpr uint32_t kTcRawBuf = kRawSbOff + 128 * kRawSbRow;  // 40960 >= kRawDnSbOff + kTcMaxSG * 512
+static_assert(kTcRawBuf >= kRawDnSbOff + kTcMaxSG * 512, "raw buffer holds the down layout");
+
+__device__ __forceinline__ void cp_async16(void* dst, const void* src) {
+  asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(smem_u32(dst)), "l"(src) : "memory");
+}
+__device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
+template <int N>
+__device__ __forceinline__ void cp_async_wait() { asm volatile("cp.async.wait_group %0;" ::"n"(N) : "memory"); }
+__device__ __forceinline__ void cp_async_wait_all() { asm volatile("cp.async.wait_all;" ::: "memory"); }
+// Barrier of the kTcThreads producer threads only (the issuer warp is not
+// in it) that also ANDs their flags, so that all of them leave or stay.
+__device__ __forceinline__ bool producer_bar_and(bool v) {
+  uint32_t r;
+  asm volatile(
+      "{ .reg .pred p, q;\n\t"
+      "setp.ne.u32 p, %1, 0;\n\t"
+      "bar.red.and.pred q, 1, %2, p;\n\t"
+      "selp.u32 %0, 1, 0, q; }"
+      : "=r"(r)
+      : "r"((uint32_t)v), "n"(kTcThreads)
+      : "memory");
+  return r != 0;
+}
+
+// Requests superstep S (64-groups S SG .. S SG + SG - 1) of tile rows
+// [r0, r0 + 128) into raw buffer buf.  MODE 0: gate/up rows (packed rows:
+// gate n, up n interleaved, row-major codes); MODE 1: down rows
+// (column-block codes: one word per row and column block).
+template <int MODE, int BITS>
+__device__ __forceinline__ void tc_issue_super(const uint8_t* rec, int H, int I, int r0, int S, int SG, uint8_t* buf) {
+  const RecordLayout L = record_layout(BITS, H, I);
+  const int t = threadIdx.x, g0 = S * SG;
+  if (MODE == 0) {
+    const int ng = H / 64;
+    const int runs = BITS == 4 ? 256 : 128;  // (row, half) runs of 16 SG bytes; 2-bit groups are one 16-byte chunk
+    for (int c = t; c < runs * SG; c += kTcThreads) {
+      const int run = c / SG, piece = c % SG;
+      const int row = BITS == 4 ? run >> 1 : run, h = BITS == 4 ? run & 1 : 0;
+      const uint8_t* src = rec + L.gu_codes + (size_t)(r0 + row) * L.gu_row_bytes +
+                           (BITS == 4 ? chunk_off<4>(ng, g0, h) : chunk_off<2>(ng, g0, 0)) + piece * 16;
+      cp_async16(buf + row * kRawRow + h * 128 + piece * 16, src);
+    }
+    const int spr = SG / 4;  // 16-byte pieces of a row's scale-bias words
+    for (int c = t; c < 128 * spr; c += kTcThreads) {
+      const int row = c / spr, piece = c % spr;
+      const uint8_t* src = rec + L.gu_sb + ((size_t)(r0 + row) * ng + g0) * 4 + piece * 16;
+      cp_async16(buf + kRawSbOff + row * kRawSbRow + piece * 16, src);
+    }
+  } else {
+    constexpr int kWpg = BITS == 4 ? 8 : 4;  // column-block words per 64-group
+    const uint32_t* codes = reinterpret_cast<const uint32_t*>(rec + L.down_codes);
+    for (int c = t; c < kWpg * SG * 32; c += kTcThreads) {
+      const int run = c >> 5, piece = c & 31;
+      cp_async16(buf + run * 512 + piece * 16, codes + (size_t)(kWpg * g0 + run) * H + r0 + 4 * piece);
+    }
+    const uint32_t* sbw = reinterpret_cast<const uint32_t*>(rec + L.down_sb);
+    for (int c = t; c < SG * 32; c += kTcThreads) {
+      const int run = c >> 5, piece = c & 31;
+      cp_async16(buf + kRawDnSbOff + run * 512 + piece * 16, sbw + (size_t)(g0 + run) * H + r0 + 4 * piece);
+    }
+  }
+}
+
 // Raw words of one thread's share of a tile step: 16 bytes of codes (up to
 // four 32-bit words) and the scale-bias word.
 struct TcRaw {
@@ -181,93 +288,74 @@ struct TcRaw {
   uint32_t sb;
 };
 
-// Thread t's share of 64-group gi of tile rows [r0, r0 + 128): row t / 2,
-// inputs 32 (t % 2) .. + 31.  MODE 0: gate/up rows (packed rows: gate n, up
-// n interleaved, row-major codes); MODE 1: down rows (column-block codes).
+// Group j of the superstep in buf, row r, inputs 32 hh .. 32 hh + 31.
 template <int MODE, int BITS>
-__device__ __forceinline__ TcRaw tc_load_raw(const uint8_t* rec, int H, int I, int r0, int gi) {
-  const RecordLayout L = record_layout(BITS, H, I);
-  const int t = threadIdx.x, r = t >> 1, hh = t & 1;
+__device__ __forceinline__ TcRaw tc_read_raw(const uint8_t* buf, int j, int r, int hh) {
   TcRaw w;
   if (MODE == 0) {
-    const int ng = H / 64, pr = r0 + r;
-    const uint8_t* row = rec + L.gu_codes + (size_t)pr * L.gu_row_bytes;
-    w.c = ld_stream(row + (BITS == 4 ? chunk_off<4>(ng, gi, hh) : chunk_off<2>(ng, gi, 0)));
+    w.c = *reinterpret_cast<const uint4*>(buf + r * kRawRow + (BITS == 4 ? hh * 128 : 0) + j * 16);
     if (BITS == 2 && hh) w.c = make_uint4(w.c.z, w.c.w, 0u, 0u);
-    w.sb = ld_stream_u32(reinterpret_cast<const uint32_t*>(rec + L.gu_sb) + (size_t)pr * ng + gi);
+    w.sb = *reinterpret_cast<const uint32_t*>(buf + kRawSbOff + r * kRawSbRow + j * 4);
   } else {
-    const int row = r0 + r;
-    const uint32_t* codes = reinterpret_cast<const uint32_t*>(rec + L.down_codes) + row;
-    if (BITS == 4) {  // words 8 gi + 4 hh .. + 3
-      w.c.x = ld_stream_u32(codes + (size_t)(8 * gi + 4 * hh + 0) * H);
-      w.c.y = ld_stream_u32(codes + (size_t)(8 * gi + 4 * hh + 1) * H);
-      w.c.z = ld_stream_u32(codes + (size_t)(8 * gi + 4 * hh + 2) * H);
-      w.c.w = ld_stream_u32(codes + (size_t)(8 * gi + 4 * hh + 3) * H);
-    } else {  // words 4 gi + 2 hh .. + 1
-      w.c.x = ld_stream_u32(codes + (size_t)(4 * gi + 2 * hh + 0) * H);
-      w.c.y = ld_stream_u32(codes + (size_t)(4 * gi + 2 * hh + 1) * H);
-      w.c.z = w.c.w = 0u;
-    }
-    w.sb = ld_stream_u32(reinterpret_cast<const uint32_t*>(rec + L.down_sb) + (size_t)gi * H + row);
+    const uint32_t* wd = reinterpret_cast<const uint32_t*>(buf);
+    if (BITS == 4)
+      w.c = make_uint4(wd[(8 * j + 4 * hh + 0) * 128 + r], wd[(8 * j + 4 * hh + 1) * 128 + r],
+                       wd[(8 * j + 4 * hh + 2) * 128 + r], wd[(8 * j + 4 * hh + 3) * 128 + r]);
+    else
+      w.c = make_uint4(wd[(4 * j + 2 * hh + 0) * 128 + r], wd[(4 * j + 2 * hh + 1) * 128 + r], 0u, 0u);
+    w.sb = *reinterpret_cast<const uint32_t*>(buf + kRawDnSbOff + (j * 128 + r) * 4);
   }
   return w;
 }
 
-// Dequantises a thread's share into the fp16 A tile.
+// Dequantises row r, inputs 32 hh .. 32 hh + 31 of a step into the fp16 A tile.
 template <int BITS>
-__device__ __forceinline__ void tc_dequant(const TcRaw& w, uint8_t* a_tile) {
-  const int t = threadIdx.x, r = t >> 1, hh = t & 1;
+__device__ __forceinline__ void tc_dequant(const TcRaw& w, uint8_t* a_tile, int r, int hh) {
   float s, b;
   sb_true(w.sb, BITS, &s, &b);
+  const __half2 b2 = __float2half2_rn(b);
   if (BITS == 4) {
+    const __half2 s1 = __float2half2_rn(s), s16 = __float2half2_rn(s * 0.0625f);
     const uint32_t wd[4] = {w.c.x, w.c.y, w.c.z, w.c.w};
 #pragma unroll
-    for (int q = 0; q < 4; ++q) {
-      float w8[8];
-      dequant_word4(wd[q], s, b, w8);
-      store_a8(a_tile, r, 4 * hh + q, w8);
-    }
+    for (int q = 0; q < 4; ++q) store_a8h(a_tile, r, 4 * hh + q, dequant_word4h(wd[q], s1, s16, b2));
   } else {
+    const __half2 sc[4] = {__float2half2_rn(s), __float2half2_rn(s * 0.25f), __float2half2_rn(s * 0.0625f),
+                           __float2half2_rn(s * 0.015625f)};
     const uint32_t wd[2] = {w.c.x, w.c.y};
 #pragma unroll
     for (int q = 0; q < 2; ++q) {
-      float w16[16];
-      dequant_word2(wd[q], s, b, w16);
-      store_a8(a_tile, r, 4 * hh + 2 * q, w16);
-      store_a8(a_tile, r, 4 * hh + 2 * q + 1, w16 + 8);
+      uint4 lo, hi;
+      dequant_word2h(wd[q], sc, b2, &lo, &hi);
+      store_a8h(a_tile, r, 4 * hh + 2 * q, lo);
+      store_a8h(a_tile, r, 4 * hh + 2 * q + 1, hi);
     }
   }
 }
 
 // ------------------------------------------------------------- the GEMM --
-constexpr int kTcStages = 3;  // shared-memory ring of A and B tiles
-constexpr int kTcAhead = 4;   // steps of raw weight words held in registers ahead of use
-
-template <int MODE, int BITS>
-__device__ __forceinline__ TcRaw tc_raw_or_zero(const uint8_t* rec, int H, int I, int r0, int gi, int steps) {
-  if (gi < steps) return tc_load_raw<MODE, BITS>(rec, H, I, r0, gi);
-  TcRaw z;
-  z.c = make_uint4(0u, 0u, 0u, 0u);
-  z.sb = 0u;
-  return z;
-}
-
 __device__ __forceinline__ void mbar_arrive(uint64_t* bar) {
   asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(smem_u32(bar)) : "memory");
 }
 
 // grid (max tensor-core items, M / 128), kTcThreads + 32 threads.  MODE 0:
 // gate/up (M = 2 I, K = H), epilogue SwiGLU -> a[slot][n].  MODE 1: down
-// (M = H, K = I) -> y[slot][row].  Warps 0..7 dequantise step s (one
-// 64-input group) into ring stage s % 3 and arrive on full[stage]; warp 8
-// (one thread) waits for the stage's A and token tile, issues the four
-// products, commits them to done[stage] and requests the token tile of step
-// s + 2.  Completion c of a stage's mbarriers belongs to step stage + 3 c,
-// so every wait's parity is (s / 3) & 1.  Bounded waits: on expiry the CTA
-// sets FMOE_STATUS_WAIT_TIMEOUT, waits (bounded) for its committed products
-// and copies, frees its tensor memory and returns.
+// (M = H, K = I) -> y[slot][row].  Warps 0..7 keep two supersteps of raw
+// codes in flight (see the raw code ring); warps w and w + 4 dequantise the
+// steps s = w (mod 4) (one 64-input group each, one half of its inputs per
+// warp, so four steps are in flight) into A stage s % 4 once the products
+// of step s - 4 are done, and arrive on full[s % 4]; warp 8 (one thread)
+// waits for the A stage and the
+// step's token tile (a ring of 4), issues the four products, commits them to
+// done[s % 4] and requests the token tile of step s + 2 into the stage the
+// products of step s - 2 read (issued two steps earlier: the issuer never
+// waits on the products it has just issued).  Completion c of an mbarrier
+// of a ring of n stages belongs to step stage + n c, so a wait's parity is
+// (s / n) & 1.  Bounded waits:
+// on expiry the CTA sets FMOE_STATUS_WAIT_TIMEOUT, waits (bounded) for its
+// committed products and copies, frees its tensor memory and returns.
 template <int MODE, int BITS>
-__device__ __forceinline__ void tc_gemm_body(const ExpertSet& es, const int4 it, const uint8_t* rec,
+__device__ __forceinline__ void tc_gemm_body(const ExpertSet& es, const int4 it, const uint8_t* rec, int r0, int gb,
                                              const uint8_t* __restrict__ staged, float* __restrict__ out,
                                              unsigned char* tsm, uint64_t* bar_b, uint64_t* bar_m, uint64_t* bar_f,
                                              uint32_t tmem, const int* s_slot, int* s_ok) {
@@ -275,59 +363,74 @@ __device__ __forceinline__ void tc_gemm_body(const ExpertSet& es, const int4 it,
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int K = MODE == 0 ? es.H : es.I;
   const int steps = K / 64;
-  const int r0 = (int)blockIdx.y * kTcRows;
   const uint32_t b_bytes = (uint32_t)N * 128;  // one 64-input step of the staged tokens
+  constexpr int nB = kTcBStages;
   const uint8_t* bsrc = staged + (size_t)it.w * 4 * K;
   auto a_st = [&](int st) { return tsm + (size_t)st * kTcATile; };
-  auto b_st = [&](int st) { return tsm + (size_t)kTcStages * kTcATile + (size_t)st * kTcMaxNp * 2 * 128; };
-  auto par = [](int s) { return (uint32_t)((s / kTcStages) & 1); };
+  auto b_st = [&](int st) { return tsm + (size_t)kTcStages * kTcATile + (size_t)st * b_bytes; };
+  auto raw_buf = [&](int S) { return tsm + (size_t)kTcStages * kTcATile + kTcBRing + (size_t)(S % kTcRawBufs) * kTcRawBuf; };
+  // parities count the CTA's steps over all of its work units (gb: steps before this one)
+  auto par = [&](int s) { return (uint32_t)(((gb + s) / kTcStages) & 1); };
+  auto parb = [&](int s) { return (uint32_t)(((gb + s) / nB) & 1); };
   if (warp < kTcThreads / 32) {
-    // ---- producers: raw words of steps s .. s + 3 in four fixed register
-    // sets, each refilled with step s + 4 right after its use
-    TcRaw rw[kTcAhead];
-#pragma unroll
-    for (int i = 0; i < kTcAhead; ++i) rw[i] = tc_raw_or_zero<MODE, BITS>(rec, es.H, es.I, r0, i, steps);
+    // ---- producers
+    const int SG = steps % kTcMaxSG == 0 ? kTcMaxSG : 4, nsup = steps / SG;
+    tc_issue_super<MODE, BITS>(rec, es.H, es.I, r0, 0, SG, raw_buf(0));
+    cp_async_commit();
+    if (nsup > 1) tc_issue_super<MODE, BITS>(rec, es.H, es.I, r0, 1, SG, raw_buf(1));
+    cp_async_commit();
     bool ok = true;
-    for (int s0 = 0; s0 < steps && ok; s0 += kTcAhead) {
-#pragma unroll
-      for (int i = 0; i < kTcAhead; ++i) {
-        const int s = s0 + i;
-        if (!ok || s >= steps) break;
-        const int st = s % kTcStages;
-        if (s >= kTcStages && !mbar_wait(&bar_m[st], par(s - kTcStages))) {  // products of step s - 3 done
+#pragma unroll 1
+    for (int S = 0; S < nsup; ++S) {
+      cp_async_wait<1>();          // this thread's copies of superstep S have landed
+      ok = producer_bar_and(ok);   // ... and everyone's; buffer (S + 2) % 3 is no longer read
+      if (!ok) break;              // a wait expired somewhere: every producer leaves here
+      if (S + 2 < nsup) tc_issue_super<MODE, BITS>(rec, es.H, es.I, r0, S + 2, SG, raw_buf(S + 2));
+      cp_async_commit();
+      const uint8_t* buf = raw_buf(S);
+      // warps w and w + 4 dequantise the steps s = w (mod 4), inputs
+      // 32 (w / 4) .. + 31 of them, always into A stage s % 4 = w % 4
+#pragma unroll 1
+      for (int j = warp & 3; j < SG; j += kTcStages) {
+        const int s = S * SG + j, st = s % kTcStages, hh = warp >> 2;
+        if (s >= kTcStages && !mbar_wait(&bar_m[st], par(s - kTcStages))) {  // products of step s - 4 done
           ok = false;
           *s_ok = 0;
           break;
         }
-        tc_dequant<BITS>(rw[i], a_st(st));
-        rw[i] = tc_raw_or_zero<MODE, BITS>(rec, es.H, es.I, r0, s + kTcAhead, steps);
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+          const int r = lane + 32 * i;
+          tc_dequant<BITS>(tc_read_raw<MODE, BITS>(buf, j, r, hh), a_st(st), r, hh);
+        }
         fence_proxy_async();  // the generic-proxy A tile is read by the tensor cores
         __syncwarp();
         if (lane == 0) mbar_arrive(&bar_f[st]);
       }
     }
+    cp_async_wait_all();  // no copy may land after the CTA is gone
+    (void)ok;
   } else if (lane == 0) {
     // ---- issuer
     const uint32_t idesc = umma_idesc_f16(kTcRows, N);
     int last_commit = -1, b_issued = -1, b_waited = -1;
     auto issue_b = [&](int s) {
-      const int st = s % kTcStages;
+      const int st = s % nB;
       b_issued = s;
       mbar_expect_tx(&bar_b[st], b_bytes);
       bulk_g2s(b_st(st), bsrc + (size_t)s * b_bytes, b_bytes, &bar_b[st]);
     };
-    issue_b(0);
-    if (steps > 1) issue_b(1);
+    for (int s = 0; s < nB - kTcBLag && s < steps; ++s) issue_b(s);
     bool ok = true;
     for (int s = 0; s < steps; ++s) {
-      const int st = s % kTcStages;
-      if (!mbar_wait(&bar_f[st], par(s)) || !mbar_wait(&bar_b[st], par(s))) {
+      const int st = s % kTcStages, sb = s % nB;
+      if (!mbar_wait(&bar_f[st], par(s)) || !mbar_wait(&bar_b[sb], parb(s))) {
         ok = false;
         break;
       }
       b_waited = s;
       tc_fence_after();
-      const uint32_t a0 = smem_u32(a_st(st)), b0 = smem_u32(b_st(st));
+      const uint32_t a0 = smem_u32(a_st(st)), b0 = smem_u32(b_st(sb));
 #pragma unroll
       for (int j = 0; j < 4; ++j) {  // K = 16 slices: two 8-input chunks each
         const uint64_t ad = umma_desc(a0 + (uint32_t)(2 * j) * (kTcRows / 8) * 128, (kTcRows / 8) * 128, 128);
@@ -336,13 +439,13 @@ __device__ __forceinline__ void tc_gemm_body(const ExpertSet& es, const int4 it,
       }
       umma_commit(&bar_m[st]);
       last_commit = s;
-      // token tile of step s + 2: its stage was read by the products of step s - 1
-      if (s + 2 < steps) {
-        if (s >= 1 && !mbar_wait(&bar_m[(s + 2) % kTcStages], par(s - 1))) {
+      // token tile of step s + nB - kTcBLag: its stage was read by the products of step s - kTcBLag
+      if (s + nB - kTcBLag < steps) {
+        if (s >= kTcBLag && !mbar_wait(&bar_m[(s - kTcBLag) % kTcStages], par(s - kTcBLag))) {
           ok = false;
           break;
         }
-        issue_b(s + 2);
+        issue_b(s + nB - kTcBLag);
       }
     }
     if (!ok) {
@@ -350,7 +453,7 @@ __device__ __forceinline__ void tc_gemm_body(const ExpertSet& es, const int4 it,
       if (last_commit >= 0)  // products complete in order: the last one covers the rest
         (void)mbar_wait(&bar_m[last_commit % kTcStages], par(last_commit));
       for (int q = b_waited + 1; q <= b_issued; ++q)  // token tiles still in flight
-        (void)mbar_wait(&bar_b[q % kTcStages], par(q));
+        (void)mbar_wait(&bar_b[q % nB], parb(q));
     }
   }
   __syncthreads();
@@ -389,27 +492,31 @@ __device__ __forceinline__ void tc_gemm_body(const ExpertSet& es, const int4 it,
   if (!ok && tid == 0) raise_status(FMOE_STATUS_WAIT_TIMEOUT);
 }
 
+// Persistent: CTA c takes the work units c, c + gridDim.x, .. of the
+// n_items[1] x (M / 128) units (item u / tiles, row tile u % tiles), so the
+// grid never holds idle CTAs; tensor memory, mbarriers and rings carry over
+// from unit to unit (steps % 4 == 0 keeps every ring stage in step).
 template <int MODE>
-__global__ void __launch_bounds__(kTcThreads + 32)
+__global__ void __launch_bounds__(kTcThreads + 32, 1)
 tc_gemm_kernel(ExpertSet es, GroupWork w, const uint8_t* __restrict__ staged, float* __restrict__ out) {
   extern __shared__ __align__(1024) unsigned char tsm[];
-  __shared__ uint64_t bar_b[kTcStages], bar_m[kTcStages], bar_f[kTcStages];
+  __shared__ uint64_t bar_b[kTcBStages], bar_m[kTcStages], bar_f[kTcStages];
   __shared__ uint32_t s_tmem;
   __shared__ int s_slot[kTcMaxNp];
   __shared__ int s_ok;
-  if ((int)blockIdx.x >= w.n_items[1]) return;
-  const int4 it = w.tc[blockIdx.x];
-  const int g = it.x, m = it.z, N = 2 * tc_np(m);
+  const int tiles = (MODE == 0 ? 2 * es.I : es.H) / kTcRows;
+  const int steps = (MODE == 0 ? es.H : es.I) / 64;
+  const int units = w.n_items[1] * tiles;
+  if ((int)blockIdx.x >= units) return;
   const int tid = threadIdx.x, warp = tid >> 5;
-  uint32_t ncols = 32;
-  while ((int)ncols < N) ncols <<= 1;
-  for (int i = tid; i < m; i += blockDim.x) s_slot[i] = w.slots[w.offset[g] + it.y + i];
+  constexpr uint32_t ncols = 2 * kTcMaxNp;  // N <= 2 kTcMaxNp fp32 columns, a power of two >= 32
+  static_assert(ncols >= 32 && (ncols & (ncols - 1)) == 0, "tensor memory allocation");
   if (tid == 0) {
     s_ok = 1;
+    for (int i = 0; i < kTcBStages; ++i) mbar_init(&bar_b[i], 1);
     for (int i = 0; i < kTcStages; ++i) {
-      mbar_init(&bar_b[i], 1);
       mbar_init(&bar_m[i], 1);
-      mbar_init(&bar_f[i], kTcThreads / 32);
+      mbar_init(&bar_f[i], 2);  // the two warps that dequantise a step
     }
     asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
   }
@@ -423,19 +530,33 @@ tc_gemm_kernel(ExpertSet es, GroupWork w, const uint8_t* __restrict__ staged, fl
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = s_tmem;
-  int bits;
-  const uint8_t* rec = group_record(es, g, &bits);
-  if (bits == 4) tc_gemm_body<MODE, 4>(es, it, rec, staged, out, tsm, bar_b, bar_m, bar_f, tmem, s_slot, &s_ok);
-  else tc_gemm_body<MODE, 2>(es, it, rec, staged, out, tsm, bar_b, bar_m, bar_f, tmem, s_slot, &s_ok);
-  tc_fence_before();
-  __syncthreads();
+  int gb = 0;
+  for (int u = blockIdx.x; u < units; u += gridDim.x, gb += steps) {
+    const int4 it = w.tc[u / tiles];
+    const int g = it.x, m = it.z, r0 = (u % tiles) * kTcRows;
+    for (int i = tid; i < m; i += blockDim.x) s_slot[i] = w.slots[w.offset[g] + it.y + i];
+    __syncthreads();
+    int bits;
+    const uint8_t* rec = group_record(es, g, &bits);
+    if (bits == 4) tc_gemm_body<MODE, 4>(es, it, rec, r0, gb, staged, out, tsm, bar_b, bar_m, bar_f, tmem, s_slot, &s_ok);
+    else tc_gemm_body<MODE, 2>(es, it, rec, r0, gb, staged, out, tsm, bar_b, bar_m, bar_f, tmem, s_slot, &s_ok);
+    // the epilogue's tensor-memory reads and s_slot uses end before the next unit
+    tc_fence_before();
+    const bool go = __syncthreads_and(s_ok != 0);
+    tc_fence_after();
+    if (!go) break;
+  }
   if (warp == 0) {
     tc_fence_after();
     asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem), "r"(ncols) : "memory");
   }
 }
 
-// Dynamic shared memory of tc_gemm_kernel: the ring of A and B tiles.
-constexpr size_t tc_smem_bytes() { return kTcStages * ((size_t)kTcATile + (size_t)kTcMaxNp * 2 * 128); }
+// Dynamic shared memory of tc_gemm_kernel: the A ring, the token-tile ring
+// and the raw code ring.
+constexpr size_t tc_smem_bytes() {
+  return (size_t)kTcStages * kTcATile + kTcBRing + (size_t)kTcRawBufs * kTcRawBuf;
+}
+static_assert(kTcBLag < kTcStages && kTcBLag < kTcBStages, "ring lags");
 
 }  // namespace fmoe
