@@ -209,8 +209,7 @@ __device__ __forceinline__ void sb_true(uint32_t sbw, int bits, float* s, float*
 //   down codes     [SG groups x words per group][128 rows] u32
 //   down s-b       [SG][128 rows] u32, at kRawDnSbOff
 constexpr int kTcStages = 4;                      // ring of A tiles
-constexpr int kTcBStages = 4;                     // ring of token tiles
-constexpr int kTcBLag = 2;                        // a token tile is refilled once the products 2 steps back are done
+constexpr int kTcBStages = kTcStages;             // token tiles ride with the A stages
 constexpr uint32_t kTcBRing = kTcBStages * kTcMaxNp * 2 * 128;
 constexpr int kTcRawBufs = 3;                     // supersteps in the raw ring
 constexpr int kTcMaxSG = 8;                       // 64-groups per superstep
@@ -338,22 +337,20 @@ __device__ __forceinline__ void mbar_arrive(uint64_t* bar) {
   asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(smem_u32(bar)) : "memory");
 }
 
-// grid (max tensor-core items, M / 128), kTcThreads + 32 threads.  MODE 0:
-// gate/up (M = 2 I, K = H), epilogue SwiGLU -> a[slot][n].  MODE 1: down
-// (M = H, K = I) -> y[slot][row].  Warps 0..7 keep two supersteps of raw
-// codes in flight (see the raw code ring); warps w and w + 4 dequantise the
-// steps s = w (mod 4) (one 64-input group each, one half of its inputs per
-// warp, so four steps are in flight) into A stage s % 4 once the products
-// of step s - 4 are done, and arrive on full[s % 4]; warp 8 (one thread)
-// waits for the A stage and the
-// step's token tile (a ring of 4), issues the four products, commits them to
-// done[s % 4] and requests the token tile of step s + 2 into the stage the
-// products of step s - 2 read (issued two steps earlier: the issuer never
-// waits on the products it has just issued).  Completion c of an mbarrier
-// of a ring of n stages belongs to step stage + n c, so a wait's parity is
-// (s / n) & 1.  Bounded waits:
-// on expiry the CTA sets FMOE_STATUS_WAIT_TIMEOUT, waits (bounded) for its
-// committed products and copies, frees its tensor memory and returns.
+// One work unit (item it, row tile r0) of tc_gemm_kernel.  MODE 0: gate/up
+// (M = 2 I, K = H), epilogue SwiGLU -> a[slot][n].  MODE 1: down (M = H,
+// K = I) -> y[slot][row].  Warps 0..7 keep two supersteps of raw codes in
+// flight (see the raw code ring); warps w and w + 4 handle the steps
+// s = w (mod 4) (one 64-input group each, one half of its inputs per warp,
+// so four steps are in flight): once the products of step s - 4 are done,
+// lane 0 of warp w requests the step's token tile into B stage s % 4, both
+// warps dequantise into A stage s % 4 and arrive on full[s % 4].  Warp 8
+// (one thread) only waits for full[s % 4] and the token tile, issues the
+// four products and commits them to done[s % 4].  Completion c of a stage's
+// mbarriers belongs to the CTA's step stage + 4 c (steps counted over its
+// work units from gb), so a wait's parity is ((gb + s) / 4) & 1.  Bounded
+// waits: on expiry the CTA sets FMOE_STATUS_WAIT_TIMEOUT, waits (bounded)
+// for its committed products and copies and leaves its work loop.
 template <int MODE, int BITS>
 __device__ __forceinline__ void tc_gemm_body(const ExpertSet& es, const int4 it, const uint8_t* rec, int r0, int gb,
                                              const uint8_t* __restrict__ staged, float* __restrict__ out,
@@ -364,14 +361,12 @@ __device__ __forceinline__ void tc_gemm_body(const ExpertSet& es, const int4 it,
   const int K = MODE == 0 ? es.H : es.I;
   const int steps = K / 64;
   const uint32_t b_bytes = (uint32_t)N * 128;  // one 64-input step of the staged tokens
-  constexpr int nB = kTcBStages;
   const uint8_t* bsrc = staged + (size_t)it.w * 4 * K;
   auto a_st = [&](int st) { return tsm + (size_t)st * kTcATile; };
   auto b_st = [&](int st) { return tsm + (size_t)kTcStages * kTcATile + (size_t)st * b_bytes; };
   auto raw_buf = [&](int S) { return tsm + (size_t)kTcStages * kTcATile + kTcBRing + (size_t)(S % kTcRawBufs) * kTcRawBuf; };
   // parities count the CTA's steps over all of its work units (gb: steps before this one)
   auto par = [&](int s) { return (uint32_t)(((gb + s) / kTcStages) & 1); };
-  auto parb = [&](int s) { return (uint32_t)(((gb + s) / nB) & 1); };
   if (warp < kTcThreads / 32) {
     // ---- producers
     const int SG = steps % kTcMaxSG == 0 ? kTcMaxSG : 4, nsup = steps / SG;
@@ -380,6 +375,7 @@ __device__ __forceinline__ void tc_gemm_body(const ExpertSet& es, const int4 it,
     if (nsup > 1) tc_issue_super<MODE, BITS>(rec, es.H, es.I, r0, 1, SG, raw_buf(1));
     cp_async_commit();
     bool ok = true;
+    int b_last = -1;  // last token tile requested by this lane
 #pragma unroll 1
     for (int S = 0; S < nsup; ++S) {
       cp_async_wait<1>();          // this thread's copies of superstep S have landed
@@ -398,6 +394,11 @@ __device__ __forceinline__ void tc_gemm_body(const ExpertSet& es, const int4 it,
           *s_ok = 0;
           break;
         }
+        if (hh == 0 && lane == 0) {  // the step's token tile into B stage s % 4 (free with A stage s % 4)
+          mbar_expect_tx(&bar_b[st], b_bytes);
+          bulk_g2s(b_st(st), bsrc + (size_t)s * b_bytes, b_bytes, &bar_b[st]);
+          b_last = s;
+        }
 #pragma unroll
         for (int i = 0; i < 4; ++i) {
           const int r = lane + 32 * i;
@@ -409,28 +410,22 @@ __device__ __forceinline__ void tc_gemm_body(const ExpertSet& es, const int4 it,
       }
     }
     cp_async_wait_all();  // no copy may land after the CTA is gone
-    (void)ok;
+    // on an early exit, the last token tile this lane requested may still be
+    // in flight (each earlier one was waited for by the issuer)
+    if (!ok && b_last >= 0) (void)mbar_wait(&bar_b[b_last % kTcStages], par(b_last));
   } else if (lane == 0) {
     // ---- issuer
     const uint32_t idesc = umma_idesc_f16(kTcRows, N);
-    int last_commit = -1, b_issued = -1, b_waited = -1;
-    auto issue_b = [&](int s) {
-      const int st = s % nB;
-      b_issued = s;
-      mbar_expect_tx(&bar_b[st], b_bytes);
-      bulk_g2s(b_st(st), bsrc + (size_t)s * b_bytes, b_bytes, &bar_b[st]);
-    };
-    for (int s = 0; s < nB - kTcBLag && s < steps; ++s) issue_b(s);
+    int last_commit = -1;
     bool ok = true;
     for (int s = 0; s < steps; ++s) {
-      const int st = s % kTcStages, sb = s % nB;
-      if (!mbar_wait(&bar_f[st], par(s)) || !mbar_wait(&bar_b[sb], parb(s))) {
+      const int st = s % kTcStages;
+      if (!mbar_wait(&bar_f[st], par(s)) || !mbar_wait(&bar_b[st], par(s))) {
         ok = false;
         break;
       }
-      b_waited = s;
       tc_fence_after();
-      const uint32_t a0 = smem_u32(a_st(st)), b0 = smem_u32(b_st(sb));
+      const uint32_t a0 = smem_u32(a_st(st)), b0 = smem_u32(b_st(st));
 #pragma unroll
       for (int j = 0; j < 4; ++j) {  // K = 16 slices: two 8-input chunks each
         const uint64_t ad = umma_desc(a0 + (uint32_t)(2 * j) * (kTcRows / 8) * 128, (kTcRows / 8) * 128, 128);
@@ -439,21 +434,11 @@ __device__ __forceinline__ void tc_gemm_body(const ExpertSet& es, const int4 it,
       }
       umma_commit(&bar_m[st]);
       last_commit = s;
-      // token tile of step s + nB - kTcBLag: its stage was read by the products of step s - kTcBLag
-      if (s + nB - kTcBLag < steps) {
-        if (s >= kTcBLag && !mbar_wait(&bar_m[(s - kTcBLag) % kTcStages], par(s - kTcBLag))) {
-          ok = false;
-          break;
-        }
-        issue_b(s + nB - kTcBLag);
-      }
     }
     if (!ok) {
       *s_ok = 0;
       if (last_commit >= 0)  // products complete in order: the last one covers the rest
         (void)mbar_wait(&bar_m[last_commit % kTcStages], par(last_commit));
-      for (int q = b_waited + 1; q <= b_issued; ++q)  // token tiles still in flight
-        (void)mbar_wait(&bar_b[q % nB], parb(q));
     }
   }
   __syncthreads();
@@ -557,6 +542,6 @@ tc_gemm_kernel(ExpertSet es, GroupWork w, const uint8_t* __restrict__ staged, fl
 constexpr size_t tc_smem_bytes() {
   return (size_t)kTcStages * kTcATile + kTcBRing + (size_t)kTcRawBufs * kTcRawBuf;
 }
-static_assert(kTcBLag < kTcStages && kTcBLag < kTcBStages, "ring lags");
+
 
 }  // namespace fmoe
