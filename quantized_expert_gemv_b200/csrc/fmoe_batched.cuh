@@ -21,6 +21,7 @@
 
 #include "fmoe.h"
 #include "fmoe_device.cuh"
+#include "fmoe_fused.cuh"  // mbarrier and bulk-copy primitives, lds_group
 #include "fmoe_layout.h"
 
 namespace fmoe {
@@ -335,6 +336,161 @@ gateup_group_kernel(ExpertSet es, GroupWork w, int bucket, int max_items, const 
   constexpr int kPairs = MB <= 4 ? 2 : 1;
   if (bits == 4) gateup_rows_multi<4, MB, kPairs>(rec, es, smem, sxs, m, a, s_slot, p0, p1);
   else gateup_rows_multi<2, MB, kPairs>(rec, es, smem, sxs, m, a, s_slot, p0, p1);
+}
+
+// ------------------------------------------- bulk-copied gate/up GEMV --
+// For the small items (m <= 4 tokens, bound by their weight bytes): a row
+// pair's codes (two contiguous rows) and scale-bias words (two contiguous
+// runs) come into shared memory by two bulk copies, so the bytes in flight
+// are set by shared memory, not by registers.  Warp w takes the pairs
+// p0 + w, p0 + w + 8, .. of the CTA's range and owns two ring slots: while
+// it works on one pair the next one is landing; its lane 0 requests the
+// pair after next into the slot it has just finished.  Needs H / 64 >= 32.
+constexpr int kGuBulkWarps = kGrpThreads / 32;
+constexpr int kGuBulkSlots = 2 * kGuBulkWarps;
+
+__host__ __device__ constexpr size_t gu_bulk_slot_bytes(int H, int bits) {
+  return (size_t)2 * H * bits / 8 + (size_t)2 * (H / 64) * 4;  // two code rows + their scale-bias words
+}
+
+template <int MB>
+__global__ void __launch_bounds__(kGrpThreads, 2)
+gateup_bulk_kernel(ExpertSet es, GroupWork w, int bucket, int max_items, const float* __restrict__ xn,
+                   const unsigned char* __restrict__ xs, float* __restrict__ a, const float* __restrict__ w_sg,
+                   float* __restrict__ gamma) {
+  extern __shared__ __align__(128) unsigned char smem[];
+  __shared__ int s_slot[MB];
+  __shared__ uint64_t full[kGuBulkSlots];
+  if ((int)blockIdx.x >= w.n_items[2 + bucket]) return;
+  const int4 it = w.bitems[(size_t)bucket * max_items + blockIdx.x];
+  const int g = it.x, m = it.z, k1 = es.k + 1;
+  const int H = es.H, I = es.I, ng = H / 64;
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  int bits;
+  const uint8_t* rec = group_record(es, g, &bits);
+  const RecordLayout L = record_layout(bits, H, I);
+  const size_t sxs = (staged_x_bytes(H) + 15) & ~(size_t)15;
+  const uint32_t code_bytes = 2u * (uint32_t)L.gu_row_bytes, sb_bytes = 8u * (uint32_t)ng;
+  const size_t slot_bytes = ((size_t)code_bytes + sb_bytes + 127) & ~(size_t)127;
+  unsigned char* ring = smem + (((size_t)MB * sxs + 127) & ~(size_t)127);
+  int p0, p1;
+  {
+    const int per = (I + gu_split(MB) - 1) / gu_split(MB);
+    p0 = min(I, (int)blockIdx.y * per);
+    p1 = min(I, p0 + per);
+  }
+  if (tid == 0) {
+    for (int i = 0; i < kGuBulkSlots; ++i) mbar_init(&full[i], 1);
+    asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+  }
+  if (tid < m) s_slot[tid] = w.slots[w.offset[g] + it.y + tid];
+  __syncthreads();
+  // pair n into slot q (lane 0 of the owning warp)
+  auto request = [&](int n, int q) {
+    uint8_t* dst = ring + (size_t)q * slot_bytes;
+    mbar_expect_tx(&full[q], code_bytes + sb_bytes);
+    bulk_g2s(dst, rec + L.gu_codes + (size_t)(2 * n) * L.gu_row_bytes, code_bytes, &full[q]);
+    bulk_g2s(dst + code_bytes, rec + L.gu_sb + (size_t)(2 * n) * ng * 4, sb_bytes, &full[q]);
+  };
+  if (lane == 0) {
+    if (p0 + warp < p1) request(p0 + warp, 2 * warp);
+    if (p0 + warp + kGuBulkWarps < p1) request(p0 + warp + kGuBulkWarps, 2 * warp + 1);
+  }
+  // the tokens' staged inputs (and the shared expert's gates) while the first pairs land
+  for (int i = 0; i < m; ++i) {
+    const uint4* src = reinterpret_cast<const uint4*>(xs + (size_t)(s_slot[i] / k1) * sxs);
+    uint4* dst = reinterpret_cast<uint4*>(smem + (size_t)i * sxs);
+    for (int j = tid; j < (int)(sxs / 16); j += kGrpThreads) dst[j] = __ldcg(src + j);
+  }
+  if (gamma && g == es.E && blockIdx.y == 0) {
+    for (int i = warp; i < m; i += kGuBulkWarps) {
+      const float* x = xn + (size_t)(s_slot[i] / k1) * H;
+      float z = 0.f;
+#pragma unroll 8
+      for (int c = lane * 4; c < H; c += 128) {
+        const float4 wv = __ldg(reinterpret_cast<const float4*>(w_sg + c));
+        const float4 v = __ldg(reinterpret_cast<const float4*>(x + c));
+        z = fmaf(wv.x, v.x, z);
+        z = fmaf(wv.y, v.y, z);
+        z = fmaf(wv.z, v.z, z);
+        z = fmaf(wv.w, v.w, z);
+      }
+      z = warp_sum(z);
+      if (lane == 0) gamma[s_slot[i] / k1] = 1.f / (1.f + expf(-z));
+    }
+  }
+  __syncthreads();
+  bool ok = true;
+  int kk = 0;
+  for (int n = p0 + warp; n < p1; n += kGuBulkWarps, ++kk) {
+    const int q = 2 * warp + (kk & 1);
+    if (!mbar_wait(&full[q], (uint32_t)((kk >> 1) & 1))) {
+      ok = false;
+      break;
+    }
+    const uint8_t* rows = ring + (size_t)q * slot_bytes;
+    const uint32_t* sbw = reinterpret_cast<const uint32_t*>(rows + code_bytes);
+    float yg[MB], yu[MB];
+#pragma unroll
+    for (int i = 0; i < MB; ++i) yg[i] = yu[i] = 0.f;
+    for (int g0 = lane; g0 < ng; g0 += 32) {
+      if (bits == 4) {
+        const GroupCodes<4> cg = lds_group<4>(rows, ng, g0), cu = lds_group<4>(rows + L.gu_row_bytes, ng, g0);
+        const uint32_t sg = sbw[g0], su = sbw[ng + g0];
+#pragma unroll
+        for (int i = 0; i < MB; ++i) {
+          if (i < m) {
+            const StagedX sx = staged_i(smem, sxs, i, H);
+            uint4 xv[8];
+            load_xv(sx, ng, g0, xv);
+            yg[i] = group_epilogue(yg[i], sg, group_dot<4>(cg, xv), sx.delta[g0], sx.xsum[g0]);
+            yu[i] = group_epilogue(yu[i], su, group_dot<4>(cu, xv), sx.delta[g0], sx.xsum[g0]);
+          }
+        }
+      } else {
+        const GroupCodes<2> cg = lds_group<2>(rows, ng, g0), cu = lds_group<2>(rows + L.gu_row_bytes, ng, g0);
+        const uint32_t sg = sbw[g0], su = sbw[ng + g0];
+#pragma unroll
+        for (int i = 0; i < MB; ++i) {
+          if (i < m) {
+            const StagedX sx = staged_i(smem, sxs, i, H);
+            uint4 xv[8];
+            load_xv(sx, ng, g0, xv);
+            yg[i] = group_epilogue(yg[i], sg, group_dot<2>(cg, xv), sx.delta[g0], sx.xsum[g0]);
+            yu[i] = group_epilogue(yu[i], su, group_dot<2>(cu, xv), sx.delta[g0], sx.xsum[g0]);
+          }
+        }
+      }
+    }
+    __syncwarp();
+    // the slot is read: it takes the pair after next
+    if (lane == 0 && n + 2 * kGuBulkWarps < p1) {
+      fence_proxy_async();
+      request(n + 2 * kGuBulkWarps, q);
+    }
+#pragma unroll
+    for (int i = 0; i < MB; ++i) {
+      if (i < m) {
+        const float gs = warp_sum(yg[i]), us = warp_sum(yu[i]);
+        if (lane == 0) a[(size_t)s_slot[i] * I + n] = silu_mul(gs, us);
+      }
+    }
+  }
+  if (!ok) {
+    // leave no copy in flight: this warp's slots still owed a completion
+    if (lane == 0) {
+      for (int j = 0; j < 2; ++j) {
+        const int n2 = p0 + warp + (kk + j) * kGuBulkWarps;
+        if (n2 < p1) (void)mbar_wait(&full[2 * warp + ((kk + j) & 1)], (uint32_t)(((kk + j) >> 1) & 1));
+      }
+      raise_status(FMOE_STATUS_WAIT_TIMEOUT);
+    }
+  }
+}
+
+__host__ __device__ constexpr size_t gu_bulk_smem(int MB, int H, int bits) {
+  return (((size_t)MB * ((staged_x_bytes(H) + 15) & ~(size_t)15) + 127) & ~(size_t)127) +
+         (size_t)kGuBulkSlots * ((gu_bulk_slot_bytes(H, bits) + 127) & ~(size_t)127);
 }
 
 // Down product of one record for one hidden row and the m tokens staged at

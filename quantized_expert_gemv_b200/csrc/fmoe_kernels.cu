@@ -641,7 +641,7 @@ static int g_tc_enabled = 1;  // tensor-core products for groups of >= kTcMinTok
 
 // Dynamic shared memory above the default 48 KB for a kernel, set once per device.
 static bool smem_optin(const void* fn, size_t bytes, int slot) {
-  static size_t done[64][8];
+  static size_t done[64][32];
   int dev = 0;
   if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return false;
   if (done[dev][slot] >= bytes) return true;
@@ -659,10 +659,23 @@ static bool grp_optin(size_t gu_smem, size_t dn_smem, int b) {
          smem_optin(reinterpret_cast<const void*>(&down_group_kernel<MB>), dn_smem, 12 + b);
 }
 
+// Small items (MB <= 4) go through the bulk-copied kernel when a row pair
+// is whole warp-widths of groups (H / 64 >= 32) and its ring fits.
+template <int MB>
+static bool gu_bulk_ok(const ExpertSet& es) {
+  if (MB > 4 || es.H / 64 < 32) return false;
+  return smem_optin(reinterpret_cast<const void*>(&gateup_bulk_kernel<MB>), gu_bulk_smem(MB, es.H, 4), 16 + MB);
+}
+
 template <int MB>
 static void grp_launch_gu(const ExpertSet& es, const GroupWork& gw, int b, int items, int grid, const float* xn,
                           const unsigned char* xs, float* a, const float* w_sg, float* gamma, size_t sxs,
                           cudaStream_t st) {
+  if (gu_bulk_ok<MB>(es)) {
+    gateup_bulk_kernel<(MB <= 4 ? MB : 4)><<<dim3(grid, gu_split(MB)), kGrpThreads, gu_bulk_smem(MB, es.H, 4), st>>>(
+        es, gw, b, items, xn, xs, a, w_sg, gamma);
+    return;
+  }
   gateup_group_kernel<MB><<<dim3(grid, gu_split(MB)), kGrpThreads, MB * sxs, st>>>(es, gw, b, items, xn, xs, a, w_sg,
                                                                              gamma);
 }
