@@ -396,6 +396,32 @@ def test_grouped_experts_many_tokens_per_expert(wl, tc_path):
     assert fm.fmoe_read_status() == 0
 
 
+@pytest.mark.parametrize("wl", [synth.Workload(n_experts=32, bits=2)], ids=["int2-32"])
+def test_batched_full_size_int2_every_item_size(wl, tc_path):
+    """hidden 4096 / inter 1024, 2-bit routed experts, 24 tokens on given
+    logits chosen so that every kind of work item occurs: experts with 2
+    tokens and with 3 tokens (the bulk-copied small-item GEMV), 4-5 tokens
+    and 6 and 24 tokens (tensor cores from 5 tokens on), and the 4-bit
+    shared expert with all 24; sampled tokens checked against the oracle."""
+    T = 24
+    lw = device_layer(wl)
+    lw_o = oracle_layer(wl, 0, slots=[wl.n_experts])
+    lg = np.zeros((T, wl.n_experts), np.float32)
+    for t in range(T):
+        picks = [0, 1 if t < 6 else 2 + t % 4, 10 + t % 8, 20 + t % 12]
+        lg[t, picks] = [4.0, 3.0, 2.0, 1.0]
+    counts = np.bincount(np.argsort(-lg, axis=1)[:, :4].ravel(), minlength=wl.n_experts)
+    assert {2, 3, 6, 24} <= set(counts.tolist()) and (counts[2:6] >= 4).all()
+    x = synth.tokens(wl, T, stream=47)
+    h, xn = dev(x), dev(x)
+    ws = fm.alloc_workspace(lw.desc, T)
+    fm.fmoe_layer_forward_logits(lw, dev(lg), h, xn, ws)
+    for t in (0, 5, 6, 13, 23):
+        check_layer_token(wl, lw_o, ws, lw.desc, T, t, x[t], x[t], host(h)[t], host(xn)[t], f"t={t}",
+                          logits_given=True)
+    assert fm.fmoe_read_status() == 0
+
+
 def test_tensor_core_and_integer_paths_differ_only_by_rounding():
     """The two implementations of the grouped products both run (their
     results are not bit-identical) and agree well inside the tolerance."""
