@@ -85,6 +85,42 @@ def batched_measure(fm, synth, np, torch, lw, wl, stream, steps=50, warmup=5, T=
             "timing": "CUDA events on the launching stream, 50 consecutive steps"}
 
 
+def small_batch_measure(fm, synth, torch, layers, wl, stream, Ts=(2, 4, 8), rotations=20):
+    """T tokens (2-15: a small decode batch or a speculative-verify step)
+    carried through the resident layer stack, routed by the layers' own
+    routers: one CUDA graph replay per rotation of the stack, CUDA events
+    around `rotations` replays.  Per T: microseconds per layer and token-
+    layers per second."""
+    out = {}
+    L = len(layers)
+    for T in Ts:
+        x = torch.from_numpy(synth.tokens(wl, T, stream=950 + T)).cuda()
+        h, xn = x.clone(), x.clone()
+        ws = fm.alloc_workspace(layers[0].desc, T)
+        g = torch.cuda.CUDAGraph()
+        with torch.cuda.stream(stream):
+            fm.fmoe_stack_forward(layers, h, xn, ws, stream=stream)
+            stream.synchronize()
+            with torch.cuda.graph(g, stream=stream):
+                fm.fmoe_stack_forward(layers, h, xn, ws, stream=stream)
+            for _ in range(3):
+                g.replay()
+        torch.cuda.synchronize()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        with torch.cuda.stream(stream):
+            e0.record(stream)
+            for _ in range(rotations):
+                g.replay()
+            e1.record(stream)
+        e1.synchronize()
+        us = e0.elapsed_time(e1) * 1e3 / (rotations * L)
+        out[str(T)] = {"us_per_layer": us, "layer_fwd_per_s": 1e6 / us, "token_layers_per_s": T * 1e6 / us}
+        del g
+    return {"workload": f"moe_stack_int4_small_batch: T tokens through the {L} resident int4 layers (routed by "
+                        f"their routers), {rotations} graph replays of the stack per T",
+            "by_T": out}
+
+
 def int2_chain_measure(fm, synth, torch, stream, layers=20, steps=2000, warmup=100):
     """The 2-bit variant of the layer stack (routed experts 2-bit, shared
     expert 4-bit), one token carried through all layers: layers/s."""
@@ -462,6 +498,7 @@ def run_ours(args):
     line["tokens_per_s"] = value / L  # one token through the L-layer stack
     if not args.no_extra and wl.n_experts == 512:
         line["batched"] = batched_measure(fm, synth, np, torch, layers[0], wl, stream)
+        line["small_batch"] = small_batch_measure(fm, synth, torch, layers, wl, stream)
         del layers, graphs, g_all
         graphs = g_all = None
         torch.cuda.empty_cache()

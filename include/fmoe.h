@@ -248,6 +248,14 @@ int fmoe_set_fused(int enable);
  * process-wide setting, returns the previous value. */
 int fmoe_set_tensor_cores(int enable);
 
+/* Largest token count T for which fmoe_layer_forward (stack == 0) or
+ * fmoe_stack_forward (stack != 0) runs the tokens one by one through the
+ * persistent T = 1 kernel (when enabled, fmoe_set_fused): 4 and 8.  Such
+ * calls compute each token exactly as a T = 1 call on that token would and
+ * leave, like T = 1, no per-expert outputs y in the workspace; larger T take
+ * the grouped path. */
+int fmoe_fused_max_tokens(int stack);
+
 /* Tokens an expert needs in a step for its products to run on the tensor
  * cores (when enabled): 5.  From about five tokens per expert the
  * integer-dot matrix-vector path is bound by its dot products rather than by

@@ -91,6 +91,7 @@ _SIGS = {
     "fmoe_fused_supported": (_i32, [_PDESC]),
     "fmoe_set_tensor_cores": (_i32, [_i32]),
     "fmoe_tc_min_tokens": (_i32, []),
+    "fmoe_fused_max_tokens": (_i32, [_i32]),
     "fmoe_layer_forward_noalloc": (_i32, [_PW, _vp, _vp, _i32, _vp]),
 }
 for _name, (_res, _args) in _SIGS.items():
@@ -325,6 +326,11 @@ def fmoe_set_tensor_cores(enable: bool) -> bool:
 def fmoe_tc_min_tokens() -> int:
     """Tokens an expert needs in a step for the tensor-core products."""
     return int(_lib.fmoe_tc_min_tokens())
+
+
+def fmoe_fused_max_tokens(stack: bool = False) -> int:
+    """Largest T run token by token through the persistent kernel (layer or stack call)."""
+    return int(_lib.fmoe_fused_max_tokens(int(bool(stack))))
 
 
 def fmoe_set_fused(enable: bool) -> bool:

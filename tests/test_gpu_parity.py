@@ -72,7 +72,7 @@ def check_layer_token(wl, lw_o, ws, desc, T, t, h_in, xn_in, h_out, xn_out, labe
     outputs y (left in the workspace by the one-kernel-per-step path only;
     the persistent kernel sums them on the fly), h' and xn' against the
     oracle."""
-    fused = T == 1 and not logits_given and fused_on() and fm.fmoe_fused_supported(desc)
+    fused = T <= fm.fmoe_fused_max_tokens() and not logits_given and fused_on() and fm.fmoe_fused_supported(desc)
     lg_d = host(fm.workspace_view(ws, desc, T, fm.WS_LOGITS))[t]
     ids_d = host(fm.workspace_view(ws, desc, T, fm.WS_IDS))[t]
     p_d = host(fm.workspace_view(ws, desc, T, fm.WS_WEIGHTS))[t]
@@ -419,6 +419,42 @@ def test_batched_full_size_int2_every_item_size(wl, tc_path):
     for t in (0, 5, 6, 13, 23):
         check_layer_token(wl, lw_o, ws, lw.desc, T, t, x[t], x[t], host(h)[t], host(xn)[t], f"t={t}",
                           logits_given=True)
+    assert fm.fmoe_read_status() == 0
+
+
+@pytest.mark.parametrize("wl", [synth.TINY, SMALL], ids=["tiny4", "small4"])
+def test_few_tokens_run_token_by_token(wl):
+    """Up to fmoe_fused_max_tokens tokens, a layer call and a stack call give
+    each token exactly the bits of a T = 1 call on that token; one token
+    more takes the grouped path and agrees within the tolerance."""
+    if not fm.fmoe_fused_supported(device_layer(wl).desc):
+        pytest.skip("persistent kernel does not fit this shape here")
+    lws = [device_layer(wl, l) for l in range(3)]
+    for stack, T in ((False, fm.fmoe_fused_max_tokens(False)), (True, fm.fmoe_fused_max_tokens(True))):
+        x = synth.tokens(wl, T + 1, stream=61)
+        want = []
+        for t in range(T + 1):
+            h1, xn1 = dev(x[t:t + 1]), dev(x[t:t + 1])
+            ws1 = fm.alloc_workspace(lws[0].desc, 1)
+            if stack:
+                fm.fmoe_stack_forward(lws, h1, xn1, ws1)
+            else:
+                fm.fmoe_layer_forward(lws[0], h1, xn1, ws1)
+            want.append((host(h1)[0], host(xn1)[0]))
+        for n in (T, T + 1):
+            h, xn = dev(x[:n]), dev(x[:n])
+            ws = fm.alloc_workspace(lws[0].desc, n)
+            if stack:
+                fm.fmoe_stack_forward(lws, h, xn, ws)
+            else:
+                fm.fmoe_layer_forward(lws[0], h, xn, ws)
+            got_h, got_xn = host(h), host(xn)
+            for t in range(n):
+                if n == T:
+                    assert np.array_equal(got_h[t], want[t][0]) and np.array_equal(got_xn[t], want[t][1]), (stack, t)
+                else:
+                    rel = np.linalg.norm(got_xn[t] - want[t][1]) / np.linalg.norm(want[t][1])
+                    assert rel <= 2e-3, (stack, t, rel)
     assert fm.fmoe_read_status() == 0
 
 
