@@ -71,6 +71,8 @@ def lib() -> ctypes.CDLL:
         L.oracle_layer_token.restype = i32
         L.oracle_quantize.argtypes = [vp, ctypes.c_size_t, i32, i32, vp, vp, vp]
         L.oracle_quantize.restype = None
+        L.oracle_quantize_f32.argtypes = [vp, ctypes.c_size_t, i32, i32, vp, vp, vp]
+        L.oracle_quantize_f32.restype = None
         L.oracle_dequantize.argtypes = [vp, vp, vp, i32, i32, i32, vp]
         L.oracle_dequantize.restype = None
         _lib = L
@@ -219,6 +221,18 @@ def quantize(w, G: int, bits: int):
     s = np.empty(w.size // G)
     b = np.empty(w.size // G)
     lib().oracle_quantize(_p(w), w.size, G, bits, _p(q), _p(s), _p(b))
+    return q, s, b
+
+
+def quantize_f32(w, G: int, bits: int):
+    """The stored-format quantiser in fp32 (oracle.c, oracle_quantize_f32):
+    returns (q uint8, scale bf16 bits uint16, bias bf16 bits uint16)."""
+    w = _c(w, np.float32).ravel()
+    n_groups = w.size // G
+    q = np.empty(w.size, np.uint8)
+    s = np.empty(n_groups, np.uint16)
+    b = np.empty(n_groups, np.uint16)
+    lib().oracle_quantize_f32(_p(w), n_groups, G, bits, _p(q), _p(s), _p(b))
     return q, s, b
 
 

@@ -288,6 +288,58 @@ void oracle_quantize(const double* w, size_t n, int G, int bits, uint8_t* q, dou
   }
 }
 
+/* fp32 -> bf16 bit pattern, round to nearest, ties to even (finite inputs). */
+static uint16_t oracle_f32_to_bf16(float f) {
+  uint32_t u;
+  memcpy(&u, &f, 4);
+  u += 0x7FFFu + ((u >> 16) & 1u);
+  return (uint16_t)(u >> 16);
+}
+
+static float oracle_bf16_f32(uint16_t h) {
+  uint32_t u = (uint32_t)h << 16;
+  float f;
+  memcpy(&f, &u, 4);
+  return f;
+}
+
+/* The stored-format quantiser (fp32 weights -> codes + bf16 scale/bias),
+ * the offline conversion step the pages' conclusion mentions, with every
+ * decision taken in fp32 exactly as written here: per group of G values
+ * lo = min (+0 for a -0 minimum), hi = max; s = (hi - lo) / (2^bits - 1)
+ * (one fp32 division),
+ * stored as bf16 (round to nearest even), b = lo stored as bf16; with the
+ * stored values S and B, q = rint((w - B) / S) (fp32 subtraction and
+ * division, ties to even) clamped to [0, 2^bits - 1], and q = 0 where S = 0.
+ * Finite inputs only. */
+void oracle_quantize_f32(const float* w, size_t n_groups, int G, int bits, uint8_t* q, uint16_t* s,
+                         uint16_t* b) {
+  const int qmax = (1 << bits) - 1;
+  for (size_t g = 0; g < n_groups; ++g) {
+    const float* x = w + g * (size_t)G;
+    float lo = x[0], hi = x[0];
+    for (int j = 1; j < G; ++j) {
+      if (x[j] < lo) lo = x[j];
+      if (x[j] > hi) hi = x[j];
+    }
+    lo = lo + 0.0f;  /* a -0 minimum is stored as +0 */
+    const float sc = (hi - lo) / (float)qmax;
+    s[g] = oracle_f32_to_bf16(sc);
+    b[g] = oracle_f32_to_bf16(lo);
+    const float S = oracle_bf16_f32(s[g]), B = oracle_bf16_f32(b[g]);
+    for (int j = 0; j < G; ++j) {
+      float c = 0.0f;
+      if (S > 0.0f) {
+        const float t = (x[j] - B) / S;
+        c = nearbyintf(t);
+        if (c < 0.0f) c = 0.0f;
+        if (c > (float)qmax) c = (float)qmax;
+      }
+      q[g * (size_t)G + j] = (uint8_t)c;
+    }
+  }
+}
+
 /* Dequantise a whole matrix: w[r][j] = q[r][j] * s[r][j/G] + b[r][j/G]. */
 void oracle_dequantize(const uint8_t* q, const uint16_t* s, const uint16_t* b, int rows,
                        int cols, int G, double* w) {

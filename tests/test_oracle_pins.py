@@ -361,6 +361,46 @@ def test_quantiser_error_at_most_half_step():
         assert np.all(np.abs(back - w) <= np.repeat(s, 64) / 2 * (1 + 1e-12))
 
 
+@pytest.mark.parametrize("bits", [4, 2])
+def test_stored_format_quantiser_recovers_exact_inputs(bits):
+    """Weights that are q * S + B with bf16 S, B (each group holding both
+    code extremes) come back as exactly q, S, B from the fp32 quantiser."""
+    r = rng(21 + bits)
+    G, n_groups = 64, 48
+    qmax = (1 << bits) - 1
+    q = r.integers(0, qmax + 1, size=(n_groups, G), dtype=np.uint8)
+    q[:, 0], q[:, 1] = 0, qmax
+    # S and B chosen so that every q * S + B is exact in fp32 and (hi - lo) / qmax == S exactly
+    S = synth.f32_to_bf16((2.0 ** r.integers(-9, -3, size=n_groups)).astype(np.float32))
+    B = synth.f32_to_bf16((-(2.0 ** r.integers(-6, 0, size=n_groups)) * r.integers(1, 4, size=n_groups)).astype(np.float32))
+    Sf, Bf = synth.bf16_to_f32(S), synth.bf16_to_f32(B)
+    w = (q.astype(np.float32) * Sf[:, None] + Bf[:, None]).astype(np.float32)
+    assert np.array_equal(w.astype(np.float64), q * Sf[:, None].astype(np.float64) + Bf[:, None])  # exact
+    q2, s2, b2 = oracle.quantize_f32(w, G, bits)
+    assert np.array_equal(q2.reshape(n_groups, G), q)
+    assert np.array_equal(s2, S) and np.array_equal(b2, B)
+
+
+def test_stored_format_quantiser_error_bound_and_special_groups():
+    """Round-trip error of the fp32 quantiser: at most S/2, plus what the
+    bf16 rounding of the scale (qmax of its half-ulp) and of the bias can
+    add; a constant group gives scale 0 and codes 0; negative and positive
+    groups alike."""
+    r = rng(22)
+    for bits in (4, 2):
+        qmax = (1 << bits) - 1
+        w = np.concatenate([r.normal(size=64 * 30), r.normal(loc=5.0, size=64 * 5), -r.uniform(1, 3, 64 * 5),
+                            np.full(64, 0.375)]).astype(np.float32)
+        q, s, b = oracle.quantize_f32(w, 64, bits)
+        S, B = synth.bf16_to_f32(s).astype(np.float64), synth.bf16_to_f32(b).astype(np.float64)
+        back = q.astype(np.float64) * np.repeat(S, 64) + np.repeat(B, 64)
+        lo = w.reshape(-1, 64).min(axis=1).astype(np.float64)
+        bound = S / 2 + qmax * S * 2.0 ** -8 + np.abs(lo) * 2.0 ** -8 + 1e-12
+        assert np.all(np.abs(back - w).reshape(-1, 64) <= bound[:, None])
+        assert s[-1] == 0 and np.all(q[-64:] == 0) and synth.bf16_to_f32(b[-1:])[0] == np.float32(0.375)
+        assert q.max() <= qmax
+
+
 # ------------------------------------------------------------ byte counts ----
 
 def _golden():
