@@ -156,6 +156,21 @@ int fmoe_pack_experts_device(const uint8_t* d_q, const uint16_t* d_scale, const 
                              int bits, int n_experts, int hidden, int inter, int group,
                              void* d_packed, size_t d_bytes, cudaStream_t stream);
 
+/* Stored-format quantiser ("What is Flash-MoE?", conclusion: the offline
+ * conversion of trained weights into the 4-bit / 2-bit expert files): the
+ * fp32 weights d_w [n_groups][group] (device, e.g. the logical expert
+ * matrices above, row-major) become codes d_q [n_groups][group] (one per
+ * byte) and bf16 bit patterns d_scale, d_bias [n_groups], the inputs of
+ * fmoe_pack_experts_device.  Per group: lo = min (+0 for -0), hi = max,
+ * scale = bf16(fp32 (hi - lo) / (2^bits - 1)), bias = bf16(lo) (round to
+ * nearest even), q = rint((w - bias) / scale) in fp32 clamped to
+ * [0, 2^bits - 1] (q = 0 for scale 0).  Finite inputs only; all pointers
+ * 16-byte aligned; asynchronous on `stream`.
+ * Errors: FMOE_ERR_INVALID_ARG (null or misaligned), FMOE_ERR_UNSUPPORTED
+ * (group != 64 or bits not 2 / 4), FMOE_ERR_CUDA. */
+int fmoe_quantize_groups(const float* d_w, size_t n_groups, int group, int bits, uint8_t* d_q,
+                         uint16_t* d_scale, uint16_t* d_bias, cudaStream_t stream);
+
 /* ----------------------------------------------------------- workspace -- */
 /* Device workspace for T tokens of a layer with descriptor d (bytes).  The
  * workspace holds intermediates (router partial sums, logits, ids, gate

@@ -91,6 +91,7 @@ _SIGS = {
     "fmoe_fused_supported": (_i32, [_PDESC]),
     "fmoe_set_tensor_cores": (_i32, [_i32]),
     "fmoe_tc_min_tokens": (_i32, []),
+    "fmoe_quantize_groups": (_i32, [_vp, _sz, _i32, _i32, _vp, _vp, _vp, _vp]),
     "fmoe_fused_max_tokens": (_i32, [_i32]),
     "fmoe_layer_forward_noalloc": (_i32, [_PW, _vp, _vp, _i32, _vp]),
 }
@@ -321,6 +322,17 @@ def fmoe_set_tensor_cores(enable: bool) -> bool:
     """Selects tensor-core products (True, default) or the integer-dot path for the
     heavily routed experts of the T > 1 path; returns the previous setting."""
     return bool(_lib.fmoe_set_tensor_cores(int(bool(enable))))
+
+
+def fmoe_quantize_groups(w, bits: int, q, scale, bias, stream=None) -> None:
+    """Quantises the fp32 device tensor w (64-value groups, contiguous) into
+    codes q (uint8, one per value) and bf16 bit patterns scale, bias (int16 or
+    uint16 tensors, one per group), caller-allocated."""
+    n = w.numel()
+    if n % 64:
+        raise ValueError("w must hold whole 64-value groups")
+    rc = _lib.fmoe_quantize_groups(_ptr(w), n // 64, 64, bits, _ptr(q), _ptr(scale), _ptr(bias), _stream(stream))
+    _check(rc, "fmoe_quantize_groups")
 
 
 def fmoe_tc_min_tokens() -> int:

@@ -19,6 +19,7 @@
 #include <cstring>
 #include <mutex>
 
+#include <cuda_bf16.h>
 #include <cuda_runtime.h>
 
 #include "fmoe.h"
@@ -411,6 +412,45 @@ combine_kernel(const float* __restrict__ y, const float* __restrict__ weights,
   const float r = 1.f / sqrtf(ss / (float)H + eps);
   for (int i = threadIdx.x; i < H; i += blockDim.x)
     xn_out[(size_t)t * H + i] = h_out[(size_t)t * H + i] * r * norm_w[i];
+}
+
+// ---------------------------------------------------------- quantiser ----
+// Stored-format quantiser: fp32 weights, 64-group min/max affine codes with
+// bf16 scale and bias (the offline conversion the pages' conclusion
+// mentions; "What is Flash-MoE?", conclusion).  One warp per group, lane l
+// holds inputs 2l, 2l+1.  Every decision in fp32 with correctly rounded
+// operations: lo = min (+0 for -0), hi = max, s = (hi - lo) / (2^bits - 1),
+// S = bf16(s), B = bf16(lo) (round to nearest even), q = rint((w - B) / S)
+// clamped to [0, 2^bits - 1], q = 0 where S = 0.
+__global__ void __launch_bounds__(256)
+quantize_groups_kernel(const float* __restrict__ w, size_t n_groups, int bits, uint8_t* __restrict__ q,
+                       uint16_t* __restrict__ scale, uint16_t* __restrict__ bias) {
+  const int lane = threadIdx.x & 31;
+  const size_t nw = ((size_t)gridDim.x * blockDim.x) >> 5;
+  const float qmax = (float)((1 << bits) - 1);
+  for (size_t g = ((size_t)blockIdx.x * blockDim.x + threadIdx.x) >> 5; g < n_groups; g += nw) {
+    const float2 v = reinterpret_cast<const float2*>(w + g * 64)[lane];
+    float lo = fminf(v.x, v.y), hi = fmaxf(v.x, v.y);
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) {
+      lo = fminf(lo, __shfl_xor_sync(0xffffffffu, lo, o));
+      hi = fmaxf(hi, __shfl_xor_sync(0xffffffffu, hi, o));
+    }
+    lo = __fadd_rn(lo, 0.0f);
+    const __nv_bfloat16 sb = __float2bfloat16_rn(__fdiv_rn(__fsub_rn(hi, lo), qmax));
+    const __nv_bfloat16 bb = __float2bfloat16_rn(lo);
+    const float S = __bfloat162float(sb), B = __bfloat162float(bb);
+    auto code = [&](float x) -> uint32_t {
+      if (!(S > 0.f)) return 0u;
+      const float c = fminf(fmaxf(rintf(__fdiv_rn(__fsub_rn(x, B), S)), 0.f), qmax);
+      return (uint32_t)c;
+    };
+    reinterpret_cast<uchar2*>(q + g * 64)[lane] = make_uchar2((unsigned char)code(v.x), (unsigned char)code(v.y));
+    if (lane == 0) {
+      scale[g] = __bfloat16_as_ushort(sb);
+      bias[g] = __bfloat16_as_ushort(bb);
+    }
+  }
 }
 
 // ------------------------------------------------------- device packer ----
@@ -1105,6 +1145,17 @@ extern "C" int fmoe_pack_experts_device(const uint8_t* d_q, const uint16_t* d_sc
   else
     pack_codes_kernel<2><<<blocks, 256, 0, stream>>>(d_q, n_experts, hidden, inter, out);
   pack_sb_kernel<<<blocks, 256, 0, stream>>>(d_scale, d_bias, bits, n_experts, hidden, inter, out);
+  return cuda_rc(cudaGetLastError());
+}
+
+extern "C" int fmoe_quantize_groups(const float* d_w, size_t n_groups, int group, int bits, uint8_t* d_q,
+                                    uint16_t* d_scale, uint16_t* d_bias, cudaStream_t stream) {
+  if (!d_w || !d_q || !d_scale || !d_bias) return FMOE_ERR_INVALID_ARG;
+  if (!aligned16(d_w) || !aligned16(d_q) || !aligned16(d_scale) || !aligned16(d_bias)) return FMOE_ERR_INVALID_ARG;
+  if (group != 64 || (bits != 4 && bits != 2)) return FMOE_ERR_UNSUPPORTED;
+  if (n_groups == 0) return FMOE_OK;
+  const size_t warps = n_groups < (size_t)148 * 64 ? n_groups : (size_t)148 * 64;
+  quantize_groups_kernel<<<(unsigned)((warps + 7) / 8), 256, 0, stream>>>(d_w, n_groups, bits, d_q, d_scale, d_bias);
   return cuda_rc(cudaGetLastError());
 }
 

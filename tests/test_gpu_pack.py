@@ -65,3 +65,61 @@ def test_device_packer_flags_bad_codes():
     fm.fmoe_read_status(clear=True)
     fm.fmoe_pack_experts_device(q, s, b, 4, 1, H, I, out)
     assert fm.fmoe_read_status(clear=True) & fm.FMOE_STATUS_BAD_PACK_INPUT
+
+
+def _quantiser_inputs(n_groups, seed):
+    """fp32 weights of the expert scale (normal, 0.02), plus groups that test
+    the edge cases: constant, signed zeros at the minimum, all negative,
+    large magnitude, exact code grids, a tiny range."""
+    r = np.random.default_rng(seed)
+    w = (r.normal(size=(n_groups, 64)) * 0.02).astype(np.float32)
+    w[0] = 0.125
+    w[1] = r.normal(size=64).astype(np.float32) ** 2
+    w[1, :3] = [-0.0, 0.0, -0.0]
+    w[2] = -r.uniform(1.0, 2.0, size=64)
+    w[3] = r.normal(size=64) * 3e4
+    w[4] = (r.integers(0, 16, size=64) * np.float32(2 ** -7) - np.float32(0.5)).astype(np.float32)
+    w[5] = np.float32(1.0) + r.uniform(0, 1e-6, size=64).astype(np.float32)
+    return w
+
+
+@pytest.mark.parametrize("bits", [4, 2])
+def test_device_quantiser_matches_oracle(bits):
+    """Codes, bf16 scales and biases bit for bit against the oracle's fp32
+    quantiser, at a full expert's worth of groups."""
+    import oracle
+    n_groups = 3 * 4096 * 1024 // 64
+    w = _quantiser_inputs(n_groups, 40 + bits)
+    q_ref, s_ref, b_ref = oracle.quantize_f32(w, 64, bits)
+    wd = torch.from_numpy(w).cuda()
+    q = torch.empty(w.size, dtype=torch.uint8, device="cuda")
+    sc = torch.empty(n_groups, dtype=torch.int16, device="cuda")
+    bi = torch.empty(n_groups, dtype=torch.int16, device="cuda")
+    fm.fmoe_quantize_groups(wd, bits, q, sc, bi)
+    assert np.array_equal(sc.cpu().numpy().view(np.uint16), s_ref)
+    assert np.array_equal(bi.cpu().numpy().view(np.uint16), b_ref)
+    assert np.array_equal(q.cpu().numpy(), q_ref)
+
+
+@pytest.mark.parametrize("bits", [4, 2])
+def test_quantise_then_pack_round_trip(bits):
+    """fp32 expert weights -> device quantiser -> device packer; unpacking
+    the records on the host gives back the quantiser's codes, scales and
+    biases."""
+    H, I, E = 256, 128, 3
+    n = 3 * H * I * E
+    w = _quantiser_inputs(n // 64, 50 + bits).ravel()
+    wd = torch.from_numpy(w).cuda()
+    q = torch.empty(n, dtype=torch.uint8, device="cuda")
+    sc = torch.empty(n // 64, dtype=torch.int16, device="cuda")
+    bi = torch.empty(n // 64, dtype=torch.int16, device="cuda")
+    fm.fmoe_quantize_groups(wd, bits, q, sc, bi)
+    nbytes = fm.fmoe_packed_bytes(bits, E, H, I, 64)
+    packed = torch.empty(nbytes, dtype=torch.uint8, device="cuda")
+    fm.fmoe_pack_experts_device(q, sc, bi, bits, E, H, I, packed)
+    torch.cuda.synchronize()
+    assert fm.fmoe_read_status() == 0
+    q2, s2, b2 = fm.fmoe_unpack_experts_host(packed.cpu().numpy(), bits, E, H, I)
+    assert np.array_equal(q2.ravel(), q.cpu().numpy())
+    assert np.array_equal(s2.ravel(), sc.cpu().numpy().view(np.uint16))
+    assert np.array_equal(b2.ravel(), bi.cpu().numpy().view(np.uint16))
