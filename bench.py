@@ -121,6 +121,35 @@ def small_batch_measure(fm, synth, torch, layers, wl, stream, Ts=(2, 4, 8), rota
             "by_T": out}
 
 
+def quantiser_measure(fm, torch, stream, experts=16, reps=10, H=4096, I=1024):
+    """The device quantiser (fp32 weights -> int4 codes + bf16 scale/bias) on
+    `experts` experts' worth of fp32 weights (3 H I each): GB/s of fp32
+    weights read (bytes moved: 4 in, 1 code + 4/64 scale-bias out per
+    weight)."""
+    n = experts * 3 * H * I
+    g = torch.Generator(device="cuda").manual_seed(5)
+    w = torch.randn(n, device="cuda", generator=g) * 0.02
+    q = torch.empty(n, dtype=torch.uint8, device="cuda")
+    sc = torch.empty(n // 64, dtype=torch.int16, device="cuda")
+    bi = torch.empty(n // 64, dtype=torch.int16, device="cuda")
+    with torch.cuda.stream(stream):
+        for _ in range(2):
+            fm.fmoe_quantize_groups(w, 4, q, sc, bi, stream=stream)
+    torch.cuda.synchronize()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    with torch.cuda.stream(stream):
+        e0.record(stream)
+        for _ in range(reps):
+            fm.fmoe_quantize_groups(w, 4, q, sc, bi, stream=stream)
+        e1.record(stream)
+    e1.synchronize()
+    s = e0.elapsed_time(e1) / 1e3 / reps
+    moved = n * 4 + n + (n // 64) * 4
+    del w, q, sc, bi
+    return {"workload": f"quantise {experts} experts' fp32 weights (hidden {H}, inter {I}) to int4 + bf16 scale/bias",
+            "ms": s * 1e3, "weights_per_s": n / s, "gbs_moved": moved / s / 1e9}
+
+
 def int2_chain_measure(fm, synth, torch, stream, layers=20, steps=2000, warmup=100):
     """The 2-bit variant of the layer stack (routed experts 2-bit, shared
     expert 4-bit), one token carried through all layers: layers/s."""
@@ -457,17 +486,16 @@ def run_ours(args):
     K2 = args.e2e_steps or min(args.steps, 2000)
     xs = synth.tokens(wl, min(K2, 64), stream=500 + rank)
     nb = xs.shape[0]
-    # per step one pinned [2, H] block (h and its normed copy xn) in, one out
-    hx_in = torch.from_numpy(np.ascontiguousarray(np.stack([xs, xs], axis=1))).pin_memory()
-    hx_out = torch.empty((nb, 2, H), dtype=torch.float32).pin_memory()
-    hx = torch.empty((2, H), dtype=torch.float32, device="cuda")
+    # per step one pinned [2, 1, H] block (h and its normed copy xn) goes in
+    # and one comes out, through the host-state entry point of the C ABI
+    hx_in = torch.from_numpy(np.ascontiguousarray(np.stack([xs, xs], axis=1)[:, :, None, :])).pin_memory()
+    hx_out = torch.empty((nb, 2, 1, H), dtype=torch.float32).pin_memory()
+    hx = torch.empty((2, 1, H), dtype=torch.float32, device="cuda")
 
     def e2e_steps(n):
         for i in range(n):
             j = i % nb
-            hx.copy_(hx_in[j], non_blocking=True)
-            fm.fmoe_layer_forward(layers[i % L], hx[0:1], hx[1:2], ws, stream=stream)
-            hx_out[j].copy_(hx, non_blocking=True)
+            fm.fmoe_layer_forward_host(layers[i % L], hx_in[j], hx_out[j], hx, ws, stream=stream)
 
     with torch.cuda.stream(stream):
         e2e_steps(min(50, K2))
@@ -482,8 +510,8 @@ def run_ours(args):
     e2e_ms = max_over_ranks(e0.elapsed_time(e1), world)
     e2e = {"value": job_rate(K2, world, e2e_ms), "unit": UNIT, "h2d_bytes_per_step": 2 * H * 4,
            "d2h_bytes_per_step": 2 * H * 4, "steps": K2,
-           "how": "per step: one pinned host [2, H] block (h, xn) -> device, fmoe_layer_forward (eager C-ABI call), "
-                  "h', xn' -> pinned host in one copy"}
+           "how": "per step: fmoe_layer_forward_host (one eager C-ABI call): a pinned host [2, H] block (h, xn) "
+                  "-> device, the layer, h', xn' -> pinned host"}
 
     line = {"metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
             "warmup": args.warmup, "ms_per_step": ms_max / args.steps, "higher_is_better": True,
@@ -499,6 +527,7 @@ def run_ours(args):
     if not args.no_extra and wl.n_experts == 512:
         line["batched"] = batched_measure(fm, synth, np, torch, layers[0], wl, stream)
         line["small_batch"] = small_batch_measure(fm, synth, torch, layers, wl, stream)
+        line["quantiser"] = quantiser_measure(fm, torch, stream)
         del layers, graphs, g_all
         graphs = g_all = None
         torch.cuda.empty_cache()

@@ -234,6 +234,19 @@ int fmoe_combine_residual_rmsnorm(const float* d_y, const float* d_weights, cons
 int fmoe_layer_forward(const fmoe_layer_weights* lw, float* d_h, float* d_xn, int T, void* d_ws,
                        size_t ws_bytes, cudaStream_t stream);
 
+/* fmoe_layer_forward for T tokens whose state lives in host memory, for a
+ * caller that feeds tokens from the host (a decode loop in plain C):
+ *   hx_in   host fp32 [2][T][H]: h rows, then the normed xn rows;
+ *   hx_out  host fp32 [2][T][H]: receives h' rows, then xn' rows;
+ *   d_hx    device fp32 [2][T][H] (caller-owned, 16-byte aligned) that the
+ *           layer runs on in place.
+ * One host-to-device copy, the layer, one device-to-host copy, all on
+ * `stream` (with pinned host buffers nothing blocks; hx_out is valid once
+ * the stream has reached the end of the call).  hx_in and hx_out may be the
+ * same buffer.  Errors: as fmoe_layer_forward (checked before any copy). */
+int fmoe_layer_forward_host(const fmoe_layer_weights* lw, const float* hx_in, float* hx_out, float* d_hx,
+                            int T, void* d_ws, size_t ws_bytes, cudaStream_t stream);
+
 /* As fmoe_layer_forward, routing on given router logits d_logits [T][E]
  * (device fp32) instead of the router product. */
 int fmoe_layer_forward_logits(const fmoe_layer_weights* lw, const float* d_logits, float* d_h,

@@ -91,6 +91,7 @@ _SIGS = {
     "fmoe_fused_supported": (_i32, [_PDESC]),
     "fmoe_set_tensor_cores": (_i32, [_i32]),
     "fmoe_tc_min_tokens": (_i32, []),
+    "fmoe_layer_forward_host": (_i32, [_vp, _vp, _vp, _vp, _i32, _vp, _sz, _vp]),
     "fmoe_quantize_groups": (_i32, [_vp, _sz, _i32, _i32, _vp, _vp, _vp, _vp]),
     "fmoe_fused_max_tokens": (_i32, [_i32]),
     "fmoe_layer_forward_noalloc": (_i32, [_PW, _vp, _vp, _i32, _vp]),
@@ -288,6 +289,17 @@ def fmoe_layer_forward(lw: LayerWeights, h, xn, ws, stream=None) -> None:
     rc = _lib.fmoe_layer_forward(ctypes.byref(c), _ptr(h), _ptr(xn), h.shape[0], _ptr(ws),
                                  ws.numel() * ws.element_size(), _stream(stream))
     _check(rc, "fmoe_layer_forward")
+
+
+def fmoe_layer_forward_host(lw: LayerWeights, hx_in, hx_out, d_hx, ws, stream=None) -> None:
+    """fmoe_layer_forward on host token state: hx_in / hx_out are (pinned) host
+    tensors [2, T, H] (h rows, then xn rows), d_hx a device tensor of the same
+    shape; one copy in, the layer, one copy out, asynchronous on `stream`."""
+    c = lw.c()
+    T = d_hx.shape[1]
+    rc = _lib.fmoe_layer_forward_host(ctypes.byref(c), _ptr(hx_in), _ptr(hx_out), _ptr(d_hx), T, _ptr(ws),
+                                      ws.numel() * ws.element_size(), _stream(stream))
+    _check(rc, "fmoe_layer_forward_host")
 
 
 def fmoe_layer_forward_logits(lw: LayerWeights, logits, h, xn, ws, stream=None) -> None:

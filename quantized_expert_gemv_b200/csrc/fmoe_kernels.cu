@@ -1120,6 +1120,23 @@ extern "C" int fmoe_layer_forward(const fmoe_layer_weights* lw, float* d_h, floa
   return layer_forward_impl(lw, nullptr, d_h, d_xn, T, d_ws, ws_bytes, stream);
 }
 
+extern "C" int fmoe_layer_forward_host(const fmoe_layer_weights* lw, const float* hx_in, float* hx_out,
+                                       float* d_hx, int T, void* d_ws, size_t ws_bytes, cudaStream_t stream) {
+  const int rc0 = weights_check(lw);
+  if (rc0 != FMOE_OK) return rc0;
+  if (!hx_in || !hx_out || !d_hx || !d_ws || T < 1 || !aligned16(d_hx) || !aligned16(d_ws))
+    return FMOE_ERR_INVALID_ARG;
+  const int H = lw->desc.hidden;
+  const WsLayout w = ws_layout(H, lw->desc.inter, lw->desc.n_experts, lw->desc.top_k, T);
+  if (ws_bytes < w.bytes) return FMOE_ERR_BUFFER_TOO_SMALL;
+  const size_t bytes = (size_t)2 * T * H * sizeof(float);
+  if (cudaMemcpyAsync(d_hx, hx_in, bytes, cudaMemcpyHostToDevice, stream) != cudaSuccess) return FMOE_ERR_CUDA;
+  const int rc = layer_forward_impl(lw, nullptr, d_hx, d_hx + (size_t)T * H, T, d_ws, ws_bytes, stream);
+  if (rc != FMOE_OK) return rc;
+  return cudaMemcpyAsync(hx_out, d_hx, bytes, cudaMemcpyDeviceToHost, stream) == cudaSuccess ? FMOE_OK
+                                                                                            : FMOE_ERR_CUDA;
+}
+
 extern "C" int fmoe_layer_forward_logits(const fmoe_layer_weights* lw, const float* d_logits,
                                          float* d_h, float* d_xn, int T, void* d_ws,
                                          size_t ws_bytes, cudaStream_t stream) {

@@ -458,6 +458,26 @@ def test_few_tokens_run_token_by_token(wl):
     assert fm.fmoe_read_status() == 0
 
 
+@pytest.mark.parametrize("T", [1, 3, 6])
+def test_host_state_entry_point_matches_device_entry_point(T):
+    """fmoe_layer_forward_host (pinned host h/xn in, h'/xn' out, one copy
+    each way) gives the bits of fmoe_layer_forward on device tensors."""
+    wl = SMALL
+    lw = device_layer(wl)
+    x = synth.tokens(wl, T, stream=63)
+    h, xn = dev(x), dev(x)
+    ws = fm.alloc_workspace(lw.desc, T)
+    fm.fmoe_layer_forward(lw, h, xn, ws)
+    hx_in = torch.from_numpy(np.stack([x, x])).pin_memory()
+    hx_out = torch.zeros_like(hx_in).pin_memory()
+    d_hx = torch.empty(hx_in.shape, dtype=torch.float32, device="cuda")
+    ws2 = fm.alloc_workspace(lw.desc, T)
+    fm.fmoe_layer_forward_host(lw, hx_in, hx_out, d_hx, ws2)
+    torch.cuda.synchronize()
+    assert np.array_equal(hx_out[0].numpy(), host(h)) and np.array_equal(hx_out[1].numpy(), host(xn))
+    assert fm.fmoe_read_status() == 0
+
+
 def test_tensor_core_and_integer_paths_differ_only_by_rounding():
     """The two implementations of the grouped products both run (their
     results are not bit-identical) and agree well inside the tolerance."""
