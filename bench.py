@@ -121,6 +121,48 @@ def small_batch_measure(fm, synth, torch, layers, wl, stream, Ts=(2, 4, 8), rota
             "by_T": out}
 
 
+def cache_measure(fm, synth, np, torch, layers, wl, stream, n_layers=4, slot_counts=(64, 256, 1024), tokens=50):
+    """Decode (T = 1) through `n_layers` layers whose routed experts live in
+    pinned host memory, with a device cache of `slots` records shared by the
+    layers (least recently used first); routing from Zipf(1)-popularity
+    Gumbel-top-k logits per layer and token.  Per cache size: layer steps/s,
+    hit rate, host-to-device expert GB/s."""
+    host = [layers[l].experts.cpu().pin_memory() for l in range(n_layers)]
+    logits = [[torch.from_numpy(synth.zipf_gumbel_logits(wl, 1000 * l + t, 1)[0]).cuda() for l in range(n_layers)]
+              for t in range(tokens)]
+    x = torch.from_numpy(synth.tokens(wl, 1, stream=960)).cuda()
+    ws = fm.alloc_workspace(layers[0].desc, 1)
+    out = {}
+    for slots in slot_counts:
+        cache = fm.ExpertCache(layers[0].desc, host, n_slots=slots, max_tokens=1)
+        h, xn = x.clone(), x.clone()
+        with torch.cuda.stream(stream):
+            for t in range(5):  # warm the cache
+                for l in range(n_layers):
+                    cache.forward(l, layers[l], h, xn, ws, logits=logits[t][l], stream=stream)
+        torch.cuda.synchronize()
+        h0, m0, b0 = cache.stats()
+        t0 = time.perf_counter()
+        with torch.cuda.stream(stream):
+            for t in range(tokens):
+                for l in range(n_layers):
+                    cache.forward(l, layers[l], h, xn, ws, logits=logits[t][l], stream=stream)
+        torch.cuda.synchronize()
+        dt = time.perf_counter() - t0
+        h1, m1, b1 = cache.stats()
+        steps = tokens * n_layers
+        out[str(slots)] = {"layer_steps_per_s": steps / dt, "hit_rate": (h1 - h0) / max(1, (h1 - h0) + (m1 - m0)),
+                           "h2d_gbs": (b1 - b0) / dt / 1e9, "slots_gb": slots * layers[0].desc.record_bytes() / 1e9}
+        cache.close()
+        del cache
+        torch.cuda.empty_cache()
+    del host
+    return {"workload": f"moe_decode_host_tier: {n_layers} int4 layers' routed experts in pinned host memory, device "
+                        f"cache of N records shared by the layers (LRU), Zipf(1) routing, {tokens} tokens",
+            "timing": "host wall clock around the steps (each step synchronises to read its routing)",
+            "by_slots": out}
+
+
 def quantiser_measure(fm, torch, stream, experts=16, reps=10, H=4096, I=1024):
     """The device quantiser (fp32 weights -> int4 codes + bf16 scale/bias) on
     `experts` experts' worth of fp32 weights (3 H I each): GB/s of fp32
@@ -528,6 +570,7 @@ def run_ours(args):
         line["batched"] = batched_measure(fm, synth, np, torch, layers[0], wl, stream)
         line["small_batch"] = small_batch_measure(fm, synth, torch, layers, wl, stream)
         line["quantiser"] = quantiser_measure(fm, torch, stream)
+        line["host_tier"] = cache_measure(fm, synth, np, torch, layers, wl, stream)
         del layers, graphs, g_all
         graphs = g_all = None
         torch.cuda.empty_cache()

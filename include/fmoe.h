@@ -171,6 +171,47 @@ int fmoe_pack_experts_device(const uint8_t* d_q, const uint16_t* d_scale, const 
 int fmoe_quantize_groups(const float* d_w, size_t n_groups, int group, int bits, uint8_t* d_q,
                          uint16_t* d_scale, uint16_t* d_bias, cudaStream_t stream);
 
+/* ------------------------------------------------ host expert tier -- */
+/* Routed experts held in host memory with a device cache of records
+ * ("What is Flash-MoE?", section "1. SSD expert streaming": experts fetched
+ * per layer from a slower tier once routing has chosen them; here the tier
+ * is host memory over PCIe and the cache is explicit, least recently used
+ * first, shared by all layers).  Opaque handle; host-side state only. */
+typedef struct fmoe_expert_cache fmoe_expert_cache;
+
+/* Creates a cache for n_layers layers of descriptor d:
+ *   h_layer_experts[l]  host: layer l's E packed routed records, back to back
+ *                       (pinned memory keeps the record copies asynchronous);
+ *   d_slots             device, caller-owned: n_slots records
+ *                       (d_slots_bytes >= n_slots * record bytes);
+ *   d_table             device, caller-owned: n_layers * E uint64 record
+ *                       addresses (written by the cache);
+ *   max_tokens          largest T of a step.
+ * Allocates two small pinned host buffers (table mirror, one step's ids);
+ * zeroes d_table synchronously.  Errors: FMOE_ERR_INVALID_ARG,
+ * FMOE_ERR_UNSUPPORTED, FMOE_ERR_BUFFER_TOO_SMALL, FMOE_ERR_CUDA. */
+int fmoe_cache_create(const fmoe_layer_desc* d, int n_layers, const void* const* h_layer_experts, int n_slots,
+                      void* d_slots, size_t d_slots_bytes, uint64_t* d_table, int max_tokens,
+                      fmoe_expert_cache** out);
+int fmoe_cache_destroy(fmoe_expert_cache* c);
+
+/* Counters since creation: expert-steps served from the slots (an expert
+ * used by several tokens of one step counts once), records copied in, and
+ * their bytes. */
+int fmoe_cache_stats(const fmoe_expert_cache* c, uint64_t* hits, uint64_t* misses, uint64_t* bytes_in);
+
+/* One layer step (layer index `layer`) for T tokens, as fmoe_layer_forward
+ * (or fmoe_layer_forward_logits when d_logits is given) with the routed
+ * records taken from the cache (lw->experts is not read): routing on the
+ * device, the step's ids copied to the host and the stream synchronised,
+ * every missing record copied into a slot (the least recently used one not
+ * needed by this step), the layer's table row uploaded, then the expert
+ * products and the combine.  Steps of one cache must be issued in order on
+ * one stream.  Errors: as fmoe_layer_forward; FMOE_ERR_BUFFER_TOO_SMALL when
+ * the slots cannot hold one step's distinct experts. */
+int fmoe_cache_layer_forward(fmoe_expert_cache* c, int layer, const fmoe_layer_weights* lw, const float* d_logits,
+                             float* d_h, float* d_xn, int T, void* d_ws, size_t ws_bytes, cudaStream_t stream);
+
 /* ----------------------------------------------------------- workspace -- */
 /* Device workspace for T tokens of a layer with descriptor d (bytes).  The
  * workspace holds intermediates (router partial sums, logits, ids, gate

@@ -91,6 +91,10 @@ _SIGS = {
     "fmoe_fused_supported": (_i32, [_PDESC]),
     "fmoe_set_tensor_cores": (_i32, [_i32]),
     "fmoe_tc_min_tokens": (_i32, []),
+    "fmoe_cache_create": (_i32, [_vp, _i32, _vp, _i32, _vp, _sz, _vp, _i32, _vp]),
+    "fmoe_cache_destroy": (_i32, [_vp]),
+    "fmoe_cache_stats": (_i32, [_vp, _vp, _vp, _vp]),
+    "fmoe_cache_layer_forward": (_i32, [_vp, _i32, _vp, _vp, _vp, _vp, _i32, _vp, _sz, _vp]),
     "fmoe_layer_forward_host": (_i32, [_vp, _vp, _vp, _vp, _i32, _vp, _sz, _vp]),
     "fmoe_quantize_groups": (_i32, [_vp, _sz, _i32, _i32, _vp, _vp, _vp, _vp]),
     "fmoe_fused_max_tokens": (_i32, [_i32]),
@@ -361,3 +365,48 @@ def fmoe_set_fused(enable: bool) -> bool:
     """Selects the persistent fused kernel (True, default) or the one-kernel-per-step
     path for T = 1; returns the previous setting."""
     return bool(_lib.fmoe_set_fused(int(bool(enable))))
+
+
+class ExpertCache:
+    """Routed experts of n layers in host memory, a device cache of n_slots
+    records (C ABI fmoe_cache_*).  host_layers: per layer a (pinned) uint8
+    CPU tensor of the layer's E packed records; the device slots and the
+    record table are allocated here, as caller-owned buffers of the ABI."""
+
+    def __init__(self, desc: LayerDesc, host_layers, n_slots: int, max_tokens: int = 64):
+        import torch
+        self.desc, self.host_layers = desc, list(host_layers)
+        rec = desc.record_bytes()
+        self.slots = torch.empty(n_slots * rec, dtype=torch.uint8, device="cuda")
+        self.table = torch.zeros(len(self.host_layers) * desc.n_experts, dtype=torch.int64, device="cuda")
+        ptrs = (ctypes.c_void_p * len(self.host_layers))(*[t.data_ptr() for t in self.host_layers])
+        h = ctypes.c_void_p()
+        d = desc.c()
+        rc = _lib.fmoe_cache_create(ctypes.byref(d), len(self.host_layers), ptrs, n_slots, _ptr(self.slots),
+                                    self.slots.numel(), _ptr(self.table), max_tokens, ctypes.byref(h))
+        _check(rc, "fmoe_cache_create")
+        self._h = h
+
+    def forward(self, layer: int, lw: LayerWeights, h, xn, ws, logits=None, stream=None) -> None:
+        c = lw.c()
+        rc = _lib.fmoe_cache_layer_forward(self._h, layer, ctypes.byref(c), _ptr(logits) if logits is not None else None,
+                                           _ptr(h), _ptr(xn), h.shape[0], _ptr(ws), ws.numel() * ws.element_size(),
+                                           _stream(stream))
+        _check(rc, "fmoe_cache_layer_forward")
+
+    def stats(self):
+        hits, misses, nbytes = ctypes.c_uint64(), ctypes.c_uint64(), ctypes.c_uint64()
+        _check(_lib.fmoe_cache_stats(self._h, ctypes.byref(hits), ctypes.byref(misses), ctypes.byref(nbytes)),
+               "fmoe_cache_stats")
+        return hits.value, misses.value, nbytes.value
+
+    def close(self) -> None:
+        if getattr(self, "_h", None):
+            _lib.fmoe_cache_destroy(self._h)
+            self._h = None
+
+    def __del__(self):
+        try:
+            self.close()
+        except Exception:
+            pass

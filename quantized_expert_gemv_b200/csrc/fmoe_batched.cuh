@@ -199,6 +199,7 @@ __device__ __forceinline__ const uint8_t* group_record(const ExpertSet& es, int 
     return es.shared;
   }
   *bits = es.bits;
+  if (es.rec_table) return reinterpret_cast<const uint8_t*>(es.rec_table[g]);
   return es.experts + (size_t)g * es.rec_bytes;
 }
 

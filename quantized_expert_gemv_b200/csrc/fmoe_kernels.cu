@@ -163,6 +163,7 @@ topk_kernel(const float* __restrict__ part, const float* __restrict__ logits_in,
 // ---------------------------------------------------------- experts ----
 struct ExpertSet {
   const uint8_t* experts;  // E records
+  const uint64_t* rec_table;  // when set: device address of routed record id (an expert cache's slots)
   const uint8_t* shared;   // one record
   size_t rec_bytes, shared_rec_bytes;
   int bits, shared_bits;
@@ -179,6 +180,7 @@ __device__ __forceinline__ const uint8_t* slot_record(const ExpertSet& es, const
   const int id = ids[(size_t)t * es.k + j];
   *bits = es.bits;
   if (id < 0 || id >= es.E) return nullptr;
+  if (es.rec_table) return reinterpret_cast<const uint8_t*>(es.rec_table[id]);
   return es.experts + (size_t)id * es.rec_bytes;
 }
 
@@ -645,6 +647,7 @@ static ExpertSet expert_set(const fmoe_layer_weights* lw) {
   const fmoe_layer_desc& d = lw->desc;
   ExpertSet es;
   es.experts = static_cast<const uint8_t*>(lw->experts);
+  es.rec_table = nullptr;
   es.shared = static_cast<const uint8_t*>(lw->shared);
   es.rec_bytes = record_layout(d.bits, d.hidden, d.inter).bytes;
   es.shared_rec_bytes = record_layout(d.shared_bits, d.hidden, d.inter).bytes;
@@ -1276,3 +1279,5 @@ extern "C" int fmoe_layer_forward_noalloc(const fmoe_layer_weights* lw, float* d
   if (rc != FMOE_OK) return rc;
   return layer_forward_impl(lw, nullptr, d_h, d_xn, T, ws, kStaticScratchBytes, stream);
 }
+
+#include "fmoe_cache.cuh"
