@@ -302,10 +302,11 @@ int fmoe_layer_forward_logits(const fmoe_layer_weights* lw, const float* d_logit
 int fmoe_stack_forward(const fmoe_layer_weights* layers, int n_layers, float* d_h, float* d_xn,
                        int T, void* d_ws, size_t ws_bytes, cudaStream_t stream);
 
-/* Chooses the implementation of the T = 1 path: enable != 0 (the default)
- * uses the persistent fused kernel wherever its shared-memory plan fits, 0
- * the one-kernel-per-step path.  Both compute the same layer; process-wide
- * setting, returns the previous value. */
+/* Chooses the implementation of the T = 1 path (and of the few-token calls
+ * that run token by token, see fmoe_fused_max_tokens): enable != 0 (the
+ * default) uses the persistent fused kernel wherever its shared-memory plan
+ * fits, 0 the one-kernel-per-step path.  Both compute the same layer;
+ * process-wide setting, returns the previous value. */
 int fmoe_set_fused(int enable);
 
 /* Chooses the expert products of the T > 1 path for experts that receive at

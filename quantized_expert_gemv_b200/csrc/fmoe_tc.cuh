@@ -6,15 +6,17 @@
 // the dequantised weights (w = code * scale + bias, rounded to fp16) and X
 // the tokens' inputs split as x = x_hi + x_lo (two fp16 values, so the
 // input keeps ~22 bits): X holds the Np hi rows, then the Np lo rows, and
-// the output for token t is D[., t] + D[., Np + t].  Per CTA: a tile of 128
-// weight rows, all N = 2 Np columns, the accumulator in tensor memory:
-//   - all 256 threads dequantise one 64-input group of the tile into shared
-//     memory (fp16, K-major core matrices of 8 rows x 16 bytes);
-//   - the staged X tile of that group arrives by one bulk copy;
+// the output for token t is D[., t] + D[., Np + t].  Persistent CTAs (one
+// per SM) take work units of (item of <= 32 tokens, tile of 128 weight
+// rows), all N = 2 Np columns, the accumulator in tensor memory:
+//   - the 256 producer threads stream the tile's raw codes into a shared
+//     ring with cp.async, two 8-group supersteps ahead, and two warps per
+//     64-input group dequantise it into a 4-stage fp16 A ring (K-major core
+//     matrices of 8 rows x 16 bytes), requesting the group's staged X tile
+//     by one bulk copy;
 //   - one thread issues the four 128 x N x 16 tcgen05.mma of the group and
-//     commits them to the stage's mbarrier (a ring of three stages, so
-//     dequantising the next groups overlaps the tensor cores; the raw
-//     weight words are loaded four groups ahead);
+//     commits them to the stage's mbarrier, so dequantising the next groups
+//     overlaps the tensor cores;
 //   - the epilogue reads the accumulator with tcgen05.ld (warp w: tensor
 //     memory lanes 32 (w % 4) ..), adds the hi and lo columns, and writes
 //     SwiGLU outputs (gate/up) or expert outputs (down).
