@@ -355,15 +355,15 @@ __host__ __device__ constexpr size_t gu_bulk_slot_bytes(int H, int bits) {
 }
 
 template <int MB>
-__global__ void __launch_bounds__(kGrpThreads, 2)
-gateup_bulk_kernel(ExpertSet es, GroupWork w, int bucket, int max_items, const float* __restrict__ xn,
-                   const unsigned char* __restrict__ xs, float* __restrict__ a, const float* __restrict__ w_sg,
-                   float* __restrict__ gamma) {
+__device__ __forceinline__ void gateup_bulk_body(const ExpertSet& es, const GroupWork& w, int bucket, int max_items,
+                                                 int item, const float* __restrict__ xn,
+                                                 const unsigned char* __restrict__ xs, float* __restrict__ a,
+                                                 const float* __restrict__ w_sg, float* __restrict__ gamma) {
   extern __shared__ __align__(128) unsigned char smem[];
   __shared__ int s_slot[MB];
   __shared__ uint64_t full[kGuBulkSlots];
-  if ((int)blockIdx.x >= w.n_items[2 + bucket]) return;
-  const int4 it = w.bitems[(size_t)bucket * max_items + blockIdx.x];
+  if (item >= w.n_items[2 + bucket]) return;
+  const int4 it = w.bitems[(size_t)bucket * max_items + item];
   const int g = it.x, m = it.z, k1 = es.k + 1;
   const int H = es.H, I = es.I, ng = H / 64;
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
@@ -489,6 +489,25 @@ gateup_bulk_kernel(ExpertSet es, GroupWork w, int bucket, int max_items, const f
   }
 }
 
+// grid (max items, gu_split(MB)): one size bucket.
+template <int MB>
+__global__ void __launch_bounds__(kGrpThreads, 2)
+gateup_bulk_kernel(ExpertSet es, GroupWork w, int bucket, int max_items, const float* __restrict__ xn,
+                   const unsigned char* __restrict__ xs, float* __restrict__ a, const float* __restrict__ w_sg,
+                   float* __restrict__ gamma) {
+  gateup_bulk_body<MB>(es, w, bucket, max_items, (int)blockIdx.x, xn, xs, a, w_sg, gamma);
+}
+
+// grid (n0 + n1, gu_split): the items of buckets 0 (<= 2 tokens) and 1
+// (<= 4 tokens) in one launch, so that neither bucket's tail idles the GPU.
+__global__ void __launch_bounds__(kGrpThreads, 2)
+gateup_bulk_small_kernel(ExpertSet es, GroupWork w, int max_items, int n0, const float* __restrict__ xn,
+                         const unsigned char* __restrict__ xs, float* __restrict__ a,
+                         const float* __restrict__ w_sg, float* __restrict__ gamma) {
+  if ((int)blockIdx.x < n0) gateup_bulk_body<2>(es, w, 0, max_items, (int)blockIdx.x, xn, xs, a, w_sg, gamma);
+  else gateup_bulk_body<4>(es, w, 1, max_items, (int)blockIdx.x - n0, xn, xs, a, w_sg, gamma);
+}
+
 __host__ __device__ constexpr size_t gu_bulk_smem(int MB, int H, int bits) {
   return (((size_t)MB * ((staged_x_bytes(H) + 15) & ~(size_t)15) + 127) & ~(size_t)127) +
          (size_t)kGuBulkSlots * ((gu_bulk_slot_bytes(H, bits) + 127) & ~(size_t)127);
@@ -526,16 +545,15 @@ __device__ __forceinline__ void down_row_multi(const uint8_t* rec, const ExpertS
   }
 }
 
-// grid (max items, H / kDnRows), one size bucket of GEMV items (m <= MB);
-// one hidden row per thread.
+// Down product of one GEMV item (m <= MB tokens) for hidden rows
+// blockIdx.y * kDnRows + thread; one hidden row per thread.
 template <int MB>
-__global__ void __launch_bounds__(kDnRows)
-down_group_kernel(ExpertSet es, GroupWork w, int bucket, int max_items, const float* __restrict__ a,
-                  float* __restrict__ y) {
+__device__ __forceinline__ void down_group_body(const ExpertSet& es, const GroupWork& w, int bucket, int max_items,
+                                                int item, const float* __restrict__ a, float* __restrict__ y) {
   extern __shared__ __align__(128) unsigned char smem[];
   __shared__ int s_slot[kGrpMaxM];
-  if ((int)blockIdx.x >= w.n_items[2 + bucket]) return;
-  const int4 it = w.bitems[(size_t)bucket * max_items + blockIdx.x];
+  if (item >= w.n_items[2 + bucket]) return;
+  const int4 it = w.bitems[(size_t)bucket * max_items + item];
   const int g = it.x, m = it.z;
   if (threadIdx.x < m) s_slot[threadIdx.x] = w.slots[w.offset[g] + it.y + threadIdx.x];
   __syncthreads();
@@ -554,6 +572,23 @@ down_group_kernel(ExpertSet es, GroupWork w, int bucket, int max_items, const fl
 #pragma unroll
   for (int i = 0; i < MB; ++i)
     if (i < m) y[(size_t)s_slot[i] * es.H + row] = yv[i];
+}
+
+
+// grid (max items, H / kDnRows), one size bucket of GEMV items (m <= MB).
+template <int MB>
+__global__ void __launch_bounds__(kDnRows)
+down_group_kernel(ExpertSet es, GroupWork w, int bucket, int max_items, const float* __restrict__ a,
+                  float* __restrict__ y) {
+  down_group_body<MB>(es, w, bucket, max_items, (int)blockIdx.x, a, y);
+}
+
+// grid (n0 + n1, H / kDnRows): buckets 0 and 1 in one launch.
+__global__ void __launch_bounds__(kDnRows)
+down_group_small_kernel(ExpertSet es, GroupWork w, int max_items, int n0, const float* __restrict__ a,
+                        float* __restrict__ y) {
+  if ((int)blockIdx.x < n0) down_group_body<2>(es, w, 0, max_items, (int)blockIdx.x, a, y);
+  else down_group_body<4>(es, w, 1, max_items, (int)blockIdx.x - n0, a, y);
 }
 
 }  // namespace fmoe

@@ -776,8 +776,19 @@ static int launch_experts(const ExpertSet& es, const float* xn, const int32_t* i
       // index the bucket lists with the full stride `items`)
       int nb[kGrpBuckets];
       for (int b = 0; b < kGrpBuckets; ++b) nb[b] = bucket_items_bound(b, slots, items, tc ? kTcMinTokens : 0);
-      if (nb[0]) grp_launch_gu<2>(es, *gw, 0, items, nb[0], xn, xs, a, w_sg, gamma, sxs, st);
-      if (nb[1]) grp_launch_gu<4>(es, *gw, 1, items, nb[1], xn, xs, a, w_sg, gamma, sxs, st);
+      // only items of <= 4 tokens: one launch for both of their buckets
+      const bool small_only = nb[2] == 0 && nb[3] == 0 && nb[0] > 0 && nb[1] > 0 && gu_bulk_ok<2>(es) &&
+                              gu_bulk_ok<4>(es) &&
+                              smem_optin(reinterpret_cast<const void*>(&gateup_bulk_small_kernel),
+                                         gu_bulk_smem(4, es.H, 4), 30) &&
+                              smem_optin(reinterpret_cast<const void*>(&down_group_small_kernel), 4 * sas, 31);
+      if (small_only) {
+        gateup_bulk_small_kernel<<<dim3(nb[0] + nb[1], gu_split(4)), kGrpThreads, gu_bulk_smem(4, es.H, 4), st>>>(
+            es, *gw, items, nb[0], xn, xs, a, w_sg, gamma);
+      } else {
+        if (nb[0]) grp_launch_gu<2>(es, *gw, 0, items, nb[0], xn, xs, a, w_sg, gamma, sxs, st);
+        if (nb[1]) grp_launch_gu<4>(es, *gw, 1, items, nb[1], xn, xs, a, w_sg, gamma, sxs, st);
+      }
       if (nb[2]) grp_launch_gu<8>(es, *gw, 2, items, nb[2], xn, xs, a, w_sg, gamma, sxs, st);
       if (nb[3]) grp_launch_gu<16>(es, *gw, 3, items, nb[3], xn, xs, a, w_sg, gamma, sxs, st);
       if (tc) {
@@ -787,8 +798,13 @@ static int launch_experts(const ExpertSet& es, const float* xn, const int32_t* i
         const int u0 = max_tc * (2 * es.I / kTcRows);
         tc_gemm_kernel<0><<<u0 < n_sm ? u0 : n_sm, kTcThreads + 32, tc_smem_bytes(), st>>>(es, *gw, tcx, a);
       }
-      if (nb[0]) grp_launch_dn<2>(es, *gw, 0, items, nb[0], a, y, sas, st);
-      if (nb[1]) grp_launch_dn<4>(es, *gw, 1, items, nb[1], a, y, sas, st);
+      if (small_only) {
+        down_group_small_kernel<<<dim3(nb[0] + nb[1], (es.H + kDnRows - 1) / kDnRows), kDnRows, 4 * sas, st>>>(
+            es, *gw, items, nb[0], a, y);
+      } else {
+        if (nb[0]) grp_launch_dn<2>(es, *gw, 0, items, nb[0], a, y, sas, st);
+        if (nb[1]) grp_launch_dn<4>(es, *gw, 1, items, nb[1], a, y, sas, st);
+      }
       if (nb[2]) grp_launch_dn<8>(es, *gw, 2, items, nb[2], a, y, sas, st);
       if (nb[3]) grp_launch_dn<16>(es, *gw, 3, items, nb[3], a, y, sas, st);
       if (tc) {
