@@ -127,6 +127,7 @@ def cache_measure(fm, synth, np, torch, layers, wl, stream, n_layers=4, slot_cou
     layers (least recently used first); routing from Zipf(1)-popularity
     Gumbel-top-k logits per layer and token.  Per cache size: layer steps/s,
     hit rate, host-to-device expert GB/s."""
+    n_layers = min(n_layers, len(layers))
     host = [layers[l].experts.cpu().pin_memory() for l in range(n_layers)]
     logits = [[torch.from_numpy(synth.zipf_gumbel_logits(wl, 1000 * l + t, 1)[0]).cuda() for l in range(n_layers)]
               for t in range(tokens)]
