@@ -186,6 +186,39 @@ def test_host_validation_before_launch(fm):
     assert fm.fmoe_error_string(fm.FMOE_ERR_UNSUPPORTED) == "unsupported shape or bit width"
 
 
+def test_host_validation_of_the_later_entry_points(fm):
+    """Quantiser, host-state layer forward and expert cache refuse bad
+    arguments on the host, before any CUDA call (runs without a GPU)."""
+    L = fm._lib
+    # quantiser: null / misaligned pointers, group and bit width, empty input
+    assert L.fmoe_quantize_groups(None, 4, 64, 4, 16, 16, 16, None) == fm.FMOE_ERR_INVALID_ARG
+    assert L.fmoe_quantize_groups(16, 4, 64, 4, 24, 16, 16, None) == fm.FMOE_ERR_INVALID_ARG
+    assert L.fmoe_quantize_groups(16, 4, 32, 4, 16, 16, 16, None) == fm.FMOE_ERR_UNSUPPORTED
+    assert L.fmoe_quantize_groups(16, 4, 64, 3, 16, 16, 16, None) == fm.FMOE_ERR_UNSUPPORTED
+    assert L.fmoe_quantize_groups(16, 0, 64, 2, 16, 16, 16, None) == fm.FMOE_OK
+    # host-state layer forward: null buffers, workspace too small
+    d = fm.LayerDesc(hidden=256, inter=128, n_experts=16, top_k=4)
+    w = fm.fmoe_layer_weights(d.c(), 16, 16, 16, 16, 16)
+    assert L.fmoe_layer_forward_host(ctypes.byref(w), None, 16, 16, 1, 16, 1 << 30, None) == fm.FMOE_ERR_INVALID_ARG
+    assert L.fmoe_layer_forward_host(ctypes.byref(w), 16, 16, 24, 1, 16, 1 << 30, None) == fm.FMOE_ERR_INVALID_ARG
+    assert L.fmoe_layer_forward_host(ctypes.byref(w), 16, 16, 16, 1, 16, 64, None) == fm.FMOE_ERR_BUFFER_TOO_SMALL
+    # expert cache: missing arguments, slots too small for n_slots records
+    dc = d.c()
+    hp = (ctypes.c_void_p * 1)(16)
+    out = ctypes.c_void_p()
+    assert L.fmoe_cache_create(None, 1, hp, 4, 16, 1 << 30, 16, 1, ctypes.byref(out)) == fm.FMOE_ERR_INVALID_ARG
+    assert L.fmoe_cache_create(ctypes.byref(dc), 1, None, 4, 16, 1 << 30, 16, 1, ctypes.byref(out)) == fm.FMOE_ERR_INVALID_ARG
+    assert L.fmoe_cache_create(ctypes.byref(dc), 1, hp, 4, 16, 64, 16, 1, ctypes.byref(out)) == fm.FMOE_ERR_BUFFER_TOO_SMALL
+    assert L.fmoe_cache_create(ctypes.byref(dc), 1, hp, 0, 16, 1 << 30, 16, 1, ctypes.byref(out)) == fm.FMOE_ERR_INVALID_ARG
+    assert L.fmoe_cache_layer_forward(None, 0, ctypes.byref(w), None, 16, 16, 1, 16, 1 << 30, None) == \
+        fm.FMOE_ERR_INVALID_ARG
+    assert L.fmoe_cache_stats(None, None, None, None) == fm.FMOE_ERR_INVALID_ARG
+    assert L.fmoe_cache_destroy(None) == fm.FMOE_ERR_INVALID_ARG
+    # the dispatch thresholds the header states
+    assert fm.fmoe_tc_min_tokens() == 5
+    assert fm.fmoe_fused_max_tokens(False) == 4 and fm.fmoe_fused_max_tokens(True) == 8
+
+
 def test_workspace_layout(fm):
     d = fm.LayerDesc()
     n1, n64 = fm.fmoe_workspace_bytes(d, 1), fm.fmoe_workspace_bytes(d, 64)
