@@ -129,14 +129,15 @@ tc_stage_kernel(GroupWork w, const float* __restrict__ src, int K, int k1, int m
     }
     *reinterpret_cast<uint4*>(base + (size_t)kc * (2 * np / 8) * 128 + (size_t)(row >> 3) * 128 + (row & 7) * 16) = out;
   }
-  if (mode == 0 && g == E && gamma) {  // token i's gate in the CTA of step i % steps, one warp each
+  if (mode == 0 && g == E && gamma) {  // token i's gate in the CTA of step i % steps, all its warps
+    __shared__ float s_part[kTcThreads / 32];
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31, steps = K / 64;
-    for (int i = s + steps * warp; i < m; i += steps * (kTcThreads / 32)) {
+    for (int i = s; i < m; i += steps) {
       const int t = slots[i] / k1;
       const float* x = src + (size_t)t * K;
       float z = 0.f;
-#pragma unroll 8
-      for (int c = lane * 4; c < K; c += 128) {
+#pragma unroll 4
+      for (int c = (int)threadIdx.x * 4; c < K; c += kTcThreads * 4) {
         const float4 wv = __ldg(reinterpret_cast<const float4*>(w_sg + c));
         const float4 v = __ldg(reinterpret_cast<const float4*>(x + c));
         z = fmaf(wv.x, v.x, z);
@@ -145,7 +146,14 @@ tc_stage_kernel(GroupWork w, const float* __restrict__ src, int K, int k1, int m
         z = fmaf(wv.w, v.w, z);
       }
       z = warp_sum(z);
-      if (lane == 0) gamma[t] = 1.f / (1.f + expf(-z));
+      if (lane == 0) s_part[warp] = z;
+      __syncthreads();
+      if (threadIdx.x == 0) {
+        float zz = 0.f;
+        for (int w = 0; w < kTcThreads / 32; ++w) zz += s_part[w];
+        gamma[t] = 1.f / (1.f + expf(-zz));
+      }
+      __syncthreads();
     }
   }
 }
