@@ -567,7 +567,9 @@ def run_ours(args):
             "roofline": roofline, "e2e": e2e, "gpu_launches": launches,
             "clocks": clk.summary()}
     line["tokens_per_s"] = value / L  # one token through the L-layer stack
-    if not args.no_extra and wl.n_experts == 512:
+    # the further measurements run on a single-GPU run only (under torchrun
+    # every rank would repeat them, pinning host memory per rank)
+    if not args.no_extra and wl.n_experts == 512 and world == 1:
         line["batched"] = batched_measure(fm, synth, np, torch, layers[0], wl, stream)
         line["small_batch"] = small_batch_measure(fm, synth, torch, layers, wl, stream)
         line["quantiser"] = quantiser_measure(fm, torch, stream)
