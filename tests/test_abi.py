@@ -226,3 +226,19 @@ def test_workspace_layout(fm):
     offs = [fm.fmoe_workspace_offset(d, 3, w) for w in range(6)]
     assert offs == sorted(offs) and all(o % 256 == 0 for o in offs)
     assert fm.fmoe_workspace_offset(d, 3, 6) == 2 ** 64 - 1
+
+
+def test_header_and_c_example_compile_as_c():
+    """include/fmoe.h is a C header: the plain-C example compiles with gcc
+    -std=c11 against it (syntax and types only; no GPU needed)."""
+    import shutil
+    import subprocess
+    gcc = shutil.which("gcc")
+    cuda_inc = "/usr/local/cuda/include"
+    if not gcc or not os.path.exists(os.path.join(cuda_inc, "cuda_runtime.h")):
+        pytest.skip("gcc or the CUDA headers are not available")
+    root = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+    src = os.path.join(root, "quantized_expert_gemv_b200", "examples", "decode_host.c")
+    r = subprocess.run([gcc, "-std=c11", "-Wall", "-Werror", "-fsyntax-only", "-I", os.path.join(root, "include"),
+                        "-I", cuda_inc, src], capture_output=True, text=True)
+    assert r.returncode == 0, r.stderr
