@@ -181,8 +181,10 @@ void oracle_expert_ffn(const oracle_expert_t* ex, int H, int I, int G, const dou
  *   S_h  = |h| + sum_k |p_k y_k| + |gamma y_s|          (the sum's own terms)
  *        + sum_k p_k S_y,k + gamma S_y,s + |y_s| S_gamma  (inputs' errors)
  *        + 1e-2                                         (inputs' 1e-5 slack)
- *   S_xn = |w| r S_h + |xn'| (rho + 1),
- *   rho  = sum_j |h'_j| S_h,j / (H (mean(h'^2) + eps))   (first-order error of r). */
+ *   S_xn = |w| r S_h + |xn'| (rho + 1e-3),
+ *   rho  = sum_j |h'_j| S_h,j / (H (mean(h'^2) + eps))   (first-order error of r);
+ * the 1e-3 |xn'| term puts 1e-6 |xn'| into the tolerance: the fp32 rounding
+ * of r and of the two products that form xn'. */
 void oracle_combine_rmsnorm(int H, int k, const double* y, const double* S_y, const double* p,
                             double gamma, double S_gamma, const double* h, const float* w,
                             double eps, double* h_out, double* xn_out, double* S_h,
@@ -211,7 +213,7 @@ void oracle_combine_rmsnorm(int H, int k, const double* y, const double* S_y, co
   rho /= (double)H * (ms + eps);
   for (int i = 0; i < H; ++i) {
     xn_out[i] = h_out[i] * r * (double)w[i];
-    S_xn[i] = fabs((double)w[i]) * r * S_h[i] + fabs(xn_out[i]) * (rho + 1.0);
+    S_xn[i] = fabs((double)w[i]) * r * S_h[i] + fabs(xn_out[i]) * (rho + 1e-3);
   }
 }
 

@@ -427,3 +427,167 @@ def test_expert_record_size_matches_pages():
     # (each printed figure rounded to 1 GB)
     delta = g["layers"] * g["experts_per_layer"] * (int4 - int2) / 2 ** 30
     assert abs(delta - (g["model_gb_int4"] - g["model_gb_int2"])) <= 1.0
+
+
+# ------------------------------------------------------------ error scales ----
+# The oracle's error scale S of an output is a first-order bound: if every
+# input of a step moves by at most eps times its own scale (and every term of
+# a sum by eps times its magnitude), the output moves by at most eps * S, and
+# some choice of signs reaches it.  Each pin below moves the inputs of one
+# step by +-eps * S and measures the response of the oracle's own value
+# function (finite differences in fp64), so the scale is tied to how the
+# output actually depends on its inputs, not to a retyped formula.
+
+EPS = 1e-7
+
+
+def _tiny_expert(seed, H=256, I=128):
+    wl = synth.Workload(hidden=H, inter=I, n_experts=4)
+    return wl, synth.expert(wl, seed % 7, seed % 4)
+
+
+def _dense(q, s, b, G):
+    return oracle.dequantize(q, s, b, G)
+
+
+def test_error_scale_of_router_and_qgemv_is_sum_of_absolute_terms():
+    """S of a dense or dequantised product is sum_j |w_j x_j|: moving every
+    x_j by eps |x_j| sign(w_j) moves y by exactly eps * S."""
+    r = rng(40)
+    W = r.normal(0, 0.02, size=(9, 192)).astype(np.float32)
+    x = r.normal(size=192)
+    y, S = oracle.gemv_f32(W, x)
+    for i in range(9):
+        d = EPS * np.abs(x) * np.sign(W[i].astype(np.float64))
+        yp, _ = oracle.gemv_f32(W, x + d)
+        assert (yp[i] - y[i]) / EPS == pytest.approx(S[i], rel=1e-6)
+    wl, ex = _tiny_expert(1)
+    n = wl.hidden * wl.inter
+    q, s, b = ex.q[:n].reshape(wl.inter, wl.hidden), ex.scale[:n // 64].reshape(wl.inter, -1), \
+        ex.bias[:n // 64].reshape(wl.inter, -1)
+    w = _dense(q, s, b, 64)
+    xq = synth.tokens(wl, 1, stream=3)[0].astype(np.float64)
+    yq, Sq = oracle.qgemv(q, s, b, 64, xq)
+    for i in (0, 17, wl.inter - 1):
+        d = EPS * np.abs(xq) * np.sign(w[i])
+        yp, _ = oracle.qgemv(q, s, b, 64, xq + d)
+        assert (yp[i] - yq[i]) / EPS == pytest.approx(Sq[i], rel=1e-6)
+
+
+def test_error_scale_of_swiglu_outputs():
+    """S_a: the worst of the four sign choices of (g +- eps S_g, u +- eps S_u)
+    moves silu(g) u by eps S_a, to first order.  A wrong derivative of silu
+    (a dropped g sigmoid'(g) term, a swapped S_g / S_u) fails here."""
+    for seed in range(3):
+        wl, ex = _tiny_expert(seed)
+        x = synth.tokens(wl, 1, stream=10 + seed)[0].astype(np.float64) * (1 + 2 * seed)
+        out = oracle.expert_ffn(ex, wl.hidden, wl.inter, 64, x)
+        g, u, a = out["g"], out["u"], out["a"]
+        for i in range(wl.inter):
+            resp = max(abs(oracle.swiglu(g[i] + sg * EPS * out["S_g"][i], u[i] + su * EPS * out["S_u"][i]) - a[i])
+                       for sg in (-1, 1) for su in (-1, 1)) / EPS
+            assert resp == pytest.approx(out["S_a"][i], rel=1e-4, abs=1e-12), (seed, i)
+
+
+def test_error_scale_of_down_products_propagates_through_down_rows():
+    """S_y of an expert output = its own terms sum_j |Wd_rj a_j| plus
+    sum_j |Wd_rj| S_a,j.  The second part is measured: moving each a_j by
+    eps S_a,j sign(Wd_rj) moves y_r by eps times it.  H != I, so summing the
+    down matrix along the wrong axis cannot pass."""
+    wl, ex = _tiny_expert(2)
+    H, I = wl.hidden, wl.inter
+    x = synth.tokens(wl, 1, stream=20)[0].astype(np.float64)
+    out = oracle.expert_ffn(ex, H, I, 64, x)
+    n = H * I
+    qd = ex.q[2 * n:].reshape(H, I)
+    sd = ex.scale[2 * n // 64:].reshape(H, I // 64)
+    bd = ex.bias[2 * n // 64:].reshape(H, I // 64)
+    wd = _dense(qd, sd, bd, 64)
+    y0, own = oracle.qgemv(qd, sd, bd, 64, out["a"])
+    assert np.array_equal(y0, out["y"])
+    for r in range(0, H, 5):
+        yp, _ = oracle.qgemv(qd, sd, bd, 64, out["a"] + EPS * out["S_a"] * np.sign(wd[r]))
+        prop = (yp[r] - y0[r]) / EPS
+        assert out["S_y"][r] - own[r] == pytest.approx(prop, rel=1e-5), r
+
+
+def test_error_scale_of_shared_gate():
+    """S_gamma = d sigmoid / dz * S_z: z +- eps S_z moves gamma by eps S_gamma."""
+    wl = synth.TINY
+    lw = _tiny_layer(wl)
+    x = synth.tokens(wl, 1, stream=4)[0].astype(np.float64) * 3
+    ref = oracle.layer_token(wl, lw, x, x)
+    z, Sz = oracle.gemv_f32(lw.w_shared_gate[None], x)
+    resp = max(abs(oracle.sigmoid(z[0] + sgn * EPS * Sz[0]) - ref["gamma"]) for sgn in (-1, 1)) / EPS
+    assert resp == pytest.approx(ref["S_gamma"], rel=1e-5)
+
+
+def test_error_scale_of_combine():
+    """S_h - 1e-2 (the 1e-2 carries the inputs' absolute 1e-5 slack) is the
+    response of h' when h moves by eps |h|, every y_k by eps (|y_k| + S_y,k)
+    and gamma by eps S_gamma towards the sign of y_s: the sum's own terms plus
+    its inputs' errors, each with its weight (p_k >= 0, gamma >= 0)."""
+    r = rng(41)
+    H, k = 64, 4
+    y = r.normal(size=(k + 1, H)) * 2
+    S_y = np.abs(r.normal(size=(k + 1, H))) * 5
+    p = r.dirichlet(np.ones(k))
+    gamma, S_gamma = 0.3, 0.7
+    h = r.normal(size=H)
+    w = (1 + 0.1 * r.normal(size=H)).astype(np.float32)
+    ho, _, Sh, _ = oracle.combine_rmsnorm(y, p, gamma, h, w, 1e-6, S_y=S_y, S_gamma=S_gamma)
+    for sgn in (1.0, -1.0):
+        rows = np.sign(y[k]) == sgn
+        yp = y + EPS * (np.abs(y) + S_y)
+        hp, _, _, _ = oracle.combine_rmsnorm(yp, p, gamma + sgn * EPS * S_gamma, h + EPS * np.abs(h), w, 1e-6,
+                                             S_y=S_y, S_gamma=S_gamma)
+        resp = (hp - ho) / EPS
+        assert np.allclose(resp[rows], Sh[rows] - 1e-2, rtol=1e-5, atol=1e-9)
+
+
+def test_error_scale_of_rmsnorm():
+    """S_xn - 1e-3 |xn'| bounds the response of xn'_i to moves of h' by at
+    most eps S_h, and the worst-case move (h'_i towards w_i, every other h'_j
+    against the sign of h'_i h'_j w_i, which moves r the same way) reaches it
+    up to the cross term of h'_i with itself, 2 |w_i| h'_i^2 r^3 S_h,i / H.
+    A missing r-error term, or one without its 1/H, fails here."""
+    r_ = rng(42)
+    H = 64
+    h = r_.normal(size=H) * 1.5
+    w = (1 + 0.1 * r_.normal(size=H)).astype(np.float32)
+    z = np.zeros((2, H))
+    # k = 1, zero expert outputs and gamma 0: h' = h, S_h = |h| + 1e-2
+    ho, xo, Sh, Sx = oracle.combine_rmsnorm(z, np.ones(1), 0.0, h, w, 1e-6)
+    assert np.array_equal(ho, h)
+    rr = 1.0 / math.sqrt(np.mean(h * h) + 1e-6)
+    bound = Sx - 1e-3 * np.abs(xo)
+    for i in range(H):
+        wi = float(w[i])
+        d = -EPS * Sh * np.sign(h) * np.sign(wi * h[i])
+        d[i] = EPS * Sh[i] * np.sign(wi)
+        _, xp, _, _ = oracle.combine_rmsnorm(z, np.ones(1), 0.0, h + d, w, 1e-6)
+        resp = abs(xp[i] - xo[i]) / EPS
+        cross = 2 * abs(wi) * h[i] ** 2 * rr ** 3 * Sh[i] / H
+        assert resp <= bound[i] * (1 + 1e-5), i
+        assert resp >= (bound[i] - cross) * (1 - 1e-5) - 1e-9, i
+    # random moves within the scales never exceed the bound
+    for t in range(20):
+        d = EPS * Sh * r_.uniform(-1, 1, size=H)
+        _, xp, _, _ = oracle.combine_rmsnorm(z, np.ones(1), 0.0, h + d, w, 1e-6)
+        assert np.all(np.abs(xp - xo) <= EPS * bound * (1 + 1e-5))
+
+
+def test_layer_error_scales_compose_the_steps():
+    """oracle_layer_token's scales are those of its steps chained: S_y of each
+    selected expert from expert_ffn, then S_h / S_xn from combine_rmsnorm with
+    those S_y and S_gamma."""
+    wl = synth.TINY
+    lw = _tiny_layer(wl)
+    x = synth.tokens(wl, 1, stream=6)[0].astype(np.float64)
+    ref = oracle.layer_token(wl, lw, x, x)
+    for j, slot in enumerate(list(ref["ids"]) + [wl.n_experts]):
+        e = oracle.expert_ffn(lw.experts[int(slot)], wl.hidden, wl.inter, 64, x)
+        assert np.array_equal(e["S_y"], ref["S_y"][j])
+    _, _, Sh, Sx = oracle.combine_rmsnorm(ref["y"], ref["p"], ref["gamma"], x, lw.norm_w, wl.eps,
+                                          S_y=ref["S_y"], S_gamma=ref["S_gamma"])
+    assert np.array_equal(Sh, ref["S_h"]) and np.array_equal(Sx, ref["S_xn"])
