@@ -12,7 +12,7 @@ INCLUDE = os.path.join(ROOT, "include")
 LIB = os.path.join(PKG, "libfmoe.so")
 
 SOURCES = ["fmoe_kernels.cu", "fmoe_pack.cpp"]
-HEADERS = ["fmoe_device.cuh", "fmoe_layout.h"]
+HEADERS = sorted(f for f in os.listdir(CSRC) if f.endswith((".cuh", ".h")))
 
 NVCC_FLAGS = [
     "-gencode", "arch=compute_100a,code=sm_100a",

@@ -46,6 +46,9 @@ struct GroupWork {
   int4* items;  // [max_items] (group, first slot within the group, tokens, 0), by group
   int4* bitems; // [kGrpBuckets][max_items] the GEMV items of each size bucket
   int4* tc;     // [max_tc]    (group, first, tokens, running sum of the items' tokens rounded up to 8)
+  float* tscale;    // [T] tensor-core staging multiplier of each token (stage_tokens_kernel)
+  float* rscale;    // [staged rows] epilogue multiplier of each tensor-core row
+  unsigned* amax;   // [staged rows] max |a| of each tensor-core row (gate/up epilogue)
 };
 
 __host__ __device__ constexpr int group_max_tc(int T, int k, int min_tokens) {
@@ -208,11 +211,28 @@ __device__ __forceinline__ StagedX staged_i(unsigned char* base, size_t stride, 
   return staged_x_at(base + (size_t)i * stride, K);
 }
 
-// Stages every token's normed input once per step (int16 groups, the
-// layout of StagedX) at xs + t * stride.  grid T.
+// Stages every token's normed input once per step (24-bit block floating
+// point groups, the layout of StagedX) at xs + t * stride.  grid T.
+// With tscale, also the token's power-of-two staging multiplier for the
+// tensor-core products (tc_row_scale of its largest magnitude).
 __global__ void __launch_bounds__(kGrpThreads)
-stage_tokens_kernel(const float* __restrict__ xn, int H, unsigned char* __restrict__ xs, size_t stride) {
-  stage_x(xn + (size_t)blockIdx.x * H, H, staged_x_at(xs + blockIdx.x * stride, H));
+stage_tokens_kernel(const float* __restrict__ xn, int H, unsigned char* __restrict__ xs, size_t stride,
+                    float* __restrict__ tscale) {
+  const float* x = xn + (size_t)blockIdx.x * H;
+  stage_x(x, H, staged_x_at(xs + blockIdx.x * stride, H));
+  if (tscale) {
+    __shared__ float s_m[kGrpThreads / 32];
+    float m = 0.f;
+    for (int i = threadIdx.x; i < H; i += blockDim.x) m = fmaxf(m, fabsf(x[i]));
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
+    if ((threadIdx.x & 31) == 0) s_m[threadIdx.x >> 5] = m;
+    __syncthreads();
+    if (threadIdx.x == 0) {
+      for (int w = 1; w < kGrpThreads / 32; ++w) m = fmaxf(m, s_m[w]);
+      tscale[blockIdx.x] = tc_row_scale(m);
+    }
+  }
 }
 
 // Gate/up row pairs [p0, p1) of one record for the m <= MB tokens staged at
@@ -255,12 +275,13 @@ __device__ __forceinline__ void gateup_rows_multi(const uint8_t* rec, const Expe
         if (i < m) {
           const StagedX sx = staged_i(sxb, sxs, i, H);
           uint4 xv[8];
-          load_xv(sx, ng, g, xv);
+          uint2 xl[8];
+          load_xv(sx, ng, g, xv, xl);
           const float d = sx.delta[g], xs = sx.xsum[g];
 #pragma unroll
           for (int q = 0; q < PAIRS; ++q) {
-            yg[q][i] = group_epilogue(yg[q][i], sg[q], group_dot<BITS>(cg[q], xv), d, xs);
-            yu[q][i] = group_epilogue(yu[q][i], su[q], group_dot<BITS>(cu[q], xv), d, xs);
+            yg[q][i] = group_epilogue(yg[q][i], sg[q], group_dot<BITS>(cg[q], xv, xl), d, xs);
+            yu[q][i] = group_epilogue(yu[q][i], su[q], group_dot<BITS>(cu[q], xv, xl), d, xs);
           }
         }
       }
@@ -443,9 +464,10 @@ __device__ __forceinline__ void gateup_bulk_body(const ExpertSet& es, const Grou
           if (i < m) {
             const StagedX sx = staged_i(smem, sxs, i, H);
             uint4 xv[8];
-            load_xv(sx, ng, g0, xv);
-            yg[i] = group_epilogue(yg[i], sg, group_dot<4>(cg, xv), sx.delta[g0], sx.xsum[g0]);
-            yu[i] = group_epilogue(yu[i], su, group_dot<4>(cu, xv), sx.delta[g0], sx.xsum[g0]);
+            uint2 xl[8];
+            load_xv(sx, ng, g0, xv, xl);
+            yg[i] = group_epilogue(yg[i], sg, group_dot<4>(cg, xv, xl), sx.delta[g0], sx.xsum[g0]);
+            yu[i] = group_epilogue(yu[i], su, group_dot<4>(cu, xv, xl), sx.delta[g0], sx.xsum[g0]);
           }
         }
       } else {
@@ -456,9 +478,10 @@ __device__ __forceinline__ void gateup_bulk_body(const ExpertSet& es, const Grou
           if (i < m) {
             const StagedX sx = staged_i(smem, sxs, i, H);
             uint4 xv[8];
-            load_xv(sx, ng, g0, xv);
-            yg[i] = group_epilogue(yg[i], sg, group_dot<2>(cg, xv), sx.delta[g0], sx.xsum[g0]);
-            yu[i] = group_epilogue(yu[i], su, group_dot<2>(cu, xv), sx.delta[g0], sx.xsum[g0]);
+            uint2 xl[8];
+            load_xv(sx, ng, g0, xv, xl);
+            yg[i] = group_epilogue(yg[i], sg, group_dot<2>(cg, xv, xl), sx.delta[g0], sx.xsum[g0]);
+            yu[i] = group_epilogue(yu[i], su, group_dot<2>(cu, xv, xl), sx.delta[g0], sx.xsum[g0]);
           }
         }
       }
@@ -533,11 +556,13 @@ __device__ __forceinline__ void down_row_multi(const uint8_t* rec, const ExpertS
     for (int i = 0; i < MB; ++i) {
       if (i < m) {
         const StagedX sx = staged_i(sab, sas, i, I);
-        int acc = 0;
+        Acc2 acc{0, 0};
 #pragma unroll
         for (int b = 0; b < kWpg; ++b) {
-          if (BITS == 4) acc += word_dot4(wd[b], sx.xs[b * ngI + g]);
-          else acc += word_dot2(wd[b], sx.xs[(2 * b) * ngI + g], sx.xs[(2 * b + 1) * ngI + g]);
+          if (BITS == 4) acc = acc + word_dot4(wd[b], sx.xs[b * ngI + g], sx.xl[b * ngI + g]);
+          else
+            acc = acc + word_dot2(wd[b], sx.xs[(2 * b) * ngI + g], sx.xs[(2 * b + 1) * ngI + g],
+                                  sx.xl[(2 * b) * ngI + g], sx.xl[(2 * b + 1) * ngI + g]);
         }
         yv[i] = group_epilogue(yv[i], sb, acc, sx.delta[g], sx.xsum[g]);
       }

@@ -1,40 +1,56 @@
 // fmoe_fused.cuh -- one persistent kernel for a stack of MoE layers, batch 1.
 //
-// One CTA per SM, launched cooperatively so that every CTA is resident and
-// grid-wide barriers are safe.  The experts' intermediate dimension is cut
-// into column blocks of w = 8 (4-bit) or 16 (2-bit) units: a block is w
-// gate/up row pairs plus the matching w columns of the down matrix, one
-// 32-bit word of codes per hidden row (the packed record stores the down
-// matrix column block by column block).  A CTA that owns a block computes
-// its w SwiGLU outputs and, from them, the block's contribution to all H
-// outputs of the down product -- no other CTA's data is needed until the
-// partial outputs are summed.  Per layer:
-//   A  xn = h' r w (every CTA, whole vector) and this CTA's router rows
-//      (fp32, the shared gate vector as row E) -> logits
-//   -- barrier B1 (all logits written); while it completes, the CTA runs
-//      its block of the shared expert
-//   D  every CTA takes the top-k of all logits itself and fetches its run of
-//      routed blocks (each block's bytes are contiguous in the record)
-//   E  routed blocks: gate/up -> a -> weighted down contribution, held in
-//      registers (each thread owns H / 512 hidden rows)
-//   F  the CTA's partial output sum_j p_j y_j + gamma y_s for all H rows ->
-//      global; barrier B2
-//   G  each CTA sums the partials of its slice of rows in a fixed order,
-//      adds the residual -> h', and its part of sum(h'^2); barrier B3
+// One CTA per SM, launched cooperatively so that every CTA is resident.  The
+// experts' intermediate dimension is cut into column blocks of w = 8 (4-bit)
+// or 16 (2-bit) units: a block is w gate/up row pairs plus the matching w
+// columns of the down matrix, one 32-bit word of codes per hidden row (the
+// packed record stores the down matrix column block by column block).  A CTA
+// that owns a block computes its w SwiGLU outputs and, from them, the
+// block's contribution to all H outputs of the down product; the CTAs'
+// partial outputs are summed at the end of the layer.  Per layer:
+//   A  (all warps) xn = h' r w from the previous layer's h' and sums of
+//      squares (exchange words), staged as 24-bit block floating point;
+//      this CTA's router rows (fp32; the shared gate vector is row E) ->
+//      logits, published as exchange words
+//   E  two warp groups in a pipeline over the CTA's blocks (shared block
+//      first, then its routed blocks), each block in one of three shared-
+//      memory slots filled by bulk copies:
+//        gate/up warps (0-7): the block's gate/up group dot products, SwiGLU,
+//          the w outputs rounded to 24-bit block floating point -> handed to
+//          the down warps through shared memory and an mbarrier
+//        down warps (8-15): first read all logits, take the top-k, issue the
+//          routed blocks' copies; then for every block the down columns of
+//          all H rows (each thread 16 rows), weighted by the block's gate
+//          weight; a finished block's slot takes the next block at once
+//   F  the CTA's partial output for all H rows -> exchange words
+//   G  (all warps) each CTA sums the partials of its slice of rows in a fixed
+//      order, adds the residual -> h' and its part of sum(h'^2), published as
+//      exchange words for the next layer's A
+// The shared block does not depend on the routing: it is fetched during the
+// previous layer and its gate/up products run while the logits travel, so
+// the routed data, which cannot be requested before the top-k, has the
+// memory system to itself.  Every CTA's routed blocks lie in one 64-group of
+// one expert (the groups are spread over the CTAs), so one 16 KB entry holds
+// their down scale-bias words, and their down products share one scale per
+// row: they are accumulated unscaled and scaled once per layer.
 // Source pages: "What is Flash-MoE?" (a2a-mcp.org), sections
 // "Understanding Mixture-of-Experts", "2. FMA-optimised dequantisation
 // kernels" and "3. Hand-tuned Metal compute shaders" (deferred command-buffer
 // submission there plays the role the persistent kernel plays here: no host
 // round trip between the steps or between layers).
 //
-// Weight bytes move global -> shared with cp.async.bulk into three block
-// slots and two scale-bias entries (mbarrier completion).  At the top-k the
-// CTA requests its first three routed blocks and asks the L2 to prefetch
-// the rest and the next layer's router rows and shared block, so HBM keeps
-// streaming while the slots turn over.  Every weight byte is read from HBM
-// once per layer.  Every wait (mbarrier or grid barrier) is bounded: on
-// expiry the CTA sets FMOE_STATUS_WAIT_TIMEOUT, waits (bounded) for its own
-// copies in flight, and returns.
+// Exchanges between CTAs (logits, partial outputs, h' with its sums of
+// squares): the writers store fp32 values, then one release-add per CTA
+// (per writing warp for the logits) on a counter of that exchange; in each
+// reading CTA one thread polls the counter with acquire loads (a short sleep
+// between polls keeps the polling traffic off the lines being written) until
+// it reaches the layer's target, and after a CTA-local barrier every thread
+// reads the values.  The counters grow over the launch's layers and the
+// last CTA to leave returns them to zero.  Every wait (mbarrier,
+// counter) is bounded: on expiry the CTA sets
+// FMOE_STATUS_WAIT_TIMEOUT, records the abort in shared memory (later waits
+// return at once, every warp still passes every named barrier), waits
+// (bounded) for its own copies in flight, and returns.
 #pragma once
 
 #include <cstdint>
@@ -47,18 +63,35 @@ namespace fmoe {
 
 constexpr int kFusedThreads = 512;
 constexpr int kFusedWarps = kFusedThreads / 32;
+constexpr int kGuThreads = 256;  // warps 0-7: gate/up, SwiGLU
+constexpr int kGuWarps = kGuThreads / 32;
+constexpr int kDnThreads = kFusedThreads - kGuThreads;  // warps 8-15: routing, copies, down products
+constexpr int kDnWarps = kDnThreads / 32;
 constexpr int kFusedMaxLayers = 32;
 constexpr int kFusedMaxK = 8;
-constexpr int kFusedMaxCtas = 160;      // partial outputs in the workspace: [kFusedMaxCtas][H]
+constexpr int kFusedMaxE = 1024;
+constexpr int kFusedMaxH = 4096;
+constexpr int kFusedMaxCtas = 160;      // partial outputs in the workspace: [kFusedMaxCtas][kFusedMaxH]
 constexpr int kFusedMaxRouterRows = 4;  // router rows (E experts + the shared gate) per CTA
-constexpr int kFusedRowsPerThread = 8;  // hidden rows per thread in the down products: H <= 4096
-constexpr int kFusedMaxRouted = 16;     // routed blocks per CTA
+constexpr int kDnQuads = 4;             // groups of 4 consecutive hidden rows per down thread: H <= 4096
+constexpr int kDnRowsT = 4 * kDnQuads;  // hidden rows per down thread
+constexpr int kDnKeys = kFusedMaxE / kDnThreads;  // logits per down thread in the top-k
 constexpr int kSlots = 3;
-constexpr int kFirstWave = 2;  // routed blocks requested at the top-k; the rest after they land
-constexpr int kSbEntries = 2;
-constexpr int kMbSb = kSlots;  // mbarriers: the slots, then the scale-bias entries
-constexpr int kMbCount = kSlots + kSbEntries;
+constexpr int kDnxWords = 16;  // per slot: hi words [0, 8), lo words [8, 12), step, step * sum
+// mbarriers
+constexpr int kMbFull = 0;                 // [kSlots] a slot's bytes have landed
+constexpr int kMbReady = kMbFull + kSlots;  // [kSlots] a slot's SwiGLU outputs are staged
+constexpr int kMbSbShared = kMbReady + kSlots;
+constexpr int kMbSbRouted = kMbSbShared + 1;
+constexpr int kMbCount = kMbSbRouted + 1;
+constexpr int kBarGu = 1, kBarDn = 2;       // named barriers of the two warp groups
 constexpr long long kWaitCycles = 4000000000LL;  // ~2 s at 2 GHz
+// exchange counters (words of the workspace's counter area)
+constexpr int kCntH = 0;      // CTAs that published h' and their sum of squares (all layers so far)
+constexpr int kCntExit = 1;   // CTAs that left the kernel
+constexpr int kCntLogit = 3;  // router logits published
+constexpr int kCntPart = 4;   // CTAs that published their partial outputs
+constexpr unsigned kPollSleepNs = 32;
 
 struct FusedLayer {
   const uint8_t* experts;
@@ -74,11 +107,13 @@ struct FusedLayer {
 // words of one 64-group of one expert (4 H bytes).
 struct FusedPlan {
   uint32_t slot[kSlots];
-  uint32_t sbe[kSbEntries];
-  uint32_t xs;     // staged int16 x of the layer
-  uint32_t logit;  // fp32 [E]
-  uint32_t cand;   // top-k candidates: u64 [warps][k]
-  uint32_t red;    // fp32 [kFusedThreads]: partial sums of the row reduction
+  uint32_t sbe[2];  // shared expert, routed experts
+  uint32_t xs;      // staged x of the layer (24-bit block floating point)
+  uint32_t logit;   // fp32 [E]
+  uint32_t cand;    // top-k candidates: u64 [kDnWarps][k]
+  uint32_t gred;    // gate/up partial sums: fp32 [2][kGuWarps][8]
+  uint32_t dnx;     // staged SwiGLU outputs per slot: u32 [kSlots][kDnxWords]
+  uint32_t red;     // fp32 [kFusedThreads]: partial sums of the row reduction
   uint32_t mbar;
   uint32_t total;
 };
@@ -94,14 +129,12 @@ struct FusedArgs {
   int32_t* ids;
   float* weights;
   float* gamma;
-  float* a;          // [(k+1)][I], shared expert last
-  // exchange words between CTAs: (epoch << 32) | fp32 bits, written and read
-  // as single 64-bit accesses, so a reader that sees the epoch it waits for
-  // holds the value that came with it (no separate flag or barrier)
-  uint64_t* x_logit;  // [E + 1]: router logits, then sigmoid(w_sg . xn)
-  uint64_t* x_part;   // [gridDim.x][H]: partial outputs
-  float* ss_part;     // [gridDim.x]: partial sums of h'^2 (behind the grid barrier)
-  unsigned* sync;     // [0] grid-barrier arrivals, [1] exits, [2] epoch of the last launch
+  float* a;           // [(k+1)][I], shared expert last
+  float* x_logit;     // [E + 1]: router logits, then sigmoid(w_sg . xn)
+  float* x_h;         // [H]: h' of the layer
+  float* x_ss;        // [gridDim.x]: per-CTA sums of h'^2
+  float* x_part;      // [gridDim.x][H]: partial outputs
+  unsigned* sync;     // counters: kCntH, kCntExit, kCntLogit, kCntPart
   FusedPlan plan;
 };
 
@@ -117,6 +150,10 @@ __device__ __forceinline__ void mbar_init(uint64_t* bar, uint32_t count) {
 __device__ __forceinline__ void mbar_expect_tx(uint64_t* bar, uint32_t bytes) {
   asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(smem_u32(bar)), "r"(bytes)
                : "memory");
+}
+
+__device__ __forceinline__ void mbar_arrive(uint64_t* bar) {
+  asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(smem_u32(bar)) : "memory");
 }
 
 __device__ __forceinline__ void bulk_g2s(void* dst, const void* src, uint32_t bytes, uint64_t* bar) {
@@ -157,65 +194,31 @@ __device__ __forceinline__ void fence_proxy_async() {
   asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
 }
 
+__device__ __forceinline__ void named_bar(int id, int threads) {
+  asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(threads) : "memory");
+}
+
 // 16-byte shared-memory load (a plain load, so the compiler may schedule it
 // freely but never above an mbarrier wait, whose asm clobbers memory).
 __device__ __forceinline__ uint4 lds128(const void* p) { return *reinterpret_cast<const uint4*>(p); }
-
-__device__ __forceinline__ float ldcg_f(const float* p) { return __ldcg(p); }
 
 __device__ __forceinline__ float4 as_float4(uint4 v) {
   return make_float4(__uint_as_float(v.x), __uint_as_float(v.y), __uint_as_float(v.z), __uint_as_float(v.w));
 }
 
-__device__ __forceinline__ uint64_t ld_relaxed64(const uint64_t* p) {
-  uint64_t v;
-  asm volatile("ld.relaxed.gpu.global.b64 %0, [%1];" : "=l"(v) : "l"(p) : "memory");
-  return v;
+__device__ __forceinline__ void cnt_release_add(unsigned* p, unsigned v) {
+  asm volatile("red.release.gpu.global.add.u32 [%0], %1;" ::"l"(p), "r"(v) : "memory");
 }
 
-__device__ __forceinline__ void st_relaxed64(uint64_t* p, uint64_t v) {
-  asm volatile("st.relaxed.gpu.global.b64 [%0], %1;" ::"l"(p), "l"(v) : "memory");
-}
-
-__device__ __forceinline__ uint64_t x_word(uint32_t epoch, float v) {
-  return ((uint64_t)epoch << 32) | __float_as_uint(v);
-}
-
-__device__ __forceinline__ bool x_ready(uint64_t w, uint32_t epoch) { return (uint32_t)(w >> 32) == epoch; }
-
-// Re-reads *p until it carries `epoch` (bounded); false on expiry.
-__device__ __forceinline__ bool x_spin(const uint64_t* p, uint32_t epoch, uint64_t* w) {
-  if (x_ready(*w, epoch)) return true;
-  const long long t0 = clock64();
-  while (clock64() - t0 < kWaitCycles) {
-    *w = ld_relaxed64(p);
-    if (x_ready(*w, epoch)) return true;
-  }
-  return false;
-}
-
-// N exchange words at p(i) (those with valid(i)): re-reads, all in one round
-// trip per pass, the ones that do not yet carry `epoch` (bounded).
-// While words are missing, only the first missing one is polled; once it
-// has arrived, the others are re-read together.
-template <int N, class Addr, class Valid>
-__device__ __forceinline__ bool x_spin_all(uint64_t (&w)[N], uint32_t epoch, Addr p, Valid valid) {
+// Bounded poll (one thread) until *p >= target; false on expiry.
+__device__ __forceinline__ bool cnt_wait(const unsigned* p, unsigned target) {
   const long long t0 = clock64();
   while (true) {
-    int miss = -1;
-#pragma unroll
-    for (int i = N - 1; i >= 0; --i)
-      if (valid(i) && !x_ready(w[i], epoch)) miss = i;
-    if (miss < 0) return true;
+    unsigned v;
+    asm volatile("ld.acquire.gpu.global.u32 %0, [%1];" : "=r"(v) : "l"(p) : "memory");
+    if ((int)(v - target) >= 0) return true;
     if (clock64() - t0 > kWaitCycles) return false;
-    uint64_t v = ld_relaxed64(p(miss));
-    while (!x_ready(v, epoch)) {
-      if (clock64() - t0 > kWaitCycles) return false;
-      v = ld_relaxed64(p(miss));
-    }
-#pragma unroll
-    for (int i = 0; i < N; ++i)
-      if (valid(i) && !x_ready(w[i], epoch)) w[i] = i == miss ? v : ld_relaxed64(p(i));
+    __nanosleep(kPollSleepNs);
   }
 }
 
@@ -225,17 +228,19 @@ __host__ __device__ __forceinline__ void share(int total, int c, int n, int* lo,
   *hi = (int)(((long long)total * (c + 1)) / n);
 }
 
+// The 64-group of the routed blocks that CTA c of nC owns when the Gr groups
+// of the k selected experts are spread over the CTAs (Gr <= nC): group j
+// goes to CTAs [floor(j nC / Gr), floor((j + 1) nC / Gr)).
+__host__ __device__ __forceinline__ int routed_group_of(int c, int nC, int Gr) {
+  return (int)(((long long)(c + 1) * Gr - 1) / nC);
+}
+
 template <int BITS>
 __device__ __forceinline__ GroupCodes<BITS> lds_group(const uint8_t* row, int ng, int g) {
   GroupCodes<BITS> gc;
   gc.c[0] = lds128(row + chunk_off<BITS>(ng, g, 0));
   if (BITS == 4) gc.c[BITS == 4 ? 1 : 0] = lds128(row + chunk_off<BITS>(ng, g, 1));
   return gc;
-}
-
-__device__ __forceinline__ void lds_xv(const StagedX& s, int ng, int g, uint4* xv) {
-#pragma unroll
-  for (int u = 0; u < 8; ++u) xv[u] = lds128(s.xs + u * ng + g);
 }
 
 // Routing key of logit v at index e: one 64-bit integer whose order is the
@@ -275,26 +280,44 @@ __device__ __forceinline__ uint64_t warp_select_keys(uint64_t* key, int k) {
   return mine;
 }
 
+// Sum over the warp of V values per lane at once (V a power of two <= 32):
+// lane l returns the total of value l >> (5 - log2 V).  Halving exchanges
+// first (V / 2 + V / 4 + ... shuffles), then a plain butterfly.
+template <int V>
+__device__ __forceinline__ float warp_sum_multi(float (&v)[V]) {
+  const int lane = threadIdx.x & 31;
+  int o = 16;
+#pragma unroll
+  for (int n = V; n > 1; n >>= 1, o >>= 1) {
+    const bool up = (lane & o) != 0;
+#pragma unroll
+    for (int i = 0; i < n / 2; ++i) {
+      const float send = up ? v[i] : v[i + n / 2];
+      const float keep = up ? v[i + n / 2] : v[i];
+      v[i] = keep + __shfl_xor_sync(0xffffffffu, send, o);
+    }
+  }
+  float r = v[0];
+  for (; o > 0; o >>= 1) r += __shfl_xor_sync(0xffffffffu, r, o);
+  return r;
+}
+
 // Geometry of a column block of an expert with BITS-bit codes.
 template <int BITS>
 struct BlockGeo {
-  static constexpr int kW = 32 / BITS;             // intermediate units per block
-  static constexpr int kPerGroup = 64 / kW;        // blocks per 64-group
-  static constexpr int kTpp = kFusedThreads / kW;  // threads per gate/up row pair
+  static constexpr int kW = 32 / BITS;       // intermediate units per block
+  static constexpr int kPerGroup = 64 / kW;  // blocks per 64-group
+  static constexpr int kPairsPerThread = kW / 4;  // a gate/up thread's row pairs per block
   __host__ __device__ static uint32_t gu_codes(int H) { return 8u * (uint32_t)H; }
   __host__ __device__ static uint32_t dn_codes(int H) { return 4u * (uint32_t)H; }
   __host__ __device__ static uint32_t gu_sb(int H) { return (uint32_t)kW * 2u * (uint32_t)(H / 64) * 4u; }
 };
 
-// Block state shared by the threads of a CTA.
-struct BlockShared {
-  float gu[kFusedWarps][4][2];  // per warp, per pair of the thread set: partial gate / up sums
-};
-
-// The staged inputs of one 64-group, kept in registers for the whole layer:
-// thread t serves group t % 64 of every gate/up row it touches.
+// The staged inputs of one 64-group, kept in registers by a gate/up thread
+// for the whole layer: thread t serves group t % 64 of every row it touches.
 struct XGroup {
   uint4 xv[8];
+  uint2 xl[8];
   float delta, xsum;
 };
 
@@ -302,123 +325,115 @@ __device__ __forceinline__ XGroup load_xgroup(const StagedX& sx, int ngH) {
   XGroup x;
   const int g = threadIdx.x & 63;
   if (g < ngH) {
-    lds_xv(sx, ngH, g, x.xv);
+#pragma unroll
+    for (int u = 0; u < 8; ++u) {
+      x.xv[u] = lds128(sx.xs + u * ngH + g);
+      x.xl[u] = sx.xl[u * ngH + g];
+    }
     x.delta = sx.delta[g];
     x.xsum = sx.xsum[g];
   } else {
 #pragma unroll
-    for (int u = 0; u < 8; ++u) x.xv[u] = make_uint4(0u, 0u, 0u, 0u);
+    for (int u = 0; u < 8; ++u) {
+      x.xv[u] = make_uint4(0u, 0u, 0u, 0u);
+      x.xl[u] = make_uint2(0u, 0u);
+    }
     x.delta = x.xsum = 0.f;
   }
   return x;
 }
 
-// One or two column blocks (NB), block n held in slots[n]: gate/up of
-// their w row pairs each, SwiGLU, each block's w outputs rounded to 16-bit
-// fixed point with its own step, then the blocks' down columns for every
-// hidden row this thread owns, block n scaled by weight[n], added to y.
-// Thread t works on group t % 64 of pairs t / 64 + 8 i (pair p = block
-// p / w, row pair p % w of it); every warp then forms all the blocks'
-// outputs itself from the per-warp sums, so one block-wide barrier separates
-// the two halves.  a_out[n] (global) receives block n's w SwiGLU outputs.
-// The slots may be refilled after the closing barrier.
-template <int B, int NB>
-__device__ __forceinline__ void run_blocks(const uint8_t* const (&slots)[2], const uint32_t* const (&dsb)[2], int H,
-                                           const XGroup& xg, const float (&weight)[2], float* const (&a_out)[2],
-                                           BlockShared& bs, float (&y)[kFusedRowsPerThread]) {
+// Gate/up part of one block (gate/up threads): thread t takes group t % 64
+// of row pairs t / 64 + 4 i (both rows of each), and writes its warp's sums
+// to gred [warp][value] (value 2 i: gate of pair i, 2 i + 1: up).
+template <int B>
+__device__ __forceinline__ void block_gateup(const uint8_t* slot, int H, const XGroup& xg, float* gred) {
+  using G = BlockGeo<B>;
+  constexpr int kV = 2 * G::kPairsPerThread;  // 4 or 8 values per thread
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  const int ngH = H / 64, g = tid & 63, ps = tid >> 6;
+  const uint32_t rb = (uint32_t)H * B / 8;
+  const uint32_t* sbw = reinterpret_cast<const uint32_t*>(slot + G::gu_codes(H) + G::dn_codes(H));
+  float v[kV];
+#pragma unroll
+  for (int i = 0; i < G::kPairsPerThread; ++i) {
+    v[2 * i] = v[2 * i + 1] = 0.f;
+    if (g < ngH) {
+      const int pl = ps + 4 * i;
+      const uint8_t* rg = slot + (size_t)(2 * pl) * rb;
+      const GroupCodes<B> cg = lds_group<B>(rg, ngH, g);
+      const GroupCodes<B> cu = lds_group<B>(rg + rb, ngH, g);
+      v[2 * i] = group_epilogue(0.f, sbw[2 * pl * ngH + g], group_dot<B>(cg, xg.xv, xg.xl), xg.delta, xg.xsum);
+      v[2 * i + 1] =
+          group_epilogue(0.f, sbw[(2 * pl + 1) * ngH + g], group_dot<B>(cu, xg.xv, xg.xl), xg.delta, xg.xsum);
+    }
+  }
+  const float r = warp_sum_multi<kV>(v);
+  constexpr int kLanesPer = 32 / kV;
+  if ((lane & (kLanesPer - 1)) == 0) gred[warp * 8 + lane / kLanesPer] = r;
+}
+
+// SwiGLU of one block from the gate/up sums (gate/up warp 0): lane p < w
+// forms a_p; the w outputs get one power-of-two step (24-bit block floating
+// point) and go to dnx (high parts, low parts, step, step * sum) for the
+// down warps, and to a_out (global).
+template <int B>
+__device__ __forceinline__ void block_swiglu(const float* gred, uint32_t* dnx, float* a_out) {
   using G = BlockGeo<B>;
   constexpr int kW = G::kW;
-  constexpr int kNP = NB * kW;   // row pairs: 8, 16 or 32
-  constexpr int kPP = kNP / 8;   // pairs per thread
-  static_assert(kNP <= 32 && kPP <= 4, "one warp forms all outputs");
-  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
-  const int ngH = H / 64;
-  const int g = tid & 63, ps = tid >> 6;
-  {
-    const uint32_t rb = (uint32_t)H * B / 8;
-    float gs[kPP], us[kPP];
+  const int lane = threadIdx.x & 31;
+  float a = 0.f;
+  if (lane < kW) {
+    const int ps = lane & 3, i = lane >> 2;
+    const float gs = gred[(2 * ps) * 8 + 2 * i] + gred[(2 * ps + 1) * 8 + 2 * i];
+    const float us = gred[(2 * ps) * 8 + 2 * i + 1] + gred[(2 * ps + 1) * 8 + 2 * i + 1];
+    a = silu_mul(gs, us);
+    a_out[lane] = a;
+  }
+  const float m = __uint_as_float(__reduce_max_sync(0xffffffffu, __float_as_uint(fabsf(a))));
+  float inv, delta;
+  bfp_step(m, &inv, &delta);
+  const int q = bfp_int(a, inv);
+  const int qsum = __reduce_add_sync(0xffffffffu, q);
+  const uint32_t hi = (uint32_t)(q >> 8) & 0xFFFFu, lo = (uint32_t)q & 0xFFu;
+  const uint32_t hi1 = __shfl_down_sync(0xffffffffu, hi, 1);
+  const uint32_t lo1 = __shfl_down_sync(0xffffffffu, lo, 1);
+  const uint32_t lo2 = __shfl_down_sync(0xffffffffu, lo, 2);
+  const uint32_t lo3 = __shfl_down_sync(0xffffffffu, lo, 3);
+  if (lane < kW && (lane & 1) == 0) dnx[lane >> 1] = hi | (hi1 << 16);
+  if (lane < kW && (lane & 3) == 0) dnx[8 + (lane >> 2)] = lo | (lo1 << 8) | (lo2 << 16) | (lo3 << 24);
+  if (lane == 0) {
+    dnx[12] = __float_as_uint(delta);
+    dnx[13] = __float_as_uint(delta * (float)qsum);
+  }
+}
+
+// Down part of one block (down threads): for the thread's row quads, the
+// block's code words times the staged SwiGLU outputs; returns the 24-bit
+// value sums in t[16] (rows 4 (t' + 256 m) + r at t[4 m + r]).
+template <int B>
+__device__ __forceinline__ void block_down(const uint8_t* slot, const uint32_t* dnx, int H, float (&t)[kDnRowsT]) {
+  using G = BlockGeo<B>;
+  const int td = threadIdx.x - kGuThreads;
+  const uint4 h0 = lds128(dnx), h1 = lds128(dnx + 4), l01 = lds128(dnx + 8);
+  const uint32_t* dc = reinterpret_cast<const uint32_t*>(slot + G::gu_codes(H));
 #pragma unroll
-    for (int pp = 0; pp < kPP; ++pp) {
-      // pair ps + 8 pp: block (8 pp) / w and row pair ps + 8 (pp % (w / 8)) of it (ps < 8)
-      constexpr int kSub = kW / 8;
-      const int n = (8 * pp) / kW, pl = ps + 8 * (pp % kSub);
-      gs[pp] = us[pp] = 0.f;
-      if (g < ngH) {
-        const uint8_t* rg = slots[n] + (size_t)(2 * pl) * rb;
-        const uint32_t* sbg = reinterpret_cast<const uint32_t*>(slots[n] + G::gu_codes(H) + G::dn_codes(H)) +
-                              2 * pl * ngH;
-        const GroupCodes<B> cg = lds_group<B>(rg, ngH, g);
-        const GroupCodes<B> cu = lds_group<B>(rg + rb, ngH, g);
-        gs[pp] = group_epilogue(0.f, sbg[g], group_dot<B>(cg, xg.xv), xg.delta, xg.xsum);
-        us[pp] = group_epilogue(0.f, sbg[ngH + g], group_dot<B>(cu, xg.xv), xg.delta, xg.xsum);
-      }
-    }
+  for (int m = 0; m < kDnQuads; ++m) {
+    const int row = 4 * (td + kDnThreads * m);
+    if (row < H) {
+      const uint4 w = lds128(dc + row);
+      const uint32_t ws[4] = {w.x, w.y, w.z, w.w};
 #pragma unroll
-    for (int pp = 0; pp < kPP; ++pp) {
-      const float gsum = warp_sum(gs[pp]), usum = warp_sum(us[pp]);
-      if (lane == 0) {
-        bs.gu[warp][pp][0] = gsum;
-        bs.gu[warp][pp][1] = usum;
+      for (int r = 0; r < 4; ++r) {
+        const Acc2 acc = B == 4 ? word_dot4(ws[r], h0, make_uint2(l01.x, l01.y))
+                                : word_dot2(ws[r], h0, h1, make_uint2(l01.x, l01.y), make_uint2(l01.z, l01.w));
+        t[4 * m + r] = acc_value(acc);
       }
+    } else {
+#pragma unroll
+      for (int r = 0; r < 4; ++r) t[4 * m + r] = 0.f;
     }
   }
-  __syncthreads();
-  // every warp: SwiGLU of all pairs (lane l < kNP: pair l, whose sums sit in
-  // warps 2 (l % 8), 2 (l % 8) + 1, slot l / 8), one fixed-point step per
-  // block, the int16 pairs of every block spread to all lanes
-  uint32_t xw[NB][8];
-  float p1[NB], p2[NB];
-  {
-    float a = 0.f;
-    if (lane < kNP) {
-      const int pw = 2 * (lane & 7), pp = lane >> 3;
-      a = silu_mul(bs.gu[pw][pp][0] + bs.gu[pw + 1][pp][0], bs.gu[pw][pp][1] + bs.gu[pw + 1][pp][1]);
-      if (warp == 0) (NB == 2 && lane >= kW ? a_out[NB - 1] : a_out[0])[lane % kW] = a;
-    }
-    const int mine = lane / kW;  // this lane's block (>= NB: none)
-    float delta_m = 0.f;
-#pragma unroll
-    for (int n = 0; n < NB; ++n) {
-      const float m = __uint_as_float(__reduce_max_sync(0xffffffffu, mine == n ? __float_as_uint(fabsf(a)) : 0u));
-      const float delta = m * (1.f / 32767.f);
-      if (mine == n) delta_m = m > 0.f ? 32767.f / m : 0.f;
-      p1[n] = weight[n] * delta;
-    }
-    int q = __float2int_rn(a * delta_m);
-    q = q > 32767 ? 32767 : (q < -32767 ? -32767 : q);
-#pragma unroll
-    for (int n = 0; n < NB; ++n) p2[n] = p1[n] * (float)__reduce_add_sync(0xffffffffu, mine == n ? q : 0);
-    const int q_hi = __shfl_down_sync(0xffffffffu, q, 1);
-    const uint32_t word = (uint32_t)(q & 0xFFFF) | ((uint32_t)q_hi << 16);
-#pragma unroll
-    for (int n = 0; n < NB; ++n) {
-#pragma unroll
-      for (int i = 0; i < 8; ++i) xw[n][i] = i < kW / 2 ? __shfl_sync(0xffffffffu, word, n * kW + 2 * i) : 0u;
-    }
-  }
-  {
-    const uint32_t* dc[NB];
-#pragma unroll
-    for (int n = 0; n < NB; ++n) dc[n] = reinterpret_cast<const uint32_t*>(slots[n] + G::gu_codes(H));
-#pragma unroll
-    for (int m = 0; m < kFusedRowsPerThread; ++m) {
-      const int i = tid + m * kFusedThreads;
-      if (i < H) {
-        float v = y[m];
-#pragma unroll
-        for (int n = 0; n < NB; ++n) {
-          const uint32_t w = dc[n][i], sbw = dsb[n][i];
-          const int acc = B == 4 ? word_dot4(w, make_uint4(xw[n][0], xw[n][1], xw[n][2], xw[n][3]))
-                                 : word_dot2(w, make_uint4(xw[n][0], xw[n][1], xw[n][2], xw[n][3]),
-                                             make_uint4(xw[n][4], xw[n][5], xw[n][6], xw[n][7]));
-          const float sc = __uint_as_float(sbw << 16), bi = __uint_as_float(sbw & 0xFFFF0000u);
-          v = fmaf(sc, p1[n] * (float)acc, fmaf(bi, p2[n], v));
-        }
-        y[m] = v;
-      }
-    }
-  }
-  __syncthreads();
 }
 
 // ------------------------------------------------------------ the kernel --
@@ -432,54 +447,69 @@ __global__ void __launch_bounds__(kFusedThreads, 1) fused_stack_kernel(const __g
   __shared__ float s_gamma;
   __shared__ float s_rp[kFusedWarps][kFusedMaxRouterRows];
   __shared__ float s_red[kFusedWarps];
-  __shared__ BlockShared s_blk;
+  __shared__ volatile int s_abort;
 
   const int c = blockIdx.x, nC = gridDim.x;
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int H = A.H, I = A.I, E = A.E, k = A.k;
-  const int ngH = H / 64;
+  const int ngH = H / 64, ngI = I / 64;
   const FusedPlan& P = A.plan;
   uint64_t* mbar = reinterpret_cast<uint64_t*>(smem + P.mbar);
   const StagedX sx = staged_x_at(smem + P.xs, H);
   float* slog = reinterpret_cast<float*>(smem + P.logit);
   uint64_t* cand = reinterpret_cast<uint64_t*>(smem + P.cand);
+  float* gred = reinterpret_cast<float*>(smem + P.gred);
+  uint32_t* dnx = reinterpret_cast<uint32_t*>(smem + P.dnx);
   float* sred = reinterpret_cast<float*>(smem + P.red);
 
-  // static work of this CTA
+  // ---- static work of this CTA ----
   const int nr = c <= E ? (E - c) / nC + 1 : 0;  // router rows c, c + nC, ... <= E (row E: shared gate)
-  const int NBr = I * BITS / 32, NBs = I * SBITS / 32;
-  const bool has_shared = c < NBs;  // shared block c
-  int q0, q1, i0, i1;
-  share(k * NBr, c, nC, &q0, &q1);  // routed blocks, expert-major
-  share(H, c, nC, &i0, &i1);        // hidden rows of the final sums
-  const int nq = q1 - q0, nd = i1 - i0;
+  const int NBs = I * SBITS / 32;
+  const int S = c < NBs ? 1 : 0;  // shared block c
+  // routed blocks: [rb0, rb1) of 64-group jg of the k selected experts'
+  // groups (expert jj = jg / ngI, group gr = jg % ngI)
+  const int Gr = k * ngI;
+  const int jg = routed_group_of(c, nC, Gr);
+  int rb0, rb1;
+  {
+    const int cs0 = (int)(((long long)jg * nC) / Gr), cs1 = (int)(((long long)(jg + 1) * nC) / Gr);
+    share(GR::kPerGroup, c - cs0, cs1 - cs0, &rb0, &rb1);
+  }
+  const int nq = rb1 - rb0, jj = jg / ngI, gr = jg % ngI;
+  const int nseq = S + nq;  // blocks per layer: the shared one first
+  int i0, i1;
+  share(H, c, nC, &i0, &i1);  // hidden rows of the final sums
+  const int nd = i1 - i0;
   const RecordLayout LR = record_layout(BITS, H, I);
   const RecordLayout LS = record_layout(SBITS, H, I);
   const bool xthr = tid * 8 < H;  // this thread holds inputs 8 tid .. 8 tid + 7
+  const bool issuer = tid == kGuThreads;  // lane 0 of the first down warp issues every copy
 
   if (tid == 0) {
     for (int i = 0; i < kMbCount; ++i) mbar_init(&mbar[i], 1);
+    s_abort = 0;
+    cand[kDnWarps * kFusedMaxK] = 0;  // NaN-logit flag of the top-k
     asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
   }
   __syncthreads();
 
-  uint32_t phase = 0;  // per mbarrier: parity of its next completion (same in every thread)
-  uint32_t armed = 0;  // lane 0 of an issuing warp: its mbarriers with copies in flight
-
-  // ---- copies (lane 0 of one warp per mbarrier: slot s <- warp s, entry e
-  // <- warp kSlots + e, so each issuer drains its own copies on abort) ----
+  // issuer: mbarriers it has armed, and per mbarrier the parity of the next
+  // phase it will arm (each phase of a copy barrier is armed once, by it)
+  uint32_t armed = 0, next_par = 0;
   auto arm = [&](int mb, uint32_t bytes) {
     mbar_expect_tx(&mbar[mb], bytes);
     armed |= 1u << mb;
+    next_par ^= 1u << mb;
   };
   // column block nb of the record `rec` into slot s
   auto issue_block = [&](int s, const uint8_t* rec, const RecordLayout& L, int nb, uint32_t gu_sb_bytes) {
     uint8_t* dst = smem + P.slot[s];
     const uint32_t gub = 8u * (uint32_t)H, dnb = 4u * (uint32_t)H;
-    arm(s, gub + dnb + gu_sb_bytes);
-    bulk_g2s(dst, rec + L.gu_codes + (size_t)nb * gub, gub, &mbar[s]);
-    bulk_g2s(dst + gub, rec + L.down_codes + (size_t)nb * dnb, dnb, &mbar[s]);
-    bulk_g2s(dst + gub + dnb, rec + L.gu_sb + (size_t)nb * gu_sb_bytes, gu_sb_bytes, &mbar[s]);
+    fence_proxy_async();
+    arm(kMbFull + s, gub + dnb + gu_sb_bytes);
+    bulk_g2s(dst, rec + L.gu_codes + (size_t)nb * gub, gub, &mbar[kMbFull + s]);
+    bulk_g2s(dst + gub, rec + L.down_codes + (size_t)nb * dnb, dnb, &mbar[kMbFull + s]);
+    bulk_g2s(dst + gub + dnb, rec + L.gu_sb + (size_t)nb * gu_sb_bytes, gu_sb_bytes, &mbar[kMbFull + s]);
   };
   auto prefetch_block = [&](const uint8_t* rec, const RecordLayout& L, int nb, uint32_t gu_sb_bytes) {
     const uint32_t gub = 8u * (uint32_t)H, dnb = 4u * (uint32_t)H;
@@ -489,78 +519,59 @@ __global__ void __launch_bounds__(kFusedThreads, 1) fused_stack_kernel(const __g
   };
   // down scale-bias words of 64-group g of a record into entry e
   auto issue_sb = [&](int e, const uint8_t* rec, const RecordLayout& L, int g) {
-    arm(kMbSb + e, 4u * (uint32_t)H);
-    bulk_g2s(smem + P.sbe[e], rec + L.down_sb + (size_t)g * H * 4, 4u * (uint32_t)H, &mbar[kMbSb + e]);
+    fence_proxy_async();
+    arm(kMbSbShared + e, 4u * (uint32_t)H);
+    bulk_g2s(smem + P.sbe[e], rec + L.down_sb + (size_t)g * H * 4, 4u * (uint32_t)H, &mbar[kMbSbShared + e]);
   };
-  // layer l's shared block -> slot 1 (warp 1), its scale-bias -> entry 0 (warp kSlots); lane 0 only
-  auto issue_shared = [&](int l) {
-    if (!has_shared) return;
-    const uint8_t* rec = A.layers[l].shared;
-    if (warp == 1) {
-      fence_proxy_async();
-      issue_block(1, rec, LS, c, GS::gu_sb(H));
-    } else if (warp == kSlots) {
-      fence_proxy_async();
-      issue_sb(0, rec, LS, c / GS::kPerGroup);
+  // block at position p of layer l (p < nseq; positions of the next layer
+  // are not requested here) into its slot
+  auto issue_pos = [&](int l, uint32_t sq, int p) {
+    const int s = (int)((sq + (uint32_t)p) % kSlots);
+    if (p < S) {
+      issue_block(s, A.layers[l].shared, LS, c, GS::gu_sb(H));
+    } else {
+      const int b = p - S;
+      issue_block(s, A.layers[l].experts + (size_t)s_ids[jj] * LR.bytes, LR, (jg % ngI) * GR::kPerGroup + rb0 + b,
+                  GR::gu_sb(H));
     }
   };
-
-  // L2 prefetch of layer l's router rows and shared block (any one thread)
-  auto prefetch_next = [&](int l) {
+  // L2 prefetch of layer l's router rows
+  auto prefetch_router = [&](int l) {
     const FusedLayer& NX = A.layers[l];
     for (int m = 0; m < nr; ++m) {
       const int row = c + m * nC;
       prefetch_l2(row < E ? NX.w_router + (size_t)row * H : NX.w_sg, 4u * (uint32_t)H);
     }
-    if (has_shared) {
-      prefetch_block(NX.shared, LS, c, GS::gu_sb(H));
-      prefetch_l2(NX.shared + LS.down_sb + (size_t)(c / GS::kPerGroup) * H * 4, 4u * (uint32_t)H);
-    }
   };
 
-  // ---- waits (all threads; the outcome is agreed block-wide) ----
-  auto wait_mb = [&](int mb) -> bool {
-    const bool ok = mbar_wait(&mbar[mb], (phase >> mb) & 1u);
-    phase ^= 1u << mb;
-    if (lane == 0 && ok) armed &= ~(1u << mb);
-    if (__syncthreads_and(ok)) return true;
-    if (tid == 0) raise_status(FMOE_STATUS_WAIT_TIMEOUT);
-    return false;
-  };
-
-  // block-wide agreement after a round of exchange reads
-  auto x_agree = [&](bool ok) -> bool {
-    if (__syncthreads_and(ok)) return true;
-    if (tid == 0) raise_status(FMOE_STATUS_WAIT_TIMEOUT);
-    return false;
-  };
-  // grid barrier after h' (every CTA needs all of it): arrive once this
-  // CTA's rows are written, wait at the start of the next layer
-  // (release/acquire on one counter, bounded spin)
-  unsigned bar_target = 0;
-  auto grid_arrive = [&]() {
-    __syncthreads();
-    bar_target += (unsigned)nC;
-    if (tid == 0) asm volatile("red.release.gpu.global.add.u32 [%0], 1;" ::"l"(A.sync) : "memory");
-  };
-  auto grid_wait = [&]() -> bool {
-    bool ok = true;
-    if (tid == 0) {
-      ok = false;
-      const long long t0 = clock64();
-      while (true) {
-        unsigned v;
-        asm volatile("ld.acquire.gpu.global.u32 %0, [%1];" : "=r"(v) : "l"(A.sync) : "memory");
-        if (v >= bar_target) { ok = true; break; }
-        if (clock64() - t0 > kWaitCycles) break;
+  // bounded mbarrier wait; false once this CTA has aborted (every later wait
+  // returns at once)
+  auto wait_mb = [&](int mb, uint32_t parity) -> bool {
+    if (s_abort) return false;
+    if (mbar_try(&mbar[mb], parity)) return true;
+    const long long t0 = clock64();
+    while (!s_abort) {
+      if (mbar_try(&mbar[mb], parity)) return true;
+      if (clock64() - t0 > kWaitCycles) {
+        s_abort = 1;
+        raise_status(FMOE_STATUS_WAIT_TIMEOUT);
+        return false;
       }
     }
-    return x_agree(ok);
+    return false;
+  };
+  // CTA-wide wait for an exchange counter (thread 0 polls)
+  auto cta_cnt_wait = [&](int which, unsigned target) -> bool {
+    bool ok = true;
+    if (tid == 0) ok = cnt_wait(A.sync + which, target);
+    if (__syncthreads_and(ok && !s_abort)) return true;
+    if (tid == 0) raise_status(FMOE_STATUS_WAIT_TIMEOUT);
+    return false;
   };
   // r = (sum of the CTAs' partial sums of h'^2 / H + eps)^(-1/2), summed in
-  // the same order in every CTA (after the grid barrier)
-  auto norm_scale = [&]() -> float {
-    float v = tid < nC ? ldcg_f(A.ss_part + tid) : 0.f;
+  // the same order in every CTA; ssv: this thread's partial (tid < nC)
+  auto norm_scale = [&](float ssv) -> float {
+    float v = tid < nC ? ssv : 0.f;
     v = warp_sum(v);
     if (lane == 0) s_red[warp] = v;
     __syncthreads();
@@ -571,15 +582,17 @@ __global__ void __launch_bounds__(kFusedThreads, 1) fused_stack_kernel(const __g
     return 1.f / sqrtf(t / (float)H + A.eps);
   };
 
-  const uint32_t base = __ldcg(A.sync + 2);  // epochs of this launch: base + 2 l + 1, base + 2 l + 2
-  if (lane == 0 && A.n_layers > 0) issue_shared(0);
+  uint32_t sq = 0;                           // blocks of earlier layers (slot of position p: (sq + p) % 3)
+  // the first layer's shared block and its down scale-bias entry
+  if (issuer && A.n_layers > 0 && S) {
+    issue_pos(0, 0u, 0);
+    issue_sb(0, A.layers[0].shared, LS, c / GS::kPerGroup);
+  }
 
-  float yr[kFusedRowsPerThread], ys[kFusedRowsPerThread];
+  float yacc[kDnRowsT];  // down threads: this CTA's partial output rows
   bool aborted = false;
   for (int l = 0; l < A.n_layers; ++l) {
     const FusedLayer& LY = A.layers[l];
-#pragma unroll
-    for (int m = 0; m < kFusedRowsPerThread; ++m) yr[m] = ys[m] = 0.f;
     // ------------------------------------------------------------- A --
     // router rows (requested before anything they do not depend on)
     float4 wr[kFusedMaxRouterRows][2];
@@ -604,53 +617,22 @@ __global__ void __launch_bounds__(kFusedThreads, 1) fused_stack_kernel(const __g
       xv[0] = v0.x; xv[1] = v0.y; xv[2] = v0.z; xv[3] = v0.w;
       xv[4] = v1.x; xv[5] = v1.y; xv[6] = v1.z; xv[7] = v1.w;
     } else {
-      if (!grid_wait()) { aborted = true; break; }  // h' of the previous layer written
+      // h' and the sums of squares of the previous layer: every CTA has published them
+      if (!cta_cnt_wait(kCntH, (unsigned)l * (unsigned)nC)) { aborted = true; break; }
       float4 h0 = make_float4(0.f, 0.f, 0.f, 0.f), h1 = h0, w0 = h0, w1 = h0;
       const float* wprev = A.layers[l - 1].norm_w;
       if (xthr) {
-        h0 = __ldcg(reinterpret_cast<const float4*>(A.h + tid * 8));
-        h1 = __ldcg(reinterpret_cast<const float4*>(A.h + tid * 8 + 4));
+        h0 = __ldcg(reinterpret_cast<const float4*>(A.x_h + tid * 8));
+        h1 = __ldcg(reinterpret_cast<const float4*>(A.x_h + tid * 8 + 4));
         w0 = __ldg(reinterpret_cast<const float4*>(wprev + tid * 8));
         w1 = __ldg(reinterpret_cast<const float4*>(wprev + tid * 8 + 4));
       }
-      const float r = norm_scale();
+      const float r = norm_scale(tid < nC ? __ldcg(A.x_ss + tid) : 0.f);
       xv[0] = h0.x * r * w0.x; xv[1] = h0.y * r * w0.y; xv[2] = h0.z * r * w0.z; xv[3] = h0.w * r * w0.w;
       xv[4] = h1.x * r * w1.x; xv[5] = h1.y * r * w1.y; xv[6] = h1.z * r * w1.z; xv[7] = h1.w * r * w1.w;
     }
-    const uint32_t e_logit = base + 2u * (uint32_t)l + 1u, e_part = e_logit + 1u;
     // stage x: 8 consecutive threads share one 64-group
-    {
-      float m = 0.f;
-#pragma unroll
-      for (int i = 0; i < 8; ++i) m = fmaxf(m, fabsf(xv[i]));
-      m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, 1));
-      m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, 2));
-      m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, 4));
-      const float inv = m > 0.f ? 32767.f / m : 0.f;
-      const float delta = m * (1.f / 32767.f);
-      int q[8], sum = 0;
-#pragma unroll
-      for (int i = 0; i < 8; ++i) {
-        int t = __float2int_rn(xv[i] * inv);
-        t = t > 32767 ? 32767 : (t < -32767 ? -32767 : t);
-        q[i] = t;
-        sum += t;
-      }
-      sum += __shfl_xor_sync(0xffffffffu, sum, 1);
-      sum += __shfl_xor_sync(0xffffffffu, sum, 2);
-      sum += __shfl_xor_sync(0xffffffffu, sum, 4);
-      if (xthr) {
-        const int g = tid >> 3, u = tid & 7;
-        sx.xs[u * ngH + g] = make_uint4((uint32_t)(q[0] & 0xFFFF) | ((uint32_t)q[1] << 16),
-                                        (uint32_t)(q[2] & 0xFFFF) | ((uint32_t)q[3] << 16),
-                                        (uint32_t)(q[4] & 0xFFFF) | ((uint32_t)q[5] << 16),
-                                        (uint32_t)(q[6] & 0xFFFF) | ((uint32_t)q[7] << 16));
-        if (u == 0) {
-          sx.delta[g] = delta;
-          sx.xsum[g] = delta * (float)sum;
-        }
-      }
-    }
+    stage_unit(xv, xthr, tid >> 3, tid & 7, ngH, sx);
     // router partial dot products, reduced in warp order
 #pragma unroll
     for (int m = 0; m < kFusedMaxRouterRows; ++m) {
@@ -666,204 +648,211 @@ __global__ void __launch_bounds__(kFusedThreads, 1) fused_stack_kernel(const __g
       if (lane == 0) s_rp[warp][m] = d;
     }
     __syncthreads();
-    if (tid < nr) {
-      float v = 0.f;
-      for (int w = 0; w < kFusedWarps; ++w) v += s_rp[w][tid];
-      const int row = c + tid * nC;
-      if (row < E) A.logits[row] = v;
-      else A.gamma[0] = v = 1.f / (1.f + expf(-v));
-      st_relaxed64(A.x_logit + row, x_word(e_logit, v));
+    if (warp == 0) {
+      if (tid < nr) {
+        float v = 0.f;
+        for (int w = 0; w < kFusedWarps; ++w) v += s_rp[w][tid];
+        const int row = c + tid * nC;
+        if (row < E) A.logits[row] = v;
+        else A.gamma[0] = v = 1.f / (1.f + expf(-v));
+        __stcg(A.x_logit + row, v);
+      }
+      __syncwarp();
+      if (lane == 0 && nr > 0) cnt_release_add(A.sync + kCntLogit, (unsigned)nr);
     }
-    const XGroup xg = load_xgroup(sx, ngH);
-    // ------------------------------------------------------------- C --
-    // while the other CTAs finish: this CTA's block of the shared expert
-    if (has_shared) {
-      if (!wait_mb(1) || !wait_mb(kMbSb + 0)) { aborted = true; break; }
-      const uint8_t* const sl[2] = {smem + P.slot[1], nullptr};
-      const uint32_t* const sb[2] = {reinterpret_cast<const uint32_t*>(smem + P.sbe[0]), nullptr};
-      const float wt[2] = {1.f, 0.f};
-      float* const ao[2] = {A.a + (size_t)k * I + (size_t)c * GS::kW, nullptr};
-      run_blocks<SBITS, 1>(sl, sb, H, xg, wt, ao, s_blk, ys);
-    }
-    // ------------------------------------------------------------- D --
-    {
-      // routing: every thread keys up to two logits; per-warp top-k, then one
-      // warp merges the warps' candidates
-      uint64_t key[2];
-      bool nan_seen = false;
-      float lv[2];
-      {
-        uint64_t lw[2], gw = 0;
-        bool ok = true;
-        if (tid == 0) gw = ld_relaxed64(A.x_logit + E);
-#pragma unroll
-        for (int i = 0; i < 2; ++i) {
-          const int e = tid + i * kFusedThreads;
-          lw[i] = e < E ? ld_relaxed64(A.x_logit + e) : 0;
-        }
-        {
-          uint64_t all3[3] = {lw[0], lw[1], gw};
-          ok = x_spin_all(all3, e_logit, [&](int i) { return A.x_logit + (i < 2 ? tid + i * kFusedThreads : E); },
-                          [&](int i) { return i < 2 ? tid + i * kFusedThreads < E : tid == 0; });
-          lw[0] = all3[0];
-          lw[1] = all3[1];
-          gw = all3[2];
-        }
-#pragma unroll
-        for (int i = 0; i < 2; ++i) lv[i] = __uint_as_float((uint32_t)lw[i]);
-        if (tid == 0) s_gamma = __uint_as_float((uint32_t)gw);
-        if (!x_agree(ok)) { aborted = true; break; }
-      }
-#pragma unroll
-      for (int i = 0; i < 2; ++i) {
-        const int e = tid + i * kFusedThreads;
-        key[i] = 0;
-        if (e < E) {
-          nan_seen |= isnan(lv[i]);
-          slog[e] = lv[i];
-          key[i] = route_key(lv[i], e);
-        }
-      }
-      const uint64_t wk = warp_select_keys<2>(key, k);
-      if (lane < k) cand[warp * k + lane] = wk;
-      nan_seen = __syncthreads_or(nan_seen);
-      if (warp == 0) {
-        uint64_t kk[4];
-#pragma unroll
-        for (int i = 0; i < 4; ++i) {
-          const int idx = lane + 32 * i;
-          kk[i] = idx < kFusedWarps * k ? cand[idx] : 0;
-        }
-        const uint64_t win = warp_select_keys<4>(kk, k);
-        const int sel = lane < k ? key_index(win) : 0;
-        const float val = lane < k ? slog[sel] : 0.f;
-        float m = -INFINITY;
-        for (int r = 0; r < k; ++r) {
-          const float vr = __shfl_sync(0xffffffffu, val, r);
-          if (!isnan(vr)) m = fmaxf(m, vr);
-        }
-        const float pe = (lane < k && !isnan(val)) ? expf(val - m) : 0.f;
-        const float z = warp_sum(pe);
-        if (lane < k) {
-          s_ids[lane] = sel;
-          s_p[lane] = z > 0.f ? pe / z : 0.f;
-          if (c == 0) {
-            A.ids[lane] = sel;
-            A.weights[lane] = s_p[lane];
-          }
-        }
-        if (c == 0 && lane == 0 && nan_seen) raise_status(FMOE_STATUS_NAN_LOGIT);
-      }
-      __syncthreads();
-    }
-    // requests: the first routed blocks into the slots, the down scale-bias
-    // of their (at most two) 64-groups, L2 prefetches of the remaining
-    // blocks and of the next layer's router rows and shared block.  A routed
-    // block q (= j * NBr + nb) lies in 64-group q / kPerGroup of the
-    // concatenated experts.
-    // Jobs are spread over the warps' lane 0 so they go out in parallel:
-    // block b < kSlots <- warp b, entry e <- warp kSlots + e, L2 prefetch of
-    // the blocks b >= kSlots <- the following warps.
-    const int key0 = q0 / GR::kPerGroup, key1 = (q1 - 1) / GR::kPerGroup;
-    const int ngI = I / 64;
-    if (lane == 0) {
-      if (warp < kFirstWave) {
-        if (warp < nq) {
-          const int q = q0 + warp;
-          fence_proxy_async();
-          issue_block(warp, LY.experts + (size_t)s_ids[q / NBr] * LR.bytes, LR, q % NBr, GR::gu_sb(H));
-        }
-      } else if (warp >= kSlots && warp < kSlots + kSbEntries) {
-        const int e = warp - kSlots;
-        if (nq > 0 && (e == 0 || key1 != key0)) {
-          const int key = e == 0 ? key0 : key1;
-          fence_proxy_async();
-          issue_sb(e, LY.experts + (size_t)s_ids[key / ngI] * LR.bytes, LR, key % ngI);
-        }
-      }
-    }
-    // the second wave (the other slots, L2 prefetch of the later blocks) goes
-    // out once the first wave has landed, so that the first blocks are not
-    // slowed by requests for the later ones
-    auto second_wave = [&]() {
-      if (lane != 0) return;
-      if (warp >= kFirstWave && warp < kSlots) {
-        if (warp < nq) {
-          const int q = q0 + warp;
-          fence_proxy_async();
-          issue_block(warp, LY.experts + (size_t)s_ids[q / NBr] * LR.bytes, LR, q % NBr, GR::gu_sb(H));
-        }
-      } else if (warp >= kSlots + kSbEntries) {
-        for (int b = kSlots + (warp - kSlots - kSbEntries); b < nq; b += kFusedWarps - kSlots - kSbEntries) {
-          const int q = q0 + b;
-          prefetch_block(LY.experts + (size_t)s_ids[q / NBr] * LR.bytes, LR, q % NBr, GR::gu_sb(H));
-        }
-      }
-    };
     // ------------------------------------------------------------- E --
-    // routed blocks two at a time (block b in slot b % kSlots); a freed slot
-    // takes block b + kSlots at once
-    {
-      unsigned sb_ready = 0;  // bit e: entry e waited for in this layer
-      for (int b = 0; b < nq; b += 2) {
-        const int nb_round = nq - b >= 2 ? 2 : 1;
-        const uint8_t* sl[2] = {nullptr, nullptr};
-        const uint32_t* sb[2] = {nullptr, nullptr};
-        float wt[2] = {0.f, 0.f};
-        float* ao[2] = {nullptr, nullptr};
-#pragma unroll
-        for (int n = 0; n < 2; ++n) {
-          if (n >= nb_round) break;
-          const int q = q0 + b + n, j = q / NBr, nbk = q % NBr;
-          const int s = (b + n) % kSlots, e = q / GR::kPerGroup == key0 ? 0 : 1;
-          if (!wait_mb(s)) { aborted = true; break; }
-          if (!(sb_ready & (1u << e))) {
-            if (!wait_mb(kMbSb + e)) { aborted = true; break; }
-            sb_ready |= 1u << e;
-          }
-          sl[n] = smem + P.slot[s];
-          sb[n] = reinterpret_cast<const uint32_t*>(smem + P.sbe[e]);
-          wt[n] = s_p[j];
-          ao[n] = A.a + (size_t)j * I + (size_t)nbk * GR::kW;
+    if (warp < kGuWarps) {
+      // ---- gate/up warps ----
+      const XGroup xg = load_xgroup(sx, ngH);
+      for (int p = 0; p < nseq; ++p) {
+        const uint32_t pos = sq + (uint32_t)p;
+        const int s = (int)(pos % kSlots);
+        const bool ok = wait_mb(kMbFull + s, (pos / kSlots) & 1u);
+        float* gb = gred + (pos & 1u) * (kGuWarps * 8);
+        const uint8_t* sl = smem + P.slot[s];
+        if (ok) {
+          if (p < S) block_gateup<SBITS>(sl, H, xg, gb);
+          else block_gateup<BITS>(sl, H, xg, gb);
         }
-        if (aborted) break;
-        if (b == 0) second_wave();
-        const uint8_t* const slc[2] = {sl[0], sl[1]};
-        const uint32_t* const sbc[2] = {sb[0], sb[1]};
-        const float wtc[2] = {wt[0], wt[1]};
-        float* const aoc[2] = {ao[0], ao[1]};
-        if (nb_round == 2) run_blocks<BITS, 2>(slc, sbc, H, xg, wtc, aoc, s_blk, yr);
-        else run_blocks<BITS, 1>(slc, sbc, H, xg, wtc, aoc, s_blk, yr);
-        // the freed slots take their next blocks
-#pragma unroll
-        for (int n = 0; n < 2; ++n) {
-          if (n >= nb_round) break;
-          const int bb = b + n, s = bb % kSlots;
-          if (warp == s && lane == 0 && bb + kSlots < nq) {
-            const int q2 = q0 + bb + kSlots;
-            fence_proxy_async();
-            issue_block(s, LY.experts + (size_t)s_ids[q2 / NBr] * LR.bytes, LR, q2 % NBr, GR::gu_sb(H));
+        named_bar(kBarGu, kGuThreads);
+        if (warp == 0) {
+          uint32_t* dx = dnx + s * kDnxWords;
+          if (p < S) block_swiglu<SBITS>(gb, dx, A.a + (size_t)k * I + (size_t)c * GS::kW);
+          else
+            block_swiglu<BITS>(gb, dx,
+                               A.a + (size_t)jj * I + (size_t)((jg % ngI) * GR::kPerGroup + rb0 + p - S) * GR::kW);
+          __syncwarp();
+          if (lane == 0) mbar_arrive(&mbar[kMbReady + s]);
+        }
+      }
+    } else {
+      // ---- down warps: routing first ----
+      const int td = tid - kGuThreads, dw = warp - kGuWarps;
+      {
+        // every CTA has published its router rows: (l + 1) (E + 1) in all
+        if (issuer) {
+          if (!cnt_wait(A.sync + kCntLogit, (unsigned)(l + 1) * (unsigned)(E + 1)) && !s_abort) {
+            s_abort = 1;
+            raise_status(FMOE_STATUS_WAIT_TIMEOUT);
           }
         }
-        // once the first round is done, the next layer's router rows and
-        // shared block may compete for HBM
-        if (b == 0 && warp == kFusedWarps - 1 && lane == 0 && l + 1 < A.n_layers) prefetch_next(l + 1);
-      }
-      if (aborted) break;
-      if (nq == 0 && warp == kFusedWarps - 1 && lane == 0 && l + 1 < A.n_layers) prefetch_next(l + 1);
-    }
-    // every slot and entry is consumed: the next layer's shared block can come in
-    if (lane == 0 && l + 1 < A.n_layers) issue_shared(l + 1);
-    // ------------------------------------------------------------- F --
-    {
-      const float gm = s_gamma;
-      uint64_t* part = A.x_part + (size_t)c * H;
+        named_bar(kBarDn, kDnThreads);
+        float lw[kDnKeys];
 #pragma unroll
-      for (int m = 0; m < kFusedRowsPerThread; ++m) {
-        const int i = tid + m * kFusedThreads;
-        if (i < H) st_relaxed64(part + i, x_word(e_part, fmaf(gm, ys[m], yr[m])));
+        for (int i = 0; i < kDnKeys; ++i) {
+          const int e = td + i * kDnThreads;
+          lw[i] = e < E ? __ldcg(A.x_logit + e) : 0.f;
+        }
+        if (td == 0) s_gamma = __ldcg(A.x_logit + E);
+        uint64_t key[kDnKeys];
+        bool nan_seen = false;
+#pragma unroll
+        for (int i = 0; i < kDnKeys; ++i) {
+          const int e = td + i * kDnThreads;
+          key[i] = 0;
+          if (e < E) {
+            const float v = lw[i];
+            nan_seen |= isnan(v);
+            slog[e] = v;
+            key[i] = route_key(v, e);
+          }
+        }
+        const uint64_t wk = warp_select_keys<kDnKeys>(key, k);
+        if (lane < k) cand[dw * k + lane] = wk;
+        nan_seen = __any_sync(0xffffffffu, nan_seen);
+        if (lane == 0 && nan_seen) cand[kDnWarps * kFusedMaxK] = 1;  // flag word after the candidates
+        named_bar(kBarDn, kDnThreads);
+        if (dw == 0) {
+          uint64_t kk[2];
+#pragma unroll
+          for (int i = 0; i < 2; ++i) {
+            const int idx = lane + 32 * i;
+            kk[i] = idx < kDnWarps * k ? cand[idx] : 0;
+          }
+          const uint64_t win = warp_select_keys<2>(kk, k);
+          const int sel = lane < k ? key_index(win) : 0;
+          const float val = lane < k ? slog[sel] : 0.f;
+          float m = -INFINITY;
+          for (int r = 0; r < k; ++r) {
+            const float vr = __shfl_sync(0xffffffffu, val, r);
+            if (!isnan(vr)) m = fmaxf(m, vr);
+          }
+          const float pe = (lane < k && !isnan(val)) ? expf(val - m) : 0.f;
+          const float z = warp_sum(pe);
+          if (lane < k) {
+            s_ids[lane] = sel;
+            s_p[lane] = z > 0.f ? pe / z : 0.f;
+            if (c == 0) {
+              A.ids[lane] = sel;
+              A.weights[lane] = s_p[lane];
+            }
+          }
+          if (c == 0 && lane == 0 && cand[kDnWarps * kFusedMaxK] != 0) raise_status(FMOE_STATUS_NAN_LOGIT);
+          __syncwarp();
+          if (lane == 0) {
+            cand[kDnWarps * kFusedMaxK] = 0;
+            // requests: the routed blocks that have a free slot, their down
+            // scale-bias entry, and L2 prefetches of the later ones
+            if (!s_abort) {
+              for (int p = S; p < nseq && p < kSlots; ++p) issue_pos(l, sq, p);
+              if (nq > 0) issue_sb(1, LY.experts + (size_t)s_ids[jj] * LR.bytes, LR, gr);
+              for (int p = kSlots; p < nseq; ++p)
+                prefetch_block(LY.experts + (size_t)s_ids[jj] * LR.bytes, LR, (jg % ngI) * GR::kPerGroup + rb0 + p - S,
+                               GR::gu_sb(H));
+              // the next layer's shared block, when its slot is already free
+              if (S && l + 1 < A.n_layers && nseq < kSlots) issue_pos(l + 1, sq + (uint32_t)nseq, 0);
+            }
+          }
+        }
+        named_bar(kBarDn, kDnThreads);
       }
+      // ---- down products, block by block ----
+#pragma unroll
+      for (int m = 0; m < kDnRowsT; ++m) yacc[m] = 0.f;
+      float uacc[kDnRowsT];  // routed blocks: sum of step * weight * value, scaled per row at the end
+#pragma unroll
+      for (int m = 0; m < kDnRowsT; ++m) uacc[m] = 0.f;
+      float p2sum = 0.f;  // routed blocks: sum of step * weight * sum xi (times the row's bias at the end)
+      const float wt_r = s_p[jj], wt_s = s_gamma;
+      for (int p = 0; p < nseq; ++p) {
+        const uint32_t pos = sq + (uint32_t)p;
+        const int s = (int)(pos % kSlots);
+        bool ok = wait_mb(kMbReady + s, (pos / kSlots) & 1u);
+        ok = ok && wait_mb(kMbFull + s, (pos / kSlots) & 1u);
+        if (p == 0 && S) ok = ok && wait_mb(kMbSbShared, (uint32_t)l & 1u);
+        // this CTA's last block has landed: the next layer's router rows may compete for HBM
+        if (issuer && p == nseq - 1 && l + 1 < A.n_layers) prefetch_router(l + 1);
+        if (ok) {
+          const uint8_t* sl = smem + P.slot[s];
+          const uint32_t* dx = dnx + s * kDnxWords;
+          float t[kDnRowsT];
+          if (p < S) {
+            block_down<SBITS>(sl, dx, H, t);
+            const float p1 = wt_s * __uint_as_float(dx[12]), p2 = wt_s * __uint_as_float(dx[13]);
+            const uint32_t* sbe = reinterpret_cast<const uint32_t*>(smem + P.sbe[0]);
+#pragma unroll
+            for (int m = 0; m < kDnQuads; ++m) {
+              const int row = 4 * (td + kDnThreads * m);
+              if (row < H) {
+                const uint4 sb = lds128(sbe + row);
+                const uint32_t sw[4] = {sb.x, sb.y, sb.z, sb.w};
+#pragma unroll
+                for (int r = 0; r < 4; ++r) {
+                  const float sc = __uint_as_float(sw[r] << 16), bi = __uint_as_float(sw[r] & 0xFFFF0000u);
+                  yacc[4 * m + r] = fmaf(sc, p1 * t[4 * m + r], fmaf(bi, p2, yacc[4 * m + r]));
+                }
+              }
+            }
+          } else {
+            block_down<BITS>(sl, dx, H, t);
+            const float p1 = wt_r * __uint_as_float(dx[12]);
+            p2sum = fmaf(wt_r, __uint_as_float(dx[13]), p2sum);
+#pragma unroll
+            for (int m = 0; m < kDnRowsT; ++m) uacc[m] = fmaf(p1, t[m], uacc[m]);
+          }
+        }
+        named_bar(kBarDn, kDnThreads);  // every down thread is done with the slot
+        if (issuer && !s_abort) {
+          // the slot takes the block three positions on: this layer's, or
+          // the next layer's shared block
+          const int pn = p + kSlots;
+          if (pn < nseq) issue_pos(l, sq, pn);
+          else if (pn == nseq && S && l + 1 < A.n_layers) issue_pos(l + 1, sq + (uint32_t)nseq, 0);
+          // the shared entry is free: the next layer's comes in
+          if (p == 0 && S && l + 1 < A.n_layers) issue_sb(0, A.layers[l + 1].shared, LS, c / GS::kPerGroup);
+        }
+      }
+      if (nseq == 0 && issuer && l + 1 < A.n_layers) prefetch_router(l + 1);
+      // ---- F: routed blocks scaled per row, partial output out ----
+      bool ok = true;
+      if (nq > 0) ok = wait_mb(kMbSbRouted, (uint32_t)l & 1u);
+      const uint32_t* sbe = reinterpret_cast<const uint32_t*>(smem + P.sbe[1]);
+      float* part = A.x_part + (size_t)c * H;
+#pragma unroll
+      for (int m = 0; m < kDnQuads; ++m) {
+        const int row = 4 * (td + kDnThreads * m);
+        if (row < H) {
+          float v[4];
+          if (nq > 0 && ok) {
+            const uint4 sb = lds128(sbe + row);
+            const uint32_t sw[4] = {sb.x, sb.y, sb.z, sb.w};
+#pragma unroll
+            for (int r = 0; r < 4; ++r) {
+              const float sc = __uint_as_float(sw[r] << 16), bi = __uint_as_float(sw[r] & 0xFFFF0000u);
+              v[r] = fmaf(sc, uacc[4 * m + r], fmaf(bi, p2sum, yacc[4 * m + r]));
+            }
+          } else {
+#pragma unroll
+            for (int r = 0; r < 4; ++r) v[r] = yacc[4 * m + r];
+          }
+          __stcg(reinterpret_cast<float4*>(part + row), make_float4(v[0], v[1], v[2], v[3]));
+        }
+      }
+      named_bar(kBarDn, kDnThreads);
+      if (issuer) cnt_release_add(A.sync + kCntPart, 1u);
     }
+    sq += (uint32_t)nseq;
+    if (__syncthreads_or(s_abort)) { aborted = true; break; }
     // ------------------------------------------------------------- G --
     {
       // rows i0 + r, r < nd: ngr threads per row each sum every ngr-th CTA's
@@ -871,58 +860,66 @@ __global__ void __launch_bounds__(kFusedThreads, 1) fused_stack_kernel(const __g
       const int ngr = nd > 0 ? kFusedThreads / nd : 0;
       const int r = nd > 0 ? tid % nd : 0, pg = nd > 0 ? tid / nd : kFusedThreads;
       const float hres = tid < nd ? A.h[i0 + tid] : 0.f;  // this CTA's own rows
-      bool ok = true;
+      if (!cta_cnt_wait(kCntPart, (unsigned)(l + 1) * (unsigned)nC)) { aborted = true; break; }
       if (pg < ngr) {
         constexpr int kLoads = (kFusedMaxCtas * 32 + kFusedThreads - 1) / kFusedThreads;  // ngr >= 512 / 32
-        uint64_t v[kLoads];
+        float v[kLoads];
 #pragma unroll
         for (int t2 = 0; t2 < kLoads; ++t2) {
           const int p = pg + t2 * ngr;
-          v[t2] = p < nC ? ld_relaxed64(A.x_part + (size_t)p * H + i0 + r) : x_word(e_part, 0.f);
+          v[t2] = p < nC ? __ldcg(A.x_part + (size_t)p * H + i0 + r) : 0.f;
         }
-        ok = x_spin_all(v, e_part, [&](int t2) { return A.x_part + (size_t)(pg + t2 * ngr) * H + i0 + r; },
-                        [&](int t2) { return pg + t2 * ngr < nC; });
         float acc = 0.f;
 #pragma unroll
-        for (int t2 = 0; t2 < kLoads; ++t2) acc += __uint_as_float((uint32_t)v[t2]);
+        for (int t2 = 0; t2 < kLoads; ++t2) acc += v[t2];
         sred[pg * nd + r] = acc;
       }
-      if (!x_agree(ok)) { aborted = true; break; }
+      __syncthreads();
       float ss = 0.f;
       if (tid < nd) {
         float v = hres;
         for (int g = 0; g < ngr; ++g) v += sred[g * nd + tid];
         A.h[i0 + tid] = v;
+        __stcg(A.x_h + i0 + tid, v);
         ss = v * v;
       }
       if (warp == 0) {
         ss = warp_sum(ss);
-        if (lane == 0) A.ss_part[c] = ss;
+        if (lane == 0) __stcg(A.x_ss + c, ss);
       }
+      __syncthreads();
+      if (tid == 0) cnt_release_add(A.sync + kCntH, 1u);
     }
-    grid_arrive();  // h' and the partial sums written
   }
 
-  if (!aborted && A.n_layers > 0 && grid_wait()) {
+  // after the last layer: every CTA's h' rows and sum of squares are written
+  bool done = !aborted && A.n_layers > 0;
+  if (done) done = cta_cnt_wait(kCntH, (unsigned)A.n_layers * (unsigned)nC);
+  if (done) {
     // epilogue: xn' of the last layer for this CTA's rows (h' written by this thread)
-    const float r_last = norm_scale();
+    const float r_last = norm_scale(tid < nC ? __ldcg(A.x_ss + tid) : 0.f);
     const float* w = A.layers[A.n_layers - 1].norm_w;
     if (tid < nd) A.xn[i0 + tid] = A.h[i0 + tid] * r_last * w[i0 + tid];
     __syncthreads();
     if (tid == 0) {
       __threadfence();
-      const unsigned prev = atomicAdd(&A.sync[1], 1u);
-      if (prev == (unsigned)nC - 1) {  // every CTA has read the epoch base and is past its last exchange
-        A.sync[2] = base + 2u * (uint32_t)A.n_layers + 2u;
-        A.sync[0] = 0;
-        A.sync[1] = 0;
+      const unsigned prev = atomicAdd(&A.sync[kCntExit], 1u);
+      if (prev == (unsigned)nC - 1) {  // every CTA is past its last counter wait
+        A.sync[kCntH] = 0;
+        A.sync[kCntLogit] = 0;
+        A.sync[kCntPart] = 0;
+        A.sync[kCntExit] = 0;
         __threadfence();
       }
     }
-  } else if (lane == 0) {
-    // drain: wait (bounded) for this issuer's copies still in flight
+  }
+  if (issuer) {
+    // drain: wait (bounded) for this issuer's copies still in flight -- the
+    // last phase armed on each barrier (earlier phases have completed: a
+    // slot or entry is re-armed only after its previous contents were used).
+    // On a clean exit these phases have completed already.
     for (int mb = 0; mb < kMbCount; ++mb)
-      if (armed & (1u << mb)) (void)mbar_wait(&mbar[mb], (phase >> mb) & 1u);
+      if (armed & (1u << mb)) (void)mbar_wait(&mbar[mb], ((next_par >> mb) & 1u) ^ 1u);
   }
 }
 
@@ -930,16 +927,14 @@ __global__ void __launch_bounds__(kFusedThreads, 1) fused_stack_kernel(const __g
 // does not fit the kernel.
 inline bool fused_plan(int H, int I, int E, int k, int bits, int sbits, int n_ctas, size_t max_smem,
                        FusedPlan* out) {
-  if (H < 64 || H % 64 || I < 64 || I % 64 || H > kFusedThreads * kFusedRowsPerThread) return false;
-  if (E < 1 || E > 2 * kFusedThreads || k < 1 || k > kFusedMaxK || k > E) return false;
+  if (H < 64 || H % 64 || I < 64 || I % 64 || H > kFusedMaxH) return false;
+  if (E < 1 || E > kFusedMaxE || k < 1 || k > kFusedMaxK || k > E) return false;
   if (n_ctas < 1 || n_ctas > kFusedMaxCtas) return false;
   if (E + 1 > kFusedMaxRouterRows * n_ctas) return false;
   auto wn = [](int b) { return 32 / b; };
-  const int nbr = I / wn(bits), nbs = I / wn(sbits);
-  if (nbs > n_ctas) return false;  // one shared block per CTA at most
-  // routed blocks per CTA; a CTA's run spans at most two 64-groups
-  const int per_cta = (k * nbr + n_ctas - 1) / n_ctas;
-  if (per_cta > kFusedMaxRouted || per_cta > 64 / wn(bits) + 1) return false;
+  const int nbs = I / wn(sbits);
+  if (nbs > n_ctas) return false;        // one shared block per CTA at most
+  if (k * (I / 64) > n_ctas) return false;  // one routed 64-group per CTA at most
   if ((H + n_ctas - 1) / n_ctas > 32) return false;  // rows per CTA in the final sums: one warp
   auto blk = [&](int b) -> long long { return 12LL * H + (long long)wn(b) * 2 * (H / 64) * 4; };
   const long long slot = blk(bits) > blk(sbits) ? blk(bits) : blk(sbits);
@@ -950,7 +945,7 @@ inline bool fused_plan(int H, int I, int E, int k, int bits, int sbits, int n_ct
     p.slot[s] = (uint32_t)o;
     o = al(o + slot);
   }
-  for (int e = 0; e < kSbEntries; ++e) {
+  for (int e = 0; e < 2; ++e) {
     p.sbe[e] = (uint32_t)o;
     o = al(o + 4LL * H);
   }
@@ -959,7 +954,11 @@ inline bool fused_plan(int H, int I, int E, int k, int bits, int sbits, int n_ct
   p.logit = (uint32_t)o;
   o = al(o + 4LL * E);
   p.cand = (uint32_t)o;
-  o = al(o + 8LL * kFusedWarps * kFusedMaxK);
+  o = al(o + 8LL * (kDnWarps * kFusedMaxK + 1));
+  p.gred = (uint32_t)o;
+  o = al(o + 4LL * 2 * kGuWarps * 8);
+  p.dnx = (uint32_t)o;
+  o = al(o + 4LL * kSlots * kDnxWords);
   p.red = (uint32_t)o;
   o = al(o + 4LL * kFusedThreads);
   p.mbar = (uint32_t)o;

@@ -213,10 +213,11 @@ __device__ __forceinline__ void gateup_rows(const uint8_t* rec, const ExpertSet&
       const uint32_t sg = ld_stream_u32(sbw + (size_t)(2 * n) * ng + g);
       const uint32_t su = ld_stream_u32(sbw + (size_t)(2 * n + 1) * ng + g);
       uint4 xv[8];
-      load_xv(sx, ng, g, xv);
+      uint2 xl[8];
+      load_xv(sx, ng, g, xv, xl);
       const float d = sx.delta[g], xs = sx.xsum[g];
-      yg = group_epilogue(yg, sg, group_dot<BITS>(cg, xv), d, xs);
-      yu = group_epilogue(yu, su, group_dot<BITS>(cu, xv), d, xs);
+      yg = group_epilogue(yg, sg, group_dot<BITS>(cg, xv, xl), d, xs);
+      yu = group_epilogue(yu, su, group_dot<BITS>(cu, xv, xl), d, xs);
     }
     for (int o = lpr >> 1; o > 0; o >>= 1) {
       yg += __shfl_xor_sync(0xffffffffu, yg, o);
@@ -245,11 +246,13 @@ __device__ __forceinline__ float down_row_cols(const uint8_t* rec, const ExpertS
 #pragma unroll
     for (int b = 0; b < kWpg; ++b) w[b] = ld_stream_u32(codes + (size_t)(g * kWpg + b) * H);
     const uint32_t sb = ld_stream_u32(sbw + (size_t)g * H);
-    int acc = 0;
+    Acc2 acc{0, 0};
 #pragma unroll
     for (int b = 0; b < kWpg; ++b) {
-      if (BITS == 4) acc += word_dot4(w[b], sx.xs[b * ngI + g]);
-      else acc += word_dot2(w[b], sx.xs[(2 * b) * ngI + g], sx.xs[(2 * b + 1) * ngI + g]);
+      if (BITS == 4) acc = acc + word_dot4(w[b], sx.xs[b * ngI + g], sx.xl[b * ngI + g]);
+      else
+        acc = acc + word_dot2(w[b], sx.xs[(2 * b) * ngI + g], sx.xs[(2 * b + 1) * ngI + g], sx.xl[(2 * b) * ngI + g],
+                              sx.xl[(2 * b + 1) * ngI + g]);
     }
     y = group_epilogue(y, sb, acc, sx.delta[g], sx.xsum[g]);
   }
@@ -557,9 +560,10 @@ __global__ void pack_sb_kernel(const uint16_t* __restrict__ scale, const uint16_
 
 // ------------------------------------------------------- host helpers ----
 struct WsLayout {
-  size_t sync, ss, x_logit, x_part, grp, part, logits, ids, weights, gamma, a, y, bytes;
+  size_t sync, x_logit, x_ss, x_h, x_part, grp, part, logits, ids, weights, gamma, a, y, bytes;
   size_t g_count, g_offset, g_slots, g_nitems, g_items, g_bitems, g_tc, g_xs;  // inside grp
   size_t tcx, tca;  // staged fp16 inputs of the tensor-core items (0 bytes when T < kTcMinTokens)
+  size_t tsc, rsc, amax;  // their staging scales (tokens, staged rows) and rows' max |a|
 };
 
 // Upper bound of the tensor-core items' token rows (sum of tokens rounded up to 8).
@@ -570,18 +574,21 @@ static size_t tc_np_bound(int T, int k) {
 
 static inline size_t align_up(size_t v, size_t a) { return (v + a - 1) / a * a; }
 
-constexpr int kMaxSMs = 1024;
-
 static WsLayout ws_layout(int H, int I, int E, int k, int T) {
   WsLayout w;
-  w.sync = 0;    // grid-barrier counter, exit counter and epoch of the fused kernel
-  w.ss = 4096;   // per-CTA partial sums of h'^2 of the fused kernel
-  size_t o = 4096 + (size_t)kMaxSMs * 4;
-  // exchange words of the fused kernel (8 bytes each)
+  w.sync = 0;  // grid-barrier counter, exit counter and epoch of the fused kernel
+  // exchange buffers of the fused kernel (fp32), at offsets and sizes that
+  // do not depend on the shape or T (its counters, at the start, decide
+  // when their contents are current)
+  size_t o = 4096;
   w.x_logit = o;
-  o = align_up(o + (size_t)(E + 1) * 8, 256);
+  o = align_up(o + (size_t)(kFusedMaxE + 1) * 4, 256);
+  w.x_ss = o;
+  o = align_up(o + (size_t)kFusedMaxCtas * 4, 256);
+  w.x_h = o;
+  o = align_up(o + (size_t)kFusedMaxH * 4, 256);
   w.x_part = o;
-  o = align_up(o + (size_t)kFusedMaxCtas * H * 8, 256);
+  o = align_up(o + (size_t)kFusedMaxCtas * kFusedMaxH * 4, 256);
   // expert groups of the T > 1 path
   w.grp = o;
   w.g_count = o;
@@ -604,6 +611,12 @@ static WsLayout ws_layout(int H, int I, int E, int k, int T) {
   o = align_up(o + tc_np_bound(T, k) * 4 * H, 256);
   w.tca = o;
   o = align_up(o + tc_np_bound(T, k) * 4 * I, 256);
+  w.tsc = o;
+  o = align_up(o + (size_t)T * 4, 256);
+  w.rsc = o;
+  o = align_up(o + tc_np_bound(T, k) * 4, 256);
+  w.amax = o;
+  o = align_up(o + tc_np_bound(T, k) * 4, 256);
   w.part = o;
   o = align_up(o + (size_t)T * (E + 1) * kRouterSplit * 4, 256);
   w.logits = o;
@@ -771,7 +784,7 @@ static int launch_experts(const ExpertSet& es, const float* xn, const int32_t* i
                       smem_optin(reinterpret_cast<const void*>(&tc_gemm_kernel<1>), tc_smem_bytes(), 3);
       const int max_tc = group_max_tc(T, es.k, kTcMinTokens);
       group_kernel<<<1, 1024, grp_smem, st>>>(ids, T, es.k, es.E, es.I, es.H, tc ? kTcMinTokens : 0, *gw, a, y);
-      stage_tokens_kernel<<<T, kGrpThreads, 0, st>>>(xn, es.H, xs, sxs);
+      stage_tokens_kernel<<<T, kGrpThreads, 0, st>>>(xn, es.H, xs, sxs, tc ? gw->tscale : nullptr);
       // a bucket's grid covers at most the items it can hold (the kernels
       // index the bucket lists with the full stride `items`)
       int nb[kGrpBuckets];
@@ -792,11 +805,12 @@ static int launch_experts(const ExpertSet& es, const float* xn, const int32_t* i
       if (nb[2]) grp_launch_gu<8>(es, *gw, 2, items, nb[2], xn, xs, a, w_sg, gamma, sxs, st);
       if (nb[3]) grp_launch_gu<16>(es, *gw, 3, items, nb[3], xn, xs, a, w_sg, gamma, sxs, st);
       if (tc) {
+        const TcScale sc{gw->rscale, gw->amax};
         tc_stage_kernel<<<dim3(max_tc, es.H / 64), kTcThreads, 0, st>>>(*gw, xn, es.H, es.k + 1, 0, tcx, es.E, w_sg,
-                                                                      gamma);
+                                                                      gamma, gw->tscale, sc);
         const int n_sm = device_sms();
         const int u0 = max_tc * (2 * es.I / kTcRows);
-        tc_gemm_kernel<0><<<u0 < n_sm ? u0 : n_sm, kTcThreads + 32, tc_smem_bytes(), st>>>(es, *gw, tcx, a);
+        tc_gemm_kernel<0><<<u0 < n_sm ? u0 : n_sm, kTcThreads + 32, tc_smem_bytes(), st>>>(es, *gw, tcx, a, sc);
       }
       if (small_only) {
         down_group_small_kernel<<<dim3(nb[0] + nb[1], (es.H + kDnRows - 1) / kDnRows), kDnRows, 4 * sas, st>>>(
@@ -808,11 +822,12 @@ static int launch_experts(const ExpertSet& es, const float* xn, const int32_t* i
       if (nb[2]) grp_launch_dn<8>(es, *gw, 2, items, nb[2], a, y, sas, st);
       if (nb[3]) grp_launch_dn<16>(es, *gw, 3, items, nb[3], a, y, sas, st);
       if (tc) {
+        const TcScale sc{gw->rscale, gw->amax};
         tc_stage_kernel<<<dim3(max_tc, es.I / 64), kTcThreads, 0, st>>>(*gw, a, es.I, es.k + 1, 1, tca, es.E, nullptr,
-                                                                      nullptr);
+                                                                      nullptr, nullptr, sc);
         const int n_sm = device_sms();
         const int u1 = max_tc * (es.H / kTcRows);
-        tc_gemm_kernel<1><<<u1 < n_sm ? u1 : n_sm, kTcThreads + 32, tc_smem_bytes(), st>>>(es, *gw, tca, y);
+        tc_gemm_kernel<1><<<u1 < n_sm ? u1 : n_sm, kTcThreads + 32, tc_smem_bytes(), st>>>(es, *gw, tca, y, sc);
       }
       return cuda_rc(cudaGetLastError());
     }
@@ -942,9 +957,10 @@ static int launch_fused(const fmoe_layer_weights* layers, int n_layers, float* h
   args.weights = reinterpret_cast<float*>(base + w.weights) + (size_t)t * d.top_k;
   args.gamma = reinterpret_cast<float*>(base + w.gamma) + t;
   args.a = reinterpret_cast<float*>(base + w.a) + (size_t)t * (d.top_k + 1) * d.inter;
-  args.x_logit = reinterpret_cast<uint64_t*>(base + w.x_logit);
-  args.x_part = reinterpret_cast<uint64_t*>(base + w.x_part);
-  args.ss_part = reinterpret_cast<float*>(base + w.ss);
+  args.x_logit = reinterpret_cast<float*>(base + w.x_logit);
+  args.x_h = reinterpret_cast<float*>(base + w.x_h);
+  args.x_ss = reinterpret_cast<float*>(base + w.x_ss);
+  args.x_part = reinterpret_cast<float*>(base + w.x_part);
   args.sync = reinterpret_cast<unsigned*>(base + w.sync);
   args.plan = fc.plan;
   for (int l0 = 0; l0 < n_layers; l0 += kFusedMaxLayers) {
@@ -984,6 +1000,9 @@ static GroupWork group_work(unsigned char* base, const WsLayout& w) {
   g.items = reinterpret_cast<int4*>(base + w.g_items);
   g.bitems = reinterpret_cast<int4*>(base + w.g_bitems);
   g.tc = reinterpret_cast<int4*>(base + w.g_tc);
+  g.tscale = reinterpret_cast<float*>(base + w.tsc);
+  g.rscale = reinterpret_cast<float*>(base + w.rsc);
+  g.amax = reinterpret_cast<unsigned*>(base + w.amax);
   return g;
 }
 

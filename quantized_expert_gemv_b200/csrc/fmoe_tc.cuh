@@ -94,6 +94,14 @@ __device__ __forceinline__ uint32_t pack_h2(float a, float b) {
 
 __host__ __device__ __forceinline__ int tc_np(int m) { return (m + 7) / 8 * 8; }
 
+// Per staged row of the tensor-core items: the multiplier that undoes the
+// row's staging scale in the epilogue, and (gate/up products) the largest
+// |a| of the row, from which the down products' staging takes its scale.
+struct TcScale {
+  float* rscale;  // [rows]
+  unsigned* amax;  // [rows], fp32 bits of max |a|
+};
+
 // ------------------------------------------------------- token staging --
 // Stages the inputs of every tensor-core item in fp16 hi / lo core matrices:
 // per 64-input step, rows 0 .. Np-1 the hi parts of the item's tokens, rows
@@ -105,12 +113,23 @@ __host__ __device__ __forceinline__ int tc_np(int m) { return (m + 7) / 8 * 8; }
 // With mode 0 the CTAs also compute gamma for the shared expert's tokens.
 __global__ void __launch_bounds__(kTcThreads)
 tc_stage_kernel(GroupWork w, const float* __restrict__ src, int K, int k1, int mode, uint8_t* __restrict__ dst,
-                int E, const float* __restrict__ w_sg, float* __restrict__ gamma) {
+                int E, const float* __restrict__ w_sg, float* __restrict__ gamma, const float* __restrict__ tscale,
+                TcScale sc) {
   if ((int)blockIdx.x >= w.n_items[1]) return;
   const int4 it = w.tc[blockIdx.x];
   const int g = it.x, m = it.z, np = tc_np(m), s = blockIdx.y;
   const int* slots = w.slots + w.offset[g] + it.y;
   uint8_t* base = dst + (size_t)it.w * 4 * K + (size_t)s * (2 * np) * 128;
+  // row scales: mode 0 the token's (stage_tokens_kernel), mode 1 from the
+  // gate/up products' max |a| of the row; the first step's CTA records the
+  // epilogue multipliers and (mode 0) clears the rows' max |a|
+  if (s == 0) {
+    for (int r = threadIdx.x; r < m; r += blockDim.x) {
+      const float f = mode == 0 ? tscale[slots[r] / k1] : tc_row_scale(__uint_as_float(sc.amax[it.w + r]));
+      sc.rscale[it.w + r] = 1.f / f;
+      if (mode == 0) sc.amax[it.w + r] = 0u;
+    }
+  }
   for (int u = threadIdx.x; u < 2 * np * 8; u += blockDim.x) {
     const int row = u >> 3, kc = u & 7;  // 8 inputs 8 kc .. 8 kc + 7 of row `row`
     const int tok = row < np ? row : row - np;
@@ -118,9 +137,10 @@ tc_stage_kernel(GroupWork w, const float* __restrict__ src, int K, int k1, int m
     if (tok < m) {
       const int slot = slots[tok];
       const float* v = src + (size_t)(mode == 0 ? slot / k1 : slot) * K + s * 64 + kc * 8;
+      const float rs = mode == 0 ? tscale[slot / k1] : tc_row_scale(__uint_as_float(sc.amax[it.w + tok]));
       const float4 a = __ldg(reinterpret_cast<const float4*>(v));
       const float4 b = __ldg(reinterpret_cast<const float4*>(v + 4));
-      float f[8] = {a.x, a.y, a.z, a.w, b.x, b.y, b.z, b.w};
+      float f[8] = {a.x * rs, a.y * rs, a.z * rs, a.w * rs, b.x * rs, b.y * rs, b.z * rs, b.w * rs};
       if (row >= np) {
 #pragma unroll
         for (int i = 0; i < 8; ++i) f[i] = f[i] - __half2float(__float2half_rn(f[i]));
@@ -343,9 +363,6 @@ __device__ __forceinline__ void tc_dequant(const TcRaw& w, uint8_t* a_tile, int 
 }
 
 // ------------------------------------------------------------- the GEMM --
-__device__ __forceinline__ void mbar_arrive(uint64_t* bar) {
-  asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(smem_u32(bar)) : "memory");
-}
 
 // One work unit (item it, row tile r0) of tc_gemm_kernel.  MODE 0: gate/up
 // (M = 2 I, K = H), epilogue SwiGLU -> a[slot][n].  MODE 1: down (M = H,
@@ -365,7 +382,7 @@ template <int MODE, int BITS>
 __device__ __forceinline__ void tc_gemm_body(const ExpertSet& es, const int4 it, const uint8_t* rec, int r0, int gb,
                                              const uint8_t* __restrict__ staged, float* __restrict__ out,
                                              unsigned char* tsm, uint64_t* bar_b, uint64_t* bar_m, uint64_t* bar_f,
-                                             uint32_t tmem, const int* s_slot, int* s_ok) {
+                                             uint32_t tmem, const int* s_slot, int* s_ok, TcScale sc) {
   const int m = it.z, np = tc_np(m), N = 2 * np;
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int K = MODE == 0 ? es.H : es.I;
@@ -474,10 +491,14 @@ __device__ __forceinline__ void tc_gemm_body(const ExpertSet& es, const int4 it,
 #pragma unroll
       for (int i = 0; i < 8; ++i) {
         const int t = ch * 8 + i;
-        const float v = hi[i] + lo[i];
+        const float v = (hi[i] + lo[i]) * (t < m ? sc.rscale[it.w + t] : 0.f);
         if (MODE == 0) {
           const float partner = __shfl_xor_sync(0xffffffffu, v, 1);  // gate row 2n, up row 2n + 1
-          if ((lane & 1) == 0 && t < m) out[(size_t)s_slot[t] * es.I + (r0 + row) / 2] = silu_mul(v, partner);
+          if ((lane & 1) == 0 && t < m) {
+            const float av = silu_mul(v, partner);
+            out[(size_t)s_slot[t] * es.I + (r0 + row) / 2] = av;
+            atomicMax(&sc.amax[it.w + t], __float_as_uint(fabsf(av)));
+          }
         } else if (t < m) {
           out[(size_t)s_slot[t] * es.H + r0 + row] = v;
         }
@@ -493,7 +514,7 @@ __device__ __forceinline__ void tc_gemm_body(const ExpertSet& es, const int4 it,
 // from unit to unit (steps % 4 == 0 keeps every ring stage in step).
 template <int MODE>
 __global__ void __launch_bounds__(kTcThreads + 32, 1)
-tc_gemm_kernel(ExpertSet es, GroupWork w, const uint8_t* __restrict__ staged, float* __restrict__ out) {
+tc_gemm_kernel(ExpertSet es, GroupWork w, const uint8_t* __restrict__ staged, float* __restrict__ out, TcScale sc) {
   extern __shared__ __align__(1024) unsigned char tsm[];
   __shared__ uint64_t bar_b[kTcBStages], bar_m[kTcStages], bar_f[kTcStages];
   __shared__ uint32_t s_tmem;
@@ -533,8 +554,8 @@ tc_gemm_kernel(ExpertSet es, GroupWork w, const uint8_t* __restrict__ staged, fl
     __syncthreads();
     int bits;
     const uint8_t* rec = group_record(es, g, &bits);
-    if (bits == 4) tc_gemm_body<MODE, 4>(es, it, rec, r0, gb, staged, out, tsm, bar_b, bar_m, bar_f, tmem, s_slot, &s_ok);
-    else tc_gemm_body<MODE, 2>(es, it, rec, r0, gb, staged, out, tsm, bar_b, bar_m, bar_f, tmem, s_slot, &s_ok);
+    if (bits == 4) tc_gemm_body<MODE, 4>(es, it, rec, r0, gb, staged, out, tsm, bar_b, bar_m, bar_f, tmem, s_slot, &s_ok, sc);
+    else tc_gemm_body<MODE, 2>(es, it, rec, r0, gb, staged, out, tsm, bar_b, bar_m, bar_f, tmem, s_slot, &s_ok, sc);
     // the epilogue's tensor-memory reads and s_slot uses end before the next unit
     tc_fence_before();
     const bool go = __syncthreads_and(s_ok != 0);

@@ -5,6 +5,9 @@ element by element, S being the oracle's error scale (the sum of absolute
 terms behind v, propagated through the later steps), and the relative L2
 error ||d - v|| / ||v|| is at most 2e-3.
 """
+import concurrent.futures
+import os
+
 import numpy as np
 
 REL = 1e-3
@@ -31,3 +34,11 @@ def check(d, v, S, what: str, rel_l2: bool = True):
             r = np.linalg.norm(d - v) / nv
             assert r <= REL_L2, f"{what}: relative L2 {r:.3g} > {REL_L2}"
     return float((err / tol).max()) if err.size else 0.0
+
+
+def pmap(fn, items):
+    """Runs fn over items on host threads (the oracle's C calls release the
+    interpreter lock) and re-raises the first failure."""
+    items = list(items)
+    with concurrent.futures.ThreadPoolExecutor(max_workers=min(16, os.cpu_count() or 4)) as ex:
+        return list(ex.map(fn, items))

@@ -80,3 +80,28 @@ def test_noalloc_rejects_tokens_beyond_scratch(small_layer):
         fm.fmoe_layer_forward_noalloc(lw, h, xn)
     assert e.value.status == fm.FMOE_ERR_BUFFER_TOO_SMALL
     assert not h.any() and not xn.any()
+
+
+def test_noalloc_scratch_shared_across_shapes():
+    """One scratch array serves every shape: a many-token call of a small
+    layer (whose grouping data land where a larger layer's persistent
+    kernel keeps its exchange words, were those placed by shape) followed by
+    a single-token call of a larger layer must give the bits of that call on
+    a fresh workspace."""
+    if not torch.cuda.is_available():
+        pytest.skip("no CUDA device")
+    small = upload_layer(SMALL, 0)
+    big_wl = synth.Workload(hidden=1024, inter=512, n_experts=64)
+    big = upload_layer(big_wl, 0)
+    assert fm.fmoe_fused_supported(big.desc)
+    fm.fmoe_read_status(clear=True)
+    xs = synth.tokens(SMALL, 8, stream=75)
+    h, xn = torch.from_numpy(xs).cuda(), torch.from_numpy(xs).cuda()
+    fm.fmoe_layer_forward_noalloc(small, h, xn)  # T = 8: the grouped path
+    xb = synth.tokens(big_wl, 1, stream=76)
+    ws = fm.alloc_workspace(big.desc, 1)
+    ref = _two_calls(lambda h, xn: fm.fmoe_layer_forward(big, h, xn, ws), xb)
+    got = _two_calls(lambda h, xn: fm.fmoe_layer_forward_noalloc(big, h, xn), xb)
+    for i in range(2):
+        assert np.array_equal(got[i][0], ref[i][0]) and np.array_equal(got[i][1], ref[i][1]), i
+    assert fm.fmoe_read_status() == 0
