@@ -20,15 +20,25 @@ import numpy as np
 
 _HERE = os.path.dirname(os.path.abspath(__file__))
 _LIB_PATH = os.path.join(_HERE, "liboracle.so")
+_OMP_LIB_PATH = os.path.join(_HERE, "liboracle_omp.so")  # timing build: output rows over threads
 
 
-def build(force: bool = False) -> str:
+def _build_one(path: str, extra, force: bool) -> str:
     src = os.path.join(_HERE, "oracle.c")
-    if force or not os.path.exists(_LIB_PATH) or os.path.getmtime(_LIB_PATH) < os.path.getmtime(src):
+    if force or not os.path.exists(path) or os.path.getmtime(path) < os.path.getmtime(src):
         subprocess.check_call(["gcc", "-O2", "-fPIC", "-shared", "-std=c11", "-fno-fast-math",
-                               "-ffp-contract=off", src, "-lm", "-o", _LIB_PATH + ".tmp"])
-        os.replace(_LIB_PATH + ".tmp", _LIB_PATH)
-    return _LIB_PATH
+                               "-ffp-contract=off", *extra, src, "-lm", "-o", path + ".tmp"])
+        os.replace(path + ".tmp", path)
+    return path
+
+
+def build(force: bool = False, omp: bool = False) -> str:
+    """Builds the plain oracle (the checks use it); with omp, also the
+    timing build whose matrix-vector rows run on OpenMP threads."""
+    path = _build_one(_LIB_PATH, [], force)
+    if omp:
+        _build_one(_OMP_LIB_PATH, ["-fopenmp", "-DORACLE_OMP"], force)
+    return path
 
 
 class _Expert(ctypes.Structure):
@@ -43,13 +53,34 @@ class _Layer(ctypes.Structure):
 
 
 _lib = None
+_libs = {}
+
+
+def set_threads(n: int) -> int:
+    """Timing only (the benchmark's CPU baseline): n > 1 switches every call
+    below to the OpenMP build on n threads, n <= 1 back to the plain build.
+    Both compute the same values.  Returns the threads in use."""
+    global _lib
+    if n <= 1:
+        _lib = _load(_LIB_PATH)
+        return 1
+    build(omp=True)
+    _lib = _load(_OMP_LIB_PATH)
+    _lib.oracle_set_threads(int(n))
+    return int(n)
 
 
 def lib() -> ctypes.CDLL:
     global _lib
     if _lib is None:
         build()
-        L = ctypes.CDLL(_LIB_PATH)
+        _lib = _load(_LIB_PATH)
+    return _lib
+
+
+def _load(path: str) -> ctypes.CDLL:
+    if path not in _libs:
+        L = ctypes.CDLL(path)
         vp, i32, dbl = ctypes.c_void_p, ctypes.c_int, ctypes.c_double
         L.oracle_bf16.restype = dbl
         L.oracle_bf16.argtypes = [ctypes.c_uint16]
@@ -75,8 +106,11 @@ def lib() -> ctypes.CDLL:
         L.oracle_quantize_f32.restype = None
         L.oracle_dequantize.argtypes = [vp, vp, vp, i32, i32, i32, vp]
         L.oracle_dequantize.restype = None
-        _lib = L
-    return _lib
+        if path == _OMP_LIB_PATH:
+            L.oracle_set_threads.argtypes = [i32]
+            L.oracle_set_threads.restype = None
+        _libs[path] = L
+    return _libs[path]
 
 
 def _c(a, dtype):

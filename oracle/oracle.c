@@ -36,6 +36,19 @@
 #include <stdint.h>
 #include <string.h>
 
+/* Timing build only (ORACLE_OMP, used by the benchmark's CPU baseline on all
+ * host cores): the independent output rows of the matrix-vector products
+ * are spread over threads.  Each row is still computed by one thread in the
+ * same order, so the results are those of the plain build bit for bit.  The
+ * checks use the plain build. */
+#ifdef ORACLE_OMP
+#include <omp.h>
+#define ORACLE_ROWS_PARALLEL _Pragma("omp parallel for schedule(static)")
+void oracle_set_threads(int n) { omp_set_num_threads(n); }
+#else
+#define ORACLE_ROWS_PARALLEL
+#endif
+
 /* Exact value of a bf16 bit pattern (bf16 is the top half of an IEEE fp32). */
 double oracle_bf16(uint16_t h) {
   uint32_t u = (uint32_t)h << 16;
@@ -52,6 +65,7 @@ double oracle_bf16(uint16_t h) {
 void oracle_qgemv(const uint8_t* q, const uint16_t* s, const uint16_t* b, int rows, int cols,
                   int G, const double* x, double* y, double* S) {
   int ng = cols / G;
+  ORACLE_ROWS_PARALLEL
   for (int r = 0; r < rows; ++r) {
     double acc = 0.0, mag = 0.0;
     for (int j = 0; j < cols; ++j) {
@@ -69,6 +83,7 @@ void oracle_qgemv(const uint8_t* q, const uint16_t* s, const uint16_t* b, int ro
  * Mixture-of-Experts" -- a router picks experts per layer) and the shared
  * expert's gate logit.  y[r] = sum_j W[r][j] x[j], S[r] = sum_j |W[r][j] x[j]|. */
 void oracle_gemv_f32(const float* W, int rows, int cols, const double* x, double* y, double* S) {
+  ORACLE_ROWS_PARALLEL
   for (int r = 0; r < rows; ++r) {
     double acc = 0.0, mag = 0.0;
     for (int j = 0; j < cols; ++j) {
@@ -157,6 +172,7 @@ void oracle_expert_ffn(const oracle_expert_t* ex, int H, int I, int G, const dou
   oracle_qgemv(qd, sd, bd, H, I, G, a, y, S_y);
   /* add |Wd| S_a: the down product sees a with its own error */
   int ngd = I / G;
+  ORACLE_ROWS_PARALLEL
   for (int r = 0; r < H; ++r) {
     double prop = 0.0;
     for (int j = 0; j < I; ++j) {

@@ -22,10 +22,10 @@
 //          routed blocks' copies; then for every block the down columns of
 //          all H rows (each thread 16 rows), weighted by the block's gate
 //          weight; a finished block's slot takes the next block at once
-//   F  the CTA's partial output for all H rows -> exchange words
-//   G  (all warps) each CTA sums the partials of its slice of rows in a fixed
-//      order, adds the residual -> h' and its part of sum(h'^2), published as
-//      exchange words for the next layer's A
+//   F  the CTA's partial output for all H rows -> the workspace
+//   G  (all warps) each CTA sums the partials of its slice of rows in a
+//      fixed order (deterministic), adds the residual -> h' and its part of
+//      sum(h'^2), published for the next layer's A
 // The shared block does not depend on the routing: it is fetched during the
 // previous layer and its gate/up products run while the logits travel, so
 // the routed data, which cannot be requested before the top-k, has the
@@ -39,15 +39,21 @@
 // submission there plays the role the persistent kernel plays here: no host
 // round trip between the steps or between layers).
 //
-// Exchanges between CTAs (logits, partial outputs, h' with its sums of
-// squares): the writers store fp32 values, then one release-add per CTA
-// (per writing warp for the logits) on a counter of that exchange; in each
-// reading CTA one thread polls the counter with acquire loads (a short sleep
-// between polls keeps the polling traffic off the lines being written) until
-// it reaches the layer's target, and after a CTA-local barrier every thread
-// reads the values.  The counters grow over the launch's layers and the
-// last CTA to leave returns them to zero.  Every wait (mbarrier,
-// counter) is bounded: on expiry the CTA sets
+// Exchanges between CTAs.  Router logits (E + 1 words, read whole by every
+// CTA): exchange words, (epoch << 32) | fp32 bits, written and read as
+// single 64-bit accesses, so a reader that sees the epoch it waits for holds
+// the value that came with it -- no fence on either side; each writing warp
+// adds to a relaxed counter after its stores, one thread per reading CTA
+// polls that counter with a short sleep between polls (polling words that
+// are still being written would slow the writers down), and only then are
+// the words read (re-read, with a sleep, while a store has not landed: the
+// counter is a hint, the epochs decide).  Partial outputs and h' (with its
+// sums of squares): fp32 with coalesced stores, then one release-add per
+// CTA on the exchange's counter; one thread per reading CTA polls it with
+// acquire loads, and after a CTA-local barrier the threads read the values
+// with 16-byte L2 loads where the layout allows.  The counters grow over the
+// launch's layers; the last CTA to leave returns them to zero.  Every wait
+// (mbarrier, counter, exchange word) is bounded: on expiry the CTA sets
 // FMOE_STATUS_WAIT_TIMEOUT, records the abort in shared memory (later waits
 // return at once, every warp still passes every named barrier), waits
 // (bounded) for its own copies in flight, and returns.
@@ -83,15 +89,18 @@ constexpr int kMbFull = 0;                 // [kSlots] a slot's bytes have lande
 constexpr int kMbReady = kMbFull + kSlots;  // [kSlots] a slot's SwiGLU outputs are staged
 constexpr int kMbSbShared = kMbReady + kSlots;
 constexpr int kMbSbRouted = kMbSbShared + 1;
-constexpr int kMbCount = kMbSbRouted + 1;
+constexpr int kMbRouter = kMbSbRouted + 1;  // the layer's router rows have landed
+constexpr int kMbCount = kMbRouter + 1;
 constexpr int kBarGu = 1, kBarDn = 2;       // named barriers of the two warp groups
 constexpr long long kWaitCycles = 4000000000LL;  // ~2 s at 2 GHz
 // exchange counters (words of the workspace's counter area)
 constexpr int kCntH = 0;      // CTAs that published h' and their sum of squares (all layers so far)
 constexpr int kCntExit = 1;   // CTAs that left the kernel
+constexpr int kEpoch = 2;     // epoch of the last launch (router-logit exchange words)
 constexpr int kCntLogit = 3;  // router logits published
 constexpr int kCntPart = 4;   // CTAs that published their partial outputs
-constexpr unsigned kPollSleepNs = 32;
+constexpr unsigned kPollSleepNs = 32;    // between polls of a counter
+constexpr unsigned kRepollSleepNs = 64;  // between re-reads of an exchange word
 
 struct FusedLayer {
   const uint8_t* experts;
@@ -130,11 +139,11 @@ struct FusedArgs {
   float* weights;
   float* gamma;
   float* a;           // [(k+1)][I], shared expert last
-  float* x_logit;     // [E + 1]: router logits, then sigmoid(w_sg . xn)
-  float* x_h;         // [H]: h' of the layer
-  float* x_ss;        // [gridDim.x]: per-CTA sums of h'^2
-  float* x_part;      // [gridDim.x][H]: partial outputs
-  unsigned* sync;     // counters: kCntH, kCntExit, kCntLogit, kCntPart
+  uint64_t* x_logit;  // [E + 1]: router logits, then sigmoid(w_sg . xn) (exchange words)
+  float* x_h;      // [H]: h' of the layer
+  float* x_ss;     // [gridDim.x]: per-CTA sums of h'^2
+  float* x_part;   // [gridDim.x][H]: partial outputs
+  unsigned* sync;  // counters kCntH, kCntExit, kCntLogit, kCntPart; logit epoch base kEpoch
   FusedPlan plan;
 };
 
@@ -210,15 +219,59 @@ __device__ __forceinline__ void cnt_release_add(unsigned* p, unsigned v) {
   asm volatile("red.release.gpu.global.add.u32 [%0], %1;" ::"l"(p), "r"(v) : "memory");
 }
 
-// Bounded poll (one thread) until *p >= target; false on expiry.
+// Bounded poll (one thread) until *p >= target, with acquire semantics when
+// ACQ; false on expiry.
+template <bool ACQ = false>
 __device__ __forceinline__ bool cnt_wait(const unsigned* p, unsigned target) {
   const long long t0 = clock64();
   while (true) {
     unsigned v;
-    asm volatile("ld.acquire.gpu.global.u32 %0, [%1];" : "=r"(v) : "l"(p) : "memory");
+    if (ACQ) asm volatile("ld.acquire.gpu.global.u32 %0, [%1];" : "=r"(v) : "l"(p) : "memory");
+    else asm volatile("ld.relaxed.gpu.global.u32 %0, [%1];" : "=r"(v) : "l"(p) : "memory");
     if ((int)(v - target) >= 0) return true;
     if (clock64() - t0 > kWaitCycles) return false;
     __nanosleep(kPollSleepNs);
+  }
+}
+
+__device__ __forceinline__ uint64_t ld_relaxed64(const uint64_t* p) {
+  uint64_t v;
+  asm volatile("ld.relaxed.gpu.global.b64 %0, [%1];" : "=l"(v) : "l"(p) : "memory");
+  return v;
+}
+
+__device__ __forceinline__ void st_relaxed64(uint64_t* p, uint64_t v) {
+  asm volatile("st.relaxed.gpu.global.b64 [%0], %1;" ::"l"(p), "l"(v) : "memory");
+}
+
+__device__ __forceinline__ void cnt_add(unsigned* p, unsigned v) {
+  asm volatile("red.relaxed.gpu.global.add.u32 [%0], %1;" ::"l"(p), "r"(v) : "memory");
+}
+
+__device__ __forceinline__ uint64_t x_word(uint32_t epoch, float v) {
+  return ((uint64_t)epoch << 32) | __float_as_uint(v);
+}
+
+__device__ __forceinline__ bool x_ready(uint64_t w, uint32_t epoch) { return (uint32_t)(w >> 32) == epoch; }
+
+__device__ __forceinline__ float x_value(uint64_t w) { return __uint_as_float((uint32_t)w); }
+
+// N exchange words at p(i) (those with valid(i)), already read once into w:
+// re-reads the ones that do not carry `epoch` yet, with a sleep between
+// rounds (bounded); false on expiry.
+template <int N, class Addr, class Valid>
+__device__ __forceinline__ bool x_settle(uint64_t (&w)[N], uint32_t epoch, Addr p, Valid valid) {
+  const long long t0 = clock64();
+  while (true) {
+    bool miss = false;
+#pragma unroll
+    for (int i = 0; i < N; ++i) miss |= valid(i) && !x_ready(w[i], epoch);
+    if (!miss) return true;
+    if (clock64() - t0 > kWaitCycles) return false;
+    __nanosleep(kRepollSleepNs);
+#pragma unroll
+    for (int i = 0; i < N; ++i)
+      if (valid(i) && !x_ready(w[i], epoch)) w[i] = ld_relaxed64(p(i));
   }
 }
 
@@ -264,17 +317,30 @@ __device__ __forceinline__ int key_index(uint64_t key) { return (int)(0xFFFFFFFF
 template <int PER>
 __device__ __forceinline__ uint64_t warp_select_keys(uint64_t* key, int k) {
   const int lane = threadIdx.x & 31;
+  // each lane sorts its keys (largest first): a round looks at the heads only
+  auto cs = [&](int i, int j) {
+    const uint64_t a = key[i], b = key[j];
+    key[i] = a > b ? a : b;
+    key[j] = a > b ? b : a;
+  };
+  if (PER >= 2) cs(0, 1);
+  if (PER == 4) {
+    cs(2, 3);
+    cs(0, 2);
+    cs(1, 3);
+    cs(1, 2);
+  }
   uint64_t mine = 0;
   for (int r = 0; r < k; ++r) {
-    uint64_t best = key[0];
-#pragma unroll
-    for (int i = 1; i < PER; ++i) best = key[i] > best ? key[i] : best;
+    const uint64_t best = key[0];
     const uint32_t hi = __reduce_max_sync(0xffffffffu, (uint32_t)(best >> 32));
     const uint32_t lo = __reduce_max_sync(0xffffffffu, (uint32_t)(best >> 32) == hi ? (uint32_t)best : 0u);
     const uint64_t win = ((uint64_t)hi << 32) | lo;
+    if (best == win) {  // keys are unique (the index is part of the key): the winning lane drops its head
 #pragma unroll
-    for (int i = 0; i < PER; ++i)
-      if (key[i] == win) key[i] = 0;
+      for (int i = 0; i + 1 < PER; ++i) key[i] = key[i + 1];
+      key[PER - 1] = 0;
+    }
     if (lane == r) mine = win;
   }
   return mine;
@@ -374,11 +440,11 @@ __device__ __forceinline__ void block_gateup(const uint8_t* slot, int H, const X
 }
 
 // SwiGLU of one block from the gate/up sums (gate/up warp 0): lane p < w
-// forms a_p; the w outputs get one power-of-two step (24-bit block floating
-// point) and go to dnx (high parts, low parts, step, step * sum) for the
-// down warps, and to a_out (global).
+// forms a_p (returned); the w outputs get one power-of-two step (24-bit
+// block floating point) and go to dnx (high parts, low parts, step,
+// step * sum) for the down warps.
 template <int B>
-__device__ __forceinline__ void block_swiglu(const float* gred, uint32_t* dnx, float* a_out) {
+__device__ __forceinline__ float block_swiglu(const float* gred, uint32_t* dnx) {
   using G = BlockGeo<B>;
   constexpr int kW = G::kW;
   const int lane = threadIdx.x & 31;
@@ -388,7 +454,6 @@ __device__ __forceinline__ void block_swiglu(const float* gred, uint32_t* dnx, f
     const float gs = gred[(2 * ps) * 8 + 2 * i] + gred[(2 * ps + 1) * 8 + 2 * i];
     const float us = gred[(2 * ps) * 8 + 2 * i + 1] + gred[(2 * ps + 1) * 8 + 2 * i + 1];
     a = silu_mul(gs, us);
-    a_out[lane] = a;
   }
   const float m = __uint_as_float(__reduce_max_sync(0xffffffffu, __float_as_uint(fabsf(a))));
   float inv, delta;
@@ -406,6 +471,7 @@ __device__ __forceinline__ void block_swiglu(const float* gred, uint32_t* dnx, f
     dnx[12] = __float_as_uint(delta);
     dnx[13] = __float_as_uint(delta * (float)qsum);
   }
+  return a;
 }
 
 // Down part of one block (down threads): for the thread's row quads, the
@@ -442,12 +508,11 @@ __global__ void __launch_bounds__(kFusedThreads, 1) fused_stack_kernel(const __g
   using GR = BlockGeo<BITS>;
   using GS = BlockGeo<SBITS>;
   extern __shared__ __align__(128) unsigned char smem[];
-  __shared__ int s_ids[kFusedMaxK];
-  __shared__ float s_p[kFusedMaxK];
   __shared__ float s_gamma;
   __shared__ float s_rp[kFusedWarps][kFusedMaxRouterRows];
   __shared__ float s_red[kFusedWarps];
   __shared__ volatile int s_abort;
+  __shared__ int s_nan;
 
   const int c = blockIdx.x, nC = gridDim.x;
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
@@ -460,7 +525,6 @@ __global__ void __launch_bounds__(kFusedThreads, 1) fused_stack_kernel(const __g
   uint64_t* cand = reinterpret_cast<uint64_t*>(smem + P.cand);
   float* gred = reinterpret_cast<float*>(smem + P.gred);
   uint32_t* dnx = reinterpret_cast<uint32_t*>(smem + P.dnx);
-  float* sred = reinterpret_cast<float*>(smem + P.red);
 
   // ---- static work of this CTA ----
   const int nr = c <= E ? (E - c) / nC + 1 : 0;  // router rows c, c + nC, ... <= E (row E: shared gate)
@@ -479,29 +543,35 @@ __global__ void __launch_bounds__(kFusedThreads, 1) fused_stack_kernel(const __g
   const int nseq = S + nq;  // blocks per layer: the shared one first
   int i0, i1;
   share(H, c, nC, &i0, &i1);  // hidden rows of the final sums
-  const int nd = i1 - i0;
   const RecordLayout LR = record_layout(BITS, H, I);
   const RecordLayout LS = record_layout(SBITS, H, I);
   const bool xthr = tid * 8 < H;  // this thread holds inputs 8 tid .. 8 tid + 7
-  const bool issuer = tid == kGuThreads;  // lane 0 of the first down warp issues every copy
+  const int td = tid - kGuThreads, dw = warp - kGuWarps;  // down threads: index and warp in the group
+  const bool issuer = tid == kGuThreads;  // the first down thread: counters and polls of the down warps
+  // copies: lane 0 of down warp s issues slot s (s < kSlots), down warps
+  // kWarpSb, kWarpSb + 1 the two scale-bias entries, kWarpRt the router
+  // rows, the warps after them the L2 prefetches -- one owner per mbarrier,
+  // owners in different warps
+  constexpr int kWarpSb = kSlots, kWarpRt = kSlots + 2, kWarpPf = kSlots + 3;
+  const bool owner = dw >= 0 && lane == 0;
 
   if (tid == 0) {
     for (int i = 0; i < kMbCount; ++i) mbar_init(&mbar[i], 1);
     s_abort = 0;
-    cand[kDnWarps * kFusedMaxK] = 0;  // NaN-logit flag of the top-k
+    s_nan = 0;
     asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
   }
   __syncthreads();
 
-  // issuer: mbarriers it has armed, and per mbarrier the parity of the next
-  // phase it will arm (each phase of a copy barrier is armed once, by it)
+  // owner lane: mbarriers it has armed, and per mbarrier the parity of the
+  // next phase it will arm (each phase of a copy barrier is armed once, by it)
   uint32_t armed = 0, next_par = 0;
   auto arm = [&](int mb, uint32_t bytes) {
     mbar_expect_tx(&mbar[mb], bytes);
     armed |= 1u << mb;
     next_par ^= 1u << mb;
   };
-  // column block nb of the record `rec` into slot s
+  // column block nb of the record `rec` into slot s (slot s's owner)
   auto issue_block = [&](int s, const uint8_t* rec, const RecordLayout& L, int nb, uint32_t gu_sb_bytes) {
     uint8_t* dst = smem + P.slot[s];
     const uint32_t gub = 8u * (uint32_t)H, dnb = 4u * (uint32_t)H;
@@ -517,30 +587,39 @@ __global__ void __launch_bounds__(kFusedThreads, 1) fused_stack_kernel(const __g
     prefetch_l2(rec + L.down_codes + (size_t)nb * dnb, dnb);
     prefetch_l2(rec + L.gu_sb + (size_t)nb * gu_sb_bytes, gu_sb_bytes);
   };
-  // down scale-bias words of 64-group g of a record into entry e
+  // down scale-bias words of 64-group g of a record into entry e (its owner)
   auto issue_sb = [&](int e, const uint8_t* rec, const RecordLayout& L, int g) {
     fence_proxy_async();
     arm(kMbSbShared + e, 4u * (uint32_t)H);
     bulk_g2s(smem + P.sbe[e], rec + L.down_sb + (size_t)g * H * 4, 4u * (uint32_t)H, &mbar[kMbSbShared + e]);
   };
-  // block at position p of layer l (p < nseq; positions of the next layer
-  // are not requested here) into its slot
-  auto issue_pos = [&](int l, uint32_t sq, int p) {
+  auto routed_nb = [&](int p) { return gr * GR::kPerGroup + rb0 + p - S; };  // block of position p >= S
+  // block at position p of layer l into its slot, by the slot's owner; rid:
+  // the selected expert of this CTA's routed group
+  auto issue_pos = [&](int l, uint32_t sq, int p, int rid) {
     const int s = (int)((sq + (uint32_t)p) % kSlots);
-    if (p < S) {
-      issue_block(s, A.layers[l].shared, LS, c, GS::gu_sb(H));
-    } else {
-      const int b = p - S;
-      issue_block(s, A.layers[l].experts + (size_t)s_ids[jj] * LR.bytes, LR, (jg % ngI) * GR::kPerGroup + rb0 + b,
-                  GR::gu_sb(H));
-    }
+    if (!owner || dw != s) return;
+    if (p < S) issue_block(s, A.layers[l].shared, LS, c, GS::gu_sb(H));
+    else issue_block(s, A.layers[l].experts + (size_t)rid * LR.bytes, LR, routed_nb(p), GR::gu_sb(H));
   };
-  // L2 prefetch of layer l's router rows
-  auto prefetch_router = [&](int l) {
+  // Layer l's router rows (rows c + m nC, row E: the shared gate vector) into
+  // the two slots that do not hold the layer's first block (sq_l: its first
+  // position): rows 0-2 in one, row 3 in the other.  Issued once every block
+  // before the layer is done; read in the layer's phase A, before the top-k
+  // requests the routed blocks into those slots.
+  auto router_row_at = [&](uint32_t sq_l, int m) -> float* {
+    const int s = (int)((sq_l + 1u + (m >= 3 ? 1u : 0u)) % kSlots);
+    return reinterpret_cast<float*>(smem + P.slot[s]) + (size_t)(m % 3) * H;
+  };
+  auto issue_router = [&](int l, uint32_t sq_l) {
+    if (!owner || dw != kWarpRt || nr == 0) return;
     const FusedLayer& NX = A.layers[l];
+    fence_proxy_async();
+    arm(kMbRouter, 4u * (uint32_t)H * (uint32_t)nr);
     for (int m = 0; m < nr; ++m) {
       const int row = c + m * nC;
-      prefetch_l2(row < E ? NX.w_router + (size_t)row * H : NX.w_sg, 4u * (uint32_t)H);
+      bulk_g2s(router_row_at(sq_l, m), row < E ? NX.w_router + (size_t)row * H : NX.w_sg, 4u * (uint32_t)H,
+               &mbar[kMbRouter]);
     }
   };
 
@@ -560,10 +639,16 @@ __global__ void __launch_bounds__(kFusedThreads, 1) fused_stack_kernel(const __g
     }
     return false;
   };
-  // CTA-wide wait for an exchange counter (thread 0 polls)
+  auto set_abort = [&]() {
+    if (!s_abort) {
+      s_abort = 1;
+      raise_status(FMOE_STATUS_WAIT_TIMEOUT);
+    }
+  };
+  // CTA-wide wait for a counter (thread 0 polls, with acquire loads)
   auto cta_cnt_wait = [&](int which, unsigned target) -> bool {
     bool ok = true;
-    if (tid == 0) ok = cnt_wait(A.sync + which, target);
+    if (tid == 0) ok = cnt_wait<true>(A.sync + which, target);
     if (__syncthreads_and(ok && !s_abort)) return true;
     if (tid == 0) raise_status(FMOE_STATUS_WAIT_TIMEOUT);
     return false;
@@ -571,8 +656,7 @@ __global__ void __launch_bounds__(kFusedThreads, 1) fused_stack_kernel(const __g
   // r = (sum of the CTAs' partial sums of h'^2 / H + eps)^(-1/2), summed in
   // the same order in every CTA; ssv: this thread's partial (tid < nC)
   auto norm_scale = [&](float ssv) -> float {
-    float v = tid < nC ? ssv : 0.f;
-    v = warp_sum(v);
+    float v = warp_sum(tid < nC ? ssv : 0.f);
     if (lane == 0) s_red[warp] = v;
     __syncthreads();
     float t = 0.f;
@@ -582,31 +666,20 @@ __global__ void __launch_bounds__(kFusedThreads, 1) fused_stack_kernel(const __g
     return 1.f / sqrtf(t / (float)H + A.eps);
   };
 
-  uint32_t sq = 0;                           // blocks of earlier layers (slot of position p: (sq + p) % 3)
-  // the first layer's shared block and its down scale-bias entry
-  if (issuer && A.n_layers > 0 && S) {
-    issue_pos(0, 0u, 0);
-    issue_sb(0, A.layers[0].shared, LS, c / GS::kPerGroup);
+  const uint32_t base = __ldcg(A.sync + kEpoch);  // logit epoch of layer l: base + l + 1
+  uint32_t sq = 0;  // blocks of earlier layers (slot of position p: (sq + p) % 3)
+  // the first layer's shared block, its down scale-bias entry and router rows
+  if (A.n_layers > 0 && S) {
+    issue_pos(0, 0u, 0, 0);
+    if (owner && dw == kWarpSb) issue_sb(0, A.layers[0].shared, LS, c / GS::kPerGroup);
   }
+  if (A.n_layers > 0) issue_router(0, 0u);
 
-  float yacc[kDnRowsT];  // down threads: this CTA's partial output rows
   bool aborted = false;
   for (int l = 0; l < A.n_layers; ++l) {
     const FusedLayer& LY = A.layers[l];
+    const uint32_t e_logit = base + (uint32_t)l + 1u;
     // ------------------------------------------------------------- A --
-    // router rows (requested before anything they do not depend on)
-    float4 wr[kFusedMaxRouterRows][2];
-#pragma unroll
-    for (int m = 0; m < kFusedMaxRouterRows; ++m) {
-      const int row = c + m * nC;
-      if (m < nr && xthr) {
-        const float* src = (row < E ? LY.w_router + (size_t)row * H : LY.w_sg) + tid * 8;
-        wr[m][0] = as_float4(ld_stream(src));
-        wr[m][1] = as_float4(ld_stream(src + 4));
-      } else {
-        wr[m][0] = wr[m][1] = make_float4(0.f, 0.f, 0.f, 0.f);
-      }
-    }
     float xv[8];
     if (l == 0) {
       float4 v0 = make_float4(0.f, 0.f, 0.f, 0.f), v1 = v0;
@@ -633,17 +706,24 @@ __global__ void __launch_bounds__(kFusedThreads, 1) fused_stack_kernel(const __g
     }
     // stage x: 8 consecutive threads share one 64-group
     stage_unit(xv, xthr, tid >> 3, tid & 7, ngH, sx);
-    // router partial dot products, reduced in warp order
+    // router partial dot products (rows in shared memory), reduced in warp order
+    if (nr > 0 && !wait_mb(kMbRouter, (uint32_t)l & 1u)) set_abort();
 #pragma unroll
     for (int m = 0; m < kFusedMaxRouterRows; ++m) {
-      float d = wr[m][0].x * xv[0];
-      d = fmaf(wr[m][0].y, xv[1], d);
-      d = fmaf(wr[m][0].z, xv[2], d);
-      d = fmaf(wr[m][0].w, xv[3], d);
-      d = fmaf(wr[m][1].x, xv[4], d);
-      d = fmaf(wr[m][1].y, xv[5], d);
-      d = fmaf(wr[m][1].z, xv[6], d);
-      d = fmaf(wr[m][1].w, xv[7], d);
+      float4 wr[2] = {make_float4(0.f, 0.f, 0.f, 0.f), make_float4(0.f, 0.f, 0.f, 0.f)};
+      if (m < nr && xthr && !s_abort) {
+        const float* rr = router_row_at(sq, m) + tid * 8;
+        wr[0] = as_float4(lds128(rr));
+        wr[1] = as_float4(lds128(rr + 4));
+      }
+      float d = wr[0].x * xv[0];
+      d = fmaf(wr[0].y, xv[1], d);
+      d = fmaf(wr[0].z, xv[2], d);
+      d = fmaf(wr[0].w, xv[3], d);
+      d = fmaf(wr[1].x, xv[4], d);
+      d = fmaf(wr[1].y, xv[5], d);
+      d = fmaf(wr[1].z, xv[6], d);
+      d = fmaf(wr[1].w, xv[7], d);
       d = warp_sum(d);
       if (lane == 0) s_rp[warp][m] = d;
     }
@@ -655,10 +735,10 @@ __global__ void __launch_bounds__(kFusedThreads, 1) fused_stack_kernel(const __g
         const int row = c + tid * nC;
         if (row < E) A.logits[row] = v;
         else A.gamma[0] = v = 1.f / (1.f + expf(-v));
-        __stcg(A.x_logit + row, v);
+        st_relaxed64(A.x_logit + row, x_word(e_logit, v));
       }
       __syncwarp();
-      if (lane == 0 && nr > 0) cnt_release_add(A.sync + kCntLogit, (unsigned)nr);
+      if (lane == 0 && nr > 0) cnt_add(A.sync + kCntLogit, (unsigned)nr);
     }
     // ------------------------------------------------------------- E --
     if (warp < kGuWarps) {
@@ -677,33 +757,37 @@ __global__ void __launch_bounds__(kFusedThreads, 1) fused_stack_kernel(const __g
         named_bar(kBarGu, kGuThreads);
         if (warp == 0) {
           uint32_t* dx = dnx + s * kDnxWords;
-          if (p < S) block_swiglu<SBITS>(gb, dx, A.a + (size_t)k * I + (size_t)c * GS::kW);
-          else
-            block_swiglu<BITS>(gb, dx,
-                               A.a + (size_t)jj * I + (size_t)((jg % ngI) * GR::kPerGroup + rb0 + p - S) * GR::kW);
+          const float a = p < S ? block_swiglu<SBITS>(gb, dx) : block_swiglu<BITS>(gb, dx);
           __syncwarp();
           if (lane == 0) mbar_arrive(&mbar[kMbReady + s]);
+          // the SwiGLU outputs to the workspace, after the hand-off (a global
+          // store before the arrive would make it wait for the store)
+          if (p < S) {
+            if (lane < GS::kW) A.a[(size_t)k * I + (size_t)c * GS::kW + lane] = a;
+          } else if (lane < GR::kW) {
+            A.a[(size_t)jj * I + (size_t)routed_nb(p) * GR::kW + lane] = a;
+          }
         }
       }
     } else {
       // ---- down warps: routing first ----
-      const int td = tid - kGuThreads, dw = warp - kGuWarps;
+      int rid;      // the selected expert of this CTA's routed group
+      float wt_r;   // its gate weight
       {
         // every CTA has published its router rows: (l + 1) (E + 1) in all
-        if (issuer) {
-          if (!cnt_wait(A.sync + kCntLogit, (unsigned)(l + 1) * (unsigned)(E + 1)) && !s_abort) {
-            s_abort = 1;
-            raise_status(FMOE_STATUS_WAIT_TIMEOUT);
-          }
-        }
+        if (issuer && !cnt_wait<false>(A.sync + kCntLogit, (unsigned)(l + 1) * (unsigned)(E + 1))) set_abort();
         named_bar(kBarDn, kDnThreads);
-        float lw[kDnKeys];
+        uint64_t lw[kDnKeys + 1];
 #pragma unroll
         for (int i = 0; i < kDnKeys; ++i) {
           const int e = td + i * kDnThreads;
-          lw[i] = e < E ? __ldcg(A.x_logit + e) : 0.f;
+          lw[i] = e < E ? ld_relaxed64(A.x_logit + e) : 0;
         }
-        if (td == 0) s_gamma = __ldcg(A.x_logit + E);
+        lw[kDnKeys] = td == 0 ? ld_relaxed64(A.x_logit + E) : 0;
+        if (!x_settle(lw, e_logit, [&](int i) { return A.x_logit + (i < kDnKeys ? td + i * kDnThreads : E); },
+                      [&](int i) { return i < kDnKeys ? td + i * kDnThreads < E : td == 0; }))
+          set_abort();
+        if (td == 0) s_gamma = x_value(lw[kDnKeys]);
         uint64_t key[kDnKeys];
         bool nan_seen = false;
 #pragma unroll
@@ -711,77 +795,69 @@ __global__ void __launch_bounds__(kFusedThreads, 1) fused_stack_kernel(const __g
           const int e = td + i * kDnThreads;
           key[i] = 0;
           if (e < E) {
-            const float v = lw[i];
+            const float v = x_value(lw[i]);
             nan_seen |= isnan(v);
             slog[e] = v;
             key[i] = route_key(v, e);
           }
         }
-        const uint64_t wk = warp_select_keys<kDnKeys>(key, k);
+        const uint64_t wk = E <= 2 * kDnThreads ? warp_select_keys<2>(key, k) : warp_select_keys<kDnKeys>(key, k);
         if (lane < k) cand[dw * k + lane] = wk;
-        nan_seen = __any_sync(0xffffffffu, nan_seen);
-        if (lane == 0 && nan_seen) cand[kDnWarps * kFusedMaxK] = 1;  // flag word after the candidates
+        if (__any_sync(0xffffffffu, nan_seen) && lane == 0) s_nan = 1;
         named_bar(kBarDn, kDnThreads);
-        if (dw == 0) {
-          uint64_t kk[2];
+        // every down warp merges the warps' candidates itself (same result in
+        // each): the top-k ids, and the softmax of their logits
+        uint64_t kk[2];
 #pragma unroll
-          for (int i = 0; i < 2; ++i) {
-            const int idx = lane + 32 * i;
-            kk[i] = idx < kDnWarps * k ? cand[idx] : 0;
-          }
-          const uint64_t win = warp_select_keys<2>(kk, k);
-          const int sel = lane < k ? key_index(win) : 0;
-          const float val = lane < k ? slog[sel] : 0.f;
-          float m = -INFINITY;
-          for (int r = 0; r < k; ++r) {
-            const float vr = __shfl_sync(0xffffffffu, val, r);
-            if (!isnan(vr)) m = fmaxf(m, vr);
-          }
-          const float pe = (lane < k && !isnan(val)) ? expf(val - m) : 0.f;
-          const float z = warp_sum(pe);
-          if (lane < k) {
-            s_ids[lane] = sel;
-            s_p[lane] = z > 0.f ? pe / z : 0.f;
-            if (c == 0) {
-              A.ids[lane] = sel;
-              A.weights[lane] = s_p[lane];
-            }
-          }
-          if (c == 0 && lane == 0 && cand[kDnWarps * kFusedMaxK] != 0) raise_status(FMOE_STATUS_NAN_LOGIT);
-          __syncwarp();
-          if (lane == 0) {
-            cand[kDnWarps * kFusedMaxK] = 0;
-            // requests: the routed blocks that have a free slot, their down
-            // scale-bias entry, and L2 prefetches of the later ones
-            if (!s_abort) {
-              for (int p = S; p < nseq && p < kSlots; ++p) issue_pos(l, sq, p);
-              if (nq > 0) issue_sb(1, LY.experts + (size_t)s_ids[jj] * LR.bytes, LR, gr);
-              for (int p = kSlots; p < nseq; ++p)
-                prefetch_block(LY.experts + (size_t)s_ids[jj] * LR.bytes, LR, (jg % ngI) * GR::kPerGroup + rb0 + p - S,
-                               GR::gu_sb(H));
-              // the next layer's shared block, when its slot is already free
-              if (S && l + 1 < A.n_layers && nseq < kSlots) issue_pos(l + 1, sq + (uint32_t)nseq, 0);
-            }
-          }
+        for (int i = 0; i < 2; ++i) {
+          const int idx = lane + 32 * i;
+          kk[i] = idx < kDnWarps * k ? cand[idx] : 0;
         }
-        named_bar(kBarDn, kDnThreads);
+        const uint64_t win = warp_select_keys<2>(kk, k);
+        const int sel = lane < k ? key_index(win) : 0;
+        const float val = lane < k ? slog[sel] : 0.f;
+        float m = -INFINITY;
+        for (int r = 0; r < k; ++r) {
+          const float vr = __shfl_sync(0xffffffffu, val, r);
+          if (!isnan(vr)) m = fmaxf(m, vr);
+        }
+        const float pe = (lane < k && !isnan(val)) ? expf(val - m) : 0.f;
+        const float z = warp_sum(pe);
+        const float pw = z > 0.f ? pe / z : 0.f;
+        rid = __shfl_sync(0xffffffffu, sel, jj);
+        wt_r = __shfl_sync(0xffffffffu, pw, jj);
+        if (c == 0 && dw == 0) {
+          if (lane < k) {
+            A.ids[lane] = sel;
+            A.weights[lane] = pw;
+          }
+          if (lane == 0 && s_nan) raise_status(FMOE_STATUS_NAN_LOGIT);
+        }
+        // requests, each by its owner: the routed blocks that have a free
+        // slot, their down scale-bias entry, L2 prefetches of the later
+        // ones, and the next layer's shared block when its slot is free
+        if (owner && !s_abort) {
+          for (int p = S; p < nseq && p < kSlots; ++p) issue_pos(l, sq, p, rid);
+          if (nq > 0 && dw == kWarpSb + 1) issue_sb(1, LY.experts + (size_t)rid * LR.bytes, LR, gr);
+          if (dw >= kWarpPf)
+            for (int p = kSlots + dw - kWarpPf; p < nseq; p += kDnWarps - kWarpPf)
+              prefetch_block(LY.experts + (size_t)rid * LR.bytes, LR, routed_nb(p), GR::gu_sb(H));
+          if (S && l + 1 < A.n_layers && nseq < kSlots) issue_pos(l + 1, sq + (uint32_t)nseq, 0, 0);
+        }
       }
       // ---- down products, block by block ----
-#pragma unroll
-      for (int m = 0; m < kDnRowsT; ++m) yacc[m] = 0.f;
+      float yacc[kDnRowsT];  // this CTA's partial output rows
       float uacc[kDnRowsT];  // routed blocks: sum of step * weight * value, scaled per row at the end
 #pragma unroll
-      for (int m = 0; m < kDnRowsT; ++m) uacc[m] = 0.f;
+      for (int m = 0; m < kDnRowsT; ++m) yacc[m] = uacc[m] = 0.f;
       float p2sum = 0.f;  // routed blocks: sum of step * weight * sum xi (times the row's bias at the end)
-      const float wt_r = s_p[jj], wt_s = s_gamma;
+      const float wt_s = s_gamma;
       for (int p = 0; p < nseq; ++p) {
         const uint32_t pos = sq + (uint32_t)p;
         const int s = (int)(pos % kSlots);
         bool ok = wait_mb(kMbReady + s, (pos / kSlots) & 1u);
         ok = ok && wait_mb(kMbFull + s, (pos / kSlots) & 1u);
         if (p == 0 && S) ok = ok && wait_mb(kMbSbShared, (uint32_t)l & 1u);
-        // this CTA's last block has landed: the next layer's router rows may compete for HBM
-        if (issuer && p == nseq - 1 && l + 1 < A.n_layers) prefetch_router(l + 1);
         if (ok) {
           const uint8_t* sl = smem + P.slot[s];
           const uint32_t* dx = dnx + s * kDnxWords;
@@ -812,17 +888,19 @@ __global__ void __launch_bounds__(kFusedThreads, 1) fused_stack_kernel(const __g
           }
         }
         named_bar(kBarDn, kDnThreads);  // every down thread is done with the slot
-        if (issuer && !s_abort) {
+        if (owner && !s_abort) {
           // the slot takes the block three positions on: this layer's, or
           // the next layer's shared block
           const int pn = p + kSlots;
-          if (pn < nseq) issue_pos(l, sq, pn);
-          else if (pn == nseq && S && l + 1 < A.n_layers) issue_pos(l + 1, sq + (uint32_t)nseq, 0);
+          if (pn < nseq) issue_pos(l, sq, pn, rid);
+          else if (pn == nseq && S && l + 1 < A.n_layers) issue_pos(l + 1, sq + (uint32_t)nseq, 0, 0);
           // the shared entry is free: the next layer's comes in
-          if (p == 0 && S && l + 1 < A.n_layers) issue_sb(0, A.layers[l + 1].shared, LS, c / GS::kPerGroup);
+          if (p == 0 && S && l + 1 < A.n_layers && dw == kWarpSb)
+            issue_sb(0, A.layers[l + 1].shared, LS, c / GS::kPerGroup);
         }
       }
-      if (nseq == 0 && issuer && l + 1 < A.n_layers) prefetch_router(l + 1);
+      // every block of the layer is done: the next layer's router rows come in
+      if (l + 1 < A.n_layers && !s_abort) issue_router(l + 1, sq + (uint32_t)nseq);
       // ---- F: routed blocks scaled per row, partial output out ----
       bool ok = true;
       if (nq > 0) ok = wait_mb(kMbSbRouted, (uint32_t)l & 1u);
@@ -857,10 +935,12 @@ __global__ void __launch_bounds__(kFusedThreads, 1) fused_stack_kernel(const __g
     {
       // rows i0 + r, r < nd: ngr threads per row each sum every ngr-th CTA's
       // partial; then one thread per row adds those sums in order
+      const int nd = i1 - i0;
       const int ngr = nd > 0 ? kFusedThreads / nd : 0;
       const int r = nd > 0 ? tid % nd : 0, pg = nd > 0 ? tid / nd : kFusedThreads;
       const float hres = tid < nd ? A.h[i0 + tid] : 0.f;  // this CTA's own rows
       if (!cta_cnt_wait(kCntPart, (unsigned)(l + 1) * (unsigned)nC)) { aborted = true; break; }
+      float* sred = reinterpret_cast<float*>(smem + P.red);
       if (pg < ngr) {
         constexpr int kLoads = (kFusedMaxCtas * 32 + kFusedThreads - 1) / kFusedThreads;  // ngr >= 512 / 32
         float v[kLoads];
@@ -886,25 +966,26 @@ __global__ void __launch_bounds__(kFusedThreads, 1) fused_stack_kernel(const __g
       if (warp == 0) {
         ss = warp_sum(ss);
         if (lane == 0) __stcg(A.x_ss + c, ss);
+        __syncwarp();
+        if (lane == 0) cnt_release_add(A.sync + kCntH, 1u);  // warp 0 wrote every row of this CTA (nd <= 32)
       }
-      __syncthreads();
-      if (tid == 0) cnt_release_add(A.sync + kCntH, 1u);
     }
   }
 
-  // after the last layer: every CTA's h' rows and sum of squares are written
+  // after the last layer: every CTA's adds have landed
   bool done = !aborted && A.n_layers > 0;
   if (done) done = cta_cnt_wait(kCntH, (unsigned)A.n_layers * (unsigned)nC);
   if (done) {
-    // epilogue: xn' of the last layer for this CTA's rows (h' written by this thread)
+    // epilogue: xn' of the last layer for this CTA's rows (h' written by this CTA)
     const float r_last = norm_scale(tid < nC ? __ldcg(A.x_ss + tid) : 0.f);
     const float* w = A.layers[A.n_layers - 1].norm_w;
-    if (tid < nd) A.xn[i0 + tid] = A.h[i0 + tid] * r_last * w[i0 + tid];
+    if (tid < i1 - i0) A.xn[i0 + tid] = A.h[i0 + tid] * r_last * w[i0 + tid];
     __syncthreads();
     if (tid == 0) {
       __threadfence();
       const unsigned prev = atomicAdd(&A.sync[kCntExit], 1u);
       if (prev == (unsigned)nC - 1) {  // every CTA is past its last counter wait
+        A.sync[kEpoch] = base + (uint32_t)A.n_layers + 1u;
         A.sync[kCntH] = 0;
         A.sync[kCntLogit] = 0;
         A.sync[kCntPart] = 0;
@@ -913,8 +994,8 @@ __global__ void __launch_bounds__(kFusedThreads, 1) fused_stack_kernel(const __g
       }
     }
   }
-  if (issuer) {
-    // drain: wait (bounded) for this issuer's copies still in flight -- the
+  if (owner) {
+    // drain: wait (bounded) for this lane's copies still in flight -- the
     // last phase armed on each barrier (earlier phases have completed: a
     // slot or entry is re-armed only after its previous contents were used).
     // On a clean exit these phases have completed already.

@@ -577,12 +577,12 @@ static inline size_t align_up(size_t v, size_t a) { return (v + a - 1) / a * a; 
 static WsLayout ws_layout(int H, int I, int E, int k, int T) {
   WsLayout w;
   w.sync = 0;  // grid-barrier counter, exit counter and epoch of the fused kernel
-  // exchange buffers of the fused kernel (fp32), at offsets and sizes that
-  // do not depend on the shape or T (its counters, at the start, decide
-  // when their contents are current)
+  // exchange buffers of the fused kernel (logit exchange words, fp32
+  // partial outputs and h'), at offsets and sizes that do not depend on the
+  // shape or T: no other kernel writes there
   size_t o = 4096;
   w.x_logit = o;
-  o = align_up(o + (size_t)(kFusedMaxE + 1) * 4, 256);
+  o = align_up(o + (size_t)(kFusedMaxE + 1) * 8, 256);
   w.x_ss = o;
   o = align_up(o + (size_t)kFusedMaxCtas * 4, 256);
   w.x_h = o;
@@ -957,7 +957,7 @@ static int launch_fused(const fmoe_layer_weights* layers, int n_layers, float* h
   args.weights = reinterpret_cast<float*>(base + w.weights) + (size_t)t * d.top_k;
   args.gamma = reinterpret_cast<float*>(base + w.gamma) + t;
   args.a = reinterpret_cast<float*>(base + w.a) + (size_t)t * (d.top_k + 1) * d.inter;
-  args.x_logit = reinterpret_cast<float*>(base + w.x_logit);
+  args.x_logit = reinterpret_cast<uint64_t*>(base + w.x_logit);
   args.x_h = reinterpret_cast<float*>(base + w.x_h);
   args.x_ss = reinterpret_cast<float*>(base + w.x_ss);
   args.x_part = reinterpret_cast<float*>(base + w.x_part);
