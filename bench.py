@@ -553,35 +553,40 @@ def run_ours(args):
                 "timing": "CUDA events on the launching stream around the timed replays"}
 
     # ---- end to end through the C ABI with host buffers (eager calls) ----
-    K2 = args.e2e_steps or min(args.steps, 2000)
-    xs = synth.tokens(wl, min(K2, 64), stream=500 + rank)
+    # A plain C decode loop: per call, one token's [2, 1, H] block (h and its
+    # normed copy xn) is copied from pinned host memory to the device, the L
+    # resident layers run, and h', xn' are copied back (fmoe_stack_forward_host).
+    # One call = L steps.
+    K2 = args.e2e_steps or max(min(args.steps, 2000), 10 * L)
+    calls = max(1, K2 // L)
+    K2 = calls * L
+    xs = synth.tokens(wl, min(calls, 64), stream=500 + rank)
     nb = xs.shape[0]
-    # per step one pinned [2, 1, H] block (h and its normed copy xn) goes in
-    # and one comes out, through the host-state entry point of the C ABI
     hx_in = torch.from_numpy(np.ascontiguousarray(np.stack([xs, xs], axis=1)[:, :, None, :])).pin_memory()
     hx_out = torch.empty((nb, 2, 1, H), dtype=torch.float32).pin_memory()
     hx = torch.empty((2, 1, H), dtype=torch.float32, device="cuda")
 
-    def e2e_steps(n):
+    def e2e_calls(n):
         for i in range(n):
             j = i % nb
-            fm.fmoe_layer_forward_host(layers[i % L], hx_in[j], hx_out[j], hx, ws, stream=stream)
+            fm.fmoe_stack_forward_host(layers, hx_in[j], hx_out[j], hx, ws, stream=stream)
 
     with torch.cuda.stream(stream):
-        e2e_steps(min(50, K2))
+        e2e_calls(min(5, calls))
     torch.cuda.synchronize()
     barrier(world)
     e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     with torch.cuda.stream(stream):
         e0.record(stream)
-        e2e_steps(K2)
+        e2e_calls(calls)
         e1.record(stream)
     e1.synchronize()
     e2e_ms = max_over_ranks(e0.elapsed_time(e1), world)
-    e2e = {"value": job_rate(K2, world, e2e_ms), "unit": UNIT, "h2d_bytes_per_step": 2 * H * 4,
-           "d2h_bytes_per_step": 2 * H * 4, "steps": K2,
-           "how": "per step: fmoe_layer_forward_host (one eager C-ABI call): a pinned host [2, H] block (h, xn) "
-                  "-> device, the layer, h', xn' -> pinned host"}
+    e2e = {"value": job_rate(K2, world, e2e_ms), "unit": UNIT, "h2d_bytes_per_step": 2 * H * 4 / L,
+           "d2h_bytes_per_step": 2 * H * 4 / L, "steps": K2, "calls": calls,
+           "how": f"per call (= {L} steps): fmoe_stack_forward_host, one eager C-ABI call: a pinned host [2, H] block "
+                  f"(h, xn) -> device, the {L} resident layers, h', xn' -> pinned host ({2 * H * 4} bytes each way "
+                  f"per call)"}
 
     line = {"metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
             "warmup": args.warmup, "ms_per_step": ms_max / args.steps, "higher_is_better": True,

@@ -302,6 +302,18 @@ int fmoe_layer_forward_logits(const fmoe_layer_weights* lw, const float* d_logit
 int fmoe_stack_forward(const fmoe_layer_weights* layers, int n_layers, float* d_h, float* d_xn,
                        int T, void* d_ws, size_t ws_bytes, cudaStream_t stream);
 
+/* fmoe_stack_forward for token state in host memory (the call a plain C
+ * decode loop makes once per token): hx_in / hx_out host fp32 [2][T][H]
+ * (h rows, then xn rows), d_hx device fp32 [2][T][H] that the stack runs on
+ * in place.  One host-to-device copy, the n_layers layers, one
+ * device-to-host copy, all on `stream`; hx_in and hx_out may be the same
+ * buffer.  Every layer must have the same hidden size.  Errors: as
+ * fmoe_stack_forward, checked before any copy, plus
+ * FMOE_ERR_BUFFER_TOO_SMALL when ws_bytes is below any layer's
+ * fmoe_workspace_bytes(desc, T). */
+int fmoe_stack_forward_host(const fmoe_layer_weights* layers, int n_layers, const float* hx_in, float* hx_out,
+                            float* d_hx, int T, void* d_ws, size_t ws_bytes, cudaStream_t stream);
+
 /* Chooses the implementation of the T = 1 path (and of the few-token calls
  * that run token by token, see fmoe_fused_max_tokens): enable != 0 (the
  * default) uses the persistent fused kernel wherever its shared-memory plan

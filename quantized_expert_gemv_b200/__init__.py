@@ -96,6 +96,7 @@ _SIGS = {
     "fmoe_cache_stats": (_i32, [_vp, _vp, _vp, _vp]),
     "fmoe_cache_layer_forward": (_i32, [_vp, _i32, _vp, _vp, _vp, _vp, _i32, _vp, _sz, _vp]),
     "fmoe_layer_forward_host": (_i32, [_vp, _vp, _vp, _vp, _i32, _vp, _sz, _vp]),
+    "fmoe_stack_forward_host": (_i32, [_PW, _i32, _vp, _vp, _vp, _i32, _vp, _sz, _vp]),
     "fmoe_quantize_groups": (_i32, [_vp, _sz, _i32, _i32, _vp, _vp, _vp, _vp]),
     "fmoe_fused_max_tokens": (_i32, [_i32]),
     "fmoe_layer_forward_noalloc": (_i32, [_PW, _vp, _vp, _i32, _vp]),
@@ -311,6 +312,16 @@ def fmoe_layer_forward_logits(lw: LayerWeights, logits, h, xn, ws, stream=None) 
     rc = _lib.fmoe_layer_forward_logits(ctypes.byref(c), _ptr(logits), _ptr(h), _ptr(xn), h.shape[0], _ptr(ws),
                                         ws.numel() * ws.element_size(), _stream(stream))
     _check(rc, "fmoe_layer_forward_logits")
+
+
+def fmoe_stack_forward_host(layers, hx_in, hx_out, d_hx, ws, stream=None) -> None:
+    """fmoe_stack_forward on host token state: hx_in / hx_out (pinned) host
+    tensors [2, T, H], d_hx a device tensor of the same shape; one copy in,
+    the layers, one copy out, asynchronous on `stream`."""
+    arr = (fmoe_layer_weights * len(layers))(*[lw.c() for lw in layers])
+    rc = _lib.fmoe_stack_forward_host(arr, len(layers), _ptr(hx_in), _ptr(hx_out), _ptr(d_hx), d_hx.shape[1],
+                                      _ptr(ws), ws.numel() * ws.element_size(), _stream(stream))
+    _check(rc, "fmoe_stack_forward_host")
 
 
 def fmoe_stack_forward(layers, h, xn, ws, stream=None) -> None:

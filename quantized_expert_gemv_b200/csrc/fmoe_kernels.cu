@@ -1269,6 +1269,28 @@ extern "C" int fmoe_stack_forward(const fmoe_layer_weights* layers, int n_layers
   return FMOE_OK;
 }
 
+extern "C" int fmoe_stack_forward_host(const fmoe_layer_weights* layers, int n_layers, const float* hx_in,
+                                       float* hx_out, float* d_hx, int T, void* d_ws, size_t ws_bytes,
+                                       cudaStream_t stream) {
+  if (!layers || n_layers < 1 || !hx_in || !hx_out || !d_hx || !d_ws || T < 1 || !aligned16(d_hx) ||
+      !aligned16(d_ws))
+    return FMOE_ERR_INVALID_ARG;
+  for (int l = 0; l < n_layers; ++l) {
+    const int rc = weights_check(&layers[l]);
+    if (rc != FMOE_OK) return rc;
+    if (layers[l].desc.hidden != layers[0].desc.hidden) return FMOE_ERR_INVALID_ARG;
+    const fmoe_layer_desc& d = layers[l].desc;
+    if (ws_bytes < ws_layout(d.hidden, d.inter, d.n_experts, d.top_k, T).bytes) return FMOE_ERR_BUFFER_TOO_SMALL;
+  }
+  const int H = layers[0].desc.hidden;
+  const size_t bytes = (size_t)2 * T * H * sizeof(float);
+  if (cudaMemcpyAsync(d_hx, hx_in, bytes, cudaMemcpyHostToDevice, stream) != cudaSuccess) return FMOE_ERR_CUDA;
+  const int rc = fmoe_stack_forward(layers, n_layers, d_hx, d_hx + (size_t)T * H, T, d_ws, ws_bytes, stream);
+  if (rc != FMOE_OK) return rc;
+  return cudaMemcpyAsync(hx_out, d_hx, bytes, cudaMemcpyDeviceToHost, stream) == cudaSuccess ? FMOE_OK
+                                                                                            : FMOE_ERR_CUDA;
+}
+
 // --------------------------------------------- fixed device scratch ----
 // Workspace of fmoe_layer_forward_noalloc: one array per device, set aside
 // when the module loads, so that the call itself reserves no memory.

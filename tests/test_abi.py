@@ -202,6 +202,12 @@ def test_host_validation_of_the_later_entry_points(fm):
     assert L.fmoe_layer_forward_host(ctypes.byref(w), None, 16, 16, 1, 16, 1 << 30, None) == fm.FMOE_ERR_INVALID_ARG
     assert L.fmoe_layer_forward_host(ctypes.byref(w), 16, 16, 24, 1, 16, 1 << 30, None) == fm.FMOE_ERR_INVALID_ARG
     assert L.fmoe_layer_forward_host(ctypes.byref(w), 16, 16, 16, 1, 16, 64, None) == fm.FMOE_ERR_BUFFER_TOO_SMALL
+    # host-state stack: no layers, null buffers, workspace too small
+    ws2 = (fm.fmoe_layer_weights * 2)(w, w)
+    assert L.fmoe_stack_forward_host(None, 1, 16, 16, 16, 1, 16, 1 << 30, None) == fm.FMOE_ERR_INVALID_ARG
+    assert L.fmoe_stack_forward_host(ws2, 2, None, 16, 16, 1, 16, 1 << 30, None) == fm.FMOE_ERR_INVALID_ARG
+    assert L.fmoe_stack_forward_host(ws2, 2, 16, 16, 24, 1, 16, 1 << 30, None) == fm.FMOE_ERR_INVALID_ARG
+    assert L.fmoe_stack_forward_host(ws2, 2, 16, 16, 16, 1, 16, 64, None) == fm.FMOE_ERR_BUFFER_TOO_SMALL
     # expert cache: missing arguments, slots too small for n_slots records
     dc = d.c()
     hp = (ctypes.c_void_p * 1)(16)

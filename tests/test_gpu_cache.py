@@ -128,3 +128,57 @@ def test_cache_too_small_for_one_step_is_an_error():
     with pytest.raises(fm.FmoeError):
         cache.forward(0, lws[0], h, xn, ws)
     cache.close()
+
+
+@pytest.mark.parametrize("T", [1, 3])
+@pytest.mark.parametrize("fused", [True, False], ids=["fused-enabled", "fused-disabled"])
+def test_cached_steps_match_oracle(T, fused):
+    """Cached layer steps against the fp64 oracle, element by element: the
+    router logits, the top-k on the device's logits, the gate weights and
+    gamma, every selected expert's SwiGLU outputs a and down outputs y, h'
+    and xn'.  Two steps per layer: the first copies its records in from host
+    memory, the second finds them in the cache.  The host tier runs the same
+    way with the persistent kernel enabled or not (it learns the routing on
+    the host before the expert products, so it always takes the
+    one-kernel-per-step products)."""
+    import oracle
+    from tests.parity import check
+    wl = SMALL
+    lws, host = _layers(wl, 2)
+    cache = fm.ExpertCache(lws[0].desc, host, n_slots=max(6, T * wl.top_k), max_tokens=T)
+    x = synth.tokens(wl, T, stream=74)
+    h, xn = torch.from_numpy(x).cuda(), torch.from_numpy(x).cuda()
+    ws = fm.alloc_workspace(lws[0].desc, T)
+    prev = fm.fmoe_set_fused(fused)
+    try:
+        for step in range(2):
+            for l in range(2):
+                h_in, xn_in = h.cpu().numpy().astype(np.float64), xn.cpu().numpy().astype(np.float64)
+                cache.forward(l, lws[l], h, xn, ws)
+                torch.cuda.synchronize()
+                view = lambda which: fm.workspace_view(ws, lws[l].desc, T, which).cpu().numpy()
+                lg, ids, p, gm = view(fm.WS_LOGITS), view(fm.WS_IDS), view(fm.WS_WEIGHTS), view(fm.WS_GAMMA)
+                a, y = view(fm.WS_A), view(fm.WS_Y)
+                lo = oracle.LayerWeights(synth.router(wl, l), synth.shared_gate(wl, l), synth.norm_weight(wl, l),
+                                         {e: synth.expert(wl, l, e) for e in range(wl.n_experts + 1)})
+                for t in range(T):
+                    label = f"step {step} layer {l} token {t}"
+                    lg_o, S_l = oracle.gemv_f32(lo.w_router, xn_in[t])
+                    check(lg[t], lg_o, S_l, f"{label} logits")
+                    ref = oracle.layer_token(wl, lo, h_in[t], xn_in[t], logits_in=lg[t])
+                    assert ref["ids"].tolist() == ids[t].tolist(), label
+                    check(p[t], ref["p"], ref["p"], f"{label} gate weights")
+                    check(gm[t], ref["gamma"], ref["gamma"] + ref["S_gamma"], f"{label} gamma", rel_l2=False)
+                    for j, slot in enumerate(list(ids[t]) + [wl.n_experts]):
+                        e = oracle.expert_ffn(lo.experts[int(slot)], wl.hidden, wl.inter, 64, xn_in[t])
+                        check(a[t, j], e["a"], e["S_a"], f"{label} a[{j}]")
+                    check(y[t], ref["y"], ref["S_y"], f"{label} y")
+                    check(h.cpu().numpy()[t], ref["h"], ref["S_h"], f"{label} h'")
+                    check(xn.cpu().numpy()[t], ref["xn"], ref["S_xn"], f"{label} xn'")
+            h.copy_(xn)
+    finally:
+        fm.fmoe_set_fused(prev)
+    hits, misses, _ = cache.stats()
+    assert hits >= 1 and misses >= 1
+    assert fm.fmoe_read_status() == 0
+    cache.close()

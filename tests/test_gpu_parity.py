@@ -486,6 +486,25 @@ def test_host_state_entry_point_matches_device_entry_point(T):
     assert fm.fmoe_read_status() == 0
 
 
+@pytest.mark.parametrize("T", [1, 2])
+def test_host_state_stack_matches_device_stack(T):
+    """fmoe_stack_forward_host (pinned host h/xn in, three layers, h'/xn'
+    out) gives the bits of fmoe_stack_forward on device tensors."""
+    wl = SMALL
+    lws = [device_layer(wl, l) for l in range(3)]
+    x = synth.tokens(wl, T, stream=64)
+    h, xn = dev(x), dev(x)
+    ws = fm.alloc_workspace(lws[0].desc, T)
+    fm.fmoe_stack_forward(lws, h, xn, ws)
+    hx = torch.from_numpy(np.stack([x, x])).pin_memory()
+    d_hx = torch.empty(hx.shape, dtype=torch.float32, device="cuda")
+    ws2 = fm.alloc_workspace(lws[0].desc, T)
+    fm.fmoe_stack_forward_host(lws, hx, hx, d_hx, ws2)  # in place on the host buffer
+    torch.cuda.synchronize()
+    assert np.array_equal(hx[0].numpy(), host(h)) and np.array_equal(hx[1].numpy(), host(xn))
+    assert fm.fmoe_read_status() == 0
+
+
 def test_tensor_core_and_integer_paths_differ_only_by_rounding():
     """The two implementations of the grouped products both run (their
     results are not bit-identical) and agree well inside the tolerance."""
