@@ -315,7 +315,7 @@ int fmoe_stack_forward_host(const fmoe_layer_weights* layers, int n_layers, cons
                             float* d_hx, int T, void* d_ws, size_t ws_bytes, cudaStream_t stream);
 
 /* Chooses the implementation of the T = 1 path (and of the few-token calls
- * that run token by token, see fmoe_fused_max_tokens): enable != 0 (the
+ * that run through the persistent kernel, see fmoe_fused_max_tokens): enable != 0 (the
  * default) uses the persistent fused kernel wherever its shared-memory plan
  * fits, 0 the one-kernel-per-step path.  Both compute the same layer;
  * process-wide setting, returns the previous value. */
@@ -331,11 +331,18 @@ int fmoe_set_fused(int enable);
 int fmoe_set_tensor_cores(int enable);
 
 /* Largest token count T for which fmoe_layer_forward (stack == 0) or
- * fmoe_stack_forward (stack != 0) runs the tokens one by one through the
- * persistent T = 1 kernel (when enabled, fmoe_set_fused): 4 and 8.  Such
- * calls compute each token exactly as a T = 1 call on that token would and
- * leave, like T = 1, no per-expert outputs y in the workspace; larger T take
- * the grouped path. */
+ * fmoe_stack_forward (stack != 0) runs the tokens through the persistent
+ * kernel (when enabled, fmoe_set_fused): 4 and 8.  Tokens go two per launch
+ * where the kernel has a two-token form for the code widths (4-bit routed
+ * and shared experts; an odd last token, and other widths, one per launch):
+ * a pair shares the router rows, the shared expert's weights and the
+ * exchanges between CTAs (section "Understanding Mixture-of-Experts" of
+ * "What is Flash-MoE?": the shared expert serves every token).  A token's
+ * result in a pair does not depend on the other token of the pair (the work
+ * is split over the CTAs by position in the pair, not by value) but is
+ * rounded differently from a one-token launch.  Such calls leave, like
+ * T = 1, no per-expert outputs y in the workspace; larger T take the grouped
+ * path. */
 int fmoe_fused_max_tokens(int stack);
 
 /* Tokens an expert needs in a step for its products to run on the tensor
@@ -363,7 +370,7 @@ int fmoe_fused_supported(const fmoe_layer_desc* d);
  * library's module is loaded on that device.
  *   lw, d_h, d_xn, T, stream  as for fmoe_layer_forward.
  * Limit: fmoe_workspace_bytes(&lw->desc, T) must not exceed 12 MiB
- * (12582912 bytes), which admits up to T = 17 tokens at hidden 4096 /
+ * (12582912 bytes), which admits up to T = 16 tokens at hidden 4096 /
  * inter 1024 / 512 experts / top-4 (from T = 5 the workspace holds the
  * tensor-core inputs, about 100 KB per token); a larger request returns
  * FMOE_ERR_BUFFER_TOO_SMALL before anything is launched.

@@ -33,6 +33,15 @@
 // one expert (the groups are spread over the CTAs), so one 16 KB entry holds
 // their down scale-bias words, and their down products share one scale per
 // row: they are accumulated unscaled and scaled once per layer.
+// Two tokens per launch (NT = 2): both tokens' xn are staged, every router
+// row is read once and dotted with both, the shared expert's blocks are
+// read once and applied to both tokens (gate/up, SwiGLU and down products
+// per token from the same codes in shared memory), and the exchanges carry
+// both tokens at once, so the chain of dependent steps is paid once for
+// the pair.  The routed 64-groups of the NT k (token, selected expert)
+// pairs are spread over the CTAs: each CTA's routed blocks belong to one
+// token and one expert.  A CTA's partial output for the other token is its
+// shared-block contribution (or zero), written as soon as it is known.
 // Source pages: "What is Flash-MoE?" (a2a-mcp.org), sections
 // "Understanding Mixture-of-Experts", "2. FMA-optimised dequantisation
 // kernels" and "3. Hand-tuned Metal compute shaders" (deferred command-buffer
@@ -78,6 +87,12 @@ constexpr int kFusedMaxK = 8;
 constexpr int kFusedMaxE = 1024;
 constexpr int kFusedMaxH = 4096;
 constexpr int kFusedMaxCtas = 160;      // partial outputs in the workspace: [kFusedMaxCtas][kFusedMaxH]
+constexpr int kFusedMaxNT = 2;          // tokens per launch
+// token strides of the exchange buffers (their sizes do not depend on the shape)
+constexpr int kXLogitStride = kFusedMaxE + 1;
+constexpr int kXSsStride = kFusedMaxCtas;
+constexpr int kXHStride = kFusedMaxH;
+constexpr size_t kXPartStride = (size_t)kFusedMaxCtas * kFusedMaxH;
 constexpr int kFusedMaxRouterRows = 4;  // router rows (E experts + the shared gate) per CTA
 constexpr int kDnQuads = 4;             // groups of 4 consecutive hidden rows per down thread: H <= 4096
 constexpr int kDnRowsT = 4 * kDnQuads;  // hidden rows per down thread
@@ -117,11 +132,12 @@ struct FusedLayer {
 struct FusedPlan {
   uint32_t slot[kSlots];
   uint32_t sbe[2];  // shared expert, routed experts
-  uint32_t xs;      // staged x of the layer (24-bit block floating point)
+  uint32_t xs;      // staged x of the layer, per token (24-bit block floating point)
+  uint32_t xs_stride;
   uint32_t logit;   // fp32 [E]
   uint32_t cand;    // top-k candidates: u64 [kDnWarps][k]
-  uint32_t gred;    // gate/up partial sums: fp32 [2][kGuWarps][8]
-  uint32_t dnx;     // staged SwiGLU outputs per slot: u32 [kSlots][kDnxWords]
+  uint32_t gred;    // gate/up partial sums: fp32 [2][NT][kGuWarps][8]
+  uint32_t dnx;     // staged SwiGLU outputs per slot and token: u32 [kSlots][NT][kDnxWords]
   uint32_t red;     // fp32 [kFusedThreads]: partial sums of the row reduction
   uint32_t mbar;
   uint32_t total;
@@ -132,17 +148,18 @@ struct FusedArgs {
   int n_layers;
   int H, I, E, k;
   float eps;
-  float* h;
-  float* xn;
-  float* logits;
-  int32_t* ids;
-  float* weights;
-  float* gamma;
-  float* a;           // [(k+1)][I], shared expert last
-  uint64_t* x_logit;  // [E + 1]: router logits, then sigmoid(w_sg . xn) (exchange words)
-  float* x_h;      // [H]: h' of the layer
-  float* x_ss;     // [gridDim.x]: per-CTA sums of h'^2
-  float* x_part;   // [gridDim.x][H]: partial outputs
+  // per token, token-major (the launch's first token at the pointer)
+  float* h;           // [NT][H]
+  float* xn;          // [NT][H]
+  float* logits;      // [NT][E]
+  int32_t* ids;       // [NT][k]
+  float* weights;     // [NT][k]
+  float* gamma;       // [NT]
+  float* a;           // [NT][(k+1)][I], shared expert last
+  uint64_t* x_logit;  // [NT][kXLogitStride]: router logits, then sigmoid(w_sg . xn) (exchange words)
+  float* x_h;      // [NT][kXHStride]: h' of the layer
+  float* x_ss;     // [NT][kXSsStride]: per-CTA sums of h'^2
+  float* x_part;   // [NT][kXPartStride]: partial outputs, [gridDim.x][H] per token
   unsigned* sync;  // counters kCntH, kCntExit, kCntLogit, kCntPart; logit epoch base kEpoch
   FusedPlan plan;
 };
@@ -503,14 +520,15 @@ __device__ __forceinline__ void block_down(const uint8_t* slot, const uint32_t* 
 }
 
 // ------------------------------------------------------------ the kernel --
-template <int BITS, int SBITS>  // routed and shared code widths
+template <int BITS, int SBITS, int NT>  // routed and shared code widths, tokens per launch
 __global__ void __launch_bounds__(kFusedThreads, 1) fused_stack_kernel(const __grid_constant__ FusedArgs A) {
+  static_assert(NT >= 1 && NT <= kFusedMaxNT, "tokens per launch");
   using GR = BlockGeo<BITS>;
   using GS = BlockGeo<SBITS>;
   extern __shared__ __align__(128) unsigned char smem[];
-  __shared__ float s_gamma;
-  __shared__ float s_rp[kFusedWarps][kFusedMaxRouterRows];
-  __shared__ float s_red[kFusedWarps];
+  __shared__ float s_gamma[NT];
+  __shared__ float s_rp[kFusedWarps][NT][kFusedMaxRouterRows];
+  __shared__ float s_red[NT][kFusedWarps];
   __shared__ volatile int s_abort;
   __shared__ int s_nan;
 
@@ -520,7 +538,7 @@ __global__ void __launch_bounds__(kFusedThreads, 1) fused_stack_kernel(const __g
   const int ngH = H / 64, ngI = I / 64;
   const FusedPlan& P = A.plan;
   uint64_t* mbar = reinterpret_cast<uint64_t*>(smem + P.mbar);
-  const StagedX sx = staged_x_at(smem + P.xs, H);
+  auto sx_of = [&](int t) { return staged_x_at(smem + P.xs + (size_t)t * P.xs_stride, H); };
   float* slog = reinterpret_cast<float*>(smem + P.logit);
   uint64_t* cand = reinterpret_cast<uint64_t*>(smem + P.cand);
   float* gred = reinterpret_cast<float*>(smem + P.gred);
@@ -530,16 +548,21 @@ __global__ void __launch_bounds__(kFusedThreads, 1) fused_stack_kernel(const __g
   const int nr = c <= E ? (E - c) / nC + 1 : 0;  // router rows c, c + nC, ... <= E (row E: shared gate)
   const int NBs = I * SBITS / 32;
   const int S = c < NBs ? 1 : 0;  // shared block c
-  // routed blocks: [rb0, rb1) of 64-group jg of the k selected experts'
-  // groups (expert jj = jg / ngI, group gr = jg % ngI)
-  const int Gr = k * ngI;
+  // routed blocks: [rb0, rb1) of 64-group jg of the NT k (token, selected
+  // expert) pairs' groups (pair = jg / ngI: token tr = pair / k, its jj-th
+  // expert; group gr = jg % ngI)
+  const int Gr = NT * k * ngI;
   const int jg = routed_group_of(c, nC, Gr);
-  int rb0, rb1;
+  int rb0, rb1, cs0;
   {
-    const int cs0 = (int)(((long long)jg * nC) / Gr), cs1 = (int)(((long long)(jg + 1) * nC) / Gr);
+    cs0 = (int)(((long long)jg * nC) / Gr);
+    const int cs1 = (int)(((long long)(jg + 1) * nC) / Gr);
     share(GR::kPerGroup, c - cs0, cs1 - cs0, &rb0, &rb1);
   }
-  const int nq = rb1 - rb0, jj = jg / ngI, gr = jg % ngI;
+  const int nq = rb1 - rb0, pair = jg / ngI, gr = jg % ngI;
+  const int tr = NT == 1 ? 0 : pair / k, jj = NT == 1 ? pair : pair % k;
+  // the CTA that writes token tr's ids and gate weights: the first of its first group
+  const bool route_writer = jj == 0 && gr == 0 && c == cs0;
   const int nseq = S + nq;  // blocks per layer: the shared one first
   int i0, i1;
   share(H, c, nC, &i0, &i1);  // hidden rows of the final sums
@@ -653,17 +676,32 @@ __global__ void __launch_bounds__(kFusedThreads, 1) fused_stack_kernel(const __g
     if (tid == 0) raise_status(FMOE_STATUS_WAIT_TIMEOUT);
     return false;
   };
-  // r = (sum of the CTAs' partial sums of h'^2 / H + eps)^(-1/2), summed in
-  // the same order in every CTA; ssv: this thread's partial (tid < nC)
-  auto norm_scale = [&](float ssv) -> float {
-    float v = warp_sum(tid < nC ? ssv : 0.f);
-    if (lane == 0) s_red[warp] = v;
-    __syncthreads();
-    float t = 0.f;
+  // per token: r = (sum of the CTAs' partial sums of h'^2 / H + eps)^(-1/2),
+  // summed in the same order in every CTA (thread t < nC holds CTA t's partials)
+  auto norm_scales = [&](float (&r)[NT]) {
 #pragma unroll
-    for (int wi = 0; wi < kFusedWarps; ++wi) t += s_red[wi];
+    for (int t = 0; t < NT; ++t) {
+      const float v = warp_sum(tid < nC ? __ldcg(A.x_ss + (size_t)t * kXSsStride + tid) : 0.f);
+      if (lane == 0) s_red[t][warp] = v;
+    }
     __syncthreads();
-    return 1.f / sqrtf(t / (float)H + A.eps);
+#pragma unroll
+    for (int t = 0; t < NT; ++t) {
+      float s = 0.f;
+#pragma unroll
+      for (int wi = 0; wi < kFusedWarps; ++wi) s += s_red[t][wi];
+      r[t] = 1.f / sqrtf(s / (float)H + A.eps);
+    }
+    __syncthreads();
+  };
+  // the down threads' rows of a partial output: quads 4 (td + kDnThreads m)
+  auto store_rows = [&](float* part, const float (&v)[kDnRowsT]) {
+#pragma unroll
+    for (int m = 0; m < kDnQuads; ++m) {
+      const int row = 4 * (td + kDnThreads * m);
+      if (row < H)
+        __stcg(reinterpret_cast<float4*>(part + row), make_float4(v[4 * m], v[4 * m + 1], v[4 * m + 2], v[4 * m + 3]));
+    }
   };
 
   const uint32_t base = __ldcg(A.sync + kEpoch);  // logit epoch of layer l: base + l + 1
@@ -680,33 +718,52 @@ __global__ void __launch_bounds__(kFusedThreads, 1) fused_stack_kernel(const __g
     const FusedLayer& LY = A.layers[l];
     const uint32_t e_logit = base + (uint32_t)l + 1u;
     // ------------------------------------------------------------- A --
-    float xv[8];
+    float xv[NT][8];
     if (l == 0) {
-      float4 v0 = make_float4(0.f, 0.f, 0.f, 0.f), v1 = v0;
-      if (xthr) {
-        v0 = __ldcg(reinterpret_cast<const float4*>(A.xn + tid * 8));
-        v1 = __ldcg(reinterpret_cast<const float4*>(A.xn + tid * 8 + 4));
+#pragma unroll
+      for (int t = 0; t < NT; ++t) {
+        float4 v0 = make_float4(0.f, 0.f, 0.f, 0.f), v1 = v0;
+        if (xthr) {
+          v0 = __ldcg(reinterpret_cast<const float4*>(A.xn + (size_t)t * H + tid * 8));
+          v1 = __ldcg(reinterpret_cast<const float4*>(A.xn + (size_t)t * H + tid * 8 + 4));
+        }
+        xv[t][0] = v0.x; xv[t][1] = v0.y; xv[t][2] = v0.z; xv[t][3] = v0.w;
+        xv[t][4] = v1.x; xv[t][5] = v1.y; xv[t][6] = v1.z; xv[t][7] = v1.w;
       }
-      xv[0] = v0.x; xv[1] = v0.y; xv[2] = v0.z; xv[3] = v0.w;
-      xv[4] = v1.x; xv[5] = v1.y; xv[6] = v1.z; xv[7] = v1.w;
     } else {
       // h' and the sums of squares of the previous layer: every CTA has published them
       if (!cta_cnt_wait(kCntH, (unsigned)l * (unsigned)nC)) { aborted = true; break; }
-      float4 h0 = make_float4(0.f, 0.f, 0.f, 0.f), h1 = h0, w0 = h0, w1 = h0;
+      float4 w0 = make_float4(0.f, 0.f, 0.f, 0.f), w1 = w0;
       const float* wprev = A.layers[l - 1].norm_w;
       if (xthr) {
-        h0 = __ldcg(reinterpret_cast<const float4*>(A.x_h + tid * 8));
-        h1 = __ldcg(reinterpret_cast<const float4*>(A.x_h + tid * 8 + 4));
         w0 = __ldg(reinterpret_cast<const float4*>(wprev + tid * 8));
         w1 = __ldg(reinterpret_cast<const float4*>(wprev + tid * 8 + 4));
       }
-      const float r = norm_scale(tid < nC ? __ldcg(A.x_ss + tid) : 0.f);
-      xv[0] = h0.x * r * w0.x; xv[1] = h0.y * r * w0.y; xv[2] = h0.z * r * w0.z; xv[3] = h0.w * r * w0.w;
-      xv[4] = h1.x * r * w1.x; xv[5] = h1.y * r * w1.y; xv[6] = h1.z * r * w1.z; xv[7] = h1.w * r * w1.w;
+      float4 hv[NT][2];
+#pragma unroll
+      for (int t = 0; t < NT; ++t) {
+        hv[t][0] = hv[t][1] = make_float4(0.f, 0.f, 0.f, 0.f);
+        if (xthr) {
+          hv[t][0] = __ldcg(reinterpret_cast<const float4*>(A.x_h + (size_t)t * kXHStride + tid * 8));
+          hv[t][1] = __ldcg(reinterpret_cast<const float4*>(A.x_h + (size_t)t * kXHStride + tid * 8 + 4));
+        }
+      }
+      float r[NT];
+      norm_scales(r);
+#pragma unroll
+      for (int t = 0; t < NT; ++t) {
+        const float4 h0 = hv[t][0], h1 = hv[t][1];
+        const float rt = r[t];
+        xv[t][0] = h0.x * rt * w0.x; xv[t][1] = h0.y * rt * w0.y; xv[t][2] = h0.z * rt * w0.z;
+        xv[t][3] = h0.w * rt * w0.w; xv[t][4] = h1.x * rt * w1.x; xv[t][5] = h1.y * rt * w1.y;
+        xv[t][6] = h1.z * rt * w1.z; xv[t][7] = h1.w * rt * w1.w;
+      }
     }
     // stage x: 8 consecutive threads share one 64-group
-    stage_unit(xv, xthr, tid >> 3, tid & 7, ngH, sx);
-    // router partial dot products (rows in shared memory), reduced in warp order
+#pragma unroll
+    for (int t = 0; t < NT; ++t) stage_unit(xv[t], xthr, tid >> 3, tid & 7, ngH, sx_of(t));
+    // router partial dot products (rows in shared memory, each read once for
+    // all tokens), reduced in warp order
     if (nr > 0 && !wait_mb(kMbRouter, (uint32_t)l & 1u)) set_abort();
 #pragma unroll
     for (int m = 0; m < kFusedMaxRouterRows; ++m) {
@@ -716,26 +773,30 @@ __global__ void __launch_bounds__(kFusedThreads, 1) fused_stack_kernel(const __g
         wr[0] = as_float4(lds128(rr));
         wr[1] = as_float4(lds128(rr + 4));
       }
-      float d = wr[0].x * xv[0];
-      d = fmaf(wr[0].y, xv[1], d);
-      d = fmaf(wr[0].z, xv[2], d);
-      d = fmaf(wr[0].w, xv[3], d);
-      d = fmaf(wr[1].x, xv[4], d);
-      d = fmaf(wr[1].y, xv[5], d);
-      d = fmaf(wr[1].z, xv[6], d);
-      d = fmaf(wr[1].w, xv[7], d);
-      d = warp_sum(d);
-      if (lane == 0) s_rp[warp][m] = d;
+#pragma unroll
+      for (int t = 0; t < NT; ++t) {
+        float d = wr[0].x * xv[t][0];
+        d = fmaf(wr[0].y, xv[t][1], d);
+        d = fmaf(wr[0].z, xv[t][2], d);
+        d = fmaf(wr[0].w, xv[t][3], d);
+        d = fmaf(wr[1].x, xv[t][4], d);
+        d = fmaf(wr[1].y, xv[t][5], d);
+        d = fmaf(wr[1].z, xv[t][6], d);
+        d = fmaf(wr[1].w, xv[t][7], d);
+        d = warp_sum(d);
+        if (lane == 0) s_rp[warp][t][m] = d;
+      }
     }
     __syncthreads();
     if (warp == 0) {
-      if (tid < nr) {
+      const int t = lane / kFusedMaxRouterRows, m = lane % kFusedMaxRouterRows;
+      if (t < NT && m < nr) {
         float v = 0.f;
-        for (int w = 0; w < kFusedWarps; ++w) v += s_rp[w][tid];
-        const int row = c + tid * nC;
-        if (row < E) A.logits[row] = v;
-        else A.gamma[0] = v = 1.f / (1.f + expf(-v));
-        st_relaxed64(A.x_logit + row, x_word(e_logit, v));
+        for (int w = 0; w < kFusedWarps; ++w) v += s_rp[w][t][m];
+        const int row = c + m * nC;
+        if (row < E) A.logits[(size_t)t * E + row] = v;
+        else A.gamma[t] = v = 1.f / (1.f + expf(-v));
+        st_relaxed64(A.x_logit + (size_t)t * kXLogitStride + row, x_word(e_logit, v));
       }
       __syncwarp();
       if (lane == 0 && nr > 0) cnt_add(A.sync + kCntLogit, (unsigned)nr);
@@ -743,51 +804,74 @@ __global__ void __launch_bounds__(kFusedThreads, 1) fused_stack_kernel(const __g
     // ------------------------------------------------------------- E --
     if (warp < kGuWarps) {
       // ---- gate/up warps ----
-      const XGroup xg = load_xgroup(sx, ngH);
+      // the staged inputs of the token of the first block: the shared block
+      // runs token 0 first, the routed blocks take token tr
+      XGroup xg = load_xgroup(sx_of(S ? 0 : tr), ngH);
       for (int p = 0; p < nseq; ++p) {
         const uint32_t pos = sq + (uint32_t)p;
         const int s = (int)(pos % kSlots);
         const bool ok = wait_mb(kMbFull + s, (pos / kSlots) & 1u);
-        float* gb = gred + (pos & 1u) * (kGuWarps * 8);
+        float* gb = gred + (pos & 1u) * (NT * kGuWarps * 8);
         const uint8_t* sl = smem + P.slot[s];
         if (ok) {
-          if (p < S) block_gateup<SBITS>(sl, H, xg, gb);
-          else block_gateup<BITS>(sl, H, xg, gb);
+          if (p < S) {
+            block_gateup<SBITS>(sl, H, xg, gb);
+#pragma unroll
+            for (int t = 1; t < NT; ++t) {
+              xg = load_xgroup(sx_of(t), ngH);
+              block_gateup<SBITS>(sl, H, xg, gb + t * (kGuWarps * 8));
+            }
+            if (NT > 1 && tr != NT - 1) xg = load_xgroup(sx_of(tr), ngH);
+          } else {
+            block_gateup<BITS>(sl, H, xg, gb);
+          }
         }
         named_bar(kBarGu, kGuThreads);
         if (warp == 0) {
-          uint32_t* dx = dnx + s * kDnxWords;
-          const float a = p < S ? block_swiglu<SBITS>(gb, dx) : block_swiglu<BITS>(gb, dx);
-          __syncwarp();
-          if (lane == 0) mbar_arrive(&mbar[kMbReady + s]);
-          // the SwiGLU outputs to the workspace, after the hand-off (a global
-          // store before the arrive would make it wait for the store)
+          uint32_t* dx = dnx + s * (NT * kDnxWords);
           if (p < S) {
-            if (lane < GS::kW) A.a[(size_t)k * I + (size_t)c * GS::kW + lane] = a;
-          } else if (lane < GR::kW) {
-            A.a[(size_t)jj * I + (size_t)routed_nb(p) * GR::kW + lane] = a;
+            float a[NT];
+#pragma unroll
+            for (int t = 0; t < NT; ++t) a[t] = block_swiglu<SBITS>(gb + t * (kGuWarps * 8), dx + t * kDnxWords);
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&mbar[kMbReady + s]);
+            // the SwiGLU outputs to the workspace, after the hand-off (a global
+            // store before the arrive would make it wait for the store)
+#pragma unroll
+            for (int t = 0; t < NT; ++t)
+              if (lane < GS::kW) A.a[((size_t)t * (k + 1) + k) * I + (size_t)c * GS::kW + lane] = a[t];
+          } else {
+            const float a = block_swiglu<BITS>(gb, dx);
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&mbar[kMbReady + s]);
+            if (lane < GR::kW) A.a[((size_t)tr * (k + 1) + jj) * I + (size_t)routed_nb(p) * GR::kW + lane] = a;
           }
         }
       }
     } else {
-      // ---- down warps: routing first ----
+      // ---- down warps: routing first (token tr's top-k; every token's gamma) ----
       int rid;      // the selected expert of this CTA's routed group
       float wt_r;   // its gate weight
       {
         // every CTA has published its router rows: (l + 1) (E + 1) in all
         if (issuer && !cnt_wait<false>(A.sync + kCntLogit, (unsigned)(l + 1) * (unsigned)(E + 1))) set_abort();
         named_bar(kBarDn, kDnThreads);
+        const uint64_t* xl_tr = A.x_logit + (size_t)tr * kXLogitStride;
         uint64_t lw[kDnKeys + 1];
 #pragma unroll
         for (int i = 0; i < kDnKeys; ++i) {
           const int e = td + i * kDnThreads;
-          lw[i] = e < E ? ld_relaxed64(A.x_logit + e) : 0;
+          lw[i] = e < E ? ld_relaxed64(xl_tr + e) : 0;
         }
-        lw[kDnKeys] = td == 0 ? ld_relaxed64(A.x_logit + E) : 0;
-        if (!x_settle(lw, e_logit, [&](int i) { return A.x_logit + (i < kDnKeys ? td + i * kDnThreads : E); },
-                      [&](int i) { return i < kDnKeys ? td + i * kDnThreads < E : td == 0; }))
+        lw[kDnKeys] = td < NT ? ld_relaxed64(A.x_logit + (size_t)td * kXLogitStride + E) : 0;
+        if (!x_settle(lw, e_logit,
+                      [&](int i) {
+                        return i < kDnKeys ? xl_tr + td + i * kDnThreads
+                                           : A.x_logit + (size_t)td * kXLogitStride + E;
+                      },
+                      [&](int i) { return i < kDnKeys ? td + i * kDnThreads < E : td < NT; }))
           set_abort();
-        if (td == 0) s_gamma = x_value(lw[kDnKeys]);
+        if (td < NT) s_gamma[td] = x_value(lw[kDnKeys]);
         uint64_t key[kDnKeys];
         bool nan_seen = false;
 #pragma unroll
@@ -826,10 +910,10 @@ __global__ void __launch_bounds__(kFusedThreads, 1) fused_stack_kernel(const __g
         const float pw = z > 0.f ? pe / z : 0.f;
         rid = __shfl_sync(0xffffffffu, sel, jj);
         wt_r = __shfl_sync(0xffffffffu, pw, jj);
-        if (c == 0 && dw == 0) {
+        if (route_writer && dw == 0) {
           if (lane < k) {
-            A.ids[lane] = sel;
-            A.weights[lane] = pw;
+            A.ids[(size_t)tr * k + lane] = sel;
+            A.weights[(size_t)tr * k + lane] = pw;
           }
           if (lane == 0 && s_nan) raise_status(FMOE_STATUS_NAN_LOGIT);
         }
@@ -845,13 +929,21 @@ __global__ void __launch_bounds__(kFusedThreads, 1) fused_stack_kernel(const __g
           if (S && l + 1 < A.n_layers && nseq < kSlots) issue_pos(l + 1, sq + (uint32_t)nseq, 0, 0);
         }
       }
+      // the other tokens' partial outputs of a CTA without a shared block: zero
+      if (NT > 1 && !S) {
+        float zr[kDnRowsT];
+#pragma unroll
+        for (int m = 0; m < kDnRowsT; ++m) zr[m] = 0.f;
+#pragma unroll
+        for (int t = 0; t < NT; ++t)
+          if (t != tr) store_rows(A.x_part + (size_t)t * kXPartStride + (size_t)c * H, zr);
+      }
       // ---- down products, block by block ----
-      float yacc[kDnRowsT];  // this CTA's partial output rows
+      float yacc[kDnRowsT];  // the shared block's contribution to token tr
       float uacc[kDnRowsT];  // routed blocks: sum of step * weight * value, scaled per row at the end
 #pragma unroll
       for (int m = 0; m < kDnRowsT; ++m) yacc[m] = uacc[m] = 0.f;
       float p2sum = 0.f;  // routed blocks: sum of step * weight * sum xi (times the row's bias at the end)
-      const float wt_s = s_gamma;
       for (int p = 0; p < nseq; ++p) {
         const uint32_t pos = sq + (uint32_t)p;
         const int s = (int)(pos % kSlots);
@@ -860,23 +952,34 @@ __global__ void __launch_bounds__(kFusedThreads, 1) fused_stack_kernel(const __g
         if (p == 0 && S) ok = ok && wait_mb(kMbSbShared, (uint32_t)l & 1u);
         if (ok) {
           const uint8_t* sl = smem + P.slot[s];
-          const uint32_t* dx = dnx + s * kDnxWords;
+          const uint32_t* dx = dnx + s * (NT * kDnxWords);
           float t[kDnRowsT];
           if (p < S) {
-            block_down<SBITS>(sl, dx, H, t);
-            const float p1 = wt_s * __uint_as_float(dx[12]), p2 = wt_s * __uint_as_float(dx[13]);
+            // the shared block: every token's down products from the same codes
             const uint32_t* sbe = reinterpret_cast<const uint32_t*>(smem + P.sbe[0]);
 #pragma unroll
-            for (int m = 0; m < kDnQuads; ++m) {
-              const int row = 4 * (td + kDnThreads * m);
-              if (row < H) {
-                const uint4 sb = lds128(sbe + row);
+            for (int tk = 0; tk < NT; ++tk) {
+              const uint32_t* dxt = dx + tk * kDnxWords;
+              block_down<SBITS>(sl, dxt, H, t);
+              const float p1 = s_gamma[tk] * __uint_as_float(dxt[12]), p2 = s_gamma[tk] * __uint_as_float(dxt[13]);
+              float v[kDnRowsT];
+#pragma unroll
+              for (int mq = 0; mq < kDnQuads; ++mq) {
+                const int row = 4 * (td + kDnThreads * mq);
+                uint4 sb = make_uint4(0u, 0u, 0u, 0u);
+                if (row < H) sb = lds128(sbe + row);
                 const uint32_t sw[4] = {sb.x, sb.y, sb.z, sb.w};
 #pragma unroll
                 for (int r = 0; r < 4; ++r) {
                   const float sc = __uint_as_float(sw[r] << 16), bi = __uint_as_float(sw[r] & 0xFFFF0000u);
-                  yacc[4 * m + r] = fmaf(sc, p1 * t[4 * m + r], fmaf(bi, p2, yacc[4 * m + r]));
+                  v[4 * mq + r] = fmaf(sc, p1 * t[4 * mq + r], bi * p2);
                 }
+              }
+              if (tk == tr) {
+#pragma unroll
+                for (int mm = 0; mm < kDnRowsT; ++mm) yacc[mm] = v[mm];
+              } else {
+                store_rows(A.x_part + (size_t)tk * kXPartStride + (size_t)c * H, v);
               }
             }
           } else {
@@ -884,7 +987,7 @@ __global__ void __launch_bounds__(kFusedThreads, 1) fused_stack_kernel(const __g
             const float p1 = wt_r * __uint_as_float(dx[12]);
             p2sum = fmaf(wt_r, __uint_as_float(dx[13]), p2sum);
 #pragma unroll
-            for (int m = 0; m < kDnRowsT; ++m) uacc[m] = fmaf(p1, t[m], uacc[m]);
+            for (int mm = 0; mm < kDnRowsT; ++mm) uacc[mm] = fmaf(p1, t[mm], uacc[mm]);
           }
         }
         named_bar(kBarDn, kDnThreads);  // every down thread is done with the slot
@@ -901,11 +1004,11 @@ __global__ void __launch_bounds__(kFusedThreads, 1) fused_stack_kernel(const __g
       }
       // every block of the layer is done: the next layer's router rows come in
       if (l + 1 < A.n_layers && !s_abort) issue_router(l + 1, sq + (uint32_t)nseq);
-      // ---- F: routed blocks scaled per row, partial output out ----
+      // ---- F: routed blocks scaled per row, token tr's partial output out ----
       bool ok = true;
       if (nq > 0) ok = wait_mb(kMbSbRouted, (uint32_t)l & 1u);
       const uint32_t* sbe = reinterpret_cast<const uint32_t*>(smem + P.sbe[1]);
-      float* part = A.x_part + (size_t)c * H;
+      float* part = A.x_part + (size_t)tr * kXPartStride + (size_t)c * H;
 #pragma unroll
       for (int m = 0; m < kDnQuads; ++m) {
         const int row = 4 * (td + kDnThreads * m);
@@ -933,39 +1036,49 @@ __global__ void __launch_bounds__(kFusedThreads, 1) fused_stack_kernel(const __g
     if (__syncthreads_or(s_abort)) { aborted = true; break; }
     // ------------------------------------------------------------- G --
     {
-      // rows i0 + r, r < nd: ngr threads per row each sum every ngr-th CTA's
-      // partial; then one thread per row adds those sums in order
-      const int nd = i1 - i0;
-      const int ngr = nd > 0 ? kFusedThreads / nd : 0;
-      const int r = nd > 0 ? tid % nd : 0, pg = nd > 0 ? tid / nd : kFusedThreads;
-      const float hres = tid < nd ? A.h[i0 + tid] : 0.f;  // this CTA's own rows
+      // values q = t nd + r (token t, row i0 + r), q < nv: ngr threads per
+      // value each sum every ngr-th CTA's partial; then warp 0 adds those
+      // sums in order (lane r: row i0 + r of every token)
+      const int nd = i1 - i0, nv = NT * nd;
+      const int ngr = nv > 0 ? kFusedThreads / nv : 0;
+      const int q = nv > 0 ? tid % nv : 0, pg = nv > 0 ? tid / nv : kFusedThreads;
+      const int tq = nd > 0 ? q / nd : 0, r = nd > 0 ? q % nd : 0;
+      float hres[NT];  // this CTA's own rows
+#pragma unroll
+      for (int t = 0; t < NT; ++t) hres[t] = tid < nd ? A.h[(size_t)t * H + i0 + tid] : 0.f;
       if (!cta_cnt_wait(kCntPart, (unsigned)(l + 1) * (unsigned)nC)) { aborted = true; break; }
       float* sred = reinterpret_cast<float*>(smem + P.red);
       if (pg < ngr) {
-        constexpr int kLoads = (kFusedMaxCtas * 32 + kFusedThreads - 1) / kFusedThreads;  // ngr >= 512 / 32
+        // ngr >= kFusedThreads / (32 NT)
+        constexpr int kLoads = (kFusedMaxCtas * 32 * NT + kFusedThreads - 1) / kFusedThreads;
+        const float* src = A.x_part + (size_t)tq * kXPartStride + i0 + r;
         float v[kLoads];
 #pragma unroll
         for (int t2 = 0; t2 < kLoads; ++t2) {
           const int p = pg + t2 * ngr;
-          v[t2] = p < nC ? __ldcg(A.x_part + (size_t)p * H + i0 + r) : 0.f;
+          v[t2] = p < nC ? __ldcg(src + (size_t)p * H) : 0.f;
         }
         float acc = 0.f;
 #pragma unroll
         for (int t2 = 0; t2 < kLoads; ++t2) acc += v[t2];
-        sred[pg * nd + r] = acc;
+        sred[pg * nv + q] = acc;
       }
       __syncthreads();
-      float ss = 0.f;
-      if (tid < nd) {
-        float v = hres;
-        for (int g = 0; g < ngr; ++g) v += sred[g * nd + tid];
-        A.h[i0 + tid] = v;
-        __stcg(A.x_h + i0 + tid, v);
-        ss = v * v;
-      }
       if (warp == 0) {
-        ss = warp_sum(ss);
-        if (lane == 0) __stcg(A.x_ss + c, ss);
+        float ss[NT];
+#pragma unroll
+        for (int t = 0; t < NT; ++t) {
+          ss[t] = 0.f;
+          if (tid < nd) {
+            float v = hres[t];
+            for (int g = 0; g < ngr; ++g) v += sred[g * nv + t * nd + tid];
+            A.h[(size_t)t * H + i0 + tid] = v;
+            __stcg(A.x_h + (size_t)t * kXHStride + i0 + tid, v);
+            ss[t] = v * v;
+          }
+          ss[t] = warp_sum(ss[t]);
+          if (lane == 0) __stcg(A.x_ss + (size_t)t * kXSsStride + c, ss[t]);
+        }
         __syncwarp();
         if (lane == 0) cnt_release_add(A.sync + kCntH, 1u);  // warp 0 wrote every row of this CTA (nd <= 32)
       }
@@ -977,9 +1090,14 @@ __global__ void __launch_bounds__(kFusedThreads, 1) fused_stack_kernel(const __g
   if (done) done = cta_cnt_wait(kCntH, (unsigned)A.n_layers * (unsigned)nC);
   if (done) {
     // epilogue: xn' of the last layer for this CTA's rows (h' written by this CTA)
-    const float r_last = norm_scale(tid < nC ? __ldcg(A.x_ss + tid) : 0.f);
+    float r_last[NT];
+    norm_scales(r_last);
     const float* w = A.layers[A.n_layers - 1].norm_w;
-    if (tid < i1 - i0) A.xn[i0 + tid] = A.h[i0 + tid] * r_last * w[i0 + tid];
+    if (tid < i1 - i0) {
+#pragma unroll
+      for (int t = 0; t < NT; ++t)
+        A.xn[(size_t)t * H + i0 + tid] = A.h[(size_t)t * H + i0 + tid] * r_last[t] * w[i0 + tid];
+    }
     __syncthreads();
     if (tid == 0) {
       __threadfence();
@@ -1004,10 +1122,11 @@ __global__ void __launch_bounds__(kFusedThreads, 1) fused_stack_kernel(const __g
   }
 }
 
-// Host-side plan: shared-memory layout for n_ctas CTAs; false if the shape
-// does not fit the kernel.
-inline bool fused_plan(int H, int I, int E, int k, int bits, int sbits, int n_ctas, size_t max_smem,
+// Host-side plan: shared-memory layout for n_ctas CTAs and nt tokens per
+// launch; false if the shape does not fit the kernel.
+inline bool fused_plan(int H, int I, int E, int k, int bits, int sbits, int nt, int n_ctas, size_t max_smem,
                        FusedPlan* out) {
+  if (nt < 1 || nt > kFusedMaxNT) return false;
   if (H < 64 || H % 64 || I < 64 || I % 64 || H > kFusedMaxH) return false;
   if (E < 1 || E > kFusedMaxE || k < 1 || k > kFusedMaxK || k > E) return false;
   if (n_ctas < 1 || n_ctas > kFusedMaxCtas) return false;
@@ -1015,7 +1134,7 @@ inline bool fused_plan(int H, int I, int E, int k, int bits, int sbits, int n_ct
   auto wn = [](int b) { return 32 / b; };
   const int nbs = I / wn(sbits);
   if (nbs > n_ctas) return false;        // one shared block per CTA at most
-  if (k * (I / 64) > n_ctas) return false;  // one routed 64-group per CTA at most
+  if (nt * k * (I / 64) > n_ctas) return false;  // one routed 64-group per CTA at most
   if ((H + n_ctas - 1) / n_ctas > 32) return false;  // rows per CTA in the final sums: one warp
   auto blk = [&](int b) -> long long { return 12LL * H + (long long)wn(b) * 2 * (H / 64) * 4; };
   const long long slot = blk(bits) > blk(sbits) ? blk(bits) : blk(sbits);
@@ -1031,15 +1150,16 @@ inline bool fused_plan(int H, int I, int E, int k, int bits, int sbits, int n_ct
     o = al(o + 4LL * H);
   }
   p.xs = (uint32_t)o;
-  o = al(o + (long long)staged_x_bytes(H));
+  p.xs_stride = (uint32_t)al((long long)staged_x_bytes(H));
+  o = al(o + (long long)nt * p.xs_stride);
   p.logit = (uint32_t)o;
   o = al(o + 4LL * E);
   p.cand = (uint32_t)o;
   o = al(o + 8LL * (kDnWarps * kFusedMaxK + 1));
   p.gred = (uint32_t)o;
-  o = al(o + 4LL * 2 * kGuWarps * 8);
+  o = al(o + 4LL * 2 * nt * kGuWarps * 8);
   p.dnx = (uint32_t)o;
-  o = al(o + 4LL * kSlots * kDnxWords);
+  o = al(o + 4LL * kSlots * nt * kDnxWords);
   p.red = (uint32_t)o;
   o = al(o + 4LL * kFusedThreads);
   p.mbar = (uint32_t)o;

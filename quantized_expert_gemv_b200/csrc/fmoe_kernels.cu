@@ -578,17 +578,17 @@ static WsLayout ws_layout(int H, int I, int E, int k, int T) {
   WsLayout w;
   w.sync = 0;  // grid-barrier counter, exit counter and epoch of the fused kernel
   // exchange buffers of the fused kernel (logit exchange words, fp32
-  // partial outputs and h'), at offsets and sizes that do not depend on the
-  // shape or T: no other kernel writes there
+  // partial outputs and h', for up to kFusedMaxNT tokens), at offsets and
+  // sizes that do not depend on the shape or T: no other kernel writes there
   size_t o = 4096;
   w.x_logit = o;
-  o = align_up(o + (size_t)(kFusedMaxE + 1) * 8, 256);
+  o = align_up(o + (size_t)kFusedMaxNT * kXLogitStride * 8, 256);
   w.x_ss = o;
-  o = align_up(o + (size_t)kFusedMaxCtas * 4, 256);
+  o = align_up(o + (size_t)kFusedMaxNT * kXSsStride * 4, 256);
   w.x_h = o;
-  o = align_up(o + (size_t)kFusedMaxH * 4, 256);
+  o = align_up(o + (size_t)kFusedMaxNT * kXHStride * 4, 256);
   w.x_part = o;
-  o = align_up(o + (size_t)kFusedMaxCtas * kFusedMaxH * 4, 256);
+  o = align_up(o + (size_t)kFusedMaxNT * kXPartStride * 4, 256);
   // expert groups of the T > 1 path
   w.grp = o;
   w.g_count = o;
@@ -856,10 +856,10 @@ static int launch_combine(const float* y, const float* weights, const float* gam
 
 // ----------------------------------------------------- fused batch-1 path --
 static int g_fused_enabled = 1;
-// Token counts up to which T > 1 runs as one persistent launch per token
-// (measured: a layer of T = 2 / 4 / 8 tokens takes 77 / 138 / 197 us on the
-// grouped path against 21.4 us per token and layer in a stack launch; a
-// single-layer launch costs ~30 us).
+// Token counts up to which T > 1 runs through the persistent kernel, two
+// tokens per launch (measured: a layer of T = 2 / 4 / 8 tokens takes
+// 77 / 138 / 197 us on the grouped path against 21.4 us per token and layer
+// in a one-token stack launch; a single-layer launch costs ~30 us).
 constexpr int kFusedTokensLayer = 4;
 constexpr int kFusedTokensStack = 8;
 
@@ -867,6 +867,9 @@ struct FusedConfig {
   bool ok;
   int n_sm;
   FusedPlan plan;
+};
+struct FusedConfigs {
+  FusedConfig nt[kFusedMaxNT + 1];  // by tokens per launch (index 0 unused)
 };
 
 static bool same_desc(const fmoe_layer_desc& a, const fmoe_layer_desc& b);
@@ -876,34 +879,40 @@ static bool same_desc(const fmoe_layer_desc& a, const fmoe_layer_desc& b);
 struct FusedCacheEntry {
   bool valid;
   fmoe_layer_desc desc;
-  FusedConfig fc;
+  FusedConfigs fc;
 };
 static FusedCacheEntry g_fused_cache[64];
 
-static FusedConfig fused_config_uncached(const fmoe_layer_desc& d, int dev);
+static FusedConfig fused_config_uncached(const fmoe_layer_desc& d, int dev, int nt);
 
-static FusedConfig fused_config(const fmoe_layer_desc& d) {
+// The configuration of the persistent kernel for nt tokens per launch.
+static FusedConfig fused_config(const fmoe_layer_desc& d, int nt = 1) {
   int dev = 0;
+  if (nt < 1 || nt > kFusedMaxNT) return FusedConfig{};
   if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return FusedConfig{};
   FusedCacheEntry& e = g_fused_cache[dev];
-  if (e.valid && same_desc(e.desc, d)) return e.fc;
-  const FusedConfig fc = fused_config_uncached(d, dev);
-  e.desc = d;
-  e.fc = fc;
-  e.valid = true;
-  return fc;
+  if (!(e.valid && same_desc(e.desc, d))) {
+    for (int n = 1; n <= kFusedMaxNT; ++n) e.fc.nt[n] = fused_config_uncached(d, dev, n);
+    e.desc = d;
+    e.valid = true;
+  }
+  return e.fc.nt[nt];
 }
 
-// The fused kernel instantiation for a pair of code widths.
-static const void* fused_kernel_for(int bits, int sbits) {
-  if (bits == 4 && sbits == 4) return reinterpret_cast<const void*>(&fused_stack_kernel<4, 4>);
-  if (bits == 2 && sbits == 4) return reinterpret_cast<const void*>(&fused_stack_kernel<2, 4>);
-  if (bits == 2 && sbits == 2) return reinterpret_cast<const void*>(&fused_stack_kernel<2, 2>);
-  if (bits == 4 && sbits == 2) return reinterpret_cast<const void*>(&fused_stack_kernel<4, 2>);
+// The fused kernel instantiation for a pair of code widths and nt tokens per
+// launch (two tokens: 4-bit codes, whose slots leave room for two tokens'
+// staged inputs).
+static const void* fused_kernel_for(int bits, int sbits, int nt) {
+  if (nt == 2) return bits == 4 && sbits == 4 ? reinterpret_cast<const void*>(&fused_stack_kernel<4, 4, 2>) : nullptr;
+  if (nt != 1) return nullptr;
+  if (bits == 4 && sbits == 4) return reinterpret_cast<const void*>(&fused_stack_kernel<4, 4, 1>);
+  if (bits == 2 && sbits == 4) return reinterpret_cast<const void*>(&fused_stack_kernel<2, 4, 1>);
+  if (bits == 2 && sbits == 2) return reinterpret_cast<const void*>(&fused_stack_kernel<2, 2, 1>);
+  if (bits == 4 && sbits == 2) return reinterpret_cast<const void*>(&fused_stack_kernel<4, 2, 1>);
   return nullptr;
 }
 
-static FusedConfig fused_config_uncached(const fmoe_layer_desc& d, int dev) {
+static FusedConfig fused_config_uncached(const fmoe_layer_desc& d, int dev, int nt) {
   FusedConfig fc{};
   int n_sm = 0, optin = 0;
   if (cudaDeviceGetAttribute(&n_sm, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess) return fc;
@@ -911,9 +920,9 @@ static FusedConfig fused_config_uncached(const fmoe_layer_desc& d, int dev) {
   if (n_sm < 1) return fc;
   if (n_sm > kFusedMaxCtas) n_sm = kFusedMaxCtas;  // one CTA per SM, at most kFusedMaxCtas of them
   const size_t max_dyn = optin > 2048 ? (size_t)optin - 1024 : 0;
-  if (!fused_plan(d.hidden, d.inter, d.n_experts, d.top_k, d.bits, d.shared_bits, n_sm, max_dyn, &fc.plan))
+  if (!fused_plan(d.hidden, d.inter, d.n_experts, d.top_k, d.bits, d.shared_bits, nt, n_sm, max_dyn, &fc.plan))
     return fc;
-  const void* kfn = fused_kernel_for(d.bits, d.shared_bits);
+  const void* kfn = fused_kernel_for(d.bits, d.shared_bits, nt);
   if (!kfn) return fc;
   if (cudaFuncSetAttribute(kfn, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)fc.plan.total) != cudaSuccess)
     return fc;
@@ -931,17 +940,18 @@ static bool same_desc(const fmoe_layer_desc& a, const fmoe_layer_desc& b) {
          a.bits == b.bits && a.shared_bits == b.shared_bits && a.group == b.group && a.eps == b.eps;
 }
 
-// Runs n_layers layers of one token with the persistent kernel: token t of
-// a T-token workspace (its rows of the logits, ids, weights, gamma and a
-// intermediates; h and xn point at the token's own row).  Returns
-// FMOE_ERR_UNSUPPORTED when the configuration does not fit it.
+// Runs n_layers layers of nt tokens with the persistent kernel: tokens
+// t .. t + nt - 1 of a T-token workspace (their rows of the logits, ids,
+// weights, gamma and a intermediates; h and xn point at token t's row, the
+// others follow).  Returns FMOE_ERR_UNSUPPORTED when the configuration does
+// not fit it.
 static int launch_fused(const fmoe_layer_weights* layers, int n_layers, float* h, float* xn, void* ws,
-                        size_t ws_bytes, cudaStream_t st, int T = 1, int t = 0) {
+                        size_t ws_bytes, cudaStream_t st, int T = 1, int t = 0, int nt = 1) {
   const fmoe_layer_desc& d = layers[0].desc;
-  const FusedConfig fc = fused_config(d);
+  const FusedConfig fc = fused_config(d, nt);
   if (!fc.ok) return FMOE_ERR_UNSUPPORTED;
   const WsLayout w = ws_layout(d.hidden, d.inter, d.n_experts, d.top_k, T);
-  if (ws_bytes < w.bytes || t < 0 || t >= T) return FMOE_ERR_BUFFER_TOO_SMALL;
+  if (ws_bytes < w.bytes || t < 0 || t + nt > T) return FMOE_ERR_BUFFER_TOO_SMALL;
   unsigned char* base = static_cast<unsigned char*>(ws);
   FusedArgs args;
   std::memset(&args, 0, sizeof(args));
@@ -985,8 +995,27 @@ static int launch_fused(const fmoe_layer_weights* layers, int n_layers, float* h
     cfg.attrs = attr;
     cfg.numAttrs = 1;
     void* kargs[] = {&args};
-    const cudaError_t e = cudaLaunchKernelExC(&cfg, fused_kernel_for(d.bits, d.shared_bits), kargs);
+    const cudaError_t e = cudaLaunchKernelExC(&cfg, fused_kernel_for(d.bits, d.shared_bits, nt), kargs);
     if (e != cudaSuccess) return FMOE_ERR_CUDA;
+  }
+  return FMOE_OK;
+}
+
+// T tokens (rows of h and xn) through n_layers layers: launches of two
+// tokens where the kernel supports them, one token otherwise.
+// FMOE_ERR_UNSUPPORTED (nothing launched) when the one-token kernel does not
+// fit the shape.
+static int launch_fused_tokens(const fmoe_layer_weights* layers, int n_layers, float* h, float* xn, int T,
+                               void* ws, size_t ws_bytes, cudaStream_t st) {
+  const fmoe_layer_desc& d = layers[0].desc;
+  if (!fused_config(d, 1).ok) return FMOE_ERR_UNSUPPORTED;
+  const bool pairs = fused_config(d, 2).ok;
+  const size_t H = (size_t)d.hidden;
+  for (int t = 0; t < T;) {
+    const int nt = pairs && T - t >= 2 ? 2 : 1;
+    const int rc = launch_fused(layers, n_layers, h + t * H, xn + t * H, ws, ws_bytes, st, T, t, nt);
+    if (rc != FMOE_OK) return rc;
+    t += nt;
   }
   return FMOE_OK;
 }
@@ -1017,14 +1046,10 @@ static int layer_forward_impl(const fmoe_layer_weights* lw, const float* logits_
   const WsLayout w = ws_layout(d.hidden, d.inter, d.n_experts, d.top_k, T);
   if (ws_bytes < w.bytes) return FMOE_ERR_BUFFER_TOO_SMALL;
   if (T <= kFusedTokensLayer && !logits_in && g_fused_enabled) {
-    // a few tokens: one persistent launch per token is faster than the
-    // grouped path's sequence of launches (rows are independent tokens)
-    for (int t = 0; t < T; ++t) {
-      rc = launch_fused(lw, 1, h + (size_t)t * d.hidden, xn + (size_t)t * d.hidden, ws, ws_bytes, st, T, t);
-      if (rc == FMOE_ERR_UNSUPPORTED && t == 0) break;
-      if (rc != FMOE_OK) return rc;
-      if (t == T - 1) return FMOE_OK;
-    }
+    // a few tokens: persistent launches of two tokens (one for an odd last
+    // token) are faster than the grouped path's sequence of launches
+    rc = launch_fused_tokens(lw, 1, h, xn, T, ws, ws_bytes, st);
+    if (rc != FMOE_ERR_UNSUPPORTED) return rc;
   }
   unsigned char* base = static_cast<unsigned char*>(ws);
   float* part = reinterpret_cast<float*>(base + w.part);
@@ -1249,17 +1274,10 @@ extern "C" int fmoe_stack_forward(const fmoe_layer_weights* layers, int n_layers
     if (!d_h || !d_xn || !d_ws || !aligned16(d_h) || !aligned16(d_xn) || !aligned16(d_ws))
       return FMOE_ERR_INVALID_ARG;
     if (uniform) {
-      // each token through the whole stack in one persistent launch (rows
-      // are independent tokens); up to kFusedTokensStack tokens this beats
-      // the grouped path layer by layer
-      const int H = layers[0].desc.hidden;
-      for (int t = 0; t < T; ++t) {
-        const int rc = launch_fused(layers, n_layers, d_h + (size_t)t * H, d_xn + (size_t)t * H, d_ws, ws_bytes,
-                                    stream, T, t);
-        if (rc == FMOE_ERR_UNSUPPORTED && t == 0) break;
-        if (rc != FMOE_OK) return rc;
-        if (t == T - 1) return FMOE_OK;
-      }
+      // the tokens through the whole stack, two per persistent launch; up to
+      // kFusedTokensStack tokens this beats the grouped path layer by layer
+      const int rc = launch_fused_tokens(layers, n_layers, d_h, d_xn, T, d_ws, ws_bytes, stream);
+      if (rc != FMOE_ERR_UNSUPPORTED) return rc;
     }
   }
   for (int l = 0; l < n_layers; ++l) {

@@ -3,7 +3,8 @@
 Twenty resident layers of hidden 4096 / inter 1024 / 512 experts (int4, and
 2-bit routed experts with a 4-bit shared expert) decode a few tokens: one
 token through the stack, the next token starting from the previous token's
-final xn' (h = xn = xn').  Three checks:
+final xn' (h = xn = xn'); and 2 or 4 independent tokens at once (two per
+persistent launch).  Three checks:
 
   - the stack entry point (one persistent launch over the 20 layers, as the
     benchmark runs it) gives the bits of the 20 single-layer launches;
@@ -84,6 +85,36 @@ def decode_on_device(wl, lws, n_tokens, stream):
         tok = layers[-1]["xn"].copy()
     assert fm.fmoe_read_status() == 0
     return x0, recs
+
+
+VIEWS = (("logits", fm.WS_LOGITS), ("ids", fm.WS_IDS), ("p", fm.WS_WEIGHTS), ("gamma", fm.WS_GAMMA),
+         ("a", fm.WS_A))
+
+
+def decode_batch_on_device(wl, lws, T, stream):
+    """T independent tokens layer by layer (fmoe_layer_forward with T rows:
+    persistent launches of two tokens), recording every layer's inputs,
+    outputs and intermediates per token; then fmoe_stack_forward on the same
+    tokens, which must give the same bits."""
+    desc = lws[0].desc
+    ws = fm.alloc_workspace(desc, T)
+    x = synth.tokens(wl, T, stream=stream)
+    h, xn = dev(x), dev(x)
+    recs = [[] for _ in range(T)]
+    for l in range(N_LAYERS):
+        h_in, xn_in = host(h), host(xn)
+        fm.fmoe_layer_forward(lws[l], h, xn, ws)
+        v = {name: host(fm.workspace_view(ws, desc, T, which)) for name, which in VIEWS}
+        h_out, xn_out = host(h), host(xn)
+        for t in range(T):
+            recs[t].append(dict(h_in=h_in[t], xn_in=xn_in[t], h=h_out[t], xn=xn_out[t],
+                                **{name: v[name][t] for name, _ in VIEWS}))
+    h2, xn2 = dev(x), dev(x)
+    fm.fmoe_stack_forward(lws, h2, xn2, fm.alloc_workspace(desc, T))
+    assert np.array_equal(host(h2), host(h)), "stack h' differs from the layer calls"
+    assert np.array_equal(host(xn2), host(xn)), "stack xn' differs from the layer calls"
+    assert fm.fmoe_read_status() == 0
+    return x, recs
 
 
 def teacher_forced(wl, rec, layer, label):
@@ -172,6 +203,29 @@ def test_stack_20_layers_int4_full_size(stack_int4):
     wl, lws = stack_int4
     assert fm.fmoe_fused_supported(lws[0].desc)
     run_chain_checks(wl, lws, 3, stream=81)
+
+
+@pytest.mark.parametrize("T", [2, 4])
+def test_stack_20_layers_int4_few_tokens(stack_int4, T):
+    """T independent tokens (two per persistent launch) through the twenty
+    int4 layers: every layer of every token teacher-forced against the
+    oracle, the stack against the layer calls bit for bit, and each token's
+    free-running fp64 chain."""
+    wl, lws = stack_int4
+    x, recs = decode_batch_on_device(wl, lws, T, stream=83 + T)
+    jobs = [(t, l) for t in range(T) for l in range(N_LAYERS)]
+    near = []
+
+    def job(i):
+        if i >= len(jobs):
+            t = i - len(jobs)
+            near.extend(free_running(wl, x[t], [recs[t]]))
+            return
+        t, l = jobs[i]
+        teacher_forced(wl, recs[t][l], l, f"T={T} token {t} layer {l}")
+
+    pmap(job, range(len(jobs) + T))
+    print(f"near ties adopted by the free-running oracle: {len(near)} {near}")
 
 
 @pytest.fixture(scope="module")

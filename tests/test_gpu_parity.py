@@ -430,39 +430,65 @@ def test_batched_full_size_int2_every_item_size(wl, tc_path):
     assert fm.fmoe_read_status() == 0
 
 
+def _run(lws, x, stack):
+    h, xn = dev(x), dev(x)
+    ws = fm.alloc_workspace(lws[0].desc, len(x))
+    if stack:
+        fm.fmoe_stack_forward(lws, h, xn, ws)
+    else:
+        fm.fmoe_layer_forward(lws[0], h, xn, ws)
+    return host(h), host(xn), ws
+
+
 @pytest.mark.parametrize("wl", [synth.TINY, SMALL], ids=["tiny4", "small4"])
-def test_few_tokens_run_token_by_token(wl):
-    """Up to fmoe_fused_max_tokens tokens, a layer call and a stack call give
-    each token exactly the bits of a T = 1 call on that token; one token
-    more takes the grouped path and agrees within the tolerance."""
+def test_few_tokens_through_persistent_kernel(wl):
+    """Up to fmoe_fused_max_tokens tokens run through the persistent kernel,
+    two per launch (4-bit layers): every token of a layer call against the
+    oracle; a stack call gives the bits of the same tokens through layer
+    calls; a token's bits do not depend on its partner in the pair; an odd
+    last token gets the bits of a T = 1 call; one token more than the
+    maximum takes the grouped path and agrees within the tolerance."""
     if not fm.fmoe_fused_supported(device_layer(wl).desc):
         pytest.skip("persistent kernel does not fit this shape here")
-    lws = [device_layer(wl, l) for l in range(3)]
-    for stack, T in ((False, fm.fmoe_fused_max_tokens(False)), (True, fm.fmoe_fused_max_tokens(True))):
-        x = synth.tokens(wl, T + 1, stream=61)
-        want = []
+    n_layers = 3
+    lws = [device_layer(wl, l) for l in range(n_layers)]
+    los = [oracle_layer(wl, l) for l in range(n_layers)]
+    Tl, Ts = fm.fmoe_fused_max_tokens(False), fm.fmoe_fused_max_tokens(True)
+    x = synth.tokens(wl, Ts + 2, stream=61)
+    # layer calls of Tl tokens (pairs), chained over the layers, each against the oracle
+    h, xn = dev(x[:Tl]), dev(x[:Tl])
+    ws = fm.alloc_workspace(lws[0].desc, Tl)
+    for l in range(n_layers):
+        h_in, xn_in = host(h), host(xn)
+        fm.fmoe_layer_forward(lws[l], h, xn, ws)
+        for t in range(Tl):
+            check_layer_token(wl, los[l], ws, lws[l].desc, Tl, t, h_in[t], xn_in[t], host(h)[t], host(xn)[t],
+                              f"layer {l} t={t}")
+    layered = (host(h), host(xn))
+    # the stack over the same tokens: the bits of the layer calls
+    sh, sxn, _ = _run(lws, x[:Tl], stack=True)
+    assert np.array_equal(sh, layered[0]) and np.array_equal(sxn, layered[1])
+    for stack in (False, True):
+        T = Ts if stack else Tl
+        got_h, got_xn, _ = _run(lws, x[:T], stack)
+        # partner independence: token 0 paired with token T instead of token 1
+        xp = x[:T].copy()
+        xp[1] = x[T]
+        ph, pxn, _ = _run(lws, xp, stack)
+        assert np.array_equal(ph[0], got_h[0]) and np.array_equal(pxn[0], got_xn[0]), stack
+        assert not np.array_equal(pxn[1], got_xn[1])
+        one = [_run(lws, x[t:t + 1], stack) for t in range(T + 1)]
+        # an odd last token runs alone: the bits of a T = 1 call
+        oh, oxn, _ = _run(lws, x[:3], stack)
+        assert np.array_equal(oh[2], one[2][0][0]) and np.array_equal(oxn[2], one[2][1][0]), stack
+        for t in range(T):
+            rel = np.linalg.norm(got_xn[t] - one[t][1][0]) / np.linalg.norm(one[t][1][0])
+            assert rel <= 2e-3, (stack, t, rel)
+        # one token more: the grouped path
+        gh, gxn, _ = _run(lws, x[:T + 1], stack)
         for t in range(T + 1):
-            h1, xn1 = dev(x[t:t + 1]), dev(x[t:t + 1])
-            ws1 = fm.alloc_workspace(lws[0].desc, 1)
-            if stack:
-                fm.fmoe_stack_forward(lws, h1, xn1, ws1)
-            else:
-                fm.fmoe_layer_forward(lws[0], h1, xn1, ws1)
-            want.append((host(h1)[0], host(xn1)[0]))
-        for n in (T, T + 1):
-            h, xn = dev(x[:n]), dev(x[:n])
-            ws = fm.alloc_workspace(lws[0].desc, n)
-            if stack:
-                fm.fmoe_stack_forward(lws, h, xn, ws)
-            else:
-                fm.fmoe_layer_forward(lws[0], h, xn, ws)
-            got_h, got_xn = host(h), host(xn)
-            for t in range(n):
-                if n == T:
-                    assert np.array_equal(got_h[t], want[t][0]) and np.array_equal(got_xn[t], want[t][1]), (stack, t)
-                else:
-                    rel = np.linalg.norm(got_xn[t] - want[t][1]) / np.linalg.norm(want[t][1])
-                    assert rel <= 2e-3, (stack, t, rel)
+            rel = np.linalg.norm(gxn[t] - one[t][1][0]) / np.linalg.norm(one[t][1][0])
+            assert rel <= 2e-3, (stack, t, rel)
     assert fm.fmoe_read_status() == 0
 
 
