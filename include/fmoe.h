@@ -294,13 +294,46 @@ int fmoe_layer_forward_logits(const fmoe_layer_weights* lw, const float* d_logit
                               float* d_xn, int T, void* d_ws, size_t ws_bytes, cudaStream_t stream);
 
 /* A stack of n_layers layers (host array of weight descriptors) for T
- * tokens, in place on d_h / d_xn: layer l + 1 reads what layer l wrote.
- * Equivalent to n_layers calls of fmoe_layer_forward.  At T = 1 with one
- * descriptor for all layers the whole stack runs as one persistent kernel
- * (cooperative launch, one CTA per SM, up to 32 layers per launch).  If that
- * kernel reports FMOE_STATUS_WAIT_TIMEOUT, re-initialise the workspace. */
+ * tokens, in place on d_h / d_xn: layer l + 1 reads what layer l wrote --
+ * the layer chain of "What is Flash-MoE?" (a2a-mcp.org), section
+ * "Understanding Mixture-of-Experts": every layer's output is the next
+ * layer's input.  The same results, bit for bit, as n_layers calls of
+ * fmoe_layer_forward.  Up to fmoe_fused_max_tokens(1) tokens with one
+ * descriptor for all layers the whole stack runs as persistent kernels
+ * (cooperative launch, one CTA per SM, two tokens and up to 32 layers per
+ * launch), which leave the last layer's intermediates in the workspace
+ * (see fmoe_stack_forward_trace for every layer's).  If a persistent kernel
+ * reports FMOE_STATUS_WAIT_TIMEOUT, re-initialise the workspace. */
 int fmoe_stack_forward(const fmoe_layer_weights* layers, int n_layers, float* d_h, float* d_xn,
                        int T, void* d_ws, size_t ws_bytes, cudaStream_t stream);
+
+/* Sections of one layer's record in a stack trace. */
+#define FMOE_TRACE_XN_IN 0   /* fp32 [T][H]: the layer's input xn */
+#define FMOE_TRACE_LOGITS 1  /* fp32 [T][E]: router logits */
+#define FMOE_TRACE_IDS 2     /* int32 [T][k]: selected experts, best first */
+#define FMOE_TRACE_WEIGHTS 3 /* fp32 [T][k]: their gate weights */
+#define FMOE_TRACE_GAMMA 4   /* fp32 [T]: shared-expert gate */
+#define FMOE_TRACE_A 5       /* fp32 [T][k+1][I]: SwiGLU outputs, shared expert last */
+#define FMOE_TRACE_H_OUT 6   /* fp32 [T][H]: the layer's output h' */
+
+/* Bytes of a trace of n_layers layers for T tokens (0 on bad arguments). */
+size_t fmoe_trace_bytes(const fmoe_layer_desc* d, int T, int n_layers);
+
+/* Byte offset of section `which` (FMOE_TRACE_*) of layer `layer`'s record
+ * in a trace ((size_t)-1 on bad arguments); records follow one another,
+ * sections are 256-byte aligned. */
+size_t fmoe_trace_offset(const fmoe_layer_desc* d, int T, int layer, int which);
+
+/* fmoe_stack_forward that also records, for every layer, its input xn, the
+ * router logits, the selected experts and gate weights, gamma, the SwiGLU
+ * outputs and its output h' into d_trace (device, 16-byte aligned, at least
+ * fmoe_trace_bytes(desc, T, n_layers) bytes, caller-owned): the values the
+ * launches themselves computed, for checking every layer of a persistent
+ * stack launch.  All layers must share one descriptor.  Errors: as
+ * fmoe_stack_forward, FMOE_ERR_INVALID_ARG for a null or misaligned trace,
+ * FMOE_ERR_BUFFER_TOO_SMALL when trace_bytes is short. */
+int fmoe_stack_forward_trace(const fmoe_layer_weights* layers, int n_layers, float* d_h, float* d_xn, int T,
+                             void* d_ws, size_t ws_bytes, void* d_trace, size_t trace_bytes, cudaStream_t stream);
 
 /* fmoe_stack_forward for token state in host memory (the call a plain C
  * decode loop makes once per token): hx_in / hx_out host fp32 [2][T][H]
@@ -346,9 +379,11 @@ int fmoe_set_tensor_cores(int enable);
 int fmoe_fused_max_tokens(int stack);
 
 /* Tokens an expert needs in a step for its products to run on the tensor
- * cores (when enabled): 5.  From about five tokens per expert the
- * integer-dot matrix-vector path is bound by its dot products rather than by
- * the expert's weight bytes. */
+ * cores (when enabled): 3.  With the 24-bit activations of the integer-dot
+ * path (two dot products per code lane), from three tokens per expert that
+ * path is bound by its dot products rather than by the expert's weight
+ * bytes, and the tensor-core products are faster (measured on the 64-token
+ * Zipf-routed step: 0.446 against 0.490 ms at a threshold of 5). */
 int fmoe_tc_min_tokens(void);
 
 /* 1 if the persistent kernel runs layers of descriptor d at T = 1 on the
@@ -370,8 +405,8 @@ int fmoe_fused_supported(const fmoe_layer_desc* d);
  * library's module is loaded on that device.
  *   lw, d_h, d_xn, T, stream  as for fmoe_layer_forward.
  * Limit: fmoe_workspace_bytes(&lw->desc, T) must not exceed 12 MiB
- * (12582912 bytes), which admits up to T = 16 tokens at hidden 4096 /
- * inter 1024 / 512 experts / top-4 (from T = 5 the workspace holds the
+ * (12582912 bytes), which admits up to T = 13 tokens at hidden 4096 /
+ * inter 1024 / 512 experts / top-4 (from T = 3 the workspace holds the
  * tensor-core inputs, about 100 KB per token); a larger request returns
  * FMOE_ERR_BUFFER_TOO_SMALL before anything is launched.
  * First call on each device: it looks up the array's device address and

@@ -44,6 +44,7 @@ FMOE_STATUS_BAD_PACK_INPUT = 0x8
 FMOE_LOGITS_GIVEN = 0x1
 
 WS_LOGITS, WS_IDS, WS_WEIGHTS, WS_GAMMA, WS_A, WS_Y = range(6)
+TRACE_XN_IN, TRACE_LOGITS, TRACE_IDS, TRACE_WEIGHTS, TRACE_GAMMA, TRACE_A, TRACE_H_OUT = range(7)
 
 LIBRARY_PATH = _LIB_PATH
 
@@ -87,6 +88,9 @@ _SIGS = {
     "fmoe_layer_forward": (_i32, [_PW, _vp, _vp, _i32, _vp, _sz, _vp]),
     "fmoe_layer_forward_logits": (_i32, [_PW, _vp, _vp, _vp, _i32, _vp, _sz, _vp]),
     "fmoe_stack_forward": (_i32, [_PW, _i32, _vp, _vp, _i32, _vp, _sz, _vp]),
+    "fmoe_stack_forward_trace": (_i32, [_PW, _i32, _vp, _vp, _i32, _vp, _sz, _vp, _sz, _vp]),
+    "fmoe_trace_bytes": (_sz, [_PDESC, _i32, _i32]),
+    "fmoe_trace_offset": (_sz, [_PDESC, _i32, _i32, _i32]),
     "fmoe_set_fused": (_i32, [_i32]),
     "fmoe_fused_supported": (_i32, [_PDESC]),
     "fmoe_set_tensor_cores": (_i32, [_i32]),
@@ -324,11 +328,45 @@ def fmoe_stack_forward_host(layers, hx_in, hx_out, d_hx, ws, stream=None) -> Non
     _check(rc, "fmoe_stack_forward_host")
 
 
-def fmoe_stack_forward(layers, h, xn, ws, stream=None) -> None:
+def fmoe_stack_forward(layers, h, xn, ws, stream=None, trace=None) -> None:
+    """The layer stack in place on h / xn; with `trace` (from alloc_trace),
+    fmoe_stack_forward_trace: every layer's input, intermediates and output."""
     arr = (fmoe_layer_weights * len(layers))(*[lw.c() for lw in layers])
-    rc = _lib.fmoe_stack_forward(arr, len(layers), _ptr(h), _ptr(xn), h.shape[0], _ptr(ws),
-                                 ws.numel() * ws.element_size(), _stream(stream))
-    _check(rc, "fmoe_stack_forward")
+    if trace is None:
+        rc = _lib.fmoe_stack_forward(arr, len(layers), _ptr(h), _ptr(xn), h.shape[0], _ptr(ws),
+                                     ws.numel() * ws.element_size(), _stream(stream))
+        _check(rc, "fmoe_stack_forward")
+        return
+    rc = _lib.fmoe_stack_forward_trace(arr, len(layers), _ptr(h), _ptr(xn), h.shape[0], _ptr(ws),
+                                       ws.numel() * ws.element_size(), _ptr(trace),
+                                       trace.numel() * trace.element_size(), _stream(stream))
+    _check(rc, "fmoe_stack_forward_trace")
+
+
+def fmoe_trace_bytes(desc: LayerDesc, T: int, n_layers: int) -> int:
+    d = desc.c()
+    return int(_lib.fmoe_trace_bytes(ctypes.byref(d), T, n_layers))
+
+
+def alloc_trace(desc: LayerDesc, T: int, n_layers: int, device="cuda"):
+    """A device buffer (uint8) for the trace of n_layers layers of T tokens."""
+    import torch
+    return torch.zeros(fmoe_trace_bytes(desc, T, n_layers), dtype=torch.uint8, device=device)
+
+
+def trace_view(trace, desc: LayerDesc, T: int, layer: int, which: int):
+    """Typed view of section `which` (TRACE_*) of layer `layer`'s record."""
+    import torch
+    k, H, I, E = desc.top_k, desc.hidden, desc.inter, desc.n_experts
+    d = desc.c()
+    off = int(_lib.fmoe_trace_offset(ctypes.byref(d), T, layer, which))
+    shapes = {TRACE_XN_IN: ((T, H), torch.float32), TRACE_LOGITS: ((T, E), torch.float32),
+              TRACE_IDS: ((T, k), torch.int32), TRACE_WEIGHTS: ((T, k), torch.float32),
+              TRACE_GAMMA: ((T,), torch.float32), TRACE_A: ((T, k + 1, I), torch.float32),
+              TRACE_H_OUT: ((T, H), torch.float32)}
+    shape, dt = shapes[which]
+    n = int(np.prod(shape))
+    return trace[off:off + 4 * n].view(dt).view(*shape)
 
 
 def fmoe_layer_forward_noalloc(lw: LayerWeights, h, xn, stream=None) -> None:

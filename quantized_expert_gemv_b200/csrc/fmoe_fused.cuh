@@ -148,7 +148,9 @@ struct FusedArgs {
   int n_layers;
   int H, I, E, k;
   float eps;
-  // per token, token-major (the launch's first token at the pointer)
+  // per token, token-major (the launch's first token at the pointer); the
+  // intermediates of layer l at their pointer + l * lstride bytes (0: every
+  // layer writes the same place)
   float* h;           // [NT][H]
   float* xn;          // [NT][H]
   float* logits;      // [NT][E]
@@ -156,6 +158,9 @@ struct FusedArgs {
   float* weights;     // [NT][k]
   float* gamma;       // [NT]
   float* a;           // [NT][(k+1)][I], shared expert last
+  float* tr_xn;       // [NT][H] per layer: the layer's input xn (nullptr: not recorded)
+  float* tr_h;        // [NT][H] per layer: the layer's output h' (nullptr: not recorded)
+  size_t lstride;
   uint64_t* x_logit;  // [NT][kXLogitStride]: router logits, then sigmoid(w_sg . xn) (exchange words)
   float* x_h;      // [NT][kXHStride]: h' of the layer
   float* x_ss;     // [NT][kXSsStride]: per-CTA sums of h'^2
@@ -634,6 +639,10 @@ __global__ void __launch_bounds__(kFusedThreads, 1) fused_stack_kernel(const __g
     const int s = (int)((sq_l + 1u + (m >= 3 ? 1u : 0u)) % kSlots);
     return reinterpret_cast<float*>(smem + P.slot[s]) + (size_t)(m % 3) * H;
   };
+  // the intermediates of layer l (per-layer records when tracing)
+  auto lay = [&](auto* p, int l) {
+    return reinterpret_cast<decltype(p)>(reinterpret_cast<char*>(p) + (size_t)l * A.lstride);
+  };
   auto issue_router = [&](int l, uint32_t sq_l) {
     if (!owner || dw != kWarpRt || nr == 0) return;
     const FusedLayer& NX = A.layers[l];
@@ -759,6 +768,14 @@ __global__ void __launch_bounds__(kFusedThreads, 1) fused_stack_kernel(const __g
         xv[t][6] = h1.z * rt * w1.z; xv[t][7] = h1.w * rt * w1.w;
       }
     }
+    if (A.tr_xn && xthr) {
+#pragma unroll
+      for (int t = 0; t < NT; ++t) {
+        float* tx = lay(A.tr_xn, l) + (size_t)t * H + tid * 8;
+        __stcg(reinterpret_cast<float4*>(tx), make_float4(xv[t][0], xv[t][1], xv[t][2], xv[t][3]));
+        __stcg(reinterpret_cast<float4*>(tx + 4), make_float4(xv[t][4], xv[t][5], xv[t][6], xv[t][7]));
+      }
+    }
     // stage x: 8 consecutive threads share one 64-group
 #pragma unroll
     for (int t = 0; t < NT; ++t) stage_unit(xv[t], xthr, tid >> 3, tid & 7, ngH, sx_of(t));
@@ -794,8 +811,8 @@ __global__ void __launch_bounds__(kFusedThreads, 1) fused_stack_kernel(const __g
         float v = 0.f;
         for (int w = 0; w < kFusedWarps; ++w) v += s_rp[w][t][m];
         const int row = c + m * nC;
-        if (row < E) A.logits[(size_t)t * E + row] = v;
-        else A.gamma[t] = v = 1.f / (1.f + expf(-v));
+        if (row < E) lay(A.logits, l)[(size_t)t * E + row] = v;
+        else lay(A.gamma, l)[t] = v = 1.f / (1.f + expf(-v));
         st_relaxed64(A.x_logit + (size_t)t * kXLogitStride + row, x_word(e_logit, v));
       }
       __syncwarp();
@@ -839,12 +856,13 @@ __global__ void __launch_bounds__(kFusedThreads, 1) fused_stack_kernel(const __g
             // store before the arrive would make it wait for the store)
 #pragma unroll
             for (int t = 0; t < NT; ++t)
-              if (lane < GS::kW) A.a[((size_t)t * (k + 1) + k) * I + (size_t)c * GS::kW + lane] = a[t];
+              if (lane < GS::kW) lay(A.a, l)[((size_t)t * (k + 1) + k) * I + (size_t)c * GS::kW + lane] = a[t];
           } else {
             const float a = block_swiglu<BITS>(gb, dx);
             __syncwarp();
             if (lane == 0) mbar_arrive(&mbar[kMbReady + s]);
-            if (lane < GR::kW) A.a[((size_t)tr * (k + 1) + jj) * I + (size_t)routed_nb(p) * GR::kW + lane] = a;
+            if (lane < GR::kW)
+              lay(A.a, l)[((size_t)tr * (k + 1) + jj) * I + (size_t)routed_nb(p) * GR::kW + lane] = a;
           }
         }
       }
@@ -912,8 +930,8 @@ __global__ void __launch_bounds__(kFusedThreads, 1) fused_stack_kernel(const __g
         wt_r = __shfl_sync(0xffffffffu, pw, jj);
         if (route_writer && dw == 0) {
           if (lane < k) {
-            A.ids[(size_t)tr * k + lane] = sel;
-            A.weights[(size_t)tr * k + lane] = pw;
+            lay(A.ids, l)[(size_t)tr * k + lane] = sel;
+            lay(A.weights, l)[(size_t)tr * k + lane] = pw;
           }
           if (lane == 0 && s_nan) raise_status(FMOE_STATUS_NAN_LOGIT);
         }
@@ -1074,6 +1092,7 @@ __global__ void __launch_bounds__(kFusedThreads, 1) fused_stack_kernel(const __g
             for (int g = 0; g < ngr; ++g) v += sred[g * nv + t * nd + tid];
             A.h[(size_t)t * H + i0 + tid] = v;
             __stcg(A.x_h + (size_t)t * kXHStride + i0 + tid, v);
+            if (A.tr_h) lay(A.tr_h, l)[(size_t)t * H + i0 + tid] = v;
             ss[t] = v * v;
           }
           ss[t] = warp_sum(ss[t]);

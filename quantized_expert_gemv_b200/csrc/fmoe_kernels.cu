@@ -635,6 +635,26 @@ static WsLayout ws_layout(int H, int I, int E, int k, int T) {
   return w;
 }
 
+// One layer's record of a stack trace (fmoe_stack_forward_trace): sections
+// in the order of the FMOE_TRACE_* constants, each 256-byte aligned.
+struct TraceLayout {
+  size_t off[7];
+  size_t bytes;
+};
+
+static TraceLayout trace_layout(int H, int I, int E, int k, int T) {
+  const size_t sz[7] = {(size_t)T * H * 4, (size_t)T * E * 4, (size_t)T * k * 4, (size_t)T * k * 4,
+                        (size_t)T * 4,     (size_t)T * (k + 1) * I * 4, (size_t)T * H * 4};
+  TraceLayout t;
+  size_t o = 0;
+  for (int i = 0; i < 7; ++i) {
+    t.off[i] = o;
+    o = align_up(o + sz[i], 256);
+  }
+  t.bytes = o;
+  return t;
+}
+
 static inline bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
 
 static bool desc_valid(const fmoe_layer_desc* d) {
@@ -946,7 +966,8 @@ static bool same_desc(const fmoe_layer_desc& a, const fmoe_layer_desc& b) {
 // others follow).  Returns FMOE_ERR_UNSUPPORTED when the configuration does
 // not fit it.
 static int launch_fused(const fmoe_layer_weights* layers, int n_layers, float* h, float* xn, void* ws,
-                        size_t ws_bytes, cudaStream_t st, int T = 1, int t = 0, int nt = 1) {
+                        size_t ws_bytes, cudaStream_t st, int T = 1, int t = 0, int nt = 1,
+                        unsigned char* trace = nullptr) {
   const fmoe_layer_desc& d = layers[0].desc;
   const FusedConfig fc = fused_config(d, nt);
   if (!fc.ok) return FMOE_ERR_UNSUPPORTED;
@@ -973,9 +994,22 @@ static int launch_fused(const fmoe_layer_weights* layers, int n_layers, float* h
   args.x_part = reinterpret_cast<float*>(base + w.x_part);
   args.sync = reinterpret_cast<unsigned*>(base + w.sync);
   args.plan = fc.plan;
+  const TraceLayout tl = trace_layout(d.hidden, d.inter, d.n_experts, d.top_k, T);
   for (int l0 = 0; l0 < n_layers; l0 += kFusedMaxLayers) {
     const int n = n_layers - l0 < kFusedMaxLayers ? n_layers - l0 : kFusedMaxLayers;
     args.n_layers = n;
+    if (trace) {
+      // this chunk's layers' records, token t's rows
+      unsigned char* tb = trace + (size_t)l0 * tl.bytes;
+      args.tr_xn = reinterpret_cast<float*>(tb + tl.off[FMOE_TRACE_XN_IN]) + (size_t)t * d.hidden;
+      args.logits = reinterpret_cast<float*>(tb + tl.off[FMOE_TRACE_LOGITS]) + (size_t)t * d.n_experts;
+      args.ids = reinterpret_cast<int32_t*>(tb + tl.off[FMOE_TRACE_IDS]) + (size_t)t * d.top_k;
+      args.weights = reinterpret_cast<float*>(tb + tl.off[FMOE_TRACE_WEIGHTS]) + (size_t)t * d.top_k;
+      args.gamma = reinterpret_cast<float*>(tb + tl.off[FMOE_TRACE_GAMMA]) + t;
+      args.a = reinterpret_cast<float*>(tb + tl.off[FMOE_TRACE_A]) + (size_t)t * (d.top_k + 1) * d.inter;
+      args.tr_h = reinterpret_cast<float*>(tb + tl.off[FMOE_TRACE_H_OUT]) + (size_t)t * d.hidden;
+      args.lstride = tl.bytes;
+    }
     for (int l = 0; l < n; ++l) {
       const fmoe_layer_weights& L = layers[l0 + l];
       args.layers[l].experts = static_cast<const uint8_t*>(L.experts);
@@ -1006,14 +1040,14 @@ static int launch_fused(const fmoe_layer_weights* layers, int n_layers, float* h
 // FMOE_ERR_UNSUPPORTED (nothing launched) when the one-token kernel does not
 // fit the shape.
 static int launch_fused_tokens(const fmoe_layer_weights* layers, int n_layers, float* h, float* xn, int T,
-                               void* ws, size_t ws_bytes, cudaStream_t st) {
+                               void* ws, size_t ws_bytes, cudaStream_t st, unsigned char* trace = nullptr) {
   const fmoe_layer_desc& d = layers[0].desc;
   if (!fused_config(d, 1).ok) return FMOE_ERR_UNSUPPORTED;
   const bool pairs = fused_config(d, 2).ok;
   const size_t H = (size_t)d.hidden;
   for (int t = 0; t < T;) {
     const int nt = pairs && T - t >= 2 ? 2 : 1;
-    const int rc = launch_fused(layers, n_layers, h + t * H, xn + t * H, ws, ws_bytes, st, T, t, nt);
+    const int rc = launch_fused(layers, n_layers, h + t * H, xn + t * H, ws, ws_bytes, st, T, t, nt, trace);
     if (rc != FMOE_OK) return rc;
     t += nt;
   }
@@ -1260,10 +1294,23 @@ extern "C" int fmoe_set_fused(int enable) {
   return prev;
 }
 
-extern "C" int fmoe_stack_forward(const fmoe_layer_weights* layers, int n_layers, float* d_h,
-                                  float* d_xn, int T, void* d_ws, size_t ws_bytes,
-                                  cudaStream_t stream) {
+// A stack of layers; with a trace, every layer's input xn, intermediates and
+// output h' recorded in its record of the trace.
+static int stack_forward_impl(const fmoe_layer_weights* layers, int n_layers, float* d_h, float* d_xn, int T,
+                              void* d_ws, size_t ws_bytes, unsigned char* trace, size_t trace_bytes,
+                              cudaStream_t stream) {
   if (!layers || n_layers < 1) return FMOE_ERR_INVALID_ARG;
+  if (trace) {
+    for (int l = 0; l < n_layers; ++l) {
+      const int rc = weights_check(&layers[l]);
+      if (rc != FMOE_OK) return rc;
+      if (!same_desc(layers[l].desc, layers[0].desc)) return FMOE_ERR_INVALID_ARG;
+    }
+    const fmoe_layer_desc& d = layers[0].desc;
+    if (T < 1 || !aligned16(trace)) return FMOE_ERR_INVALID_ARG;
+    if (trace_bytes < (size_t)n_layers * trace_layout(d.hidden, d.inter, d.n_experts, d.top_k, T).bytes)
+      return FMOE_ERR_BUFFER_TOO_SMALL;
+  }
   if (T >= 1 && T <= kFusedTokensStack && g_fused_enabled) {
     bool uniform = true;
     for (int l = 0; l < n_layers; ++l) {
@@ -1276,15 +1323,62 @@ extern "C" int fmoe_stack_forward(const fmoe_layer_weights* layers, int n_layers
     if (uniform) {
       // the tokens through the whole stack, two per persistent launch; up to
       // kFusedTokensStack tokens this beats the grouped path layer by layer
-      const int rc = launch_fused_tokens(layers, n_layers, d_h, d_xn, T, d_ws, ws_bytes, stream);
+      const int rc = launch_fused_tokens(layers, n_layers, d_h, d_xn, T, d_ws, ws_bytes, stream, trace);
       if (rc != FMOE_ERR_UNSUPPORTED) return rc;
     }
   }
   for (int l = 0; l < n_layers; ++l) {
+    const fmoe_layer_desc& d = layers[l].desc;
+    const TraceLayout tl = trace_layout(d.hidden, d.inter, d.n_experts, d.top_k, T);
+    unsigned char* rec = trace ? trace + (size_t)l * tl.bytes : nullptr;
+    const size_t hb = (size_t)T * d.hidden * 4;
+    if (rec && cudaMemcpyAsync(rec + tl.off[FMOE_TRACE_XN_IN], d_xn, hb, cudaMemcpyDeviceToDevice, stream) !=
+                   cudaSuccess)
+      return FMOE_ERR_CUDA;
     const int rc = fmoe_layer_forward(&layers[l], d_h, d_xn, T, d_ws, ws_bytes, stream);
     if (rc != FMOE_OK) return rc;
+    if (rec) {
+      // the layer's intermediates, as it left them in the workspace
+      const WsLayout w = ws_layout(d.hidden, d.inter, d.n_experts, d.top_k, T);
+      const unsigned char* base = static_cast<const unsigned char*>(d_ws);
+      const size_t src[5] = {w.logits, w.ids, w.weights, w.gamma, w.a};
+      const size_t n[5] = {(size_t)T * d.n_experts * 4, (size_t)T * d.top_k * 4, (size_t)T * d.top_k * 4,
+                           (size_t)T * 4, (size_t)T * (d.top_k + 1) * d.inter * 4};
+      for (int i = 0; i < 5; ++i)
+        if (cudaMemcpyAsync(rec + tl.off[FMOE_TRACE_LOGITS + i], base + src[i], n[i], cudaMemcpyDeviceToDevice,
+                            stream) != cudaSuccess)
+          return FMOE_ERR_CUDA;
+      if (cudaMemcpyAsync(rec + tl.off[FMOE_TRACE_H_OUT], d_h, hb, cudaMemcpyDeviceToDevice, stream) != cudaSuccess)
+        return FMOE_ERR_CUDA;
+    }
   }
   return FMOE_OK;
+}
+
+extern "C" int fmoe_stack_forward(const fmoe_layer_weights* layers, int n_layers, float* d_h,
+                                  float* d_xn, int T, void* d_ws, size_t ws_bytes,
+                                  cudaStream_t stream) {
+  return stack_forward_impl(layers, n_layers, d_h, d_xn, T, d_ws, ws_bytes, nullptr, 0, stream);
+}
+
+extern "C" size_t fmoe_trace_bytes(const fmoe_layer_desc* d, int T, int n_layers) {
+  if (!desc_valid(d) || T < 1 || n_layers < 1) return 0;
+  return (size_t)n_layers * trace_layout(d->hidden, d->inter, d->n_experts, d->top_k, T).bytes;
+}
+
+extern "C" size_t fmoe_trace_offset(const fmoe_layer_desc* d, int T, int layer, int which) {
+  if (!desc_valid(d) || T < 1 || layer < 0 || which < FMOE_TRACE_XN_IN || which > FMOE_TRACE_H_OUT)
+    return (size_t)-1;
+  const TraceLayout tl = trace_layout(d->hidden, d->inter, d->n_experts, d->top_k, T);
+  return (size_t)layer * tl.bytes + tl.off[which];
+}
+
+extern "C" int fmoe_stack_forward_trace(const fmoe_layer_weights* layers, int n_layers, float* d_h, float* d_xn,
+                                        int T, void* d_ws, size_t ws_bytes, void* d_trace, size_t trace_bytes,
+                                        cudaStream_t stream) {
+  if (!d_trace) return FMOE_ERR_INVALID_ARG;
+  return stack_forward_impl(layers, n_layers, d_h, d_xn, T, d_ws, ws_bytes, static_cast<unsigned char*>(d_trace),
+                            trace_bytes, stream);
 }
 
 extern "C" int fmoe_stack_forward_host(const fmoe_layer_weights* layers, int n_layers, const float* hx_in,

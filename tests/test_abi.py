@@ -221,7 +221,7 @@ def test_host_validation_of_the_later_entry_points(fm):
     assert L.fmoe_cache_stats(None, None, None, None) == fm.FMOE_ERR_INVALID_ARG
     assert L.fmoe_cache_destroy(None) == fm.FMOE_ERR_INVALID_ARG
     # the dispatch thresholds the header states
-    assert fm.fmoe_tc_min_tokens() == 5
+    assert fm.fmoe_tc_min_tokens() == 3
     assert fm.fmoe_fused_max_tokens(False) == 4 and fm.fmoe_fused_max_tokens(True) == 8
 
 
@@ -232,6 +232,37 @@ def test_workspace_layout(fm):
     offs = [fm.fmoe_workspace_offset(d, 3, w) for w in range(6)]
     assert offs == sorted(offs) and all(o % 256 == 0 for o in offs)
     assert fm.fmoe_workspace_offset(d, 3, 6) == 2 ** 64 - 1
+
+
+def test_trace_layout_and_validation(fm):
+    """A stack trace: one record per layer, sections in the declared order,
+    256-byte aligned, sized for T tokens; bad arguments refused on the host."""
+    L = fm._lib
+    d = fm.LayerDesc()
+    T, n = 3, 5
+    H, I, E, k = d.hidden, d.inter, d.n_experts, d.top_k
+    rec = fm.fmoe_trace_bytes(d, T, 1)
+    assert fm.fmoe_trace_bytes(d, T, n) == n * rec
+    sizes = [T * H * 4, T * E * 4, T * k * 4, T * k * 4, T * 4, T * (k + 1) * I * 4, T * H * 4]
+    dc = d.c()
+    offs = [L.fmoe_trace_offset(ctypes.byref(dc), T, 2, w) for w in range(7)]
+    assert all(o % 256 == 0 for o in offs)
+    assert offs[0] == 2 * rec
+    for w in range(6):
+        assert offs[w + 1] >= offs[w] + sizes[w]
+    assert 2 * rec + rec >= offs[6] + sizes[6]
+    assert L.fmoe_trace_offset(ctypes.byref(dc), T, 0, 7) == 2 ** 64 - 1
+    assert L.fmoe_trace_offset(ctypes.byref(dc), T, -1, 0) == 2 ** 64 - 1
+    assert L.fmoe_trace_bytes(ctypes.byref(dc), 0, 1) == 0
+    # trace entry point: null or misaligned trace, trace too small
+    dd = fm.LayerDesc(hidden=256, inter=128, n_experts=16, top_k=4)
+    w = fm.fmoe_layer_weights(dd.c(), 16, 16, 16, 16, 16)
+    w2 = (fm.fmoe_layer_weights * 2)(w, w)
+    assert L.fmoe_stack_forward_trace(w2, 2, 16, 16, 1, 16, 1 << 30, None, 1 << 30, None) == fm.FMOE_ERR_INVALID_ARG
+    assert L.fmoe_stack_forward_trace(w2, 2, 16, 16, 1, 16, 1 << 30, 24, 1 << 30, None) == fm.FMOE_ERR_INVALID_ARG
+    need = fm.fmoe_trace_bytes(dd, 1, 2)
+    assert L.fmoe_stack_forward_trace(w2, 2, 16, 16, 1, 16, 1 << 30, 16, need - 1, None) == \
+        fm.FMOE_ERR_BUFFER_TOO_SMALL
 
 
 def test_header_and_c_example_compile_as_c():

@@ -1,15 +1,16 @@
 """Full-size layer chains against the oracle: the launch the benchmark times.
 
 Twenty resident layers of hidden 4096 / inter 1024 / 512 experts (int4, and
-2-bit routed experts with a 4-bit shared expert) decode a few tokens: one
-token through the stack, the next token starting from the previous token's
-final xn' (h = xn = xn'); and 2 or 4 independent tokens at once (two per
-persistent launch).  Three checks:
+2-bit routed experts with a 4-bit shared expert) run as one persistent stack
+launch (fmoe_stack_forward, traced: every layer's input xn, router logits,
+selected experts, gate weights, gamma, SwiGLU outputs and output h' as the
+launch computed them).  Tokens are decoded one at a time -- each next token
+starting from the previous token's final xn' (h = xn = xn') -- or 2 and 4
+independent tokens at once (two per persistent launch).  Checks:
 
-  - the stack entry point (one persistent launch over the 20 layers, as the
-    benchmark runs it) gives the bits of the 20 single-layer launches;
+  - the stack's first layer gives the bits of a single-layer call;
   - teacher-forced: every layer of every token against the oracle fed the
-    device's own fp32 inputs of that layer (router logits, top-k ids on the
+    launch's own fp32 inputs of that layer (router logits, top-k ids on the
     device's logits, gate weights, gamma, every expert's SwiGLU outputs a,
     h' and xn' element by element);
   - free-running: an fp64 oracle chain carrying its own state through all
@@ -34,6 +35,9 @@ fm = pytest.importorskip("quantized_expert_gemv_b200")
 
 N_LAYERS = 20
 
+SECTIONS = (("xn_in", fm.TRACE_XN_IN), ("logits", fm.TRACE_LOGITS), ("ids", fm.TRACE_IDS),
+            ("p", fm.TRACE_WEIGHTS), ("gamma", fm.TRACE_GAMMA), ("a", fm.TRACE_A), ("h", fm.TRACE_H_OUT))
+
 
 @pytest.fixture(scope="module", autouse=True)
 def _cuda():
@@ -57,64 +61,55 @@ def layer_base(wl, layer):
                                {wl.n_experts: synth.expert(wl, layer, wl.n_experts)})
 
 
-def decode_on_device(wl, lws, n_tokens, stream):
-    """Each token layer by layer (fmoe_layer_forward, T = 1), recording every
-    layer's inputs, outputs and intermediates; then the same token through
-    fmoe_stack_forward from the same start, which must give the same bits."""
+def traced_stack(lws, x):
+    """x [T][H] through the stack (h = xn = x), traced.  Returns per token the
+    list of per-layer records (h_in, xn_in, logits, ids, p, gamma, a, h, xn)."""
     desc = lws[0].desc
-    ws = fm.alloc_workspace(desc, 1)
-    ws2 = fm.alloc_workspace(desc, 1)
+    T = len(x)
+    ws = fm.alloc_workspace(desc, T)
+    tr = fm.alloc_trace(desc, T, N_LAYERS)
+    h, xn = dev(x), dev(x)
+    fm.fmoe_stack_forward(lws, h, xn, ws, trace=tr)
+    per_layer = [{name: host(fm.trace_view(tr, desc, T, l, which)) for name, which in SECTIONS}
+                 for l in range(N_LAYERS)]
+    h_fin, xn_fin = host(h), host(xn)
+    recs = [[] for _ in range(T)]
+    for l, v in enumerate(per_layer):
+        xn_out = per_layer[l + 1]["xn_in"] if l + 1 < N_LAYERS else xn_fin
+        h_in = x if l == 0 else per_layer[l - 1]["h"]
+        for t in range(T):
+            r = {name: v[name][t] for name, _ in SECTIONS}
+            r.update(h_in=h_in[t], xn=xn_out[t])
+            recs[t].append(r)
+    assert np.array_equal(per_layer[-1]["h"], h_fin), "traced h' of the last layer differs from the output"
+    assert np.array_equal(per_layer[0]["xn_in"], x), "traced input of the first layer differs from the input"
+    assert fm.fmoe_read_status() == 0
+    return recs
+
+
+def first_layer_matches_layer_call(lws, x, rec0):
+    """The stack's first layer against fmoe_layer_forward on the same tokens, bit for bit."""
+    T = len(x)
+    h, xn = dev(x), dev(x)
+    fm.fmoe_layer_forward(lws[0], h, xn, fm.alloc_workspace(lws[0].desc, T))
+    for t in range(T):
+        assert np.array_equal(host(h)[t], rec0[t]["h"]), f"token {t}: first layer h' differs from a layer call"
+        assert np.array_equal(host(xn)[t], rec0[t]["xn"]), f"token {t}: first layer xn' differs from a layer call"
+
+
+def decode_on_device(wl, lws, n_tokens, stream):
+    """Tokens one at a time through the traced stack, each starting from the
+    previous token's final xn'."""
     x0 = synth.tokens(wl, 1, stream=stream)[0]
     tok = x0.copy()
     recs = []
     for t in range(n_tokens):
-        h, xn = dev(tok[None]), dev(tok[None])
-        layers = []
-        for l in range(N_LAYERS):
-            h_in, xn_in = host(h)[0], host(xn)[0]
-            fm.fmoe_layer_forward(lws[l], h, xn, ws)
-            view = lambda which: host(fm.workspace_view(ws, desc, 1, which))[0]
-            layers.append(dict(h_in=h_in, xn_in=xn_in, h=host(h)[0], xn=host(xn)[0], logits=view(fm.WS_LOGITS),
-                               ids=view(fm.WS_IDS), p=view(fm.WS_WEIGHTS), gamma=view(fm.WS_GAMMA),
-                               a=view(fm.WS_A)))
-        h2, xn2 = dev(tok[None]), dev(tok[None])
-        fm.fmoe_stack_forward(lws, h2, xn2, ws2)
-        assert np.array_equal(host(h2)[0], layers[-1]["h"]), f"token {t}: stack h' differs from the layer calls"
-        assert np.array_equal(host(xn2)[0], layers[-1]["xn"]), f"token {t}: stack xn' differs from the layer calls"
-        recs.append(layers)
-        tok = layers[-1]["xn"].copy()
-    assert fm.fmoe_read_status() == 0
+        r = traced_stack(lws, tok[None])[0]
+        if t == 0:
+            first_layer_matches_layer_call(lws, tok[None], [r[0]])
+        recs.append(r)
+        tok = r[-1]["xn"].copy()
     return x0, recs
-
-
-VIEWS = (("logits", fm.WS_LOGITS), ("ids", fm.WS_IDS), ("p", fm.WS_WEIGHTS), ("gamma", fm.WS_GAMMA),
-         ("a", fm.WS_A))
-
-
-def decode_batch_on_device(wl, lws, T, stream):
-    """T independent tokens layer by layer (fmoe_layer_forward with T rows:
-    persistent launches of two tokens), recording every layer's inputs,
-    outputs and intermediates per token; then fmoe_stack_forward on the same
-    tokens, which must give the same bits."""
-    desc = lws[0].desc
-    ws = fm.alloc_workspace(desc, T)
-    x = synth.tokens(wl, T, stream=stream)
-    h, xn = dev(x), dev(x)
-    recs = [[] for _ in range(T)]
-    for l in range(N_LAYERS):
-        h_in, xn_in = host(h), host(xn)
-        fm.fmoe_layer_forward(lws[l], h, xn, ws)
-        v = {name: host(fm.workspace_view(ws, desc, T, which)) for name, which in VIEWS}
-        h_out, xn_out = host(h), host(xn)
-        for t in range(T):
-            recs[t].append(dict(h_in=h_in[t], xn_in=xn_in[t], h=h_out[t], xn=xn_out[t],
-                                **{name: v[name][t] for name, _ in VIEWS}))
-    h2, xn2 = dev(x), dev(x)
-    fm.fmoe_stack_forward(lws, h2, xn2, fm.alloc_workspace(desc, T))
-    assert np.array_equal(host(h2), host(h)), "stack h' differs from the layer calls"
-    assert np.array_equal(host(xn2), host(xn)), "stack xn' differs from the layer calls"
-    assert fm.fmoe_read_status() == 0
-    return x, recs
 
 
 def teacher_forced(wl, rec, layer, label):
@@ -170,21 +165,23 @@ def free_running(wl, x0, recs):
     return near_ties
 
 
-def run_chain_checks(wl, lws, n_tokens, stream):
-    x0, recs = decode_on_device(wl, lws, n_tokens, stream)
-    jobs = [(t, l) for t in range(n_tokens) for l in range(N_LAYERS)]
-    out = {}
+def check_chains(wl, starts, seqs, label):
+    """Teacher-forced checks of every (token, layer) and the free-running
+    chain of every decode sequence: seqs[i] is a list of tokens decoded one
+    after the other from starts[i], each token a list of layer records."""
+    jobs = [(i, t, l) for i, seq in enumerate(seqs) for t in range(len(seq)) for l in range(N_LAYERS)]
+    near = []
 
-    def job(i):
-        if i == len(jobs):
-            out["near_ties"] = free_running(wl, x0, recs)
+    def job(n):
+        if n >= len(jobs):
+            i = n - len(jobs)
+            near.extend(free_running(wl, starts[i], seqs[i]))
             return
-        t, l = jobs[i]
-        teacher_forced(wl, recs[t][l], l, f"token {t} layer {l}")
+        i, t, l = jobs[n]
+        teacher_forced(wl, seqs[i][t][l], l, f"{label} seq {i} token {t} layer {l}")
 
-    pmap(job, range(len(jobs) + 1))
-    print(f"near ties adopted by the free-running oracle: {len(out['near_ties'])} {out['near_ties']}")
-    return out["near_ties"]
+    pmap(job, range(len(jobs) + len(seqs)))
+    print(f"{label}: near ties adopted by the free-running oracle: {len(near)} {near}")
 
 
 @pytest.fixture(scope="module")
@@ -202,30 +199,21 @@ def test_stack_20_layers_int4_full_size(stack_int4):
     """Twenty int4 layers (72.5 GB resident), three tokens decoded."""
     wl, lws = stack_int4
     assert fm.fmoe_fused_supported(lws[0].desc)
-    run_chain_checks(wl, lws, 3, stream=81)
+    x0, recs = decode_on_device(wl, lws, 3, stream=81)
+    check_chains(wl, [x0], [recs], "int4")
 
 
 @pytest.mark.parametrize("T", [2, 4])
 def test_stack_20_layers_int4_few_tokens(stack_int4, T):
     """T independent tokens (two per persistent launch) through the twenty
     int4 layers: every layer of every token teacher-forced against the
-    oracle, the stack against the layer calls bit for bit, and each token's
-    free-running fp64 chain."""
+    oracle, the first layer against a layer call bit for bit, and each
+    token's free-running fp64 chain."""
     wl, lws = stack_int4
-    x, recs = decode_batch_on_device(wl, lws, T, stream=83 + T)
-    jobs = [(t, l) for t in range(T) for l in range(N_LAYERS)]
-    near = []
-
-    def job(i):
-        if i >= len(jobs):
-            t = i - len(jobs)
-            near.extend(free_running(wl, x[t], [recs[t]]))
-            return
-        t, l = jobs[i]
-        teacher_forced(wl, recs[t][l], l, f"T={T} token {t} layer {l}")
-
-    pmap(job, range(len(jobs) + T))
-    print(f"near ties adopted by the free-running oracle: {len(near)} {near}")
+    x = synth.tokens(wl, T, stream=83 + T)
+    recs = traced_stack(lws, x)
+    first_layer_matches_layer_call(lws, x, [r[0] for r in recs])
+    check_chains(wl, list(x), [[r] for r in recs], f"int4 T={T}")
 
 
 @pytest.fixture(scope="module")
@@ -244,4 +232,5 @@ def test_stack_20_layers_int2_full_size(stack_int2):
     two tokens decoded."""
     wl, lws = stack_int2
     assert fm.fmoe_fused_supported(lws[0].desc)
-    run_chain_checks(wl, lws, 2, stream=82)
+    x0, recs = decode_on_device(wl, lws, 2, stream=82)
+    check_chains(wl, [x0], [recs], "int2")

@@ -73,15 +73,21 @@ def check_layer_token(wl, lw_o, ws, desc, T, t, h_in, xn_in, h_out, xn_out, labe
     the persistent kernel sums them on the fly), h' and xn' against the
     oracle."""
     fused = T <= fm.fmoe_fused_max_tokens() and not logits_given and fused_on() and fm.fmoe_fused_supported(desc)
+    v = {name: host(fm.workspace_view(ws, desc, T, which))[t]
+         for name, which in (("logits", fm.WS_LOGITS), ("ids", fm.WS_IDS), ("p", fm.WS_WEIGHTS),
+                             ("gamma", fm.WS_GAMMA), ("a", fm.WS_A), ("y", fm.WS_Y))}
+    if fused:
+        del v["y"]
+    return check_layer_values(wl, lw_o, v, h_in, xn_in, h_out, xn_out, label, logits_given)
+
+
+def check_layer_values(wl, lw_o, v, h_in, xn_in, h_out, xn_out, label, logits_given=False):
+    """check_layer_token on the intermediates v (logits, ids, p, gamma, a and,
+    when present, y) of one token's layer step."""
     layer = getattr(lw_o, "layer", 0)
     # a private copy of the layer: experts generated for this check are dropped with it
     lw_o = oracle.LayerWeights(lw_o.w_router, lw_o.w_shared_gate, lw_o.norm_w, dict(lw_o.experts))
-    lg_d = host(fm.workspace_view(ws, desc, T, fm.WS_LOGITS))[t]
-    ids_d = host(fm.workspace_view(ws, desc, T, fm.WS_IDS))[t]
-    p_d = host(fm.workspace_view(ws, desc, T, fm.WS_WEIGHTS))[t]
-    a_d = host(fm.workspace_view(ws, desc, T, fm.WS_A))[t]
-    y_d = host(fm.workspace_view(ws, desc, T, fm.WS_Y))[t]
-    gamma_d = host(fm.workspace_view(ws, desc, T, fm.WS_GAMMA))[t]
+    lg_d, ids_d, p_d, a_d, gamma_d = v["logits"], v["ids"], v["p"], v["a"], v["gamma"]
     if not logits_given:
         lg_o, S_l = oracle.gemv_f32(lw_o.w_router, xn_in.astype(np.float64))
         check(lg_d, lg_o, S_l, f"{label} logits")
@@ -96,11 +102,42 @@ def check_layer_token(wl, lw_o, ws, desc, T, t, h_in, xn_in, h_out, xn_out, labe
     for j, slot in enumerate(list(ids_d) + [wl.n_experts]):
         e = oracle.expert_ffn(lw_o.experts[int(slot)], wl.hidden, wl.inter, wl.group, xn_in)
         check(a_d[j], e["a"], e["S_a"], f"{label} a[{j}]")
-    if not fused:
-        check(y_d, ref["y"], ref["S_y"], f"{label} y")
+    if "y" in v:
+        check(v["y"], ref["y"], ref["S_y"], f"{label} y")
     check(h_out, ref["h"], ref["S_h"], f"{label} h'")
     check(xn_out, ref["xn"], ref["S_xn"], f"{label} xn'")
     return ref
+
+
+TRACE_SECTIONS = (("xn_in", fm.TRACE_XN_IN), ("logits", fm.TRACE_LOGITS), ("ids", fm.TRACE_IDS),
+                  ("p", fm.TRACE_WEIGHTS), ("gamma", fm.TRACE_GAMMA), ("a", fm.TRACE_A), ("h", fm.TRACE_H_OUT))
+
+
+def traced_stack_check(wl, lws, los, x, label):
+    """x [T][H] through the stack (h = xn = x) with a trace; every layer of
+    every token checked teacher-forced on the values the launch recorded.
+    Returns the final h', xn'."""
+    desc = lws[0].desc
+    T, L = len(x), len(lws)
+    ws = fm.alloc_workspace(desc, T)
+    tr = fm.alloc_trace(desc, T, L)
+    h, xn = dev(x), dev(x)
+    fm.fmoe_stack_forward(lws, h, xn, ws, trace=tr)
+    rec = [{name: host(fm.trace_view(tr, desc, T, l, which)) for name, which in TRACE_SECTIONS} for l in range(L)]
+    h_fin, xn_fin = host(h), host(xn)
+    assert np.array_equal(rec[-1]["h"], h_fin)
+    jobs = [(l, t) for l in range(L) for t in range(T)]
+
+    def job(j):
+        l, t = jobs[j]
+        h_in = x[t] if l == 0 else rec[l - 1]["h"][t]
+        xn_out = rec[l + 1]["xn_in"][t] if l + 1 < L else xn_fin[t]
+        v = {name: rec[l][name][t] for name in ("logits", "ids", "p", "gamma", "a")}
+        check_layer_values(wl, los[l], v, h_in, rec[l]["xn_in"][t], rec[l]["h"][t], xn_out,
+                           f"{label} stack layer {l} t={t}")
+
+    pmap(job, range(len(jobs)))
+    return h_fin, xn_fin
 
 
 # ------------------------------------------------------------------ routing --
@@ -443,16 +480,18 @@ def _run(lws, x, stack):
 @pytest.mark.parametrize("wl", [synth.TINY, SMALL], ids=["tiny4", "small4"])
 def test_few_tokens_through_persistent_kernel(wl):
     """Up to fmoe_fused_max_tokens tokens run through the persistent kernel,
-    two per launch (4-bit layers): every token of a layer call against the
-    oracle; a stack call gives the bits of the same tokens through layer
-    calls; a token's bits do not depend on its partner in the pair; an odd
-    last token gets the bits of a T = 1 call; one token more than the
-    maximum takes the grouped path and agrees within the tolerance."""
+    two per launch (4-bit layers): every token of a layer call, and every
+    layer of every token of a traced stack call, against the oracle; a
+    token's bits do not depend on its partner in the pair; an odd last
+    token gets the bits of a T = 1 call; one token more than the maximum
+    takes the grouped path and agrees within the tolerance."""
     if not fm.fmoe_fused_supported(device_layer(wl).desc):
         pytest.skip("persistent kernel does not fit this shape here")
     n_layers = 3
     lws = [device_layer(wl, l) for l in range(n_layers)]
     los = [oracle_layer(wl, l) for l in range(n_layers)]
+    for l, lo in enumerate(los):
+        lo.layer = l
     Tl, Ts = fm.fmoe_fused_max_tokens(False), fm.fmoe_fused_max_tokens(True)
     x = synth.tokens(wl, Ts + 2, stream=61)
     # layer calls of Tl tokens (pairs), chained over the layers, each against the oracle
@@ -464,10 +503,8 @@ def test_few_tokens_through_persistent_kernel(wl):
         for t in range(Tl):
             check_layer_token(wl, los[l], ws, lws[l].desc, Tl, t, h_in[t], xn_in[t], host(h)[t], host(xn)[t],
                               f"layer {l} t={t}")
-    layered = (host(h), host(xn))
-    # the stack over the same tokens: the bits of the layer calls
-    sh, sxn, _ = _run(lws, x[:Tl], stack=True)
-    assert np.array_equal(sh, layered[0]) and np.array_equal(sxn, layered[1])
+    # the stack over Ts tokens, every layer of every token checked on its trace
+    traced_stack_check(wl, lws, los, x[:Ts], "few tokens")
     for stack in (False, True):
         T = Ts if stack else Tl
         got_h, got_xn, _ = _run(lws, x[:T], stack)
@@ -558,11 +595,11 @@ def test_tensor_core_and_integer_paths_differ_only_by_rounding():
 
 @pytest.mark.parametrize("wl", [synth.TINY, TINY2, SMALL, SMALL2], ids=["tiny4", "tiny2", "small4", "small2"])
 def test_stack_chain_teacher_forced_and_free_running(wl, path):
-    """A 4-layer stack decoding 3 tokens: h, xn carried layer to layer, each
-    next token starting from the previous token's final xn'.  Each layer is
-    checked teacher-forced on the device's inputs; fmoe_stack_forward must
-    equal the layer-by-layer calls bit for bit; the free-running fp64 chain
-    must agree in relative L2."""
+    """A 4-layer stack decoding 3 tokens, each next token starting from the
+    previous token's final xn'.  Layer by layer (fmoe_layer_forward) and as
+    one traced stack call per token: every layer checked teacher-forced on
+    the device's inputs; the stack gives the bits of the layer calls; the
+    decode agrees with the free-running fp64 chain in relative L2."""
     L, steps = 4, 3
     lws = [device_layer(wl, l) for l in range(L)]
     los = [oracle_layer(wl, l) for l in range(L)]
@@ -575,10 +612,13 @@ def test_stack_chain_teacher_forced_and_free_running(wl, path):
     h, xn = dev(tok[None]), dev(tok[None])
     free_h = tok.astype(np.float64)
     free_xn = tok.astype(np.float64)
+    first = None
     for s in range(steps):
         for l in range(L):
             h_in, xn_in = host(h)[0], host(xn)[0]
             fm.fmoe_layer_forward(lws[l], h, xn, ws)
+            if s == 0 and l == 0:
+                first = (host(h)[0], host(xn)[0])
             check_layer_token(wl, los[l], ws, lws[l].desc, 1, 0, h_in, xn_in, host(h)[0], host(xn)[0],
                               f"step {s} layer {l}")
             ref = oracle.layer_token(wl, los[l], free_h, free_xn, expert_fn=lambda e, l=l: synth.expert(wl, l, e))
@@ -588,12 +628,18 @@ def test_stack_chain_teacher_forced_and_free_running(wl, path):
     final_layered = host(xn)[0]
     rel = np.linalg.norm(final_layered - free_xn) / np.linalg.norm(free_xn)
     assert rel <= 2e-3, rel
-    # the stack entry point gives the same bits
-    h2, xn2 = dev(x0[None]), dev(x0[None])
+    # the stack entry point, traced, one call per token: the same bits
+    tok = x0.copy()
     for s in range(steps):
-        fm.fmoe_stack_forward(lws, h2, xn2, ws)
-        h2.copy_(xn2)
-    assert np.array_equal(host(xn2)[0], final_layered)
+        if s == 0:
+            tr = fm.alloc_trace(lws[0].desc, 1, 1)
+            h1, xn1 = dev(tok[None]), dev(tok[None])
+            fm.fmoe_stack_forward(lws[:1], h1, xn1, ws, trace=tr)
+            assert np.array_equal(host(h1)[0], first[0]) and np.array_equal(host(xn1)[0], first[1])
+        _, xn_s = traced_stack_check(wl, lws, los, tok[None], f"step {s}")
+        tok = xn_s[0].copy()
+    assert np.array_equal(tok, final_layered)
+    assert fm.fmoe_read_status() == 0
 
 
 # ---------------------------------------------------------- outlier inputs --
