@@ -16,7 +16,8 @@
 //     by one bulk copy;
 //   - one thread issues the four 128 x N x 16 tcgen05.mma of the group and
 //     commits them to the stage's mbarrier, so dequantising the next groups
-//     overlaps the tensor cores;
+//     overlaps the tensor cores (at N <= 64 the issue rate of these small
+//     products, about 75 ns each, bounds the kernel: measured per step);
 //   - the epilogue reads the accumulator with tcgen05.ld (warp w: tensor
 //     memory lanes 32 (w % 4) ..), adds the hi and lo columns, and writes
 //     SwiGLU outputs (gate/up) or expert outputs (down).
@@ -47,6 +48,14 @@ constexpr int kTcRows = 128;      // weight rows per CTA (the MMA's M)
 constexpr uint32_t kTcATile = kTcRows * 64 * 2;  // fp16 A tile of one 64-input group
 
 // ------------------------------------------------------------ primitives --
+// K-major, 128-byte swizzle (layout type 2 in bits 61-63): 8-row atoms of
+// 128-byte lines, SBO = 1024 bytes between atoms (LBO unused).  A K = 16
+// slice at byte offset 32 j of the lines starts 32 j bytes on.
+__device__ __forceinline__ uint64_t umma_desc_sw128(uint32_t saddr) {
+  return (uint64_t)((saddr >> 4) & 0x3FFFu) | (1ull << 16) | ((uint64_t)(1024 >> 4) << 32) | (1ull << 46) |
+         (2ull << 61);
+}
+
 __device__ __forceinline__ uint64_t umma_desc(uint32_t saddr, uint32_t lbo, uint32_t sbo) {
   // K-major, no swizzle: core matrices of 8 rows x 16 bytes; lbo = distance
   // between the two 8-element halves of a K = 16 slice, sbo = between
@@ -192,9 +201,12 @@ __device__ __forceinline__ uint32_t deq_pair(uint32_t fields, __half2 s2, __half
   return *reinterpret_cast<const uint32_t*>(&w);
 }
 
-// 16-byte fp16 store of inputs 8 c .. 8 c + 7 of row r into the A tile.
+// 16-byte fp16 store of inputs 8 c .. 8 c + 7 of row r into the A tile:
+// K-major with the 128-byte swizzle -- a row's 64 inputs are one 128-byte
+// line, 8 rows an atom of 1024 bytes, and the 16-byte chunk c of row r sits
+// at chunk position c ^ (r % 8) (the tile is 1024-byte aligned).
 __device__ __forceinline__ void store_a8h(uint8_t* a_tile, int r, int c, uint4 h) {
-  *reinterpret_cast<uint4*>(a_tile + (size_t)c * (kTcRows / 8) * 128 + (r >> 3) * 128 + (r & 7) * 16) = h;
+  *reinterpret_cast<uint4*>(a_tile + (r >> 3) * 1024 + (r & 7) * 128 + ((c ^ (r & 7)) << 4)) = h;
 }
 
 // The eight weights of a 4-bit word (field 2a+b holds input 4b+a: byte j
@@ -225,8 +237,8 @@ __device__ __forceinline__ void sb_true(uint32_t sbw, int bits, float* s, float*
 
 // ------------------------------------------------------ raw code ring --
 // The producers stream the tile's raw codes and scale-bias words into a
-// shared-memory ring of three "supersteps" of SG = 8 (or 4) 64-groups each,
-// two supersteps ahead of the one being dequantised.  A superstep's bytes
+// shared-memory ring of four "supersteps" of SG = 4 64-groups each, three
+// supersteps ahead of the one being dequantised.  A superstep's bytes
 // are copied in runs that are contiguous in global memory -- a row's SG
 // groups (gate/up codes: two 16 SG byte runs per row, one per half of the
 // 32-byte group), or 128 rows of one column-block word (down codes) -- so
@@ -234,19 +246,20 @@ __device__ __forceinline__ void sb_true(uint32_t sbw, int bits, float* s, float*
 // copies are laid out so that the dequantising warps (lane l: rows l,
 // l + 32, l + 64, l + 96, one half of the group's inputs) read without bank
 // conflicts:
-//   gate/up codes  [128 rows][2 halves][SG groups][16 B], row stride 272 B
+//   gate/up codes  [128 rows][2 halves][SG groups][16 B], row stride 144 B
 //   gate/up s-b    [128 rows][SG words], row stride 48 B, at kRawSbOff
 //   down codes     [SG groups x words per group][128 rows] u32
 //   down s-b       [SG][128 rows] u32, at kRawDnSbOff
 constexpr int kTcStages = 4;                      // ring of A tiles
-constexpr int kTcBStages = kTcStages;             // token tiles ride with the A stages
+constexpr int kTcBStages = 2 * kTcStages;         // ring of token tiles: requested kTcStages steps ahead
 constexpr uint32_t kTcBRing = kTcBStages * kTcMaxNp * 2 * 128;
-constexpr int kTcRawBufs = 3;                     // supersteps in the raw ring
-constexpr int kTcMaxSG = 8;                       // 64-groups per superstep
-constexpr uint32_t kRawRow = 272, kRawSbRow = 48;
-constexpr uint32_t kRawSbOff = 128 * kRawRow;                 // 34816
-constexpr uint32_t kRawDnSbOff = 8 * kTcMaxSG * 128 * 4;     // 32768
-constexpr uint32_t kTcRawBuf = kRawSbOff + 128 * kRawSbRow;  // 40960 >= kRawDnSbOff + kTcMaxSG * 512
+constexpr int kTcRawBufs = 4;                     // supersteps in the raw ring
+constexpr int kTcMaxSG = 4;                       // 64-groups per superstep
+constexpr uint32_t kRawHalf = kTcMaxSG * 16;      // one half of a row's groups
+constexpr uint32_t kRawRow = 2 * kRawHalf + 16, kRawSbRow = 48;
+constexpr uint32_t kRawSbOff = 128 * kRawRow;                 // 18432
+constexpr uint32_t kRawDnSbOff = 8 * kTcMaxSG * 128 * 4;     // 16384
+constexpr uint32_t kTcRawBuf = kRawSbOff + 128 * kRawSbRow;  // 24576 >= kRawDnSbOff + kTcMaxSG * 512
 static_assert(kTcRawBuf >= kRawDnSbOff + kTcMaxSG * 512, "raw buffer holds the down layout");
 
 __device__ __forceinline__ void cp_async16(void* dst, const void* src) {
@@ -287,7 +300,7 @@ __device__ __forceinline__ void tc_issue_super(const uint8_t* rec, int H, int I,
       const int row = BITS == 4 ? run >> 1 : run, h = BITS == 4 ? run & 1 : 0;
       const uint8_t* src = rec + L.gu_codes + (size_t)(r0 + row) * L.gu_row_bytes +
                            (BITS == 4 ? chunk_off<4>(ng, g0, h) : chunk_off<2>(ng, g0, 0)) + piece * 16;
-      cp_async16(buf + row * kRawRow + h * 128 + piece * 16, src);
+      cp_async16(buf + row * kRawRow + h * kRawHalf + piece * 16, src);
     }
     const int spr = SG / 4;  // 16-byte pieces of a row's scale-bias words
     for (int c = t; c < 128 * spr; c += kTcThreads) {
@@ -322,7 +335,7 @@ template <int MODE, int BITS>
 __device__ __forceinline__ TcRaw tc_read_raw(const uint8_t* buf, int j, int r, int hh) {
   TcRaw w;
   if (MODE == 0) {
-    w.c = *reinterpret_cast<const uint4*>(buf + r * kRawRow + (BITS == 4 ? hh * 128 : 0) + j * 16);
+    w.c = *reinterpret_cast<const uint4*>(buf + r * kRawRow + (BITS == 4 ? hh * kRawHalf : 0) + j * 16);
     if (BITS == 2 && hh) w.c = make_uint4(w.c.z, w.c.w, 0u, 0u);
     w.sb = *reinterpret_cast<const uint32_t*>(buf + kRawSbOff + r * kRawSbRow + j * 4);
   } else {
@@ -366,16 +379,20 @@ __device__ __forceinline__ void tc_dequant(const TcRaw& w, uint8_t* a_tile, int 
 
 // One work unit (item it, row tile r0) of tc_gemm_kernel.  MODE 0: gate/up
 // (M = 2 I, K = H), epilogue SwiGLU -> a[slot][n].  MODE 1: down (M = H,
-// K = I) -> y[slot][row].  Warps 0..7 keep two supersteps of raw codes in
+// K = I) -> y[slot][row].  Warps 0..7 keep three supersteps of raw codes in
 // flight (see the raw code ring); warps w and w + 4 handle the steps
 // s = w (mod 4) (one 64-input group each, one half of its inputs per warp,
 // so four steps are in flight): once the products of step s - 4 are done,
-// lane 0 of warp w requests the step's token tile into B stage s % 4, both
-// warps dequantise into A stage s % 4 and arrive on full[s % 4].  Warp 8
-// (one thread) only waits for full[s % 4] and the token tile, issues the
-// four products and commits them to done[s % 4].  Completion c of a stage's
-// mbarriers belongs to the CTA's step stage + 4 c (steps counted over its
-// work units from gb), so a wait's parity is ((gb + s) / 4) & 1.  Bounded
+// lane 0 of warp w requests the token tile of step s + 4 into the B stage
+// that held step s - 4's (the first four steps' tiles are requested with
+// them), both warps dequantise into A stage s % 4 and arrive
+// on full[s % 4].  So a token tile is in flight for four steps, not on the
+// critical path of its own step.  Warp 8 (one thread) only waits for
+// full[s % 4] and the token tile, issues the four products and commits them
+// to done[s % 4].  Completion c of an A stage's mbarriers belongs to the
+// CTA's step stage + 4 c (steps counted over its work units from gb), so a
+// wait's parity is ((gb + s) / 4) & 1; step s's token tile is in B stage
+// (gb + s) % 8, parity ((gb + s) / 8) & 1.  Bounded
 // waits: on expiry the CTA sets FMOE_STATUS_WAIT_TIMEOUT, waits (bounded)
 // for its committed products and copies and leaves its work loop.
 template <int MODE, int BITS>
@@ -394,21 +411,30 @@ __device__ __forceinline__ void tc_gemm_body(const ExpertSet& es, const int4 it,
   auto raw_buf = [&](int S) { return tsm + (size_t)kTcStages * kTcATile + kTcBRing + (size_t)(S % kTcRawBufs) * kTcRawBuf; };
   // parities count the CTA's steps over all of its work units (gb: steps before this one)
   auto par = [&](int s) { return (uint32_t)(((gb + s) / kTcStages) & 1); };
+  auto par_b = [&](int s) { return (uint32_t)(((gb + s) / kTcBStages) & 1); };
+  auto st_b = [&](int s) { return (gb + s) % kTcBStages; };
+  auto request_b = [&](int s) {
+    const int st = st_b(s);
+    mbar_expect_tx(&bar_b[st], b_bytes);
+    bulk_g2s(b_st(st), bsrc + (size_t)s * b_bytes, b_bytes, &bar_b[st]);
+  };
   if (warp < kTcThreads / 32) {
     // ---- producers
-    const int SG = steps % kTcMaxSG == 0 ? kTcMaxSG : 4, nsup = steps / SG;
-    tc_issue_super<MODE, BITS>(rec, es.H, es.I, r0, 0, SG, raw_buf(0));
-    cp_async_commit();
-    if (nsup > 1) tc_issue_super<MODE, BITS>(rec, es.H, es.I, r0, 1, SG, raw_buf(1));
-    cp_async_commit();
+    const int SG = kTcMaxSG, nsup = steps / SG;  // steps: a multiple of 4
+#pragma unroll
+    for (int S = 0; S < kTcRawBufs - 1; ++S) {
+      if (S < nsup) tc_issue_super<MODE, BITS>(rec, es.H, es.I, r0, S, SG, raw_buf(S));
+      cp_async_commit();
+    }
     bool ok = true;
     int b_last = -1;  // last token tile requested by this lane
 #pragma unroll 1
     for (int S = 0; S < nsup; ++S) {
-      cp_async_wait<1>();          // this thread's copies of superstep S have landed
-      ok = producer_bar_and(ok);   // ... and everyone's; buffer (S + 2) % 3 is no longer read
-      if (!ok) break;              // a wait expired somewhere: every producer leaves here
-      if (S + 2 < nsup) tc_issue_super<MODE, BITS>(rec, es.H, es.I, r0, S + 2, SG, raw_buf(S + 2));
+      cp_async_wait<kTcRawBufs - 2>();  // this thread's copies of superstep S have landed
+      ok = producer_bar_and(ok);        // ... and everyone's; buffer (S + 3) % 4 is no longer read
+      if (!ok) break;                   // a wait expired somewhere: every producer leaves here
+      if (S + kTcRawBufs - 1 < nsup)
+        tc_issue_super<MODE, BITS>(rec, es.H, es.I, r0, S + kTcRawBufs - 1, SG, raw_buf(S + kTcRawBufs - 1));
       cp_async_commit();
       const uint8_t* buf = raw_buf(S);
       // warps w and w + 4 dequantise the steps s = w (mod 4), inputs
@@ -421,10 +447,10 @@ __device__ __forceinline__ void tc_gemm_body(const ExpertSet& es, const int4 it,
           *s_ok = 0;
           break;
         }
-        if (hh == 0 && lane == 0) {  // the step's token tile into B stage s % 4 (free with A stage s % 4)
-          mbar_expect_tx(&bar_b[st], b_bytes);
-          bulk_g2s(b_st(st), bsrc + (size_t)s * b_bytes, b_bytes, &bar_b[st]);
-          b_last = s;
+        if (hh == 0 && lane == 0) {  // token tiles: this step's (the first four), and step s + 4's
+          if (s < kTcStages) request_b(s);
+          if (s + kTcStages < steps) request_b(s + kTcStages);
+          b_last = s + kTcStages < steps ? s + kTcStages : s;
         }
 #pragma unroll
         for (int i = 0; i < 4; ++i) {
@@ -437,28 +463,38 @@ __device__ __forceinline__ void tc_gemm_body(const ExpertSet& es, const int4 it,
       }
     }
     cp_async_wait_all();  // no copy may land after the CTA is gone
-    // on an early exit, the last token tile this lane requested may still be
-    // in flight (each earlier one was waited for by the issuer)
-    if (!ok && b_last >= 0) (void)mbar_wait(&bar_b[b_last % kTcStages], par(b_last));
+    // on an early exit, the last two token tiles this lane requested may
+    // still be in flight (each earlier one was waited for by the issuer)
+    if (!ok && b_last >= 0) {
+      (void)mbar_wait(&bar_b[st_b(b_last)], par_b(b_last));
+      if (b_last >= kTcStages) (void)mbar_wait(&bar_b[st_b(b_last - kTcStages)], par_b(b_last - kTcStages));
+    }
   } else if (lane == 0) {
-    // ---- issuer
+    // ---- issuer: the fewest instructions per step (it shares its SM
+    // sub-partition with dequantising warps).  The descriptors of stage 0
+    // are built once; a stage, and a K = 16 slice inside it, add constant
+    // amounts to their address fields (shared addresses < 256 KB fit the
+    // 14-bit field, so no carry leaves it).
     const uint32_t idesc = umma_idesc_f16(kTcRows, N);
+    const uint64_t ad0 = umma_desc_sw128(smem_u32(a_st(0)));
+    const uint64_t bd0 = umma_desc(smem_u32(b_st(0)), (uint32_t)(N / 8) * 128, 128);
+    constexpr uint64_t kAStage = kTcATile >> 4, kASlice = 32 >> 4;
+    const uint64_t b_stage = b_bytes >> 4, b_slice = (uint64_t)(2 * (N / 8) * 128) >> 4;
     int last_commit = -1;
     bool ok = true;
     for (int s = 0; s < steps; ++s) {
-      const int st = s % kTcStages;
-      if (!mbar_wait(&bar_f[st], par(s)) || !mbar_wait(&bar_b[st], par(s))) {
+      const int st = s % kTcStages, sb = st_b(s);
+      if (!mbar_wait(&bar_f[st], par(s)) || !mbar_wait(&bar_b[sb], par_b(s))) {
         ok = false;
         break;
       }
       tc_fence_after();
-      const uint32_t a0 = smem_u32(a_st(st)), b0 = smem_u32(b_st(st));
-#pragma unroll
-      for (int j = 0; j < 4; ++j) {  // K = 16 slices: two 8-input chunks each
-        const uint64_t ad = umma_desc(a0 + (uint32_t)(2 * j) * (kTcRows / 8) * 128, (kTcRows / 8) * 128, 128);
-        const uint64_t bd = umma_desc(b0 + (uint32_t)(2 * j) * (uint32_t)(N / 8) * 128, (uint32_t)(N / 8) * 128, 128);
-        umma_f16(tmem, ad, bd, idesc, s > 0 || j > 0);
-      }
+      const uint64_t ad = ad0 + (uint64_t)st * kAStage, bd = bd0 + (uint64_t)sb * b_stage;
+      // K = 16 slices (two 8-input chunks each)
+      umma_f16(tmem, ad, bd, idesc, s > 0);
+      umma_f16(tmem, ad + kASlice, bd + b_slice, idesc, true);
+      umma_f16(tmem, ad + 2 * kASlice, bd + 2 * b_slice, idesc, true);
+      umma_f16(tmem, ad + 3 * kASlice, bd + 3 * b_slice, idesc, true);
       umma_commit(&bar_m[st]);
       last_commit = s;
     }
