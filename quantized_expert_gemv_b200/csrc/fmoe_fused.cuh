@@ -117,6 +117,8 @@ constexpr int kCntPart = 4;   // CTAs that published their partial outputs
 constexpr unsigned kPollSleepNs = 32;    // between polls of a counter
 constexpr unsigned kRepollSleepNs = 64;  // between re-reads of an exchange word
 
+constexpr int kTimelinePoints = 48;
+
 struct FusedLayer {
   const uint8_t* experts;
   const uint8_t* shared;
@@ -524,6 +526,28 @@ __device__ __forceinline__ void block_down(const uint8_t* slot, const uint32_t* 
   }
 }
 
+// ------------------------------------------------------------ timeline --
+// Built with FMOE_TIMELINE (quantized_expert_gemv_b200/timeline.py): each
+// CTA records the global timer (ns) at the phase boundaries of one layer of
+// a launch, g_fmoe_ts[CTA][point]; the points are listed in timeline.py.
+// Without it FMOE_TS compiles to nothing.
+#ifdef FMOE_TIMELINE
+__device__ unsigned long long g_fmoe_ts[kFusedMaxCtas][kTimelinePoints];
+__device__ int g_fmoe_ts_layer;
+#define FMOE_TS(i)                                                                   \
+  do {                                                                               \
+    if (l == g_fmoe_ts_layer) {                                                      \
+      unsigned long long t_;                                                         \
+      asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t_)::"memory");               \
+      g_fmoe_ts[blockIdx.x][(i)] = t_;                                               \
+    }                                                                                \
+  } while (0)
+#else
+#define FMOE_TS(i) \
+  do {             \
+  } while (0)
+#endif
+
 // ------------------------------------------------------------ the kernel --
 template <int BITS, int SBITS, int NT>  // routed and shared code widths, tokens per launch
 __global__ void __launch_bounds__(kFusedThreads, 1) fused_stack_kernel(const __grid_constant__ FusedArgs A) {
@@ -725,6 +749,7 @@ __global__ void __launch_bounds__(kFusedThreads, 1) fused_stack_kernel(const __g
   bool aborted = false;
   for (int l = 0; l < A.n_layers; ++l) {
     const FusedLayer& LY = A.layers[l];
+    if (tid == 0) FMOE_TS(0);
     const uint32_t e_logit = base + (uint32_t)l + 1u;
     // ------------------------------------------------------------- A --
     float xv[NT][8];
@@ -742,6 +767,7 @@ __global__ void __launch_bounds__(kFusedThreads, 1) fused_stack_kernel(const __g
     } else {
       // h' and the sums of squares of the previous layer: every CTA has published them
       if (!cta_cnt_wait(kCntH, (unsigned)l * (unsigned)nC)) { aborted = true; break; }
+      if (tid == 0) FMOE_TS(1);
       float4 w0 = make_float4(0.f, 0.f, 0.f, 0.f), w1 = w0;
       const float* wprev = A.layers[l - 1].norm_w;
       if (xthr) {
@@ -768,6 +794,7 @@ __global__ void __launch_bounds__(kFusedThreads, 1) fused_stack_kernel(const __g
         xv[t][6] = h1.z * rt * w1.z; xv[t][7] = h1.w * rt * w1.w;
       }
     }
+    if (tid == 0) FMOE_TS(2);
     if (A.tr_xn && xthr) {
 #pragma unroll
       for (int t = 0; t < NT; ++t) {
@@ -781,7 +808,9 @@ __global__ void __launch_bounds__(kFusedThreads, 1) fused_stack_kernel(const __g
     for (int t = 0; t < NT; ++t) stage_unit(xv[t], xthr, tid >> 3, tid & 7, ngH, sx_of(t));
     // router partial dot products (rows in shared memory, each read once for
     // all tokens), reduced in warp order
+    if (tid == 0) FMOE_TS(3);
     if (nr > 0 && !wait_mb(kMbRouter, (uint32_t)l & 1u)) set_abort();
+    if (tid == 0) FMOE_TS(4);
 #pragma unroll
     for (int m = 0; m < kFusedMaxRouterRows; ++m) {
       float4 wr[2] = {make_float4(0.f, 0.f, 0.f, 0.f), make_float4(0.f, 0.f, 0.f, 0.f)};
@@ -805,6 +834,7 @@ __global__ void __launch_bounds__(kFusedThreads, 1) fused_stack_kernel(const __g
       }
     }
     __syncthreads();
+    if (tid == 0) FMOE_TS(5);
     if (warp == 0) {
       const int t = lane / kFusedMaxRouterRows, m = lane % kFusedMaxRouterRows;
       if (t < NT && m < nr) {
@@ -818,6 +848,7 @@ __global__ void __launch_bounds__(kFusedThreads, 1) fused_stack_kernel(const __g
       __syncwarp();
       if (lane == 0 && nr > 0) cnt_add(A.sync + kCntLogit, (unsigned)nr);
     }
+    if (tid == 0) FMOE_TS(6);
     // ------------------------------------------------------------- E --
     if (warp < kGuWarps) {
       // ---- gate/up warps ----
@@ -828,6 +859,7 @@ __global__ void __launch_bounds__(kFusedThreads, 1) fused_stack_kernel(const __g
         const uint32_t pos = sq + (uint32_t)p;
         const int s = (int)(pos % kSlots);
         const bool ok = wait_mb(kMbFull + s, (pos / kSlots) & 1u);
+        if (tid == 0 && p < 5) FMOE_TS(7 + p);
         float* gb = gred + (pos & 1u) * (NT * kGuWarps * 8);
         const uint8_t* sl = smem + P.slot[s];
         if (ok) {
@@ -845,6 +877,7 @@ __global__ void __launch_bounds__(kFusedThreads, 1) fused_stack_kernel(const __g
         }
         named_bar(kBarGu, kGuThreads);
         if (warp == 0) {
+          if (lane == 0 && p < 5) FMOE_TS(12 + p);
           uint32_t* dx = dnx + s * (NT * kDnxWords);
           if (p < S) {
             float a[NT];
@@ -874,6 +907,7 @@ __global__ void __launch_bounds__(kFusedThreads, 1) fused_stack_kernel(const __g
         // every CTA has published its router rows: (l + 1) (E + 1) in all
         if (issuer && !cnt_wait<false>(A.sync + kCntLogit, (unsigned)(l + 1) * (unsigned)(E + 1))) set_abort();
         named_bar(kBarDn, kDnThreads);
+        if (issuer) FMOE_TS(17);
         const uint64_t* xl_tr = A.x_logit + (size_t)tr * kXLogitStride;
         uint64_t lw[kDnKeys + 1];
 #pragma unroll
@@ -906,6 +940,7 @@ __global__ void __launch_bounds__(kFusedThreads, 1) fused_stack_kernel(const __g
         const uint64_t wk = E <= 2 * kDnThreads ? warp_select_keys<2>(key, k) : warp_select_keys<kDnKeys>(key, k);
         if (lane < k) cand[dw * k + lane] = wk;
         if (__any_sync(0xffffffffu, nan_seen) && lane == 0) s_nan = 1;
+        if (issuer) FMOE_TS(18);
         named_bar(kBarDn, kDnThreads);
         // every down warp merges the warps' candidates itself (same result in
         // each): the top-k ids, and the softmax of their logits
@@ -935,6 +970,7 @@ __global__ void __launch_bounds__(kFusedThreads, 1) fused_stack_kernel(const __g
           }
           if (lane == 0 && s_nan) raise_status(FMOE_STATUS_NAN_LOGIT);
         }
+        if (issuer) FMOE_TS(19);
         // requests, each by its owner: the routed blocks that have a free
         // slot, their down scale-bias entry, L2 prefetches of the later
         // ones, and the next layer's shared block when its slot is free
@@ -947,6 +983,7 @@ __global__ void __launch_bounds__(kFusedThreads, 1) fused_stack_kernel(const __g
           if (S && l + 1 < A.n_layers && nseq < kSlots) issue_pos(l + 1, sq + (uint32_t)nseq, 0, 0);
         }
       }
+      if (issuer) FMOE_TS(20);
       // the other tokens' partial outputs of a CTA without a shared block: zero
       if (NT > 1 && !S) {
         float zr[kDnRowsT];
@@ -968,6 +1005,7 @@ __global__ void __launch_bounds__(kFusedThreads, 1) fused_stack_kernel(const __g
         bool ok = wait_mb(kMbReady + s, (pos / kSlots) & 1u);
         ok = ok && wait_mb(kMbFull + s, (pos / kSlots) & 1u);
         if (p == 0 && S) ok = ok && wait_mb(kMbSbShared, (uint32_t)l & 1u);
+        if (issuer && p < 5) FMOE_TS(21 + p);
         if (ok) {
           const uint8_t* sl = smem + P.slot[s];
           const uint32_t* dx = dnx + s * (NT * kDnxWords);
@@ -1009,6 +1047,7 @@ __global__ void __launch_bounds__(kFusedThreads, 1) fused_stack_kernel(const __g
           }
         }
         named_bar(kBarDn, kDnThreads);  // every down thread is done with the slot
+        if (issuer && p < 5) FMOE_TS(26 + p);
         if (owner && !s_abort) {
           // the slot takes the block three positions on: this layer's, or
           // the next layer's shared block
@@ -1047,9 +1086,11 @@ __global__ void __launch_bounds__(kFusedThreads, 1) fused_stack_kernel(const __g
           __stcg(reinterpret_cast<float4*>(part + row), make_float4(v[0], v[1], v[2], v[3]));
         }
       }
+      if (issuer) FMOE_TS(31);
       named_bar(kBarDn, kDnThreads);
       if (issuer) cnt_release_add(A.sync + kCntPart, 1u);
     }
+    if (issuer) FMOE_TS(32);
     sq += (uint32_t)nseq;
     if (__syncthreads_or(s_abort)) { aborted = true; break; }
     // ------------------------------------------------------------- G --
@@ -1065,6 +1106,7 @@ __global__ void __launch_bounds__(kFusedThreads, 1) fused_stack_kernel(const __g
 #pragma unroll
       for (int t = 0; t < NT; ++t) hres[t] = tid < nd ? A.h[(size_t)t * H + i0 + tid] : 0.f;
       if (!cta_cnt_wait(kCntPart, (unsigned)(l + 1) * (unsigned)nC)) { aborted = true; break; }
+      if (tid == 0) FMOE_TS(33);
       float* sred = reinterpret_cast<float*>(smem + P.red);
       if (pg < ngr) {
         // ngr >= kFusedThreads / (32 NT)
@@ -1082,6 +1124,7 @@ __global__ void __launch_bounds__(kFusedThreads, 1) fused_stack_kernel(const __g
         sred[pg * nv + q] = acc;
       }
       __syncthreads();
+      if (tid == 0) FMOE_TS(34);
       if (warp == 0) {
         float ss[NT];
 #pragma unroll
@@ -1101,6 +1144,7 @@ __global__ void __launch_bounds__(kFusedThreads, 1) fused_stack_kernel(const __g
         __syncwarp();
         if (lane == 0) cnt_release_add(A.sync + kCntH, 1u);  // warp 0 wrote every row of this CTA (nd <= 32)
       }
+      if (tid == 0) FMOE_TS(35);
     }
   }
 

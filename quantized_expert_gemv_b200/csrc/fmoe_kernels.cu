@@ -1450,3 +1450,14 @@ extern "C" int fmoe_layer_forward_noalloc(const fmoe_layer_weights* lw, float* d
 }
 
 #include "fmoe_cache.cuh"
+
+#ifdef FMOE_TIMELINE
+// Timeline build only (see fmoe_fused.cuh): the layer to record, and the
+// records of the last launch, [kFusedMaxCtas][kTimelinePoints] u64 ns.
+extern "C" int fmoe_timeline_layer(int layer) {
+  return cudaMemcpyToSymbol(g_fmoe_ts_layer, &layer, sizeof(int)) == cudaSuccess ? FMOE_OK : FMOE_ERR_CUDA;
+}
+extern "C" int fmoe_timeline_read(void* host) {
+  return cudaMemcpyFromSymbol(host, g_fmoe_ts, sizeof(g_fmoe_ts)) == cudaSuccess ? FMOE_OK : FMOE_ERR_CUDA;
+}
+#endif

@@ -225,6 +225,13 @@ def test_host_validation_of_the_later_entry_points(fm):
     assert fm.fmoe_fused_max_tokens(False) == 4 and fm.fmoe_fused_max_tokens(True) == 8
 
 
+def test_product_library_has_no_timeline_build(fm):
+    """The timer reads of the per-phase timeline exist only in the separate
+    FMOE_TIMELINE build (quantized_expert_gemv_b200/timeline.py)."""
+    assert not hasattr(fm._lib, "fmoe_timeline_read")
+    assert not hasattr(fm._lib, "fmoe_timeline_layer")
+
+
 def test_workspace_layout(fm):
     d = fm.LayerDesc()
     n1, n64 = fm.fmoe_workspace_bytes(d, 1), fm.fmoe_workspace_bytes(d, 64)
