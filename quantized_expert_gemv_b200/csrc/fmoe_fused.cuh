@@ -807,10 +807,14 @@ __global__ void __launch_bounds__(kFusedThreads, 1) fused_stack_kernel(const __g
 #pragma unroll
     for (int t = 0; t < NT; ++t) stage_unit(xv[t], xthr, tid >> 3, tid & 7, ngH, sx_of(t));
     // router partial dot products (rows in shared memory, each read once for
-    // all tokens), reduced in warp order
+    // all tokens): value t R + m of a thread is token t's product with row
+    // m; each warp reduces all of them at once, then warp 0 adds the warps'
+    // sums in warp order
     if (tid == 0) FMOE_TS(3);
     if (nr > 0 && !wait_mb(kMbRouter, (uint32_t)l & 1u)) set_abort();
     if (tid == 0) FMOE_TS(4);
+    constexpr int kRV = NT * kFusedMaxRouterRows;  // values per thread: a power of two
+    float dv[kRV];
 #pragma unroll
     for (int m = 0; m < kFusedMaxRouterRows; ++m) {
       float4 wr[2] = {make_float4(0.f, 0.f, 0.f, 0.f), make_float4(0.f, 0.f, 0.f, 0.f)};
@@ -829,8 +833,15 @@ __global__ void __launch_bounds__(kFusedThreads, 1) fused_stack_kernel(const __g
         d = fmaf(wr[1].y, xv[t][5], d);
         d = fmaf(wr[1].z, xv[t][6], d);
         d = fmaf(wr[1].w, xv[t][7], d);
-        d = warp_sum(d);
-        if (lane == 0) s_rp[warp][t][m] = d;
+        dv[t * kFusedMaxRouterRows + m] = d;
+      }
+    }
+    {
+      const float d = warp_sum_multi<kRV>(dv);  // lane l: the total of value l / (32 / kRV)
+      constexpr int kLanesPer = 32 / kRV;
+      if ((lane & (kLanesPer - 1)) == 0) {
+        const int v = lane / kLanesPer;
+        s_rp[warp][v / kFusedMaxRouterRows][v % kFusedMaxRouterRows] = d;
       }
     }
     __syncthreads();
