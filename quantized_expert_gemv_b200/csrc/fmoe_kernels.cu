@@ -830,7 +830,7 @@ static int launch_experts(const ExpertSet& es, const float* xn, const int32_t* i
                                                                       gamma, gw->tscale, sc);
         const int n_sm = device_sms();
         const int u0 = max_tc * (2 * es.I / kTcRows);
-        tc_gemm_kernel<0><<<u0 < n_sm ? u0 : n_sm, kTcThreads + 32, tc_smem_bytes(), st>>>(es, *gw, tcx, a, sc);
+        tc_gemm_kernel<0><<<u0 < n_sm ? u0 : n_sm, kTcBlock, tc_smem_bytes(), st>>>(es, *gw, tcx, a, sc);
       }
       if (small_only) {
         down_group_small_kernel<<<dim3(nb[0] + nb[1], (es.H + kDnRows - 1) / kDnRows), kDnRows, 4 * sas, st>>>(
@@ -847,7 +847,7 @@ static int launch_experts(const ExpertSet& es, const float* xn, const int32_t* i
                                                                       nullptr, nullptr, sc);
         const int n_sm = device_sms();
         const int u1 = max_tc * (es.H / kTcRows);
-        tc_gemm_kernel<1><<<u1 < n_sm ? u1 : n_sm, kTcThreads + 32, tc_smem_bytes(), st>>>(es, *gw, tca, y, sc);
+        tc_gemm_kernel<1><<<u1 < n_sm ? u1 : n_sm, kTcBlock, tc_smem_bytes(), st>>>(es, *gw, tca, y, sc);
       }
       return cuda_rc(cudaGetLastError());
     }

@@ -43,7 +43,17 @@ namespace fmoe {
 
 constexpr int kTcMinTokens = 3;   // from 3 tokens per expert the tensor-core path is faster (measured, 24-bit inputs)
 constexpr int kTcMaxNp = kTcItemMax;  // tokens per tensor-core item (N = 2 Np <= 64)
-constexpr int kTcThreads = 256;
+constexpr int kTcThreads = 256;  // producer threads (8 warps)
+// The CTA has 12 warps.  Warps are spread over the SM's four sub-partitions
+// by index modulo 4; the issuing thread (warp 0) gets sub-partition 0 to
+// itself (warps 4 and 8 only join the barriers and the epilogue), the eight
+// producer warps sit on sub-partitions 1-3, so the MMA issue loop is not
+// starved of issue slots by the dequantisation (measured: ~0.65 us per step
+// when it shared a sub-partition with two producer warps).
+constexpr int kTcBlock = 384;
+__host__ __device__ constexpr int tc_producer_of(int warp) {  // producer index 0..7 of a warp, or -1
+  return (warp & 3) == 0 || warp == 11 ? -1 : warp - 1 - warp / 4;
+}
 constexpr int kTcRows = 128;      // weight rows per CTA (the MMA's M)
 constexpr uint32_t kTcATile = kTcRows * 64 * 2;  // fp16 A tile of one 64-input group
 
@@ -289,9 +299,10 @@ __device__ __forceinline__ bool producer_bar_and(bool v) {
 // gate n, up n interleaved, row-major codes); MODE 1: down rows
 // (column-block codes: one word per row and column block).
 template <int MODE, int BITS>
-__device__ __forceinline__ void tc_issue_super(const uint8_t* rec, int H, int I, int r0, int S, int SG, uint8_t* buf) {
+__device__ __forceinline__ void tc_issue_super(const uint8_t* rec, int H, int I, int r0, int S, int SG, uint8_t* buf,
+                                               int t) {
   const RecordLayout L = record_layout(BITS, H, I);
-  const int t = threadIdx.x, g0 = S * SG;
+  const int g0 = S * SG;
   if (MODE == 0) {
     const int ng = H / 64;
     const int runs = BITS == 4 ? 256 : 128;  // (row, half) runs of 16 SG bytes; 2-bit groups are one 16-byte chunk
@@ -418,12 +429,13 @@ __device__ __forceinline__ void tc_gemm_body(const ExpertSet& es, const int4 it,
     mbar_expect_tx(&bar_b[st], b_bytes);
     bulk_g2s(b_st(st), bsrc + (size_t)s * b_bytes, b_bytes, &bar_b[st]);
   };
-  if (warp < kTcThreads / 32) {
+  const int pw = tc_producer_of(warp), pt = pw * 32 + lane;  // producer warp / thread index
+  if (pw >= 0) {
     // ---- producers
     const int SG = kTcMaxSG, nsup = steps / SG;  // steps: a multiple of 4
 #pragma unroll
     for (int S = 0; S < kTcRawBufs - 1; ++S) {
-      if (S < nsup) tc_issue_super<MODE, BITS>(rec, es.H, es.I, r0, S, SG, raw_buf(S));
+      if (S < nsup) tc_issue_super<MODE, BITS>(rec, es.H, es.I, r0, S, SG, raw_buf(S), pt);
       cp_async_commit();
     }
     bool ok = true;
@@ -434,14 +446,14 @@ __device__ __forceinline__ void tc_gemm_body(const ExpertSet& es, const int4 it,
       ok = producer_bar_and(ok);        // ... and everyone's; buffer (S + 3) % 4 is no longer read
       if (!ok) break;                   // a wait expired somewhere: every producer leaves here
       if (S + kTcRawBufs - 1 < nsup)
-        tc_issue_super<MODE, BITS>(rec, es.H, es.I, r0, S + kTcRawBufs - 1, SG, raw_buf(S + kTcRawBufs - 1));
+        tc_issue_super<MODE, BITS>(rec, es.H, es.I, r0, S + kTcRawBufs - 1, SG, raw_buf(S + kTcRawBufs - 1), pt);
       cp_async_commit();
       const uint8_t* buf = raw_buf(S);
       // warps w and w + 4 dequantise the steps s = w (mod 4), inputs
       // 32 (w / 4) .. + 31 of them, always into A stage s % 4 = w % 4
 #pragma unroll 1
-      for (int j = warp & 3; j < SG; j += kTcStages) {
-        const int s = S * SG + j, st = s % kTcStages, hh = warp >> 2;
+      for (int j = pw & 3; j < SG; j += kTcStages) {
+        const int s = S * SG + j, st = s % kTcStages, hh = pw >> 2;
         if (s >= kTcStages && !mbar_wait(&bar_m[st], par(s - kTcStages))) {  // products of step s - 4 done
           ok = false;
           *s_ok = 0;
@@ -469,9 +481,8 @@ __device__ __forceinline__ void tc_gemm_body(const ExpertSet& es, const int4 it,
       (void)mbar_wait(&bar_b[st_b(b_last)], par_b(b_last));
       if (b_last >= kTcStages) (void)mbar_wait(&bar_b[st_b(b_last - kTcStages)], par_b(b_last - kTcStages));
     }
-  } else if (lane == 0) {
-    // ---- issuer: the fewest instructions per step (it shares its SM
-    // sub-partition with dequantising warps).  The descriptors of stage 0
+  } else if (warp == 0 && lane == 0) {
+    // ---- issuer: the fewest instructions per step.  The descriptors of stage 0
     // are built once; a stage, and a K = 16 slice inside it, add constant
     // amounts to their address fields (shared addresses < 256 KB fit the
     // 14-bit field, so no carry leaves it).
@@ -549,8 +560,12 @@ __device__ __forceinline__ void tc_gemm_body(const ExpertSet& es, const int4 it,
 // grid never holds idle CTAs; tensor memory, mbarriers and rings carry over
 // from unit to unit (steps % 4 == 0 keeps every ring stage in step).
 template <int MODE>
-__global__ void __launch_bounds__(kTcThreads + 32, 1)
+__global__ void __launch_bounds__(kTcBlock, 1)
 tc_gemm_kernel(ExpertSet es, GroupWork w, const uint8_t* __restrict__ staged, float* __restrict__ out, TcScale sc) {
+  static_assert(tc_producer_of(1) == 0 && tc_producer_of(3) == 2 && tc_producer_of(5) == 3 &&
+                    tc_producer_of(7) == 5 && tc_producer_of(9) == 6 && tc_producer_of(10) == 7 &&
+                    tc_producer_of(0) < 0 && tc_producer_of(4) < 0 && tc_producer_of(8) < 0 && tc_producer_of(11) < 0,
+                "producer warps");
   extern __shared__ __align__(1024) unsigned char tsm[];
   __shared__ uint64_t bar_b[kTcBStages], bar_m[kTcStages], bar_f[kTcStages];
   __shared__ uint32_t s_tmem;
