@@ -308,9 +308,11 @@ __device__ __forceinline__ void gateup_rows_multi(const uint8_t* rec, const Expe
 // Item (group, first, m): the group's slots first .. first + m - 1; the
 // tokens' staged inputs are copied from xs (stage_tokens_kernel).  Also
 // computes gamma[t] = sigmoid(w_sg . xn[t]) for the shared expert's tokens
-// when gamma is given.
+// when gamma is given.  Used for hidden sizes below 2048 (larger ones take
+// gateup_bulk_kernel); one CTA per SM's worth of registers, so that the
+// 24-bit dot products of MB tokens do not spill.
 template <int MB>
-__global__ void __launch_bounds__(kGrpThreads, MB <= 4 ? 2 : 1)
+__global__ void __launch_bounds__(kGrpThreads, 1)
 gateup_group_kernel(ExpertSet es, GroupWork w, int bucket, int max_items, const float* __restrict__ xn,
                     const unsigned char* __restrict__ xs, float* __restrict__ a, const float* __restrict__ w_sg,
                     float* __restrict__ gamma) {
