@@ -549,6 +549,8 @@ __device__ __forceinline__ void down_row_multi(const uint8_t* rec, const ExpertS
   const RecordLayout L = record_layout(BITS, H, I);
   const uint32_t* codes = reinterpret_cast<const uint32_t*>(rec + L.down_codes) + row;
   const uint32_t* sbw = reinterpret_cast<const uint32_t*>(rec + L.down_sb) + row;
+  // unrolled so that several groups' loads are in flight per thread
+#pragma unroll 4
   for (int g = 0; g < ngI; ++g) {
     uint32_t wd[kWpg];
 #pragma unroll

@@ -529,6 +529,26 @@ def test_few_tokens_through_persistent_kernel(wl):
     assert fm.fmoe_read_status() == 0
 
 
+@pytest.mark.parametrize("wl", [SMALL, SMALL2], ids=["small4", "small2"])
+def test_stack_trace_beyond_persistent_tokens(wl):
+    """A traced stack of more tokens than the persistent kernel takes (the
+    grouped path, layer by layer, the trace copied from the workspace):
+    every layer of every token against the oracle, and the traced stack
+    gives the bits of the untraced one."""
+    L = 3
+    lws = [device_layer(wl, l) for l in range(L)]
+    los = [oracle_layer(wl, l) for l in range(L)]
+    for l, lo in enumerate(los):
+        lo.layer = l
+    T = fm.fmoe_fused_max_tokens(True) + 2
+    x = synth.tokens(wl, T, stream=67)
+    h_t, xn_t = traced_stack_check(wl, lws, los, x, "grouped")
+    h, xn = dev(x), dev(x)
+    fm.fmoe_stack_forward(lws, h, xn, fm.alloc_workspace(lws[0].desc, T))
+    assert np.array_equal(host(h), h_t) and np.array_equal(host(xn), xn_t)
+    assert fm.fmoe_read_status() == 0
+
+
 @pytest.mark.parametrize("T", [1, 3, 6])
 def test_host_state_entry_point_matches_device_entry_point(T):
     """fmoe_layer_forward_host (pinned host h/xn in, h'/xn' out, one copy
