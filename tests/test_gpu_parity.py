@@ -310,6 +310,29 @@ def test_layer_forward_tiny(wl, T, path):
     assert fm.fmoe_read_status() == 0
 
 
+@pytest.mark.parametrize("wl,T", [(synth.Workload(hidden=1024, inter=512, n_experts=1024, top_k=8), 1),
+                                  (synth.Workload(hidden=1024, inter=512, n_experts=1024, top_k=8), 6),
+                                  (synth.Workload(hidden=256, inter=256, n_experts=64, top_k=1), 1),
+                                  (synth.Workload(hidden=256, inter=256, n_experts=64, top_k=1), 3),
+                                  (synth.Workload(hidden=256, inter=256, n_experts=4, top_k=4), 1),
+                                  (synth.Workload(hidden=256, inter=256, n_experts=4, top_k=4), 2)],
+                         ids=["E1024-k8-T1", "E1024-k8-T6", "k1-T1", "k1-T3", "k=E-T1", "k=E-T2"])
+def test_layer_forward_routing_extremes(wl, T, path):
+    """The largest routing the library takes (1024 experts, top-8; the
+    persistent kernel's router rows do not cover it, so the one-kernel-per-
+    step path runs), top-1, and every expert selected (k = E): every output
+    of every token against the oracle."""
+    lw = device_layer(wl)
+    lw_o = oracle_layer(wl, 0, slots=[wl.n_experts])
+    x = synth.tokens(wl, T, stream=71)
+    h, xn = dev(x), dev(x)
+    ws = fm.alloc_workspace(lw.desc, T)
+    fm.fmoe_layer_forward(lw, h, xn, ws)
+    pmap(lambda t: check_layer_token(wl, lw_o, ws, lw.desc, T, t, x[t], x[t], host(h)[t], host(xn)[t], f"t={t}"),
+         range(T))
+    assert fm.fmoe_read_status() == 0
+
+
 @pytest.fixture(scope="module")
 def full_layer():
     wl = synth.LAYER
