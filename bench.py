@@ -381,17 +381,17 @@ def job_rate(units_per_rank: int, world: int, ms_max: float) -> float:
 
 
 # ----------------------------------------------------------- CPU baseline --
-def oracle_layer_steps(max_steps: int, seconds: float, layers: int):
+def oracle_layer_steps(max_steps: int, seconds: float, layers: int, wl=None):
     """Times the fp64 oracle, as it stands, on the host (one thread or, after
     oracle.set_threads, the OpenMP timing build): successive
-    single-token layer forwards of the benchmark workload through the layer
-    stack, until `max_steps` are done or `seconds` of oracle time are spent.
-    The selected experts are regenerated on demand; generation is not timed.
-    Returns (steps done, seconds spent in the oracle)."""
+    single-token layer forwards of the benchmark workload (or `wl`) through
+    the layer stack, until `max_steps` are done or `seconds` of oracle time
+    are spent.  The selected experts are regenerated on demand; generation is
+    not timed.  Returns (steps done, seconds spent in the oracle)."""
     import numpy as np
     import oracle
     import synth
-    wl = synth.LAYER
+    wl = wl or synth.LAYER
     done, spent = 0, 0.0
     cache = {}
     while done < max_steps and spent < seconds:
@@ -410,6 +410,33 @@ def oracle_layer_steps(max_steps: int, seconds: float, layers: int):
     return done, spent
 
 
+def oracle_batched_tokens(n_tokens: int, T: int = 64):
+    """Times the fp64 oracle on the first n_tokens tokens of the 64-token
+    Zipf-routed step of the batched measurement (the same routing draw,
+    given logits): per token the layer with its selected experts, which the
+    oracle computes token by token.  Expert generation is not timed.
+    Returns (tokens done, seconds spent in the oracle)."""
+    import numpy as np
+    import oracle
+    import synth
+    wl = synth.LAYER
+    lg = synth.zipf_gumbel_logits(wl, 0, T)[0]
+    xs = synth.tokens(wl, T, stream=900)
+    lw = oracle.LayerWeights(synth.router(wl, 0), synth.shared_gate(wl, 0), synth.norm_weight(wl, 0),
+                             {wl.n_experts: synth.expert(wl, 0, wl.n_experts)})
+    spent = 0.0
+    for t in range(n_tokens):
+        ids, _, _ = oracle.topk_softmax(lg[t].astype(np.float64), wl.top_k)
+        for e in ids:
+            if int(e) not in lw.experts:
+                lw.experts[int(e)] = synth.expert(wl, 0, int(e))
+        x = xs[t].astype(np.float64)
+        t0 = time.perf_counter()
+        oracle.layer_token(wl, lw, x, x, logits_in=lg[t])
+        spent += time.perf_counter() - t0
+    return n_tokens, spent
+
+
 def host_cores() -> int:
     """Cores this process may run on (the affinity mask, not the machine)."""
     try:
@@ -426,13 +453,23 @@ def cpu_baseline(seconds: float, layers: int) -> dict:
     cores = host_cores()
     oracle.set_threads(cores)
     done, spent = oracle_layer_steps(10 ** 6, seconds / 2, layers)
+    # the other workloads, on all cores, small bounded samples
+    import synth
+    d2, s2 = oracle_layer_steps(10 ** 6, min(3.0, seconds / 5), layers, wl=synth.LAYER_INT2)
+    nb, sb = oracle_batched_tokens(8)
     oracle.set_threads(1)
     done1, spent1 = oracle_layer_steps(10 ** 6, seconds / 2, layers)
     return {"value": done / spent, "unit": UNIT, "cores": cores, "kind": "oracle",
             "sample": f"{done} single-token layer forwards of the benchmark workload (fp64 C oracle, OpenMP over "
                       f"output rows on {cores} cores; expert generation excluded), {spent:.1f} s",
             "single_thread": {"value": done1 / spent1, "unit": UNIT, "cores": 1,
-                              "sample": f"{done1} layer forwards on one thread, {spent1:.1f} s"}}
+                              "sample": f"{done1} layer forwards on one thread, {spent1:.1f} s"},
+            "int4_chain_tokens_per_s": done / spent / layers,
+            "int2_chain": {"layer_fwd_per_s": d2 / s2, "tokens_per_s": d2 / s2 / layers, "cores": cores,
+                           "sample": f"{d2} layer forwards of 2-bit routed / 4-bit shared layers, {s2:.1f} s"},
+            "batched": {"tokens_per_s": nb / sb, "ms_per_64_token_step": 64 * sb / nb * 1e3, "cores": cores,
+                        "sample": f"the first {nb} tokens of the 64-token Zipf step (given logits), "
+                                  f"{sb:.1f} s; the oracle computes token by token"}}
 
 
 def run_reference(args):
