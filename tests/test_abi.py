@@ -286,3 +286,22 @@ def test_header_and_c_example_compile_as_c():
     r = subprocess.run([gcc, "-std=c11", "-Wall", "-Werror", "-fsyntax-only", "-I", os.path.join(root, "include"),
                         "-I", cuda_inc, src], capture_output=True, text=True)
     assert r.returncode == 0, r.stderr
+
+
+def test_timeline_points_match_the_kernel():
+    """Every timer point of the persistent kernel has a name in the timeline
+    tool, and every named point is recorded somewhere in the kernel."""
+    import re
+    from pathlib import Path
+    from quantized_expert_gemv_b200 import timeline
+    src = (Path(__file__).resolve().parents[1] / "quantized_expert_gemv_b200" / "csrc" / "fmoe_fused.cuh").read_text()
+    used = set()
+    calls = re.findall(r"FMOE_TS\(([0-9][^)]*)\)", src)
+    assert len(calls) == src.count("FMOE_TS(") - 2  # all but the two macro definitions
+    for expr in calls:
+        m = re.fullmatch(r"(\d+)(?: \+ p)?", expr.strip())
+        assert m, expr
+        base = int(m.group(1))
+        used.update(range(base, base + 5) if "+ p" in expr else [base])
+    assert used == set(timeline.POINTS), sorted(used ^ set(timeline.POINTS))
+    assert max(used) < timeline.N_POINTS
