@@ -254,7 +254,7 @@ def workload_config(layers: int, experts: int = 512) -> dict:
 # DRAM bytes (read + write) of one full-size int4 layer of fused_stack_kernel,
 # from an ncu capture (profiles/fused_stack_kernel_int4_batch1.md), valid for
 # the kernel sources whose digest is given; any later change to them voids it.
-TRAFFIC_PER_LAYER = {"sources_sha256_16": "850bd1180038bdb9", "bytes": 44_008_960}
+TRAFFIC_PER_LAYER = {"sources_sha256_16": "9aba729bf237347f", "bytes": 43_996_672}
 TRAFFIC_SOURCES = ("fmoe_fused.cuh", "fmoe_device.cuh", "fmoe_layout.h")  # the kernel's sources
 
 

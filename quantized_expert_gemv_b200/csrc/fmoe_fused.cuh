@@ -1,4 +1,4 @@
-// fmoe_fused.cuh -- one persistent kernel for a stack of MoE layers, batch 1.
+// fmoe_fused.cuh -- one persistent kernel for a stack of MoE layers, one or two tokens.
 //
 // One CTA per SM, launched cooperatively so that every CTA is resident.  The
 // experts' intermediate dimension is cut into column blocks of w = 8 (4-bit)
