@@ -406,7 +406,7 @@ def fmoe_tc_min_tokens() -> int:
 
 
 def fmoe_fused_max_tokens(stack: bool = False) -> int:
-    """Largest T run token by token through the persistent kernel (layer or stack call)."""
+    """Largest T that runs through the persistent kernel (layer or stack call), two tokens per launch."""
     return int(_lib.fmoe_fused_max_tokens(int(bool(stack))))
 
 

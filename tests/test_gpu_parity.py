@@ -367,9 +367,9 @@ def test_layer_forward_full_size_int2(wl, path):
 def test_fused_and_per_step_paths_agree(full_layer):
     """The persistent kernel and the one-kernel-per-step path route alike and
     agree to well inside the oracle tolerance.  They are not bit-identical:
-    the persistent kernel rounds the SwiGLU outputs to 16-bit fixed point
-    per column block of 8 units, the per-step path per 64-group, and it sums
-    the expert outputs in another order."""
+    the persistent kernel stages the SwiGLU outputs as 24-bit block floating
+    point per column block of 8 units, the per-step path per 64-group, and it
+    sums the expert outputs in another order."""
     wl, lw, _ = full_layer
     x = synth.tokens(wl, 1, stream=35)
     outs = {}
