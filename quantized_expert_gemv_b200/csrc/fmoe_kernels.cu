@@ -1,15 +1,27 @@
 // fmoe_kernels.cu -- sm_100a kernels and the C ABI of the quantised MoE
 // expert forward (see include/fmoe.h for the contract of every entry point).
 //
-// Kernels, in the order one layer runs them:
-//   router_partial_kernel  fp32 router rows x normed input, split along H
-//   topk_kernel            sums the splits, warp top-k, softmax of the k
-//                          selected logits, shared-expert sigmoid gate
-//   gateup_kernel          dequantising gate/up products of every selected
-//                          expert and the shared expert, fused SwiGLU
-//   down_kernel            dequantising down product
-//   combine_kernel         weighted combine + residual + shared gate, then the
-//                          two-pass RMSNorm
+// Which kernels run a layer:
+//   - one or two tokens (and up to fmoe_fused_max_tokens in pairs): the
+//     persistent fused_stack_kernel (fmoe_fused.cuh), whole layers and
+//     layer stacks in one cooperative launch;
+//   - otherwise (or with fmoe_set_fused(0)), one kernel per step, in the
+//     order one layer runs them:
+//       router_partial_kernel  fp32 router rows x normed input, split along H
+//       topk_kernel            sums the splits, warp top-k, softmax of the k
+//                              selected logits, shared-expert sigmoid gate
+//       gateup_kernel          dequantising gate/up products of every
+//                              selected expert and the shared expert, fused
+//                              SwiGLU (T = 1)
+//       down_kernel            dequantising down product (T = 1)
+//       combine_kernel         weighted combine + residual + shared gate,
+//                              then the two-pass RMSNorm
+//     with T > 1 the expert products group the slots by expert first
+//     (fmoe_batched.cuh: integer-dot GEMVs; fmoe_tc.cuh: tcgen05 GEMM for
+//     experts with fmoe_tc_min_tokens or more tokens);
+//   - off the layer: the packer (pack_codes_kernel, pack_sb_kernel) and the
+//     quantiser (quantize_groups_kernel); the host expert tier's cache
+//     (fmoe_cache.cuh).
 // Source pages: "What is Flash-MoE?" (a2a-mcp.org), sections "Understanding
 // Mixture-of-Experts" (top-4 of 512 plus one shared expert),
 // "2. FMA-optimised dequantisation kernels" and "3. Hand-tuned Metal compute
@@ -874,12 +886,13 @@ static int launch_combine(const float* y, const float* weights, const float* gam
   return cuda_rc(cudaGetLastError());
 }
 
-// ----------------------------------------------------- fused batch-1 path --
+// ------------------------------------------------- persistent-kernel path --
 static int g_fused_enabled = 1;
 // Token counts up to which T > 1 runs through the persistent kernel, two
 // tokens per launch (measured: a layer of T = 2 / 4 / 8 tokens takes
-// 77 / 138 / 197 us on the grouped path against 21.4 us per token and layer
-// in a one-token stack launch; a single-layer launch costs ~30 us).
+// 77 / 138 / 197 us on the grouped path against 31.9 / 60.3 / 124.7 us per
+// layer in stack launches of token pairs; a single-layer launch costs
+// ~34 us).
 constexpr int kFusedTokensLayer = 4;
 constexpr int kFusedTokensStack = 8;
 
