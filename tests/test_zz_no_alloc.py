@@ -2,9 +2,10 @@
 against fmoe_layer_forward with a caller workspace.
 
 Both run the same kernels, so two calls in a row (the second reading what
-the first wrote) must give bit-identical h and xn on both paths: at T = 1
-(persistent kernel where the shape admits it), at T = 3 (one kernel per
-step), and at the largest T the 12 MiB scratch admits.  A T beyond that is
+the first wrote) must give bit-identical h and xn, with the persistent
+kernel enabled and disabled: at T = 1, at T = 3 (a pair and a single token
+through the persistent kernel, or one kernel per step), and at the largest
+T the 12 MiB scratch admits (the grouped path).  A T beyond that is
 refused on the host before anything is launched.  The file name sorts last
 so that the test also runs after everything else in the suite has used the
 library.
