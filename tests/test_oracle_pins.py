@@ -190,6 +190,23 @@ def test_topk_weights_sum_to_one_and_follow_logit_order():
         assert set(ids.tolist()) == set(np.argsort(-lg, kind="stable")[:4].tolist())
 
 
+def test_topk_one_selects_the_maximum_with_weight_one():
+    lg = np.linspace(-1, 1, 64)[::-1].copy()
+    lg[37] = 5.0
+    ids, p, _ = oracle.topk_softmax(lg, 1)
+    assert ids.tolist() == [37] and p.tolist() == [1.0]
+
+
+def test_topk_of_every_logit_is_the_full_softmax_in_descending_order():
+    # k = E: every expert selected; the weights are the softmax over all of
+    # them, listed from the largest logit down (ties: lower index first)
+    lg = np.array([0.5, 2.0, -1.0, 2.0, 0.0])
+    ids, p, _ = oracle.topk_softmax(lg, 5)
+    assert ids.tolist() == [1, 3, 0, 4, 2]
+    e = np.exp(lg - lg.max())
+    assert np.allclose(p, (e / e.sum())[[1, 3, 0, 4, 2]], rtol=1e-15)
+
+
 def test_topk_nan_is_never_selected_and_is_reported():
     lg = np.linspace(1, 0, 16)
     lg[0] = np.nan
