@@ -608,3 +608,25 @@ def test_layer_error_scales_compose_the_steps():
     _, _, Sh, Sx = oracle.combine_rmsnorm(ref["y"], ref["p"], ref["gamma"], x, lw.norm_w, wl.eps,
                                           S_y=ref["S_y"], S_gamma=ref["S_gamma"])
     assert np.array_equal(Sh, ref["S_h"]) and np.array_equal(Sx, ref["S_xn"])
+
+
+def test_openmp_timing_build_computes_the_same_values():
+    """The OpenMP build that the CPU baseline times (output rows over
+    threads) gives the plain build's values bit for bit: the rows are
+    independent, each summed in the same order."""
+    wl = synth.TINY
+    lw = oracle.LayerWeights(synth.router(wl, 0), synth.shared_gate(wl, 0), synth.norm_weight(wl, 0),
+                             dict(zip(range(wl.n_experts + 1), synth.experts(wl, 0, range(wl.n_experts + 1)))))
+    x = synth.tokens(wl, 3, stream=5).astype(np.float64)
+    keys = ("h", "xn", "S_h", "S_xn", "p", "gamma")
+    try:
+        oracle.set_threads(1)
+        plain = [oracle.layer_token(wl, lw, x[t], x[t]) for t in range(3)]
+        oracle.set_threads(4)
+        omp = [oracle.layer_token(wl, lw, x[t], x[t]) for t in range(3)]
+    finally:
+        oracle.set_threads(1)
+    for a, b in zip(plain, omp):
+        assert a["ids"].tolist() == b["ids"].tolist()
+        for k in keys:
+            assert np.array_equal(np.asarray(a[k]), np.asarray(b[k])), k
