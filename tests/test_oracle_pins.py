@@ -351,6 +351,27 @@ def test_layer_logits_given_routes_on_them():
     assert out["ids"].tolist() == [11, 4, 9, 0]
 
 
+def test_layer_residual_enters_only_the_sum():
+    """The router, the shared gate and every expert read the normed input xn
+    only; the residual stream h is added to their combined output.  So with
+    xn fixed, moving h changes nothing but h', by exactly the move."""
+    wl = synth.TINY
+    lw = _tiny_layer(wl)
+    x = synth.tokens(wl, 1, stream=7)[0].astype(np.float64)
+    h1 = synth.tokens(wl, 1, stream=8)[0].astype(np.float64) * 4
+    h2 = -3 * h1 + 1.0
+    a = oracle.layer_token(wl, lw, h1, x)
+    b = oracle.layer_token(wl, lw, h2, x)
+    assert a["ids"].tolist() == b["ids"].tolist()
+    for key in ("logits", "p", "gamma", "y"):
+        assert np.array_equal(a[key], b[key]), key
+    moved = b["h"] - a["h"]
+    assert np.allclose(moved, h2 - h1, rtol=1e-13, atol=1e-13 * np.abs(h1).max())
+    # and the router reads xn: the same h with another xn routes differently
+    c = oracle.layer_token(wl, lw, h1, x[::-1].copy())
+    assert not np.array_equal(a["logits"], c["logits"])
+
+
 # -------------------------------------------------- quantiser round trip ----
 
 @pytest.mark.parametrize("bits", [4, 2])
@@ -416,6 +437,63 @@ def test_stored_format_quantiser_error_bound_and_special_groups():
         assert np.all(np.abs(back - w).reshape(-1, 64) <= bound[:, None])
         assert s[-1] == 0 and np.all(q[-64:] == 0) and synth.bf16_to_f32(b[-1:])[0] == np.float32(0.375)
         assert q.max() <= qmax
+
+
+def test_stored_format_quantiser_rounds_bf16_to_nearest_even():
+    """The stored scale and bias are the nearest bf16 values, ties to the
+    even significand (bf16 keeps 8 significant bits: 1 + 2^-8 lies halfway
+    between 1 and 1 + 2^-7).  Groups of 64 built so that the fp32 minimum and
+    the fp32 scale (hi - lo) / 15 are exactly such halfway values."""
+    G = 64
+
+    def group(lo, span):
+        g = np.linspace(0.0, 1.0, G).astype(np.float32) * np.float32(span) + np.float32(lo)
+        g[0], g[-1] = lo, np.float32(lo) + np.float32(span)
+        return g
+
+    cases = [  # (minimum, hi - lo, expected bias bits, expected scale bits)
+        (1 + 2.0 ** -8, 15 * (1 + 2.0 ** -8), 0x3F80, 0x3F80),       # ties down to even
+        (1 + 3 * 2.0 ** -8, 15 * (1 + 3 * 2.0 ** -8), 0x3F82, 0x3F82),  # ties up to even
+        (-(1 + 2.0 ** -8), 15 * 0.5, 0xBF80, 0x3F00),                # negative tie, exact scale
+        (1 + 2.0 ** -8 + 2.0 ** -20, 15 * (1 + 2.0 ** -8 + 2.0 ** -20), 0x3F81, 0x3F81),  # above the tie
+    ]
+    w = np.concatenate([group(lo, span) for lo, span, _, _ in cases])
+    for (lo, span, _, _), g in zip(cases, w.reshape(-1, G)):
+        assert g.min() == np.float32(lo) and np.float32(g.max() - g.min()) / np.float32(15) == np.float32(span / 15)
+    _, s, b = oracle.quantize_f32(w, G, 4)
+    assert [int(v) for v in b] == [c[2] for c in cases]
+    assert [int(v) for v in s] == [c[3] for c in cases]
+
+
+@pytest.mark.parametrize("bits", [4, 2])
+def test_stored_format_quantiser_picks_the_nearest_stored_grid_point(bits):
+    """Each code selects, among the points c * S + B (c = 0 .. 2^bits - 1) of
+    the STORED bf16 scale S and bias B, the one nearest the weight, up to the
+    fp32 rounding of (w - B) / S: codes taken from the unrounded scale or
+    minimum miss it by up to a few hundredths of S."""
+    r = rng(23 + bits)
+    qmax = (1 << bits) - 1
+    w = np.concatenate([r.normal(size=64 * 60), r.normal(loc=-3.0, scale=0.2, size=64 * 20)]).astype(np.float32)
+    q, s, b = oracle.quantize_f32(w, 64, bits)
+    S = np.repeat(synth.bf16_to_f32(s).astype(np.float64), 64)
+    B = np.repeat(synth.bf16_to_f32(b).astype(np.float64), 64)
+    grid = np.arange(qmax + 1)[None, :] * S[:, None] + B[:, None]
+    best = np.abs(grid - w.astype(np.float64)[:, None]).min(axis=1)
+    got = np.abs(q.astype(np.float64) * S + B - w)
+    assert np.all(got <= best + 1e-5 * S)
+
+
+def test_stored_format_quantiser_stores_a_negative_zero_minimum_as_plus_zero():
+    """A group whose minimum is -0 stores bias +0 (bits 0), the reading the
+    oracle states; its codes are those of the +0 minimum."""
+    g = np.linspace(0.0, 1.5, 64).astype(np.float32)
+    g[0] = -0.0
+    q, s, b = oracle.quantize_f32(g, 64, 4)
+    g2 = g.copy()
+    g2[0] = 0.0
+    q2, s2, b2 = oracle.quantize_f32(g2, 64, 4)
+    assert int(b[0]) == 0 and int(b2[0]) == 0
+    assert np.array_equal(q, q2) and np.array_equal(s, s2)
 
 
 # ------------------------------------------------------------ byte counts ----
