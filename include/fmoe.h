@@ -270,8 +270,10 @@ int fmoe_combine_residual_rmsnorm(const float* d_y, const float* d_weights, cons
  * the normed input d_xn [T][H], writes h' to d_h and xn' to d_xn.  All steps
  * run on the device with no host round trip; the call is safe to capture in
  * a CUDA graph.  The intermediates stay in the workspace (see
- * fmoe_workspace_offset).  Errors: FMOE_ERR_INVALID_ARG, FMOE_ERR_UNSUPPORTED,
- * FMOE_ERR_CUDA. */
+ * fmoe_workspace_offset).  d_h and d_xn must not overlap (the same buffer
+ * for both would leave xn' where h' belongs): FMOE_ERR_INVALID_ARG when
+ * their T x H rows share a byte.  Errors: FMOE_ERR_INVALID_ARG,
+ * FMOE_ERR_UNSUPPORTED, FMOE_ERR_CUDA. */
 int fmoe_layer_forward(const fmoe_layer_weights* lw, float* d_h, float* d_xn, int T, void* d_ws,
                        size_t ws_bytes, cudaStream_t stream);
 
@@ -303,7 +305,8 @@ int fmoe_layer_forward_logits(const fmoe_layer_weights* lw, const float* d_logit
  * (cooperative launch, one CTA per SM, two tokens and up to 32 layers per
  * launch), which leave the last layer's intermediates in the workspace
  * (see fmoe_stack_forward_trace for every layer's).  If a persistent kernel
- * reports FMOE_STATUS_WAIT_TIMEOUT, re-initialise the workspace. */
+ * reports FMOE_STATUS_WAIT_TIMEOUT, re-initialise the workspace.  Errors:
+ * as fmoe_layer_forward (d_h and d_xn must not overlap). */
 int fmoe_stack_forward(const fmoe_layer_weights* layers, int n_layers, float* d_h, float* d_xn,
                        int T, void* d_ws, size_t ws_bytes, cudaStream_t stream);
 

@@ -162,7 +162,7 @@ extern "C" int fmoe_cache_layer_forward(fmoe_expert_cache* c, int layer, const f
       !aligned16(lw->w_router) || !aligned16(lw->w_shared_gate) || !aligned16(lw->norm_w))
     return FMOE_ERR_INVALID_ARG;
   if (!d_h || !d_xn || !d_ws || !aligned16(d_h) || !aligned16(d_xn) || !aligned16(d_ws) ||
-      (d_logits && !aligned16(d_logits)))
+      (d_logits && !aligned16(d_logits)) || !disjoint(d_h, d_xn, (size_t)T * d.hidden * 4))
     return FMOE_ERR_INVALID_ARG;
   const WsLayout w = ws_layout(d.hidden, d.inter, d.n_experts, d.top_k, T);
   if (ws_bytes < w.bytes) return FMOE_ERR_BUFFER_TOO_SMALL;

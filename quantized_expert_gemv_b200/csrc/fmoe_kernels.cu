@@ -669,6 +669,14 @@ static TraceLayout trace_layout(int H, int I, int E, int k, int T) {
 
 static inline bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
 
+// Two device ranges of `bytes` bytes each share no byte.  The layer and stack
+// calls read h and xn and write h' and xn' over them in place, so their token
+// rows must be apart (the same buffer for both would give xn' in place of h').
+static inline bool disjoint(const void* a, const void* b, size_t bytes) {
+  const uintptr_t x = reinterpret_cast<uintptr_t>(a), y = reinterpret_cast<uintptr_t>(b);
+  return x + bytes <= y || y + bytes <= x;
+}
+
 static bool desc_valid(const fmoe_layer_desc* d) {
   return d && d->hidden > 0 && d->inter > 0 && d->n_experts >= 1 && d->n_experts <= kMaxE &&
          d->top_k >= 1 && d->top_k <= kMaxK && d->top_k <= d->n_experts && d->eps >= 0.f;
@@ -1089,6 +1097,7 @@ static int layer_forward_impl(const fmoe_layer_weights* lw, const float* logits_
   const fmoe_layer_desc& d = lw->desc;
   if (T < 1 || !h || !xn || !ws || !aligned16(h) || !aligned16(xn) || !aligned16(ws))
     return FMOE_ERR_INVALID_ARG;
+  if (!disjoint(h, xn, (size_t)T * d.hidden * 4)) return FMOE_ERR_INVALID_ARG;
   if (logits_in && !aligned16(logits_in)) return FMOE_ERR_INVALID_ARG;
   const WsLayout w = ws_layout(d.hidden, d.inter, d.n_experts, d.top_k, T);
   if (ws_bytes < w.bytes) return FMOE_ERR_BUFFER_TOO_SMALL;
@@ -1312,7 +1321,9 @@ extern "C" int fmoe_set_fused(int enable) {
 static int stack_forward_impl(const fmoe_layer_weights* layers, int n_layers, float* d_h, float* d_xn, int T,
                               void* d_ws, size_t ws_bytes, unsigned char* trace, size_t trace_bytes,
                               cudaStream_t stream) {
-  if (!layers || n_layers < 1) return FMOE_ERR_INVALID_ARG;
+  if (!layers || n_layers < 1 || !desc_valid(&layers[0].desc)) return FMOE_ERR_INVALID_ARG;
+  if (T >= 1 && d_h && d_xn && !disjoint(d_h, d_xn, (size_t)T * layers[0].desc.hidden * 4))
+    return FMOE_ERR_INVALID_ARG;
   if (trace) {
     for (int l = 0; l < n_layers; ++l) {
       const int rc = weights_check(&layers[l]);
@@ -1454,6 +1465,7 @@ extern "C" int fmoe_layer_forward_noalloc(const fmoe_layer_weights* lw, float* d
                                           cudaStream_t stream) {
   if (!lw || !desc_valid(&lw->desc) || T < 1) return FMOE_ERR_INVALID_ARG;
   const fmoe_layer_desc& d = lw->desc;
+  if (!d_h || !d_xn || !disjoint(d_h, d_xn, (size_t)T * d.hidden * 4)) return FMOE_ERR_INVALID_ARG;
   if (ws_layout(d.hidden, d.inter, d.n_experts, d.top_k, T).bytes > kStaticScratchBytes)
     return FMOE_ERR_BUFFER_TOO_SMALL;
   void* ws = nullptr;

@@ -150,6 +150,9 @@ def test_packer_rejects_bad_input(fm):
     assert e.value.status == fm.FMOE_ERR_UNSUPPORTED
 
 
+H_, XN_ = 1 << 20, (1 << 20) + 1024  # distinct device addresses of one 256-float token row each
+
+
 def test_host_validation_before_launch(fm):
     """Bad arguments are refused on the host (no CUDA call is made, so this
     runs without a GPU)."""
@@ -160,9 +163,19 @@ def test_host_validation_before_launch(fm):
     # null activation pointers
     assert L.fmoe_layer_forward(ctypes.byref(w), None, None, 1, 16, 1 << 30, None) == fm.FMOE_ERR_INVALID_ARG
     # misaligned workspace
-    assert L.fmoe_layer_forward(ctypes.byref(w), 16, 16, 1, 17, 1 << 30, None) == fm.FMOE_ERR_INVALID_ARG
+    assert L.fmoe_layer_forward(ctypes.byref(w), H_, XN_, 1, 17, 1 << 30, None) == fm.FMOE_ERR_INVALID_ARG
     # workspace too small
-    assert L.fmoe_layer_forward(ctypes.byref(w), 16, 16, 1, 16, 64, None) == fm.FMOE_ERR_BUFFER_TOO_SMALL
+    assert L.fmoe_layer_forward(ctypes.byref(w), H_, XN_, 1, 16, 64, None) == fm.FMOE_ERR_BUFFER_TOO_SMALL
+    # h and xn overlapping (one token of H = 256 floats is 1 KiB): refused,
+    # rows that only touch are not
+    for xn in (H_, H_ + 1008, H_ - 1008):
+        assert L.fmoe_layer_forward(ctypes.byref(w), H_, xn, 1, 16, 64, None) == fm.FMOE_ERR_INVALID_ARG
+        assert L.fmoe_layer_forward_logits(ctypes.byref(w), 16, H_, xn, 1, 16, 64, None) == fm.FMOE_ERR_INVALID_ARG
+        assert L.fmoe_stack_forward(ctypes.byref(w), 1, H_, xn, 1, 16, 64, None) == fm.FMOE_ERR_INVALID_ARG
+        assert L.fmoe_layer_forward_noalloc(ctypes.byref(w), H_, xn, 1, None) == fm.FMOE_ERR_INVALID_ARG
+    assert L.fmoe_layer_forward(ctypes.byref(w), H_, XN_, 2, 16, 64, None) == fm.FMOE_ERR_INVALID_ARG  # 2 tokens
+    for xn in (H_ + 1024, H_ - 1024):
+        assert L.fmoe_layer_forward(ctypes.byref(w), H_, xn, 1, 16, 64, None) == fm.FMOE_ERR_BUFFER_TOO_SMALL
     # k > 8, k > E, E > 1024, T < 1
     for bad in (dict(top_k=9, n_experts=16), dict(top_k=5, n_experts=4), dict(n_experts=2048)):
         dd = fm.LayerDesc(hidden=256, inter=128, **{**dict(n_experts=16, top_k=4), **bad})
@@ -265,11 +278,12 @@ def test_trace_layout_and_validation(fm):
     dd = fm.LayerDesc(hidden=256, inter=128, n_experts=16, top_k=4)
     w = fm.fmoe_layer_weights(dd.c(), 16, 16, 16, 16, 16)
     w2 = (fm.fmoe_layer_weights * 2)(w, w)
-    assert L.fmoe_stack_forward_trace(w2, 2, 16, 16, 1, 16, 1 << 30, None, 1 << 30, None) == fm.FMOE_ERR_INVALID_ARG
-    assert L.fmoe_stack_forward_trace(w2, 2, 16, 16, 1, 16, 1 << 30, 24, 1 << 30, None) == fm.FMOE_ERR_INVALID_ARG
+    assert L.fmoe_stack_forward_trace(w2, 2, H_, XN_, 1, 16, 1 << 30, None, 1 << 30, None) == fm.FMOE_ERR_INVALID_ARG
+    assert L.fmoe_stack_forward_trace(w2, 2, H_, XN_, 1, 16, 1 << 30, 24, 1 << 30, None) == fm.FMOE_ERR_INVALID_ARG
     need = fm.fmoe_trace_bytes(dd, 1, 2)
-    assert L.fmoe_stack_forward_trace(w2, 2, 16, 16, 1, 16, 1 << 30, 16, need - 1, None) == \
+    assert L.fmoe_stack_forward_trace(w2, 2, H_, XN_, 1, 16, 1 << 30, 16, need - 1, None) == \
         fm.FMOE_ERR_BUFFER_TOO_SMALL
+    assert L.fmoe_stack_forward_trace(w2, 2, H_, H_, 1, 16, 1 << 30, 16, need, None) == fm.FMOE_ERR_INVALID_ARG
 
 
 def test_header_and_c_example_compile_as_c():
