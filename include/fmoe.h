@@ -260,8 +260,9 @@ int fmoe_expert_forward(const fmoe_layer_weights* lw, const float* d_xn, int T,
 /* Combine + residual + shared gate, then RMSNorm, for T tokens:
  *   h_out[t] = h[t] + sum_j weights[t][j] y[t][j] + gamma[t] y[t][k]
  *   xn_out[t] = h_out[t] * (mean(h_out[t]^2) + eps)^(-1/2) * norm_w
- * All device fp32; y [T][k+1][H]; h_out may alias h and xn_out may alias
- * neither y nor h.  Errors: FMOE_ERR_INVALID_ARG, FMOE_ERR_CUDA. */
+ * All device fp32; y [T][k+1][H].  h_out may be h itself (in place);
+ * otherwise neither output may share a byte with y, h or the other output
+ * (FMOE_ERR_INVALID_ARG).  Errors: FMOE_ERR_INVALID_ARG, FMOE_ERR_CUDA. */
 int fmoe_combine_residual_rmsnorm(const float* d_y, const float* d_weights, const float* d_gamma,
                                   const float* d_h, const float* d_norm_w, float eps, int T, int k,
                                   int H, float* d_h_out, float* d_xn_out, cudaStream_t stream);

@@ -669,13 +669,15 @@ static TraceLayout trace_layout(int H, int I, int E, int k, int T) {
 
 static inline bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
 
-// Two device ranges of `bytes` bytes each share no byte.  The layer and stack
-// calls read h and xn and write h' and xn' over them in place, so their token
-// rows must be apart (the same buffer for both would give xn' in place of h').
-static inline bool disjoint(const void* a, const void* b, size_t bytes) {
+// The device ranges [a, a + na) and [b, b + nb) share no byte.  The layer and
+// stack calls read h and xn and write h' and xn' over them in place, so their
+// token rows must be apart (the same buffer for both would give xn' in place
+// of h').
+static inline bool disjoint(const void* a, size_t na, const void* b, size_t nb) {
   const uintptr_t x = reinterpret_cast<uintptr_t>(a), y = reinterpret_cast<uintptr_t>(b);
-  return x + bytes <= y || y + bytes <= x;
+  return x + na <= y || y + nb <= x;
 }
+static inline bool disjoint(const void* a, const void* b, size_t bytes) { return disjoint(a, bytes, b, bytes); }
 
 static bool desc_valid(const fmoe_layer_desc* d) {
   return d && d->hidden > 0 && d->inter > 0 && d->n_experts >= 1 && d->n_experts <= kMaxE &&
@@ -1230,7 +1232,12 @@ extern "C" int fmoe_combine_residual_rmsnorm(const float* d_y, const float* d_we
   const void* ps[] = {d_y, d_weights, d_gamma, d_h, d_norm_w, d_h_out, d_xn_out};
   for (const void* p : ps)
     if (!p || !aligned16(p)) return FMOE_ERR_INVALID_ARG;
-  if (d_xn_out == d_h || d_xn_out == d_y) return FMOE_ERR_INVALID_ARG;
+  // h_out may be h itself (in place); otherwise the outputs share no byte
+  // with each other, with h or with y
+  const size_t rows = (size_t)T * H * 4, ys = (size_t)T * (k + 1) * H * 4;
+  if (!disjoint(d_xn_out, d_h, rows) || !disjoint(d_xn_out, d_h_out, rows) || !disjoint(d_xn_out, rows, d_y, ys) ||
+      !disjoint(d_h_out, rows, d_y, ys) || (d_h_out != d_h && !disjoint(d_h_out, d_h, rows)))
+    return FMOE_ERR_INVALID_ARG;
   return launch_combine(d_y, d_weights, d_gamma, d_h, d_norm_w, eps, T, k, H, d_h_out, d_xn_out, stream);
 }
 

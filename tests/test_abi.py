@@ -192,9 +192,16 @@ def test_host_validation_before_launch(fm):
     # route: k > 8 unsupported, null outputs invalid
     assert L.fmoe_route_topk(16, 16, 1, 256, 16, 9, 0, 16, 16, 16, 16, 1 << 20, None) == fm.FMOE_ERR_UNSUPPORTED
     assert L.fmoe_route_topk(16, 16, 1, 256, 16, 4, 0, None, 16, 16, 16, 1 << 20, None) == fm.FMOE_ERR_INVALID_ARG
-    # combine: output aliasing its inputs
-    assert L.fmoe_combine_residual_rmsnorm(16, 16, 16, 32, 16, ctypes.c_float(1e-6), 1, 4, 256, 32, 32,
-                                           None) == fm.FMOE_ERR_INVALID_ARG
+    # combine: an output overlapping an input or the other output (one
+    # token of H = 256: rows of 1 KiB, y of 5 KiB); h_out = h is in place
+    Y = 1 << 24
+    comb = lambda y, h, ho, xo: L.fmoe_combine_residual_rmsnorm(y, 16, 16, h, 16, ctypes.c_float(1e-6), 1, 4, 256,
+                                                                ho, xo, None)
+    assert comb(Y, 32, 32, 32) == fm.FMOE_ERR_INVALID_ARG            # xn_out = h
+    assert comb(Y, H_, XN_, XN_) == fm.FMOE_ERR_INVALID_ARG          # xn_out = h_out
+    assert comb(Y, H_, H_, Y + 4096) == fm.FMOE_ERR_INVALID_ARG      # xn_out inside y
+    assert comb(Y, H_, Y - 512, XN_) == fm.FMOE_ERR_INVALID_ARG      # h_out runs into y
+    assert comb(Y, H_, H_ + 512, XN_ + 1024) == fm.FMOE_ERR_INVALID_ARG  # h_out half over h
     assert L.fmoe_stack_forward(None, 1, 16, 16, 1, 16, 1 << 30, None) == fm.FMOE_ERR_INVALID_ARG
     assert fm.fmoe_error_string(fm.FMOE_ERR_UNSUPPORTED) == "unsupported shape or bit width"
 
