@@ -50,7 +50,7 @@ extern "C" {
 /* ---------------------------------------------------------------- status -- */
 #define FMOE_OK 0
 #define FMOE_ERR_INVALID_ARG 1   /* null pointer, bad size, misaligned pointer */
-#define FMOE_ERR_UNSUPPORTED 2   /* a shape or bit width this build does not run */
+#define FMOE_ERR_UNSUPPORTED 2   /* a shape or bit width the library does not run */
 #define FMOE_ERR_CUDA 3          /* a CUDA runtime call failed */
 #define FMOE_ERR_DEVICE_STATUS 4 /* the device status word is non-zero */
 #define FMOE_ERR_BUFFER_TOO_SMALL 5
