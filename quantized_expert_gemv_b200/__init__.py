@@ -119,16 +119,60 @@ def _check(rc: int, where: str) -> None:
 
 
 def _ptr(x):
-    """Device or host pointer of a torch tensor / numpy array (None -> NULL)."""
+    """Device or host pointer of a torch tensor / numpy array (None -> NULL;
+    an int is taken as a raw address)."""
     if x is None:
         return None
     if isinstance(x, np.ndarray):
-        assert x.flags["C_CONTIGUOUS"], "array must be contiguous"
+        if not x.flags["C_CONTIGUOUS"]:
+            raise ValueError("array must be contiguous")
         return ctypes.c_void_p(x.ctypes.data)
     if isinstance(x, int):
         return ctypes.c_void_p(x)
-    assert x.is_contiguous(), "tensor must be contiguous"
+    if not x.is_contiguous():
+        raise ValueError("tensor must be contiguous")
     return ctypes.c_void_p(x.data_ptr())
+
+
+_DT = {"f32": (np.float32, "float32"), "i32": (np.int32, "int32")}
+
+
+def _need(x, name: str, n: int, dt: str | None = "f32", cuda: bool = True, exact: bool = True) -> None:
+    """Refuses (ValueError) a buffer that a C call would read or write out of
+    its bounds, as the wrong element type or in the wrong memory, before the
+    call: x must be contiguous, hold exactly (exact) or at least n elements
+    of type dt (dt None: n counts bytes, any type), and live on a CUDA device
+    (cuda) or in host memory.  Raw int addresses are the caller's own."""
+    if isinstance(x, int):
+        return
+    if x is None:
+        raise ValueError(f"{name}: missing")
+    if isinstance(x, np.ndarray):
+        where, contiguous, size, nbytes = "cpu", x.flags["C_CONTIGUOUS"], x.size, x.nbytes
+        dt_ok = dt is None or x.dtype == np.dtype(_DT[dt][0])
+    else:
+        where, contiguous = x.device.type, x.is_contiguous()
+        size, nbytes = x.numel(), x.numel() * x.element_size()
+        dt_ok = dt is None or str(x.dtype) == "torch." + _DT[dt][1]
+    if where != ("cuda" if cuda else "cpu"):
+        raise ValueError(f"{name}: must be in {'CUDA device' if cuda else 'host'} memory")
+    if not contiguous:
+        raise ValueError(f"{name}: must be contiguous")
+    if not dt_ok:
+        raise ValueError(f"{name}: must hold {_DT[dt][1]} elements, not {x.dtype}")
+    have = size if dt is not None else nbytes
+    if (have != n) if exact else (have < n):
+        unit = "elements" if dt is not None else "bytes"
+        raise ValueError(f"{name}: holds {have} {unit}, the call needs {'' if exact else 'at least '}{n}")
+
+
+def _tokens(lw_or_desc, h, xn, name_h: str = "h", name_xn: str = "xn") -> int:
+    """T of the token buffers h, xn [T][hidden] (fp32, device)."""
+    H = lw_or_desc.hidden
+    T = int(h.shape[0]) if len(getattr(h, "shape", ())) >= 1 else 0
+    _need(h, name_h, T * H)
+    _need(xn, name_xn, T * H)
+    return T
 
 
 def _stream(stream):
@@ -229,6 +273,12 @@ class LayerWeights:
 
     def c(self) -> fmoe_layer_weights:
         if self._c is None:
+            d = self.desc
+            _need(self.experts, "experts", d.n_experts * d.record_bytes(), None, exact=False)
+            _need(self.shared, "shared", d.record_bytes(shared=True), None, exact=False)
+            _need(self.w_router, "w_router", d.n_experts * d.hidden)
+            _need(self.w_shared_gate, "w_shared_gate", d.hidden)
+            _need(self.norm_w, "norm_w", d.hidden)
             self._c = fmoe_layer_weights(self.desc.c(), self.experts.data_ptr(), self.shared.data_ptr(),
                                          self.w_router.data_ptr(), self.w_shared_gate.data_ptr(),
                                          self.norm_w.data_ptr())
@@ -272,6 +322,13 @@ def workspace_view(ws, desc: LayerDesc, T: int, which: int):
 def fmoe_route_topk(xn, w_router, k: int, logits, ids, weights, ws=None, flags: int = 0, stream=None) -> None:
     T, E = logits.shape
     H = w_router.shape[1] if w_router is not None else 64
+    _need(logits, "logits", T * E)
+    _need(ids, "ids", T * k, "i32")
+    _need(weights, "weights", T * k)
+    if not flags & FMOE_LOGITS_GIVEN:
+        _need(w_router, "w_router", E * H)
+        _need(xn, "xn", T * H)
+        _need(ws, "ws", 0, None, exact=False)
     nbytes = ws.numel() * ws.element_size() if ws is not None else 0
     rc = _lib.fmoe_route_topk(_ptr(xn), _ptr(w_router), T, H, E, k, flags, _ptr(logits), _ptr(ids),
                               _ptr(weights), _ptr(ws), nbytes, _stream(stream))
@@ -280,6 +337,12 @@ def fmoe_route_topk(xn, w_router, k: int, logits, ids, weights, ws=None, flags: 
 
 def fmoe_expert_forward(lw: LayerWeights, xn, ids, y, gamma, ws, stream=None) -> None:
     T = xn.shape[0]
+    k, H = lw.desc.top_k, lw.desc.hidden
+    _need(xn, "xn", T * H)
+    _need(ids, "ids", T * k, "i32")
+    _need(y, "y", T * (k + 1) * H)
+    _need(gamma, "gamma", T)
+    _need(ws, "ws", 0, None, exact=False)
     c = lw.c()
     rc = _lib.fmoe_expert_forward(ctypes.byref(c), _ptr(xn), T, _ptr(ids), lw.desc.top_k, _ptr(y), _ptr(gamma),
                                   _ptr(ws), ws.numel() * ws.element_size(), _stream(stream))
@@ -288,14 +351,22 @@ def fmoe_expert_forward(lw: LayerWeights, xn, ids, y, gamma, ws, stream=None) ->
 
 def fmoe_combine_residual_rmsnorm(y, weights, gamma, h, norm_w, eps: float, h_out, xn_out, stream=None) -> None:
     T, k1, H = y.shape
+    _need(y, "y", T * k1 * H)
+    _need(weights, "weights", T * (k1 - 1))
+    _need(gamma, "gamma", T)
+    _need(norm_w, "norm_w", H)
+    for name, t in (("h", h), ("h_out", h_out), ("xn_out", xn_out)):
+        _need(t, name, T * H)
     rc = _lib.fmoe_combine_residual_rmsnorm(_ptr(y), _ptr(weights), _ptr(gamma), _ptr(h), _ptr(norm_w), eps, T,
                                             k1 - 1, H, _ptr(h_out), _ptr(xn_out), _stream(stream))
     _check(rc, "fmoe_combine_residual_rmsnorm")
 
 
 def fmoe_layer_forward(lw: LayerWeights, h, xn, ws, stream=None) -> None:
+    T = _tokens(lw.desc, h, xn)
+    _need(ws, "ws", 0, None, exact=False)
     c = lw.c()
-    rc = _lib.fmoe_layer_forward(ctypes.byref(c), _ptr(h), _ptr(xn), h.shape[0], _ptr(ws),
+    rc = _lib.fmoe_layer_forward(ctypes.byref(c), _ptr(h), _ptr(xn), T, _ptr(ws),
                                  ws.numel() * ws.element_size(), _stream(stream))
     _check(rc, "fmoe_layer_forward")
 
@@ -304,16 +375,24 @@ def fmoe_layer_forward_host(lw: LayerWeights, hx_in, hx_out, d_hx, ws, stream=No
     """fmoe_layer_forward on host token state: hx_in / hx_out are (pinned) host
     tensors [2, T, H] (h rows, then xn rows), d_hx a device tensor of the same
     shape; one copy in, the layer, one copy out, asynchronous on `stream`."""
+    T = int(d_hx.shape[1])
+    n = 2 * T * lw.desc.hidden
+    _need(d_hx, "d_hx", n)
+    _need(hx_in, "hx_in", n, cuda=False)
+    _need(hx_out, "hx_out", n, cuda=False)
+    _need(ws, "ws", 0, None, exact=False)
     c = lw.c()
-    T = d_hx.shape[1]
     rc = _lib.fmoe_layer_forward_host(ctypes.byref(c), _ptr(hx_in), _ptr(hx_out), _ptr(d_hx), T, _ptr(ws),
                                       ws.numel() * ws.element_size(), _stream(stream))
     _check(rc, "fmoe_layer_forward_host")
 
 
 def fmoe_layer_forward_logits(lw: LayerWeights, logits, h, xn, ws, stream=None) -> None:
+    T = _tokens(lw.desc, h, xn)
+    _need(logits, "logits", T * lw.desc.n_experts)
+    _need(ws, "ws", 0, None, exact=False)
     c = lw.c()
-    rc = _lib.fmoe_layer_forward_logits(ctypes.byref(c), _ptr(logits), _ptr(h), _ptr(xn), h.shape[0], _ptr(ws),
+    rc = _lib.fmoe_layer_forward_logits(ctypes.byref(c), _ptr(logits), _ptr(h), _ptr(xn), T, _ptr(ws),
                                         ws.numel() * ws.element_size(), _stream(stream))
     _check(rc, "fmoe_layer_forward_logits")
 
@@ -322,8 +401,14 @@ def fmoe_stack_forward_host(layers, hx_in, hx_out, d_hx, ws, stream=None) -> Non
     """fmoe_stack_forward on host token state: hx_in / hx_out (pinned) host
     tensors [2, T, H], d_hx a device tensor of the same shape; one copy in,
     the layers, one copy out, asynchronous on `stream`."""
+    T = int(d_hx.shape[1])
+    n = 2 * T * layers[0].desc.hidden
+    _need(d_hx, "d_hx", n)
+    _need(hx_in, "hx_in", n, cuda=False)
+    _need(hx_out, "hx_out", n, cuda=False)
+    _need(ws, "ws", 0, None, exact=False)
     arr = (fmoe_layer_weights * len(layers))(*[lw.c() for lw in layers])
-    rc = _lib.fmoe_stack_forward_host(arr, len(layers), _ptr(hx_in), _ptr(hx_out), _ptr(d_hx), d_hx.shape[1],
+    rc = _lib.fmoe_stack_forward_host(arr, len(layers), _ptr(hx_in), _ptr(hx_out), _ptr(d_hx), T,
                                       _ptr(ws), ws.numel() * ws.element_size(), _stream(stream))
     _check(rc, "fmoe_stack_forward_host")
 
@@ -331,13 +416,17 @@ def fmoe_stack_forward_host(layers, hx_in, hx_out, d_hx, ws, stream=None) -> Non
 def fmoe_stack_forward(layers, h, xn, ws, stream=None, trace=None) -> None:
     """The layer stack in place on h / xn; with `trace` (from alloc_trace),
     fmoe_stack_forward_trace: every layer's input, intermediates and output."""
+    T = _tokens(layers[0].desc, h, xn)
+    _need(ws, "ws", 0, None, exact=False)
+    if trace is not None:
+        _need(trace, "trace", 0, None, exact=False)
     arr = (fmoe_layer_weights * len(layers))(*[lw.c() for lw in layers])
     if trace is None:
-        rc = _lib.fmoe_stack_forward(arr, len(layers), _ptr(h), _ptr(xn), h.shape[0], _ptr(ws),
+        rc = _lib.fmoe_stack_forward(arr, len(layers), _ptr(h), _ptr(xn), T, _ptr(ws),
                                      ws.numel() * ws.element_size(), _stream(stream))
         _check(rc, "fmoe_stack_forward")
         return
-    rc = _lib.fmoe_stack_forward_trace(arr, len(layers), _ptr(h), _ptr(xn), h.shape[0], _ptr(ws),
+    rc = _lib.fmoe_stack_forward_trace(arr, len(layers), _ptr(h), _ptr(xn), T, _ptr(ws),
                                        ws.numel() * ws.element_size(), _ptr(trace),
                                        trace.numel() * trace.element_size(), _stream(stream))
     _check(rc, "fmoe_stack_forward_trace")
@@ -372,8 +461,9 @@ def trace_view(trace, desc: LayerDesc, T: int, layer: int, which: int):
 def fmoe_layer_forward_noalloc(lw: LayerWeights, h, xn, stream=None) -> None:
     """fmoe_layer_forward with the library's fixed per-device scratch instead of a
     caller workspace (nothing is allocated; calls on one device must not overlap)."""
+    T = _tokens(lw.desc, h, xn)
     c = lw.c()
-    rc = _lib.fmoe_layer_forward_noalloc(ctypes.byref(c), _ptr(h), _ptr(xn), h.shape[0], _stream(stream))
+    rc = _lib.fmoe_layer_forward_noalloc(ctypes.byref(c), _ptr(h), _ptr(xn), T, _stream(stream))
     _check(rc, "fmoe_layer_forward_noalloc")
 
 
@@ -437,11 +527,29 @@ class ExpertCache:
         self._h = h
 
     def forward(self, layer: int, lw: LayerWeights, h, xn, ws, logits=None, stream=None) -> None:
-        c = lw.c()
+        T = _tokens(lw.desc, h, xn)
+        _need(ws, "ws", 0, None, exact=False)
+        if logits is not None:
+            _need(logits, "logits", T * lw.desc.n_experts)
+        c = self._weights(lw)
         rc = _lib.fmoe_cache_layer_forward(self._h, layer, ctypes.byref(c), _ptr(logits) if logits is not None else None,
-                                           _ptr(h), _ptr(xn), h.shape[0], _ptr(ws), ws.numel() * ws.element_size(),
+                                           _ptr(h), _ptr(xn), T, _ptr(ws), ws.numel() * ws.element_size(),
                                            _stream(stream))
         _check(rc, "fmoe_cache_layer_forward")
+
+    @staticmethod
+    def _weights(lw: LayerWeights) -> fmoe_layer_weights:
+        """The C descriptor of lw for a cached layer: its routed records come
+        from the cache, so lw.experts may be None (it is not read); the other
+        buffers are checked as for a resident layer."""
+        d = lw.desc
+        _need(lw.shared, "shared", d.record_bytes(shared=True), None, exact=False)
+        _need(lw.w_router, "w_router", d.n_experts * d.hidden)
+        _need(lw.w_shared_gate, "w_shared_gate", d.hidden)
+        _need(lw.norm_w, "norm_w", d.hidden)
+        return fmoe_layer_weights(d.c(), lw.experts.data_ptr() if lw.experts is not None else None,
+                                  lw.shared.data_ptr(), lw.w_router.data_ptr(), lw.w_shared_gate.data_ptr(),
+                                  lw.norm_w.data_ptr())
 
     def stats(self):
         hits, misses, nbytes = ctypes.c_uint64(), ctypes.c_uint64(), ctypes.c_uint64()

@@ -326,3 +326,66 @@ def test_timeline_points_match_the_kernel():
         used.update(range(base, base + 5) if "+ p" in expr else [base])
     assert used == set(timeline.POINTS), sorted(used ^ set(timeline.POINTS))
     assert max(used) < timeline.N_POINTS
+
+
+def test_binding_refuses_bad_buffers_before_the_call(fm):
+    """The Python binding checks each buffer a call reads or writes (memory
+    kind, contiguity, element type, size) and raises ValueError before the
+    library is called: a token buffer shorter than T x hidden, or a weight
+    tensor shorter than the records the descriptor names, would otherwise be
+    read or written past its end on the device.  Runs without a GPU."""
+    import torch
+    need = fm._need
+    # host buffers: pass when right, refused for each kind of mismatch
+    need(torch.zeros(4, 256), "h", 4 * 256, cuda=False)
+    need(np.zeros((4, 256), np.float32), "h", 4 * 256, cuda=False)
+    need(torch.zeros(3, dtype=torch.int32), "ids", 3, "i32", cuda=False)
+    need(torch.zeros(100, dtype=torch.uint8), "ws", 64, None, cuda=False, exact=False)
+    bad = [
+        (torch.zeros(4, 255), "holds 1020 elements, the call needs 1024"),
+        (torch.zeros(4, 257), "holds 1028 elements, the call needs 1024"),
+        (torch.zeros(4, 256, dtype=torch.float64), "must hold float32"),
+        (torch.zeros(4, 256, dtype=torch.bfloat16), "must hold float32"),
+        (torch.zeros(256, 4).t(), "must be contiguous"),
+        (np.zeros((4, 256), np.float64), "must hold float32"),
+        (np.zeros((256, 4), np.float32).T, "must be contiguous"),
+        (None, "missing"),
+    ]
+    for x, msg in bad:
+        with pytest.raises(ValueError, match=msg):
+            need(x, "h", 4 * 256, cuda=False)
+    with pytest.raises(ValueError, match="at least 64"):
+        need(torch.zeros(63, dtype=torch.uint8), "ws", 64, None, cuda=False, exact=False)
+    with pytest.raises(ValueError, match="host memory"):
+        need(torch.zeros(4, 256, device="meta"), "hx_in", 4 * 256, cuda=False)
+    need(1 << 20, "h", 4 * 256)  # a raw address is the caller's own
+    # device buffers given as host tensors: refused before the library is called
+    d = fm.LayerDesc(hidden=256, inter=128, n_experts=16, top_k=4)
+    H, E, k = d.hidden, d.n_experts, d.top_k
+    lw = fm.LayerWeights(d, torch.zeros(E * d.record_bytes(), dtype=torch.uint8),
+                         torch.zeros(d.record_bytes(shared=True), dtype=torch.uint8),
+                         torch.zeros(E, H), torch.zeros(H), torch.ones(H))
+    h, xn, ws = torch.zeros(2, H), torch.zeros(2, H), torch.zeros(1 << 20, dtype=torch.uint8)
+    with pytest.raises(ValueError, match="h: must be in CUDA device memory"):
+        fm.fmoe_layer_forward(lw, h, xn, ws)
+    with pytest.raises(ValueError, match="h: must be in CUDA device memory"):
+        fm.fmoe_stack_forward([lw, lw], h, xn, ws)
+    with pytest.raises(ValueError, match="h: must be in CUDA device memory"):
+        fm.fmoe_layer_forward_noalloc(lw, h, xn)
+    with pytest.raises(ValueError, match="d_hx: must be in CUDA device memory"):
+        fm.fmoe_layer_forward_host(lw, torch.zeros(2, 2, H), torch.zeros(2, 2, H), torch.zeros(2, 2, H), ws)
+    with pytest.raises(ValueError, match="experts: must be in CUDA device memory"):
+        lw.c()
+    with pytest.raises(ValueError, match="y: must be in CUDA device memory"):
+        fm.fmoe_combine_residual_rmsnorm(torch.zeros(2, k + 1, H), torch.zeros(2, k), torch.zeros(2), h,
+                                         torch.ones(H), 1e-6, h, xn)
+    with pytest.raises(ValueError, match="logits: must be in CUDA device memory"):
+        fm.fmoe_route_topk(None, None, k, torch.zeros(2, E), torch.zeros(2, k, dtype=torch.int32), torch.zeros(2, k),
+                           flags=fm.FMOE_LOGITS_GIVEN)
+    with pytest.raises(ValueError, match="xn: must be in CUDA device memory"):
+        fm.fmoe_expert_forward(lw, xn, torch.zeros(2, k, dtype=torch.int32), torch.zeros(2, k + 1, H),
+                               torch.zeros(2), ws)
+    # a cached layer's descriptor does not need device experts, only the rest
+    lw_cached = fm.LayerWeights(d, None, lw.shared, lw.w_router, lw.w_shared_gate, lw.norm_w)
+    with pytest.raises(ValueError, match="shared: must be in CUDA device memory"):
+        fm.ExpertCache._weights(lw_cached)
