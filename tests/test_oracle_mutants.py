@@ -107,7 +107,19 @@ MUTANTS = [
      "int slot = (t < k) ? ids[t] : 0;"),
     ("layer: shared gate's error without the sigmoid derivative",
      "double S_gamma = gamma * (1.0 - gamma) * S_z;", "double S_gamma = gamma * S_z;"),
+    ("topk: an expert selected twice", "if (ids[u] == e) taken = 1;", "if (ids[u] == e) taken = 0;"),
+    ("topk: NaN logit given a weight", "p[t] = isnan(l) ? 0.0 : exp(l - m);", "p[t] = exp(l - m);"),
+    ("gemv_f32: error scale without absolute values", "      mag += fabs(t);", "      mag += t;"),
+    ("S_y: own terms dropped", "    S_y[r] += prop;", "    S_y[r] = prop;"),
+    ("S_h: weighted terms without absolute values", "mag += fabs(p[t] * yt);", "mag += p[t] * yt;"),
+    ("S_h: the inputs' slack dropped", "S_h[i] = mag + 1e-2;", "S_h[i] = mag;"),
+    ("rmsnorm: normalises the residual input instead of h'", "xn_out[i] = h_out[i] * r * (double)w[i];",
+     "xn_out[i] = h[i] * r * (double)w[i];"),
     # quantisers (the offline conversion)
+    ("quantize: scale over 2^bits steps", "double sc = (hi - lo) / qmax;", "double sc = (hi - lo) / (qmax + 1);"),
+    ("quantize_f32: scale and bias stored in each other's place",
+     "    s[g] = oracle_f32_to_bf16(sc);\n    b[g] = oracle_f32_to_bf16(lo);",
+     "    s[g] = oracle_f32_to_bf16(lo);\n    b[g] = oracle_f32_to_bf16(sc);"),
     ("quantize: codes truncated instead of rounded", "double c = sc > 0.0 ? nearbyint((w[g0 + j] - lo) / sc) : 0.0;",
      "double c = sc > 0.0 ? floor((w[g0 + j] - lo) / sc) : 0.0;"),
     ("quantize_f32: bf16 ties rounded away from zero", "u += 0x7FFFu + ((u >> 16) & 1u);", "u += 0x8000u;"),

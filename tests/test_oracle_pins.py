@@ -215,6 +215,18 @@ def test_topk_nan_is_never_selected_and_is_reported():
     assert nan and ids.tolist() == [1, 2, 3, 4]
 
 
+def test_topk_with_fewer_numbers_than_k_gives_nan_weight_zero():
+    """NaN ranks below every number (the reading: NaN as -inf): with three
+    numbers among six logits, top-4 takes the three numbers in order and
+    then the lowest-index NaN, whose weight is exp(-inf) = 0; the numbers'
+    weights are the softmax of the three."""
+    lg = np.array([np.nan, 1.0, np.nan, 0.5, np.nan, 2.0])
+    ids, p, nan = oracle.topk_softmax(lg, 4)
+    assert nan and ids.tolist() == [5, 1, 3, 0]
+    e = np.exp(np.array([2.0, 1.0, 0.5]) - 2.0)
+    assert np.allclose(p[:3], e / e.sum(), rtol=1e-15) and p[3] == 0.0
+
+
 # ------------------------------------------------------- SwiGLU / sigmoid ----
 
 def test_sigmoid_and_swiglu_closed_forms():
