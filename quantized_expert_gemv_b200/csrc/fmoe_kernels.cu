@@ -27,6 +27,7 @@
 // "2. FMA-optimised dequantisation kernels" and "3. Hand-tuned Metal compute
 // shaders" (dequantising matrix-vector products, fused SwiGLU, MoE combine +
 // residual + sigmoid gating, two-pass RMSNorm feeding the next layer).
+#include <atomic>
 #include <cstdint>
 #include <cstring>
 #include <mutex>
@@ -735,13 +736,18 @@ static int launch_topk(const float* part, const float* logits_in, int T, int E, 
   return cuda_rc(cudaGetLastError());
 }
 
-static int g_tc_enabled = 1;  // tensor-core products for groups of >= kTcMinTokens tokens
+// Tensor-core products for groups of >= kTcMinTokens tokens (a process-wide
+// switch; calls from several host threads read it while one may set it).
+static std::atomic<int> g_tc_enabled{1};
 
-// Dynamic shared memory above the default 48 KB for a kernel, set once per device.
+// Dynamic shared memory above the default 48 KB for a kernel, set once per
+// device (under a lock: calls may come from several host threads).
 static bool smem_optin(const void* fn, size_t bytes, int slot) {
   static size_t done[64][32];
+  static std::mutex mu;
   int dev = 0;
   if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return false;
+  std::lock_guard<std::mutex> lock(mu);
   if (done[dev][slot] >= bytes) return true;
   if (cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)bytes) != cudaSuccess) return false;
   done[dev][slot] = bytes;
@@ -897,7 +903,7 @@ static int launch_combine(const float* y, const float* weights, const float* gam
 }
 
 // ------------------------------------------------- persistent-kernel path --
-static int g_fused_enabled = 1;
+static std::atomic<int> g_fused_enabled{1};  // process-wide, as g_tc_enabled
 // Token counts up to which T > 1 runs through the persistent kernel, two
 // tokens per launch (measured: a layer of T = 2 / 4 / 8 tokens takes
 // 77 / 138 / 197 us on the grouped path against 31.9 / 60.3 / 124.7 us per
@@ -918,13 +924,16 @@ struct FusedConfigs {
 static bool same_desc(const fmoe_layer_desc& a, const fmoe_layer_desc& b);
 
 // Per-device cache of the last configuration (shape checks and the
-// attribute / occupancy queries run once per shape, not per call).
+// attribute / occupancy queries run once per shape, not per call).  Host
+// threads that run layers of different shapes on one device share an entry,
+// so it is read and replaced under a lock.
 struct FusedCacheEntry {
   bool valid;
   fmoe_layer_desc desc;
   FusedConfigs fc;
 };
 static FusedCacheEntry g_fused_cache[64];
+static std::mutex g_fused_cache_mu;
 
 static FusedConfig fused_config_uncached(const fmoe_layer_desc& d, int dev, int nt);
 
@@ -933,6 +942,7 @@ static FusedConfig fused_config(const fmoe_layer_desc& d, int nt = 1) {
   int dev = 0;
   if (nt < 1 || nt > kFusedMaxNT) return FusedConfig{};
   if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return FusedConfig{};
+  std::lock_guard<std::mutex> lock(g_fused_cache_mu);
   FusedCacheEntry& e = g_fused_cache[dev];
   if (!(e.valid && same_desc(e.desc, d))) {
     for (int n = 1; n <= kFusedMaxNT; ++n) e.fc.nt[n] = fused_config_uncached(d, dev, n);
@@ -1307,21 +1317,13 @@ extern "C" int fmoe_fused_supported(const fmoe_layer_desc* d) {
   return fused_config(*d).ok ? 1 : 0;
 }
 
-extern "C" int fmoe_set_tensor_cores(int enable) {
-  const int prev = g_tc_enabled;
-  g_tc_enabled = enable ? 1 : 0;
-  return prev;
-}
+extern "C" int fmoe_set_tensor_cores(int enable) { return g_tc_enabled.exchange(enable ? 1 : 0); }
 
 extern "C" int fmoe_tc_min_tokens(void) { return kTcMinTokens; }
 
 extern "C" int fmoe_fused_max_tokens(int stack) { return stack ? kFusedTokensStack : kFusedTokensLayer; }
 
-extern "C" int fmoe_set_fused(int enable) {
-  const int prev = g_fused_enabled;
-  g_fused_enabled = enable ? 1 : 0;
-  return prev;
-}
+extern "C" int fmoe_set_fused(int enable) { return g_fused_enabled.exchange(enable ? 1 : 0); }
 
 // A stack of layers; with a trace, every layer's input xn, intermediates and
 // output h' recorded in its record of the trace.
