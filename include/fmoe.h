@@ -26,8 +26,14 @@
  *     caller owns every buffer; no entry point allocates device memory.
  *   - Device pointers must be 16-byte aligned.
  *   - Device-side work is enqueued on the caller's stream and is
- *     asynchronous: no entry point synchronises, except the packer, which
- *     waits for its own host-to-device copy.
+ *     asynchronous: no entry point synchronises, except the host-memory
+ *     packer (it waits for its own host-to-device copies), fmoe_read_status
+ *     (it waits for the device) and the expert cache (it reads each step's
+ *     routing on the host, and zeroes its table at creation).
+ *   - Calls may come from several host threads.  A workspace, a trace, an
+ *     expert cache and the no-allocation scratch of a device serve one call
+ *     at a time (or calls ordered on one stream); fmoe_set_fused and
+ *     fmoe_set_tensor_cores are process-wide switches.
  *   - Faults detected on the device (an expert id outside [0, E), a NaN
  *     router logit, an exhausted wait) set bits of a sticky per-device
  *     status word; kernels never trap.  Read and clear it with
