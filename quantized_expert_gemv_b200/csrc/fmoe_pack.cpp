@@ -18,6 +18,15 @@
 
 namespace fmoe {
 
+// 32-bit words of a packed record by byte copies: the host buffers carry no
+// alignment guarantee, and a 4-byte memcpy compiles to one move.
+static inline void st32(uint8_t* base, size_t word, uint32_t v) { std::memcpy(base + 4 * word, &v, 4); }
+static inline uint32_t ld32(const uint8_t* base, size_t word) {
+  uint32_t v;
+  std::memcpy(&v, base + 4 * word, 4);
+  return v;
+}
+
 static inline float bf16_bits_to_f32(uint16_t h) {
   uint32_t u = (uint32_t)h << 16;
   float f;
@@ -113,26 +122,26 @@ static int pack_expert(int bits, int H, int I, const uint8_t* q, const uint16_t*
     for (int m = 0; m < 2; ++m) {
       pack_row(bits, H, q + m * n + (size_t)r * H, dst + L.gu_codes + (size_t)(2 * r + m) * L.gu_row_bytes);
       const size_t gpr = (size_t)H / 64;
-      uint32_t* sb = reinterpret_cast<uint32_t*>(dst + L.gu_sb) + (size_t)(2 * r + m) * gpr;
+      uint8_t* sb = dst + L.gu_sb + (size_t)(2 * r + m) * gpr * 4;
       for (size_t g = 0; g < gpr; ++g) {
         uint16_t s;
         if (!bf16_scale_pow2(sc[m * ng + (size_t)r * gpr + g], shift, &s)) return FMOE_ERR_INVALID_ARG;
-        sb[g] = (uint32_t)s | ((uint32_t)bi[m * ng + (size_t)r * gpr + g] << 16);
+        st32(sb, g, (uint32_t)s | ((uint32_t)bi[m * ng + (size_t)r * gpr + g] << 16));
       }
     }
   // down matrix, column-block major: word (nb, r) holds inputs
   // [nb * per_word, (nb + 1) * per_word) of row r; scale-bias word (g, r)
   const int per_word = 32 / bits;
-  uint32_t* dw = reinterpret_cast<uint32_t*>(dst + L.down_codes);
-  uint32_t* dsb = reinterpret_cast<uint32_t*>(dst + L.down_sb);
+  uint8_t* dw = dst + L.down_codes;
+  uint8_t* dsb = dst + L.down_sb;
   const size_t gpr = (size_t)I / 64;
   for (int r = 0; r < H; ++r) {
     const uint8_t* qr = q + 2 * n + (size_t)r * I;
-    for (int nb = 0; nb < I / per_word; ++nb) dw[(size_t)nb * H + r] = pack_word(bits, qr + (size_t)nb * per_word);
+    for (int nb = 0; nb < I / per_word; ++nb) st32(dw, (size_t)nb * H + r, pack_word(bits, qr + (size_t)nb * per_word));
     for (size_t g = 0; g < gpr; ++g) {
       uint16_t s;
       if (!bf16_scale_pow2(sc[2 * ng + (size_t)r * gpr + g], shift, &s)) return FMOE_ERR_INVALID_ARG;
-      dsb[g * H + r] = (uint32_t)s | ((uint32_t)bi[2 * ng + (size_t)r * gpr + g] << 16);
+      st32(dsb, g * H + r, (uint32_t)s | ((uint32_t)bi[2 * ng + (size_t)r * gpr + g] << 16));
     }
   }
   return FMOE_OK;
@@ -147,22 +156,23 @@ static int unpack_expert(int bits, int H, int I, const uint8_t* src, uint8_t* q,
     for (int m = 0; m < 2; ++m) {
       unpack_row(bits, H, src + L.gu_codes + (size_t)(2 * r + m) * L.gu_row_bytes, q + m * n + (size_t)r * H);
       const size_t gpr = (size_t)H / 64;
-      const uint32_t* sb = reinterpret_cast<const uint32_t*>(src + L.gu_sb) + (size_t)(2 * r + m) * gpr;
+      const uint8_t* sb = src + L.gu_sb + (size_t)(2 * r + m) * gpr * 4;
       for (size_t g = 0; g < gpr; ++g) {
-        if (!bf16_unscale_pow2((uint16_t)(sb[g] & 0xFFFFu), shift, &sc[m * ng + (size_t)r * gpr + g]))
+        const uint32_t w = ld32(sb, g);
+        if (!bf16_unscale_pow2((uint16_t)(w & 0xFFFFu), shift, &sc[m * ng + (size_t)r * gpr + g]))
           return FMOE_ERR_INVALID_ARG;
-        bi[m * ng + (size_t)r * gpr + g] = (uint16_t)(sb[g] >> 16);
+        bi[m * ng + (size_t)r * gpr + g] = (uint16_t)(w >> 16);
       }
     }
   const int per_word = 32 / bits;
-  const uint32_t* dw = reinterpret_cast<const uint32_t*>(src + L.down_codes);
-  const uint32_t* dsb = reinterpret_cast<const uint32_t*>(src + L.down_sb);
+  const uint8_t* dw = src + L.down_codes;
+  const uint8_t* dsb = src + L.down_sb;
   const size_t gpr = (size_t)I / 64;
   for (int r = 0; r < H; ++r) {
     uint8_t* qr = q + 2 * n + (size_t)r * I;
-    for (int nb = 0; nb < I / per_word; ++nb) unpack_word(bits, dw[(size_t)nb * H + r], qr + (size_t)nb * per_word);
+    for (int nb = 0; nb < I / per_word; ++nb) unpack_word(bits, ld32(dw, (size_t)nb * H + r), qr + (size_t)nb * per_word);
     for (size_t g = 0; g < gpr; ++g) {
-      const uint32_t w = dsb[g * H + r];
+      const uint32_t w = ld32(dsb, g * H + r);
       if (!bf16_unscale_pow2((uint16_t)(w & 0xFFFFu), shift, &sc[2 * ng + (size_t)r * gpr + g]))
         return FMOE_ERR_INVALID_ARG;
       bi[2 * ng + (size_t)r * gpr + g] = (uint16_t)(w >> 16);

@@ -64,6 +64,14 @@ def test_pack_unpack_round_trip(fm, bits, H, I):
     assert packed.nbytes == fm.fmoe_packed_bytes(bits, 2, H, I)
     q2, s2, b2 = fm.fmoe_unpack_experts_host(packed, bits, 2, H, I)
     assert np.array_equal(q2, q) and np.array_equal(s2, s) and np.array_equal(b2, b)
+    # a host buffer at an odd address gives the same bytes and unpacks the same
+    raw = np.zeros(packed.nbytes + 3, np.uint8)
+    odd = raw[3:]
+    assert odd.ctypes.data % 4 != 0
+    fm.fmoe_pack_experts_host(q, s, b, bits, 2, H, I, out=odd)
+    assert np.array_equal(odd, packed)
+    q3, s3, b3 = fm.fmoe_unpack_experts_host(odd, bits, 2, H, I)
+    assert np.array_equal(q3, q) and np.array_equal(s3, s) and np.array_equal(b3, b)
 
 
 @pytest.mark.parametrize("bits", [4, 2])
