@@ -172,6 +172,14 @@ def test_every_mutant_text_occurs_once():
         assert old != new
 
 
+@pytest.fixture(scope="module", autouse=True)
+def _generator_built():
+    """The children share the input generator's library: built once here,
+    not by several children at the same time."""
+    import synth
+    synth.lib()
+
+
 def test_unchanged_copy_passes_the_pins(tmp_path):
     path = _copy_oracle(str(tmp_path), _source())
     rc, out, where = _run_pins(path)
