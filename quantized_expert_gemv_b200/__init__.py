@@ -4,7 +4,7 @@ A thin ctypes layer over the C ABI declared in include/fmoe.h: it converts
 torch tensors / numpy arrays to pointers and checks status codes.  Every step
 of the computation runs in the library's CUDA kernels; there is no Python or
 CPU fallback.  If libfmoe.so has not been built, importing this package
-raises ImportError (build it with ``python -m quantized_expert_gemv_b200.build``
+raises ImportError (build it with ``python quantized_expert_gemv_b200/build.py``
 or ``__graft_entry__.build()``).
 
 PyTorch is used only for device memory and streams: device arguments are
@@ -25,7 +25,7 @@ _LIB_PATH = os.path.join(_PKG, "libfmoe.so")
 if not os.path.exists(_LIB_PATH):
     raise ImportError(
         f"{_LIB_PATH} is missing: the CUDA library has not been built "
-        "(run `python -m quantized_expert_gemv_b200.build`). There is no fallback.")
+        "(run `python quantized_expert_gemv_b200/build.py`). There is no fallback.")
 
 _lib = ctypes.CDLL(_LIB_PATH)
 

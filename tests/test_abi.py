@@ -15,8 +15,13 @@ ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
 
 @pytest.fixture(scope="module")
 def fm():
-    from quantized_expert_gemv_b200 import build
-    build.build()
+    # the builder by its path: importing the package needs the library it builds
+    import importlib.util
+    spec = importlib.util.spec_from_file_location(
+        "fmoe_library_build", os.path.join(ROOT, "quantized_expert_gemv_b200", "build.py"))
+    builder = importlib.util.module_from_spec(spec)
+    spec.loader.exec_module(builder)
+    builder.build()
     import quantized_expert_gemv_b200 as m
     return m
 
