@@ -9,18 +9,21 @@
 // the output for token t is D[., t] + D[., Np + t].  Persistent CTAs (one
 // per SM) take work units of (item of <= 32 tokens, tile of 128 weight
 // rows), all N = 2 Np columns, the accumulator in tensor memory:
-//   - the 256 producer threads stream the tile's raw codes into a shared
-//     ring with cp.async, two 8-group supersteps ahead, and two warps per
-//     64-input group dequantise it into a 4-stage fp16 A ring (K-major core
-//     matrices of 8 rows x 16 bytes), requesting the group's staged X tile
-//     by one bulk copy;
-//   - one thread issues the four 128 x N x 16 tcgen05.mma of the group and
-//     commits them to the stage's mbarrier, so dequantising the next groups
-//     overlaps the tensor cores (at N <= 64 the issue rate of these small
-//     products, about 75 ns each, bounds the kernel: measured per step);
-//   - the epilogue reads the accumulator with tcgen05.ld (warp w: tensor
-//     memory lanes 32 (w % 4) ..), adds the hi and lo columns, and writes
-//     SwiGLU outputs (gate/up) or expert outputs (down).
+//   - the eight producer warps stream the tile's raw codes with 16-byte
+//     cp.async into a ring of four supersteps of 4 groups (three supersteps
+//     ahead), and two warps per 64-input group dequantise it into a 4-stage
+//     fp16 A ring (K-major, 128-byte swizzle); the group's staged X tile
+//     comes by one bulk copy into an 8-stage ring, requested four steps
+//     ahead;
+//   - one thread (warp 0, alone on its SM sub-partition) issues the four
+//     128 x N x 16 tcgen05.mma of the group and commits them to the stage's
+//     mbarrier, so dequantising the next groups overlaps the tensor cores
+//     (at N <= 64 the issue rate of these small products, about 75 ns each,
+//     bounds the kernel: measured per step);
+//   - the epilogue (warps 0-7) reads the accumulator with tcgen05.ld (warp
+//     w: tensor memory lanes 32 (w % 4) .., the token columns split between
+//     warps w and w + 4), adds the hi and lo columns, and writes SwiGLU
+//     outputs (gate/up) or expert outputs (down).
 // Error bound per output: w is rounded once (relative 2^-12), x keeps 22
 // bits, the fp32 accumulation adds at most K 2^-24 of the sum of |w x|:
 // below 5e-4 of that sum at K = 4096, inside the 1e-3 tolerance.
