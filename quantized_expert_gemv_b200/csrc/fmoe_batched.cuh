@@ -4,10 +4,13 @@
 // shared-expert slots are sorted by expert (group_kernel, in token order
 // within an expert, so every result is deterministic).  Each expert's
 // weights are then read once per step for all of its tokens:
-//   - groups with fewer than kTcMinTokens tokens, in work items of up to
-//     kGrpMaxM tokens, go through the integer-dot GEMV (gateup_group_kernel,
-//     down_group_kernel): one load of a weight row serves every token of the
-//     item;
+//   - groups with fewer than kTcMinTokens tokens (all groups, with the
+//     tensor cores switched off), in work items of up to kGrpMaxM tokens, go
+//     through the integer-dot GEMV: gate/up row pairs by bulk copy into
+//     per-warp slots for items of up to 4 tokens (gateup_bulk_small_kernel,
+//     gateup_bulk_kernel), by direct loads for larger ones
+//     (gateup_group_kernel), and down_group_kernel; one load of a weight row
+//     serves every token of the item;
 //   - groups with at least kTcMinTokens tokens are dense enough for the
 //     tensor cores (fmoe_tc.cuh): their items are listed separately.
 // Slot s = t (k + 1) + j addresses a [T][k+1][I] and y [T][k+1][H] exactly as
