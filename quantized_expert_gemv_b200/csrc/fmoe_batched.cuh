@@ -7,9 +7,10 @@
 //   - groups with fewer than kTcMinTokens tokens (all groups, with the
 //     tensor cores switched off), in work items of up to kGrpMaxM tokens, go
 //     through the integer-dot GEMV: gate/up row pairs by bulk copy into
-//     per-warp slots for items of up to 4 tokens (gateup_bulk_small_kernel,
-//     gateup_bulk_kernel), by direct loads for larger ones
-//     (gateup_group_kernel), and down_group_kernel; one load of a weight row
+//     per-warp slots for items of up to 4 tokens when a row holds at least
+//     32 groups (gateup_bulk_small_kernel, gateup_bulk_kernel), by direct
+//     loads otherwise (gateup_group_kernel), then the down products
+//     (down_group_small_kernel, down_group_kernel); one load of a weight row
 //     serves every token of the item;
 //   - groups with at least kTcMinTokens tokens are dense enough for the
 //     tensor cores (fmoe_tc.cuh): their items are listed separately.
