@@ -45,3 +45,30 @@ def test_max_over_ranks_and_job_rate_on_two_gloo_ranks():
 def test_job_rate_single_rank():
     import bench
     assert bench.job_rate(4000, 1, 80.0) == pytest.approx(50_000.0)
+
+
+def test_reference_arm_prints_the_contract_line_on_rank_0_only():
+    """`bench.py --impl reference` (the CPU oracle timed on the host cores)
+    prints one JSON line with the metric, the reference tag, its CPU
+    baseline and an end-to-end entry without copies; a rank other than 0
+    exits 0 without work.  Needs no GPU."""
+    import json
+    import subprocess
+    import sys
+    root = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+    env = {k: v for k, v in os.environ.items() if k not in ("RANK", "WORLD_SIZE", "LOCAL_RANK")}
+    cmd = [sys.executable, "bench.py", "--impl", "reference", "--steps", "2", "--warmup", "3"]
+    p = subprocess.run(cmd, cwd=root, env=env, capture_output=True, text=True, timeout=600)
+    assert p.returncode == 0, p.stderr[-2000:]
+    lines = [l for l in p.stdout.splitlines() if l.startswith("{")]
+    assert len(lines) == 1, p.stdout
+    d = json.loads(lines[0])
+    assert d["impl"] == "reference" and d["unit"] == "layer_fwd/s" and d["value"] > 0
+    assert d["higher_is_better"] is True and d["vs_baseline"] is None and d["warmup"] == 3
+    assert d["config"]["workload"].startswith("moe_layer_int4_batch1")
+    cb = d["cpu_baseline"]
+    assert cb["kind"] == "oracle" and cb["cores"] >= 1 and cb["value"] == d["value"] and cb["sample"]
+    assert d["e2e"] == {"value": d["value"], "unit": d["unit"], "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}
+    p1 = subprocess.run(cmd, cwd=root, env=dict(env, RANK="1", WORLD_SIZE="2", LOCAL_RANK="1"), capture_output=True,
+                        text=True, timeout=600)
+    assert p1.returncode == 0 and not any(l.startswith("{") for l in p1.stdout.splitlines())
