@@ -72,3 +72,34 @@ def test_reference_arm_prints_the_contract_line_on_rank_0_only():
     p1 = subprocess.run(cmd, cwd=root, env=dict(env, RANK="1", WORLD_SIZE="2", LOCAL_RANK="1"), capture_output=True,
                         text=True, timeout=600)
     assert p1.returncode == 0 and not any(l.startswith("{") for l in p1.stdout.splitlines())
+
+
+def test_clock_sampler_reads_clocks_and_decodes_reasons_from_nvml(monkeypatch):
+    """The benchmark's clock record against a fake NVML (no GPU): the
+    median SM clock of the samples, the maximum clock, and the names of the
+    active clock-event reason bits (sw_power_cap kept, slowdowns named)."""
+    import sys
+    import types
+
+    import bench
+    clocks = iter([1965, 1800, 1965, 1965, 1500] + [1965] * 1000)
+    reasons = iter([0x0, 0x4, 0x8 | 0x40] + [0x0] * 1000)
+    fake = types.SimpleNamespace(
+        NVML_CLOCK_SM=1,
+        nvmlInit=lambda: None,
+        nvmlDeviceGetHandleByPciBusId=lambda bus: "h",
+        nvmlDeviceGetHandleByIndex=lambda i: "h",
+        nvmlDeviceGetMaxClockInfo=lambda h, kind: 1965,
+        nvmlDeviceGetClockInfo=lambda h, kind: next(clocks),
+        nvmlDeviceGetCurrentClocksEventReasons=lambda h: next(reasons))
+    monkeypatch.setitem(sys.modules, "pynvml", fake)
+    s = bench.ClockSampler(0, period=3600.0)  # samples at entry and exit only
+    assert s.ok
+    with s:
+        pass
+    s._sample()
+    s._sample()
+    out = s.summary()
+    assert out["sm_max_mhz"] == 1965 and out["samples"] == 4
+    assert out["sm_mhz"] == 1965  # median of 1965, 1800, 1965, 1965
+    assert out["reasons"] == ["hw_slowdown", "hw_thermal_slowdown", "sw_power_cap"]
