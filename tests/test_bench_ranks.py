@@ -103,3 +103,23 @@ def test_clock_sampler_reads_clocks_and_decodes_reasons_from_nvml(monkeypatch):
     assert out["sm_max_mhz"] == 1965 and out["samples"] == 4
     assert out["sm_mhz"] == 1965  # median of 1965, 1800, 1965, 1965
     assert out["reasons"] == ["hw_slowdown", "hw_thermal_slowdown", "sw_power_cap"]
+
+
+def test_roofline_denominator_and_traffic_record(monkeypatch, tmp_path):
+    """The roofline's peak comes from the measured-peaks file when there is
+    one (else the stated fallback), and the recorded DRAM traffic is
+    reported only while the kernel sources match the digest it was taken
+    with."""
+    import json
+
+    import bench
+    (tmp_path / "MEASURED_PEAKS.json").write_text(json.dumps({"hbm_gbs": 6123.5}))
+    monkeypatch.setattr(bench, "ROOT", str(tmp_path))
+    assert bench.measured_peak() == (6123.5, "measured")
+    (tmp_path / "MEASURED_PEAKS.json").unlink()
+    assert bench.measured_peak() == (bench.FALLBACK_HBM_GBS, "fallback")
+    monkeypatch.undo()
+    rec = bench.TRAFFIC_PER_LAYER
+    assert bench.measured_traffic(20) in (20 * rec["bytes"], None)
+    monkeypatch.setattr(bench, "TRAFFIC_PER_LAYER", dict(rec, sources_sha256_16="0" * 16))
+    assert bench.measured_traffic(20) is None
