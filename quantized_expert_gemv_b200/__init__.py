@@ -198,8 +198,21 @@ def fmoe_packed_bytes(bits: int, n_experts: int, hidden: int, inter: int, group:
     return int(_lib.fmoe_packed_bytes(bits, n_experts, hidden, inter, group))
 
 
+def _pack_inputs(q, scale, bias, bits: int, n_experts: int, hidden: int, inter: int, group: int, cuda: bool) -> None:
+    """The logical codes (one byte each) and bf16 scale / bias (two bytes
+    each, per group) that a packer reads must all be there; checked when the
+    shape is one the library packs (otherwise its status says why)."""
+    if n_experts < 1 or group < 1 or fmoe_packed_bytes(bits, n_experts, hidden, inter, group) <= 0:
+        return
+    n = n_experts * 3 * hidden * inter
+    _need(q, "q", n, None, cuda=cuda, exact=False)
+    _need(scale, "scale", 2 * (n // group), None, cuda=cuda, exact=False)
+    _need(bias, "bias", 2 * (n // group), None, cuda=cuda, exact=False)
+
+
 def fmoe_pack_experts_host(q: np.ndarray, scale: np.ndarray, bias: np.ndarray, bits: int, n_experts: int,
                            hidden: int, inter: int, group: int = 64, out: np.ndarray | None = None) -> np.ndarray:
+    _pack_inputs(q, scale, bias, bits, n_experts, hidden, inter, group, cuda=False)
     n = fmoe_packed_bytes(bits, n_experts, hidden, inter, group)
     if out is None:
         out = np.empty(max(n, 1), np.uint8)
@@ -211,6 +224,9 @@ def fmoe_pack_experts_host(q: np.ndarray, scale: np.ndarray, bias: np.ndarray, b
 
 def fmoe_unpack_experts_host(packed: np.ndarray, bits: int, n_experts: int, hidden: int, inter: int,
                              group: int = 64):
+    if n_experts >= 1 and fmoe_packed_bytes(bits, n_experts, hidden, inter, group) > 0:
+        _need(packed, "packed", fmoe_packed_bytes(bits, n_experts, hidden, inter, group), None, cuda=False,
+              exact=False)
     n = hidden * inter
     q = np.empty(n_experts * 3 * n, np.uint8)
     s = np.empty(n_experts * 3 * n // group, np.uint16)
@@ -223,6 +239,8 @@ def fmoe_unpack_experts_host(packed: np.ndarray, bits: int, n_experts: int, hidd
 def fmoe_pack_experts(q, scale, bias, bits: int, n_experts: int, hidden: int, inter: int, d_packed,
                       group: int = 64, stream=None, byte_offset: int = 0) -> None:
     """Packs host logical experts into the device tensor d_packed (at byte_offset)."""
+    _pack_inputs(q, scale, bias, bits, n_experts, hidden, inter, group, cuda=False)
+    _need(d_packed, "d_packed", byte_offset, None, exact=False)
     dst = d_packed.data_ptr() + byte_offset
     avail = d_packed.numel() * d_packed.element_size() - byte_offset
     rc = _lib.fmoe_pack_experts(_ptr(q), _ptr(scale), _ptr(bias), bits, n_experts, hidden, inter, group,
@@ -233,6 +251,8 @@ def fmoe_pack_experts(q, scale, bias, bits: int, n_experts: int, hidden: int, in
 def fmoe_pack_experts_device(d_q, d_scale, d_bias, bits: int, n_experts: int, hidden: int, inter: int, d_packed,
                              group: int = 64, stream=None, byte_offset: int = 0) -> None:
     """Packs logical experts already on the device into d_packed (at byte_offset)."""
+    _pack_inputs(d_q, d_scale, d_bias, bits, n_experts, hidden, inter, group, cuda=True)
+    _need(d_packed, "d_packed", byte_offset, None, exact=False)
     dst = d_packed.data_ptr() + byte_offset
     avail = d_packed.numel() * d_packed.element_size() - byte_offset
     rc = _lib.fmoe_pack_experts_device(_ptr(d_q), _ptr(d_scale), _ptr(d_bias), bits, n_experts, hidden, inter,
@@ -486,6 +506,10 @@ def fmoe_quantize_groups(w, bits: int, q, scale, bias, stream=None) -> None:
     n = w.numel()
     if n % 64:
         raise ValueError("w must hold whole 64-value groups")
+    _need(w, "w", n)
+    _need(q, "q", n, None, exact=False)
+    _need(scale, "scale", 2 * (n // 64), None, exact=False)
+    _need(bias, "bias", 2 * (n // 64), None, exact=False)
     rc = _lib.fmoe_quantize_groups(_ptr(w), n // 64, 64, bits, _ptr(q), _ptr(scale), _ptr(bias), _stream(stream))
     _check(rc, "fmoe_quantize_groups")
 

@@ -398,6 +398,21 @@ def test_binding_refuses_bad_buffers_before_the_call(fm):
     with pytest.raises(ValueError, match="xn: must be in CUDA device memory"):
         fm.fmoe_expert_forward(lw, xn, torch.zeros(2, k, dtype=torch.int32), torch.zeros(2, k + 1, H),
                                torch.zeros(2), ws)
+    # packers: the codes and scales of every expert must be there (shape
+    # supported); an unsupported shape is still the library's to refuse
+    q = np.zeros(3 * H * 128, np.uint8)
+    sb = np.zeros(3 * H * 128 // 64, np.uint16)
+    with pytest.raises(ValueError, match="q: holds"):
+        fm.fmoe_pack_experts_host(q, sb, sb, 4, 2, H, 128)
+    with pytest.raises(ValueError, match="scale: holds"):
+        fm.fmoe_pack_experts_host(np.zeros(2 * 3 * H * 128, np.uint8), sb, sb, 4, 2, H, 128)
+    with pytest.raises(ValueError, match="packed: holds"):
+        fm.fmoe_unpack_experts_host(np.zeros(100, np.uint8), 4, 1, H, 128)
+    with pytest.raises(ValueError, match="q: must be in CUDA device memory"):
+        fm.fmoe_pack_experts_device(q, sb, sb, 4, 1, H, 128, torch.zeros(10, dtype=torch.uint8))
+    with pytest.raises(ValueError, match="w: must be in CUDA device memory"):
+        fm.fmoe_quantize_groups(torch.zeros(128), 4, torch.zeros(128, dtype=torch.uint8),
+                                torch.zeros(2, dtype=torch.int16), torch.zeros(2, dtype=torch.int16))
     # a cached layer's descriptor does not need device experts, only the rest
     lw_cached = fm.LayerWeights(d, None, lw.shared, lw.w_router, lw.w_shared_gate, lw.norm_w)
     with pytest.raises(ValueError, match="shared: must be in CUDA device memory"):
