@@ -540,6 +540,8 @@ class ExpertCache:
         import torch
         self.desc, self.host_layers = desc, list(host_layers)
         rec = desc.record_bytes()
+        for l, t in enumerate(self.host_layers):
+            _need(t, f"host_layers[{l}]", desc.n_experts * rec, None, cuda=False, exact=False)
         self.slots = torch.empty(n_slots * rec, dtype=torch.uint8, device="cuda")
         self.table = torch.zeros(len(self.host_layers) * desc.n_experts, dtype=torch.int64, device="cuda")
         ptrs = (ctypes.c_void_p * len(self.host_layers))(*[t.data_ptr() for t in self.host_layers])

@@ -413,6 +413,10 @@ def test_binding_refuses_bad_buffers_before_the_call(fm):
     with pytest.raises(ValueError, match="w: must be in CUDA device memory"):
         fm.fmoe_quantize_groups(torch.zeros(128), 4, torch.zeros(128, dtype=torch.uint8),
                                 torch.zeros(2, dtype=torch.int16), torch.zeros(2, dtype=torch.int16))
+    # the host tier's layers must hold every routed record
+    with pytest.raises(ValueError, match=r"host_layers\[1\]: holds"):
+        fm.ExpertCache(d, [torch.zeros(E * d.record_bytes(), dtype=torch.uint8),
+                           torch.zeros(E * d.record_bytes() - 1, dtype=torch.uint8)], n_slots=4)
     # a cached layer's descriptor does not need device experts, only the rest
     lw_cached = fm.LayerWeights(d, None, lw.shared, lw.w_router, lw.w_shared_gate, lw.norm_w)
     with pytest.raises(ValueError, match="shared: must be in CUDA device memory"):
